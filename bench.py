@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the STAR-KV paged low-rank decode step on B200.
+
+One step = the whole hot path over one batch: compress-and-append of one new
+token per sequence into the paged K/V code pools, then single-token paged
+decode over the updated cache, for every layer of the workload.  Inputs are
+seeded and synthetic with the shapes of the pages' kernel benchmark (32-head
+MHA, head_size 128, rank 64, fp16, block size 16).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 3] [--impl ours|reference]
+
+Multi-GPU runs are independent replicas (the path has no exchange step): each
+rank owns its own cache and batch, timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "compressed-KV paged decode tokens/s at 1 B200; HBM GB/s as % of ~8 TB/s peak"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+WORKLOAD_NAMES = {
+    2: "single-layer decode: 32 heads, head_size 128, K rank 64/head, V joint rank 2048, fp16, "
+       "block_size 16, batch 16, seq_len 2048",
+    3: "single-layer decode: 32 heads, head_size 128, K rank 64/head, V joint rank 2048, fp16, "
+       "block_size 16, batch 64, seq_len 8192",
+    4: "continuous batching: 32 heads, head_size 128, batch 48, seq_len ~U[512,16384], 3 layers "
+       "K rank {32,64,96}, V rank 32r, fp16, block_size 16",
+    5: "Llama-2-7B attention path: 32 layers, 32 heads, head_size 128, batch 8, context 32768, "
+       "K rank 64/head, V rank 2048, fp16, block_size 16",
+}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", type=int, default=3, choices=[2, 3, 4, 5])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="budget of the oracle CPU-baseline sample")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# --------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [x.strip() for x in line.split(",")]
+                    if len(parts) < 10:
+                        continue
+                    if self.uuid and self.uuid not in parts[1]:
+                        continue
+                    rows.append(parts)
+            os.unlink(self.path)
+        except Exception:
+            return None
+        if not rows:
+            return None
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------ our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import rank_compressed_kv_star_b200 as S
+    from rank_compressed_kv_star_b200 import build
+    from starkv_inputs import device as D, workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    if rank == 0:
+        build.build()
+        build.build_inputs()
+    if world > 1:
+        dist.barrier()
+    S.load_library()
+
+    wl = W.workload(args.workload)
+    layers = []
+    for li in range(len(wl.layers)):
+        Ld = D.device_layer(wl, li)
+        Ld["desc"] = S.layer_desc(Ld["H"], Ld["d"], Ld["r"], Ld["R"], Ld["nb"], Ld["tables"].shape[1])
+        layers.append(Ld)
+    B = wl.batch
+    max_len = wl.max_seq_len
+    wsb = max(S.starkv_decode_workspace_bytes(L["desc"], B, max_len) for L in layers)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    outs = [torch.empty((B, L["H"], L["d"]), dtype=torch.float16, device="cuda") for L in layers]
+    stream = torch.cuda.current_stream()
+    n_ev = 6
+
+    def step(evs=None, app_evs=None, li_prof=None):
+        for li, L in enumerate(layers):
+            if app_evs is not None:
+                app_evs[li][0].record(stream)
+            S.starkv_compress_append(L["desc"], B, L["k"], L["v"], L["A_K"], L["A_V"], L["tables"],
+                                     L["ctx_lens"], L["k_cache"], L["v_cache"], stream=stream)
+            if app_evs is not None:
+                app_evs[li][1].record(stream)
+            if evs is not None:
+                S.starkv_paged_decode_profiled(L["desc"], B, max_len, L["q"], L["B_K"], L["B_V"],
+                                               L["k_cache"], L["v_cache"], L["tables"], L["seq_lens"],
+                                               L["scale"], ws, wsb, outs[li], evs[li], stream=stream)
+            else:
+                S.starkv_paged_decode(L["desc"], B, max_len, L["q"], L["B_K"], L["B_V"], L["k_cache"],
+                                      L["v_cache"], L["tables"], L["seq_lens"], L["scale"], ws, wsb,
+                                      outs[li], stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    st, flags = S.starkv_decode_check(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device status {S.STATUS[st]} flags {flags}")
+
+    # ---------------- device-timed region: inputs resident, codes >> L2 per step
+    K = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in layers] for _ in range(K)]
+    app_evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in layers] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t0.record(stream)
+    for i in range(K):
+        step(evs[i], app_evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1) / K
+    st, flags = S.starkv_decode_check(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device status {S.STATUS[st]} flags {flags}")
+
+    names = ["absorb", "kpass", "reduce", "vpass", "upproj"]
+    per = {n: 0.0 for n in names}
+    per["append"] = 0.0
+    for i in range(K):
+        for li in range(len(layers)):
+            e = evs[i][li]
+            for j, n in enumerate(names):
+                per[n] += e[j].elapsed_time(e[j + 1])
+            per["append"] += app_evs[i][li][0].elapsed_time(app_evs[i][li][1])
+    per = {n: v / K for n, v in per.items()}             # ms per step (all layers)
+
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # ---------------- algorithmic bytes
+    T_sum = int(wl.seq_lens.sum())
+    k_bytes = sum(T_sum * L["H"] * L["r"] * 2 for L in layers)
+    v_bytes = sum(T_sum * L["R"] * 2 for L in layers)
+    proj_bytes = sum(L["B_K"].numel() * 2 + L["B_V"].numel() * 2 + L["A_K"].numel() * 2 + L["A_V"].numel() * 2
+                     for L in layers)
+    act_bytes = sum(B * L["H"] * L["d"] * 2 * 4 for L in layers)   # q, k, v in; out
+    step_bytes = k_bytes + v_bytes + proj_bytes + act_bytes
+    peak, peak_kind = measured_peaks()
+    kp_gbs = k_bytes / (per["kpass"] * 1e-3) / 1e9
+    vp_gbs = v_bytes / (per["vpass"] * 1e-3) / 1e9
+    dom = "kpass" if per["kpass"] >= per["vpass"] else "vpass"
+    dom_bytes, dom_gbs = (k_bytes, kp_gbs) if dom == "kpass" else (v_bytes, vp_gbs)
+
+    # ---------------- end to end through the public API with host buffers
+    Ke = max(1, min(args.e2e_steps, K))
+    host_in = []
+    for L in layers:
+        host_in.append({n: L[n].cpu().pin_memory() for n in ("q", "k", "v", "tables", "seq_lens", "ctx_lens")})
+    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    h2d = sum(t.numel() * t.element_size() for h in host_in for t in h.values())
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(Ke):
+        for li, L in enumerate(layers):
+            for n, t in host_in[li].items():
+                L[n].copy_(t, non_blocking=True)
+        step()
+        for li in range(len(layers)):
+            host_out[li].copy_(outs[li], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / Ke
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    assert np.isfinite(host_out[0].float().numpy()).all()
+
+    cpu = None
+    if rank == 0 and world == 1:
+        cpu = cpu_baseline(wl, args.cpu_seconds)
+
+    value = world * B / (ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "accum": "f32", "data": "synthetic",
+        "config": {"workload": f"cfg{args.workload}: {WORKLOAD_NAMES[args.workload]}", "batch": B,
+                   "max_seq_len": max_len, "layers": len(layers),
+                   "step": "compress-append of one token per sequence + paged decode, every layer",
+                   "l2": "inputs larger than L2 (code pools of %.2f GiB read per step)" % ((k_bytes + v_bytes) / 2**30),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "hbm": {"step_algorithmic_bytes": step_bytes,
+                "step_GBps": round(step_bytes / (ms * 1e-3) / 1e9, 1),
+                "frac_of_8TBps": round(step_bytes / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4),
+                "frac_of_peak": round(step_bytes / (ms * 1e-3) / 1e9 / peak, 4), "peak_kind": peak_kind},
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": round(dom_gbs, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(dom_gbs / peak, 4), "traffic": None,
+                     "algorithmic_bytes_per_launch": dom_bytes // len(layers), "peak_kind": peak_kind},
+        "kernels_ms_per_step": {n: round(v, 5) for n, v in per.items()},
+        "kernels_GBps": {"kpass": round(kp_gbs, 1), "vpass": round(vp_gbs, 1)},
+        "e2e": {"value": round(world * B / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
+        "gpu_launches": K * len(layers) * 6,
+        "clocks": clk,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# -------------------------------------------------------- CPU baseline
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def prepare_seq(wl, b, layer, proj_cache):
+    """Host inputs of one sequence of one layer: a private paged pool holding its pages
+    under a shuffled block-table row (generation is not part of any timing)."""
+    from starkv_inputs import workloads as W
+    sh = wl.layers[layer]
+    ctx = int(wl.ctx_lens[b])
+    T = ctx + (1 if wl.append else 0)
+    cK, cV = W.seq_codes(wl, layer, b, ctx)
+    n_pages = -(-T // 16)
+    row = np.random.default_rng(b).permutation(n_pages).astype(np.int32)
+    kc = np.full((n_pages, 16, sh.num_heads, sh.k_rank), np.nan, np.float16)
+    vc = np.full((n_pages, 16, sh.v_rank), np.nan, np.float16)
+    W.place_host(kc, row, cK)
+    W.place_host(vc, row, cV)
+    if layer not in proj_cache:
+        proj_cache[layer] = W.projections(wl, layer)
+    q, k, v = (W.activation(wl, layer, a)[b:b + 1] for a in (W.ACT_Q, W.ACT_K, W.ACT_V))
+    return dict(kc=kc, vc=vc, row=row, q=q, k=k, v=v, ctx=ctx, T=T, proj=proj_cache[layer],
+                append=wl.append, H=sh.num_heads)
+
+
+def oracle_eval(st, heads=None):
+    """Timed oracle work for one prepared sequence: append, block-table walk, decode of `heads`."""
+    from oracle import starkv_oracle as O
+    A_K, A_V, B_K, B_V = st["proj"]
+    t0 = time.perf_counter()
+    kc, vc = st["kc"], st["vc"]
+    if st["append"]:
+        _, _, kc, vc = O.compress_append(st["k"], st["v"], A_K, A_V, st["row"][None],
+                                         np.array([st["ctx"]]), kc, vc)
+    cK = O.gather(kc, st["row"], st["T"])
+    cV = O.gather(vc, st["row"], st["T"])
+    O.attend_codes_reordered(st["q"][0], B_K, B_V, cK, cV, 1.0 / np.sqrt(st["q"].shape[2]), heads=heads)
+    return time.perf_counter() - t0
+
+
+def _prepared(wl, n_seq=4):
+    proj = {}
+    n_layers = len(wl.layers)
+    out = []
+    for i in range(n_seq):
+        layer = i % n_layers
+        b = (i * 7919) % wl.batch
+        out.append(prepare_seq(wl, b, layer, proj))
+    return out
+
+
+def cpu_baseline(wl, budget_s):
+    seqs = _prepared(wl)
+    done, spent = 0, 0.0
+    while spent < budget_s:
+        spent += oracle_eval(seqs[done % len(seqs)])
+        done += 1
+    n_layers = len(wl.layers)
+    tok_per_s = done / spent / n_layers          # one decode token = one sequence through every layer
+    return {"value": round(tok_per_s, 4), "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{done} (sequence, layer) append+decode evaluations of this workload in fp64 "
+                      f"(explicit K, reordered V), cycling over {len(seqs)} prepared sequences; "
+                      f"{spent:.1f} s of oracle time, code generation excluded"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    from starkv_inputs import workloads as W
+    wl = W.workload(args.workload)
+    seqs = _prepared(wl)
+    n_layers = len(wl.layers)
+    H = seqs[0]["H"]
+    per_step_budget = min(2.0, 120.0 / (args.steps + args.warmup))
+    # heads per step sized from one calibration evaluation
+    t_full = oracle_eval(seqs[0])
+    n_heads = int(max(1, min(H, round(H * per_step_budget / max(t_full, 1e-6)))))
+    times, frac = [], []
+    for i in range(args.warmup + args.steps):
+        h0 = (i * n_heads) % H
+        heads = [(h0 + j) % H for j in range(n_heads)]
+        sec = oracle_eval(seqs[i % len(seqs)], heads=heads)
+        if i >= args.warmup:
+            times.append(sec)
+            frac.append(n_heads / H)
+    tokens = sum(frac) / n_layers
+    value = tokens / sum(times)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * sum(times) / len(times), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"cfg{args.workload}: {WORKLOAD_NAMES[args.workload]}", "batch": wl.batch,
+                   "max_seq_len": wl.max_seq_len, "layers": n_layers},
+        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": _blas_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: one sequence's append, block-table walk and decode of "
+                                   f"{n_heads}/{H} heads for one layer, fp64 oracle"},
+        "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

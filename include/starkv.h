@@ -1,0 +1,210 @@
+/*
+ * starkv.h -- C ABI of the STAR-KV paged low-rank decode library (sm_100a).
+ *
+ * STAR-KV stores, per layer, a low-rank projection of the K/V cache instead of
+ * the full-dimension cache: head-wise for K and joint across heads for V,
+ * kept in a compressed paged format (Proxima README, "Low-rank KV Cache
+ * Compression for vLLM", opening method paragraph; tenosra.com/proxima, first
+ * paragraph).  This library implements the two per-token steps of that cache:
+ *
+ *   compress-and-append : codes of each sequence's new token written into the
+ *                         paged pools;
+ *   paged decode        : single-query attention computed straight from the
+ *                         codes, never materialising full keys or values.
+ *
+ * Formulation (head_dim d, H heads, K rank r per head, V joint rank R):
+ *   c_K[h] = k_h . A_K[h]         A_K[h] : d x r        (head-wise K)
+ *   c_V    = v . A_V              A_V    : (H*d) x R    (joint V, v = concat_h v_h)
+ *   q~_h   = scale * q_h . B_K[h]^T,  B_K[h] : r x d    (query absorbed into K codes)
+ *   s[h,t] = q~_h . c_K[t,h]
+ *   p[h,:] = softmax_t(s[h,:])
+ *   out_h  = (sum_t p[h,t] c_V[t]) . B_V[:, h*d:(h+1)*d],  B_V : R x (H*d)
+ * which equals softmax attention over the decompressed keys k^_h = c_K[h].B_K[h]
+ * and values v^ = c_V.B_V.
+ *
+ * Paged format: pages of block_size = 16 tokens (README, KV-cache block
+ * paragraph: block size 16); token t of sequence b is in slot t % 16 of
+ * physical page block_tables[b][t / 16] (PagedAttention block-level
+ * management, botdigit.com explainer, "How Dynamic KV-Cache Compaction Works").
+ * Layouts (row-major, fp16): K pool [num_blocks][16][H][r];
+ *                            V pool [num_blocks][16][R].
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    allocates no memory and keeps no state between calls.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued asynchronously; a call returning STARKV_OK means the
+ *    launches were accepted, not that they finished.
+ *  - Argument and shape problems are reported synchronously, before any launch,
+ *    and leave all buffers untouched.  Launch failures return STARKV_ERR_CUDA.
+ *  - Device code never traps.  Data problems the host cannot see (a block id
+ *    outside [0, num_blocks), a length above the table's capacity, a timed-out
+ *    internal wait) set bits of a device status word that
+ *    starkv_decode_check() reads back; the affected output is undefined.
+ */
+#ifndef STARKV_H_
+#define STARKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  STARKV_OK = 0,
+  STARKV_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad scale */
+  STARKV_ERR_UNSUPPORTED = 2,  /* shape outside what the kernels implement */
+  STARKV_ERR_WORKSPACE = 3,    /* workspace null or smaller than required */
+  STARKV_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  STARKV_ERR_DEVICE_CHECK = 5, /* device status word reported a data problem */
+  STARKV_ERR_TIMEOUT = 6       /* an internal device wait ran out of time */
+} starkv_status;
+
+/* Device status word bits (starkv_decode_check). */
+#define STARKV_FLAG_BAD_BLOCK_ID 0x1  /* block id outside [0, num_blocks) */
+#define STARKV_FLAG_BAD_SEQ_LEN 0x2   /* seq_len < 0 or > max_blocks_per_seq*16 or > max_seq_len */
+#define STARKV_FLAG_TIMEOUT 0x4       /* a pipeline wait exceeded its bound */
+
+/* One layer's cache geometry.  Ranks may differ from layer to layer. */
+typedef struct {
+  int32_t num_heads;          /* H: 1..64, power of two (query and KV heads; MHA) */
+  int32_t head_dim;           /* d: 32, 64, 128 or 256 */
+  int32_t k_rank;             /* r: multiple of 16, 16..256 */
+  int32_t v_rank;             /* R: multiple of 64, 64..8192 */
+  int32_t block_size;         /* must be 16 */
+  int32_t num_blocks;         /* pages in each pool */
+  int32_t max_blocks_per_seq; /* row length of block_tables */
+} starkv_layer_desc;
+
+/*
+ * starkv_compress_append -- write the codes of one new token per sequence.
+ *
+ * Computes c_K[b,h,:] = k[b,h,:] . A_K[h] and c_V[b,:] = v[b,:] . A_V with fp32
+ * accumulation, rounds them to fp16 (round to nearest even) and stores them in
+ * slot positions[b] % 16 of page block_tables[b][positions[b] / 16] of the K
+ * and V pools.  Nothing else in the pools is written.
+ *
+ *   k, v          fp16 [batch][H][d]  (v read as the concatenation [batch][H*d])
+ *   A_K           fp16 [H][d][r]
+ *   A_V           fp16 [H*d][R]
+ *   block_tables  int32 [batch][max_blocks_per_seq]
+ *   positions     int32 [batch]: the sequence length BEFORE this append
+ *   k_cache       fp16 [num_blocks][16][H][r]   (in/out)
+ *   v_cache       fp16 [num_blocks][16][R]      (in/out)
+ *
+ * Targets must be distinct slots (no page shared between sequences).  A target
+ * whose position or block id is out of range is skipped.  batch == 0 is a
+ * no-op.  Cites: README method paragraph ("stored in a compressed paged format").
+ */
+starkv_status starkv_compress_append(const starkv_layer_desc* desc, int32_t batch, const void* k,
+                                     const void* v, const void* A_K, const void* A_V,
+                                     const int32_t* block_tables, const int32_t* positions,
+                                     void* k_cache, void* v_cache, void* stream);
+
+/*
+ * starkv_decode_workspace_bytes -- device scratch needed by starkv_paged_decode
+ * for this layer geometry, batch size and length bound (0 on invalid input).
+ * Depends on the SM count of the current device.
+ */
+size_t starkv_decode_workspace_bytes(const starkv_layer_desc* desc, int32_t batch,
+                                     int32_t max_seq_len);
+
+/*
+ * starkv_paged_decode -- single-token decode attention from the paged codes.
+ *
+ *   q             fp16 [batch][H][d]
+ *   B_K           fp16 [H][r][d]
+ *   B_V           fp16 [R][H*d]
+ *   k_cache       fp16 [num_blocks][16][H][r]
+ *   v_cache       fp16 [num_blocks][16][R]
+ *   block_tables  int32 [batch][max_blocks_per_seq]
+ *   seq_lens      int32 [batch]: tokens to attend over (after any append)
+ *   max_seq_len   host-side upper bound of every seq_lens[b]
+ *                 (<= max_blocks_per_seq*16); sizes grids and scratch
+ *   scale         softmax scale (normally 1/sqrt(head_dim)); finite, > 0
+ *   workspace     device scratch of at least starkv_decode_workspace_bytes()
+ *                 bytes, 256-byte aligned; contents on entry are ignored
+ *   out           fp16 [batch][H][d]
+ *
+ * Slots at or past seq_lens[b] are never read.  seq_lens[b] == 0 gives a zero
+ * output row.  Accumulation is fp32; attention weights enter the V contraction
+ * as fp16.  Calls that share a workspace must be ordered on one stream.
+ */
+starkv_status starkv_paged_decode(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len,
+                                  const void* q, const void* B_K, const void* B_V,
+                                  const void* k_cache, const void* v_cache,
+                                  const int32_t* block_tables, const int32_t* seq_lens, float scale,
+                                  void* workspace, size_t workspace_bytes, void* out, void* stream);
+
+/*
+ * starkv_paged_decode_profiled -- starkv_paged_decode that also records CUDA
+ * events on `stream` around its kernels, for per-kernel timing.
+ * stage_events: HOST array of 6 cudaEvent_t (as void*; a NULL entry is
+ * skipped) recorded before the query absorption, after it, after the K pass,
+ * after the split reduction, after the V pass and after the up-projection.
+ * The events are not recorded when the call returns an error before launching
+ * or when max_seq_len == 0.  Otherwise identical to starkv_paged_decode.
+ */
+starkv_status starkv_paged_decode_profiled(const starkv_layer_desc* desc, int32_t batch,
+                                           int32_t max_seq_len, const void* q, const void* B_K,
+                                           const void* B_V, const void* k_cache, const void* v_cache,
+                                           const int32_t* block_tables, const int32_t* seq_lens,
+                                           float scale, void* workspace, size_t workspace_bytes,
+                                           void* out, void* stream, void* const* stage_events);
+
+/*
+ * starkv_decode_check -- synchronise `stream` and read the device status word
+ * the last decode on `workspace` left.  *flags_out receives STARKV_FLAG_* bits
+ * (0 when clean).  Returns STARKV_OK when clean, STARKV_ERR_TIMEOUT when the
+ * timeout bit is set, STARKV_ERR_DEVICE_CHECK for other bits.
+ */
+starkv_status starkv_decode_check(const void* workspace, void* stream, int32_t* flags_out);
+
+/*
+ * Workspace layout (byte offsets into the decode workspace), exposed so that
+ * tests can inspect intermediate results.  Values for one (desc, batch,
+ * max_seq_len) on the current device.
+ */
+typedef struct {
+  size_t total_bytes;
+  size_t status_off;  /* int32 status word */
+  size_t prefix_off;  /* int32 [batch+1] prefix sums of pages per sequence */
+  size_t qt_off;      /* fp32 [batch][H][r]: log2(e)*scale*q.B_K^T */
+  size_t logits_off;  /* fp32 [batch][t_pad][H]: base-2 logits s*log2(e) */
+  size_t ml_off;      /* fp32 [k_slots][H][2]: per-segment (max, sum exp2) */
+  size_t stats_off;   /* fp32 [batch][H][2]: (global max, 1/sum) */
+  size_t zpart_off;   /* fp32 [n_rranges][v_slots][H][r_range]: partial sum_t p c_V */
+  int32_t t_pad;      /* logits row capacity (multiple of 16) */
+  int32_t k_ctas;     /* CTAs of the K pass (stream partition) */
+  int32_t k_slots;    /* k_ctas + batch */
+  int32_t v_ctas;     /* CTAs of the V pass per R range */
+  int32_t v_slots;    /* v_ctas + batch */
+  int32_t n_rranges;  /* R ranges of the V pass */
+  int32_t r_range;    /* V rank handled per R range */
+} starkv_workspace_layout;
+
+starkv_status starkv_decode_workspace_layout(const starkv_layer_desc* desc, int32_t batch,
+                                             int32_t max_seq_len, starkv_workspace_layout* out);
+
+/* Human-readable name of a status code (static storage). */
+const char* starkv_status_string(starkv_status status);
+
+/*
+ * starkv_rank_from_spectrum -- adaptive rank by soft-thresholding: the number
+ * of singular values strictly greater than tau ("learned soft-thresholding for
+ * adaptive rank control", README opening line).  Host function; s is a HOST
+ * array of n doubles (n >= 0, s may be NULL when n == 0).  Returns -1 on
+ * invalid input.
+ */
+int32_t starkv_rank_from_spectrum(const double* s, int32_t n, double tau);
+
+/* Library version, 10000*major + 100*minor + patch. */
+int32_t starkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STARKV_H_ */

@@ -1,0 +1,195 @@
+"""Python binding of libstarkv (STAR-KV paged low-rank decode on sm_100a).
+
+Argument marshalling only: every function forwards to the C entry point of the
+same name in ``libstarkv.so`` (declared in ``include/starkv.h``).  Tensor
+arguments may be torch tensors (their ``data_ptr()`` is passed) or raw integer
+device addresses; ``stream`` may be a ``torch.cuda.Stream``, a raw
+``cudaStream_t`` integer or ``None`` (the current torch stream).  There is no
+fallback: if the shared library cannot be loaded, importing the functions
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libstarkv.so")
+
+STATUS = {
+    0: "STARKV_OK", 1: "STARKV_ERR_INVALID_ARG", 2: "STARKV_ERR_UNSUPPORTED",
+    3: "STARKV_ERR_WORKSPACE", 4: "STARKV_ERR_CUDA", 5: "STARKV_ERR_DEVICE_CHECK",
+    6: "STARKV_ERR_TIMEOUT",
+}
+FLAG_BAD_BLOCK_ID, FLAG_BAD_SEQ_LEN, FLAG_TIMEOUT = 1, 2, 4
+
+EXPORTED = (
+    "starkv_compress_append", "starkv_decode_workspace_bytes", "starkv_paged_decode",
+    "starkv_paged_decode_profiled",
+    "starkv_decode_check", "starkv_decode_workspace_layout", "starkv_status_string",
+    "starkv_rank_from_spectrum", "starkv_version",
+)
+
+
+class StarkvError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class LayerDesc(ctypes.Structure):
+    _fields_ = [("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("k_rank", ctypes.c_int32), ("v_rank", ctypes.c_int32),
+                ("block_size", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
+                ("max_blocks_per_seq", ctypes.c_int32)]
+
+
+class WorkspaceLayout(ctypes.Structure):
+    _fields_ = [("total_bytes", ctypes.c_size_t), ("status_off", ctypes.c_size_t),
+                ("prefix_off", ctypes.c_size_t), ("qt_off", ctypes.c_size_t),
+                ("logits_off", ctypes.c_size_t), ("ml_off", ctypes.c_size_t),
+                ("stats_off", ctypes.c_size_t), ("zpart_off", ctypes.c_size_t),
+                ("t_pad", ctypes.c_int32), ("k_ctas", ctypes.c_int32), ("k_slots", ctypes.c_int32),
+                ("v_ctas", ctypes.c_int32), ("v_slots", ctypes.c_int32),
+                ("n_rranges", ctypes.c_int32), ("r_range", ctypes.c_int32)]
+
+
+def layer_desc(num_heads, head_dim, k_rank, v_rank, num_blocks, max_blocks_per_seq,
+               block_size=16) -> LayerDesc:
+    return LayerDesc(num_heads, head_dim, k_rank, v_rank, block_size, num_blocks,
+                     max_blocks_per_seq)
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libstarkv.so (raises OSError when it is missing: no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise OSError(f"libstarkv.so not found at {path}; build it with "
+                      "`python -m rank_compressed_kv_star_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    DP = ctypes.POINTER(LayerDesc)
+    lib.starkv_compress_append.argtypes = [DP, I32, P, P, P, P, P, P, P, P, P]
+    lib.starkv_compress_append.restype = ctypes.c_int
+    lib.starkv_decode_workspace_bytes.argtypes = [DP, I32, I32]
+    lib.starkv_decode_workspace_bytes.restype = SZ
+    lib.starkv_paged_decode.argtypes = [DP, I32, I32, P, P, P, P, P, P, P, ctypes.c_float,
+                                        P, SZ, P, P]
+    lib.starkv_paged_decode.restype = ctypes.c_int
+    lib.starkv_paged_decode_profiled.argtypes = [DP, I32, I32, P, P, P, P, P, P, P, ctypes.c_float,
+                                                 P, SZ, P, P, ctypes.POINTER(P)]
+    lib.starkv_paged_decode_profiled.restype = ctypes.c_int
+    lib.starkv_decode_check.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
+    lib.starkv_decode_check.restype = ctypes.c_int
+    lib.starkv_decode_workspace_layout.argtypes = [DP, I32, I32, ctypes.POINTER(WorkspaceLayout)]
+    lib.starkv_decode_workspace_layout.restype = ctypes.c_int
+    lib.starkv_status_string.argtypes = [ctypes.c_int]
+    lib.starkv_status_string.restype = ctypes.c_char_p
+    lib.starkv_rank_from_spectrum.argtypes = [ctypes.POINTER(ctypes.c_double), I32, ctypes.c_double]
+    lib.starkv_rank_from_spectrum.restype = I32
+    lib.starkv_version.argtypes = []
+    lib.starkv_version.restype = I32
+    _lib = lib
+    return lib
+
+
+def _desc_ref(desc):
+    return ctypes.byref(desc) if desc is not None else None
+
+
+def _ptr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise StarkvError(status, where)
+
+
+def starkv_compress_append(desc: LayerDesc, batch: int, k, v, A_K, A_V, block_tables, positions,
+                           k_cache, v_cache, stream=None, check: bool = True) -> int:
+    st = load_library().starkv_compress_append(
+        _desc_ref(desc), batch, _ptr(k), _ptr(v), _ptr(A_K), _ptr(A_V), _ptr(block_tables),
+        _ptr(positions), _ptr(k_cache), _ptr(v_cache), _stream(stream))
+    if check:
+        _check(st, "starkv_compress_append")
+    return st
+
+
+def starkv_decode_workspace_bytes(desc: LayerDesc, batch: int, max_seq_len: int) -> int:
+    return int(load_library().starkv_decode_workspace_bytes(_desc_ref(desc), batch, max_seq_len))
+
+
+def starkv_decode_workspace_layout(desc: LayerDesc, batch: int, max_seq_len: int) -> WorkspaceLayout:
+    out = WorkspaceLayout()
+    _check(load_library().starkv_decode_workspace_layout(_desc_ref(desc), batch, max_seq_len,
+                                                         ctypes.byref(out)),
+           "starkv_decode_workspace_layout")
+    return out
+
+
+def starkv_paged_decode(desc: LayerDesc, batch: int, max_seq_len: int, q, B_K, B_V, k_cache,
+                        v_cache, block_tables, seq_lens, scale: float, workspace,
+                        workspace_bytes: int, out, stream=None, check: bool = True) -> int:
+    st = load_library().starkv_paged_decode(
+        _desc_ref(desc), batch, max_seq_len, _ptr(q), _ptr(B_K), _ptr(B_V), _ptr(k_cache),
+        _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), float(scale), _ptr(workspace),
+        int(workspace_bytes), _ptr(out), _stream(stream))
+    if check:
+        _check(st, "starkv_paged_decode")
+    return st
+
+
+def starkv_paged_decode_profiled(desc: LayerDesc, batch: int, max_seq_len: int, q, B_K, B_V,
+                                 k_cache, v_cache, block_tables, seq_lens, scale: float, workspace,
+                                 workspace_bytes: int, out, stage_events, stream=None,
+                                 check: bool = True) -> int:
+    """``stage_events``: six ``torch.cuda.Event`` (or raw cudaEvent_t ints / None)."""
+    raw = [None if e is None else (e if isinstance(e, int) else e.cuda_event) for e in stage_events]
+    arr = (ctypes.c_void_p * 6)(*raw)
+    st = load_library().starkv_paged_decode_profiled(
+        _desc_ref(desc), batch, max_seq_len, _ptr(q), _ptr(B_K), _ptr(B_V), _ptr(k_cache),
+        _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), float(scale), _ptr(workspace),
+        int(workspace_bytes), _ptr(out), _stream(stream), arr)
+    if check:
+        _check(st, "starkv_paged_decode_profiled")
+    return st
+
+
+def starkv_decode_check(workspace, stream=None) -> tuple[int, int]:
+    """Returns (status, flags) after synchronising the stream."""
+    flags = ctypes.c_int32(0)
+    st = load_library().starkv_decode_check(_ptr(workspace), _stream(stream), ctypes.byref(flags))
+    return st, flags.value
+
+
+def starkv_status_string(status: int) -> str:
+    return load_library().starkv_status_string(status).decode()
+
+
+def starkv_rank_from_spectrum(s, tau: float) -> int:
+    vals = [float(x) for x in s]
+    arr = (ctypes.c_double * len(vals))(*vals) if vals else None
+    return int(load_library().starkv_rank_from_spectrum(arr, len(vals), float(tau)))
+
+
+def starkv_version() -> int:
+    return int(load_library().starkv_version())

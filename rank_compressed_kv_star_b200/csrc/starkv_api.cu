@@ -1,0 +1,436 @@
+// C-ABI entry points of libstarkv: argument validation, launch planning,
+// workspace layout and launch sequencing on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/starkv.h"
+#include "append_kernels.cuh"
+#include "decode_kernels.cuh"
+
+namespace starkv {
+namespace {
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return 148; }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int pow2_ceil(int x) { int p = 1; while (p < x) p <<= 1; return p; }
+
+starkv_status check_desc(const starkv_layer_desc* d) {
+  if (!d) return STARKV_ERR_INVALID_ARG;
+  if (d->num_heads <= 0 || d->head_dim <= 0 || d->k_rank <= 0 || d->v_rank <= 0 || d->num_blocks <= 0 ||
+      d->max_blocks_per_seq <= 0)
+    return STARKV_ERR_INVALID_ARG;
+  if (d->block_size != 16) return STARKV_ERR_UNSUPPORTED;
+  if (!is_pow2(d->num_heads) || d->num_heads > 64) return STARKV_ERR_UNSUPPORTED;
+  if (!(d->head_dim == 32 || d->head_dim == 64 || d->head_dim == 128 || d->head_dim == 256))
+    return STARKV_ERR_UNSUPPORTED;
+  if (d->k_rank % 16 != 0 || d->k_rank > 256) return STARKV_ERR_UNSUPPORTED;
+  if (d->v_rank % 64 != 0 || d->v_rank > 8192) return STARKV_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(d->num_blocks) * 16 > INT32_MAX) return STARKV_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(d->max_blocks_per_seq) * 16 > INT32_MAX) return STARKV_ERR_UNSUPPORTED;
+  return STARKV_OK;
+}
+
+// ------------------------------------------------------------------ planning
+struct DecodePlan {
+  int H, d, r, R, B, MB, NB, cap, n_pages_max, t_pad, npad;
+  // K pass
+  int L, CPL, tps, k_stages, k_ctas;
+  uint32_t k_stage_bytes;
+  size_t k_smem;
+  // V pass
+  int n_rr, r_range, r_range_pad, n_chunks, n_mtiles, v_stages, v_ctas, v_per_sm;
+  uint32_t vtile, ltile, ptile, tmem_cols;
+  size_t v_smem;
+  // up-projection
+  int bpt;
+  starkv_workspace_layout ws;
+};
+
+void plan_kpass_shape(int r, int* L, int* CPL) {
+  const int cp = r / 8;
+  if (cp == 2) { *L = 2; *CPL = 1; }
+  else if (cp == 4) { *L = 4; *CPL = 1; }
+  else if (cp <= 8) { *L = 8; *CPL = 1; }
+  else if (cp == 12) { *L = 4; *CPL = 3; }
+  else if (cp <= 16) { *L = 8; *CPL = 2; }
+  else if (cp <= 24) { *L = 8; *CPL = 3; }
+  else { *L = 8; *CPL = 4; }
+}
+
+starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_seq_len, DecodePlan* pl) {
+  starkv_status st = check_desc(d);
+  if (st != STARKV_OK) return st;
+  if (batch < 0 || max_seq_len < 0) return STARKV_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(max_seq_len) > static_cast<int64_t>(d->max_blocks_per_seq) * 16)
+    return STARKV_ERR_INVALID_ARG;
+  DecodePlan& p = *pl;
+  std::memset(&p, 0, sizeof(p));
+  p.H = d->num_heads; p.d = d->head_dim; p.r = d->k_rank; p.R = d->v_rank;
+  p.B = batch; p.MB = d->max_blocks_per_seq; p.NB = d->num_blocks;
+  p.cap = max_seq_len;
+  p.n_pages_max = (max_seq_len + 15) / 16;
+  p.t_pad = p.n_pages_max * 16;
+  p.npad = p.H < 16 ? 16 : p.H;
+  const int sms = device_sm_count();
+
+  // K pass: ~32 KiB ring stages of whole tokens, ~200 KiB of ring, one CTA per SM
+  plan_kpass_shape(p.r, &p.L, &p.CPL);
+  const uint32_t tok = static_cast<uint32_t>(p.H) * p.r * 2;
+  p.tps = 16;
+  while (p.tps > 1 && p.tps * tok > 32768u) p.tps >>= 1;
+  p.k_stage_bytes = p.tps * tok;
+  p.k_stages = static_cast<int>(200u * 1024u / p.k_stage_bytes);
+  if (p.k_stages > 8) p.k_stages = 8;
+  if (p.k_stages < 2) p.k_stages = 2;
+  p.k_smem = static_cast<size_t>(p.k_stages) * p.k_stage_bytes + p.k_stages * sizeof(StageMeta) +
+             2 * p.k_stages * sizeof(uint64_t) + (kKConsumers / p.L) * sizeof(float2);
+  p.k_ctas = sms;
+
+  // V pass: R split into ranges of <= 1024 rows (128-row UMMA tiles)
+  if (p.R <= 1024) { p.n_rr = 1; p.r_range = p.R; }
+  else {
+    p.n_rr = (p.R + 1023) / 1024;
+    p.r_range = ((p.R + p.n_rr - 1) / p.n_rr + 127) / 128 * 128;
+  }
+  p.r_range_pad = (p.r_range + 127) / 128 * 128;
+  p.n_chunks = p.r_range_pad / 64;
+  p.n_mtiles = p.r_range_pad / 128;
+  p.vtile = static_cast<uint32_t>(p.r_range_pad) * 16 * 2;
+  p.ltile = 16u * p.H * 4;
+  p.ptile = static_cast<uint32_t>(p.npad) * 16 * 2;
+  p.tmem_cols = static_cast<uint32_t>(pow2_ceil(p.n_mtiles * p.npad < 32 ? 32 : p.n_mtiles * p.npad));
+  const uint32_t stage = p.vtile + p.ltile + p.ptile;
+  p.v_stages = static_cast<int>((105u * 1024u) / stage);
+  if (p.v_stages > 8) p.v_stages = 8;
+  if (p.v_stages < 2) p.v_stages = 2;
+  p.v_smem = 1024 + static_cast<size_t>(p.v_stages) * stage + p.v_stages * sizeof(StageMeta) +
+             (3 * p.v_stages + 3) * sizeof(uint64_t) + 2 * p.npad * sizeof(float);
+  int per_sm = static_cast<int>((227u * 1024u) / (p.v_smem + 1024));
+  if (per_sm > static_cast<int>(512 / p.tmem_cols)) per_sm = 512 / p.tmem_cols;
+  if (per_sm < 1) per_sm = 1;
+  if (per_sm > 2) per_sm = 2;
+  p.v_per_sm = per_sm;
+  p.v_ctas = sms * per_sm / p.n_rr;
+  if (p.v_ctas < 1) p.v_ctas = 1;
+
+  p.bpt = kUpBT * (p.d / 2) / 256;
+
+  // workspace layout
+  starkv_workspace_layout& w = p.ws;
+  size_t off = 0;
+  w.status_off = off; off += 256;
+  w.prefix_off = off; off = align_up(off + (static_cast<size_t>(batch) + 1) * 4, 256);
+  const size_t teff_off = off; off = align_up(off + static_cast<size_t>(batch) * 4, 256);
+  (void)teff_off;
+  w.qt_off = off; off = align_up(off + static_cast<size_t>(batch) * p.H * p.r * 4, 256);
+  w.logits_off = off; off = align_up(off + static_cast<size_t>(batch) * p.t_pad * p.H * 4, 256);
+  w.k_ctas = p.k_ctas;
+  w.k_slots = p.k_ctas + batch;
+  w.ml_off = off; off = align_up(off + static_cast<size_t>(w.k_slots) * p.H * 2 * 4, 256);
+  w.stats_off = off; off = align_up(off + static_cast<size_t>(batch) * p.H * 2 * 4, 256);
+  w.v_ctas = p.v_ctas;
+  w.v_slots = p.v_ctas + batch;
+  w.n_rranges = p.n_rr;
+  w.r_range = p.r_range;
+  w.zpart_off = off;
+  off = align_up(off + static_cast<size_t>(p.n_rr) * w.v_slots * p.H * p.r_range * 4, 256);
+  w.t_pad = p.t_pad;
+  w.total_bytes = off;
+  return STARKV_OK;
+}
+
+size_t teff_offset(const DecodePlan& p) {
+  return align_up(p.ws.prefix_off + (static_cast<size_t>(p.B) + 1) * 4, 256);
+}
+
+// ------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// V pool viewed as a 2-D matrix [num_blocks*16 rows][R] of fp16; boxes of
+// 64 columns x 16 rows (one page, one 128-byte-wide chunk) with 128B swizzle.
+bool encode_vpool_map(CUtensorMap* map, const void* v_cache, int R, int NB) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(R), static_cast<cuuint64_t>(NB) * 16};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(R) * 2};
+  cuuint32_t box[2] = {64, 16};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(v_cache), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------ kernel attributes
+template <typename K>
+bool set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) ==
+         cudaSuccess;
+}
+
+template <int L, int CPL>
+cudaError_t launch_kpass(const DecodePlan& pl, const KPassParams& kp, cudaStream_t s) {
+  if (!set_smem(kpass_kernel<L, CPL>, pl.k_smem)) return cudaGetLastError();
+  kpass_kernel<L, CPL><<<pl.k_ctas, kKThreads, pl.k_smem, s>>>(kp);
+  return cudaGetLastError();
+}
+
+template <int BPT>
+cudaError_t launch_upproj(const DecodePlan& pl, const UpProjParams& up, cudaStream_t s) {
+  dim3 grid(pl.H, (pl.B + kUpBT - 1) / kUpBT);
+  upproj_kernel<BPT><<<grid, 256, 0, s>>>(up);
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace starkv
+
+using namespace starkv;
+
+extern "C" {
+
+const char* starkv_status_string(starkv_status s) {
+  switch (s) {
+    case STARKV_OK: return "STARKV_OK";
+    case STARKV_ERR_INVALID_ARG: return "STARKV_ERR_INVALID_ARG";
+    case STARKV_ERR_UNSUPPORTED: return "STARKV_ERR_UNSUPPORTED";
+    case STARKV_ERR_WORKSPACE: return "STARKV_ERR_WORKSPACE";
+    case STARKV_ERR_CUDA: return "STARKV_ERR_CUDA";
+    case STARKV_ERR_DEVICE_CHECK: return "STARKV_ERR_DEVICE_CHECK";
+    case STARKV_ERR_TIMEOUT: return "STARKV_ERR_TIMEOUT";
+  }
+  return "STARKV_UNKNOWN_STATUS";
+}
+
+int32_t starkv_version(void) { return 100; }
+
+int32_t starkv_rank_from_spectrum(const double* s, int32_t n, double tau) {
+  if (n < 0 || (n > 0 && !s) || std::isnan(tau)) return -1;
+  int32_t c = 0;
+  for (int32_t i = 0; i < n; ++i)
+    if (s[i] > tau) ++c;
+  return c;
+}
+
+starkv_status starkv_compress_append(const starkv_layer_desc* desc, int32_t batch, const void* k, const void* v,
+                                     const void* A_K, const void* A_V, const int32_t* block_tables,
+                                     const int32_t* positions, void* k_cache, void* v_cache, void* stream) {
+  starkv_status st = check_desc(desc);
+  if (st != STARKV_OK) return st;
+  if (batch < 0) return STARKV_ERR_INVALID_ARG;
+  if (batch == 0) return STARKV_OK;
+  if (!k || !v || !A_K || !A_V || !block_tables || !positions || !k_cache || !v_cache)
+    return STARKV_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(A_K) || !aligned16(A_V) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+      (reinterpret_cast<uintptr_t>(positions) & 3u))
+    return STARKV_ERR_INVALID_ARG;
+  if (desc->k_rank > 256) return STARKV_ERR_UNSUPPORTED;
+  AppendParams p;
+  p.k = static_cast<const __half*>(k);
+  p.v = static_cast<const __half*>(v);
+  p.A_K = static_cast<const __half*>(A_K);
+  p.A_V = static_cast<const __half*>(A_V);
+  p.tables = block_tables;
+  p.positions = positions;
+  p.k_cache = static_cast<__half*>(k_cache);
+  p.v_cache = static_cast<__half*>(v_cache);
+  p.B = batch; p.H = desc->num_heads; p.d = desc->head_dim; p.r = desc->k_rank; p.R = desc->v_rank;
+  p.MB = desc->max_blocks_per_seq; p.NB = desc->num_blocks;
+  p.nvx = p.R / kAppNC;
+  p.nby = (batch + kAppBT - 1) / kAppBT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  append_kernel<<<p.nvx * p.nby + p.H, 256, 0, s>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
+  return STARKV_OK;
+}
+
+size_t starkv_decode_workspace_bytes(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len) {
+  DecodePlan pl;
+  if (make_plan(desc, batch, max_seq_len, &pl) != STARKV_OK) return 0;
+  return pl.ws.total_bytes;
+}
+
+starkv_status starkv_decode_workspace_layout(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len,
+                                             starkv_workspace_layout* out) {
+  if (!out) return STARKV_ERR_INVALID_ARG;
+  DecodePlan pl;
+  starkv_status st = make_plan(desc, batch, max_seq_len, &pl);
+  if (st != STARKV_OK) return st;
+  *out = pl.ws;
+  return STARKV_OK;
+}
+
+namespace {
+starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len, const void* q,
+                          const void* B_K, const void* B_V, const void* k_cache, const void* v_cache,
+                          const int32_t* block_tables, const int32_t* seq_lens, float scale, void* workspace,
+                          size_t workspace_bytes, void* out, void* stream, void* const* stage_events) {
+  DecodePlan pl;
+  starkv_status st = make_plan(desc, batch, max_seq_len, &pl);
+  if (st != STARKV_OK) return st;
+  if (!(std::isfinite(scale) && scale > 0.f)) return STARKV_ERR_INVALID_ARG;
+  if (batch == 0) return STARKV_OK;
+  if (!q || !B_K || !B_V || !k_cache || !v_cache || !block_tables || !seq_lens || !out)
+    return STARKV_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(B_K) || !aligned16(B_V) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(out) || (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return STARKV_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < pl.ws.total_bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return STARKV_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* status = reinterpret_cast<int32_t*>(ws + pl.ws.status_off);
+  int32_t* prefix = reinterpret_cast<int32_t*>(ws + pl.ws.prefix_off);
+  int32_t* teff = reinterpret_cast<int32_t*>(ws + teff_offset(pl));
+  float* qt = reinterpret_cast<float*>(ws + pl.ws.qt_off);
+  float* logits = reinterpret_cast<float*>(ws + pl.ws.logits_off);
+  float* ml = reinterpret_cast<float*>(ws + pl.ws.ml_off);
+  float* stats = reinterpret_cast<float*>(ws + pl.ws.stats_off);
+  float* zpart = reinterpret_cast<float*>(ws + pl.ws.zpart_off);
+
+  if (max_seq_len == 0) {
+    if (cudaMemsetAsync(status, 0, 4, s) != cudaSuccess ||
+        cudaMemsetAsync(out, 0, static_cast<size_t>(batch) * pl.H * pl.d * 2, s) != cudaSuccess)
+      return STARKV_ERR_CUDA;
+    return STARKV_OK;
+  }
+
+  CUtensorMap vmap;
+  if (!encode_vpool_map(&vmap, v_cache, pl.R, pl.NB)) return STARKV_ERR_CUDA;
+  auto mark = [&](int i) {
+    if (stage_events && stage_events[i]) cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), s);
+  };
+  mark(0);
+
+  AbsorbParams ap;
+  ap.q = static_cast<const __half*>(q);
+  ap.B_K = static_cast<const __half*>(B_K);
+  ap.seq_lens = seq_lens;
+  ap.qt = qt; ap.prefix = prefix; ap.teff = teff; ap.status = status;
+  ap.B = batch; ap.H = pl.H; ap.d = pl.d; ap.r = pl.r; ap.cap = pl.cap;
+  ap.coef = scale * kLog2e;
+  absorb_kernel<<<pl.H, 256, 0, s>>>(ap);
+  if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
+  mark(1);
+
+  KPassParams kp;
+  kp.k_cache = static_cast<const __half*>(k_cache);
+  kp.tables = block_tables; kp.teff = teff; kp.prefix = prefix; kp.qt = qt;
+  kp.logits = logits; kp.ml = ml; kp.status = status;
+  kp.B = batch; kp.H = pl.H; kp.r = pl.r; kp.MB = pl.MB; kp.NB = pl.NB; kp.t_pad = pl.t_pad;
+  kp.tps = pl.tps; kp.stages = pl.k_stages; kp.stage_bytes = pl.k_stage_bytes;
+  cudaError_t e;
+  if (pl.L == 2) e = launch_kpass<2, 1>(pl, kp, s);
+  else if (pl.L == 4 && pl.CPL == 1) e = launch_kpass<4, 1>(pl, kp, s);
+  else if (pl.L == 4) e = launch_kpass<4, 3>(pl, kp, s);
+  else if (pl.CPL == 1) e = launch_kpass<8, 1>(pl, kp, s);
+  else if (pl.CPL == 2) e = launch_kpass<8, 2>(pl, kp, s);
+  else if (pl.CPL == 3) e = launch_kpass<8, 3>(pl, kp, s);
+  else e = launch_kpass<8, 4>(pl, kp, s);
+  if (e != cudaSuccess) return STARKV_ERR_CUDA;
+  mark(2);
+
+  ReduceParams rp;
+  rp.ml = ml; rp.prefix = prefix; rp.stats = stats;
+  rp.B = batch; rp.H = pl.H; rp.k_grid = pl.k_ctas;
+  reduce_kernel<<<(batch * pl.H + 255) / 256, 256, 0, s>>>(rp);
+  if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
+  mark(3);
+
+  VPassParams vp;
+  vp.tables = block_tables; vp.teff = teff; vp.prefix = prefix; vp.logits = logits; vp.stats = stats;
+  vp.zpart = zpart; vp.status = status;
+  vp.B = batch; vp.H = pl.H; vp.npad = pl.npad; vp.MB = pl.MB; vp.NB = pl.NB; vp.R = pl.R;
+  vp.t_pad = pl.t_pad; vp.r_range = pl.r_range; vp.n_rr = pl.n_rr; vp.v_slots = pl.ws.v_slots;
+  vp.stages = pl.v_stages; vp.n_chunks = pl.n_chunks; vp.n_mtiles = pl.n_mtiles; vp.tmem_cols = pl.tmem_cols;
+  vp.vtile_bytes = pl.vtile; vp.ltile_bytes = pl.ltile; vp.ptile_bytes = pl.ptile;
+  if (!set_smem(vpass_kernel, pl.v_smem)) return STARKV_ERR_CUDA;
+  vpass_kernel<<<dim3(pl.v_ctas, pl.n_rr), kVThreads, pl.v_smem, s>>>(vmap, vp);
+  if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
+  mark(4);
+
+  UpProjParams up;
+  up.zpart = zpart; up.prefix = prefix;
+  up.B_V = static_cast<const __half*>(B_V);
+  up.out = static_cast<__half*>(out);
+  up.B = batch; up.H = pl.H; up.d = pl.d; up.R = pl.R; up.r_range = pl.r_range; up.v_slots = pl.ws.v_slots;
+  up.v_grid = pl.v_ctas;
+  if (pl.bpt == 1) e = launch_upproj<1>(pl, up, s);
+  else if (pl.bpt == 2) e = launch_upproj<2>(pl, up, s);
+  else if (pl.bpt == 4) e = launch_upproj<4>(pl, up, s);
+  else e = launch_upproj<8>(pl, up, s);
+  if (e != cudaSuccess) return STARKV_ERR_CUDA;
+  mark(5);
+  return STARKV_OK;
+}
+}  // namespace
+
+starkv_status starkv_paged_decode(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len,
+                                  const void* q, const void* B_K, const void* B_V, const void* k_cache,
+                                  const void* v_cache, const int32_t* block_tables, const int32_t* seq_lens,
+                                  float scale, void* workspace, size_t workspace_bytes, void* out, void* stream) {
+  return decode_impl(desc, batch, max_seq_len, q, B_K, B_V, k_cache, v_cache, block_tables, seq_lens, scale,
+                     workspace, workspace_bytes, out, stream, nullptr);
+}
+
+starkv_status starkv_paged_decode_profiled(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len,
+                                           const void* q, const void* B_K, const void* B_V, const void* k_cache,
+                                           const void* v_cache, const int32_t* block_tables,
+                                           const int32_t* seq_lens, float scale, void* workspace,
+                                           size_t workspace_bytes, void* out, void* stream,
+                                           void* const* stage_events) {
+  return decode_impl(desc, batch, max_seq_len, q, B_K, B_V, k_cache, v_cache, block_tables, seq_lens, scale,
+                     workspace, workspace_bytes, out, stream, stage_events);
+}
+
+starkv_status starkv_decode_check(const void* workspace, void* stream, int32_t* flags_out) {
+  if (!workspace || !flags_out) return STARKV_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t flags = 0;
+  if (cudaMemcpyAsync(&flags, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return STARKV_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return STARKV_ERR_CUDA;
+  *flags_out = flags;
+  if (flags & STARKV_FLAG_TIMEOUT) return STARKV_ERR_TIMEOUT;
+  if (flags) return STARKV_ERR_DEVICE_CHECK;
+  return STARKV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,122 @@
+"""The C-ABI library without a GPU: it loads, exports every declared entry point
+and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import rank_compressed_kv_star_b200 as S
+from oracle import starkv_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from rank_compressed_kv_star_b200 import build
+    build.build()
+    return S.load_library()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "starkv.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(starkv_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(S.EXPORTED) <= set(names)
+
+
+def test_status_strings_and_version(lib):
+    for code, name in S.STATUS.items():
+        assert S.starkv_status_string(code) == name
+    assert S.starkv_version() >= 100
+
+
+def test_rank_from_spectrum_matches_oracle(lib):
+    rng = np.random.default_rng(0)
+    for _ in range(50):
+        s = np.sort(rng.random(rng.integers(0, 80)))[::-1]
+        tau = float(rng.random())
+        assert S.starkv_rank_from_spectrum(s, tau) == O.rank_from_spectrum(s, tau)
+    assert lib.starkv_rank_from_spectrum(None, -1, 0.0) == -1
+    assert S.starkv_rank_from_spectrum([1.0], float("nan")) == -1
+
+
+def _desc(**kw):
+    base = dict(num_heads=32, head_dim=128, k_rank=64, v_rank=2048, num_blocks=1000,
+                max_blocks_per_seq=64)
+    base.update(kw)
+    return S.layer_desc(**base)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(block_size=32), 2), (dict(num_heads=48), 2), (dict(head_dim=96), 2),
+    (dict(k_rank=40), 2), (dict(v_rank=100), 2), (dict(num_heads=0), 1), (dict(num_blocks=0), 1),
+    (dict(k_rank=272), 2), (dict(v_rank=8256), 2),
+])
+def test_descriptor_validation(lib, kw, expect):
+    d = _desc(**kw)
+    fake = 1 << 20
+    st = S.starkv_paged_decode(d, 1, 16, fake, fake, fake, fake, fake, fake, fake, 0.1, fake,
+                               1 << 30, fake, stream=0, check=False)
+    assert st == expect
+    assert S.starkv_decode_workspace_bytes(d, 1, 16) == 0
+    st = S.starkv_compress_append(d, 1, fake, fake, fake, fake, fake, fake, fake, fake, stream=0,
+                                  check=False)
+    assert st == expect
+
+
+def test_decode_argument_errors(lib):
+    d = _desc()
+    fake = 1 << 20
+    need = S.starkv_decode_workspace_bytes(d, 4, 1024)
+    assert need > 0
+    args = [d, 4, 1024, fake, fake, fake, fake, fake, fake, fake, 0.1, fake, need, fake]
+    def call(i, v):
+        a = list(args); a[i] = v
+        return S.starkv_paged_decode(*a, stream=0, check=False)
+    assert call(1, -1) == 1                      # negative batch
+    assert call(2, 64 * 16 + 1) == 1             # max_seq_len above table capacity
+    assert call(10, 0.0) == 1 and call(10, float("inf")) == 1
+    assert call(3, None) == 1                    # null q
+    assert call(3, fake + 2) == 1                # misaligned q
+    assert call(12, need - 1) == 3               # workspace too small
+    assert call(11, None) == 3                   # null workspace
+    assert call(11, fake + 128) == 3             # workspace not 256-byte aligned
+    assert S.starkv_paged_decode(None, 4, 1024, *args[3:], stream=0, check=False) == 1
+
+
+def test_append_argument_errors(lib):
+    d = _desc()
+    fake = 1 << 20
+    args = [d, 4, fake, fake, fake, fake, fake, fake, fake, fake]
+    for i in range(2, 10):
+        a = list(args); a[i] = None
+        assert S.starkv_compress_append(*a, stream=0, check=False) == 1
+    a = list(args); a[1] = -3
+    assert S.starkv_compress_append(*a, stream=0, check=False) == 1
+    a = list(args); a[1] = 0
+    assert S.starkv_compress_append(*a, stream=0, check=False) == 0   # empty batch: no-op
+
+
+def test_workspace_layout_is_consistent(lib):
+    d = _desc(max_blocks_per_seq=600, num_blocks=40000)
+    lay = S.starkv_decode_workspace_layout(d, 64, 8192)
+    assert lay.total_bytes == S.starkv_decode_workspace_bytes(d, 64, 8192)
+    offs = [lay.status_off, lay.prefix_off, lay.qt_off, lay.logits_off, lay.ml_off, lay.stats_off,
+            lay.zpart_off]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert lay.t_pad == 8192 and lay.k_slots == lay.k_ctas + 64 and lay.v_slots == lay.v_ctas + 64
+    assert lay.n_rranges * lay.r_range >= 2048
+    assert lay.logits_off + 64 * 8192 * 32 * 4 <= lay.ml_off
+    # grows with batch and length
+    assert S.starkv_decode_workspace_bytes(d, 65, 8192) > lay.total_bytes
+    assert S.starkv_decode_workspace_bytes(d, 64, 8200) > lay.total_bytes

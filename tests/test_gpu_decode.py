@@ -1,0 +1,328 @@
+"""GPU parity of the C-ABI path against the CPU fp64 oracle (B200, sm_100a).
+
+Tolerances (stated for the fp16-output path with fp32 accumulation): for
+decode outputs, max |gpu - oracle| <= 2e-3 and relative L2 error <= 1e-3 over
+the compared rows.  Appended codes: placement and every untouched byte
+bit-exact; code values within one fp16 ulp of the fp64 code.  Paging
+invariances (page permutation, identity vs shuffled table) are bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import rank_compressed_kv_star_b200 as S
+from oracle import starkv_oracle as O
+from starkv_inputs import device as D, gen, workloads as W
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, REL_L2 = 2e-3, 1e-3
+
+
+def rel_l2(got, ref):
+    return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+def desc_of(L):
+    return S.layer_desc(L["H"], L["d"], L["r"], L["R"], L["nb"], L["tables"].shape[1])
+
+
+def run_decode(L, seq_lens=None, max_seq_len=None, q=None):
+    seq_lens = L["seq_lens"] if seq_lens is None else seq_lens
+    B = seq_lens.shape[0]
+    if max_seq_len is None:
+        max_seq_len = int(seq_lens.max().item()) if B else 0
+    desc = desc_of(L)
+    wsb = S.starkv_decode_workspace_bytes(desc, B, max_seq_len)
+    ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device="cuda")
+    out = torch.full((B, L["H"], L["d"]), float("nan"), dtype=torch.float16, device="cuda")
+    S.starkv_paged_decode(desc, B, max_seq_len, L["q"] if q is None else q, L["B_K"], L["B_V"],
+                          L["k_cache"], L["v_cache"], L["tables"], seq_lens, L["scale"], ws, wsb, out)
+    st, flags = S.starkv_decode_check(ws)
+    assert st == 0, (S.STATUS[st], flags)
+    return out.float().cpu().numpy().astype(np.float64), ws, desc
+
+
+def oracle_rows(wl, layer, L_host_q, A_np, bs, seq_lens, appended=None, q=None):
+    """fp64 oracle for sequences `bs` (codes regenerated on the host)."""
+    A_K, A_V, B_K, B_V = A_np
+    qn = L_host_q if q is None else q
+    out = {}
+    for b in bs:
+        T = int(seq_lens[b])
+        if T == 0:
+            out[b] = np.zeros(qn.shape[1:])
+            continue
+        ctx = int(wl.ctx_lens[b])
+        cK, cV = W.seq_codes(wl, layer, b, min(ctx, T))
+        cK, cV = cK.astype(np.float64), cV.astype(np.float64)
+        if T > ctx:  # the step's appended token (oracle's own fp16 codes)
+            aK, aV = appended
+            cK = np.concatenate([cK, aK[b][None].astype(np.float64)])
+            cV = np.concatenate([cV, aV[b][None].astype(np.float64)])
+        out[b] = O.attend_codes_reordered(qn[b], B_K, B_V, cK, cV, 1.0 / np.sqrt(qn.shape[2]))
+    return out
+
+
+def assert_close(got_rows, ref_rows):
+    g = np.stack([got_rows[b] for b in sorted(ref_rows)])
+    r = np.stack([ref_rows[b] for b in sorted(ref_rows)])
+    err = np.abs(g - r).max()
+    rl = rel_l2(g, r)
+    assert np.isfinite(g).all()
+    assert err <= MAX_ABS, err
+    assert rl <= REL_L2, rl
+    return err, rl
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built(cuda_ok):
+    from rank_compressed_kv_star_b200 import build
+    build.build()
+    build.build_inputs()
+    S.load_library()
+
+
+# ------------------------------------------------------------- generator twin
+
+def test_device_generator_matches_host_bits():
+    spec = gen.spectrum_f32(64)
+    for key, rows, row_len, off in [(gen.stream_key(1, 2), 37, 64 * 4, 0),
+                                    (gen.stream_key(9), 5, 2048, 123), (123456789, 3, 64, 1 << 20)]:
+        out = torch.empty(rows * row_len, dtype=torch.float16, device="cuda")
+        D.gen_codes(key, rows, row_len, torch.from_numpy(spec).cuda(), out, row_offset=off)
+        host = gen.codes_f16(key, rows, row_len, spec, row_offset=off)
+        assert np.array_equal(out.cpu().numpy().view(np.uint16), host.reshape(-1).view(np.uint16))
+
+
+def test_device_pools_match_host_pools():
+    wl = W.workload(1)
+    Lh = W.host_layer(wl, 0)
+    Ld = D.device_layer(wl, 0, tables=Lh["tables"], nb=Lh["nb"])
+    assert np.array_equal(Ld["k_cache"].cpu().numpy().view(np.uint16), Lh["k_cache"].view(np.uint16))
+    assert np.array_equal(Ld["v_cache"].cpu().numpy().view(np.uint16), Lh["v_cache"].view(np.uint16))
+
+
+# ------------------------------------------------------------------ decode
+
+def _full_check(wl, layer=0):
+    Lh = W.host_layer(wl, layer)
+    Ld = D.device_layer(wl, layer, tables=Lh["tables"], nb=Lh["nb"])
+    got, ws, desc = run_decode(Ld)
+    ref = O.decode_explicit(Lh["q"], Lh["B_K"], Lh["B_V"], Lh["k_cache"], Lh["v_cache"],
+                            Lh["tables"], Lh["seq_lens"], Lh["scale"])
+    err, rl = assert_close({b: got[b] for b in range(wl.batch)}, {b: ref[b] for b in range(wl.batch)})
+    return Lh, Ld, got, ws, desc, err, rl
+
+
+def test_decode_tiny_workload():
+    _full_check(W.workload(1))
+
+
+def test_decode_tiny_intermediates():
+    """Logits, softmax statistics and the weighted code sums against the oracle's stages."""
+    wl = W.workload(1)
+    Lh = W.host_layer(wl, 0)
+    Ld = D.device_layer(wl, 0, tables=Lh["tables"], nb=Lh["nb"])
+    got, ws, desc = run_decode(Ld)
+    lay = S.starkv_decode_workspace_layout(desc, wl.batch, wl.max_seq_len)
+    wsn = ws.cpu().numpy()
+    H, r, R = Lh["H"], Lh["r"], Lh["R"]
+    logits = wsn[lay.logits_off:].view(np.float32)[:wl.batch * lay.t_pad * H].reshape(wl.batch, lay.t_pad, H)
+    stats = wsn[lay.stats_off:].view(np.float32)[:wl.batch * H * 2].reshape(wl.batch, H, 2)
+    for b in range(wl.batch):
+        T = int(Lh["seq_lens"][b])
+        st = O.decode_stages(Lh["q"][b], Lh["B_K"], Lh["B_V"], O.gather(Lh["k_cache"], Lh["tables"][b], T),
+                             O.gather(Lh["v_cache"], Lh["tables"][b], T), Lh["scale"])
+        s2 = st["s"] * np.log2(np.e)             # base-2 logits [H][T]
+        np.testing.assert_allclose(logits[b, :T].T, s2, rtol=0, atol=1e-4)
+        M = s2.max(axis=1)
+        Lsum = np.exp2(s2 - M[:, None]).sum(axis=1)
+        np.testing.assert_allclose(stats[b, :, 0], M, rtol=0, atol=1e-4)
+        np.testing.assert_allclose(stats[b, :, 1], 1.0 / Lsum, rtol=1e-4)
+
+
+def test_decode_ragged_multitile():
+    sh = W.LayerShape(32, 128, 64, 2048)
+    wl = W.custom("ragged", 2024, sh, [1, 15, 16, 17, 300, 0, 1000], append=False)
+    _full_check(wl)
+
+
+@pytest.mark.parametrize("r,R", [(32, 1024), (96, 3072), (16, 64), (128, 512)])
+def test_decode_rank_variants(r, R):
+    sh = W.LayerShape(32, 128, r, R)
+    wl = W.custom(f"r{r}", 300 + r, sh, [5, 33, 160, 511], append=False)
+    _full_check(wl)
+
+
+def test_decode_small_heads_and_dims():
+    sh = W.LayerShape(8, 64, 32, 256)
+    wl = W.custom("h8", 55, sh, [3, 64, 129], append=False)
+    _full_check(wl)
+
+
+def test_decode_empty_and_zero_batch():
+    sh = W.LayerShape(32, 128, 64, 2048)
+    wl = W.custom("empties", 7, sh, [0, 0, 40, 0], append=False)
+    Lh, Ld, got, *_ = _full_check(wl)
+    assert np.array_equal(got[[0, 1, 3]], np.zeros_like(got[[0, 1, 3]]))
+    # batch 0 and max_seq_len 0 are accepted and launch nothing / zero the output
+    z = torch.zeros(0, dtype=torch.int32, device="cuda")
+    run_decode(Ld, seq_lens=z, max_seq_len=0)
+    zeros4 = torch.zeros(4, dtype=torch.int32, device="cuda")
+    out, *_ = run_decode(Ld, seq_lens=zeros4, max_seq_len=0)
+    assert np.array_equal(out, np.zeros_like(out))
+
+
+def test_decode_page_permutation_bit_identical():
+    sh = W.LayerShape(32, 128, 64, 2048)
+    wl = W.custom("perm", 91, sh, [77, 300, 1, 129], append=False)
+    Lh = W.host_layer(wl, 0)
+    Ld = D.device_layer(wl, 0, tables=Lh["tables"], nb=Lh["nb"])
+    base, *_ = run_decode(Ld)
+    perm = torch.from_numpy(np.random.default_rng(4).permutation(Lh["nb"])).cuda()
+    kc = torch.empty_like(Ld["k_cache"]); kc[perm] = Ld["k_cache"]
+    vc = torch.empty_like(Ld["v_cache"]); vc[perm] = Ld["v_cache"]
+    L2 = dict(Ld, k_cache=kc, v_cache=vc, tables=perm[Ld["tables"].long()].int().contiguous())
+    got, *_ = run_decode(L2)
+    assert np.array_equal(got, base)
+
+
+def test_decode_contiguous_equals_paged():
+    sh = W.LayerShape(32, 128, 64, 2048)
+    wl = W.custom("contig", 92, sh, [50, 200, 33], append=False)
+    Lh = W.host_layer(wl, 0)
+    Ld = D.device_layer(wl, 0, tables=Lh["tables"], nb=Lh["nb"])
+    shuffled, *_ = run_decode(Ld)
+    # identity layout: sequence b's pages are consecutive, in order
+    need = [-(-int(t) // 16) for t in wl.seq_lens]
+    ident = np.zeros_like(Lh["tables"])
+    start = 0
+    for b, n in enumerate(need):
+        ident[b, :n] = np.arange(start, start + n)
+        ident[b, n:] = Lh["nb"] - 1
+        start += n
+    Li = D.device_layer(wl, 0, tables=ident, nb=Lh["nb"])
+    got, *_ = run_decode(Li)
+    assert np.array_equal(got, shuffled)
+
+
+def test_decode_softmax_stress_needle():
+    """Large logits and a planted token whose K code lines up with the query."""
+    sh = W.LayerShape(32, 128, 64, 2048)
+    wl = W.custom("needle", 93, sh, [700, 1300], append=False)
+    Lh = W.host_layer(wl, 0)
+    q = (Lh["q"].astype(np.float32) * 32).astype(np.float16)
+    for b, t in [(0, 5), (1, 1299)]:
+        pg, sl = Lh["tables"][b][t // 16], t % 16
+        qt = np.stack([Lh["B_K"][h].astype(np.float64) @ q[b, h].astype(np.float64) for h in range(32)])
+        Lh["k_cache"][pg, sl] = (qt / np.abs(qt).max(axis=1, keepdims=True) * 4).astype(np.float16)
+    Ld = D.device_layer(wl, 0, tables=Lh["tables"], nb=Lh["nb"])
+    Ld["k_cache"].copy_(torch.from_numpy(Lh["k_cache"]))
+    Ld["q"] = torch.from_numpy(q).cuda()
+    got, *_ = run_decode(Ld)
+    ref = O.decode_explicit(q, Lh["B_K"], Lh["B_V"], Lh["k_cache"], Lh["v_cache"], Lh["tables"],
+                            Lh["seq_lens"], Lh["scale"])
+    assert_close({b: got[b] for b in range(2)}, {b: ref[b] for b in range(2)})
+
+
+def test_decode_bad_block_id_is_flagged():
+    sh = W.LayerShape(32, 128, 64, 2048)
+    wl = W.custom("bad", 94, sh, [40], append=False)
+    Lh = W.host_layer(wl, 0)
+    Ld = D.device_layer(wl, 0, tables=Lh["tables"], nb=Lh["nb"])
+    bad = Ld["tables"].clone()
+    bad[0, 1] = Lh["nb"] + 5
+    desc = desc_of(Ld)
+    wsb = S.starkv_decode_workspace_bytes(desc, 1, 40)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    out = torch.empty((1, 32, 128), dtype=torch.float16, device="cuda")
+    S.starkv_paged_decode(desc, 1, 40, Ld["q"], Ld["B_K"], Ld["B_V"], Ld["k_cache"], Ld["v_cache"],
+                          bad, Ld["seq_lens"], Ld["scale"], ws, wsb, out)
+    st, flags = S.starkv_decode_check(ws)
+    assert S.STATUS[st] == "STARKV_ERR_DEVICE_CHECK" and flags & S.FLAG_BAD_BLOCK_ID
+    # a clean call on the same workspace clears the word
+    run_decode(Ld)
+
+
+def test_host_side_errors_launch_nothing():
+    sh = W.LayerShape(32, 128, 64, 2048)
+    wl = W.custom("err", 95, sh, [40], append=False)
+    Ld = D.device_layer(wl, 0)
+    desc = desc_of(Ld)
+    wsb = S.starkv_decode_workspace_bytes(desc, 1, 40)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    out = torch.zeros((1, 32, 128), dtype=torch.float16, device="cuda")
+    args = [desc, 1, 40, Ld["q"], Ld["B_K"], Ld["B_V"], Ld["k_cache"], Ld["v_cache"], Ld["tables"],
+            Ld["seq_lens"], Ld["scale"], ws, wsb, out]
+    a = list(args); a[12] = wsb - 1
+    assert S.starkv_paged_decode(*a, check=False) == 3
+    a = list(args); a[10] = float("nan")
+    assert S.starkv_paged_decode(*a, check=False) == 1
+    a = list(args); a[2] = 10 ** 6
+    assert S.starkv_paged_decode(*a, check=False) == 1
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out).item() == 0
+
+
+# ------------------------------------------------------------------ append
+
+def _append_check(wl, layer=0):
+    Lh = W.host_layer(wl, layer)
+    Ld = D.device_layer(wl, layer, tables=Lh["tables"], nb=Lh["nb"])
+    desc = desc_of(Ld)
+    before_k = Ld["k_cache"].clone()
+    before_v = Ld["v_cache"].clone()
+    S.starkv_compress_append(desc, wl.batch, Ld["k"], Ld["v"], Ld["A_K"], Ld["A_V"], Ld["tables"],
+                             Ld["ctx_lens"], Ld["k_cache"], Ld["v_cache"])
+    torch.cuda.synchronize()
+    cK, cV = O.compress(Lh["k"], Lh["v"], Lh["A_K"], Lh["A_V"])
+    pos = wl.ctx_lens
+    rows = np.array([Lh["tables"][b][pos[b] // 16] * 16 + pos[b] % 16 for b in range(wl.batch)])
+    kf_new = Ld["k_cache"].view(-1, Lh["H"] * Lh["r"]).cpu().numpy()
+    vf_new = Ld["v_cache"].view(-1, Lh["R"]).cpu().numpy()
+    kf_old = before_k.view(-1, Lh["H"] * Lh["r"]).cpu().numpy()
+    vf_old = before_v.view(-1, Lh["R"]).cpu().numpy()
+    mask = np.ones(kf_new.shape[0], bool)
+    mask[rows] = False
+    assert np.array_equal(kf_new[mask].view(np.uint16), kf_old[mask].view(np.uint16))
+    assert np.array_equal(vf_new[mask].view(np.uint16), vf_old[mask].view(np.uint16))
+    for want, got in ((cK.reshape(wl.batch, -1), kf_new[rows]), (cV, vf_new[rows])):
+        got = got.astype(np.float64)
+        ulp = np.spacing(np.abs(want).astype(np.float16)).astype(np.float64)
+        assert np.all(np.abs(got - want) <= ulp), np.max(np.abs(got - want) / ulp)
+        assert np.abs(got - want).max() <= MAX_ABS
+        assert rel_l2(got, want) <= REL_L2
+    return Lh, Ld, (cK.astype(np.float16), cV.astype(np.float16))
+
+
+def test_append_tiny():
+    _append_check(W.custom("app", 31, W.LayerShape(4, 64, 16, 64), [37, 100, 0, 15]))
+
+
+@pytest.mark.parametrize("layer", [0, 1, 2])
+def test_append_then_decode_continuous_batching_subset(layer):
+    """Batch-48 mixed-length workload's three rank profiles, first 6 sequences."""
+    full = W.workload(4)
+    wl = W.Workload("cb-subset", full.seed, 6, full.layers, full.ctx_lens[:6])
+    Lh, Ld, appended = _append_check(wl, layer)
+    got, *_ = run_decode(Ld)
+    ref = oracle_rows(wl, layer, Lh["q"], Ld["A_np"], range(6), wl.seq_lens, appended)
+    assert_close({b: got[b] for b in range(6)}, ref)
+
+
+# ---------------------------------------------------- full-size workloads
+
+@pytest.mark.parametrize("idx,sample", [(2, range(16)), (3, [0, 31, 63])])
+def test_decode_full_size_sampled(idx, sample):
+    wl = W.workload(idx)
+    Ld = D.device_layer(wl, 0)
+    S.starkv_compress_append(desc_of(Ld), wl.batch, Ld["k"], Ld["v"], Ld["A_K"], Ld["A_V"],
+                             Ld["tables"], Ld["ctx_lens"], Ld["k_cache"], Ld["v_cache"])
+    got, *_ = run_decode(Ld)
+    A_K, A_V, B_K, B_V = Ld["A_np"]
+    cK, cV = O.compress(Ld["k"].cpu().numpy(), Ld["v"].cpu().numpy(), A_K, A_V)
+    ref = oracle_rows(wl, 0, Ld["q"].cpu().numpy(), Ld["A_np"], sample, wl.seq_lens,
+                      (cK.astype(np.float16), cV.astype(np.float16)))
+    assert_close({b: got[b] for b in sample}, ref)
+    assert np.isfinite(got).all()
