@@ -184,6 +184,14 @@ def run_ours(args):
     K = args.steps
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in layers] for _ in range(K)]
     app_evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in layers] for _ in range(K)]
+    # torch creates the underlying cudaEvent at the first record: do that now so
+    # the raw handles handed to the library are valid
+    for step_evs in (evs, app_evs):
+        for per_step in step_evs:
+            for per_layer in per_step:
+                for e in per_layer:
+                    e.record(stream)
+    torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     uuid = None
     try:
@@ -269,7 +277,7 @@ def run_ours(args):
     assert np.isfinite(host_out[0].float().numpy()).all()
 
     cpu = None
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
         cpu = cpu_baseline(wl, args.cpu_seconds)
 
     value = world * B / (ms * 1e-3)
@@ -293,7 +301,7 @@ def run_ours(args):
         "kernels_GBps": {"kpass": round(kp_gbs, 1), "vpass": round(vp_gbs, 1)},
         "e2e": {"value": round(world * B / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
-        "gpu_launches": K * len(layers) * 6,
+        "gpu_launches": K * len(layers) * 7,   # append: V GEMM + K codes; decode: 5
         "clocks": clk,
     }
     if cpu is not None:

@@ -66,6 +66,8 @@ typedef enum {
 #define STARKV_FLAG_BAD_BLOCK_ID 0x1  /* block id outside [0, num_blocks) */
 #define STARKV_FLAG_BAD_SEQ_LEN 0x2   /* seq_len < 0 or > max_blocks_per_seq*16 or > max_seq_len */
 #define STARKV_FLAG_TIMEOUT 0x4       /* a pipeline wait exceeded its bound */
+/* Bits 8..15 accompany STARKV_FLAG_TIMEOUT and name the internal wait(s) that
+ * ran out (diagnostic only; the numbering is not part of the stable ABI). */
 
 /* One layer's cache geometry.  Ranks may differ from layer to layer. */
 typedef struct {
@@ -173,9 +175,10 @@ typedef struct {
   size_t prefix_off;  /* int32 [batch+1] prefix sums of pages per sequence */
   size_t qt_off;      /* fp32 [batch][H][r]: log2(e)*scale*q.B_K^T */
   size_t logits_off;  /* fp32 [batch][t_pad][H]: base-2 logits s*log2(e) */
-  size_t ml_off;      /* fp32 [k_slots][H][2]: per-segment (max, sum exp2) */
-  size_t stats_off;   /* fp32 [batch][H][2]: (global max, 1/sum) */
-  size_t zpart_off;   /* fp32 [n_rranges][v_slots][H][r_range]: partial sum_t p c_V */
+  size_t mpart_off;   /* fp32 [k_slots][H]: max of the base-2 logits per segment */
+  size_t mx_off;      /* fp32 [batch][H]: max of the base-2 logits per sequence */
+  size_t lpart_off;   /* fp32 [v_slots][H]: per segment, sum of the fp16 weights exp2(s - max) */
+  size_t zpart_off;   /* fp32 [n_rranges][v_slots][H][r_range]: per segment, sum_t w c_V */
   int32_t t_pad;      /* logits row capacity (multiple of 16) */
   int32_t k_ctas;     /* CTAs of the K pass (stream partition) */
   int32_t k_slots;    /* k_ctas + batch */

@@ -47,8 +47,9 @@ class LayerDesc(ctypes.Structure):
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [("total_bytes", ctypes.c_size_t), ("status_off", ctypes.c_size_t),
                 ("prefix_off", ctypes.c_size_t), ("qt_off", ctypes.c_size_t),
-                ("logits_off", ctypes.c_size_t), ("ml_off", ctypes.c_size_t),
-                ("stats_off", ctypes.c_size_t), ("zpart_off", ctypes.c_size_t),
+                ("logits_off", ctypes.c_size_t), ("mpart_off", ctypes.c_size_t),
+                ("mx_off", ctypes.c_size_t), ("lpart_off", ctypes.c_size_t),
+                ("zpart_off", ctypes.c_size_t),
                 ("t_pad", ctypes.c_int32), ("k_ctas", ctypes.c_int32), ("k_slots", ctypes.c_int32),
                 ("v_ctas", ctypes.c_int32), ("v_slots", ctypes.c_int32),
                 ("n_rranges", ctypes.c_int32), ("r_range", ctypes.c_int32)]

@@ -5,114 +5,201 @@
 // Both are accumulated in fp32, rounded to fp16 (nearest even) and stored in
 // slot pos % 16 of page block_table[b][pos / 16] (Proxima README, method
 // paragraph: codes "stored in a compressed paged format").
+//
+// The joint V projection is a dense GEMM over the batch,
+//   C_V^T (R x B) = A_V^T (R x H*d) . V^T (H*d x B),
+// run on tcgen05 tensor cores: one CTA per (128-row tile of R, K range),
+// A tiles are 64x64 boxes of A_V (MN-major, 128B swizzle), B tiles 64-column
+// boxes of the batch's v rows (K-major, 128B swizzle), the fp32 accumulator
+// lives in tensor memory.  The K ranges of one R tile form a thread-block
+// cluster and are summed through distributed shared memory in a fixed order,
+// so the result does not depend on scheduling.
 #pragma once
+#include <cooperative_groups.h>
 #include <cstdint>
 #include <cuda_fp16.h>
 
+#include "ptx.cuh"
+
 namespace starkv {
 
-struct AppendParams {
-  const __half* k;         // [B][H][d]
-  const __half* v;         // [B][H*d]
-  const __half* A_K;       // [H][d][r]
-  const __half* A_V;       // [H*d][R]
+struct AppendTarget {
   const int32_t* tables;   // [B][MB]
   const int32_t* positions;
-  __half* k_cache;         // [NB][16][H][r]
-  __half* v_cache;         // [NB][16][R]
-  int B, H, d, r, R, MB, NB;
-  int nvx, nby;            // V column tiles (64 wide) and batch tiles (16)
+  int MB, NB;
 };
 
-constexpr int kAppBT = 16;   // sequences per V tile
-constexpr int kAppNC = 64;   // code columns per V tile
-constexpr int kAppJC = 256;  // input rows staged per pass
-
 // Physical row (page*16 + slot) of sequence b's append target, or -1.
-__device__ __forceinline__ int64_t append_row(const AppendParams& p, int b) {
-  const int32_t pos = p.positions[b];
-  if (pos < 0 || pos / 16 >= p.MB) return -1;
-  const int32_t phys = p.tables[static_cast<size_t>(b) * p.MB + pos / 16];
-  if (phys < 0 || phys >= p.NB) return -1;
+__device__ __forceinline__ int64_t append_row(const AppendTarget& a, int b) {
+  const int32_t pos = a.positions[b];
+  if (pos < 0 || pos / 16 >= a.MB) return -1;
+  const int32_t phys = a.tables[static_cast<size_t>(b) * a.MB + pos / 16];
+  if (phys < 0 || phys >= a.NB) return -1;
   return static_cast<int64_t>(phys) * 16 + (pos % 16);
 }
 
-// grid: nvx*nby V tiles followed by H K blocks; 256 threads.
-__global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
+// ------------------------------------------------------------ V codes (TC)
+struct AppendVParams {
+  AppendTarget tgt;
+  __half* v_cache;         // [NB][16][R]
+  int B, HD, R;
+  int k_per_cta;           // rows of H*d per CTA (multiple of 64)
+  int npad;                // UMMA N: batch tile padded to a multiple of 16 (<= 256)
+  int stages;
+  uint32_t tmem_cols;
+};
+
+constexpr int kAppThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kAppKC = 64;         // rows of H*d per pipeline stage
+
+// grid (ceil(R/128), KS, ceil(B/256)), cluster (1, KS, 1)
+__global__ void __launch_bounds__(kAppThreads, 1)
+append_v_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap vmap,
+                AppendVParams p) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages;
+  const uint32_t a_bytes = 2u * kAppKC * 128u;                 // two 64x64 fp16 boxes
+  const uint32_t b_bytes = static_cast<uint32_t>(p.npad) * 128u;
+  const uint32_t stage_bytes = a_bytes + b_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * stage_bytes);
+  uint64_t* empty = full + S;
+  uint64_t* done = empty + S;
+  float* part = reinterpret_cast<float*>(smem);                 // [npad][128], reuses the ring
+  __shared__ uint32_t taddr_s;
+
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nv_blocks = p.nvx * p.nby;
-  if (static_cast<int>(blockIdx.x) < nv_blocks) {
-    // ---- V: 64 code columns x 16 sequences; 8 warps split the H*d rows of each pass
-    __shared__ __align__(16) __half vs[kAppJC][kAppBT];
-    __shared__ float red[8][kAppNC][kAppBT + 1];
-    const int nx = blockIdx.x % p.nvx, by = blockIdx.x / p.nvx;
-    const int n0 = nx * kAppNC, b0 = by * kAppBT;
-    const int HD = p.H * p.d;
-    float acc[kAppBT][2];
-#pragma unroll
-    for (int u = 0; u < kAppBT; ++u) acc[u][0] = acc[u][1] = 0.f;
-    for (int jc = 0; jc < HD; jc += kAppJC) {
-      __syncthreads();
-      for (int x = tid; x < kAppJC * kAppBT; x += 256) {
-        const int bb = x / kAppJC, jj = x % kAppJC;
-        const int b = b0 + bb, j = jc + jj;
-        vs[jj][bb] = (b < p.B && j < HD) ? p.v[static_cast<size_t>(b) * HD + j] : __float2half_rn(0.f);
-      }
-      __syncthreads();
-      const int jn = min(kAppJC, HD - jc);
-      for (int jj = warp * (kAppJC / 8); jj < (warp + 1) * (kAppJC / 8) && jj < jn; ++jj) {
-        const float2 a = __half22float2(
-            *reinterpret_cast<const __half2*>(p.A_V + static_cast<size_t>(jc + jj) * p.R + n0 + 2 * lane));
-        const uint4* vr = reinterpret_cast<const uint4*>(&vs[jj][0]);
-        const uint4 w0 = vr[0], w1 = vr[1];
-        const __half2* h0 = reinterpret_cast<const __half2*>(&w0);
-        const __half2* h1 = reinterpret_cast<const __half2*>(&w1);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float2 x0 = __half22float2(h0[u]);
-          const float2 x1 = __half22float2(h1[u]);
-          acc[2 * u][0] = fmaf(x0.x, a.x, acc[2 * u][0]);
-          acc[2 * u][1] = fmaf(x0.x, a.y, acc[2 * u][1]);
-          acc[2 * u + 1][0] = fmaf(x0.y, a.x, acc[2 * u + 1][0]);
-          acc[2 * u + 1][1] = fmaf(x0.y, a.y, acc[2 * u + 1][1]);
-          acc[8 + 2 * u][0] = fmaf(x1.x, a.x, acc[8 + 2 * u][0]);
-          acc[8 + 2 * u][1] = fmaf(x1.x, a.y, acc[8 + 2 * u][1]);
-          acc[8 + 2 * u + 1][0] = fmaf(x1.y, a.x, acc[8 + 2 * u + 1][0]);
-          acc[8 + 2 * u + 1][1] = fmaf(x1.y, a.y, acc[8 + 2 * u + 1][1]);
-        }
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kAppBT; ++u) {
-      red[warp][2 * lane][u] = acc[u][0];
-      red[warp][2 * lane + 1][u] = acc[u][1];
-    }
-    __syncthreads();
-    for (int x = tid; x < kAppNC * kAppBT; x += 256) {
-      const int c = x % kAppNC, bb = x / kAppNC;
-      const int b = b0 + bb;
-      if (b >= p.B) continue;
-      float s = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) s += red[w][c][bb];
-      const int64_t row = append_row(p, b);
-      if (row >= 0) p.v_cache[row * p.R + n0 + c] = __float2half_rn(s);
-    }
-    return;
+  const int mt = blockIdx.x;                  // 128-row tile of R
+  const int ks = blockIdx.y;                  // K range (cluster rank)
+  const int KS = gridDim.y;
+  const int b0 = blockIdx.z * 256;
+  const int k0 = ks * p.k_per_cta;
+  const int k1 = min(p.HD, k0 + p.k_per_cta);
+  const int n_stages = k1 > k0 ? (k1 - k0 + kAppKC - 1) / kAppKC : 0;
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(done, 1);
+    fence_mbar_init();
   }
-  // ---- K: one block per head; thread = (rank index, sequence lane)
-  const int h = blockIdx.x - nv_blocks;
+  if (warp == 1) {
+    tmem_alloc(&taddr_s, p.tmem_cols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t taddr = taddr_s;
+  bool ok = true;
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&amap);
+    prefetch_tensormap(&vmap);
+    const uint64_t pol = policy_evict_last();
+    for (int i = 0; i < n_stages; ++i) {
+      const int s = i % S;
+      if (i >= S && !mbar_wait(&empty[s], ((i / S) - 1) & 1)) { ok = false; break; }
+      uint8_t* st = smem + static_cast<size_t>(s) * stage_bytes;
+      const int kr = k0 + i * kAppKC;
+      mbar_arrive_expect_tx(&full[s], stage_bytes);
+      tma_load_2d(st, &amap, mt * 128, kr, &full[s], pol);
+      tma_load_2d(st + kAppKC * 128, &amap, mt * 128 + 64, kr, &full[s], pol);
+      tma_load_2d(st + a_bytes, &vmap, kr, b0, &full[s], pol);
+    }
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t idesc = idesc_f16_f32(128, p.npad, /*a_mn_major=*/true, /*b_mn_major=*/false);
+    for (int i = 0; i < n_stages; ++i) {
+      const int s = i % S;
+      if (!mbar_wait(&full[s], (i / S) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
+      const uint32_t sb = sa + a_bytes;
+#pragma unroll
+      for (int kk = 0; kk < kAppKC / 16; ++kk) {
+        const uint64_t adesc = smem_desc(sa + kk * 16u * 128u, kAppKC * 128u, 1024u, kSwizzle128B);
+        const uint64_t bdesc = smem_desc(sb + kk * 32u, 16u, 1024u, kSwizzle128B);
+        umma_f16_ss(taddr, adesc, bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(&empty[s]);
+    }
+    umma_commit(done);
+  }
+  __syncthreads();
+  // every warp observes the accumulator completion (or an empty K range)
+  if (!mbar_wait(done, 0)) ok = false;
+  tc_fence_after();
+  if (warp >= 2) {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;            // row of the R tile
+    for (int c0 = 0; c0 < p.npad; c0 += 16) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x16(taddr + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        part[(c0 + j) * 128 + row] = (n_stages > 0 && ok) ? __uint_as_float(v[j]) : 0.f;
+    }
+  }
+  tc_fence_before();
+  cluster.sync();
+  // rank ks sums rows (batch entries) [ks*npad/KS, (ks+1)*npad/KS) over the cluster, in rank order
+  const int per = (p.npad + KS - 1) / KS;
+  const int n_lo = ks * per, n_hi = min(p.npad, n_lo + per);
+  for (int x = tid; x < (n_hi - n_lo) * 128; x += kAppThreads) {
+    const int n = n_lo + x / 128, rrow = x % 128;
+    const int b = b0 + n;
+    const int rg = mt * 128 + rrow;
+    if (b >= p.B || rg >= p.R) continue;
+    float acc = 0.f;
+    for (int c = 0; c < KS; ++c) acc += cluster.map_shared_rank(part, c)[n * 128 + rrow];
+    const int64_t dst = append_row(p.tgt, b);
+    if (dst >= 0) p.v_cache[dst * p.R + rg] = __float2half_rn(acc);
+  }
+  cluster.sync();   // nobody leaves while others still read its partials
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(taddr, p.tmem_cols);
+  }
+}
+
+// ------------------------------------------------------------ K codes
+struct AppendKParams {
+  AppendTarget tgt;
+  const __half* k;         // [B][H][d]
+  const __half* A_K;       // [H][d][r]
+  __half* k_cache;         // [NB][16][H][r]
+  int B, H, d, r;
+};
+
+// grid (H), 256 threads; dynamic smem: A_K[h] (d*r halves) + k[:, h, :] (B*d halves)
+__global__ void __launch_bounds__(256) append_k_kernel(AppendKParams p) {
+  extern __shared__ __align__(16) uint8_t ks_smem[];
+  __half* As = reinterpret_cast<__half*>(ks_smem);              // [d][r]
+  __half* ksm = As + static_cast<size_t>(p.d) * p.r;            // [B][d]
+  const int h = blockIdx.x, tid = threadIdx.x;
+  const uint4* asrc = reinterpret_cast<const uint4*>(p.A_K + static_cast<size_t>(h) * p.d * p.r);
+  for (int x = tid; x < p.d * p.r / 8; x += 256) reinterpret_cast<uint4*>(As)[x] = asrc[x];
+  for (int x = tid; x < p.B * p.d / 8; x += 256) {
+    const int b = x / (p.d / 8), c = x % (p.d / 8);
+    reinterpret_cast<uint4*>(ksm)[x] =
+        reinterpret_cast<const uint4*>(p.k + (static_cast<size_t>(b) * p.H + h) * p.d)[c];
+  }
+  __syncthreads();
   const int i = tid % p.r;
   const int bpar = 256 / p.r;
   const int bs = tid / p.r;
   if (bs >= bpar) return;
-  const __half* A = p.A_K + static_cast<size_t>(h) * p.d * p.r + i;
   for (int b = bs; b < p.B; b += bpar) {
-    const __half* krow = p.k + (static_cast<size_t>(b) * p.H + h) * p.d;
-    float acc = 0.f;
-    for (int j = 0; j < p.d; ++j) acc = fmaf(__half2float(krow[j]), __half2float(A[static_cast<size_t>(j) * p.r]), acc);
-    const int64_t row = append_row(p, b);
-    if (row >= 0) p.k_cache[(row * p.H + h) * p.r + i] = __float2half_rn(acc);
+    const __half* kr = ksm + static_cast<size_t>(b) * p.d;
+    float a0 = 0.f, a1 = 0.f;
+    for (int j = 0; j < p.d; j += 2) {
+      a0 = fmaf(__half2float(kr[j]), __half2float(As[j * p.r + i]), a0);
+      a1 = fmaf(__half2float(kr[j + 1]), __half2float(As[(j + 1) * p.r + i]), a1);
+    }
+    const int64_t row = append_row(p.tgt, b);
+    if (row >= 0) p.k_cache[(row * p.H + h) * p.r + i] = __float2half_rn(a0 + a1);
   }
 }
 

@@ -2,10 +2,11 @@
 //
 // One decode is five launches on the caller's stream:
 //   1. absorb      q~ = log2(e)*scale * q . B_K[h]^T; page prefix sums; status reset
-//   2. kpass       base-2 logits s = q~ . c_K over the K pages, per-segment (max, sum exp2)
-//   3. reduce      per (b, h): global max M and 1/L with L = sum exp2(s - M)
-//   4. vpass       Z = sum_t p c_V on tcgen05 tensor cores, p = exp2(s - M)/L in fp16
-//   5. upproj      out_h = Z_h . B_V[:, h*d:(h+1)*d] -> fp16
+//   2. kpass       base-2 logits s = q~ . c_K over the K pages, per-segment max
+//   3. reduce      per (b, h): global max M of the logits
+//   4. vpass       Z = sum_t w c_V on tcgen05 tensor cores with w = fp16(exp2(s - M)),
+//                  and the normaliser L = sum_t w
+//   5. upproj      out_h = (Z_h . B_V[:, h*d:(h+1)*d]) / L -> fp16
 //
 // The formulation (head-wise K with the query absorbed, joint V applied after
 // the weighted sum of codes) follows the STAR-KV description in the Proxima
@@ -57,6 +58,16 @@ __device__ __forceinline__ int32_t seq_of_page(const int32_t* prefix, int32_t B,
 }
 
 __device__ __forceinline__ void set_flag(int32_t* status, int32_t f) { atomicOr(status, f); }
+
+// Timeout at pipeline wait `site`: the timeout bit plus a per-site bit (8..15)
+// that tells where the pipeline stopped.
+enum WaitSite : int32_t {
+  kSiteKEmpty = 0, kSiteKFull = 1, kSiteVEmpty = 2, kSiteVPready = 3, kSiteVTfree = 4,
+  kSiteVFull = 5, kSiteVZdone = 6, kSiteVMdone = 7
+};
+__device__ __forceinline__ void set_timeout(int32_t* status, WaitSite site) {
+  atomicOr(status, STARKV_FLAG_TIMEOUT | (1 << (8 + site)));
+}
 
 // ====================================================================== absorb
 struct AbsorbParams {
@@ -139,23 +150,43 @@ struct KPassParams {
   const int32_t* prefix;      // [B+1]
   const float* qt;            // [B][H][r]
   float* logits;              // [B][t_pad][H]
-  float* ml;                  // [k_slots][H][2]
+  float* mpart;               // [k_slots][H]: max of the base-2 logits per segment
   int32_t* status;
-  int B, H, r, MB, NB, t_pad;
+  int B, H, log2H, r, MB, NB, t_pad;
   int tps;                    // tokens per ring stage
   int stages;
   uint32_t stage_bytes;       // tps*H*r*2
 };
 
-constexpr int kKConsumers = 512;            // 16 warps of dot products
+constexpr int kKConsumers = 256;            // 8 warps of dot products
 constexpr int kKThreads = kKConsumers + 32; // + one producer warp
 
 struct StageMeta { int32_t b, t0, nt, flags; };
 
-// L lanes share one (token, head) dot product of length r; each lane reads CPL
-// 16-byte chunks (8 codes each).  The head of a thread is fixed:
-// (kKConsumers / L) is a multiple of H.
-template <int L, int CPL>
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)),
+        "l"(*reinterpret_cast<uint64_t*>(&c)));
+  return *reinterpret_cast<float2*>(&d);
+}
+
+// First chunk a thread visits, chosen so that the 8 threads sharing a
+// shared-memory wavefront (8 consecutive rows of r*2 bytes, 16-byte reads)
+// hit 8 different bank groups: bank group of (row, chunk) is
+// (row*CP + chunk) mod 8 with CP = r/8 chunks per row.
+__device__ __forceinline__ int chunk_rotation(int tid, int cp, int L) {
+  if (L > 1 || cp % 8 == 0) return tid & 7;
+  if (cp % 4 == 0) return (tid >> 1) & 3;
+  return (tid >> 2) & 1;
+}
+
+// One (token, head) dot product of length r per L threads: each thread reads
+// CPT 16-byte chunks (8 codes) of its row in a rotated order and accumulates
+// with packed fp32 FMAs against its head's absorbed query held in registers.
+// The head of a thread is fixed because (kKConsumers / L) is a multiple of H.
+template <int L, int CPT>
 __global__ void __launch_bounds__(kKThreads, 1) kpass_kernel(KPassParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int S = p.stages;
@@ -163,7 +194,7 @@ __global__ void __launch_bounds__(kKThreads, 1) kpass_kernel(KPassParams p) {
   StageMeta* meta = reinterpret_cast<StageMeta*>(smem + static_cast<size_t>(S) * p.stage_bytes);
   uint64_t* full = reinterpret_cast<uint64_t*>(meta + S);
   uint64_t* empty = full + S;
-  float2* red = reinterpret_cast<float2*>(empty + S);       // [kKConsumers / L]
+  float* red = reinterpret_cast<float*>(empty + S);         // [kKConsumers / L]
   __shared__ volatile int32_t abort_flag;
 
   const int tid = threadIdx.x;
@@ -217,7 +248,7 @@ __global__ void __launch_bounds__(kKThreads, 1) kpass_kernel(KPassParams p) {
       if (ok) { meta[s] = StageMeta{-1, 0, 0, 0}; mbar_arrive(&full[s]); }
     }
     if (!ok) {
-      set_flag(p.status, STARKV_FLAG_TIMEOUT);
+      set_timeout(p.status, kSiteKEmpty);
       abort_flag = 1;
       // let copies already in flight land before the CTA can exit
       const uint32_t first = k > static_cast<uint32_t>(S) ? k - S : 0;
@@ -227,82 +258,79 @@ __global__ void __launch_bounds__(kKThreads, 1) kpass_kernel(KPassParams p) {
   }
 
   // -------------------------------------------------------------- consumers
-  constexpr int kGroups = kKConsumers / L;  // (token, head) pairs per iteration
-  const int grp = tid / L;
+  constexpr int kPairsPerPass = kKConsumers / L;
+  const int pair0 = tid / L;
   const int sub = tid % L;
-  const int head = grp % p.H;
-  const int cp = p.r >> 3;                  // 16-byte chunks per (token, head)
-  const int iters = (p.tps * p.H + kGroups - 1) / kGroups;
-  float qv[CPL * 8];
-  float m = -INFINITY, l = 0.f;
+  const int head = pair0 & (p.H - 1);
+  const int cp = p.r >> 3;                  // 16-byte chunks per (token, head) row
+  const int rot = chunk_rotation(tid, cp, L);
+  const int passes = (p.tps * p.H + kPairsPerPass - 1) / kPairsPerPass;
+  float2 qv[CPT * 4];
+  float m = -INFINITY;
   int cur_b = -1;
 
   for (uint32_t k = 0;; ++k) {
     const int s = k % S;
     if (!mbar_wait(&full[s], (k / S) & 1) || abort_flag) {
-      set_flag(p.status, STARKV_FLAG_TIMEOUT);
+      set_timeout(p.status, kSiteKFull);
       break;
     }
     const StageMeta mt = meta[s];
-    if (mt.b != cur_b) {
+    if (mt.b != cur_b || mt.b < 0) {   // new sequence, or the end marker (b < 0)
       if (cur_b >= 0) {
-        // flush (max, sum) of the finished segment: slot = sequence + CTA
-        if (sub == 0) red[grp] = make_float2(m, l);
+        // per-segment max for every head: slot = sequence + CTA
+        if (sub == 0) red[pair0] = m;
         named_bar_sync(1, kKConsumers);
         if (tid < p.H) {
           float M = -INFINITY;
-          for (int g = tid; g < kGroups; g += p.H) M = fmaxf(M, red[g].x);
-          float Ls = 0.f;
-          for (int g = tid; g < kGroups; g += p.H)
-            if (red[g].x != -INFINITY) Ls += red[g].y * exp2f(red[g].x - M);
-          float* dst = p.ml + (static_cast<size_t>(cur_b + cta) * p.H + tid) * 2;
-          dst[0] = M;
-          dst[1] = Ls;
+          for (int g = tid; g < kPairsPerPass; g += p.H) M = fmaxf(M, red[g]);
+          p.mpart[static_cast<size_t>(cur_b + cta) * p.H + tid] = M;
         }
         named_bar_sync(1, kKConsumers);
       }
       if (mt.b < 0) break;
       cur_b = mt.b;
       m = -INFINITY;
-      l = 0.f;
       const float* qsrc = p.qt + (static_cast<size_t>(cur_b) * p.H + head) * p.r;
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) {
-        const int ch = sub + c * L;
+      for (int c = 0; c < CPT; ++c) {
+        const int cc = c + rot < CPT ? c + rot : c + rot - CPT;
+        const int ch = sub * CPT + cc;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) qv[c * 8 + e] = ch < cp ? qsrc[ch * 8 + e] : 0.f;
+        for (int u = 0; u < 4; ++u)
+          qv[c * 4 + u] = ch < cp ? make_float2(qsrc[ch * 8 + 2 * u], qsrc[ch * 8 + 2 * u + 1])
+                                  : make_float2(0.f, 0.f);
       }
     }
     const uint8_t* st = ring + static_cast<size_t>(s) * p.stage_bytes;
-    for (int it = 0; it < iters; ++it) {
-      const int pair = it * kGroups + grp;
-      const int t = pair / p.H;          // token within the stage; pair % H == head
+    for (int ps = 0; ps < passes; ++ps) {
+      const int pair = ps * kPairsPerPass + pair0;
+      const int t = pair >> p.log2H;     // token within the stage; pair & (H-1) == head
       const bool valid = t < mt.nt;
-      float acc = 0.f;
+      float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
       if (valid) {
         const uint8_t* row = st + static_cast<size_t>(pair) * p.r * 2;
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-          const int ch = sub + c * L;
+        for (int c = 0; c < CPT; ++c) {
+          const int cc = c + rot < CPT ? c + rot : c + rot - CPT;
+          const int ch = sub * CPT + cc;
           if (ch < cp) {
             const uint4 w = *reinterpret_cast<const uint4*>(row + ch * 16);
             const __half2* h2 = reinterpret_cast<const __half2*>(&w);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float2 f = __half22float2(h2[u]);
-              acc = fmaf(f.x, qv[c * 8 + 2 * u], acc);
-              acc = fmaf(f.y, qv[c * 8 + 2 * u + 1], acc);
-            }
+            a0 = ffma2(__half22float2(h2[0]), qv[c * 4 + 0], a0);
+            a1 = ffma2(__half22float2(h2[1]), qv[c * 4 + 1], a1);
+            a2 = ffma2(__half22float2(h2[2]), qv[c * 4 + 2], a2);
+            a3 = ffma2(__half22float2(h2[3]), qv[c * 4 + 3], a3);
           }
         }
       }
+      float acc = ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
 #pragma unroll
       for (int o = L / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (valid) {
         if (sub == 0)
           p.logits[(static_cast<size_t>(cur_b) * p.t_pad + mt.t0 + t) * p.H + head] = acc;
-        if (acc > m) { l = l * exp2f(m - acc) + 1.f; m = acc; }
-        else { l += exp2f(acc - m); }
+        m = fmaxf(m, acc);
       }
     }
     __syncwarp();
@@ -312,9 +340,9 @@ __global__ void __launch_bounds__(kKThreads, 1) kpass_kernel(KPassParams p) {
 
 // ====================================================================== reduce
 struct ReduceParams {
-  const float* ml;        // [k_slots][H][2]
+  const float* mpart;     // [k_slots][H]
   const int32_t* prefix;  // [B+1]
-  float* stats;           // [B][H][2]: (M, 1/L)
+  float* mx;              // [B][H]: max of the base-2 logits of each sequence and head
   int B, H, k_grid;
 };
 
@@ -322,22 +350,15 @@ __global__ void __launch_bounds__(256) reduce_kernel(ReduceParams p) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= p.B * p.H) return;
   const int b = idx / p.H, h = idx % p.H;
-  float* dst = p.stats + static_cast<size_t>(idx) * 2;
   const int32_t f0 = p.prefix[b], f1 = p.prefix[b + 1];
-  if (f1 == f0) { dst[0] = 0.f; dst[1] = 0.f; return; }
+  if (f1 == f0) { p.mx[idx] = 0.f; return; }
   Partition pt;
   pt.P = p.prefix[p.B];
   pt.G = static_cast<int32_t>(pt.P < p.k_grid ? pt.P : p.k_grid);
   const int32_t i0 = part_owner(f0, pt), i1 = part_owner(f1 - 1, pt);
   float M = -INFINITY;
-  for (int32_t i = i0; i <= i1; ++i) M = fmaxf(M, p.ml[(static_cast<size_t>(b + i) * p.H + h) * 2]);
-  float L = 0.f;
-  for (int32_t i = i0; i <= i1; ++i) {
-    const float* e = p.ml + (static_cast<size_t>(b + i) * p.H + h) * 2;
-    L += e[1] * exp2f(e[0] - M);
-  }
-  dst[0] = M;
-  dst[1] = 1.f / L;
+  for (int32_t i = i0; i <= i1; ++i) M = fmaxf(M, p.mpart[static_cast<size_t>(b + i) * p.H + h]);
+  p.mx[idx] = M;
 }
 
 // ======================================================================= vpass
@@ -352,8 +373,9 @@ struct VPassParams {
   const int32_t* teff;
   const int32_t* prefix;
   const float* logits;    // [B][t_pad][H]
-  const float* stats;     // [B][H][2]
-  float* zpart;           // [n_rr][v_slots][H][r_range]
+  const float* mx;        // [B][H]
+  float* zpart;           // [n_rr][v_slots][H][r_range]: sum_t w c_V per segment
+  float* lpart;           // [v_slots][H]: sum_t w per segment (written by R range 0)
   int32_t* status;
   int B, H, npad, MB, NB, R, t_pad, r_range, n_rr, v_slots, stages;
   int n_chunks;           // 64-wide chunks per R range (r_range_pad/64); the last range may hold fewer
@@ -383,7 +405,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
   uint64_t* tfree = zdone + 1;
   uint64_t* mdone = tfree + 1;
   float* sM = reinterpret_cast<float*>(mdone + 1);                      // [npad]
-  float* sI = sM + p.npad;                                              // [npad]
+  float* sRed = sM + p.npad;                                            // [128]
   __shared__ uint32_t taddr_s;
   __shared__ volatile int32_t abort_flag;
 
@@ -456,7 +478,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
         if (ok) { meta[s] = StageMeta{-1, 0, 0, 0}; mbar_arrive(&full[s]); }
       }
       if (!ok) {
-        set_flag(p.status, STARKV_FLAG_TIMEOUT);
+        set_timeout(p.status, kSiteVEmpty);
         abort_flag = 1;
         const uint32_t first = k > static_cast<uint32_t>(S) ? k - S : 0;
         for (uint32_t kk = first; kk < k; ++kk) mbar_wait(&full[kk % S], (kk / S) & 1);
@@ -471,11 +493,11 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
       uint32_t accumulate = 0;
       for (uint32_t k = 0;; ++k) {
         const int s = k % S;
-        if (!mbar_wait(&pready[s], (k / S) & 1) || abort_flag) { set_flag(p.status, STARKV_FLAG_TIMEOUT); break; }
+        if (!mbar_wait(&pready[s], (k / S) & 1) || abort_flag) { set_timeout(p.status, kSiteVPready); break; }
         const StageMeta mt = meta[s];
         if (mt.b < 0) break;
         if (mt.flags & kFirst) {
-          if (seg > 0 && !mbar_wait(tfree, (seg - 1) & 1)) { set_flag(p.status, STARKV_FLAG_TIMEOUT); break; }
+          if (seg > 0 && !mbar_wait(tfree, (seg - 1) & 1)) { set_timeout(p.status, kSiteVTfree); break; }
           accumulate = 0;
         }
         tc_fence_after();
@@ -492,42 +514,47 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
       }
       // every MMA issued has completed before the CTA can release TMEM
       umma_commit(mdone);
-      if (!mbar_wait(mdone, 0)) set_flag(p.status, STARKV_FLAG_TIMEOUT);
+      if (!mbar_wait(mdone, 0)) set_timeout(p.status, kSiteVMdone);
     }
   } else {
     // ------------------------------------------ weights + epilogue (128 thr)
     const int et = tid - 64;             // 0..127
     const int q = warp & 3;              // TMEM lane quarter of this warp
     const uint32_t lbo_b = static_cast<uint32_t>(p.npad / 8) * 128u;
-    const int entries = kBlock * p.npad;
+    // this thread's weights: head h_w (fixed), tokens t_w0, t_w0 + t_step, ...
+    const int h_w = et % p.npad;
+    const int t_w0 = et / p.npad;
+    const int t_step = 128 / p.npad;
+    float lsum = 0.f;
     uint32_t seg = 0;
     for (uint32_t k = 0;; ++k) {
       const int s = k % S;
       if (!mbar_wait(&full[s], (k / S) & 1) || abort_flag) {
-        set_flag(p.status, STARKV_FLAG_TIMEOUT);
+        set_timeout(p.status, kSiteVFull);
         abort_flag = 1;
         break;
       }
       const StageMeta mt = meta[s];
       if (mt.b < 0) { mbar_arrive(&pready[s]); break; }
       if (mt.flags & kFirst) {
-        named_bar_sync(2, 128);  // everyone is done with the previous segment's stats
-        for (int h = et; h < p.npad; h += 128) {
-          const bool in = h < p.H;
-          sM[h] = in ? p.stats[(static_cast<size_t>(mt.b) * p.H + h) * 2] : 0.f;
-          sI[h] = in ? p.stats[(static_cast<size_t>(mt.b) * p.H + h) * 2 + 1] : 0.f;
-        }
+        named_bar_sync(2, 128);  // everyone is done with the previous segment's max
+        for (int h = et; h < p.npad; h += 128)
+          sM[h] = h < p.H ? p.mx[static_cast<size_t>(mt.b) * p.H + h] : 0.f;
         named_bar_sync(2, 128);
+        lsum = 0.f;
       }
       const float* lt = reinterpret_cast<const float*>(ltiles + static_cast<size_t>(s) * p.ltile_bytes);
       uint8_t* pt_s = ptiles + static_cast<size_t>(s) * p.ptile_bytes;
-      for (int e = et; e < entries; e += 128) {
-        const int t = e / p.npad, h = e % p.npad;
-        float w = 0.f;
-        if (t < mt.nt && h < p.H) w = exp2f(lt[t * p.H + h] - sM[h]) * sI[h];
-        const uint32_t off = static_cast<uint32_t>(t >> 3) * lbo_b + static_cast<uint32_t>(h >> 3) * 128u +
-                             static_cast<uint32_t>(h & 7) * 16u + static_cast<uint32_t>(t & 7) * 2u;
-        *reinterpret_cast<__half*>(pt_s + off) = __float2half_rn(w);
+      const float m_h = sM[h_w];
+      for (int t = t_w0; t < kBlock; t += t_step) {
+        // unnormalised weight exp2(s - M) <= 1, rounded to fp16 for the MMA; the
+        // normaliser sums exactly the rounded weights
+        __half w = __float2half_rn(0.f);
+        if (t < mt.nt && h_w < p.H) w = __float2half_rn(exp2f(lt[t * p.H + h_w] - m_h));
+        lsum += __half2float(w);
+        const uint32_t off = static_cast<uint32_t>(t >> 3) * lbo_b + static_cast<uint32_t>(h_w >> 3) * 128u +
+                             static_cast<uint32_t>(h_w & 7) * 16u + static_cast<uint32_t>(t & 7) * 2u;
+        *reinterpret_cast<__half*>(pt_s + off) = w;
       }
       if (mt.nt < kBlock) {
         // tokens past the sequence end: zero their rows of the V tile so that
@@ -546,7 +573,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
       mbar_arrive(&pready[s]);
       if (mt.flags & kLast) {
         if (!mbar_wait(zdone, seg & 1)) {
-          set_flag(p.status, STARKV_FLAG_TIMEOUT);
+          set_timeout(p.status, kSiteVZdone);
           abort_flag = 1;
           break;
         }
@@ -570,6 +597,15 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
         }
         tc_fence_before();
         mbar_arrive(tfree);
+        // per-segment normaliser of every head
+        sRed[et] = lsum;
+        named_bar_sync(2, 128);
+        if (rr == 0 && et < p.H) {
+          float Ls = 0.f;
+          for (int i = et; i < 128; i += p.npad) Ls += sRed[i];
+          p.lpart[slot * p.H + et] = Ls;
+        }
+        named_bar_sync(2, 128);
         ++seg;
       }
     }
@@ -584,6 +620,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
 // ====================================================================== upproj
 struct UpProjParams {
   const float* zpart;     // [n_rr][v_slots][H][r_range]
+  const float* lpart;     // [v_slots][H]
   const int32_t* prefix;
   const __half* B_V;      // [R][H*d]
   __half* out;            // [B][H][d]
@@ -591,13 +628,24 @@ struct UpProjParams {
 };
 
 constexpr int kUpBT = 16;   // sequences per CTA
-constexpr int kUpRC = 512;  // R rows staged per pass
+constexpr int kUpRC = 128;  // rows of B_V (and Z) staged per chunk
 
-// grid (H, ceil(B/16)), 256 threads; thread = (column pair, group of BPT sequences)
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// grid (H, ceil(B/16)), 256 threads; dynamic smem 2 x (kUpRC*d halves + kUpRC*16 floats).
+// out[b,h,:] = (sum over the V-pass partials of sequence b) . B_V[:, h*d:(h+1)*d]
 template <int BPT>
 __global__ void __launch_bounds__(256) upproj_kernel(UpProjParams p) {
-  __shared__ __align__(16) float zs[kUpRC][kUpBT];
+  extern __shared__ __align__(16) uint8_t up_smem[];
+  __half* bvs = reinterpret_cast<__half*>(up_smem);                          // [2][kUpRC][d]
+  float* zs = reinterpret_cast<float*>(up_smem + 2 * kUpRC * p.d * 2);       // [2][kUpRC][kUpBT]
   __shared__ int32_t i0s[kUpBT], i1s[kUpBT];
+  __shared__ float invl[kUpBT];
   const int h = blockIdx.x;
   const int bt0 = blockIdx.y * kUpBT;
   const int tid = threadIdx.x;
@@ -616,31 +664,67 @@ __global__ void __launch_bounds__(256) upproj_kernel(UpProjParams p) {
     }
     i0s[tid] = a;
     i1s[tid] = z;
+    float Ls = 0.f;
+    for (int32_t i = a; i <= z; ++i) Ls += p.lpart[static_cast<size_t>(b + i) * p.H + h];
+    invl[tid] = Ls > 0.f ? 1.f / Ls : 0.f;
   }
-  float acc[BPT][2];
-#pragma unroll
-  for (int u = 0; u < BPT; ++u) acc[u][0] = acc[u][1] = 0.f;
+  __syncthreads();
   const size_t hd = static_cast<size_t>(p.H) * p.d;
-  for (int j0 = 0; j0 < p.R; j0 += kUpRC) {
+  const int n_chunks = (p.R + kUpRC - 1) / kUpRC;
+  const int vec_per_row = p.d / 8;  // 16-byte pieces of one B_V row slice
+
+  auto load_bv = [&](int chunk, int buf) {
+    const int j0 = chunk * kUpRC;
     const int jn = min(kUpRC, p.R - j0);
-    __syncthreads();
+    __half* dst = bvs + static_cast<size_t>(buf) * kUpRC * p.d;
+    for (int x = tid; x < jn * vec_per_row; x += 256) {
+      const int j = x / vec_per_row, v = x % vec_per_row;
+      cp_async16(dst + j * p.d + v * 8, p.B_V + static_cast<size_t>(j0 + j) * hd + static_cast<size_t>(h) * p.d + v * 8);
+    }
+  };
+  auto load_z = [&](int chunk, int buf) {
+    const int j0 = chunk * kUpRC;
+    const int jn = min(kUpRC, p.R - j0);
+    float* dst = zs + static_cast<size_t>(buf) * kUpRC * kUpBT;
     for (int x = tid; x < jn * kUpBT; x += 256) {
       const int bt = x / jn, j = j0 + x % jn;
       const int b = bt0 + bt;
       float z = 0.f;
       if (b < p.B) {
         const int rrg = j / p.r_range, jj = j % p.r_range;
-        for (int32_t i = i0s[bt]; i <= i1s[bt]; ++i)
-          z += p.zpart[((static_cast<size_t>(rrg) * p.v_slots + b + i) * p.H + h) * p.r_range + jj];
+        const float* src = p.zpart + ((static_cast<size_t>(rrg) * p.v_slots + b) * p.H + h) * p.r_range + jj;
+        const size_t slot_stride = static_cast<size_t>(p.H) * p.r_range;
+        for (int32_t i = i0s[bt]; i <= i1s[bt]; ++i) z += src[static_cast<size_t>(i) * slot_stride];
       }
-      zs[j - j0][bt] = z;
+      dst[(j - j0) * kUpBT + bt] = z;
+    }
+  };
+
+  float acc[BPT][2];
+#pragma unroll
+  for (int u = 0; u < BPT; ++u) acc[u][0] = acc[u][1] = 0.f;
+  load_bv(0, 0);
+  cp_async_commit();
+  load_z(0, 0);
+  for (int c = 0; c < n_chunks; ++c) {
+    const int buf = c & 1;
+    if (c + 1 < n_chunks) {
+      load_bv(c + 1, buf ^ 1);
+      cp_async_commit();
+      load_z(c + 1, buf ^ 1);
+      cp_async_wait_1();
+    } else {
+      cp_async_wait_0();
     }
     __syncthreads();
     if (grp * BPT < kUpBT) {
-      const __half* bv = p.B_V + static_cast<size_t>(j0) * hd + static_cast<size_t>(h) * p.d + 2 * c2;
+      const int jn = min(kUpRC, p.R - c * kUpRC);
+      const __half* bv = bvs + static_cast<size_t>(buf) * kUpRC * p.d + 2 * c2;
+      const float* zr0 = zs + static_cast<size_t>(buf) * kUpRC * kUpBT + grp * BPT;
+#pragma unroll 4
       for (int j = 0; j < jn; ++j) {
-        const float2 w = __half22float2(*reinterpret_cast<const __half2*>(bv + j * hd));
-        const float* zr = &zs[j][grp * BPT];
+        const float2 w = __half22float2(*reinterpret_cast<const __half2*>(bv + j * p.d));
+        const float* zr = zr0 + j * kUpBT;
 #pragma unroll
         for (int u = 0; u < BPT; ++u) {
           acc[u][0] = fmaf(zr[u], w.x, acc[u][0]);
@@ -648,14 +732,16 @@ __global__ void __launch_bounds__(256) upproj_kernel(UpProjParams p) {
         }
       }
     }
+    __syncthreads();
   }
   if (grp * BPT < kUpBT) {
 #pragma unroll
     for (int u = 0; u < BPT; ++u) {
       const int b = bt0 + grp * BPT + u;
+      const float il = invl[grp * BPT + u];
       if (b < p.B)
         *reinterpret_cast<__half2*>(p.out + (static_cast<size_t>(b) * p.H + h) * p.d + 2 * c2) =
-            __floats2half2_rn(acc[u][0], acc[u][1]);
+            __floats2half2_rn(acc[u][0] * il, acc[u][1] * il);
     }
   }
 }

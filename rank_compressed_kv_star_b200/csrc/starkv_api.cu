@@ -51,7 +51,7 @@ starkv_status check_desc(const starkv_layer_desc* d) {
 struct DecodePlan {
   int H, d, r, R, B, MB, NB, cap, n_pages_max, t_pad, npad;
   // K pass
-  int L, CPL, tps, k_stages, k_ctas;
+  int L, CPT, log2H, tps, k_stages, k_ctas;
   uint32_t k_stage_bytes;
   size_t k_smem;
   // V pass
@@ -63,15 +63,14 @@ struct DecodePlan {
   starkv_workspace_layout ws;
 };
 
-void plan_kpass_shape(int r, int* L, int* CPL) {
+// Threads per (token, head) dot product and 16-byte chunks per thread.
+void plan_kpass_shape(int r, int* L, int* CPT) {
   const int cp = r / 8;
-  if (cp == 2) { *L = 2; *CPL = 1; }
-  else if (cp == 4) { *L = 4; *CPL = 1; }
-  else if (cp <= 8) { *L = 8; *CPL = 1; }
-  else if (cp == 12) { *L = 4; *CPL = 3; }
-  else if (cp <= 16) { *L = 8; *CPL = 2; }
-  else if (cp <= 24) { *L = 8; *CPL = 3; }
-  else { *L = 8; *CPL = 4; }
+  if (cp <= 4) { *L = 1; *CPT = 4; }        // r <= 32
+  else if (cp <= 8) { *L = 1; *CPT = 8; }   // r <= 64
+  else if (cp <= 12) { *L = 1; *CPT = 12; } // r <= 96
+  else if (cp <= 16) { *L = 2; *CPT = 8; }  // r <= 128
+  else { *L = 4; *CPT = 8; }                // r <= 256
 }
 
 starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_seq_len, DecodePlan* pl) {
@@ -90,17 +89,20 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   p.npad = p.H < 16 ? 16 : p.H;
   const int sms = device_sm_count();
 
-  // K pass: ~32 KiB ring stages of whole tokens, ~200 KiB of ring, one CTA per SM
-  plan_kpass_shape(p.r, &p.L, &p.CPL);
+  // K pass: ring stages of whole tokens (<= 48 KiB, ideally one full pass of
+  // the 256 dot-product threads), ~200 KiB of ring, one CTA per SM
+  plan_kpass_shape(p.r, &p.L, &p.CPT);
+  p.log2H = 0;
+  while ((1 << p.log2H) < p.H) ++p.log2H;
   const uint32_t tok = static_cast<uint32_t>(p.H) * p.r * 2;
   p.tps = 16;
-  while (p.tps > 1 && p.tps * tok > 32768u) p.tps >>= 1;
+  while (p.tps > 1 && p.tps * tok > 49152u) p.tps >>= 1;
   p.k_stage_bytes = p.tps * tok;
   p.k_stages = static_cast<int>(200u * 1024u / p.k_stage_bytes);
   if (p.k_stages > 8) p.k_stages = 8;
   if (p.k_stages < 2) p.k_stages = 2;
   p.k_smem = static_cast<size_t>(p.k_stages) * p.k_stage_bytes + p.k_stages * sizeof(StageMeta) +
-             2 * p.k_stages * sizeof(uint64_t) + (kKConsumers / p.L) * sizeof(float2);
+             2 * p.k_stages * sizeof(uint64_t) + (kKConsumers / p.L) * sizeof(float);
   p.k_ctas = sms;
 
   // V pass: R split into ranges of <= 1024 rows (128-row UMMA tiles)
@@ -121,7 +123,7 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   if (p.v_stages > 8) p.v_stages = 8;
   if (p.v_stages < 2) p.v_stages = 2;
   p.v_smem = 1024 + static_cast<size_t>(p.v_stages) * stage + p.v_stages * sizeof(StageMeta) +
-             (3 * p.v_stages + 3) * sizeof(uint64_t) + 2 * p.npad * sizeof(float);
+             (3 * p.v_stages + 3) * sizeof(uint64_t) + (p.npad + 128) * sizeof(float);
   int per_sm = static_cast<int>((227u * 1024u) / (p.v_smem + 1024));
   if (per_sm > static_cast<int>(512 / p.tmem_cols)) per_sm = 512 / p.tmem_cols;
   if (per_sm < 1) per_sm = 1;
@@ -143,10 +145,11 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   w.logits_off = off; off = align_up(off + static_cast<size_t>(batch) * p.t_pad * p.H * 4, 256);
   w.k_ctas = p.k_ctas;
   w.k_slots = p.k_ctas + batch;
-  w.ml_off = off; off = align_up(off + static_cast<size_t>(w.k_slots) * p.H * 2 * 4, 256);
-  w.stats_off = off; off = align_up(off + static_cast<size_t>(batch) * p.H * 2 * 4, 256);
+  w.mpart_off = off; off = align_up(off + static_cast<size_t>(w.k_slots) * p.H * 4, 256);
+  w.mx_off = off; off = align_up(off + static_cast<size_t>(batch) * p.H * 4, 256);
   w.v_ctas = p.v_ctas;
   w.v_slots = p.v_ctas + batch;
+  w.lpart_off = off; off = align_up(off + static_cast<size_t>(w.v_slots) * p.H * 4, 256);
   w.n_rranges = p.n_rr;
   w.r_range = p.r_range;
   w.zpart_off = off;
@@ -181,19 +184,26 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// V pool viewed as a 2-D matrix [num_blocks*16 rows][R] of fp16; boxes of
-// 64 columns x 16 rows (one page, one 128-byte-wide chunk) with 128B swizzle.
-bool encode_vpool_map(CUtensorMap* map, const void* v_cache, int R, int NB) {
+// Row-major fp16 matrix [rows][cols] as a 2-D tensor map with boxes of
+// box_cols (x 2 bytes = 128 bytes) by box_rows and the 128-byte swizzle.
+bool encode_2d_map(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                   uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(R), static_cast<cuuint64_t>(NB) * 16};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(R) * 2};
-  cuuint32_t box[2] = {64, 16};
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(v_cache), dims, strides, box, estr,
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// V pool viewed as a 2-D matrix [num_blocks*16 rows][R] of fp16; boxes of
+// 64 columns x 16 rows (one page, one 128-byte-wide chunk).
+bool encode_vpool_map(CUtensorMap* map, const void* v_cache, int R, int NB) {
+  return encode_2d_map(map, v_cache, static_cast<uint64_t>(R), static_cast<uint64_t>(NB) * 16, 64, 16);
 }
 
 // ------------------------------------------------------ kernel attributes
@@ -213,7 +223,9 @@ cudaError_t launch_kpass(const DecodePlan& pl, const KPassParams& kp, cudaStream
 template <int BPT>
 cudaError_t launch_upproj(const DecodePlan& pl, const UpProjParams& up, cudaStream_t s) {
   dim3 grid(pl.H, (pl.B + kUpBT - 1) / kUpBT);
-  upproj_kernel<BPT><<<grid, 256, 0, s>>>(up);
+  const size_t smem = 2 * (static_cast<size_t>(kUpRC) * pl.d * 2 + static_cast<size_t>(kUpRC) * kUpBT * 4);
+  if (!set_smem(upproj_kernel<BPT>, smem)) return cudaGetLastError();
+  upproj_kernel<BPT><<<grid, 256, smem, s>>>(up);
   return cudaGetLastError();
 }
 
@@ -260,23 +272,71 @@ starkv_status starkv_compress_append(const starkv_layer_desc* desc, int32_t batc
       !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
       (reinterpret_cast<uintptr_t>(positions) & 3u))
     return STARKV_ERR_INVALID_ARG;
-  if (desc->k_rank > 256) return STARKV_ERR_UNSUPPORTED;
-  AppendParams p;
-  p.k = static_cast<const __half*>(k);
-  p.v = static_cast<const __half*>(v);
-  p.A_K = static_cast<const __half*>(A_K);
-  p.A_V = static_cast<const __half*>(A_V);
-  p.tables = block_tables;
-  p.positions = positions;
-  p.k_cache = static_cast<__half*>(k_cache);
-  p.v_cache = static_cast<__half*>(v_cache);
-  p.B = batch; p.H = desc->num_heads; p.d = desc->head_dim; p.r = desc->k_rank; p.R = desc->v_rank;
-  p.MB = desc->max_blocks_per_seq; p.NB = desc->num_blocks;
-  p.nvx = p.R / kAppNC;
-  p.nby = (batch + kAppBT - 1) / kAppBT;
+  const int H = desc->num_heads, d = desc->head_dim, r = desc->k_rank, R = desc->v_rank;
+  const int HD = H * d;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  append_kernel<<<p.nvx * p.nby + p.H, 256, 0, s>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
+  AppendTarget tgt{block_tables, positions, desc->max_blocks_per_seq, desc->num_blocks};
+
+  // ---- joint V codes: tcgen05 GEMM, split-K over a cluster
+  CUtensorMap amap, vmap;
+  const int n_bt = (batch + 255) / 256;
+  const int bt_rows = batch < 256 ? batch : 256;
+  const int npad = (bt_rows + 15) / 16 * 16;
+  if (!encode_2d_map(&amap, A_V, static_cast<uint64_t>(R), static_cast<uint64_t>(HD), 64, kAppKC) ||
+      !encode_2d_map(&vmap, v, static_cast<uint64_t>(HD), static_cast<uint64_t>(batch), 64,
+                     static_cast<uint32_t>(npad)))
+    return STARKV_ERR_CUDA;
+  const int n_mt = (R + 127) / 128;
+  const int sms = device_sm_count();
+  int KS = 1;
+  while (KS < 8 && n_mt * n_bt * KS * 2 <= sms && (HD / kAppKC) >= KS * 2) KS *= 2;
+  AppendVParams vp;
+  vp.tgt = tgt;
+  vp.v_cache = static_cast<__half*>(v_cache);
+  vp.B = batch; vp.HD = HD; vp.R = R;
+  vp.k_per_cta = ((HD + KS * kAppKC - 1) / (KS * kAppKC)) * kAppKC;
+  vp.npad = npad;
+  vp.stages = 4;
+  vp.tmem_cols = static_cast<uint32_t>(pow2_ceil(npad < 32 ? 32 : npad));
+  const size_t stage_bytes = 2u * kAppKC * 128u + static_cast<size_t>(npad) * 128u;
+  const size_t smem = 1024 + vp.stages * stage_bytes + (2 * vp.stages + 1) * sizeof(uint64_t);
+  if (!set_smem(append_v_kernel, smem)) return STARKV_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_mt, KS, n_bt);
+  cfg.blockDim = dim3(kAppThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = KS;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, append_v_kernel, amap, vmap, vp) != cudaSuccess) {
+    cudaGetLastError();
+    return STARKV_ERR_CUDA;
+  }
+
+  // ---- head-wise K codes
+  AppendKParams kp;
+  kp.tgt = tgt;
+  kp.k = static_cast<const __half*>(k);
+  kp.A_K = static_cast<const __half*>(A_K);
+  kp.k_cache = static_cast<__half*>(k_cache);
+  kp.H = H; kp.d = d; kp.r = r;
+  const int bchunk = 256;
+  for (int b0 = 0; b0 < batch; b0 += bchunk) {
+    AppendKParams kq = kp;
+    kq.B = batch - b0 < bchunk ? batch - b0 : bchunk;
+    kq.k = kp.k + static_cast<size_t>(b0) * H * d;
+    kq.tgt.tables = block_tables + static_cast<size_t>(b0) * desc->max_blocks_per_seq;
+    kq.tgt.positions = positions + b0;
+    const size_t ksm = (static_cast<size_t>(d) * r + static_cast<size_t>(kq.B) * d) * 2;
+    if (!set_smem(append_k_kernel, ksm)) return STARKV_ERR_CUDA;
+    append_k_kernel<<<H, 256, ksm, s>>>(kq);
+    if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
+  }
   return STARKV_OK;
 }
 
@@ -321,8 +381,9 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   int32_t* teff = reinterpret_cast<int32_t*>(ws + teff_offset(pl));
   float* qt = reinterpret_cast<float*>(ws + pl.ws.qt_off);
   float* logits = reinterpret_cast<float*>(ws + pl.ws.logits_off);
-  float* ml = reinterpret_cast<float*>(ws + pl.ws.ml_off);
-  float* stats = reinterpret_cast<float*>(ws + pl.ws.stats_off);
+  float* mpart = reinterpret_cast<float*>(ws + pl.ws.mpart_off);
+  float* mx = reinterpret_cast<float*>(ws + pl.ws.mx_off);
+  float* lpart = reinterpret_cast<float*>(ws + pl.ws.lpart_off);
   float* zpart = reinterpret_cast<float*>(ws + pl.ws.zpart_off);
 
   if (max_seq_len == 0) {
@@ -353,30 +414,28 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   KPassParams kp;
   kp.k_cache = static_cast<const __half*>(k_cache);
   kp.tables = block_tables; kp.teff = teff; kp.prefix = prefix; kp.qt = qt;
-  kp.logits = logits; kp.ml = ml; kp.status = status;
-  kp.B = batch; kp.H = pl.H; kp.r = pl.r; kp.MB = pl.MB; kp.NB = pl.NB; kp.t_pad = pl.t_pad;
+  kp.logits = logits; kp.mpart = mpart; kp.status = status;
+  kp.B = batch; kp.H = pl.H; kp.log2H = pl.log2H; kp.r = pl.r; kp.MB = pl.MB; kp.NB = pl.NB; kp.t_pad = pl.t_pad;
   kp.tps = pl.tps; kp.stages = pl.k_stages; kp.stage_bytes = pl.k_stage_bytes;
   cudaError_t e;
-  if (pl.L == 2) e = launch_kpass<2, 1>(pl, kp, s);
-  else if (pl.L == 4 && pl.CPL == 1) e = launch_kpass<4, 1>(pl, kp, s);
-  else if (pl.L == 4) e = launch_kpass<4, 3>(pl, kp, s);
-  else if (pl.CPL == 1) e = launch_kpass<8, 1>(pl, kp, s);
-  else if (pl.CPL == 2) e = launch_kpass<8, 2>(pl, kp, s);
-  else if (pl.CPL == 3) e = launch_kpass<8, 3>(pl, kp, s);
-  else e = launch_kpass<8, 4>(pl, kp, s);
+  if (pl.L == 1 && pl.CPT == 4) e = launch_kpass<1, 4>(pl, kp, s);
+  else if (pl.L == 1 && pl.CPT == 8) e = launch_kpass<1, 8>(pl, kp, s);
+  else if (pl.L == 1) e = launch_kpass<1, 12>(pl, kp, s);
+  else if (pl.L == 2) e = launch_kpass<2, 8>(pl, kp, s);
+  else e = launch_kpass<4, 8>(pl, kp, s);
   if (e != cudaSuccess) return STARKV_ERR_CUDA;
   mark(2);
 
   ReduceParams rp;
-  rp.ml = ml; rp.prefix = prefix; rp.stats = stats;
+  rp.mpart = mpart; rp.prefix = prefix; rp.mx = mx;
   rp.B = batch; rp.H = pl.H; rp.k_grid = pl.k_ctas;
   reduce_kernel<<<(batch * pl.H + 255) / 256, 256, 0, s>>>(rp);
   if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
   mark(3);
 
   VPassParams vp;
-  vp.tables = block_tables; vp.teff = teff; vp.prefix = prefix; vp.logits = logits; vp.stats = stats;
-  vp.zpart = zpart; vp.status = status;
+  vp.tables = block_tables; vp.teff = teff; vp.prefix = prefix; vp.logits = logits; vp.mx = mx;
+  vp.zpart = zpart; vp.lpart = lpart; vp.status = status;
   vp.B = batch; vp.H = pl.H; vp.npad = pl.npad; vp.MB = pl.MB; vp.NB = pl.NB; vp.R = pl.R;
   vp.t_pad = pl.t_pad; vp.r_range = pl.r_range; vp.n_rr = pl.n_rr; vp.v_slots = pl.ws.v_slots;
   vp.stages = pl.v_stages; vp.n_chunks = pl.n_chunks; vp.n_mtiles = pl.n_mtiles; vp.tmem_cols = pl.tmem_cols;
@@ -387,7 +446,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   mark(4);
 
   UpProjParams up;
-  up.zpart = zpart; up.prefix = prefix;
+  up.zpart = zpart; up.lpart = lpart; up.prefix = prefix;
   up.B_V = static_cast<const __half*>(B_V);
   up.out = static_cast<__half*>(out);
   up.B = batch; up.H = pl.H; up.d = pl.d; up.R = pl.R; up.r_range = pl.r_range; up.v_slots = pl.ws.v_slots;
