@@ -155,7 +155,7 @@ def run_ours(args):
     ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
     outs = [torch.empty((B, L["H"], L["d"]), dtype=torch.float16, device="cuda") for L in layers]
     stream = torch.cuda.current_stream()
-    n_ev = 6
+    n_ev = 7
 
     def step(evs=None, app_evs=None, li_prof=None):
         for li, L in enumerate(layers):
@@ -217,7 +217,7 @@ def run_ours(args):
     if st != 0:
         raise RuntimeError(f"device status {S.STATUS[st]} flags {flags}")
 
-    names = ["absorb", "kpass", "reduce", "vpass", "upproj"]
+    names = ["absorb", "kpass", "reduce", "vpass", "zfinal", "upproj"]
     per = {n: 0.0 for n in names}
     per["append"] = 0.0
     for i in range(K):
@@ -301,7 +301,7 @@ def run_ours(args):
         "kernels_GBps": {"kpass": round(kp_gbs, 1), "vpass": round(vp_gbs, 1)},
         "e2e": {"value": round(world * B / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
-        "gpu_launches": K * len(layers) * 7,   # append: V GEMM + K codes; decode: 5
+        "gpu_launches": K * len(layers) * 8,   # append: V GEMM + K codes; decode: 6
         "clocks": clk,
     }
     if cpu is not None:

@@ -143,11 +143,12 @@ starkv_status starkv_paged_decode(const starkv_layer_desc* desc, int32_t batch, 
 /*
  * starkv_paged_decode_profiled -- starkv_paged_decode that also records CUDA
  * events on `stream` around its kernels, for per-kernel timing.
- * stage_events: HOST array of 6 cudaEvent_t (as void*; a NULL entry is
+ * stage_events: HOST array of 7 cudaEvent_t (as void*; a NULL entry is
  * skipped) recorded before the query absorption, after it, after the K pass,
- * after the split reduction, after the V pass and after the up-projection.
- * The events are not recorded when the call returns an error before launching
- * or when max_seq_len == 0.  Otherwise identical to starkv_paged_decode.
+ * after the split reduction, after the V pass, after the Z finalisation and
+ * after the up-projection.  The events are not recorded when the call returns
+ * an error before launching or when max_seq_len == 0.  Otherwise identical to
+ * starkv_paged_decode.
  */
 starkv_status starkv_paged_decode_profiled(const starkv_layer_desc* desc, int32_t batch,
                                            int32_t max_seq_len, const void* q, const void* B_K,
@@ -179,6 +180,8 @@ typedef struct {
   size_t mx_off;      /* fp32 [batch][H]: max of the base-2 logits per sequence */
   size_t lpart_off;   /* fp32 [v_slots][H]: per segment, sum of the fp16 weights exp2(s - max) */
   size_t zpart_off;   /* fp32 [n_rranges][v_slots][H][r_range]: per segment, sum_t w c_V */
+  size_t zhi_off;     /* fp16 [H][batch][R]: Z/L rounded to fp16 */
+  size_t zlo_off;     /* fp16 [H][batch][R]: Z/L minus its fp16 rounding, in fp16 */
   int32_t t_pad;      /* logits row capacity (multiple of 16) */
   int32_t k_ctas;     /* CTAs of the K pass (stream partition) */
   int32_t k_slots;    /* k_ctas + batch */

@@ -1,12 +1,13 @@
 // Decode kernels of the STAR-KV paged low-rank cache (sm_100a).
 //
-// One decode is five launches on the caller's stream:
+// One decode is six launches on the caller's stream:
 //   1. absorb      q~ = log2(e)*scale * q . B_K[h]^T; page prefix sums; status reset
 //   2. kpass       base-2 logits s = q~ . c_K over the K pages, per-segment max
 //   3. reduce      per (b, h): global max M of the logits
 //   4. vpass       Z = sum_t w c_V on tcgen05 tensor cores with w = fp16(exp2(s - M)),
 //                  and the normaliser L = sum_t w
-//   5. upproj      out_h = (Z_h . B_V[:, h*d:(h+1)*d]) / L -> fp16
+//   5. zfinal      Z / L summed over segments, split into fp16 hi + lo
+//   6. upproj      out_h = (Z_h / L) . B_V[:, h*d:(h+1)*d] on tcgen05 -> fp16
 //
 // The formulation (head-wise K with the query absorbed, joint V applied after
 // the weighted sum of codes) follows the STAR-KV description in the Proxima
@@ -23,6 +24,7 @@
 // up-projection visit the CTAs overlapping sequence b in increasing i, so every
 // result is independent of which physical pages hold the codes.
 #pragma once
+#include <cooperative_groups.h>
 #include <cstdint>
 #include <cuda_fp16.h>
 
@@ -82,12 +84,18 @@ struct AbsorbParams {
   float coef;             // scale * log2(e)
 };
 
-// grid (H), 256 threads.  CTA 0 also writes the page prefix sums and resets the
-// status word (every later kernel of the decode runs after this one).
+// grid (H, ceil(B/64)), 256 threads.  CTA (0, 0) also writes the page prefix
+// sums and resets the status word (every later kernel of the decode runs after
+// this one).  Thread = (rank index i, lane over the tile's sequences); its row
+// B_K[h][i][:] is held in registers and the tile's q rows are staged in shared
+// memory.
+constexpr int kAbsBT = 64;
+
+template <int D>
 __global__ void __launch_bounds__(256) absorb_kernel(AbsorbParams p) {
   const int h = blockIdx.x;
   const int tid = threadIdx.x;
-  if (h == 0) {
+  if (h == 0 && blockIdx.y == 0) {
     __shared__ int32_t part[256];
     __shared__ int32_t bad;
     if (tid == 0) bad = 0;
@@ -116,29 +124,41 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbParams p) {
       acc += (p.teff[b] + kBlock - 1) / kBlock;
     }
   }
+  __shared__ __align__(16) __half qs[kAbsBT * D];
+  const int bt0 = blockIdx.y * kAbsBT;
+  const int nb = min(kAbsBT, p.B - bt0);
+  for (int x = tid; x < nb * (D / 8); x += 256) {
+    const int bb = x / (D / 8), c = x % (D / 8);
+    reinterpret_cast<uint4*>(qs)[x] =
+        reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(bt0 + bb) * p.H + h) * D)[c];
+  }
+  __syncthreads();
   // q~[b,h,i] = coef * sum_j q[b,h,j] * B_K[h][i][j]
   const int i = tid % p.r;
   const int bpar = 256 / p.r;
   const int bs = tid / p.r;
   if (bs >= bpar) return;
-  const __half* brow = p.B_K + (static_cast<size_t>(h) * p.r + i) * p.d;
-  for (int b = bs; b < p.B; b += bpar) {
-    const __half* qrow = p.q + (static_cast<size_t>(b) * p.H + h) * p.d;
-    float acc = 0.f;
-    for (int j = 0; j < p.d; j += 8) {
-      const uint4 bw = *reinterpret_cast<const uint4*>(brow + j);
-      const uint4 qw = *reinterpret_cast<const uint4*>(qrow + j);
-      const __half2* b2 = reinterpret_cast<const __half2*>(&bw);
+  uint4 brow[D / 8];
+  const uint4* bsrc = reinterpret_cast<const uint4*>(p.B_K + (static_cast<size_t>(h) * p.r + i) * D);
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) brow[c] = bsrc[c];
+  for (int bb = bs; bb < nb; bb += bpar) {
+    const uint4* qrow = reinterpret_cast<const uint4*>(qs + bb * D);
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 qw = qrow[c];
+      const __half2* b2 = reinterpret_cast<const __half2*>(&brow[c]);
       const __half2* q2 = reinterpret_cast<const __half2*>(&qw);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const float2 bf = __half22float2(b2[u]);
         const float2 qf = __half22float2(q2[u]);
-        acc = fmaf(qf.x, bf.x, acc);
-        acc = fmaf(qf.y, bf.y, acc);
+        a0 = fmaf(qf.x, bf.x, a0);
+        a1 = fmaf(qf.y, bf.y, a1);
       }
     }
-    p.qt[(static_cast<size_t>(b) * p.H + h) * p.r + i] = acc * p.coef;
+    p.qt[(static_cast<size_t>(bt0 + bb) * p.H + h) * p.r + i] = (a0 + a1) * p.coef;
   }
 }
 
@@ -617,132 +637,191 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
   }
 }
 
-// ====================================================================== upproj
-struct UpProjParams {
+// ==================================================================== zfinal
+// Z / L per (sequence, head): the V-pass partials of the sequence's segments
+// summed in segment order, scaled by 1/L (L = the summed fp16 weights), and
+// split into fp16 hi + lo halves for the up-projection's B operand (hi + lo
+// keeps about 22 bits of the fp32 value).  Z / L is a convex combination of
+// fp16 codes, so both halves are in range.  Layout [H][B][R] (head-major) so
+// that one head's rows of a batch tile are contiguous.
+struct ZFinalParams {
   const float* zpart;     // [n_rr][v_slots][H][r_range]
   const float* lpart;     // [v_slots][H]
   const int32_t* prefix;
-  const __half* B_V;      // [R][H*d]
-  __half* out;            // [B][H][d]
-  int B, H, d, R, r_range, v_slots, v_grid;
+  __half* zhi;            // [H][B][R]
+  __half* zlo;            // [H][B][R]
+  int B, H, R, r_range, v_slots, v_grid;
 };
 
-constexpr int kUpBT = 16;   // sequences per CTA
-constexpr int kUpRC = 128;  // rows of B_V (and Z) staged per chunk
-
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-// grid (H, ceil(B/16)), 256 threads; dynamic smem 2 x (kUpRC*d halves + kUpRC*16 floats).
-// out[b,h,:] = (sum over the V-pass partials of sequence b) . B_V[:, h*d:(h+1)*d]
-template <int BPT>
-__global__ void __launch_bounds__(256) upproj_kernel(UpProjParams p) {
-  extern __shared__ __align__(16) uint8_t up_smem[];
-  __half* bvs = reinterpret_cast<__half*>(up_smem);                          // [2][kUpRC][d]
-  float* zs = reinterpret_cast<float*>(up_smem + 2 * kUpRC * p.d * 2);       // [2][kUpRC][kUpBT]
-  __shared__ int32_t i0s[kUpBT], i1s[kUpBT];
-  __shared__ float invl[kUpBT];
-  const int h = blockIdx.x;
-  const int bt0 = blockIdx.y * kUpBT;
-  const int tid = threadIdx.x;
-  const int half_d = p.d / 2;
-  const int c2 = tid % half_d;
-  const int grp = tid / half_d;
-  Partition pt;
-  pt.P = p.prefix[p.B];
-  pt.G = static_cast<int32_t>(pt.P < p.v_grid ? pt.P : p.v_grid);
-  if (tid < kUpBT) {
-    const int b = bt0 + tid;
-    int32_t a = 0, z = -1;
-    if (b < p.B && p.prefix[b + 1] > p.prefix[b]) {
-      a = part_owner(p.prefix[b], pt);
-      z = part_owner(p.prefix[b + 1] - 1, pt);
-    }
-    i0s[tid] = a;
-    i1s[tid] = z;
+// grid (ceil(R/1024), B*H), 256 threads x 4 consecutive rows of R
+__global__ void __launch_bounds__(256) zfinal_kernel(ZFinalParams p) {
+  const int bh = blockIdx.y;
+  const int b = bh / p.H, h = bh % p.H;
+  const int j = (blockIdx.x * 256 + threadIdx.x) * 4;
+  if (j >= p.R) return;
+  const size_t dst = (static_cast<size_t>(h) * p.B + b) * p.R + j;
+  float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int32_t f0 = p.prefix[b], f1 = p.prefix[b + 1];
+  if (f1 > f0) {
+    Partition pt;
+    pt.P = p.prefix[p.B];
+    pt.G = static_cast<int32_t>(pt.P < p.v_grid ? pt.P : p.v_grid);
+    const int32_t i0 = part_owner(f0, pt), i1 = part_owner(f1 - 1, pt);
     float Ls = 0.f;
-    for (int32_t i = a; i <= z; ++i) Ls += p.lpart[static_cast<size_t>(b + i) * p.H + h];
-    invl[tid] = Ls > 0.f ? 1.f / Ls : 0.f;
+    for (int32_t i = i0; i <= i1; ++i) Ls += p.lpart[static_cast<size_t>(b + i) * p.H + h];
+    const int rrg = j / p.r_range, jj = j % p.r_range;
+    const size_t stride = static_cast<size_t>(p.H) * p.r_range;
+    const float* src = p.zpart + ((static_cast<size_t>(rrg) * p.v_slots + b + i0) * p.H + h) * p.r_range + jj;
+    for (int32_t i = i0; i <= i1; ++i, src += stride) {
+      const float4 v = *reinterpret_cast<const float4*>(src);
+      z.x += v.x; z.y += v.y; z.z += v.z; z.w += v.w;
+    }
+    const float il = 1.f / Ls;
+    z.x *= il; z.y *= il; z.z *= il; z.w *= il;
+  }
+  const __half2 h01 = __floats2half2_rn(z.x, z.y), h23 = __floats2half2_rn(z.z, z.w);
+  const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+  const __half2 l01 = __floats2half2_rn(z.x - f01.x, z.y - f01.y);
+  const __half2 l23 = __floats2half2_rn(z.z - f23.x, z.w - f23.y);
+  uint2 hv, lv;
+  hv.x = *reinterpret_cast<const uint32_t*>(&h01); hv.y = *reinterpret_cast<const uint32_t*>(&h23);
+  lv.x = *reinterpret_cast<const uint32_t*>(&l01); lv.y = *reinterpret_cast<const uint32_t*>(&l23);
+  *reinterpret_cast<uint2*>(p.zhi + dst) = hv;
+  *reinterpret_cast<uint2*>(p.zlo + dst) = lv;
+}
+
+// ====================================================================== upproj
+// out_h^T (d x B) = B_V^h^T (d x R) . (Z_h / L)^T (R x B) on tcgen05 tensor
+// cores, two MMAs per K step (hi and lo halves of Z / L).  A = B_V^h^T from
+// 64x64 TMA boxes of B_V (MN-major, 128B swizzle); B from 64-column boxes of
+// the head's Z rows (K-major, 128B swizzle).  R is split over a cluster whose
+// partial sums are added through distributed shared memory in rank order.
+struct UpProjParams {
+  __half* out;            // [B][H][d]
+  int B, H, d, R;
+  int n_mt;               // 128-row tiles of d
+  int k_per_cta;          // rows of R per CTA (multiple of 64)
+  int npad;               // UMMA N (batch tile padded to 16)
+  int stages;
+  uint32_t tmem_cols;
+};
+
+constexpr int kUpThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kUpKC = 64;        // rows of R per stage
+
+// grid (H * n_mt * n_bt, KS), cluster (1, KS, 1)
+__global__ void __launch_bounds__(kUpThreads, 1)
+upproj_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__ CUtensorMap zhimap,
+              const __grid_constant__ CUtensorMap zlomap, UpProjParams p) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages;
+  const uint32_t a_bytes = 2u * kUpKC * 128u;                 // two 64x64 boxes of B_V
+  const uint32_t z_bytes = static_cast<uint32_t>(p.npad) * 128u;  // one 64-column box of Z rows
+  const uint32_t stage_bytes = a_bytes + 2 * z_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * stage_bytes);
+  uint64_t* empty = full + S;
+  uint64_t* done = empty + S;
+  float* part = reinterpret_cast<float*>(smem);              // [npad][128], reuses the ring
+  __shared__ uint32_t taddr_s;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int xi = blockIdx.x;
+  const int h = xi % p.H; xi /= p.H;
+  const int mt = xi % p.n_mt;
+  const int bt = xi / p.n_mt;
+  const int ks = blockIdx.y, KS = gridDim.y;
+  const int b0 = bt * 256;
+  const int k0 = ks * p.k_per_cta;
+  const int k1 = min(p.R, k0 + p.k_per_cta);
+  const int n_stages = k1 > k0 ? (k1 - k0 + kUpKC - 1) / kUpKC : 0;
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&taddr_s, p.tmem_cols);
+    tmem_relinquish();
+    tc_fence_before();
   }
   __syncthreads();
-  const size_t hd = static_cast<size_t>(p.H) * p.d;
-  const int n_chunks = (p.R + kUpRC - 1) / kUpRC;
-  const int vec_per_row = p.d / 8;  // 16-byte pieces of one B_V row slice
+  tc_fence_after();
+  const uint32_t taddr = taddr_s;
+  bool ok = true;
 
-  auto load_bv = [&](int chunk, int buf) {
-    const int j0 = chunk * kUpRC;
-    const int jn = min(kUpRC, p.R - j0);
-    __half* dst = bvs + static_cast<size_t>(buf) * kUpRC * p.d;
-    for (int x = tid; x < jn * vec_per_row; x += 256) {
-      const int j = x / vec_per_row, v = x % vec_per_row;
-      cp_async16(dst + j * p.d + v * 8, p.B_V + static_cast<size_t>(j0 + j) * hd + static_cast<size_t>(h) * p.d + v * 8);
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&bvmap);
+    prefetch_tensormap(&zhimap);
+    prefetch_tensormap(&zlomap);
+    const uint64_t pol = policy_evict_first();
+    const int col = h * p.d + mt * 128;
+    const int zrow = h * p.B + b0;
+    for (int i = 0; i < n_stages; ++i) {
+      const int s = i % S;
+      if (i >= S && !mbar_wait(&empty[s], ((i / S) - 1) & 1)) { ok = false; break; }
+      uint8_t* st = smem + static_cast<size_t>(s) * stage_bytes;
+      const int kr = k0 + i * kUpKC;
+      mbar_arrive_expect_tx(&full[s], stage_bytes);
+      tma_load_2d(st, &bvmap, col, kr, &full[s], pol);
+      tma_load_2d(st + kUpKC * 128, &bvmap, col + 64, kr, &full[s], pol);
+      tma_load_2d(st + a_bytes, &zhimap, kr, zrow, &full[s], pol);
+      tma_load_2d(st + a_bytes + z_bytes, &zlomap, kr, zrow, &full[s], pol);
     }
-  };
-  auto load_z = [&](int chunk, int buf) {
-    const int j0 = chunk * kUpRC;
-    const int jn = min(kUpRC, p.R - j0);
-    float* dst = zs + static_cast<size_t>(buf) * kUpRC * kUpBT;
-    for (int x = tid; x < jn * kUpBT; x += 256) {
-      const int bt = x / jn, j = j0 + x % jn;
-      const int b = bt0 + bt;
-      float z = 0.f;
-      if (b < p.B) {
-        const int rrg = j / p.r_range, jj = j % p.r_range;
-        const float* src = p.zpart + ((static_cast<size_t>(rrg) * p.v_slots + b) * p.H + h) * p.r_range + jj;
-        const size_t slot_stride = static_cast<size_t>(p.H) * p.r_range;
-        for (int32_t i = i0s[bt]; i <= i1s[bt]; ++i) z += src[static_cast<size_t>(i) * slot_stride];
-      }
-      dst[(j - j0) * kUpBT + bt] = z;
-    }
-  };
-
-  float acc[BPT][2];
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t idesc = idesc_f16_f32(128, p.npad, /*a_mn_major=*/true, /*b_mn_major=*/false);
+    for (int i = 0; i < n_stages; ++i) {
+      const int s = i % S;
+      if (!mbar_wait(&full[s], (i / S) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
+      const uint32_t shi = sa + a_bytes, slo = shi + z_bytes;
 #pragma unroll
-  for (int u = 0; u < BPT; ++u) acc[u][0] = acc[u][1] = 0.f;
-  load_bv(0, 0);
-  cp_async_commit();
-  load_z(0, 0);
-  for (int c = 0; c < n_chunks; ++c) {
-    const int buf = c & 1;
-    if (c + 1 < n_chunks) {
-      load_bv(c + 1, buf ^ 1);
-      cp_async_commit();
-      load_z(c + 1, buf ^ 1);
-      cp_async_wait_1();
-    } else {
-      cp_async_wait_0();
-    }
-    __syncthreads();
-    if (grp * BPT < kUpBT) {
-      const int jn = min(kUpRC, p.R - c * kUpRC);
-      const __half* bv = bvs + static_cast<size_t>(buf) * kUpRC * p.d + 2 * c2;
-      const float* zr0 = zs + static_cast<size_t>(buf) * kUpRC * kUpBT + grp * BPT;
-#pragma unroll 4
-      for (int j = 0; j < jn; ++j) {
-        const float2 w = __half22float2(*reinterpret_cast<const __half2*>(bv + j * p.d));
-        const float* zr = zr0 + j * kUpBT;
-#pragma unroll
-        for (int u = 0; u < BPT; ++u) {
-          acc[u][0] = fmaf(zr[u], w.x, acc[u][0]);
-          acc[u][1] = fmaf(zr[u], w.y, acc[u][1]);
-        }
+      for (int kk = 0; kk < kUpKC / 16; ++kk) {
+        const uint64_t adesc = smem_desc(sa + kk * 16u * 128u, kUpKC * 128u, 1024u, kSwizzle128B);
+        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+        umma_f16_ss(taddr, adesc, smem_desc(shi + kk * 32u, 16u, 1024u, kSwizzle128B), idesc, acc);
+        umma_f16_ss(taddr, adesc, smem_desc(slo + kk * 32u, 16u, 1024u, kSwizzle128B), idesc, 1u);
       }
+      umma_commit(&empty[s]);
     }
-    __syncthreads();
+    umma_commit(done);
   }
-  if (grp * BPT < kUpBT) {
+  __syncthreads();
+  if (!mbar_wait(done, 0)) ok = false;
+  tc_fence_after();
+  if (warp >= 2) {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    for (int c0 = 0; c0 < p.npad; c0 += 16) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x16(taddr + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
+      tmem_ld_wait();
 #pragma unroll
-    for (int u = 0; u < BPT; ++u) {
-      const int b = bt0 + grp * BPT + u;
-      const float il = invl[grp * BPT + u];
-      if (b < p.B)
-        *reinterpret_cast<__half2*>(p.out + (static_cast<size_t>(b) * p.H + h) * p.d + 2 * c2) =
-            __floats2half2_rn(acc[u][0] * il, acc[u][1] * il);
+      for (int jx = 0; jx < 16; ++jx)
+        part[(c0 + jx) * 128 + row] = (n_stages > 0 && ok) ? __uint_as_float(v[jx]) : 0.f;
     }
+  }
+  tc_fence_before();
+  cluster.sync();
+  const int per = (p.npad + KS - 1) / KS;
+  const int n_lo = ks * per, n_hi = min(p.npad, n_lo + per);
+  for (int x = tid; x < (n_hi - n_lo) * 128; x += kUpThreads) {
+    const int n = n_lo + x / 128, m = x % 128;
+    const int b = b0 + n;
+    const int dm = mt * 128 + m;
+    if (b >= p.B || dm >= p.d) continue;
+    float acc = 0.f;
+    for (int c = 0; c < KS; ++c) acc += cluster.map_shared_rank(part, c)[n * 128 + m];
+    p.out[(static_cast<size_t>(b) * p.H + h) * p.d + dm] = __float2half_rn(acc);
+  }
+  cluster.sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(taddr, p.tmem_cols);
   }
 }
 

@@ -58,8 +58,10 @@ struct DecodePlan {
   int n_rr, r_range, r_range_pad, n_chunks, n_mtiles, v_stages, v_ctas, v_per_sm;
   uint32_t vtile, ltile, ptile, tmem_cols;
   size_t v_smem;
-  // up-projection
-  int bpt;
+  // up-projection (tcgen05, split-K cluster)
+  int up_mt, up_bt, up_npad, up_ks, up_kpc, up_stages;
+  uint32_t up_tmem;
+  size_t up_smem;
   starkv_workspace_layout ws;
 };
 
@@ -132,7 +134,26 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   p.v_ctas = sms * per_sm / p.n_rr;
   if (p.v_ctas < 1) p.v_ctas = 1;
 
-  p.bpt = kUpBT * (p.d / 2) / 256;
+  p.up_mt = (p.d + 127) / 128;
+  p.up_bt = (batch + 255) / 256;
+  {
+    const int rows = batch < 256 ? batch : 256;
+    p.up_npad = rows < 16 ? 16 : (rows + 15) / 16 * 16;
+  }
+  p.up_ks = 1;
+  while (p.up_ks < 8 && p.H * p.up_mt * p.up_bt * p.up_ks * 2 <= sms && p.R / kUpKC >= p.up_ks * 2) p.up_ks *= 2;
+  p.up_kpc = ((p.R + p.up_ks * kUpKC - 1) / (p.up_ks * kUpKC)) * kUpKC;
+  {
+    // stage: two 64x64 B_V boxes + hi and lo Z boxes (npad rows x 128 B); the
+    // epilogue's [npad][128] fp32 partial reuses the ring (>= 2 stages always hold it)
+    const size_t stage = 2u * kUpKC * 128u + 2u * static_cast<size_t>(p.up_npad) * 128u;
+    p.up_stages = static_cast<int>((160u * 1024u) / stage);
+    if (p.up_stages > 4) p.up_stages = 4;
+    if (p.up_stages < 2) p.up_stages = 2;
+    while (static_cast<size_t>(p.up_stages) * stage < static_cast<size_t>(p.up_npad) * 512u) ++p.up_stages;
+    p.up_tmem = static_cast<uint32_t>(pow2_ceil(p.up_npad < 32 ? 32 : p.up_npad));
+    p.up_smem = 1024 + p.up_stages * stage + (2 * p.up_stages + 1) * sizeof(uint64_t);
+  }
 
   // workspace layout
   starkv_workspace_layout& w = p.ws;
@@ -154,6 +175,8 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   w.r_range = p.r_range;
   w.zpart_off = off;
   off = align_up(off + static_cast<size_t>(p.n_rr) * w.v_slots * p.H * p.r_range * 4, 256);
+  w.zhi_off = off; off = align_up(off + static_cast<size_t>(p.H) * batch * p.R * 2, 256);
+  w.zlo_off = off; off = align_up(off + static_cast<size_t>(p.H) * batch * p.R * 2, 256);
   w.t_pad = p.t_pad;
   w.total_bytes = off;
   return STARKV_OK;
@@ -220,13 +243,21 @@ cudaError_t launch_kpass(const DecodePlan& pl, const KPassParams& kp, cudaStream
   return cudaGetLastError();
 }
 
-template <int BPT>
-cudaError_t launch_upproj(const DecodePlan& pl, const UpProjParams& up, cudaStream_t s) {
-  dim3 grid(pl.H, (pl.B + kUpBT - 1) / kUpBT);
-  const size_t smem = 2 * (static_cast<size_t>(kUpRC) * pl.d * 2 + static_cast<size_t>(kUpRC) * kUpBT * 4);
-  if (!set_smem(upproj_kernel<BPT>, smem)) return cudaGetLastError();
-  upproj_kernel<BPT><<<grid, 256, smem, s>>>(up);
-  return cudaGetLastError();
+cudaError_t launch_cluster(const void* kernel_fn, dim3 grid, dim3 block, size_t smem, int cluster_y, cudaStream_t s,
+                           void** args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = cluster_y;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, kernel_fn, args);
 }
 
 }  // namespace
@@ -393,8 +424,16 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
     return STARKV_OK;
   }
 
-  CUtensorMap vmap;
+  __half* zhi = reinterpret_cast<__half*>(ws + pl.ws.zhi_off);
+  __half* zlo = reinterpret_cast<__half*>(ws + pl.ws.zlo_off);
+  CUtensorMap vmap, bvmap, zhimap, zlomap;
   if (!encode_vpool_map(&vmap, v_cache, pl.R, pl.NB)) return STARKV_ERR_CUDA;
+  if (!encode_2d_map(&bvmap, B_V, static_cast<uint64_t>(pl.H) * pl.d, static_cast<uint64_t>(pl.R), 64, kUpKC) ||
+      !encode_2d_map(&zhimap, zhi, static_cast<uint64_t>(pl.R), static_cast<uint64_t>(pl.H) * batch, 64,
+                     static_cast<uint32_t>(pl.up_npad)) ||
+      !encode_2d_map(&zlomap, zlo, static_cast<uint64_t>(pl.R), static_cast<uint64_t>(pl.H) * batch, 64,
+                     static_cast<uint32_t>(pl.up_npad)))
+    return STARKV_ERR_CUDA;
   auto mark = [&](int i) {
     if (stage_events && stage_events[i]) cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), s);
   };
@@ -407,7 +446,13 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   ap.qt = qt; ap.prefix = prefix; ap.teff = teff; ap.status = status;
   ap.B = batch; ap.H = pl.H; ap.d = pl.d; ap.r = pl.r; ap.cap = pl.cap;
   ap.coef = scale * kLog2e;
-  absorb_kernel<<<pl.H, 256, 0, s>>>(ap);
+  {
+    const dim3 grid(pl.H, (batch + kAbsBT - 1) / kAbsBT);
+    if (pl.d == 32) absorb_kernel<32><<<grid, 256, 0, s>>>(ap);
+    else if (pl.d == 64) absorb_kernel<64><<<grid, 256, 0, s>>>(ap);
+    else if (pl.d == 128) absorb_kernel<128><<<grid, 256, 0, s>>>(ap);
+    else absorb_kernel<256><<<grid, 256, 0, s>>>(ap);
+  }
   if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
   mark(1);
 
@@ -445,18 +490,29 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
   mark(4);
 
-  UpProjParams up;
-  up.zpart = zpart; up.lpart = lpart; up.prefix = prefix;
-  up.B_V = static_cast<const __half*>(B_V);
-  up.out = static_cast<__half*>(out);
-  up.B = batch; up.H = pl.H; up.d = pl.d; up.R = pl.R; up.r_range = pl.r_range; up.v_slots = pl.ws.v_slots;
-  up.v_grid = pl.v_ctas;
-  if (pl.bpt == 1) e = launch_upproj<1>(pl, up, s);
-  else if (pl.bpt == 2) e = launch_upproj<2>(pl, up, s);
-  else if (pl.bpt == 4) e = launch_upproj<4>(pl, up, s);
-  else e = launch_upproj<8>(pl, up, s);
-  if (e != cudaSuccess) return STARKV_ERR_CUDA;
+  ZFinalParams zf;
+  zf.zpart = zpart; zf.lpart = lpart; zf.prefix = prefix; zf.zhi = zhi; zf.zlo = zlo;
+  zf.B = batch; zf.H = pl.H; zf.R = pl.R; zf.r_range = pl.r_range; zf.v_slots = pl.ws.v_slots;
+  zf.v_grid = pl.v_ctas;
+  zfinal_kernel<<<dim3((pl.R + 1023) / 1024, batch * pl.H), 256, 0, s>>>(zf);
+  if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
   mark(5);
+
+  UpProjParams up;
+  up.out = static_cast<__half*>(out);
+  up.B = batch; up.H = pl.H; up.d = pl.d; up.R = pl.R;
+  up.n_mt = pl.up_mt; up.k_per_cta = pl.up_kpc; up.npad = pl.up_npad;
+  up.stages = pl.up_stages; up.tmem_cols = pl.up_tmem;
+  if (!set_smem(upproj_kernel, pl.up_smem)) return STARKV_ERR_CUDA;
+  {
+    void* args[] = {&bvmap, &zhimap, &zlomap, &up};
+    if (launch_cluster(reinterpret_cast<const void*>(upproj_kernel), dim3(pl.H * pl.up_mt * pl.up_bt, pl.up_ks),
+                       dim3(kUpThreads), pl.up_smem, pl.up_ks, s, args) != cudaSuccess) {
+      cudaGetLastError();
+      return STARKV_ERR_CUDA;
+    }
+  }
+  mark(6);
   return STARKV_OK;
 }
 }  // namespace
