@@ -44,18 +44,23 @@ def build_inputs(force: bool = False, verbose: bool = False) -> str:
     return GEN_LIB
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    if not force and not _stale(LIB, DEPS):
-        return LIB
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
+          defines: dict | None = None, out: str | None = None) -> str:
+    """Builds libstarkv.so; ``defines`` override launch-shape macros, ``out`` the path."""
+    target = out or LIB
+    if not force and not defines and not _stale(target, DEPS):
+        return target
     cmd = [NVCC, *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-           "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp", *SOURCES]
+           "-I", os.path.join(ROOT, "include"), "-o", target + ".tmp", *SOURCES]
+    for k, v in (defines or {}).items():
+        cmd.append(f"-D{k}={v}")
     if ptxas_info:
         cmd.insert(1, "-Xptxas=-v")
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(target + ".tmp", target)
+    return target
 
 
 if __name__ == "__main__":

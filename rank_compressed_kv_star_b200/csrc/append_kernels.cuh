@@ -173,33 +173,41 @@ struct AppendKParams {
   int B, H, d, r;
 };
 
-// grid (H), 256 threads; dynamic smem: A_K[h] (d*r halves) + k[:, h, :] (B*d halves)
+// grid (H, ceil(B/kAppKB)), 256 threads; dynamic smem: A_K[h] (d*r halves) +
+// the tile's k[:, h, :] rows (kAppKB*d halves).  Thread = (rank index, lane
+// over the tile's sequences).
+constexpr int kAppKB = 8;
+
 __global__ void __launch_bounds__(256) append_k_kernel(AppendKParams p) {
   extern __shared__ __align__(16) uint8_t ks_smem[];
   __half* As = reinterpret_cast<__half*>(ks_smem);              // [d][r]
-  __half* ksm = As + static_cast<size_t>(p.d) * p.r;            // [B][d]
+  __half* ksm = As + static_cast<size_t>(p.d) * p.r;            // [kAppKB][d]
   const int h = blockIdx.x, tid = threadIdx.x;
+  const int bt0 = blockIdx.y * kAppKB;
+  const int nb = min(kAppKB, p.B - bt0);
   const uint4* asrc = reinterpret_cast<const uint4*>(p.A_K + static_cast<size_t>(h) * p.d * p.r);
   for (int x = tid; x < p.d * p.r / 8; x += 256) reinterpret_cast<uint4*>(As)[x] = asrc[x];
-  for (int x = tid; x < p.B * p.d / 8; x += 256) {
+  for (int x = tid; x < nb * p.d / 8; x += 256) {
     const int b = x / (p.d / 8), c = x % (p.d / 8);
     reinterpret_cast<uint4*>(ksm)[x] =
-        reinterpret_cast<const uint4*>(p.k + (static_cast<size_t>(b) * p.H + h) * p.d)[c];
+        reinterpret_cast<const uint4*>(p.k + (static_cast<size_t>(bt0 + b) * p.H + h) * p.d)[c];
   }
   __syncthreads();
   const int i = tid % p.r;
   const int bpar = 256 / p.r;
   const int bs = tid / p.r;
   if (bs >= bpar) return;
-  for (int b = bs; b < p.B; b += bpar) {
+  for (int b = bs; b < nb; b += bpar) {
     const __half* kr = ksm + static_cast<size_t>(b) * p.d;
-    float a0 = 0.f, a1 = 0.f;
-    for (int j = 0; j < p.d; j += 2) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    for (int j = 0; j < p.d; j += 4) {
       a0 = fmaf(__half2float(kr[j]), __half2float(As[j * p.r + i]), a0);
       a1 = fmaf(__half2float(kr[j + 1]), __half2float(As[(j + 1) * p.r + i]), a1);
+      a2 = fmaf(__half2float(kr[j + 2]), __half2float(As[(j + 2) * p.r + i]), a2);
+      a3 = fmaf(__half2float(kr[j + 3]), __half2float(As[(j + 3) * p.r + i]), a3);
     }
-    const int64_t row = append_row(p.tgt, b);
-    if (row >= 0) p.k_cache[(row * p.H + h) * p.r + i] = __float2half_rn(a0 + a1);
+    const int64_t row = append_row(p.tgt, bt0 + b);
+    if (row >= 0) p.k_cache[(row * p.H + h) * p.r + i] = __float2half_rn((a0 + a1) + (a2 + a3));
   }
 }
 

@@ -84,12 +84,12 @@ struct AbsorbParams {
   float coef;             // scale * log2(e)
 };
 
-// grid (H, ceil(B/64)), 256 threads.  CTA (0, 0) also writes the page prefix
+// grid (H, ceil(B/16)), 256 threads.  CTA (0, 0) also writes the page prefix
 // sums and resets the status word (every later kernel of the decode runs after
 // this one).  Thread = (rank index i, lane over the tile's sequences); its row
 // B_K[h][i][:] is held in registers and the tile's q rows are staged in shared
 // memory.
-constexpr int kAbsBT = 64;
+constexpr int kAbsBT = 16;
 
 template <int D>
 __global__ void __launch_bounds__(256) absorb_kernel(AbsorbParams p) {
@@ -206,8 +206,12 @@ __device__ __forceinline__ int chunk_rotation(int tid, int cp, int L) {
 // CPT 16-byte chunks (8 codes) of its row in a rotated order and accumulates
 // with packed fp32 FMAs against its head's absorbed query held in registers.
 // The head of a thread is fixed because (kKConsumers / L) is a multiple of H.
+#ifndef STARKV_K_CTAS_PER_SM
+#define STARKV_K_CTAS_PER_SM 1
+#endif
+
 template <int L, int CPT>
-__global__ void __launch_bounds__(kKThreads, 1) kpass_kernel(KPassParams p) {
+__global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(KPassParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int S = p.stages;
   uint8_t* ring = smem;

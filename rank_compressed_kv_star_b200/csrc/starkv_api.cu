@@ -12,6 +12,23 @@
 #include "append_kernels.cuh"
 #include "decode_kernels.cuh"
 
+// Launch-shape defaults (overridable at build time for tuning sweeps).
+#ifndef STARKV_K_CTAS_PER_SM
+#define STARKV_K_CTAS_PER_SM 1
+#endif
+#ifndef STARKV_K_STAGE_CAP
+#define STARKV_K_STAGE_CAP 65536
+#endif
+#ifndef STARKV_K_RING_BYTES
+#define STARKV_K_RING_BYTES (200 * 1024 / STARKV_K_CTAS_PER_SM)
+#endif
+#ifndef STARKV_V_RRANGE
+#define STARKV_V_RRANGE 1024
+#endif
+#ifndef STARKV_V_RING_BYTES
+#define STARKV_V_RING_BYTES (105 * 1024)
+#endif
+
 namespace starkv {
 namespace {
 
@@ -91,26 +108,27 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   p.npad = p.H < 16 ? 16 : p.H;
   const int sms = device_sm_count();
 
-  // K pass: ring stages of whole tokens (<= 48 KiB, ideally one full pass of
-  // the 256 dot-product threads), ~200 KiB of ring, one CTA per SM
+  // K pass: ring stages of whole tokens, up to one whole 16-token page per bulk
+  // copy (64 KiB at H=32, r=64: large copies measured fastest), ~200 KiB of
+  // ring, one CTA per SM
   plan_kpass_shape(p.r, &p.L, &p.CPT);
   p.log2H = 0;
   while ((1 << p.log2H) < p.H) ++p.log2H;
   const uint32_t tok = static_cast<uint32_t>(p.H) * p.r * 2;
   p.tps = 16;
-  while (p.tps > 1 && p.tps * tok > 49152u) p.tps >>= 1;
+  while (p.tps > 1 && p.tps * tok > static_cast<uint32_t>(STARKV_K_STAGE_CAP)) p.tps >>= 1;
   p.k_stage_bytes = p.tps * tok;
-  p.k_stages = static_cast<int>(200u * 1024u / p.k_stage_bytes);
+  p.k_stages = static_cast<int>(static_cast<uint32_t>(STARKV_K_RING_BYTES) / p.k_stage_bytes);
   if (p.k_stages > 8) p.k_stages = 8;
   if (p.k_stages < 2) p.k_stages = 2;
   p.k_smem = static_cast<size_t>(p.k_stages) * p.k_stage_bytes + p.k_stages * sizeof(StageMeta) +
              2 * p.k_stages * sizeof(uint64_t) + (kKConsumers / p.L) * sizeof(float);
-  p.k_ctas = sms;
+  p.k_ctas = sms * STARKV_K_CTAS_PER_SM;
 
   // V pass: R split into ranges of <= 1024 rows (128-row UMMA tiles)
-  if (p.R <= 1024) { p.n_rr = 1; p.r_range = p.R; }
+  if (p.R <= STARKV_V_RRANGE) { p.n_rr = 1; p.r_range = p.R; }
   else {
-    p.n_rr = (p.R + 1023) / 1024;
+    p.n_rr = (p.R + STARKV_V_RRANGE - 1) / STARKV_V_RRANGE;
     p.r_range = ((p.R + p.n_rr - 1) / p.n_rr + 127) / 128 * 128;
   }
   p.r_range_pad = (p.r_range + 127) / 128 * 128;
@@ -121,7 +139,7 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   p.ptile = static_cast<uint32_t>(p.npad) * 16 * 2;
   p.tmem_cols = static_cast<uint32_t>(pow2_ceil(p.n_mtiles * p.npad < 32 ? 32 : p.n_mtiles * p.npad));
   const uint32_t stage = p.vtile + p.ltile + p.ptile;
-  p.v_stages = static_cast<int>((105u * 1024u) / stage);
+  p.v_stages = static_cast<int>(static_cast<uint32_t>(STARKV_V_RING_BYTES) / stage);
   if (p.v_stages > 8) p.v_stages = 8;
   if (p.v_stages < 2) p.v_stages = 2;
   p.v_smem = 1024 + static_cast<size_t>(p.v_stages) * stage + p.v_stages * sizeof(StageMeta) +
@@ -356,18 +374,11 @@ starkv_status starkv_compress_append(const starkv_layer_desc* desc, int32_t batc
   kp.A_K = static_cast<const __half*>(A_K);
   kp.k_cache = static_cast<__half*>(k_cache);
   kp.H = H; kp.d = d; kp.r = r;
-  const int bchunk = 256;
-  for (int b0 = 0; b0 < batch; b0 += bchunk) {
-    AppendKParams kq = kp;
-    kq.B = batch - b0 < bchunk ? batch - b0 : bchunk;
-    kq.k = kp.k + static_cast<size_t>(b0) * H * d;
-    kq.tgt.tables = block_tables + static_cast<size_t>(b0) * desc->max_blocks_per_seq;
-    kq.tgt.positions = positions + b0;
-    const size_t ksm = (static_cast<size_t>(d) * r + static_cast<size_t>(kq.B) * d) * 2;
-    if (!set_smem(append_k_kernel, ksm)) return STARKV_ERR_CUDA;
-    append_k_kernel<<<H, 256, ksm, s>>>(kq);
-    if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
-  }
+  kp.B = batch;
+  const size_t ksm = (static_cast<size_t>(d) * r + static_cast<size_t>(kAppKB) * d) * 2;
+  if (!set_smem(append_k_kernel, ksm)) return STARKV_ERR_CUDA;
+  append_k_kernel<<<dim3(H, (batch + kAppKB - 1) / kAppKB), 256, ksm, s>>>(kp);
+  if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
   return STARKV_OK;
 }
 
