@@ -158,6 +158,31 @@ starkv_status starkv_paged_decode_profiled(const starkv_layer_desc* desc, int32_
                                            void* out, void* stream, void* const* stage_events);
 
 /*
+ * starkv_paged_decode_static -- starkv_paged_decode for callers that cannot
+ * allocate device memory at decode time: an engine that has already handed
+ * nearly all GPU memory to its paged KV pool, or a C host with no allocator to
+ * provide scratch.  Same arguments and results as starkv_paged_decode minus
+ * the workspace: the scratch is a fixed 64 MiB device array inside the library
+ * (held by every GPU that loads the library until the process exits).  This
+ * call allocates nothing.
+ *  - Problems whose starkv_decode_workspace_bytes() exceeds 64 MiB are
+ *    rejected with STARKV_ERR_WORKSPACE before any launch.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any
+ *    stream capture.
+ *  - All calls share the one array per device: calls that overlap on the GPU
+ *    (different streams, or concurrent host threads on one device) race and
+ *    give undefined results.  Calls ordered on one stream are safe.
+ *  - The device status word is not exposed for this variant.
+ * The method pages have no counterpart to this entry point.
+ */
+starkv_status starkv_paged_decode_static(const starkv_layer_desc* desc, int32_t batch,
+                                         int32_t max_seq_len, const void* q, const void* B_K,
+                                         const void* B_V, const void* k_cache, const void* v_cache,
+                                         const int32_t* block_tables, const int32_t* seq_lens,
+                                         float scale, void* out, void* stream);
+
+/*
  * starkv_decode_check -- synchronise `stream` and read the device status word
  * the last decode on `workspace` left.  *flags_out receives STARKV_FLAG_* bits
  * (0 when clean).  Returns STARKV_OK when clean, STARKV_ERR_TIMEOUT when the

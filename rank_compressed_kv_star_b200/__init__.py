@@ -25,7 +25,7 @@ FLAG_BAD_BLOCK_ID, FLAG_BAD_SEQ_LEN, FLAG_TIMEOUT = 1, 2, 4
 
 EXPORTED = (
     "starkv_compress_append", "starkv_decode_workspace_bytes", "starkv_paged_decode",
-    "starkv_paged_decode_profiled",
+    "starkv_paged_decode_profiled", "starkv_paged_decode_static",
     "starkv_decode_check", "starkv_decode_workspace_layout", "starkv_status_string",
     "starkv_rank_from_spectrum", "starkv_version",
 )
@@ -86,6 +86,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.starkv_paged_decode_profiled.argtypes = [DP, I32, I32, P, P, P, P, P, P, P, ctypes.c_float,
                                                  P, SZ, P, P, ctypes.POINTER(P)]
     lib.starkv_paged_decode_profiled.restype = ctypes.c_int
+    lib.starkv_paged_decode_static.argtypes = [DP, I32, I32, P, P, P, P, P, P, P, ctypes.c_float, P, P]
+    lib.starkv_paged_decode_static.restype = ctypes.c_int
     lib.starkv_decode_check.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
     lib.starkv_decode_check.restype = ctypes.c_int
     lib.starkv_decode_workspace_layout.argtypes = [DP, I32, I32, ctypes.POINTER(WorkspaceLayout)]
@@ -173,6 +175,18 @@ def starkv_paged_decode_profiled(desc: LayerDesc, batch: int, max_seq_len: int, 
         int(workspace_bytes), _ptr(out), _stream(stream), arr)
     if check:
         _check(st, "starkv_paged_decode_profiled")
+    return st
+
+
+def starkv_paged_decode_static(desc: LayerDesc, batch: int, max_seq_len: int, q, B_K, B_V, k_cache,
+                               v_cache, block_tables, seq_lens, scale: float, out, stream=None,
+                               check: bool = True) -> int:
+    """Decode with the library's fixed device scratch (no workspace argument)."""
+    st = load_library().starkv_paged_decode_static(
+        _desc_ref(desc), batch, max_seq_len, _ptr(q), _ptr(B_K), _ptr(B_V), _ptr(k_cache),
+        _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), float(scale), _ptr(out), _stream(stream))
+    if check:
+        _check(st, "starkv_paged_decode_static")
     return st
 
 

@@ -546,6 +546,54 @@ starkv_status starkv_paged_decode_profiled(const starkv_layer_desc* desc, int32_
                      workspace, workspace_bytes, out, stream, stage_events);
 }
 
+// ---------------------------------------------------------------------------
+// Decode without a caller-provided workspace.  Some callers cannot allocate
+// device memory when they decode: a serving engine that reserved nearly all of
+// the GPU's memory for its paged KV pool up front (a later cudaMalloc fails or
+// eats into the pool), or a plain C host that has no allocator of its own to
+// hand out scratch.  For them the scratch lives in this fixed device array,
+// which every GPU that loads the library holds until the process exits.
+#define STARKV_STATIC_WS_BYTES (64ull << 20)
+static __device__ __align__(256) uint8_t g_starkv_static_ws[STARKV_STATIC_WS_BYTES];
+
+namespace {
+std::mutex g_static_ws_mu;
+void* g_static_ws_ptr[64] = {};
+
+// Device address of the array on the current device, looked up once per device
+// (host code may not use the symbol itself: it names a host-side stand-in).
+void* static_ws_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_static_ws_mu);
+  if (!g_static_ws_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_starkv_static_ws) != cudaSuccess || !ptr) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_static_ws_ptr[dev] = ptr;
+  }
+  return g_static_ws_ptr[dev];
+}
+}  // namespace
+
+starkv_status starkv_paged_decode_static(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len,
+                                         const void* q, const void* B_K, const void* B_V, const void* k_cache,
+                                         const void* v_cache, const int32_t* block_tables,
+                                         const int32_t* seq_lens, float scale, void* out, void* stream) {
+  DecodePlan pl;
+  starkv_status st = make_plan(desc, batch, max_seq_len, &pl);
+  if (st != STARKV_OK) return st;
+  if (pl.ws.total_bytes > STARKV_STATIC_WS_BYTES) return STARKV_ERR_WORKSPACE;
+  if (batch == 0) return decode_impl(desc, batch, max_seq_len, q, B_K, B_V, k_cache, v_cache, block_tables,
+                                     seq_lens, scale, nullptr, 0, out, stream, nullptr);
+  void* ws = static_ws_address();
+  if (!ws) return STARKV_ERR_CUDA;
+  return decode_impl(desc, batch, max_seq_len, q, B_K, B_V, k_cache, v_cache, block_tables, seq_lens, scale, ws,
+                     STARKV_STATIC_WS_BYTES, out, stream, nullptr);
+}
+
 starkv_status starkv_decode_check(const void* workspace, void* stream, int32_t* flags_out) {
   if (!workspace || !flags_out) return STARKV_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
