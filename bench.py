@@ -53,6 +53,9 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="budget of the oracle CPU-baseline sample")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="profiling only: override the batch with uniform lengths --seq")
+    ap.add_argument("--seq", type=int, default=0)
     return ap.parse_args()
 
 
@@ -144,6 +147,9 @@ def run_ours(args):
     S.load_library()
 
     wl = W.workload(args.workload)
+    if args.batch:
+        wl = W.Workload(f"{wl.name} (override: batch {args.batch}, length {args.seq})", wl.seed,
+                        args.batch, wl.layers[:1], np.full(args.batch, args.seq - 1, dtype=np.int64))
     layers = []
     for li in range(len(wl.layers)):
         Ld = D.device_layer(wl, li)
@@ -285,7 +291,8 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16", "accum": "f32", "data": "synthetic",
-        "config": {"workload": f"cfg{args.workload}: {WORKLOAD_NAMES[args.workload]}", "batch": B,
+        "config": {"workload": (f"cfg{args.workload}: {WORKLOAD_NAMES[args.workload]}" if not args.batch
+                                else wl.name), "batch": B,
                    "max_seq_len": max_len, "layers": len(layers),
                    "step": "compress-append of one token per sequence + paged decode, every layer",
                    "l2": "inputs larger than L2 (code pools of %.2f GiB read per step)" % ((k_bytes + v_bytes) / 2**30),

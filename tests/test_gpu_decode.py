@@ -332,16 +332,27 @@ def test_append_then_decode_continuous_batching_subset(layer):
 
 # ---------------------------------------------------- full-size workloads
 
-@pytest.mark.parametrize("idx,sample", [(2, range(16)), (3, [0, 31, 63])])
-def test_decode_full_size_sampled(idx, sample):
+@pytest.mark.parametrize("idx,layer,sample", [
+    (2, 0, list(range(16))),            # batch 16, context 2048: every sequence
+    (3, 0, [0, 31, 63]),                # batch 64, context 8192
+    (4, 0, [0, 17, 47]),                # batch 48, mixed lengths, r=32 / R=1024
+    (4, 1, [5, 23]),                    #   r=64 / R=2048
+    (4, 2, [11, 40]),                   #   r=96 / R=3072
+    (5, 0, [0, 7]),                     # 32-layer 7B attention path, first layer
+    (5, 31, [3]),                       #   last layer
+])
+def test_decode_full_size_sampled(idx, layer, sample):
+    """Full-size workloads in the benchmark's launch configuration, sampled rows."""
     wl = W.workload(idx)
-    Ld = D.device_layer(wl, 0)
+    Ld = D.device_layer(wl, layer)
     S.starkv_compress_append(desc_of(Ld), wl.batch, Ld["k"], Ld["v"], Ld["A_K"], Ld["A_V"],
                              Ld["tables"], Ld["ctx_lens"], Ld["k_cache"], Ld["v_cache"])
     got, *_ = run_decode(Ld)
     A_K, A_V, B_K, B_V = Ld["A_np"]
     cK, cV = O.compress(Ld["k"].cpu().numpy(), Ld["v"].cpu().numpy(), A_K, A_V)
-    ref = oracle_rows(wl, 0, Ld["q"].cpu().numpy(), Ld["A_np"], sample, wl.seq_lens,
+    ref = oracle_rows(wl, layer, Ld["q"].cpu().numpy(), Ld["A_np"], sample, wl.seq_lens,
                       (cK.astype(np.float16), cV.astype(np.float16)))
     assert_close({b: got[b] for b in sample}, ref)
     assert np.isfinite(got).all()
+    del Ld
+    torch.cuda.empty_cache()
