@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--workload", type=int, default=3, choices=[2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--profile-steps", type=int, default=300,
+                    help="steps of the event-instrumented region giving per-kernel times")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="budget of the oracle CPU-baseline sample")
     ap.add_argument("--batch", type=int, default=0,
@@ -161,7 +163,7 @@ def run_ours(args):
     ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
     outs = [torch.empty((B, L["H"], L["d"]), dtype=torch.float16, device="cuda") for L in layers]
     stream = torch.cuda.current_stream()
-    n_ev = 7
+    n_ev = 6
 
     def step(evs=None, app_evs=None, li_prof=None):
         for li, L in enumerate(layers):
@@ -188,16 +190,6 @@ def run_ours(args):
 
     # ---------------- device-timed region: inputs resident, codes >> L2 per step
     K = args.steps
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in layers] for _ in range(K)]
-    app_evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in layers] for _ in range(K)]
-    # torch creates the underlying cudaEvent at the first record: do that now so
-    # the raw handles handed to the library are valid
-    for step_evs in (evs, app_evs):
-        for per_step in step_evs:
-            for per_layer in per_step:
-                for e in per_layer:
-                    e.record(stream)
-    torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     uuid = None
     try:
@@ -212,7 +204,7 @@ def run_ours(args):
     time.sleep(0.3)
     t0.record(stream)
     for i in range(K):
-        step(evs[i], app_evs[i])
+        step()
     t1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -223,16 +215,32 @@ def run_ours(args):
     if st != 0:
         raise RuntimeError(f"device status {S.STATUS[st]} flags {flags}")
 
-    names = ["absorb", "kpass", "reduce", "vpass", "zfinal", "upproj"]
+    # ---------------- per-kernel durations: a second timed region of the same
+    # steps with CUDA events recorded between the kernels on the launching stream
+    Kp = max(1, min(K, args.profile_steps))
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in layers] for _ in range(Kp)]
+    app_evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in layers] for _ in range(Kp)]
+    # torch creates the underlying cudaEvent at the first record: do that now so
+    # the raw handles handed to the library are valid
+    for step_evs in (evs, app_evs):
+        for per_step in step_evs:
+            for per_layer in per_step:
+                for e in per_layer:
+                    e.record(stream)
+    torch.cuda.synchronize()
+    for i in range(Kp):
+        step(evs[i], app_evs[i])
+    torch.cuda.synchronize()
+    names = ["absorb", "kpass", "vpass", "zfinal", "upproj"]
     per = {n: 0.0 for n in names}
     per["append"] = 0.0
-    for i in range(K):
+    for i in range(Kp):
         for li in range(len(layers)):
             e = evs[i][li]
             for j, n in enumerate(names):
                 per[n] += e[j].elapsed_time(e[j + 1])
             per["append"] += app_evs[i][li][0].elapsed_time(app_evs[i][li][1])
-    per = {n: v / K for n, v in per.items()}             # ms per step (all layers)
+    per = {n: v / Kp for n, v in per.items()}             # ms per step (all layers)
 
     if world > 1:
         t = torch.tensor([ms], device="cuda", dtype=torch.float64)
@@ -305,10 +313,11 @@ def run_ours(args):
                      "unit": "GB/s", "frac": round(dom_gbs / peak, 4), "traffic": None,
                      "algorithmic_bytes_per_launch": dom_bytes // len(layers), "peak_kind": peak_kind},
         "kernels_ms_per_step": {n: round(v, 5) for n, v in per.items()},
+        "kernels_timing": f"CUDA events between kernels over {Kp} further steps (vpass includes the split reduction)",
         "kernels_GBps": {"kpass": round(kp_gbs, 1), "vpass": round(vp_gbs, 1)},
         "e2e": {"value": round(world * B / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
-        "gpu_launches": K * len(layers) * 8,   # append: V GEMM + K codes; decode: 6
+        "gpu_launches": K * len(layers) * 7,   # append: V GEMM + K codes; decode: 5
         "clocks": clk,
     }
     if cpu is not None:

@@ -93,6 +93,8 @@ append_v_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
   tc_fence_after();
   const uint32_t taddr = taddr_s;
   bool ok = true;
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&amap);
@@ -183,6 +185,8 @@ __global__ void __launch_bounds__(256) append_k_kernel(AppendKParams p) {
   __half* As = reinterpret_cast<__half*>(ks_smem);              // [d][r]
   __half* ksm = As + static_cast<size_t>(p.d) * p.r;            // [kAppKB][d]
   const int h = blockIdx.x, tid = threadIdx.x;
+  griddep_wait();
+  griddep_launch_dependents();
   const int bt0 = blockIdx.y * kAppKB;
   const int nb = min(kAppKB, p.B - bt0);
   const uint4* asrc = reinterpret_cast<const uint4*>(p.A_K + static_cast<size_t>(h) * p.d * p.r);

@@ -1,13 +1,14 @@
 // Decode kernels of the STAR-KV paged low-rank cache (sm_100a).
 //
-// One decode is six launches on the caller's stream:
+// One decode is five launches on the caller's stream, each launched with
+// programmatic stream serialisation (see griddep_wait):
 //   1. absorb      q~ = log2(e)*scale * q . B_K[h]^T; page prefix sums; status reset
 //   2. kpass       base-2 logits s = q~ . c_K over the K pages, per-segment max
-//   3. reduce      per (b, h): global max M of the logits
-//   4. vpass       Z = sum_t w c_V on tcgen05 tensor cores with w = fp16(exp2(s - M)),
+//   3. vpass       split reduction M = max over the sequence's K segments, then
+//                  Z = sum_t w c_V on tcgen05 tensor cores with w = fp16(exp2(s - M)),
 //                  and the normaliser L = sum_t w
-//   5. zfinal      Z / L summed over segments, split into fp16 hi + lo
-//   6. upproj      out_h = (Z_h / L) . B_V[:, h*d:(h+1)*d] on tcgen05 -> fp16
+//   4. zfinal      Z / L summed over segments, split into fp16 hi + lo
+//   5. upproj      out_h = (Z_h / L) . B_V[:, h*d:(h+1)*d] on tcgen05 -> fp16
 //
 // The formulation (head-wise K with the query absorbed, joint V applied after
 // the weighted sum of codes) follows the STAR-KV description in the Proxima
@@ -95,6 +96,8 @@ template <int D>
 __global__ void __launch_bounds__(256) absorb_kernel(AbsorbParams p) {
   const int h = blockIdx.x;
   const int tid = threadIdx.x;
+  griddep_wait();
+  griddep_launch_dependents();
   if (h == 0 && blockIdx.y == 0) {
     __shared__ int32_t part[256];
     __shared__ int32_t bad;
@@ -229,6 +232,8 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
     fence_mbar_init();
   }
   __syncthreads();
+  griddep_wait();
+  griddep_launch_dependents();
 
   Partition pt;
   pt.P = p.prefix[p.B];
@@ -362,29 +367,6 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
   }
 }
 
-// ====================================================================== reduce
-struct ReduceParams {
-  const float* mpart;     // [k_slots][H]
-  const int32_t* prefix;  // [B+1]
-  float* mx;              // [B][H]: max of the base-2 logits of each sequence and head
-  int B, H, k_grid;
-};
-
-__global__ void __launch_bounds__(256) reduce_kernel(ReduceParams p) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= p.B * p.H) return;
-  const int b = idx / p.H, h = idx % p.H;
-  const int32_t f0 = p.prefix[b], f1 = p.prefix[b + 1];
-  if (f1 == f0) { p.mx[idx] = 0.f; return; }
-  Partition pt;
-  pt.P = p.prefix[p.B];
-  pt.G = static_cast<int32_t>(pt.P < p.k_grid ? pt.P : p.k_grid);
-  const int32_t i0 = part_owner(f0, pt), i1 = part_owner(f1 - 1, pt);
-  float M = -INFINITY;
-  for (int32_t i = i0; i <= i1; ++i) M = fmaxf(M, p.mpart[static_cast<size_t>(b + i) * p.H + h]);
-  p.mx[idx] = M;
-}
-
 // ======================================================================= vpass
 // Z^T (R-range rows x heads) += C_V^T (R-range x 16 tokens) . P^T (16 x heads)
 // per page, with A = the V page slice as an MN-major 128B-swizzled operand
@@ -397,11 +379,12 @@ struct VPassParams {
   const int32_t* teff;
   const int32_t* prefix;
   const float* logits;    // [B][t_pad][H]
-  const float* mx;        // [B][H]
+  const float* mpart;     // [k_slots][H]: K-pass per-segment max of the logits
   float* zpart;           // [n_rr][v_slots][H][r_range]: sum_t w c_V per segment
   float* lpart;           // [v_slots][H]: sum_t w per segment (written by R range 0)
   int32_t* status;
   int B, H, npad, MB, NB, R, t_pad, r_range, n_rr, v_slots, stages;
+  int k_grid;             // CTAs of the K pass (its partition gives the segments to reduce)
   int n_chunks;           // 64-wide chunks per R range (r_range_pad/64); the last range may hold fewer
   int n_mtiles;           // r_range_pad / 128
   uint32_t tmem_cols;
@@ -434,9 +417,14 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
   __shared__ volatile int32_t abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  griddep_wait();
+  griddep_launch_dependents();
   Partition pt;
   pt.P = p.prefix[p.B];
   pt.G = static_cast<int32_t>(pt.P < gridDim.x ? pt.P : gridDim.x);
+  Partition ptk;            // the K pass's partition of the same pages
+  ptk.P = pt.P;
+  ptk.G = static_cast<int32_t>(pt.P < p.k_grid ? pt.P : p.k_grid);
   const int cta = blockIdx.x;
   const int rr = blockIdx.y;
   if (cta >= pt.G) return;  // uniform across the CTA: nothing allocated yet
@@ -562,8 +550,17 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
       if (mt.b < 0) { mbar_arrive(&pready[s]); break; }
       if (mt.flags & kFirst) {
         named_bar_sync(2, 128);  // everyone is done with the previous segment's max
-        for (int h = et; h < p.npad; h += 128)
-          sM[h] = h < p.H ? p.mx[static_cast<size_t>(mt.b) * p.H + h] : 0.f;
+        // max of the sequence's logits: the split reduction over its K-pass segments
+        const int32_t f0 = p.prefix[mt.b], f1 = p.prefix[mt.b + 1];
+        const int32_t i0 = part_owner(f0, ptk), i1 = part_owner(f1 - 1, ptk);
+        for (int h = et; h < p.npad; h += 128) {
+          float M = 0.f;
+          if (h < p.H) {
+            M = -INFINITY;
+            for (int32_t i = i0; i <= i1; ++i) M = fmaxf(M, p.mpart[static_cast<size_t>(mt.b + i) * p.H + h]);
+          }
+          sM[h] = M;
+        }
         named_bar_sync(2, 128);
         lsum = 0.f;
       }
@@ -659,6 +656,7 @@ struct ZFinalParams {
 
 // grid (ceil(R/1024), B*H), 256 threads x 4 consecutive rows of R
 __global__ void __launch_bounds__(256) zfinal_kernel(ZFinalParams p) {
+  griddep_wait();
   const int bh = blockIdx.y;
   const int b = bh / p.H, h = bh % p.H;
   const int j = (blockIdx.x * 256 + threadIdx.x) * 4;
@@ -671,15 +669,23 @@ __global__ void __launch_bounds__(256) zfinal_kernel(ZFinalParams p) {
     pt.P = p.prefix[p.B];
     pt.G = static_cast<int32_t>(pt.P < p.v_grid ? pt.P : p.v_grid);
     const int32_t i0 = part_owner(f0, pt), i1 = part_owner(f1 - 1, pt);
-    float Ls = 0.f;
-    for (int32_t i = i0; i <= i1; ++i) Ls += p.lpart[static_cast<size_t>(b + i) * p.H + h];
     const int rrg = j / p.r_range, jj = j % p.r_range;
     const size_t stride = static_cast<size_t>(p.H) * p.r_range;
     const float* src = p.zpart + ((static_cast<size_t>(rrg) * p.v_slots + b + i0) * p.H + h) * p.r_range + jj;
-    for (int32_t i = i0; i <= i1; ++i, src += stride) {
-      const float4 v = *reinterpret_cast<const float4*>(src);
-      z.x += v.x; z.y += v.y; z.z += v.z; z.w += v.w;
+    // issue up to four segment loads before summing them in segment order
+    for (int32_t i = i0; i <= i1; i += 4) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        v[u] = i + u <= i1 ? *reinterpret_cast<const float4*>(src + static_cast<size_t>(i - i0 + u) * stride)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (i + u <= i1) { z.x += v[u].x; z.y += v[u].y; z.z += v[u].z; z.w += v[u].w; }
+      }
     }
+    float Ls = 0.f;
+    for (int32_t i = i0; i <= i1; ++i) Ls += p.lpart[static_cast<size_t>(b + i) * p.H + h];
     const float il = 1.f / Ls;
     z.x *= il; z.y *= il; z.z *= il; z.w *= il;
   }
@@ -756,6 +762,8 @@ upproj_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
   tc_fence_after();
   const uint32_t taddr = taddr_s;
   bool ok = true;
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&bvmap);

@@ -121,6 +121,19 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ------------------------------------------------ programmatic dependent launch
+// A grid launched with programmatic stream serialisation may start before the
+// previous grid in the stream has finished.  griddep_wait() blocks until that
+// grid has completed and its memory is visible; every kernel here calls it
+// before touching memory a previous kernel may write or read.  (Both are no-ops
+// for a normal launch.)
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next grid in the stream begin launching (it still waits for this
+// grid's completion in its own griddep_wait()).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_dst, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(

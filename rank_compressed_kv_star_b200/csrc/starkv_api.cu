@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/starkv.h"
 #include "append_kernels.cuh"
@@ -185,7 +186,6 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   w.k_ctas = p.k_ctas;
   w.k_slots = p.k_ctas + batch;
   w.mpart_off = off; off = align_up(off + static_cast<size_t>(w.k_slots) * p.H * 4, 256);
-  w.mx_off = off; off = align_up(off + static_cast<size_t>(batch) * p.H * 4, 256);
   w.v_ctas = p.v_ctas;
   w.v_slots = p.v_ctas + batch;
   w.lpart_off = off; off = align_up(off + static_cast<size_t>(w.v_slots) * p.H * 4, 256);
@@ -248,34 +248,60 @@ bool encode_vpool_map(CUtensorMap* map, const void* v_cache, int R, int NB) {
 }
 
 // ------------------------------------------------------ kernel attributes
+// Raises a kernel's dynamic shared-memory limit once per device (and again only
+// when a larger size is needed).
 template <typename K>
 bool set_smem(K kernel, size_t bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) ==
-         cudaSuccess;
+  static std::mutex mu;
+  static int set_bytes[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) { cudaGetLastError(); return false; }
+  std::lock_guard<std::mutex> lock(mu);
+  if (set_bytes[dev] >= static_cast<int>(bytes)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  set_bytes[dev] = static_cast<int>(bytes);
+  return true;
 }
 
-template <int L, int CPL>
-cudaError_t launch_kpass(const DecodePlan& pl, const KPassParams& kp, cudaStream_t s) {
-  if (!set_smem(kpass_kernel<L, CPL>, pl.k_smem)) return cudaGetLastError();
-  kpass_kernel<L, CPL><<<pl.k_ctas, kKThreads, pl.k_smem, s>>>(kp);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_cluster(const void* kernel_fn, dim3 grid, dim3 block, size_t smem, int cluster_y, cudaStream_t s,
-                           void** args) {
+// Every kernel is launched with programmatic stream serialisation: the grid may
+// start while the previous grid in the stream drains, and waits for it inside
+// (griddep_wait) before touching memory.  cluster_y > 1 adds a (1, cluster_y, 1)
+// thread-block cluster.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster_y,
+                   Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = cluster_y;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_y > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = 1;
+    attr[n].val.clusterDim.y = static_cast<unsigned>(cluster_y);
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelExC(&cfg, kernel_fn, args);
+  cfg.numAttrs = n;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) cudaGetLastError();
+  return e;
+}
+
+template <int L, int CPT>
+cudaError_t launch_kpass(const DecodePlan& pl, const KPassParams& kp, cudaStream_t s) {
+  if (!set_smem(kpass_kernel<L, CPT>, pl.k_smem)) return cudaErrorInvalidValue;
+  return launch(kpass_kernel<L, CPT>, dim3(pl.k_ctas), dim3(kKThreads), pl.k_smem, s, 1, kp);
 }
 
 }  // namespace
@@ -350,22 +376,8 @@ starkv_status starkv_compress_append(const starkv_layer_desc* desc, int32_t batc
   const size_t stage_bytes = 2u * kAppKC * 128u + static_cast<size_t>(npad) * 128u;
   const size_t smem = 1024 + vp.stages * stage_bytes + (2 * vp.stages + 1) * sizeof(uint64_t);
   if (!set_smem(append_v_kernel, smem)) return STARKV_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_mt, KS, n_bt);
-  cfg.blockDim = dim3(kAppThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = KS;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, append_v_kernel, amap, vmap, vp) != cudaSuccess) {
-    cudaGetLastError();
+  if (launch(append_v_kernel, dim3(n_mt, KS, n_bt), dim3(kAppThreads), smem, s, KS, amap, vmap, vp) != cudaSuccess)
     return STARKV_ERR_CUDA;
-  }
 
   // ---- head-wise K codes
   AppendKParams kp;
@@ -377,8 +389,8 @@ starkv_status starkv_compress_append(const starkv_layer_desc* desc, int32_t batc
   kp.B = batch;
   const size_t ksm = (static_cast<size_t>(d) * r + static_cast<size_t>(kAppKB) * d) * 2;
   if (!set_smem(append_k_kernel, ksm)) return STARKV_ERR_CUDA;
-  append_k_kernel<<<dim3(H, (batch + kAppKB - 1) / kAppKB), 256, ksm, s>>>(kp);
-  if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
+  if (launch(append_k_kernel, dim3(H, (batch + kAppKB - 1) / kAppKB), dim3(256), ksm, s, 1, kp) != cudaSuccess)
+    return STARKV_ERR_CUDA;
   return STARKV_OK;
 }
 
@@ -424,7 +436,6 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   float* qt = reinterpret_cast<float*>(ws + pl.ws.qt_off);
   float* logits = reinterpret_cast<float*>(ws + pl.ws.logits_off);
   float* mpart = reinterpret_cast<float*>(ws + pl.ws.mpart_off);
-  float* mx = reinterpret_cast<float*>(ws + pl.ws.mx_off);
   float* lpart = reinterpret_cast<float*>(ws + pl.ws.lpart_off);
   float* zpart = reinterpret_cast<float*>(ws + pl.ws.zpart_off);
 
@@ -459,12 +470,13 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   ap.coef = scale * kLog2e;
   {
     const dim3 grid(pl.H, (batch + kAbsBT - 1) / kAbsBT);
-    if (pl.d == 32) absorb_kernel<32><<<grid, 256, 0, s>>>(ap);
-    else if (pl.d == 64) absorb_kernel<64><<<grid, 256, 0, s>>>(ap);
-    else if (pl.d == 128) absorb_kernel<128><<<grid, 256, 0, s>>>(ap);
-    else absorb_kernel<256><<<grid, 256, 0, s>>>(ap);
+    cudaError_t ea;
+    if (pl.d == 32) ea = launch(absorb_kernel<32>, grid, dim3(256), 0, s, 1, ap);
+    else if (pl.d == 64) ea = launch(absorb_kernel<64>, grid, dim3(256), 0, s, 1, ap);
+    else if (pl.d == 128) ea = launch(absorb_kernel<128>, grid, dim3(256), 0, s, 1, ap);
+    else ea = launch(absorb_kernel<256>, grid, dim3(256), 0, s, 1, ap);
+    if (ea != cudaSuccess) return STARKV_ERR_CUDA;
   }
-  if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
   mark(1);
 
   KPassParams kp;
@@ -482,32 +494,26 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   if (e != cudaSuccess) return STARKV_ERR_CUDA;
   mark(2);
 
-  ReduceParams rp;
-  rp.mpart = mpart; rp.prefix = prefix; rp.mx = mx;
-  rp.B = batch; rp.H = pl.H; rp.k_grid = pl.k_ctas;
-  reduce_kernel<<<(batch * pl.H + 255) / 256, 256, 0, s>>>(rp);
-  if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
-  mark(3);
-
   VPassParams vp;
-  vp.tables = block_tables; vp.teff = teff; vp.prefix = prefix; vp.logits = logits; vp.mx = mx;
+  vp.tables = block_tables; vp.teff = teff; vp.prefix = prefix; vp.logits = logits; vp.mpart = mpart;
   vp.zpart = zpart; vp.lpart = lpart; vp.status = status;
   vp.B = batch; vp.H = pl.H; vp.npad = pl.npad; vp.MB = pl.MB; vp.NB = pl.NB; vp.R = pl.R;
   vp.t_pad = pl.t_pad; vp.r_range = pl.r_range; vp.n_rr = pl.n_rr; vp.v_slots = pl.ws.v_slots;
+  vp.k_grid = pl.k_ctas;
   vp.stages = pl.v_stages; vp.n_chunks = pl.n_chunks; vp.n_mtiles = pl.n_mtiles; vp.tmem_cols = pl.tmem_cols;
   vp.vtile_bytes = pl.vtile; vp.ltile_bytes = pl.ltile; vp.ptile_bytes = pl.ptile;
   if (!set_smem(vpass_kernel, pl.v_smem)) return STARKV_ERR_CUDA;
-  vpass_kernel<<<dim3(pl.v_ctas, pl.n_rr), kVThreads, pl.v_smem, s>>>(vmap, vp);
-  if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
-  mark(4);
+  if (launch(vpass_kernel, dim3(pl.v_ctas, pl.n_rr), dim3(kVThreads), pl.v_smem, s, 1, vmap, vp) != cudaSuccess)
+    return STARKV_ERR_CUDA;
+  mark(3);
 
   ZFinalParams zf;
   zf.zpart = zpart; zf.lpart = lpart; zf.prefix = prefix; zf.zhi = zhi; zf.zlo = zlo;
   zf.B = batch; zf.H = pl.H; zf.R = pl.R; zf.r_range = pl.r_range; zf.v_slots = pl.ws.v_slots;
   zf.v_grid = pl.v_ctas;
-  zfinal_kernel<<<dim3((pl.R + 1023) / 1024, batch * pl.H), 256, 0, s>>>(zf);
-  if (cudaGetLastError() != cudaSuccess) return STARKV_ERR_CUDA;
-  mark(5);
+  if (launch(zfinal_kernel, dim3((pl.R + 1023) / 1024, batch * pl.H), dim3(256), 0, s, 1, zf) != cudaSuccess)
+    return STARKV_ERR_CUDA;
+  mark(4);
 
   UpProjParams up;
   up.out = static_cast<__half*>(out);
@@ -515,15 +521,10 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   up.n_mt = pl.up_mt; up.k_per_cta = pl.up_kpc; up.npad = pl.up_npad;
   up.stages = pl.up_stages; up.tmem_cols = pl.up_tmem;
   if (!set_smem(upproj_kernel, pl.up_smem)) return STARKV_ERR_CUDA;
-  {
-    void* args[] = {&bvmap, &zhimap, &zlomap, &up};
-    if (launch_cluster(reinterpret_cast<const void*>(upproj_kernel), dim3(pl.H * pl.up_mt * pl.up_bt, pl.up_ks),
-                       dim3(kUpThreads), pl.up_smem, pl.up_ks, s, args) != cudaSuccess) {
-      cudaGetLastError();
-      return STARKV_ERR_CUDA;
-    }
-  }
-  mark(6);
+  if (launch(upproj_kernel, dim3(pl.H * pl.up_mt * pl.up_bt, pl.up_ks), dim3(kUpThreads), pl.up_smem, s, pl.up_ks,
+             bvmap, zhimap, zlomap, up) != cudaSuccess)
+    return STARKV_ERR_CUDA;
+  mark(5);
   return STARKV_OK;
 }
 }  // namespace

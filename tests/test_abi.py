@@ -111,8 +111,8 @@ def test_workspace_layout_is_consistent(lib):
     d = _desc(max_blocks_per_seq=600, num_blocks=40000)
     lay = S.starkv_decode_workspace_layout(d, 64, 8192)
     assert lay.total_bytes == S.starkv_decode_workspace_bytes(d, 64, 8192)
-    offs = [lay.status_off, lay.prefix_off, lay.qt_off, lay.logits_off, lay.mpart_off, lay.mx_off,
-            lay.lpart_off, lay.zpart_off]
+    offs = [lay.status_off, lay.prefix_off, lay.qt_off, lay.logits_off, lay.mpart_off,
+            lay.lpart_off, lay.zpart_off, lay.zhi_off, lay.zlo_off]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     assert lay.t_pad == 8192 and lay.k_slots == lay.k_ctas + 64 and lay.v_slots == lay.v_ctas + 64
     assert lay.n_rranges * lay.r_range >= 2048

@@ -122,7 +122,7 @@ def test_decode_tiny_workload():
 
 
 def test_decode_tiny_intermediates():
-    """Logits, per-sequence max and softmax normaliser against the oracle's stages."""
+    """Logits, per-segment maxima and softmax normaliser against the oracle's stages."""
     wl = W.workload(1)
     Lh = W.host_layer(wl, 0)
     Ld = D.device_layer(wl, 0, tables=Lh["tables"], nb=Lh["nb"])
@@ -132,11 +132,12 @@ def test_decode_tiny_intermediates():
     H = Lh["H"]
     f32 = lambda off, n: wsn[off:off + 4 * n].view(np.float32)
     logits = f32(lay.logits_off, wl.batch * lay.t_pad * H).reshape(wl.batch, lay.t_pad, H)
-    mx = f32(lay.mx_off, wl.batch * H).reshape(wl.batch, H)
+    mpart = f32(lay.mpart_off, lay.k_slots * H).reshape(lay.k_slots, H)
     lpart = f32(lay.lpart_off, lay.v_slots * H).reshape(lay.v_slots, H)
     prefix = wsn[lay.prefix_off:lay.prefix_off + 4 * (wl.batch + 1)].view(np.int32)
-    P, G = int(prefix[-1]), min(lay.v_ctas, int(prefix[-1]))
-    owner = lambda x: min(G - 1, ((x + 1) * G + P - 1) // P - 1)
+    P = int(prefix[-1])
+    Gv, Gk = min(lay.v_ctas, P), min(lay.k_ctas, P)
+    owner = lambda x, G: min(G - 1, ((x + 1) * G + P - 1) // P - 1)
     for b in range(wl.batch):
         T = int(Lh["seq_lens"][b])
         st = O.decode_stages(Lh["q"][b], Lh["B_K"], Lh["B_V"], O.gather(Lh["k_cache"], Lh["tables"][b], T),
@@ -144,9 +145,10 @@ def test_decode_tiny_intermediates():
         s2 = st["s"] * np.log2(np.e)             # base-2 logits [H][T]
         np.testing.assert_allclose(logits[b, :T].T, s2, rtol=0, atol=1e-4)
         M = s2.max(axis=1)
-        np.testing.assert_allclose(mx[b], M, rtol=0, atol=1e-4)
+        ksegs = range(owner(int(prefix[b]), Gk), owner(int(prefix[b + 1]) - 1, Gk) + 1)
+        np.testing.assert_allclose(np.max([mpart[b + i] for i in ksegs], axis=0), M, rtol=0, atol=1e-4)
         Lsum = np.exp2(s2 - M[:, None]).sum(axis=1)
-        segs = range(owner(int(prefix[b])), owner(int(prefix[b + 1]) - 1) + 1)
+        segs = range(owner(int(prefix[b]), Gv), owner(int(prefix[b + 1]) - 1, Gv) + 1)
         Lgpu = sum(lpart[b + i] for i in segs)
         np.testing.assert_allclose(Lgpu, Lsum, rtol=2e-3)
 
