@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <utility>
 
@@ -248,22 +249,24 @@ bool encode_vpool_map(CUtensorMap* map, const void* v_cache, int R, int NB) {
 }
 
 // ------------------------------------------------------ kernel attributes
-// Raises a kernel's dynamic shared-memory limit once per device (and again only
-// when a larger size is needed).
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device), and
+// again only when a larger size is needed.
 template <typename K>
 bool set_smem(K kernel, size_t bytes) {
   static std::mutex mu;
-  static int set_bytes[64] = {};
+  static std::map<std::pair<const void*, int>, int> set_bytes;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) { cudaGetLastError(); return false; }
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return false; }
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
   std::lock_guard<std::mutex> lock(mu);
-  if (set_bytes[dev] >= static_cast<int>(bytes)) return true;
+  auto it = set_bytes.find(key);
+  if (it != set_bytes.end() && it->second >= static_cast<int>(bytes)) return true;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
       cudaSuccess) {
     cudaGetLastError();
     return false;
   }
-  set_bytes[dev] = static_cast<int>(bytes);
+  set_bytes[key] = static_cast<int>(bytes);
   return true;
 }
 
