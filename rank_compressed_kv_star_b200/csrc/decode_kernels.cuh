@@ -297,6 +297,7 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
   float2 qv[CPT * 4];
   float m = -INFINITY;
   int cur_b = -1;
+  const uint64_t keep = policy_evict_last();   // logits: read back by the V pass
 
   for (uint32_t k = 0;; ++k) {
     const int s = k % S;
@@ -358,7 +359,7 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
       for (int o = L / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (valid) {
         if (sub == 0)
-          p.logits[(static_cast<size_t>(cur_b) * p.t_pad + mt.t0 + t) * p.H + head] = acc;
+          st_global_hint(p.logits + (static_cast<size_t>(cur_b) * p.t_pad + mt.t0 + t) * p.H + head, acc, keep);
         m = fmaxf(m, acc);
       }
     }
@@ -539,6 +540,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
     const int t_step = 128 / p.npad;
     float lsum = 0.f;
     uint32_t seg = 0;
+    const uint64_t keep = policy_evict_last();   // Z partials: read back by zfinal
     for (uint32_t k = 0;; ++k) {
       const int s = k % S;
       if (!mbar_wait(&full[s], (k / S) & 1) || abort_flag) {
@@ -612,7 +614,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
             if (j < p.r_range && rr * p.r_range + j < p.R) {
               const int hn = min(32, p.H - h0);
               for (int hh = 0; hh < hn; ++hh)
-                zb[static_cast<size_t>(h0 + hh) * p.r_range + j] = __uint_as_float(v[hh]);
+                st_global_hint(zb + static_cast<size_t>(h0 + hh) * p.r_range + j, __uint_as_float(v[hh]), keep);
             }
           }
         }
@@ -696,8 +698,9 @@ __global__ void __launch_bounds__(256) zfinal_kernel(ZFinalParams p) {
   uint2 hv, lv;
   hv.x = *reinterpret_cast<const uint32_t*>(&h01); hv.y = *reinterpret_cast<const uint32_t*>(&h23);
   lv.x = *reinterpret_cast<const uint32_t*>(&l01); lv.y = *reinterpret_cast<const uint32_t*>(&l23);
-  *reinterpret_cast<uint2*>(p.zhi + dst) = hv;
-  *reinterpret_cast<uint2*>(p.zlo + dst) = lv;
+  const uint64_t keep = policy_evict_last();   // read by the up-projection next
+  st_global_hint(reinterpret_cast<uint2*>(p.zhi + dst), hv, keep);
+  st_global_hint(reinterpret_cast<uint2*>(p.zlo + dst), lv, keep);
 }
 
 // ====================================================================== upproj

@@ -110,6 +110,16 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   return p;
 }
 
+// Global stores with an L2 eviction-priority hint (intermediates that the next
+// kernel reads once: keep them in L2 while the code streams pass through).
+__device__ __forceinline__ void st_global_hint(float* p, float v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(policy) : "memory");
+}
+__device__ __forceinline__ void st_global_hint(uint2* p, uint2 v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;" ::"l"(p), "r"(v.x), "r"(v.y), "l"(policy)
+               : "memory");
+}
+
 // Generic-proxy writes to shared memory become visible to the async proxy
 // (TMA engine, tensor cores) after this fence.
 __device__ __forceinline__ void fence_proxy_async_smem() {
