@@ -143,10 +143,10 @@ starkv_status starkv_paged_decode(const starkv_layer_desc* desc, int32_t batch, 
 /*
  * starkv_paged_decode_profiled -- starkv_paged_decode that also records CUDA
  * events on `stream` around its kernels, for per-kernel timing.
- * stage_events: HOST array of 5 cudaEvent_t (as void*; a NULL entry is
+ * stage_events: HOST array of 6 cudaEvent_t (as void*; a NULL entry is
  * skipped) recorded before the query absorption, after it, after the K pass,
- * after the V pass (which includes the split reduction and the Z
- * finalisation) and after the up-projection.  Events between the kernels keep
+ * after the V pass (which includes the split reduction), after the Z
+ * finalisation and after the up-projection.  Events between the kernels keep
  * them from overlapping their launches, so this variant can be slightly slower
  * than starkv_paged_decode.  The events are not recorded when the call returns
  * an error before launching or when max_seq_len == 0.  Otherwise identical to
@@ -204,8 +204,7 @@ typedef struct {
   size_t qt_off;      /* fp32 [batch][H][r]: log2(e)*scale*q.B_K^T */
   size_t logits_off;  /* fp32 [batch][t_pad][H]: base-2 logits s*log2(e) */
   size_t mpart_off;   /* fp32 [k_slots][H]: max of the base-2 logits per segment */
-  size_t lpart_off;   /* fp32 [n_rranges][v_slots][H]: per segment, sum of the fp16 weights exp2(s - max) */
-  size_t counters_off; /* int32 [n_rranges][batch]: V-pass segments completed */
+  size_t lpart_off;   /* fp32 [v_slots][H]: per segment, sum of the fp16 weights exp2(s - max) */
   size_t zpart_off;   /* fp32 [n_rranges][v_slots][H][r_range]: per segment, sum_t w c_V */
   size_t zhi_off;     /* fp16 [H][batch][R]: Z/L rounded to fp16 */
   size_t zlo_off;     /* fp16 [H][batch][R]: Z/L minus its fp16 rounding, in fp16 */

@@ -48,7 +48,7 @@ class WorkspaceLayout(ctypes.Structure):
     _fields_ = [("total_bytes", ctypes.c_size_t), ("status_off", ctypes.c_size_t),
                 ("prefix_off", ctypes.c_size_t), ("qt_off", ctypes.c_size_t),
                 ("logits_off", ctypes.c_size_t), ("mpart_off", ctypes.c_size_t),
-                ("lpart_off", ctypes.c_size_t), ("counters_off", ctypes.c_size_t),
+                ("lpart_off", ctypes.c_size_t),
                 ("zpart_off", ctypes.c_size_t), ("zhi_off", ctypes.c_size_t),
                 ("zlo_off", ctypes.c_size_t),
                 ("t_pad", ctypes.c_int32), ("k_ctas", ctypes.c_int32), ("k_slots", ctypes.c_int32),
@@ -166,10 +166,10 @@ def starkv_paged_decode_profiled(desc: LayerDesc, batch: int, max_seq_len: int, 
                                  k_cache, v_cache, block_tables, seq_lens, scale: float, workspace,
                                  workspace_bytes: int, out, stage_events, stream=None,
                                  check: bool = True) -> int:
-    """``stage_events``: five ``torch.cuda.Event`` (or raw cudaEvent_t ints / None)."""
+    """``stage_events``: six ``torch.cuda.Event`` (or raw cudaEvent_t ints / None)."""
     raw = [None if e is None else (e if isinstance(e, int) else e.cuda_event) for e in stage_events]
-    assert len(raw) == 5
-    arr = (ctypes.c_void_p * 5)(*raw)
+    assert len(raw) == 6
+    arr = (ctypes.c_void_p * 6)(*raw)
     st = load_library().starkv_paged_decode_profiled(
         _desc_ref(desc), batch, max_seq_len, _ptr(q), _ptr(B_K), _ptr(B_V), _ptr(k_cache),
         _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), float(scale), _ptr(workspace),

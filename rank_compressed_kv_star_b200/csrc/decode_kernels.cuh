@@ -1,14 +1,14 @@
 // Decode kernels of the STAR-KV paged low-rank cache (sm_100a).
 //
-// One decode is four launches on the caller's stream, each launched with
+// One decode is five launches on the caller's stream, each launched with
 // programmatic stream serialisation (see griddep_wait):
 //   1. absorb      q~ = log2(e)*scale * q . B_K[h]^T; page prefix sums; status reset
 //   2. kpass       base-2 logits s = q~ . c_K over the K pages, per-segment max
 //   3. vpass       split reduction M = max over the sequence's K segments, then
-//                  Z = sum_t w c_V on tcgen05 tensor cores with w = fp16(exp2(s - M))
-//                  and the normaliser L = sum_t w; the CTA finishing a sequence's
-//                  last segment sums the partials and writes Z / L as fp16 hi + lo
-//   4. upproj      out_h = (Z_h / L) . B_V[:, h*d:(h+1)*d] on tcgen05 -> fp16
+//                  Z = sum_t w c_V on tcgen05 tensor cores with w = fp16(exp2(s - M)),
+//                  and the normaliser L = sum_t w
+//   4. zfinal      Z / L summed over segments, split into fp16 hi + lo
+//   5. upproj      out_h = (Z_h / L) . B_V[:, h*d:(h+1)*d] on tcgen05 -> fp16
 //
 // The formulation (head-wise K with the query absorbed, joint V applied after
 // the weighted sum of codes) follows the STAR-KV description in the Proxima
@@ -80,8 +80,6 @@ struct AbsorbParams {
   float* qt;              // [B][H][r]
   int32_t* prefix;        // [B+1]
   int32_t* teff;          // [B] clamped lengths
-  int32_t* counters;      // [n_counters]: V-pass segment counters, reset here
-  int n_counters;
   int32_t* status;
   int B, H, d, r, cap;    // cap = min(max_seq_len, max_blocks_per_seq*16)
   float coef;             // scale * log2(e)
@@ -128,7 +126,6 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbParams p) {
       p.prefix[b] = acc;
       acc += (p.teff[b] + kBlock - 1) / kBlock;
     }
-    for (int i = tid; i < p.n_counters; i += 256) p.counters[i] = 0;
   }
   __shared__ __align__(16) __half qs[kAbsBT * D];
   const int bt0 = blockIdx.y * kAbsBT;
@@ -385,10 +382,7 @@ struct VPassParams {
   const float* logits;    // [B][t_pad][H]
   const float* mpart;     // [k_slots][H]: K-pass per-segment max of the logits
   float* zpart;           // [n_rr][v_slots][H][r_range]: sum_t w c_V per segment
-  float* lpart;           // [n_rr][v_slots][H]: sum_t w per segment
-  int32_t* counters;      // [n_rr][B]: segments of (sequence, R range) written so far
-  __half* zhi;            // [H][B][R]: Z / L rounded to fp16
-  __half* zlo;            // [H][B][R]: Z / L minus zhi, in fp16
+  float* lpart;           // [v_slots][H]: sum_t w per segment (written by R range 0)
   int32_t* status;
   int B, H, npad, MB, NB, R, t_pad, r_range, n_rr, v_slots, stages;
   int k_grid;             // CTAs of the K pass (its partition gives the segments to reduce)
@@ -420,8 +414,6 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
   uint64_t* mdone = tfree + 1;
   float* sM = reinterpret_cast<float*>(mdone + 1);                      // [npad]
   float* sRed = sM + p.npad;                                            // [128]
-  float* sInvL = sRed + 128;                                            // [npad]
-  __shared__ int32_t s_last;
   __shared__ uint32_t taddr_s;
   __shared__ volatile int32_t abort_flag;
 
@@ -631,59 +623,12 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
         // per-segment normaliser of every head
         sRed[et] = lsum;
         named_bar_sync(2, 128);
-        if (et < p.H) {
+        if (rr == 0 && et < p.H) {
           float Ls = 0.f;
           for (int i = et; i < 128; i += p.npad) Ls += sRed[i];
-          p.lpart[(static_cast<size_t>(rr) * p.v_slots + slot) * p.H + et] = Ls;
+          p.lpart[slot * p.H + et] = Ls;
         }
         named_bar_sync(2, 128);
-        // the CTA that writes the last segment of (sequence, R range) finishes it:
-        // partials summed in segment order, times 1/L, split into fp16 hi + lo
-        const int32_t f0 = p.prefix[mt.b], f1 = p.prefix[mt.b + 1];
-        const int32_t i0 = part_owner(f0, pt), i1 = part_owner(f1 - 1, pt);
-        __threadfence();            // this thread's partial stores before the count
-        named_bar_sync(2, 128);
-        if (et == 0) {
-          const int32_t done_before = atomicAdd(&p.counters[rr * p.B + mt.b], 1);
-          s_last = done_before == i1 - i0;
-          if (s_last) __threadfence();
-        }
-        named_bar_sync(2, 128);
-        if (s_last) {
-          if (et < p.H) {
-            float Ls = 0.f;
-            for (int32_t i = i0; i <= i1; ++i)
-              Ls += __ldcg(p.lpart + (static_cast<size_t>(rr) * p.v_slots + mt.b + i) * p.H + et);
-            sInvL[et] = 1.f / Ls;
-          }
-          named_bar_sync(2, 128);
-          const int rq = p.r_range / 4;
-          const size_t seg_stride = static_cast<size_t>(p.H) * p.r_range;
-          const float* zbase = p.zpart + (static_cast<size_t>(rr) * p.v_slots + mt.b + i0) * seg_stride;
-          for (int x = et; x < p.H * rq; x += 128) {
-            const int h = x / rq, j = (x % rq) * 4;
-            if (rr * p.r_range + j >= p.R) continue;
-            const float4* src = reinterpret_cast<const float4*>(zbase + static_cast<size_t>(h) * p.r_range + j);
-            float4 z = __ldcg(src);
-            for (int32_t i = 1; i <= i1 - i0; ++i) {
-              const float4 v = __ldcg(src + static_cast<size_t>(i) * (seg_stride / 4));
-              z.x += v.x; z.y += v.y; z.z += v.z; z.w += v.w;
-            }
-            const float il = sInvL[h];
-            z.x *= il; z.y *= il; z.z *= il; z.w *= il;
-            const __half2 h01 = __floats2half2_rn(z.x, z.y), h23 = __floats2half2_rn(z.z, z.w);
-            const float2 g01 = __half22float2(h01), g23 = __half22float2(h23);
-            const __half2 l01 = __floats2half2_rn(z.x - g01.x, z.y - g01.y);
-            const __half2 l23 = __floats2half2_rn(z.z - g23.x, z.w - g23.y);
-            uint2 hv, lv;
-            hv.x = *reinterpret_cast<const uint32_t*>(&h01); hv.y = *reinterpret_cast<const uint32_t*>(&h23);
-            lv.x = *reinterpret_cast<const uint32_t*>(&l01); lv.y = *reinterpret_cast<const uint32_t*>(&l23);
-            const size_t dst = (static_cast<size_t>(h) * p.B + mt.b) * p.R + rr * p.r_range + j;
-            st_global_hint(reinterpret_cast<uint2*>(p.zhi + dst), hv, keep);
-            st_global_hint(reinterpret_cast<uint2*>(p.zlo + dst), lv, keep);
-          }
-          named_bar_sync(2, 128);
-        }
         ++seg;
       }
     }
@@ -695,6 +640,69 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
   }
 }
 
+// ==================================================================== zfinal
+// Z / L per (sequence, head): the V-pass partials of the sequence's segments
+// summed in segment order, scaled by 1/L (L = the summed fp16 weights), and
+// split into fp16 hi + lo halves for the up-projection's B operand (hi + lo
+// keeps about 22 bits of the fp32 value).  Z / L is a convex combination of
+// fp16 codes, so both halves are in range.  Layout [H][B][R] (head-major) so
+// that one head's rows of a batch tile are contiguous.
+struct ZFinalParams {
+  const float* zpart;     // [n_rr][v_slots][H][r_range]
+  const float* lpart;     // [v_slots][H]
+  const int32_t* prefix;
+  __half* zhi;            // [H][B][R]
+  __half* zlo;            // [H][B][R]
+  int B, H, R, r_range, v_slots, v_grid;
+};
+
+// grid (ceil(R/1024), B*H), 256 threads x 4 consecutive rows of R
+__global__ void __launch_bounds__(256) zfinal_kernel(ZFinalParams p) {
+  griddep_wait();
+  const int bh = blockIdx.y;
+  const int b = bh / p.H, h = bh % p.H;
+  const int j = (blockIdx.x * 256 + threadIdx.x) * 4;
+  if (j >= p.R) return;
+  const size_t dst = (static_cast<size_t>(h) * p.B + b) * p.R + j;
+  float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int32_t f0 = p.prefix[b], f1 = p.prefix[b + 1];
+  if (f1 > f0) {
+    Partition pt;
+    pt.P = p.prefix[p.B];
+    pt.G = static_cast<int32_t>(pt.P < p.v_grid ? pt.P : p.v_grid);
+    const int32_t i0 = part_owner(f0, pt), i1 = part_owner(f1 - 1, pt);
+    const int rrg = j / p.r_range, jj = j % p.r_range;
+    const size_t stride = static_cast<size_t>(p.H) * p.r_range;
+    const float* src = p.zpart + ((static_cast<size_t>(rrg) * p.v_slots + b + i0) * p.H + h) * p.r_range + jj;
+    // issue up to four segment loads before summing them in segment order
+    for (int32_t i = i0; i <= i1; i += 4) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        v[u] = i + u <= i1 ? *reinterpret_cast<const float4*>(src + static_cast<size_t>(i - i0 + u) * stride)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (i + u <= i1) { z.x += v[u].x; z.y += v[u].y; z.z += v[u].z; z.w += v[u].w; }
+      }
+    }
+    float Ls = 0.f;
+    for (int32_t i = i0; i <= i1; ++i) Ls += p.lpart[static_cast<size_t>(b + i) * p.H + h];
+    const float il = 1.f / Ls;
+    z.x *= il; z.y *= il; z.z *= il; z.w *= il;
+  }
+  const __half2 h01 = __floats2half2_rn(z.x, z.y), h23 = __floats2half2_rn(z.z, z.w);
+  const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+  const __half2 l01 = __floats2half2_rn(z.x - f01.x, z.y - f01.y);
+  const __half2 l23 = __floats2half2_rn(z.z - f23.x, z.w - f23.y);
+  uint2 hv, lv;
+  hv.x = *reinterpret_cast<const uint32_t*>(&h01); hv.y = *reinterpret_cast<const uint32_t*>(&h23);
+  lv.x = *reinterpret_cast<const uint32_t*>(&l01); lv.y = *reinterpret_cast<const uint32_t*>(&l23);
+  const uint64_t keep = policy_evict_last();   // read by the up-projection next
+  st_global_hint(reinterpret_cast<uint2*>(p.zhi + dst), hv, keep);
+  st_global_hint(reinterpret_cast<uint2*>(p.zlo + dst), lv, keep);
+}
+
 // ====================================================================== upproj
 // out_h^T (d x B) = B_V^h^T (d x R) . (Z_h / L)^T (R x B) on tcgen05 tensor
 // cores, two MMAs per K step (hi and lo halves of Z / L).  A = B_V^h^T from
@@ -702,7 +710,6 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
 // the head's Z rows (K-major, 128B swizzle).  R is split over a cluster whose
 // partial sums are added through distributed shared memory in rank order.
 struct UpProjParams {
-  const int32_t* prefix;  // [B+1]: empty sequences get zero rows
   __half* out;            // [B][H][d]
   int B, H, d, R;
   int n_mt;               // 128-row tiles of d
@@ -824,7 +831,6 @@ upproj_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
     if (b >= p.B || dm >= p.d) continue;
     float acc = 0.f;
     for (int c = 0; c < KS; ++c) acc += cluster.map_shared_rank(part, c)[n * 128 + m];
-    if (p.prefix[b + 1] == p.prefix[b]) acc = 0.f;   // no tokens: no Z was produced
     p.out[(static_cast<size_t>(b) * p.H + h) * p.d + dm] = __float2half_rn(acc);
   }
   cluster.sync();

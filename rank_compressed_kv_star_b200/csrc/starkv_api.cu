@@ -145,7 +145,7 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   if (p.v_stages > 8) p.v_stages = 8;
   if (p.v_stages < 2) p.v_stages = 2;
   p.v_smem = 1024 + static_cast<size_t>(p.v_stages) * stage + p.v_stages * sizeof(StageMeta) +
-             (3 * p.v_stages + 3) * sizeof(uint64_t) + (2 * p.npad + 128) * sizeof(float);
+             (3 * p.v_stages + 3) * sizeof(uint64_t) + (p.npad + 128) * sizeof(float);
   int per_sm = static_cast<int>((227u * 1024u) / (p.v_smem + 1024));
   if (per_sm > static_cast<int>(512 / p.tmem_cols)) per_sm = 512 / p.tmem_cols;
   if (per_sm < 1) per_sm = 1;
@@ -189,8 +189,7 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   w.mpart_off = off; off = align_up(off + static_cast<size_t>(w.k_slots) * p.H * 4, 256);
   w.v_ctas = p.v_ctas;
   w.v_slots = p.v_ctas + batch;
-  w.lpart_off = off; off = align_up(off + static_cast<size_t>(p.n_rr) * w.v_slots * p.H * 4, 256);
-  w.counters_off = off; off = align_up(off + static_cast<size_t>(p.n_rr) * batch * 4, 256);
+  w.lpart_off = off; off = align_up(off + static_cast<size_t>(w.v_slots) * p.H * 4, 256);
   w.n_rranges = p.n_rr;
   w.r_range = p.r_range;
   w.zpart_off = off;
@@ -441,7 +440,6 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   float* logits = reinterpret_cast<float*>(ws + pl.ws.logits_off);
   float* mpart = reinterpret_cast<float*>(ws + pl.ws.mpart_off);
   float* lpart = reinterpret_cast<float*>(ws + pl.ws.lpart_off);
-  int32_t* counters = reinterpret_cast<int32_t*>(ws + pl.ws.counters_off);
   float* zpart = reinterpret_cast<float*>(ws + pl.ws.zpart_off);
 
   if (max_seq_len == 0) {
@@ -471,7 +469,6 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   ap.B_K = static_cast<const __half*>(B_K);
   ap.seq_lens = seq_lens;
   ap.qt = qt; ap.prefix = prefix; ap.teff = teff; ap.status = status;
-  ap.counters = counters; ap.n_counters = pl.n_rr * batch;
   ap.B = batch; ap.H = pl.H; ap.d = pl.d; ap.r = pl.r; ap.cap = pl.cap;
   ap.coef = scale * kLog2e;
   {
@@ -503,7 +500,6 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   VPassParams vp;
   vp.tables = block_tables; vp.teff = teff; vp.prefix = prefix; vp.logits = logits; vp.mpart = mpart;
   vp.zpart = zpart; vp.lpart = lpart; vp.status = status;
-  vp.counters = counters; vp.zhi = zhi; vp.zlo = zlo;
   vp.B = batch; vp.H = pl.H; vp.npad = pl.npad; vp.MB = pl.MB; vp.NB = pl.NB; vp.R = pl.R;
   vp.t_pad = pl.t_pad; vp.r_range = pl.r_range; vp.n_rr = pl.n_rr; vp.v_slots = pl.ws.v_slots;
   vp.k_grid = pl.k_ctas;
@@ -514,8 +510,15 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
     return STARKV_ERR_CUDA;
   mark(3);
 
+  ZFinalParams zf;
+  zf.zpart = zpart; zf.lpart = lpart; zf.prefix = prefix; zf.zhi = zhi; zf.zlo = zlo;
+  zf.B = batch; zf.H = pl.H; zf.R = pl.R; zf.r_range = pl.r_range; zf.v_slots = pl.ws.v_slots;
+  zf.v_grid = pl.v_ctas;
+  if (launch(zfinal_kernel, dim3((pl.R + 1023) / 1024, batch * pl.H), dim3(256), 0, s, 1, zf) != cudaSuccess)
+    return STARKV_ERR_CUDA;
+  mark(4);
+
   UpProjParams up;
-  up.prefix = prefix;
   up.out = static_cast<__half*>(out);
   up.B = batch; up.H = pl.H; up.d = pl.d; up.R = pl.R;
   up.n_mt = pl.up_mt; up.k_per_cta = pl.up_kpc; up.npad = pl.up_npad;
@@ -524,7 +527,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   if (launch(upproj_kernel, dim3(pl.H * pl.up_mt * pl.up_bt, pl.up_ks), dim3(kUpThreads), pl.up_smem, s, pl.up_ks,
              bvmap, zhimap, zlomap, up) != cudaSuccess)
     return STARKV_ERR_CUDA;
-  mark(4);
+  mark(5);
   return STARKV_OK;
 }
 }  // namespace
