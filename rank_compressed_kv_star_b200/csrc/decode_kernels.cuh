@@ -656,51 +656,79 @@ struct ZFinalParams {
   int B, H, R, r_range, v_slots, v_grid;
 };
 
-// grid (ceil(R/1024), B*H), 256 threads x 4 consecutive rows of R
+// grid (ceil(R/2048), B*H), 256 threads x 8 consecutive rows of R.  Thread 0
+// looks up the sequence's segments and 1/L once for the CTA.
 __global__ void __launch_bounds__(256) zfinal_kernel(ZFinalParams p) {
   griddep_wait();
+  __shared__ int32_t s_i0, s_i1;
+  __shared__ float s_il;
   const int bh = blockIdx.y;
   const int b = bh / p.H, h = bh % p.H;
-  const int j = (blockIdx.x * 256 + threadIdx.x) * 4;
+  if (threadIdx.x == 0) {
+    const int32_t f0 = p.prefix[b], f1 = p.prefix[b + 1];
+    int32_t i0 = 0, i1 = -1;
+    float il = 0.f;
+    if (f1 > f0) {
+      Partition pt;
+      pt.P = p.prefix[p.B];
+      pt.G = static_cast<int32_t>(pt.P < p.v_grid ? pt.P : p.v_grid);
+      i0 = part_owner(f0, pt);
+      i1 = part_owner(f1 - 1, pt);
+      float Ls = 0.f;
+      for (int32_t i = i0; i <= i1; ++i) Ls += p.lpart[static_cast<size_t>(b + i) * p.H + h];
+      il = 1.f / Ls;
+    }
+    s_i0 = i0;
+    s_i1 = i1;
+    s_il = il;
+  }
+  __syncthreads();
+  const int j = (blockIdx.x * 256 + threadIdx.x) * 8;
   if (j >= p.R) return;
-  const size_t dst = (static_cast<size_t>(h) * p.B + b) * p.R + j;
-  float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-  const int32_t f0 = p.prefix[b], f1 = p.prefix[b + 1];
-  if (f1 > f0) {
-    Partition pt;
-    pt.P = p.prefix[p.B];
-    pt.G = static_cast<int32_t>(pt.P < p.v_grid ? pt.P : p.v_grid);
-    const int32_t i0 = part_owner(f0, pt), i1 = part_owner(f1 - 1, pt);
+  const int32_t i0 = s_i0, i1 = s_i1;
+  float z[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) z[u] = 0.f;
+  if (i1 >= i0) {
     const int rrg = j / p.r_range, jj = j % p.r_range;
     const size_t stride = static_cast<size_t>(p.H) * p.r_range;
     const float* src = p.zpart + ((static_cast<size_t>(rrg) * p.v_slots + b + i0) * p.H + h) * p.r_range + jj;
-    // issue up to four segment loads before summing them in segment order
+    // all loads of up to four segments are issued before they are summed in segment order
     for (int32_t i = i0; i <= i1; i += 4) {
-      float4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        v[u] = i + u <= i1 ? *reinterpret_cast<const float4*>(src + static_cast<size_t>(i - i0 + u) * stride)
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 v[4][2];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        if (i + u <= i1) { z.x += v[u].x; z.y += v[u].y; z.z += v[u].z; z.w += v[u].w; }
+        const float4* q = reinterpret_cast<const float4*>(src + static_cast<size_t>(i - i0 + u) * stride);
+        const bool in = i + u <= i1;
+        v[u][0] = in ? q[0] : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[u][1] = in ? q[1] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (i + u <= i1) {
+          z[0] += v[u][0].x; z[1] += v[u][0].y; z[2] += v[u][0].z; z[3] += v[u][0].w;
+          z[4] += v[u][1].x; z[5] += v[u][1].y; z[6] += v[u][1].z; z[7] += v[u][1].w;
+        }
       }
     }
-    float Ls = 0.f;
-    for (int32_t i = i0; i <= i1; ++i) Ls += p.lpart[static_cast<size_t>(b + i) * p.H + h];
-    const float il = 1.f / Ls;
-    z.x *= il; z.y *= il; z.z *= il; z.w *= il;
+    const float il = s_il;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) z[u] *= il;
   }
-  const __half2 h01 = __floats2half2_rn(z.x, z.y), h23 = __floats2half2_rn(z.z, z.w);
-  const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
-  const __half2 l01 = __floats2half2_rn(z.x - f01.x, z.y - f01.y);
-  const __half2 l23 = __floats2half2_rn(z.z - f23.x, z.w - f23.y);
-  uint2 hv, lv;
-  hv.x = *reinterpret_cast<const uint32_t*>(&h01); hv.y = *reinterpret_cast<const uint32_t*>(&h23);
-  lv.x = *reinterpret_cast<const uint32_t*>(&l01); lv.y = *reinterpret_cast<const uint32_t*>(&l23);
-  const uint64_t keep = policy_evict_last();   // read by the up-projection next
-  st_global_hint(reinterpret_cast<uint2*>(p.zhi + dst), hv, keep);
-  st_global_hint(reinterpret_cast<uint2*>(p.zlo + dst), lv, keep);
+  uint4 hv, lv;
+  uint32_t* hw = reinterpret_cast<uint32_t*>(&hv);
+  uint32_t* lw = reinterpret_cast<uint32_t*>(&lv);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const __half2 hh = __floats2half2_rn(z[2 * u], z[2 * u + 1]);
+    const float2 g = __half22float2(hh);
+    const __half2 ll = __floats2half2_rn(z[2 * u] - g.x, z[2 * u + 1] - g.y);
+    hw[u] = *reinterpret_cast<const uint32_t*>(&hh);
+    lw[u] = *reinterpret_cast<const uint32_t*>(&ll);
+  }
+  const size_t dst = (static_cast<size_t>(h) * p.B + b) * p.R + j;
+  *reinterpret_cast<uint4*>(p.zhi + dst) = hv;
+  *reinterpret_cast<uint4*>(p.zlo + dst) = lv;
 }
 
 // ====================================================================== upproj

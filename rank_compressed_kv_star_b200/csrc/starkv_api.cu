@@ -514,7 +514,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   zf.zpart = zpart; zf.lpart = lpart; zf.prefix = prefix; zf.zhi = zhi; zf.zlo = zlo;
   zf.B = batch; zf.H = pl.H; zf.R = pl.R; zf.r_range = pl.r_range; zf.v_slots = pl.ws.v_slots;
   zf.v_grid = pl.v_ctas;
-  if (launch(zfinal_kernel, dim3((pl.R + 1023) / 1024, batch * pl.H), dim3(256), 0, s, 1, zf) != cudaSuccess)
+  if (launch(zfinal_kernel, dim3((pl.R + 2047) / 2048, batch * pl.H), dim3(256), 0, s, 1, zf) != cudaSuccess)
     return STARKV_ERR_CUDA;
   mark(4);
 
