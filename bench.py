@@ -61,6 +61,22 @@ def parse_args():
     return ap.parse_args()
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank float across the process group (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(world: int, batch_per_rank: int, ms_per_step_max: float) -> float:
+    """Replicas: every rank decodes its own batch; the job's rate uses the slowest rank's time."""
+    return world * batch_per_rank / (ms_per_step_max * 1e-3)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -242,10 +258,7 @@ def run_ours(args):
             per["append"] += app_evs[i][li][0].elapsed_time(app_evs[i][li][1])
     per = {n: v / Kp for n, v in per.items()}             # ms per step (all layers)
 
-    if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, device="cuda")
 
     # ---------------- algorithmic bytes
     T_sum = int(wl.seq_lens.sum())
@@ -283,18 +296,14 @@ def run_ours(args):
             host_out[li].copy_(outs[li], non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / Ke
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke, device="cuda")
     assert np.isfinite(host_out[0].float().numpy()).all()
 
     cpu = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
         cpu = cpu_baseline(wl, args.cpu_seconds)
 
-    value = world * B / (ms * 1e-3)
+    value = whole_job_tokens_per_s(world, B, ms)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
@@ -315,7 +324,7 @@ def run_ours(args):
         "kernels_ms_per_step": {n: round(v, 5) for n, v in per.items()},
         "kernels_timing": f"CUDA events between kernels over {Kp} further steps (vpass includes the split reduction)",
         "kernels_GBps": {"kpass": round(kp_gbs, 1), "vpass": round(vp_gbs, 1)},
-        "e2e": {"value": round(world * B / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(whole_job_tokens_per_s(world, B, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
         "gpu_launches": K * len(layers) * 7,   # append: V GEMM + K codes; decode: 5
         "clocks": clk,

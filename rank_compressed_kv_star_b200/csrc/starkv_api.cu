@@ -30,6 +30,9 @@
 #ifndef STARKV_V_RING_BYTES
 #define STARKV_V_RING_BYTES (105 * 1024)
 #endif
+#ifndef STARKV_UP_CTAS_PER_SM
+#define STARKV_UP_CTAS_PER_SM 1
+#endif
 
 namespace starkv {
 namespace {
@@ -161,13 +164,15 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
     p.up_npad = rows < 16 ? 16 : (rows + 15) / 16 * 16;
   }
   p.up_ks = 1;
-  while (p.up_ks < 8 && p.H * p.up_mt * p.up_bt * p.up_ks * 2 <= sms && p.R / kUpKC >= p.up_ks * 2) p.up_ks *= 2;
+  while (p.up_ks < 8 && p.H * p.up_mt * p.up_bt * p.up_ks * 2 <= sms * STARKV_UP_CTAS_PER_SM &&
+         p.R / kUpKC >= p.up_ks * 2)
+    p.up_ks *= 2;
   p.up_kpc = ((p.R + p.up_ks * kUpKC - 1) / (p.up_ks * kUpKC)) * kUpKC;
   {
     // stage: two 64x64 B_V boxes + hi and lo Z boxes (npad rows x 128 B); the
     // epilogue's [npad][128] fp32 partial reuses the ring (>= 2 stages always hold it)
     const size_t stage = 2u * kUpKC * 128u + 2u * static_cast<size_t>(p.up_npad) * 128u;
-    p.up_stages = static_cast<int>((160u * 1024u) / stage);
+    p.up_stages = static_cast<int>((160u * 1024u / STARKV_UP_CTAS_PER_SM) / stage);
     if (p.up_stages > 4) p.up_stages = 4;
     if (p.up_stages < 2) p.up_stages = 2;
     while (static_cast<size_t>(p.up_stages) * stage < static_cast<size_t>(p.up_npad) * 512u) ++p.up_stages;
