@@ -77,6 +77,17 @@ def whole_job_tokens_per_s(world: int, batch_per_rank: int, ms_per_step_max: flo
     return world * batch_per_rank / (ms_per_step_max * 1e-3)
 
 
+# DRAM bytes (read + write) per processed token measured by one ncu capture of
+# the streaming kernels on the batch-32, context-8192 case (32 heads, K rank 64,
+# V rank 2048); traffic grows in proportion to the tokens processed.  Valid
+# only for that geometry and for the kernels as they were captured.
+NCU_TRAFFIC_PER_TOKEN = {
+    "kpass": (1.074168e9 + 6.671104e6) / (32 * 8192),
+    "vpass": (1.107514e9 + 5.822976e6) / (32 * 8192),
+}
+NCU_TRAFFIC_GEOMETRY = (32, 64, 2048)   # (heads, K rank, V rank)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -273,6 +284,9 @@ def run_ours(args):
     vp_gbs = v_bytes / (per["vpass"] * 1e-3) / 1e9
     dom = "kpass" if per["kpass"] >= per["vpass"] else "vpass"
     dom_bytes, dom_gbs = (k_bytes, kp_gbs) if dom == "kpass" else (v_bytes, vp_gbs)
+    traffic = None
+    if len(layers) == 1 and (layers[0]["H"], layers[0]["r"], layers[0]["R"]) == NCU_TRAFFIC_GEOMETRY:
+        traffic = round(NCU_TRAFFIC_PER_TOKEN[dom] * T_sum)
 
     # ---------------- end to end through the public API with host buffers
     Ke = max(1, min(args.e2e_steps, K))
@@ -319,7 +333,7 @@ def run_ours(args):
                 "frac_of_8TBps": round(step_bytes / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4),
                 "frac_of_peak": round(step_bytes / (ms * 1e-3) / 1e9 / peak, 4), "peak_kind": peak_kind},
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": round(dom_gbs, 1), "peak": peak,
-                     "unit": "GB/s", "frac": round(dom_gbs / peak, 4), "traffic": None,
+                     "unit": "GB/s", "frac": round(dom_gbs / peak, 4), "traffic": traffic,
                      "algorithmic_bytes_per_launch": dom_bytes // len(layers), "peak_kind": peak_kind},
         "kernels_ms_per_step": {n: round(v, 5) for n, v in per.items()},
         "kernels_timing": f"CUDA events between kernels over {Kp} further steps (vpass includes the split reduction)",
