@@ -232,6 +232,24 @@ const char* starkv_status_string(starkv_status status);
  */
 int32_t starkv_rank_from_spectrum(const double* s, int32_t n, double tau);
 
+/*
+ * Capacity arithmetic (host functions, no GPU).  A token costs, in every layer,
+ * H*r fp16 K codes plus R fp16 V codes; a full-rank cache is the case r = d,
+ * R = H*d (2*2*H*d bytes per layer).  The README's boot log for the
+ * uncompressed 7B cache is the worked example: 6.99 GiB of KV memory, 16-token
+ * blocks, 32 layers x 512 KiB -> 894 blocks = 14,304 tokens ("Low-rank KV
+ * Cache Compression for vLLM", measured results at 8192 context).
+ *
+ * starkv_kv_bytes_per_token: 2 * sum_l (num_heads[l]*k_ranks[l] + v_ranks[l]);
+ *   HOST arrays of n_layers entries; -1 on invalid input (n_layers <= 0, null
+ *   array, non-positive entry).
+ * starkv_num_blocks: floor(budget_bytes / (block_size * bytes_per_token));
+ *   -1 on invalid input (negative budget, non-positive sizes).
+ */
+int64_t starkv_kv_bytes_per_token(int32_t n_layers, const int32_t* num_heads,
+                                  const int32_t* k_ranks, const int32_t* v_ranks);
+int64_t starkv_num_blocks(int64_t budget_bytes, int64_t bytes_per_token, int32_t block_size);
+
 /* Library version, 10000*major + 100*minor + patch. */
 int32_t starkv_version(void);
 

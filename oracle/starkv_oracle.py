@@ -256,3 +256,19 @@ def rank_from_spectrum(s, tau: float) -> int:
     """
     s = np.asarray(s, dtype=np.float64)
     return int(np.count_nonzero(s > tau))
+
+
+# ----------------------------------------------------------------- capacity
+
+def kv_bytes_per_token(num_heads, k_ranks, v_ranks) -> int:
+    """fp16 bytes one token occupies in the compressed cache, summed over layers.
+
+    Per layer a token stores H*r head-wise K codes and R joint V codes (the
+    paged format above), 2 bytes each.  A full-rank cache is r = d, R = H*d.
+    """
+    return sum(2 * (h * r + R) for h, r, R in zip(num_heads, k_ranks, v_ranks))
+
+
+def num_blocks(budget_bytes: int, bytes_per_token: int, block_size: int = BLOCK_SIZE) -> int:
+    """Whole blocks of ``block_size`` tokens that fit in ``budget_bytes``."""
+    return budget_bytes // (block_size * bytes_per_token)

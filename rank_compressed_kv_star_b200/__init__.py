@@ -27,7 +27,7 @@ EXPORTED = (
     "starkv_compress_append", "starkv_decode_workspace_bytes", "starkv_paged_decode",
     "starkv_paged_decode_profiled", "starkv_paged_decode_static",
     "starkv_decode_check", "starkv_decode_workspace_layout", "starkv_status_string",
-    "starkv_rank_from_spectrum", "starkv_version",
+    "starkv_rank_from_spectrum", "starkv_version", "starkv_kv_bytes_per_token", "starkv_num_blocks",
 )
 
 
@@ -96,6 +96,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.starkv_status_string.restype = ctypes.c_char_p
     lib.starkv_rank_from_spectrum.argtypes = [ctypes.POINTER(ctypes.c_double), I32, ctypes.c_double]
     lib.starkv_rank_from_spectrum.restype = I32
+    I64 = ctypes.c_int64
+    IP = ctypes.POINTER(ctypes.c_int32)
+    lib.starkv_kv_bytes_per_token.argtypes = [I32, IP, IP, IP]
+    lib.starkv_kv_bytes_per_token.restype = I64
+    lib.starkv_num_blocks.argtypes = [I64, I64, I32]
+    lib.starkv_num_blocks.restype = I64
     lib.starkv_version.argtypes = []
     lib.starkv_version.restype = I32
     _lib = lib
@@ -206,6 +212,17 @@ def starkv_rank_from_spectrum(s, tau: float) -> int:
     vals = [float(x) for x in s]
     arr = (ctypes.c_double * len(vals))(*vals) if vals else None
     return int(load_library().starkv_rank_from_spectrum(arr, len(vals), float(tau)))
+
+
+def starkv_kv_bytes_per_token(num_heads, k_ranks, v_ranks) -> int:
+    """Compressed cache bytes per token over the layers (one entry per layer)."""
+    n = len(num_heads)
+    arr = lambda xs: (ctypes.c_int32 * n)(*[int(x) for x in xs]) if n else None
+    return int(load_library().starkv_kv_bytes_per_token(n, arr(num_heads), arr(k_ranks), arr(v_ranks)))
+
+
+def starkv_num_blocks(budget_bytes: int, bytes_per_token: int, block_size: int = 16) -> int:
+    return int(load_library().starkv_num_blocks(int(budget_bytes), int(bytes_per_token), block_size))
 
 
 def starkv_version() -> int:

@@ -334,6 +334,22 @@ const char* starkv_status_string(starkv_status s) {
 
 int32_t starkv_version(void) { return 100; }
 
+int64_t starkv_kv_bytes_per_token(int32_t n_layers, const int32_t* num_heads, const int32_t* k_ranks,
+                                  const int32_t* v_ranks) {
+  if (n_layers <= 0 || !num_heads || !k_ranks || !v_ranks) return -1;
+  int64_t codes = 0;
+  for (int32_t l = 0; l < n_layers; ++l) {
+    if (num_heads[l] <= 0 || k_ranks[l] <= 0 || v_ranks[l] <= 0) return -1;
+    codes += static_cast<int64_t>(num_heads[l]) * k_ranks[l] + v_ranks[l];
+  }
+  return 2 * codes;
+}
+
+int64_t starkv_num_blocks(int64_t budget_bytes, int64_t bytes_per_token, int32_t block_size) {
+  if (budget_bytes < 0 || bytes_per_token <= 0 || block_size <= 0) return -1;
+  return budget_bytes / (static_cast<int64_t>(block_size) * bytes_per_token);
+}
+
 int32_t starkv_rank_from_spectrum(const double* s, int32_t n, double tau) {
   if (n < 0 || (n > 0 && !s) || std::isnan(tau)) return -1;
   int32_t c = 0;
