@@ -106,6 +106,21 @@ starkv_status starkv_compress_append(const starkv_layer_desc* desc, int32_t batc
                                      void* k_cache, void* v_cache, void* stream);
 
 /*
+ * starkv_compress_store -- compress n_tokens rows of k, v (for instance a
+ * prompt at prefill) and store each row's codes at an explicit flat slot:
+ * slot_mapping[i] = page * 16 + offset, int32 [n_tokens].  Same arithmetic,
+ * layouts and rounding as starkv_compress_append; rows whose slot is outside
+ * [0, num_blocks*16) are skipped; targets must be distinct.  k, v fp16
+ * [n_tokens][H][d].  Cites: README method paragraph (codes "stored in a
+ * compressed paged format"); the flat slot is the paged address
+ * block_table[b][t/16]*16 + t%16 precomputed by the caller.
+ */
+starkv_status starkv_compress_store(const starkv_layer_desc* desc, int32_t n_tokens, const void* k,
+                                    const void* v, const void* A_K, const void* A_V,
+                                    const int32_t* slot_mapping, void* k_cache, void* v_cache,
+                                    void* stream);
+
+/*
  * starkv_decode_workspace_bytes -- device scratch needed by starkv_paged_decode
  * for this layer geometry, batch size and length bound (0 on invalid input).
  * Depends on the SM count of the current device.

@@ -96,6 +96,21 @@ def compress_append(k, v, A_K, A_V, tables, positions, k_cache, v_cache):
     return c_K, c_V, kc, vc
 
 
+def compress_store(k, v, A_K, A_V, slot_mapping, k_cache, v_cache, block_size=BLOCK_SIZE):
+    """Compress rows and store their fp16 codes at flat slots ``page*16 + offset``.
+
+    Returns ``(c_K, c_V, new_k_cache, new_v_cache)`` (inputs not modified).
+    """
+    c_K, c_V = compress(k, v, A_K, A_V)
+    kc = np.array(k_cache, copy=True)
+    vc = np.array(v_cache, copy=True)
+    for i, sl in enumerate(slot_mapping):
+        page, off = divmod(int(sl), block_size)
+        kc[page, off] = c_K[i].astype(np.float16)
+        vc[page, off] = c_V[i].astype(np.float16)
+    return c_K, c_V, kc, vc
+
+
 # ------------------------------------------------------------ decompression
 
 def decompress_k(c_K_seq: np.ndarray, B_K: np.ndarray) -> np.ndarray:

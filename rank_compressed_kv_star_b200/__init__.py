@@ -24,7 +24,8 @@ STATUS = {
 FLAG_BAD_BLOCK_ID, FLAG_BAD_SEQ_LEN, FLAG_TIMEOUT = 1, 2, 4
 
 EXPORTED = (
-    "starkv_compress_append", "starkv_decode_workspace_bytes", "starkv_paged_decode",
+    "starkv_compress_append", "starkv_compress_store", "starkv_decode_workspace_bytes",
+    "starkv_paged_decode",
     "starkv_paged_decode_profiled", "starkv_paged_decode_static",
     "starkv_decode_check", "starkv_decode_workspace_layout", "starkv_status_string",
     "starkv_rank_from_spectrum", "starkv_version", "starkv_kv_bytes_per_token", "starkv_num_blocks",
@@ -78,6 +79,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     DP = ctypes.POINTER(LayerDesc)
     lib.starkv_compress_append.argtypes = [DP, I32, P, P, P, P, P, P, P, P, P]
     lib.starkv_compress_append.restype = ctypes.c_int
+    lib.starkv_compress_store.argtypes = [DP, I32, P, P, P, P, P, P, P, P]
+    lib.starkv_compress_store.restype = ctypes.c_int
     lib.starkv_decode_workspace_bytes.argtypes = [DP, I32, I32]
     lib.starkv_decode_workspace_bytes.restype = SZ
     lib.starkv_paged_decode.argtypes = [DP, I32, I32, P, P, P, P, P, P, P, ctypes.c_float,
@@ -141,6 +144,16 @@ def starkv_compress_append(desc: LayerDesc, batch: int, k, v, A_K, A_V, block_ta
         _ptr(positions), _ptr(k_cache), _ptr(v_cache), _stream(stream))
     if check:
         _check(st, "starkv_compress_append")
+    return st
+
+
+def starkv_compress_store(desc: LayerDesc, n_tokens: int, k, v, A_K, A_V, slot_mapping, k_cache,
+                          v_cache, stream=None, check: bool = True) -> int:
+    st = load_library().starkv_compress_store(
+        _desc_ref(desc), n_tokens, _ptr(k), _ptr(v), _ptr(A_K), _ptr(A_V), _ptr(slot_mapping),
+        _ptr(k_cache), _ptr(v_cache), _stream(stream))
+    if check:
+        _check(st, "starkv_compress_store")
     return st
 
 

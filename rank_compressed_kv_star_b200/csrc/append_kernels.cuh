@@ -23,14 +23,21 @@
 
 namespace starkv {
 
+// Where row b's codes go: either an explicit flat slot (page*16 + offset) per
+// row, or (block table row, position) per sequence.
 struct AppendTarget {
+  const int32_t* slots;    // [B] flat slots, or null to use tables/positions
   const int32_t* tables;   // [B][MB]
   const int32_t* positions;
   int MB, NB;
 };
 
-// Physical row (page*16 + slot) of sequence b's append target, or -1.
+// Physical row (page*16 + slot) of row b's target, or -1 when out of range.
 __device__ __forceinline__ int64_t append_row(const AppendTarget& a, int b) {
+  if (a.slots) {
+    const int32_t sl = a.slots[b];
+    return (sl < 0 || sl >= a.NB * 16) ? -1 : static_cast<int64_t>(sl);
+  }
   const int32_t pos = a.positions[b];
   if (pos < 0 || pos / 16 >= a.MB) return -1;
   const int32_t phys = a.tables[static_cast<size_t>(b) * a.MB + pos / 16];

@@ -358,23 +358,24 @@ int32_t starkv_rank_from_spectrum(const double* s, int32_t n, double tau) {
   return c;
 }
 
-starkv_status starkv_compress_append(const starkv_layer_desc* desc, int32_t batch, const void* k, const void* v,
-                                     const void* A_K, const void* A_V, const int32_t* block_tables,
-                                     const int32_t* positions, void* k_cache, void* v_cache, void* stream) {
+namespace {
+// Compress rows of k, v and store their codes at the target rows (see AppendTarget).
+starkv_status compress_store_impl(const starkv_layer_desc* desc, int32_t batch, const void* k, const void* v,
+                                  const void* A_K, const void* A_V, AppendTarget tgt, void* k_cache,
+                                  void* v_cache, void* stream) {
   starkv_status st = check_desc(desc);
   if (st != STARKV_OK) return st;
   if (batch < 0) return STARKV_ERR_INVALID_ARG;
   if (batch == 0) return STARKV_OK;
-  if (!k || !v || !A_K || !A_V || !block_tables || !positions || !k_cache || !v_cache)
-    return STARKV_ERR_INVALID_ARG;
+  if (!k || !v || !A_K || !A_V || !k_cache || !v_cache) return STARKV_ERR_INVALID_ARG;
+  if (!tgt.slots && (!tgt.tables || !tgt.positions)) return STARKV_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v) || !aligned16(A_K) || !aligned16(A_V) || !aligned16(k_cache) ||
-      !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
-      (reinterpret_cast<uintptr_t>(positions) & 3u))
+      !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(tgt.tables) & 3u) ||
+      (reinterpret_cast<uintptr_t>(tgt.positions) & 3u) || (reinterpret_cast<uintptr_t>(tgt.slots) & 3u))
     return STARKV_ERR_INVALID_ARG;
   const int H = desc->num_heads, d = desc->head_dim, r = desc->k_rank, R = desc->v_rank;
   const int HD = H * d;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  AppendTarget tgt{block_tables, positions, desc->max_blocks_per_seq, desc->num_blocks};
 
   // ---- joint V codes: tcgen05 GEMM, split-K over a cluster
   CUtensorMap amap, vmap;
@@ -416,6 +417,25 @@ starkv_status starkv_compress_append(const starkv_layer_desc* desc, int32_t batc
   if (launch(append_k_kernel, dim3(H, (batch + kAppKB - 1) / kAppKB), dim3(256), ksm, s, 1, kp) != cudaSuccess)
     return STARKV_ERR_CUDA;
   return STARKV_OK;
+}
+}  // namespace
+
+starkv_status starkv_compress_append(const starkv_layer_desc* desc, int32_t batch, const void* k, const void* v,
+                                     const void* A_K, const void* A_V, const int32_t* block_tables,
+                                     const int32_t* positions, void* k_cache, void* v_cache, void* stream) {
+  if (batch > 0 && (!block_tables || !positions)) return STARKV_ERR_INVALID_ARG;
+  AppendTarget tgt{nullptr, block_tables, positions, desc ? desc->max_blocks_per_seq : 0,
+                   desc ? desc->num_blocks : 0};
+  return compress_store_impl(desc, batch, k, v, A_K, A_V, tgt, k_cache, v_cache, stream);
+}
+
+starkv_status starkv_compress_store(const starkv_layer_desc* desc, int32_t n_tokens, const void* k, const void* v,
+                                    const void* A_K, const void* A_V, const int32_t* slot_mapping, void* k_cache,
+                                    void* v_cache, void* stream) {
+  if (n_tokens > 0 && !slot_mapping) return STARKV_ERR_INVALID_ARG;
+  AppendTarget tgt{slot_mapping, nullptr, nullptr, desc ? desc->max_blocks_per_seq : 0,
+                   desc ? desc->num_blocks : 0};
+  return compress_store_impl(desc, n_tokens, k, v, A_K, A_V, tgt, k_cache, v_cache, stream);
 }
 
 size_t starkv_decode_workspace_bytes(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len) {

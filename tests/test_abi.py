@@ -120,3 +120,16 @@ def test_workspace_layout_is_consistent(lib):
     # grows with batch and length
     assert S.starkv_decode_workspace_bytes(d, 65, 8192) > lay.total_bytes
     assert S.starkv_decode_workspace_bytes(d, 64, 8200) > lay.total_bytes
+
+
+def test_compress_store_argument_errors(lib):
+    d = _desc()
+    fake = 1 << 20
+    args = [d, 8, fake, fake, fake, fake, fake, fake, fake]
+    a = list(args); a[6] = None                    # no slot mapping
+    assert S.starkv_compress_store(*a, stream=0, check=False) == 1
+    a = list(args); a[6] = fake + 2                # misaligned slot mapping
+    assert S.starkv_compress_store(*a, stream=0, check=False) == 1
+    a = list(args); a[1] = 0
+    assert S.starkv_compress_store(*a, stream=0, check=False) == 0
+    assert S.starkv_compress_store(_desc(block_size=8), *args[1:], stream=0, check=False) == 2

@@ -332,6 +332,51 @@ def test_append_then_decode_continuous_batching_subset(layer):
     assert_close({b: got[b] for b in range(6)}, ref)
 
 
+def test_compress_store_prefill_then_decode():
+    """A 600-token prompt compressed by slot mapping (three 256-row tiles), then decoded."""
+    sh = W.LayerShape(32, 128, 64, 2048)
+    T = 600
+    wl = W.custom("prefill", 4242, sh, [T], append=False)
+    tables, nb, _ = W.block_tables(wl.seed, np.array([T]), -(-T // 16) + 2)
+    A_K, A_V, B_K, B_V = W.projections(wl, 0)
+    key = gen.stream_key(wl.seed, 99)
+    kx = gen.codes_f16(key, T, 32 * 128, None).reshape(T, 32, 128)
+    vx = gen.codes_f16(key + 1, T, 32 * 128, None).reshape(T, 32, 128)
+    slots = np.array([tables[0][t // 16] * 16 + t % 16 for t in range(T)], dtype=np.int32)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    kc = torch.full((nb, 16, 32, 64), float("nan"), dtype=torch.float16, device="cuda")
+    vc = torch.full((nb, 16, 2048), float("nan"), dtype=torch.float16, device="cuda")
+    desc = S.layer_desc(32, 128, 64, 2048, nb, tables.shape[1])
+    S.starkv_compress_store(desc, T, dev(kx), dev(vx), dev(A_K), dev(A_V), dev(slots), kc, vc)
+    torch.cuda.synchronize()
+    cK, cV, kc_ref, vc_ref = O.compress_store(kx, vx, A_K, A_V, slots, np.full((nb, 16, 32, 64), np.nan, np.float16),
+                                              np.full((nb, 16, 2048), np.nan, np.float16))
+    kg, vg = kc.cpu().numpy(), vc.cpu().numpy()
+    assert np.array_equal(np.isnan(kg), np.isnan(kc_ref)) and np.array_equal(np.isnan(vg), np.isnan(vc_ref))
+    kgot = kg.reshape(-1, 32 * 64)[slots].astype(np.float64)
+    vgot = vg.reshape(-1, 2048)[slots].astype(np.float64)
+    for got, want in ((kgot, cK.reshape(T, -1)), (vgot, cV)):
+        assert np.abs(got - want).max() <= MAX_ABS and rel_l2(got, want) <= REL_L2
+    q = gen.codes_f16(key + 2, 1, 32 * 128, None).reshape(1, 32, 128)
+    L = dict(H=32, d=128, r=64, R=2048, nb=nb, tables=dev(tables), seq_lens=dev(np.array([T], np.int32)),
+             k_cache=kc, v_cache=vc, q=dev(q), B_K=dev(B_K), B_V=dev(B_V), scale=1 / np.sqrt(128))
+    got, *_ = run_decode(L)
+    ref = O.decode_explicit(q, B_K, B_V, kc_ref, vc_ref, tables, [T], 1 / np.sqrt(128))
+    assert_close({0: got[0]}, {0: ref[0]})
+
+
+def test_decode_and_append_batch_over_256():
+    """300 short sequences: several 256-row batch tiles in the append GEMM and the up-projection."""
+    sh = W.LayerShape(32, 128, 64, 2048)
+    rng = np.random.default_rng(5)
+    wl = W.custom("wide", 5150, sh, rng.integers(1, 48, size=300), append=True)
+    Lh, Ld, appended = _append_check(wl)
+    got, *_ = run_decode(Ld)
+    sample = [0, 1, 255, 256, 257, 299]
+    ref = oracle_rows(wl, 0, Lh["q"], Ld["A_np"], sample, wl.seq_lens, appended)
+    assert_close({b: got[b] for b in sample}, ref)
+
+
 # ---------------------------------------------------- full-size workloads
 
 @pytest.mark.parametrize("idx,layer,sample", [

@@ -383,3 +383,15 @@ def test_planted_slot_mistake_is_caught(monkeypatch):
     monkeypatch.setattr(O, "gather", _mut_slot_shift)
     with pytest.raises((AssertionError, IndexError)):
         check_contiguous_equals_paged()
+
+
+def test_slot_mapped_store_equals_block_table_append():
+    sh = W.LayerShape(4, 64, 16, 64)
+    wl = W.custom("store", 41, sh, [37, 100, 0, 15], append=True)
+    L = W.host_layer(wl, 0)
+    pos = L["ctx_lens"]
+    slots = [int(L["tables"][b][pos[b] // 16]) * 16 + int(pos[b] % 16) for b in range(wl.batch)]
+    a = O.compress_append(L["k"], L["v"], L["A_K"], L["A_V"], L["tables"], pos, L["k_cache"], L["v_cache"])
+    s = O.compress_store(L["k"], L["v"], L["A_K"], L["A_V"], slots, L["k_cache"], L["v_cache"])
+    for x, y in zip(a[2:], s[2:]):
+        assert np.array_equal(x.view(np.uint16), y.view(np.uint16))
