@@ -26,6 +26,14 @@ What it computes (written from the method's description, not from any code):
 * Decode: single-token attention of the new query over the sequence's cached
   tokens, textbook softmax with scale ``1/sqrt(head_dim)``.
 
+* Grouped-query attention: the README lists Qwen, Mistral, Gemma and Llama-3
+  support (wpnews.pro README, status paragraph), families whose layers have
+  fewer KV heads than query heads.  Reading taken: K and V are compressed per
+  *KV* head (head-wise A_K[j] for each of the Hkv KV heads, joint A_V over the
+  Hkv*head_dim concatenated values), and query head ``h`` attends with KV head
+  ``h // (H / Hkv)`` (consecutive query heads share a KV head).  With
+  ``Hkv == H`` everything below is plain multi-head attention.
+
 Readings where the pages are silent (also listed in the design notes):
 K page layout ``[num_blocks][16][H][r]``, V page layout ``[num_blocks][16][R]``
 (token-major inside a page, one block table shared by both pools);
@@ -39,6 +47,15 @@ from __future__ import annotations
 import numpy as np
 
 BLOCK_SIZE = 16
+
+
+# ------------------------------------------------------------------ heads
+
+def kv_head(h: int, num_heads: int, num_kv_heads: int) -> int:
+    """KV head that query head ``h`` reads (consecutive groups of H/Hkv heads)."""
+    if num_heads % num_kv_heads:
+        raise ValueError("query heads must be a multiple of KV heads")
+    return h // (num_heads // num_kv_heads)
 
 
 # ------------------------------------------------------------------ paging
@@ -62,8 +79,8 @@ def gather(cache: np.ndarray, table_row: np.ndarray, T: int) -> np.ndarray:
 def compress(k: np.ndarray, v: np.ndarray, A_K: np.ndarray, A_V: np.ndarray):
     """Codes of new tokens.
 
-    k, v: ``[B][H][d]``; A_K ``[H][d][r]`` (head-wise); A_V ``[H*d][R]`` (joint).
-    Returns fp64 ``c_K [B][H][r]`` and ``c_V [B][R]``.
+    k, v: ``[B][Hkv][d]``; A_K ``[Hkv][d][r]`` (head-wise); A_V ``[Hkv*d][R]``
+    (joint).  Returns fp64 ``c_K [B][Hkv][r]`` and ``c_V [B][R]``.
     """
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -114,7 +131,7 @@ def compress_store(k, v, A_K, A_V, slot_mapping, k_cache, v_cache, block_size=BL
 # ------------------------------------------------------------ decompression
 
 def decompress_k(c_K_seq: np.ndarray, B_K: np.ndarray) -> np.ndarray:
-    """``k_hat[t, h, :] = c_K[t, h, :] . B_K[h]``; returns ``[T][H][d]``."""
+    """``k_hat[t, j, :] = c_K[t, j, :] . B_K[j]`` per KV head j; returns ``[T][Hkv][d]``."""
     B_K = np.asarray(B_K, dtype=np.float64)
     T, H, _ = c_K_seq.shape
     out = np.empty((T, H, B_K.shape[2]))
@@ -124,7 +141,7 @@ def decompress_k(c_K_seq: np.ndarray, B_K: np.ndarray) -> np.ndarray:
 
 
 def decompress_v(c_V_seq: np.ndarray, B_V: np.ndarray) -> np.ndarray:
-    """``v_hat[t, :] = c_V[t, :] . B_V``; returns ``[T][H*d]``."""
+    """``v_hat[t, :] = c_V[t, :] . B_V``; returns ``[T][Hkv*d]``."""
     return c_V_seq @ np.asarray(B_V, dtype=np.float64)
 
 
@@ -150,11 +167,13 @@ def decode_explicit(q, B_K, B_V, k_cache, v_cache, tables, seq_lens, scale):
     """Definition of decode: decompress K and V explicitly, then attend.
 
     For every sequence: walk the block table, gather the codes of its
-    ``seq_lens[b]`` tokens, rebuild ``k_hat``/``v_hat`` and run textbook
-    softmax attention per head.  Returns fp64 ``[B][H][d]``.
+    ``seq_lens[b]`` tokens, rebuild ``k_hat``/``v_hat`` per KV head and run
+    textbook softmax attention per query head with its KV head.  Returns
+    fp64 ``[B][H][d]`` (H query heads; Hkv = ``B_K.shape[0]``).
     """
     q = np.asarray(q, dtype=np.float64)
     Bsz, H, d = q.shape
+    Hkv = np.shape(B_K)[0]
     out = np.zeros((Bsz, H, d))
     for b in range(Bsz):
         T = int(seq_lens[b])
@@ -163,9 +182,10 @@ def decode_explicit(q, B_K, B_V, k_cache, v_cache, tables, seq_lens, scale):
         c_K = gather(k_cache, tables[b], T)
         c_V = gather(v_cache, tables[b], T)
         k_hat = decompress_k(c_K, B_K)
-        v_hat = decompress_v(c_V, B_V).reshape(T, H, d)
+        v_hat = decompress_v(c_V, B_V).reshape(T, Hkv, d)
         for h in range(H):
-            out[b, h] = attention_head(q[b, h], k_hat[:, h, :], v_hat[:, h, :], scale)
+            j = kv_head(h, H, Hkv)
+            out[b, h] = attention_head(q[b, h], k_hat[:, j, :], v_hat[:, j, :], scale)
     return out
 
 
@@ -174,13 +194,14 @@ def attend_codes_reordered(q_b, B_K, B_V, c_K, c_V, scale, heads=None):
 
     K is still decompressed explicitly.  For V the weighted sum is taken over
     the codes first, ``z_h = sum_t p_t c_V[t]``, and then projected,
-    ``o_h = z_h . B_V[:, h*d:(h+1)*d]`` (associativity of the matrix product;
-    agreement with :func:`decode_explicit` is a pinned test).  Returns
-    ``[len(heads)][d]`` fp64.
+    ``o_h = z_h . B_V[:, j*d:(j+1)*d]`` with ``j`` the head's KV head
+    (associativity of the matrix product; agreement with
+    :func:`decode_explicit` is a pinned test).  Returns ``[len(heads)][d]`` fp64.
     """
     q_b = np.asarray(q_b, dtype=np.float64)
     B_V = np.asarray(B_V, dtype=np.float64)
     H, d = q_b.shape
+    Hkv = np.shape(B_K)[0]
     heads = range(H) if heads is None else heads
     T = c_K.shape[0]
     out = np.zeros((len(heads), d))
@@ -188,10 +209,11 @@ def attend_codes_reordered(q_b, B_K, B_V, c_K, c_V, scale, heads=None):
         return out
     B_K = np.asarray(B_K, dtype=np.float64)
     for i, h in enumerate(heads):
-        k_hat_h = c_K[:, h, :] @ B_K[h]
+        j = kv_head(h, H, Hkv)
+        k_hat_h = c_K[:, j, :] @ B_K[j]
         p = softmax(scale * (k_hat_h @ q_b[h]))
         z = p @ c_V
-        out[i] = z @ B_V[:, h * d:(h + 1) * d]
+        out[i] = z @ B_V[:, j * d:(j + 1) * d]
     return out
 
 
@@ -213,6 +235,7 @@ def decode_contiguous(q, B_K, B_V, c_K_list, c_V_list, scale):
     """Decode over per-sequence contiguous code arrays (no paging)."""
     q = np.asarray(q, dtype=np.float64)
     Bsz, H, d = q.shape
+    Hkv = np.shape(B_K)[0]
     out = np.zeros((Bsz, H, d))
     for b in range(Bsz):
         c_K = np.asarray(c_K_list[b], dtype=np.float64)
@@ -221,42 +244,47 @@ def decode_contiguous(q, B_K, B_V, c_K_list, c_V_list, scale):
         if T == 0:
             continue
         k_hat = decompress_k(c_K, B_K)
-        v_hat = decompress_v(c_V, B_V).reshape(T, H, d)
+        v_hat = decompress_v(c_V, B_V).reshape(T, Hkv, d)
         for h in range(H):
-            out[b, h] = attention_head(q[b, h], k_hat[:, h, :], v_hat[:, h, :], scale)
+            j = kv_head(h, H, Hkv)
+            out[b, h] = attention_head(q[b, h], k_hat[:, j, :], v_hat[:, j, :], scale)
     return out
 
 
 def attention_uncompressed(q, k_list, v_list, scale):
-    """Plain multi-head single-query attention over full K/V ``[T][H][d]``."""
+    """Plain single-query attention over full K/V ``[T][Hkv][d]`` (grouped when Hkv < H)."""
     q = np.asarray(q, dtype=np.float64)
     Bsz, H, d = q.shape
     out = np.zeros((Bsz, H, d))
     for b in range(Bsz):
         k = np.asarray(k_list[b], dtype=np.float64)
         v = np.asarray(v_list[b], dtype=np.float64)
+        Hkv = k.shape[1]
         for h in range(H):
-            out[b, h] = attention_head(q[b, h], k[:, h, :], v[:, h, :], scale)
+            j = kv_head(h, H, Hkv)
+            out[b, h] = attention_head(q[b, h], k[:, j, :], v[:, j, :], scale)
     return out
 
 
 def decode_stages(q_b, B_K, B_V, c_K, c_V, scale):
     """Intermediate quantities of one sequence in absorbed form, for diagnosis.
 
-    ``q_tilde[h] = scale * q_h . B_K[h]^T`` (r-vector), ``s[h, t] =
-    q_tilde[h] . c_K[t, h]``, ``p = softmax_t(s)``, ``z[h] = p[h] . c_V`` and
-    ``o[h] = z[h] . B_V[:, h*d:(h+1)*d]``.  The scores here are natural-log
-    logits (no base-2 change).
+    With ``j = g(h)`` the query head's KV head: ``q_tilde[h] = scale * q_h .
+    B_K[j]^T`` (r-vector), ``s[h, t] = q_tilde[h] . c_K[t, j]``, ``p =
+    softmax_t(s)``, ``z[h] = p[h] . c_V`` and ``o[h] = z[h] . B_V[:,
+    j*d:(j+1)*d]``.  The scores here are natural-log logits (no base-2 change).
     """
     q_b = np.asarray(q_b, dtype=np.float64)
     B_K = np.asarray(B_K, dtype=np.float64)
     B_V = np.asarray(B_V, dtype=np.float64)
     H, d = q_b.shape
-    q_tilde = np.stack([scale * (B_K[h] @ q_b[h]) for h in range(H)])
-    s = np.einsum("hr,thr->ht", q_tilde, c_K)
+    Hkv = B_K.shape[0]
+    g = [kv_head(h, H, Hkv) for h in range(H)]
+    q_tilde = np.stack([scale * (B_K[g[h]] @ q_b[h]) for h in range(H)])
+    s = np.stack([c_K[:, g[h], :] @ q_tilde[h] for h in range(H)])
     p = softmax(s)
     z = p @ c_V
-    o = np.stack([z[h] @ B_V[:, h * d:(h + 1) * d] for h in range(H)])
+    o = np.stack([z[h] @ B_V[:, g[h] * d:(g[h] + 1) * d] for h in range(H)])
     return dict(q_tilde=q_tilde, s=s, p=p, z=z, o=o)
 
 
@@ -279,7 +307,8 @@ def kv_bytes_per_token(num_heads, k_ranks, v_ranks) -> int:
     """fp16 bytes one token occupies in the compressed cache, summed over layers.
 
     Per layer a token stores H*r head-wise K codes and R joint V codes (the
-    paged format above), 2 bytes each.  A full-rank cache is r = d, R = H*d.
+    paged format above), 2 bytes each, with H the layer's KV heads.  A
+    full-rank cache is r = d, R = H*d.
     """
     return sum(2 * (h * r + R) for h, r, R in zip(num_heads, k_ranks, v_ranks))
 

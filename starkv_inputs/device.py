@@ -61,33 +61,34 @@ def device_layer(wl: W.Workload, layer: int, device="cuda", tables=None, nb=None
     """
     sh = wl.layers[layer]
     H, d, r, R = sh.num_heads, sh.head_dim, sh.k_rank, sh.v_rank
+    Hkv = sh.kv_heads
     if tables is None:
         tables, nb, _ = W.block_tables(wl.seed, wl.seq_lens, wl.max_blocks_per_seq, wl.decoy_frac)
-    k_cache = torch.empty((nb, W.BLOCK_SIZE, H, r), dtype=torch.float16, device=device)
+    k_cache = torch.empty((nb, W.BLOCK_SIZE, Hkv, r), dtype=torch.float16, device=device)
     v_cache = torch.empty((nb, W.BLOCK_SIZE, R), dtype=torch.float16, device=device)
     if fill_nan:
         k_cache.fill_(float("nan"))
         v_cache.fill_(float("nan"))
     kspec = torch.from_numpy(W.k_spectrum(sh)).to(device)
     vspec = torch.from_numpy(W.v_spectrum(sh)).to(device)
-    kflat = k_cache.view(nb * W.BLOCK_SIZE, H * r)
+    kflat = k_cache.view(nb * W.BLOCK_SIZE, Hkv * r)
     vflat = v_cache.view(nb * W.BLOCK_SIZE, R)
     tmax = int(wl.ctx_lens.max()) if wl.batch else 0
-    tk = torch.empty(max(tmax, 1) * H * r, dtype=torch.float16, device=device)
+    tk = torch.empty(max(tmax, 1) * Hkv * r, dtype=torch.float16, device=device)
     tv = torch.empty(max(tmax, 1) * R, dtype=torch.float16, device=device)
     for b in range(wl.batch):
         T = int(wl.ctx_lens[b])
         if T == 0:
             continue
-        gen_codes(W.code_key(wl, layer, W.POOL_K, b), T, H * r, kspec, tk)
+        gen_codes(W.code_key(wl, layer, W.POOL_K, b), T, Hkv * r, kspec, tk)
         gen_codes(W.code_key(wl, layer, W.POOL_V, b), T, R, vspec, tv)
         rows = torch.from_numpy(slot_rows(tables[b], T)).to(device)
-        kflat.index_copy_(0, rows, tk[:T * H * r].view(T, H * r))
+        kflat.index_copy_(0, rows, tk[:T * Hkv * r].view(T, Hkv * r))
         vflat.index_copy_(0, rows, tv[:T * R].view(T, R))
     A_K, A_V, B_K, B_V = W.projections(wl, layer)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
     return dict(
-        H=H, d=d, r=r, R=R, nb=nb, tables_np=tables,
+        H=H, Hkv=Hkv, d=d, r=r, R=R, nb=nb, tables_np=tables,
         tables=dev(tables.astype(np.int32)),
         ctx_lens=dev(wl.ctx_lens.astype(np.int32)), seq_lens=dev(wl.seq_lens.astype(np.int32)),
         k_cache=k_cache, v_cache=v_cache,

@@ -27,10 +27,15 @@ POOL_K, POOL_V, ACT_Q, ACT_K, ACT_V = 0, 1, 2, 3, 4
 
 @dataclass
 class LayerShape:
-    num_heads: int
+    num_heads: int          # query heads
     head_dim: int
     k_rank: int
     v_rank: int
+    num_kv_heads: int = 0   # 0: as many KV heads as query heads
+
+    @property
+    def kv_heads(self) -> int:
+        return self.num_kv_heads or self.num_heads
 
 
 @dataclass
@@ -131,13 +136,13 @@ def layer_seed(wl: Workload, layer: int) -> int:
 
 
 def projections(wl: Workload, layer: int):
-    """fp16 projections of one layer: A_K [H][d][r], A_V [H*d][R], B_K [H][r][d], B_V [R][H*d].
+    """fp16 projections of one layer: A_K [Hkv][d][r], A_V [Hkv*d][R], B_K [Hkv][r][d], B_V [R][Hkv*d].
 
     A_K[h] and A_V are the orthonormal Q factors of seeded Gaussians, rounded
     to fp16; B is the transpose of the rounded A.
     """
     sh = wl.layers[layer]
-    H, d, r, R = sh.num_heads, sh.head_dim, sh.k_rank, sh.v_rank
+    H, d, r, R = sh.kv_heads, sh.head_dim, sh.k_rank, sh.v_rank
     s = layer_seed(wl, layer)
     A_K = np.stack([gen.orthonormal_f64(s * 131 + h, d, r) for h in range(H)]).astype(np.float16)
     A_V = gen.orthonormal_f64(s * 131 + 977, H * d, R).astype(np.float16)
@@ -147,11 +152,12 @@ def projections(wl: Workload, layer: int):
 
 
 def activation(wl: Workload, layer: int, which: int) -> np.ndarray:
-    """q, k or v of the step's new token: fp16 ~N(0,1), shape [B][H][d]."""
+    """q ([B][H][d], query heads) or k, v ([B][Hkv][d], KV heads) of the step's new token: fp16 ~N(0,1)."""
     sh = wl.layers[layer]
     key = gen.stream_key(wl.seed, layer, which)
-    n = sh.num_heads * sh.head_dim
-    return gen.codes_f16(key, wl.batch, n, None).reshape(wl.batch, sh.num_heads, sh.head_dim)
+    heads = sh.num_heads if which == ACT_Q else sh.kv_heads
+    n = heads * sh.head_dim
+    return gen.codes_f16(key, wl.batch, n, None).reshape(wl.batch, heads, sh.head_dim)
 
 
 def code_key(wl: Workload, layer: int, pool: int, b: int) -> int:
@@ -169,10 +175,10 @@ def v_spectrum(sh: LayerShape) -> np.ndarray:
 def seq_codes(wl: Workload, layer: int, b: int, n_tokens: int, t0: int = 0):
     """Logical codes of tokens ``t0 .. t0+n_tokens-1`` of sequence ``b``.
 
-    Returns ``(cK [n][H][r], cV [n][R])`` fp16.
+    Returns ``(cK [n][Hkv][r], cV [n][R])`` fp16.
     """
     sh = wl.layers[layer]
-    H, r, R = sh.num_heads, sh.k_rank, sh.v_rank
+    H, r, R = sh.kv_heads, sh.k_rank, sh.v_rank
     cK = gen.codes_f16(code_key(wl, layer, POOL_K, b), n_tokens, H * r, k_spectrum(sh),
                        row_offset=t0).reshape(n_tokens, H, r)
     cV = gen.codes_f16(code_key(wl, layer, POOL_V, b), n_tokens, R, v_spectrum(sh),
@@ -195,9 +201,10 @@ def host_layer(wl: Workload, layer: int, tables=None, nb=None):
     """
     sh = wl.layers[layer]
     H, d, r, R = sh.num_heads, sh.head_dim, sh.k_rank, sh.v_rank
+    Hkv = sh.kv_heads
     if tables is None:
         tables, nb, _ = block_tables(wl.seed, wl.seq_lens, wl.max_blocks_per_seq, wl.decoy_frac)
-    k_cache = np.full((nb, BLOCK_SIZE, H, r), np.nan, dtype=np.float16)
+    k_cache = np.full((nb, BLOCK_SIZE, Hkv, r), np.nan, dtype=np.float16)
     v_cache = np.full((nb, BLOCK_SIZE, R), np.nan, dtype=np.float16)
     for b in range(wl.batch):
         T = int(wl.ctx_lens[b])
@@ -206,7 +213,7 @@ def host_layer(wl: Workload, layer: int, tables=None, nb=None):
         place_host(v_cache, tables[b], cV)
     A_K, A_V, B_K, B_V = projections(wl, layer)
     return dict(
-        H=H, d=d, r=r, R=R, nb=nb, tables=tables,
+        H=H, Hkv=Hkv, d=d, r=r, R=R, nb=nb, tables=tables,
         ctx_lens=wl.ctx_lens.astype(np.int32), seq_lens=wl.seq_lens.astype(np.int32),
         k_cache=k_cache, v_cache=v_cache,
         q=activation(wl, layer, ACT_Q), k=activation(wl, layer, ACT_K),

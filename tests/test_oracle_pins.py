@@ -31,34 +31,41 @@ def _paged_fp64(codes_list, tables, nb, row_shape):
     return pool
 
 
-def _full_rank_case(seed=5, H=4, d=16, lens=(1, 19, 40)):
-    """Uncompressed K/V, orthogonal A (fp64), B = A^T, codes = k.A exactly."""
+def _full_rank_case(seed=5, H=4, d=16, lens=(1, 19, 40), Hkv=None):
+    """Uncompressed K/V, orthogonal A (fp64), B = A^T, codes = k.A exactly.
+
+    ``Hkv`` KV heads (default ``H``) carry K and V; q has ``H`` query heads.
+    """
+    Hkv = Hkv or H
     rng = np.random.default_rng(seed)
     Bsz = len(lens)
     q = rng.standard_normal((Bsz, H, d))
-    k_full = [rng.standard_normal((T, H, d)) for T in lens]
-    v_full = [rng.standard_normal((T, H, d)) for T in lens]
-    A_K = np.stack([_orth(rng, d) for _ in range(H)])
-    A_V = _orth(rng, H * d)
+    k_full = [rng.standard_normal((T, Hkv, d)) for T in lens]
+    v_full = [rng.standard_normal((T, Hkv, d)) for T in lens]
+    A_K = np.stack([_orth(rng, d) for _ in range(Hkv)])
+    A_V = _orth(rng, Hkv * d)
     B_K = np.transpose(A_K, (0, 2, 1)).copy()
     B_V = A_V.T.copy()
-    cK = [np.stack([k[:, h, :] @ A_K[h] for h in range(H)], axis=1) for k in k_full]
-    cV = [v.reshape(v.shape[0], H * d) @ A_V for v in v_full]
+    cK = [np.stack([k[:, h, :] @ A_K[h] for h in range(Hkv)], axis=1) for k in k_full]
+    cV = [v.reshape(v.shape[0], Hkv * d) @ A_V for v in v_full]
     tables, nb, _ = W.block_tables(seed, np.array(lens), max(1, -(-max(lens) // 16)) + 1)
-    kc = _paged_fp64(cK, tables, nb, (H, d))
-    vc = _paged_fp64(cV, tables, nb, (H * d,))
+    kc = _paged_fp64(cK, tables, nb, (Hkv, d))
+    vc = _paged_fp64(cV, tables, nb, (Hkv * d,))
     return dict(q=q, k_full=k_full, v_full=v_full, A_K=A_K, A_V=A_V, B_K=B_K, B_V=B_V,
                 cK=cK, cV=cV, tables=tables, kc=kc, vc=vc, lens=np.array(lens),
                 scale=1.0 / math.sqrt(d))
 
 
 def _sdpa(q, k_list, v_list, scale):
+    """torch fp64 scaled-dot-product attention; grouped query heads when K/V have fewer heads."""
     out = []
     for b in range(q.shape[0]):
         qt = torch.from_numpy(q[b][:, None, :])                     # [H][1][d]
-        kt = torch.from_numpy(np.transpose(k_list[b], (1, 0, 2)).copy())  # [H][T][d]
+        kt = torch.from_numpy(np.transpose(k_list[b], (1, 0, 2)).copy())  # [Hkv][T][d]
         vt = torch.from_numpy(np.transpose(v_list[b], (1, 0, 2)).copy())
-        o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=scale)
+        gqa = kt.shape[0] != qt.shape[0]
+        o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=scale,
+                                                             enable_gqa=gqa)
         out.append(o[:, 0, :].numpy())
     return np.stack(out)
 
@@ -75,6 +82,42 @@ def check_full_rank(decode=None):
 
 def test_full_rank_orthonormal_equals_library_attention():
     check_full_rank()
+
+
+def check_full_rank_gqa(decode=None):
+    """Grouped queries: 8 query heads over 2 KV heads, against torch's own GQA attention."""
+    c = _full_rank_case(seed=6, H=8, Hkv=2, lens=(1, 17, 33))
+    decode = decode or O.decode_explicit
+    got = decode(c["q"], c["B_K"], c["B_V"], c["kc"], c["vc"], c["tables"], c["lens"], c["scale"])
+    ref = _sdpa(c["q"], c["k_full"], c["v_full"], c["scale"])
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_full_rank_grouped_query_equals_library_attention():
+    check_full_rank_gqa()
+    check_full_rank_gqa(O.decode_reordered)
+
+
+def test_grouped_query_equals_mha_with_repeated_kv_heads():
+    """Hkv KV heads shared by groups of H/Hkv query heads == MHA on repeated KV heads."""
+    H, Hkv = 8, 2
+    G = H // Hkv
+    sh = W.LayerShape(H, 32, 16, 64, num_kv_heads=Hkv)
+    wl = W.custom("gqa", 91, sh, [1, 16, 45], append=False)
+    L = W.host_layer(wl, 0)
+    d = L["d"]
+    B_K_rep = np.repeat(L["B_K"], G, axis=0)                   # [H][r][d]
+    kc_rep = np.repeat(L["k_cache"], G, axis=2)                # [NB][16][H][r]
+    B_V_rep = np.concatenate([L["B_V"][:, (h // G) * d:(h // G + 1) * d] for h in range(H)],
+                             axis=1)                            # [R][H*d]
+    got = O.decode_explicit(L["q"], L["B_K"], L["B_V"], L["k_cache"], L["v_cache"], L["tables"],
+                            L["seq_lens"], L["scale"])
+    want = O.decode_explicit(L["q"], B_K_rep, B_V_rep, kc_rep, L["v_cache"], L["tables"],
+                             L["seq_lens"], L["scale"])
+    np.testing.assert_array_equal(got, want)
+    np.testing.assert_allclose(
+        O.decode_reordered(L["q"], L["B_K"], L["B_V"], L["k_cache"], L["v_cache"], L["tables"],
+                           L["seq_lens"], L["scale"]), want, rtol=0, atol=1e-12 * np.abs(want).max())
 
 
 def test_uncompressed_attention_matches_library():
@@ -377,6 +420,13 @@ def _mut_slot_shift(cache, table_row, T):
 def test_planted_decode_mistakes_are_caught(mutant, pin):
     with pytest.raises(AssertionError):
         pin(mutant)
+
+
+def test_planted_interleaved_kv_heads_are_caught(monkeypatch):
+    """Query head h reading KV head h % Hkv (interleaved groups) instead of h // G."""
+    monkeypatch.setattr(O, "kv_head", lambda h, H, Hkv: h % Hkv)
+    with pytest.raises(AssertionError):
+        check_full_rank_gqa()
 
 
 def test_planted_slot_mistake_is_caught(monkeypatch):
