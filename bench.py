@@ -40,6 +40,8 @@ WORKLOAD_NAMES = {
        "K rank {32,64,96}, V rank 32r, fp16, block_size 16",
     5: "Llama-2-7B attention path: 32 layers, 32 heads, head_size 128, batch 8, context 32768, "
        "K rank 64/head, V rank 2048, fp16, block_size 16",
+    6: "grouped-query layer: 32 query heads over 8 KV heads, head_size 128, K rank 64/KV head, "
+       "V joint rank 512, fp16, block_size 16, batch 64, seq_len 8192",
 }
 
 
@@ -48,7 +50,7 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", type=int, default=3, choices=[2, 3, 4, 5])
+    ap.add_argument("--workload", type=int, default=3, choices=[2, 3, 4, 5, 6])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--profile-steps", type=int, default=300,
@@ -85,7 +87,7 @@ NCU_TRAFFIC_PER_TOKEN = {
     "kpass": (1.074168e9 + 6.671104e6) / (32 * 8192),
     "vpass": (1.107514e9 + 5.822976e6) / (32 * 8192),
 }
-NCU_TRAFFIC_GEOMETRY = (32, 64, 2048)   # (heads, K rank, V rank)
+NCU_TRAFFIC_GEOMETRY = (32, 32, 64, 2048)   # (query heads, KV heads, K rank, V rank)
 
 
 def measured_peaks():
@@ -182,7 +184,8 @@ def run_ours(args):
     layers = []
     for li in range(len(wl.layers)):
         Ld = D.device_layer(wl, li)
-        Ld["desc"] = S.layer_desc(Ld["H"], Ld["d"], Ld["r"], Ld["R"], Ld["nb"], Ld["tables"].shape[1])
+        Ld["desc"] = S.layer_desc(Ld["H"], Ld["d"], Ld["r"], Ld["R"], Ld["nb"], Ld["tables"].shape[1],
+                                  num_kv_heads=Ld["Hkv"])
         layers.append(Ld)
     B = wl.batch
     max_len = wl.max_seq_len
@@ -273,11 +276,11 @@ def run_ours(args):
 
     # ---------------- algorithmic bytes
     T_sum = int(wl.seq_lens.sum())
-    k_bytes = sum(T_sum * L["H"] * L["r"] * 2 for L in layers)
+    k_bytes = sum(T_sum * L["Hkv"] * L["r"] * 2 for L in layers)
     v_bytes = sum(T_sum * L["R"] * 2 for L in layers)
     proj_bytes = sum(L["B_K"].numel() * 2 + L["B_V"].numel() * 2 + L["A_K"].numel() * 2 + L["A_V"].numel() * 2
                      for L in layers)
-    act_bytes = sum(B * L["H"] * L["d"] * 2 * 4 for L in layers)   # q, k, v in; out
+    act_bytes = sum(B * (L["H"] + L["Hkv"]) * L["d"] * 2 * 2 for L in layers)   # q, out; k, v
     step_bytes = k_bytes + v_bytes + proj_bytes + act_bytes
     peak, peak_kind = measured_peaks()
     kp_gbs = k_bytes / (per["kpass"] * 1e-3) / 1e9
@@ -285,7 +288,7 @@ def run_ours(args):
     dom = "kpass" if per["kpass"] >= per["vpass"] else "vpass"
     dom_bytes, dom_gbs = (k_bytes, kp_gbs) if dom == "kpass" else (v_bytes, vp_gbs)
     traffic = None
-    if len(layers) == 1 and (layers[0]["H"], layers[0]["r"], layers[0]["R"]) == NCU_TRAFFIC_GEOMETRY:
+    if len(layers) == 1 and (layers[0]["H"], layers[0]["Hkv"], layers[0]["r"], layers[0]["R"]) == NCU_TRAFFIC_GEOMETRY:
         traffic = round(NCU_TRAFFIC_PER_TOKEN[dom] * T_sum)
 
     # ---------------- end to end through the public API with host buffers
@@ -374,7 +377,7 @@ def prepare_seq(wl, b, layer, proj_cache):
     cK, cV = W.seq_codes(wl, layer, b, ctx)
     n_pages = -(-T // 16)
     row = np.random.default_rng(b).permutation(n_pages).astype(np.int32)
-    kc = np.full((n_pages, 16, sh.num_heads, sh.k_rank), np.nan, np.float16)
+    kc = np.full((n_pages, 16, sh.kv_heads, sh.k_rank), np.nan, np.float16)
     vc = np.full((n_pages, 16, sh.v_rank), np.nan, np.float16)
     W.place_host(kc, row, cK)
     W.place_host(vc, row, cV)

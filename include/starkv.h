@@ -12,13 +12,14 @@
  *   paged decode        : single-query attention computed straight from the
  *                         codes, never materialising full keys or values.
  *
- * Formulation (head_dim d, H heads, K rank r per head, V joint rank R):
- *   c_K[h] = k_h . A_K[h]         A_K[h] : d x r        (head-wise K)
- *   c_V    = v . A_V              A_V    : (H*d) x R    (joint V, v = concat_h v_h)
- *   q~_h   = scale * q_h . B_K[h]^T,  B_K[h] : r x d    (query absorbed into K codes)
- *   s[h,t] = q~_h . c_K[t,h]
+ * Formulation (head_dim d, H query heads, Hkv KV heads with query head h
+ * reading KV head g(h) = h / (H/Hkv), K rank r per KV head, V joint rank R):
+ *   c_K[j] = k_j . A_K[j]         A_K[j] : d x r          (head-wise K, j < Hkv)
+ *   c_V    = v . A_V              A_V    : (Hkv*d) x R    (joint V, v = concat_j v_j)
+ *   q~_h   = scale * q_h . B_K[g(h)]^T,  B_K[j] : r x d   (query absorbed into K codes)
+ *   s[h,t] = q~_h . c_K[t,g(h)]
  *   p[h,:] = softmax_t(s[h,:])
- *   out_h  = (sum_t p[h,t] c_V[t]) . B_V[:, h*d:(h+1)*d],  B_V : R x (H*d)
+ *   out_h  = (sum_t p[h,t] c_V[t]) . B_V[:, g(h)*d:(g(h)+1)*d],  B_V : R x (Hkv*d)
  * which equals softmax attention over the decompressed keys k^_h = c_K[h].B_K[h]
  * and values v^ = c_V.B_V.
  *
@@ -26,8 +27,10 @@
  * paragraph: block size 16); token t of sequence b is in slot t % 16 of
  * physical page block_tables[b][t / 16] (PagedAttention block-level
  * management, botdigit.com explainer, "How Dynamic KV-Cache Compaction Works").
- * Layouts (row-major, fp16): K pool [num_blocks][16][H][r];
+ * Layouts (row-major, fp16): K pool [num_blocks][16][Hkv][r];
  *                            V pool [num_blocks][16][R].
+ * With Hkv = H this is multi-head attention; the pages' benchmark (32-head MHA)
+ * is that case.
  *
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
@@ -71,13 +74,16 @@ typedef enum {
 
 /* One layer's cache geometry.  Ranks may differ from layer to layer. */
 typedef struct {
-  int32_t num_heads;          /* H: 1..64, power of two (query and KV heads; MHA) */
+  int32_t num_heads;          /* H: query heads, 1..64, power of two */
   int32_t head_dim;           /* d: 32, 64, 128 or 256 */
   int32_t k_rank;             /* r: multiple of 16, 16..256 */
   int32_t v_rank;             /* R: multiple of 64, 64..8192 */
   int32_t block_size;         /* must be 16 */
   int32_t num_blocks;         /* pages in each pool */
   int32_t max_blocks_per_seq; /* row length of block_tables */
+  int32_t num_kv_heads;       /* Hkv: KV heads (grouped-query attention), a power of two
+                                 dividing H; 0 means Hkv = H (multi-head attention).
+                                 Query head h uses KV head h / (H / Hkv). */
 } starkv_layer_desc;
 
 /*
@@ -88,12 +94,12 @@ typedef struct {
  * slot positions[b] % 16 of page block_tables[b][positions[b] / 16] of the K
  * and V pools.  Nothing else in the pools is written.
  *
- *   k, v          fp16 [batch][H][d]  (v read as the concatenation [batch][H*d])
- *   A_K           fp16 [H][d][r]
- *   A_V           fp16 [H*d][R]
+ *   k, v          fp16 [batch][Hkv][d]  (v read as the concatenation [batch][Hkv*d])
+ *   A_K           fp16 [Hkv][d][r]
+ *   A_V           fp16 [Hkv*d][R]
  *   block_tables  int32 [batch][max_blocks_per_seq]
  *   positions     int32 [batch]: the sequence length BEFORE this append
- *   k_cache       fp16 [num_blocks][16][H][r]   (in/out)
+ *   k_cache       fp16 [num_blocks][16][Hkv][r]   (in/out)
  *   v_cache       fp16 [num_blocks][16][R]      (in/out)
  *
  * Targets must be distinct slots (no page shared between sequences).  A target
@@ -111,7 +117,7 @@ starkv_status starkv_compress_append(const starkv_layer_desc* desc, int32_t batc
  * slot_mapping[i] = page * 16 + offset, int32 [n_tokens].  Same arithmetic,
  * layouts and rounding as starkv_compress_append; rows whose slot is outside
  * [0, num_blocks*16) are skipped; targets must be distinct.  k, v fp16
- * [n_tokens][H][d].  Cites: README method paragraph (codes "stored in a
+ * [n_tokens][Hkv][d].  Cites: README method paragraph (codes "stored in a
  * compressed paged format"); the flat slot is the paged address
  * block_table[b][t/16]*16 + t%16 precomputed by the caller.
  */
@@ -132,9 +138,9 @@ size_t starkv_decode_workspace_bytes(const starkv_layer_desc* desc, int32_t batc
  * starkv_paged_decode -- single-token decode attention from the paged codes.
  *
  *   q             fp16 [batch][H][d]
- *   B_K           fp16 [H][r][d]
- *   B_V           fp16 [R][H*d]
- *   k_cache       fp16 [num_blocks][16][H][r]
+ *   B_K           fp16 [Hkv][r][d]
+ *   B_V           fp16 [R][Hkv*d]
+ *   k_cache       fp16 [num_blocks][16][Hkv][r]
  *   v_cache       fp16 [num_blocks][16][R]
  *   block_tables  int32 [batch][max_blocks_per_seq]
  *   seq_lens      int32 [batch]: tokens to attend over (after any append)
@@ -230,6 +236,9 @@ typedef struct {
   int32_t v_slots;    /* v_ctas + batch */
   int32_t n_rranges;  /* R ranges of the V pass */
   int32_t r_range;    /* V rank handled per R range */
+  int32_t k_tensor;   /* 1: the K pass runs on tensor cores (grouped queries), 0: CUDA cores */
+  size_t qth_off;     /* fp16 [batch][2H][r]: q~ in fp16 (rows h) and its remainder (rows H+h);
+                         used by the tensor-core K pass only (0 otherwise) */
 } starkv_workspace_layout;
 
 starkv_status starkv_decode_workspace_layout(const starkv_layer_desc* desc, int32_t batch,
@@ -249,13 +258,15 @@ int32_t starkv_rank_from_spectrum(const double* s, int32_t n, double tau);
 
 /*
  * Capacity arithmetic (host functions, no GPU).  A token costs, in every layer,
- * H*r fp16 K codes plus R fp16 V codes; a full-rank cache is the case r = d,
- * R = H*d (2*2*H*d bytes per layer).  The README's boot log for the
+ * Hkv*r fp16 K codes plus R fp16 V codes (Hkv = the layer's KV heads, equal to
+ * its query heads without grouping); a full-rank cache is the case r = d,
+ * R = Hkv*d (2*2*Hkv*d bytes per layer).  The README's boot log for the
  * uncompressed 7B cache is the worked example: 6.99 GiB of KV memory, 16-token
  * blocks, 32 layers x 512 KiB -> 894 blocks = 14,304 tokens ("Low-rank KV
  * Cache Compression for vLLM", measured results at 8192 context).
  *
- * starkv_kv_bytes_per_token: 2 * sum_l (num_heads[l]*k_ranks[l] + v_ranks[l]);
+ * starkv_kv_bytes_per_token: 2 * sum_l (num_heads[l]*k_ranks[l] + v_ranks[l]),
+ *   num_heads[l] being layer l's KV heads;
  *   HOST arrays of n_layers entries; -1 on invalid input (n_layers <= 0, null
  *   array, non-positive entry).
  * starkv_num_blocks: floor(budget_bytes / (block_size * bytes_per_token));

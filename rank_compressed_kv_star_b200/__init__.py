@@ -42,7 +42,7 @@ class LayerDesc(ctypes.Structure):
     _fields_ = [("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("k_rank", ctypes.c_int32), ("v_rank", ctypes.c_int32),
                 ("block_size", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
-                ("max_blocks_per_seq", ctypes.c_int32)]
+                ("max_blocks_per_seq", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32)]
 
 
 class WorkspaceLayout(ctypes.Structure):
@@ -54,13 +54,15 @@ class WorkspaceLayout(ctypes.Structure):
                 ("zlo_off", ctypes.c_size_t),
                 ("t_pad", ctypes.c_int32), ("k_ctas", ctypes.c_int32), ("k_slots", ctypes.c_int32),
                 ("v_ctas", ctypes.c_int32), ("v_slots", ctypes.c_int32),
-                ("n_rranges", ctypes.c_int32), ("r_range", ctypes.c_int32)]
+                ("n_rranges", ctypes.c_int32), ("r_range", ctypes.c_int32),
+                ("k_tensor", ctypes.c_int32), ("qth_off", ctypes.c_size_t)]
 
 
 def layer_desc(num_heads, head_dim, k_rank, v_rank, num_blocks, max_blocks_per_seq,
-               block_size=16) -> LayerDesc:
+               block_size=16, num_kv_heads=0) -> LayerDesc:
+    """``num_kv_heads`` 0 means multi-head attention (as many KV heads as query heads)."""
     return LayerDesc(num_heads, head_dim, k_rank, v_rank, block_size, num_blocks,
-                     max_blocks_per_seq)
+                     max_blocks_per_seq, num_kv_heads)
 
 
 _lib = None

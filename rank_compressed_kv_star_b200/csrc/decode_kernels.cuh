@@ -78,10 +78,12 @@ struct AbsorbParams {
   const __half* B_K;      // [H][r][d]
   const int32_t* seq_lens;
   float* qt;              // [B][H][r]
+  __half* qth;            // [B][2H][r]: fp16 q~ (row h) and fp16 of its remainder (row H+h); may be null
   int32_t* prefix;        // [B+1]
   int32_t* teff;          // [B] clamped lengths
   int32_t* status;
   int B, H, d, r, cap;    // cap = min(max_seq_len, max_blocks_per_seq*16)
+  int log2G;              // query heads per KV head = 1 << log2G
   float coef;             // scale * log2(e)
 };
 
@@ -142,7 +144,7 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbParams p) {
   const int bs = tid / p.r;
   if (bs >= bpar) return;
   uint4 brow[D / 8];
-  const uint4* bsrc = reinterpret_cast<const uint4*>(p.B_K + (static_cast<size_t>(h) * p.r + i) * D);
+  const uint4* bsrc = reinterpret_cast<const uint4*>(p.B_K + (static_cast<size_t>(h >> p.log2G) * p.r + i) * D);
 #pragma unroll
   for (int c = 0; c < D / 8; ++c) brow[c] = bsrc[c];
   for (int bb = bs; bb < nb; bb += bpar) {
@@ -161,7 +163,14 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbParams p) {
         a1 = fmaf(qf.y, bf.y, a1);
       }
     }
-    p.qt[(static_cast<size_t>(bt0 + bb) * p.H + h) * p.r + i] = (a0 + a1) * p.coef;
+    const float v = (a0 + a1) * p.coef;
+    p.qt[(static_cast<size_t>(bt0 + bb) * p.H + h) * p.r + i] = v;
+    if (p.qth) {
+      const __half hi = __float2half_rn(v);
+      __half* row = p.qth + (static_cast<size_t>(bt0 + bb) * 2 * p.H + h) * p.r + i;
+      row[0] = hi;
+      row[static_cast<size_t>(p.H) * p.r] = __float2half_rn(v - __half2float(hi));
+    }
   }
 }
 
@@ -176,9 +185,10 @@ struct KPassParams {
   float* mpart;               // [k_slots][H]: max of the base-2 logits per segment
   int32_t* status;
   int B, H, log2H, r, MB, NB, t_pad;
-  int tps;                    // tokens per ring stage
+  int Hkv, log2G;             // KV heads (codes per token) and log2(query heads per KV head)
+  int tps;                    // tokens per ring stage (> 16: whole pages of one sequence)
   int stages;
-  uint32_t stage_bytes;       // tps*H*r*2
+  uint32_t stage_bytes;       // tps*Hkv*r*2
 };
 
 constexpr int kKConsumers = 256;            // 8 warps of dot products
@@ -245,29 +255,61 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
     // ------------------------------------------------------------ producer
     if (lane != 0) return;
     const uint64_t pol = policy_evict_first();
-    const uint32_t tok_bytes = static_cast<uint32_t>(p.H) * p.r * 2;
+    const uint32_t tok_bytes = static_cast<uint32_t>(p.Hkv) * p.r * 2;
     uint32_t k = 0;
     bool ok = true;
     if (has_work) {
       const int64_t p0 = part_begin(cta, pt), p1 = part_begin(cta + 1, pt);
       int32_t b = seq_of_page(p.prefix, p.B, p0);
-      for (int64_t pg_g = p0; pg_g < p1 && ok; ++pg_g) {
-        while (p.prefix[b + 1] <= pg_g) ++b;
-        const int32_t pg = static_cast<int32_t>(pg_g - p.prefix[b]);
-        const int32_t T = p.teff[b];
-        int32_t phys = p.tables[static_cast<size_t>(b) * p.MB + pg];
-        if (phys < 0 || phys >= p.NB) { set_flag(p.status, STARKV_FLAG_BAD_BLOCK_ID); phys = 0; }
-        const int32_t tend = min(pg * kBlock + kBlock, T);
-        for (int32_t t0 = pg * kBlock; t0 < tend; t0 += p.tps, ++k) {
+      const size_t page_elems = static_cast<size_t>(kBlock) * p.Hkv * p.r;
+      if (p.tps <= kBlock) {
+        // a page is split over several stages
+        for (int64_t pg_g = p0; pg_g < p1 && ok; ++pg_g) {
+          while (p.prefix[b + 1] <= pg_g) ++b;
+          const int32_t pg = static_cast<int32_t>(pg_g - p.prefix[b]);
+          const int32_t T = p.teff[b];
+          int32_t phys = p.tables[static_cast<size_t>(b) * p.MB + pg];
+          if (phys < 0 || phys >= p.NB) { set_flag(p.status, STARKV_FLAG_BAD_BLOCK_ID); phys = 0; }
+          const int32_t tend = min(pg * kBlock + kBlock, T);
+          for (int32_t t0 = pg * kBlock; t0 < tend; t0 += p.tps, ++k) {
+            const int s = k % S;
+            if (k >= static_cast<uint32_t>(S) && !mbar_wait(&empty[s], ((k / S) - 1) & 1)) { ok = false; break; }
+            const int32_t nt = min(p.tps, tend - t0);
+            meta[s] = StageMeta{b, t0, nt, 0};
+            const uint32_t bytes = static_cast<uint32_t>(nt) * tok_bytes;
+            mbar_arrive_expect_tx(&full[s], bytes);
+            const __half* src = p.k_cache + static_cast<size_t>(phys) * page_elems +
+                                static_cast<size_t>(t0 - pg * kBlock) * p.Hkv * p.r;
+            bulk_g2s(ring + static_cast<size_t>(s) * p.stage_bytes, src, bytes, &full[s], pol);
+          }
+        }
+      } else {
+        // a stage gathers up to tps/16 consecutive pages of one sequence, one
+        // bulk copy per page, placed back to back (token-major, as in a page)
+        const int pps = p.tps / kBlock;
+        int64_t pg_g = p0;
+        while (pg_g < p1 && ok) {
+          while (p.prefix[b + 1] <= pg_g) ++b;
+          const int32_t pg = static_cast<int32_t>(pg_g - p.prefix[b]);
+          const int32_t T = p.teff[b];
+          const int64_t stop = min(p1, static_cast<int64_t>(p.prefix[b + 1]));
+          const int n_pg = static_cast<int>(min(static_cast<int64_t>(pps), stop - pg_g));
+          const int32_t t0 = pg * kBlock;
+          const int32_t nt = min(n_pg * kBlock, T - t0);
           const int s = k % S;
           if (k >= static_cast<uint32_t>(S) && !mbar_wait(&empty[s], ((k / S) - 1) & 1)) { ok = false; break; }
-          const int32_t nt = min(p.tps, tend - t0);
           meta[s] = StageMeta{b, t0, nt, 0};
-          const uint32_t bytes = static_cast<uint32_t>(nt) * tok_bytes;
-          mbar_arrive_expect_tx(&full[s], bytes);
-          const __half* src = p.k_cache + (static_cast<size_t>(phys) * kBlock + (t0 - pg * kBlock)) *
-                                              static_cast<size_t>(p.H) * p.r;
-          bulk_g2s(ring + static_cast<size_t>(s) * p.stage_bytes, src, bytes, &full[s], pol);
+          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nt) * tok_bytes);
+          for (int i = 0; i < n_pg; ++i) {
+            int32_t phys = p.tables[static_cast<size_t>(b) * p.MB + pg + i];
+            if (phys < 0 || phys >= p.NB) { set_flag(p.status, STARKV_FLAG_BAD_BLOCK_ID); phys = 0; }
+            const int32_t ti = min(kBlock, nt - i * kBlock);
+            bulk_g2s(ring + static_cast<size_t>(s) * p.stage_bytes + static_cast<size_t>(i) * kBlock * tok_bytes,
+                     p.k_cache + static_cast<size_t>(phys) * page_elems, static_cast<uint32_t>(ti) * tok_bytes,
+                     &full[s], pol);
+          }
+          ++k;
+          pg_g += n_pg;
         }
       }
     }
@@ -339,7 +381,8 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
       const bool valid = t < mt.nt;
       float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
       if (valid) {
-        const uint8_t* row = st + static_cast<size_t>(pair) * p.r * 2;
+        // code row (token t, KV head of this query head); rows are r*2 bytes
+        const uint8_t* row = st + static_cast<size_t>((t << (p.log2H - p.log2G)) + (head >> p.log2G)) * p.r * 2;
 #pragma unroll
         for (int c = 0; c < CPT; ++c) {
           const int cc = c + rot < CPT ? c + rot : c + rot - CPT;
@@ -365,6 +408,294 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
+  }
+}
+
+// ============================================================== kpass (tensor)
+// Grouped-query K pass on tcgen05.  With G = H/Hkv query heads per KV head the
+// logits of a run of tokens are a small GEMM, S[(j,t), h] = c_K[t, j] . q~_h.
+// A tile is 128 code rows: tpt = 128/Hkv tokens of one sequence times the Hkv
+// KV heads, head-major (row j*tpt + t), loaded by TMA as 3-D boxes
+// {64 codes, 1 head, min(16, tpt) tokens} with the 128-byte swizzle, which is
+// the K-major operand layout.  B holds the sequence's absorbed queries for all
+// H heads split into an fp16 high part (row h) and the fp16 rounding of the
+// remainder (row H+h), so D[row, h] + D[row, H+h] is c_K . q~_h with q~ carried
+// to about 22 bits and fp32 accumulation.  A row uses only the G columns of its
+// own KV head; the tensor cores compute all 2H, which at G >= 2 still costs
+// less than the HBM time of the tile.  The epilogue (4 warps, one TMEM lane
+// quarter each) adds hi + lo, stores each row's G logits as one contiguous
+// vector and keeps the row's running maxima, merged per (sequence, CTA)
+// segment in shared memory.  Several accumulators let the tensor cores run
+// ahead of the epilogue.
+struct KPassTCParams {
+  const int32_t* tables;      // [B][MB]
+  const int32_t* teff;        // [B]
+  const int32_t* prefix;      // [B+1]
+  float* logits;              // [B][t_pad][H]
+  float* mpart;               // [k_slots][H]
+  int32_t* status;
+  int B, H, log2G, log2Hkv, MB, NB, t_pad;
+  int log2tpt;                // tokens per tile = 128 / Hkv
+  int ksteps;                 // UMMA K steps of 16 codes: ceil(r/16)
+  int kb;                     // 64-code column blocks: ceil(r/64)
+  int npad;                   // UMMA N = max(16, 2H)
+  int acc_cols;               // TMEM columns per accumulator (npad + 16 of slack for the epilogue reads)
+  int nacc;                   // accumulators in TMEM (2..4)
+  int ncol;                   // query-head columns of one lane quarter: max(G, H/4)
+  int stages;
+  uint32_t a_bytes;           // kb * 128 rows * 128 bytes
+  uint32_t b_bytes;           // kb * npad * 128 bytes
+  uint32_t tmem_cols;
+};
+
+constexpr int kKTCThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kKTCSegBufs = 6;     // segment-maximum buffers (warps run at most nacc <= 4 tiles apart)
+
+// Calls f(b, t0, nt, last) for the K-pass tiles of pages [p0, p1) in order:
+// tokens [t0, t0+nt) of sequence b, `last` on the final tile of the
+// (sequence, CTA) segment.  Stops when f returns false.
+template <typename F>
+__device__ __forceinline__ void for_each_k_tile(const KPassTCParams& p, int64_t p0, int64_t p1, F&& f) {
+  const int tpt = 1 << p.log2tpt;
+  int32_t b = seq_of_page(p.prefix, p.B, p0);
+  int64_t x = p0;
+  while (x < p1) {
+    while (p.prefix[b + 1] <= x) ++b;
+    const int64_t seg_end = min(p1, static_cast<int64_t>(p.prefix[b + 1]));
+    const int32_t base = p.prefix[b];
+    const int32_t ts = static_cast<int32_t>(x - base) * kBlock;
+    const int32_t te = min(static_cast<int32_t>(seg_end - base) * kBlock, p.teff[b]);
+    for (int32_t t0 = ts; t0 < te; t0 += tpt)
+      if (!f(b, t0, min(tpt, te - t0), t0 + tpt >= te)) return;
+    x = seg_end;
+  }
+}
+
+// Float maximum into shared memory through the integer atomics (ordered bit
+// patterns: max over signed ints for v >= 0, min over unsigned for v < 0).
+__device__ __forceinline__ void smem_atomic_max_f32(float* addr, float v) {
+  if (__float_as_int(v) >= 0) atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));
+  else atomicMin(reinterpret_cast<unsigned int*>(addr), __float_as_uint(v));
+}
+
+template <int G>   // query heads per KV head
+__global__ void __launch_bounds__(kKTCThreads, 1)
+kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                KPassTCParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages;
+  const uint32_t stage_bytes = p.a_bytes + p.b_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * stage_bytes);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;     // [4] accumulator ready
+  uint64_t* tempty = tfull + 4;    // [4] accumulator drained (4 epilogue warps)
+  uint64_t* mmadone = tempty + 4;
+  float* segmax = reinterpret_cast<float*>(mmadone + 1);          // [kKTCSegBufs][H]
+  int32_t* segcnt = reinterpret_cast<int32_t*>(segmax + kKTCSegBufs * p.H);
+  __shared__ uint32_t taddr_s;
+  __shared__ volatile int32_t abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 4; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
+    mbar_init(mmadone, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int i = tid; i < kKTCSegBufs * p.H; i += kKTCThreads) segmax[i] = -INFINITY;
+  if (tid < kKTCSegBufs) segcnt[tid] = 0;
+  griddep_wait();
+  griddep_launch_dependents();
+  Partition pt;
+  pt.P = p.prefix[p.B];
+  pt.G = static_cast<int32_t>(pt.P < gridDim.x ? pt.P : gridDim.x);
+  const int cta = blockIdx.x;
+  if (cta >= pt.G) return;   // uniform over the CTA
+  if (warp == 1) {
+    tmem_alloc(&taddr_s, p.tmem_cols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t taddr = taddr_s;
+  const int64_t p0 = part_begin(cta, pt), p1 = part_begin(cta + 1, pt);
+  const int tpt = 1 << p.log2tpt;
+  const int tb = tpt < kBlock ? tpt : kBlock;       // tokens per TMA box
+  const int Hkv = 1 << p.log2Hkv;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&kmap);
+      prefetch_tensormap(&qmap);
+      const uint64_t stream = policy_evict_first();
+      const uint64_t reuse = policy_evict_last();   // q~ tiles: read again for every tile
+      const uint32_t box_bytes = static_cast<uint32_t>(tb) * 128u;
+      uint32_t k = 0;
+      bool ok = true;
+      for_each_k_tile(p, p0, p1, [&](int32_t b, int32_t t0, int32_t nt, bool) {
+        const int s = k % S;
+        if (k >= static_cast<uint32_t>(S) && !mbar_wait(&empty[s], ((k / S) - 1) & 1)) { ok = false; return false; }
+        uint8_t* st = smem + static_cast<size_t>(s) * stage_bytes;
+        const int nbox = (nt + tb - 1) / tb;
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox * Hkv * p.kb) * box_bytes + p.b_bytes);
+        for (int c = 0; c < nbox; ++c) {
+          const int32_t t = t0 + c * tb;
+          int32_t phys = p.tables[static_cast<size_t>(b) * p.MB + (t >> 4)];
+          if (phys < 0 || phys >= p.NB) { set_flag(p.status, STARKV_FLAG_BAD_BLOCK_ID); phys = 0; }
+          const int32_t row = phys * kBlock + (t & (kBlock - 1));
+          for (int j = 0; j < Hkv; ++j)
+            for (int a = 0; a < p.kb; ++a)
+              tma_load_3d(st + static_cast<size_t>(a) * 16384 + static_cast<size_t>((j << p.log2tpt) + c * tb) * 128,
+                          &kmap, a * 64, j, row, &full[s], stream);
+        }
+        for (int a = 0; a < p.kb; ++a)
+          tma_load_2d(st + p.a_bytes + static_cast<size_t>(a) * p.npad * 128, &qmap, a * 64, b * 2 * p.H,
+                      &full[s], reuse);
+        ++k;
+        return true;
+      });
+      if (!ok) {
+        set_timeout(p.status, kSiteKEmpty);
+        abort_flag = 1;
+        const uint32_t first = k > static_cast<uint32_t>(S) ? k - S : 0;
+        for (uint32_t kk = first; kk < k; ++kk) mbar_wait(&full[kk % S], (kk / S) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16_f32(128, p.npad, /*a_mn_major=*/false, /*b_mn_major=*/false);
+      uint32_t k = 0;
+      bool ok = true;
+      for_each_k_tile(p, p0, p1, [&](int32_t, int32_t, int32_t, bool) {
+        const int s = k % S;
+        const uint32_t acc = k % p.nacc, use = k / p.nacc;
+        if (use > 0 && !mbar_wait(&tempty[acc], (use - 1) & 1)) { ok = false; return false; }
+        if (!mbar_wait(&full[s], (k / S) & 1) || abort_flag) { ok = false; return false; }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
+        const uint32_t sb = sa + p.a_bytes;
+        const uint32_t d = taddr + static_cast<uint32_t>(acc * p.acc_cols);
+        for (int ks = 0; ks < p.ksteps; ++ks) {
+          const uint32_t a = ks >> 2, kk = ks & 3;
+          umma_f16_ss(d, smem_desc(sa + a * 16384u + kk * 32u, 16u, 1024u, kSwizzle128B),
+                      smem_desc(sb + a * static_cast<uint32_t>(p.npad) * 128u + kk * 32u, 16u, 1024u, kSwizzle128B),
+                      idesc, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
+        umma_commit(&tfull[acc]);
+        ++k;
+        return true;
+      });
+      if (!ok) { set_timeout(p.status, kSiteKFull); abort_flag = 1; }
+      umma_commit(mmadone);
+      mbar_wait(mmadone, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // Columns [col0, col0 + ncol) of a lane quarter are the query heads of its
+    // KV heads; the lane owns the G of them at offset jl*G.
+    constexpr int NCH = G >= 16 ? G / 16 : 1;        // 16-column chunks read per tile
+    constexpr int HQ = G >= 16 ? 1 : 16 / G;         // KV heads a 16-column chunk spans
+    const int q = warp & 3;                          // TMEM lane quarter of this warp
+    const int rho = q * 32 + lane;                   // tile row
+    const int jq = (q * 32) >> p.log2tpt;            // first KV head of the quarter
+    const int jl = (rho >> p.log2tpt) - jq;          // this row's KV head, relative to jq
+    const int tl = rho & (tpt - 1);                  // token of this row within the tile
+    const int col0 = jq * G;                         // first query head of the quarter
+    const uint64_t keep = policy_evict_last();       // logits: read back by the V pass
+    float m[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) m[g] = -INFINITY;
+    uint32_t k = 0, seg = 0;
+    bool ok = true;
+    for_each_k_tile(p, p0, p1, [&](int32_t b, int32_t t0, int32_t nt, bool last) {
+      const uint32_t acc = k % p.nacc, use = k / p.nacc;
+      if (!mbar_wait(&tfull[acc], use & 1) || abort_flag) { ok = false; return false; }
+      tc_fence_after();
+      const bool valid = tl < nt;
+      float* lrow = p.logits + (static_cast<size_t>(b) * p.t_pad + t0 + tl) * p.H + col0 + jl * G;
+      const uint32_t tbase = taddr + (static_cast<uint32_t>(q * 32) << 16) + acc * p.acc_cols + col0;
+#pragma unroll
+      for (int ch = 0; ch < NCH; ++ch) {
+        uint32_t hi[32], lo[32];
+        tmem_ld_32x32b_x16(tbase + ch * 16, hi);
+        tmem_ld_32x32b_x16(tbase + p.H + ch * 16, lo);
+        tmem_ld_wait();
+        float v[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) v[c] = __uint_as_float(hi[c]) + __uint_as_float(lo[c]);
+        constexpr int GC = G >= 16 ? 16 : G;          // owned values in this chunk
+        float o[GC];
+#pragma unroll
+        for (int g = 0; g < GC; ++g) o[g] = v[g];
+#pragma unroll
+        for (int x = 1; x < HQ; ++x)
+          if (jl == x) {
+#pragma unroll
+            for (int g = 0; g < GC; ++g) o[g] = v[x * GC + g];
+          }
+        if (valid) {
+#pragma unroll
+          for (int g = 0; g < GC; ++g) m[ch * 16 + g] = fmaxf(m[ch * 16 + g], o[g]);
+          if constexpr (GC >= 4) {
+#pragma unroll
+            for (int g = 0; g < GC; g += 4)
+              st_global_hint(reinterpret_cast<float4*>(lrow + ch * 16 + g),
+                             make_float4(o[g], o[g + 1], o[g + 2], o[g + 3]), keep);
+          } else {
+            st_global_hint(reinterpret_cast<uint2*>(lrow), make_uint2(__float_as_uint(o[0]), __float_as_uint(o[1])),
+                           keep);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (last) {
+        // merge the quarter's maxima into the segment buffer; the last warp writes the segment out
+        float* sm = segmax + (seg % kKTCSegBufs) * p.H;
+        const int n_own = (p.ncol + G - 1) / G;       // KV heads in this quarter
+#pragma unroll
+        for (int x = 0; x < HQ; ++x) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float w = warp_max_f32(jl == x ? m[g] : -INFINITY);
+            if (lane == 0 && x < n_own && w > -INFINITY) smem_atomic_max_f32(sm + col0 + x * G + g, w);
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) m[g] = -INFINITY;
+        int32_t prev = 0;
+        if (lane == 0) {
+          __threadfence_block();
+          prev = atomicAdd(&segcnt[seg % kKTCSegBufs], 1);
+          __threadfence_block();
+        }
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        if (prev == 3) {
+          for (int h = lane; h < p.H; h += 32) {
+            p.mpart[static_cast<size_t>(b + cta) * p.H + h] = sm[h];
+            sm[h] = -INFINITY;
+          }
+          __syncwarp();
+          if (lane == 0) segcnt[seg % kKTCSegBufs] = 0;
+        }
+        ++seg;
+      }
+      ++k;
+      return true;
+    });
+    if (!ok) set_timeout(p.status, kSiteKFull);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(taddr, p.tmem_cols);
   }
 }
 
@@ -740,6 +1071,7 @@ __global__ void __launch_bounds__(256) zfinal_kernel(ZFinalParams p) {
 struct UpProjParams {
   __half* out;            // [B][H][d]
   int B, H, d, R;
+  int log2G;              // query head h reads B_V columns of KV head h >> log2G
   int n_mt;               // 128-row tiles of d
   int k_per_cta;          // rows of R per CTA (multiple of 64)
   int npad;               // UMMA N (batch tile padded to 16)
@@ -801,7 +1133,7 @@ upproj_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
     prefetch_tensormap(&zhimap);
     prefetch_tensormap(&zlomap);
     const uint64_t pol = policy_evict_first();
-    const int col = h * p.d + mt * 128;
+    const int col = (h >> p.log2G) * p.d + mt * 128;
     const int zrow = h * p.B + b0;
     for (int i = 0; i < n_stages; ++i) {
       const int s = i % S;

@@ -21,6 +21,9 @@
 #ifndef STARKV_K_STAGE_CAP
 #define STARKV_K_STAGE_CAP 65536
 #endif
+#ifndef STARKV_KTC_RING_BYTES
+#define STARKV_KTC_RING_BYTES (192 * 1024)
+#endif
 #ifndef STARKV_K_RING_BYTES
 #define STARKV_K_RING_BYTES (200 * 1024 / STARKV_K_CTAS_PER_SM)
 #endif
@@ -50,6 +53,7 @@ int device_sm_count() {
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int kv_heads(const starkv_layer_desc* d) { return d->num_kv_heads > 0 ? d->num_kv_heads : d->num_heads; }
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int pow2_ceil(int x) { int p = 1; while (p < x) p <<= 1; return p; }
 
@@ -60,6 +64,9 @@ starkv_status check_desc(const starkv_layer_desc* d) {
     return STARKV_ERR_INVALID_ARG;
   if (d->block_size != 16) return STARKV_ERR_UNSUPPORTED;
   if (!is_pow2(d->num_heads) || d->num_heads > 64) return STARKV_ERR_UNSUPPORTED;
+  if (d->num_kv_heads < 0) return STARKV_ERR_INVALID_ARG;
+  if (d->num_kv_heads > 0 && (!is_pow2(d->num_kv_heads) || d->num_kv_heads > d->num_heads))
+    return STARKV_ERR_UNSUPPORTED;
   if (!(d->head_dim == 32 || d->head_dim == 64 || d->head_dim == 128 || d->head_dim == 256))
     return STARKV_ERR_UNSUPPORTED;
   if (d->k_rank % 16 != 0 || d->k_rank > 256) return STARKV_ERR_UNSUPPORTED;
@@ -71,11 +78,16 @@ starkv_status check_desc(const starkv_layer_desc* d) {
 
 // ------------------------------------------------------------------ planning
 struct DecodePlan {
-  int H, d, r, R, B, MB, NB, cap, n_pages_max, t_pad, npad;
+  int H, Hkv, log2G, d, r, R, B, MB, NB, cap, n_pages_max, t_pad, npad;
   // K pass
   int L, CPT, log2H, tps, k_stages, k_ctas;
   uint32_t k_stage_bytes;
   size_t k_smem;
+  // K pass on tensor cores (grouped queries)
+  bool ktc;
+  int ktc_log2tpt, ktc_ksteps, ktc_kb, ktc_npad, ktc_acc_cols, ktc_nacc, ktc_ncol, ktc_stages;
+  uint32_t ktc_a_bytes, ktc_b_bytes, ktc_tmem;
+  size_t ktc_smem;
   // V pass
   int n_rr, r_range, r_range_pad, n_chunks, n_mtiles, v_stages, v_ctas, v_per_sm;
   uint32_t vtile, ltile, ptile, tmem_cols;
@@ -106,6 +118,9 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   DecodePlan& p = *pl;
   std::memset(&p, 0, sizeof(p));
   p.H = d->num_heads; p.d = d->head_dim; p.r = d->k_rank; p.R = d->v_rank;
+  p.Hkv = kv_heads(d);
+  p.log2G = 0;
+  while ((p.Hkv << p.log2G) < p.H) ++p.log2G;
   p.B = batch; p.MB = d->max_blocks_per_seq; p.NB = d->num_blocks;
   p.cap = max_seq_len;
   p.n_pages_max = (max_seq_len + 15) / 16;
@@ -119,9 +134,11 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   plan_kpass_shape(p.r, &p.L, &p.CPT);
   p.log2H = 0;
   while ((1 << p.log2H) < p.H) ++p.log2H;
-  const uint32_t tok = static_cast<uint32_t>(p.H) * p.r * 2;
+  const uint32_t tok = static_cast<uint32_t>(p.Hkv) * p.r * 2;   // code bytes per token
   p.tps = 16;
   while (p.tps > 1 && p.tps * tok > static_cast<uint32_t>(STARKV_K_STAGE_CAP)) p.tps >>= 1;
+  // small pages: several whole pages per stage (up to 8), same byte budget
+  while (p.tps >= 16 && p.tps < 128 && 2u * p.tps * tok <= static_cast<uint32_t>(STARKV_K_STAGE_CAP)) p.tps <<= 1;
   p.k_stage_bytes = p.tps * tok;
   p.k_stages = static_cast<int>(static_cast<uint32_t>(STARKV_K_RING_BYTES) / p.k_stage_bytes);
   if (p.k_stages > 8) p.k_stages = 8;
@@ -129,6 +146,32 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   p.k_smem = static_cast<size_t>(p.k_stages) * p.k_stage_bytes + p.k_stages * sizeof(StageMeta) +
              2 * p.k_stages * sizeof(uint64_t) + (kKConsumers / p.L) * sizeof(float);
   p.k_ctas = sms * STARKV_K_CTAS_PER_SM;
+
+  // Grouped queries (G >= 2) with at most 16 KV heads: the K pass runs on the
+  // tensor cores when two stages fit in shared memory.
+  p.ktc = false;
+  if (p.log2G >= 1 && p.Hkv <= 16) {
+    int log2Hkv = 0;
+    while ((1 << log2Hkv) < p.Hkv) ++log2Hkv;
+    p.ktc_log2tpt = 7 - log2Hkv;
+    p.ktc_ksteps = (p.r + 15) / 16;
+    p.ktc_kb = (p.r + 63) / 64;
+    p.ktc_npad = 2 * p.H < 16 ? 16 : 2 * p.H;
+    p.ktc_acc_cols = p.ktc_npad + 16;
+    const int G = 1 << p.log2G;
+    p.ktc_ncol = G > p.H / 4 ? G : p.H / 4;
+    p.ktc_nacc = 512 / p.ktc_acc_cols;
+    if (p.ktc_nacc > 4) p.ktc_nacc = 4;
+    p.ktc_a_bytes = static_cast<uint32_t>(p.ktc_kb) * 128u * 128u;
+    p.ktc_b_bytes = static_cast<uint32_t>(p.ktc_kb) * p.ktc_npad * 128u;
+    const uint32_t stage = p.ktc_a_bytes + p.ktc_b_bytes;
+    p.ktc_stages = static_cast<int>(static_cast<uint32_t>(STARKV_KTC_RING_BYTES) / stage);
+    if (p.ktc_stages > 8) p.ktc_stages = 8;
+    p.ktc_tmem = static_cast<uint32_t>(pow2_ceil(p.ktc_nacc * p.ktc_acc_cols));
+    p.ktc_smem = 1024 + static_cast<size_t>(p.ktc_stages) * stage + (2 * p.ktc_stages + 9) * sizeof(uint64_t) +
+                 (kKTCSegBufs * p.H + kKTCSegBufs) * sizeof(float);
+    p.ktc = p.ktc_stages >= 2 && p.ktc_nacc >= 2 && p.ktc_tmem <= 512;
+  }
 
   // V pass: R split into ranges of <= 1024 rows (128-row UMMA tiles)
   if (p.R <= STARKV_V_RRANGE) { p.n_rr = 1; p.r_range = p.R; }
@@ -157,7 +200,7 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   p.v_ctas = sms * per_sm / p.n_rr;
   if (p.v_ctas < 1) p.v_ctas = 1;
 
-  p.up_mt = (p.d + 127) / 128;
+  p.up_mt = (p.d + 127) / 128;    // 128-row tiles of d (rows past d are ignored)
   p.up_bt = (batch + 255) / 256;
   {
     const int rows = batch < 256 ? batch : 256;
@@ -201,6 +244,9 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   off = align_up(off + static_cast<size_t>(p.n_rr) * w.v_slots * p.H * p.r_range * 4, 256);
   w.zhi_off = off; off = align_up(off + static_cast<size_t>(p.H) * batch * p.R * 2, 256);
   w.zlo_off = off; off = align_up(off + static_cast<size_t>(p.H) * batch * p.R * 2, 256);
+  w.k_tensor = p.ktc ? 1 : 0;
+  w.qth_off = 0;
+  if (p.ktc) { w.qth_off = off; off = align_up(off + static_cast<size_t>(batch) * 2 * p.H * p.r * 2, 256); }
   w.t_pad = p.t_pad;
   w.total_bytes = off;
   return STARKV_OK;
@@ -251,6 +297,23 @@ bool encode_2d_map(CUtensorMap* map, const void* base, uint64_t cols, uint64_t r
 // 64 columns x 16 rows (one page, one 128-byte-wide chunk).
 bool encode_vpool_map(CUtensorMap* map, const void* v_cache, int R, int NB) {
   return encode_2d_map(map, v_cache, static_cast<uint64_t>(R), static_cast<uint64_t>(NB) * 16, 64, 16);
+}
+
+// K pool [num_blocks*16 tokens][Hkv][r] fp16 as a 3-D tensor map {r, Hkv,
+// tokens} with boxes {64 codes, 1 head, box_tokens} and the 128-byte swizzle
+// (codes past r read as zero).
+bool encode_kpool_map(CUtensorMap* map, const void* k_cache, int r, int Hkv, int NB, uint32_t box_tokens) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(r), static_cast<cuuint64_t>(Hkv),
+                        static_cast<cuuint64_t>(NB) * 16};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(r) * 2, static_cast<cuuint64_t>(Hkv) * r * 2};
+  cuuint32_t box[3] = {64, 1, box_tokens};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult res = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(k_cache), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return res == CUDA_SUCCESS;
 }
 
 // ------------------------------------------------------ kernel attributes
@@ -304,6 +367,25 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
   if (e != cudaSuccess) cudaGetLastError();
   return e;
+}
+
+template <int G>
+cudaError_t launch_kpass_tc_g(const DecodePlan& pl, const CUtensorMap& kmap, const CUtensorMap& qmap,
+                              const KPassTCParams& tp, cudaStream_t s) {
+  if (!set_smem(kpass_tc_kernel<G>, pl.ktc_smem)) return cudaErrorInvalidValue;
+  return launch(kpass_tc_kernel<G>, dim3(pl.k_ctas), dim3(kKTCThreads), pl.ktc_smem, s, 1, kmap, qmap, tp);
+}
+
+cudaError_t launch_kpass_tc(const DecodePlan& pl, const CUtensorMap& kmap, const CUtensorMap& qmap,
+                            const KPassTCParams& tp, cudaStream_t s) {
+  switch (pl.log2G) {
+    case 1: return launch_kpass_tc_g<2>(pl, kmap, qmap, tp, s);
+    case 2: return launch_kpass_tc_g<4>(pl, kmap, qmap, tp, s);
+    case 3: return launch_kpass_tc_g<8>(pl, kmap, qmap, tp, s);
+    case 4: return launch_kpass_tc_g<16>(pl, kmap, qmap, tp, s);
+    case 5: return launch_kpass_tc_g<32>(pl, kmap, qmap, tp, s);
+    default: return launch_kpass_tc_g<64>(pl, kmap, qmap, tp, s);
+  }
 }
 
 template <int L, int CPT>
@@ -373,7 +455,7 @@ starkv_status compress_store_impl(const starkv_layer_desc* desc, int32_t batch, 
       !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(tgt.tables) & 3u) ||
       (reinterpret_cast<uintptr_t>(tgt.positions) & 3u) || (reinterpret_cast<uintptr_t>(tgt.slots) & 3u))
     return STARKV_ERR_INVALID_ARG;
-  const int H = desc->num_heads, d = desc->head_dim, r = desc->k_rank, R = desc->v_rank;
+  const int H = kv_heads(desc), d = desc->head_dim, r = desc->k_rank, R = desc->v_rank;   // codes per KV head
   const int HD = H * d;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
@@ -494,7 +576,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   __half* zlo = reinterpret_cast<__half*>(ws + pl.ws.zlo_off);
   CUtensorMap vmap, bvmap, zhimap, zlomap;
   if (!encode_vpool_map(&vmap, v_cache, pl.R, pl.NB)) return STARKV_ERR_CUDA;
-  if (!encode_2d_map(&bvmap, B_V, static_cast<uint64_t>(pl.H) * pl.d, static_cast<uint64_t>(pl.R), 64, kUpKC) ||
+  if (!encode_2d_map(&bvmap, B_V, static_cast<uint64_t>(pl.Hkv) * pl.d, static_cast<uint64_t>(pl.R), 64, kUpKC) ||
       !encode_2d_map(&zhimap, zhi, static_cast<uint64_t>(pl.R), static_cast<uint64_t>(pl.H) * batch, 64,
                      static_cast<uint32_t>(pl.up_npad)) ||
       !encode_2d_map(&zlomap, zlo, static_cast<uint64_t>(pl.R), static_cast<uint64_t>(pl.H) * batch, 64,
@@ -510,7 +592,9 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   ap.B_K = static_cast<const __half*>(B_K);
   ap.seq_lens = seq_lens;
   ap.qt = qt; ap.prefix = prefix; ap.teff = teff; ap.status = status;
-  ap.B = batch; ap.H = pl.H; ap.d = pl.d; ap.r = pl.r; ap.cap = pl.cap;
+  __half* qth = pl.ktc ? reinterpret_cast<__half*>(ws + pl.ws.qth_off) : nullptr;
+  ap.qth = qth;
+  ap.B = batch; ap.H = pl.H; ap.d = pl.d; ap.r = pl.r; ap.cap = pl.cap; ap.log2G = pl.log2G;
   ap.coef = scale * kLog2e;
   {
     const dim3 grid(pl.H, (batch + kAbsBT - 1) / kAbsBT);
@@ -528,9 +612,26 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   kp.tables = block_tables; kp.teff = teff; kp.prefix = prefix; kp.qt = qt;
   kp.logits = logits; kp.mpart = mpart; kp.status = status;
   kp.B = batch; kp.H = pl.H; kp.log2H = pl.log2H; kp.r = pl.r; kp.MB = pl.MB; kp.NB = pl.NB; kp.t_pad = pl.t_pad;
+  kp.Hkv = pl.Hkv; kp.log2G = pl.log2G;
   kp.tps = pl.tps; kp.stages = pl.k_stages; kp.stage_bytes = pl.k_stage_bytes;
   cudaError_t e;
-  if (pl.L == 1 && pl.CPT == 4) e = launch_kpass<1, 4>(pl, kp, s);
+  if (pl.ktc) {
+    CUtensorMap kmap, qmap;
+    const uint32_t tpt = 1u << pl.ktc_log2tpt;
+    if (!encode_kpool_map(&kmap, k_cache, pl.r, pl.Hkv, pl.NB, tpt < 16 ? tpt : 16) ||
+        !encode_2d_map(&qmap, qth, static_cast<uint64_t>(pl.r), static_cast<uint64_t>(batch) * 2 * pl.H, 64,
+                       static_cast<uint32_t>(pl.ktc_npad)))
+      return STARKV_ERR_CUDA;
+    KPassTCParams tp;
+    tp.tables = block_tables; tp.teff = teff; tp.prefix = prefix;
+    tp.logits = logits; tp.mpart = mpart; tp.status = status;
+    tp.B = batch; tp.H = pl.H; tp.log2G = pl.log2G; tp.log2Hkv = pl.log2H - pl.log2G;
+    tp.MB = pl.MB; tp.NB = pl.NB; tp.t_pad = pl.t_pad;
+    tp.log2tpt = pl.ktc_log2tpt; tp.ksteps = pl.ktc_ksteps; tp.kb = pl.ktc_kb; tp.npad = pl.ktc_npad;
+    tp.acc_cols = pl.ktc_acc_cols; tp.nacc = pl.ktc_nacc; tp.ncol = pl.ktc_ncol; tp.stages = pl.ktc_stages;
+    tp.a_bytes = pl.ktc_a_bytes; tp.b_bytes = pl.ktc_b_bytes; tp.tmem_cols = pl.ktc_tmem;
+    e = launch_kpass_tc(pl, kmap, qmap, tp, s);
+  } else if (pl.L == 1 && pl.CPT == 4) e = launch_kpass<1, 4>(pl, kp, s);
   else if (pl.L == 1 && pl.CPT == 8) e = launch_kpass<1, 8>(pl, kp, s);
   else if (pl.L == 1) e = launch_kpass<1, 12>(pl, kp, s);
   else if (pl.L == 2) e = launch_kpass<2, 8>(pl, kp, s);
@@ -561,7 +662,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
 
   UpProjParams up;
   up.out = static_cast<__half*>(out);
-  up.B = batch; up.H = pl.H; up.d = pl.d; up.R = pl.R;
+  up.B = batch; up.H = pl.H; up.d = pl.d; up.R = pl.R; up.log2G = pl.log2G;
   up.n_mt = pl.up_mt; up.k_per_cta = pl.up_kpc; up.npad = pl.up_npad;
   up.stages = pl.up_stages; up.tmem_cols = pl.up_tmem;
   if (!set_smem(upproj_kernel, pl.up_smem)) return STARKV_ERR_CUDA;

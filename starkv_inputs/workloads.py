@@ -70,7 +70,13 @@ def _llama_layer(r: int, R: int) -> LayerShape:
 
 
 def workload(idx: int) -> Workload:
-    """The five workloads (1-based like the configuration list they come from)."""
+    """The five benchmark workloads (1-based), plus 6: a grouped-query layer.
+
+    Workload 6 has Llama-3-8B attention heads (32 query heads over 8 KV heads,
+    head_dim 128) compressed at the same ratios as the 7B layers (K rank 64 of
+    128, V rank 512 of the 1024 concatenated KV-head dims), batch 64 at
+    context 8192.
+    """
     if idx == 1:
         return Workload("tiny: H4 d64 r16 R64, B2, T{37,100}", 1001, 2,
                         [LayerShape(4, 64, 16, 64)],
@@ -92,6 +98,10 @@ def workload(idx: int) -> Workload:
         return Workload("Llama-2-7B attention path: 32 layers, B8, T32768, r64 R2048", 1005, 8,
                         [_llama_layer(64, 2048) for _ in range(32)],
                         np.full(8, 32767, dtype=np.int64))
+    if idx == 6:
+        return Workload("grouped-query layer: H32 Hkv8 d128 r64 R512, B64, T8192", 1006, 64,
+                        [LayerShape(32, 128, 64, 512, num_kv_heads=8)],
+                        np.full(64, 8191, dtype=np.int64))
     raise ValueError(idx)
 
 

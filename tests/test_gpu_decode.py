@@ -26,7 +26,8 @@ def rel_l2(got, ref):
 
 
 def desc_of(L):
-    return S.layer_desc(L["H"], L["d"], L["r"], L["R"], L["nb"], L["tables"].shape[1])
+    return S.layer_desc(L["H"], L["d"], L["r"], L["R"], L["nb"], L["tables"].shape[1],
+                        num_kv_heads=L.get("Hkv", 0))
 
 
 def run_decode(L, seq_lens=None, max_seq_len=None, q=None):
@@ -121,13 +122,19 @@ def test_decode_tiny_workload():
     _full_check(W.workload(1))
 
 
-def test_decode_tiny_intermediates():
-    """Logits, per-segment maxima and softmax normaliser against the oracle's stages."""
-    wl = W.workload(1)
+@pytest.mark.parametrize("gqa", [False, True])
+def test_decode_tiny_intermediates(gqa):
+    """Logits, per-segment maxima and softmax normaliser against the oracle's stages.
+
+    The grouped-query case (8 query heads over 2 KV heads) runs the tensor-core K pass.
+    """
+    wl = (W.custom("tiny-gqa", 1011, W.LayerShape(8, 64, 16, 128, num_kv_heads=2), [37, 100, 290],
+                   append=False) if gqa else W.workload(1))
     Lh = W.host_layer(wl, 0)
     Ld = D.device_layer(wl, 0, tables=Lh["tables"], nb=Lh["nb"])
     got, ws, desc = run_decode(Ld)
     lay = S.starkv_decode_workspace_layout(desc, wl.batch, wl.max_seq_len)
+    assert lay.k_tensor == (1 if gqa else 0)
     wsn = ws.cpu().numpy()
     H = Lh["H"]
     f32 = lambda off, n: wsn[off:off + 4 * n].view(np.float32)
@@ -290,9 +297,10 @@ def _append_check(wl, layer=0):
     cK, cV = O.compress(Lh["k"], Lh["v"], Lh["A_K"], Lh["A_V"])
     pos = wl.ctx_lens
     rows = np.array([Lh["tables"][b][pos[b] // 16] * 16 + pos[b] % 16 for b in range(wl.batch)])
-    kf_new = Ld["k_cache"].view(-1, Lh["H"] * Lh["r"]).cpu().numpy()
+    Hkv = Lh["Hkv"]
+    kf_new = Ld["k_cache"].view(-1, Hkv * Lh["r"]).cpu().numpy()
     vf_new = Ld["v_cache"].view(-1, Lh["R"]).cpu().numpy()
-    kf_old = before_k.view(-1, Lh["H"] * Lh["r"]).cpu().numpy()
+    kf_old = before_k.view(-1, Hkv * Lh["r"]).cpu().numpy()
     vf_old = before_v.view(-1, Lh["R"]).cpu().numpy()
     mask = np.ones(kf_new.shape[0], bool)
     mask[rows] = False
@@ -303,10 +311,10 @@ def _append_check(wl, layer=0):
     # order-free accumulation
     kk, vv = Lh["k"].astype(np.float64), Lh["v"].astype(np.float64)
     absK = np.stack([np.abs(kk[:, h, :]) @ np.abs(Lh["A_K"][h].astype(np.float64))
-                     for h in range(Lh["H"])], axis=1).reshape(wl.batch, -1)
+                     for h in range(Hkv)], axis=1).reshape(wl.batch, -1)
     absV = np.abs(vv.reshape(wl.batch, -1)) @ np.abs(Lh["A_V"].astype(np.float64))
     for want, got, absum, K in ((cK.reshape(wl.batch, -1), kf_new[rows], absK, Lh["d"]),
-                                (cV, vf_new[rows], absV, Lh["H"] * Lh["d"])):
+                                (cV, vf_new[rows], absV, Hkv * Lh["d"])):
         got = got.astype(np.float64)
         ulp = np.spacing(np.abs(want).astype(np.float16)).astype(np.float64)
         gamma = K * 2.0 ** -24 / (1 - K * 2.0 ** -24)
@@ -365,6 +373,60 @@ def test_compress_store_prefill_then_decode():
     assert_close({0: got[0]}, {0: ref[0]})
 
 
+# ------------------------------------------------ grouped-query attention
+
+@pytest.mark.parametrize("H,Hkv,d,r,R", [
+    (32, 8, 128, 64, 512),      # Llama-3-8B-like heads, 4 query heads per KV head
+    (32, 16, 128, 64, 1024),    # 2 per KV head
+    (16, 1, 128, 64, 128),      # one KV head (multi-query)
+    (64, 8, 128, 128, 1024),    # 8 per KV head, r = d
+    (8, 2, 64, 16, 128),        # small pages: 8-page K stages
+])
+def test_decode_grouped_query(H, Hkv, d, r, R):
+    sh = W.LayerShape(H, d, r, R, num_kv_heads=Hkv)
+    wl = W.custom(f"gqa{H}x{Hkv}", 600 + H + Hkv, sh, [1, 15, 16, 17, 300, 0, 1000, 129], append=False)
+    _full_check(wl)
+
+
+def test_append_then_decode_grouped_query():
+    sh = W.LayerShape(32, 128, 64, 512, num_kv_heads=8)
+    wl = W.custom("gqa-app", 777, sh, [37, 100, 0, 15, 2000, 4095], append=True)
+    Lh, Ld, appended = _append_check(wl)
+    got, *_ = run_decode(Ld)
+    ref = oracle_rows(wl, 0, Lh["q"], Ld["A_np"], range(wl.batch), wl.seq_lens, appended)
+    assert_close({b: got[b] for b in range(wl.batch)}, ref)
+
+
+def test_decode_grouped_query_equals_repeated_kv_heads_on_gpu():
+    """Hkv KV heads against the same inputs repeated to H KV heads: the MHA kernels' output."""
+    H, Hkv, d, r, R = 16, 4, 64, 32, 256
+    G = H // Hkv
+    sh = W.LayerShape(H, d, r, R, num_kv_heads=Hkv)
+    wl = W.custom("gqa-rep", 808, sh, [5, 70, 333], append=False)
+    Lh = W.host_layer(wl, 0)
+    Ld = D.device_layer(wl, 0, tables=Lh["tables"], nb=Lh["nb"])
+    got, *_ = run_decode(Ld)
+    rep = dict(Ld)
+    rep["Hkv"] = H
+    rep["k_cache"] = Ld["k_cache"].repeat_interleave(G, dim=2).contiguous()
+    rep["B_K"] = Ld["B_K"].repeat_interleave(G, dim=0).contiguous()
+    rep["B_V"] = torch.cat([Ld["B_V"][:, (h // G) * d:(h // G + 1) * d] for h in range(H)], 1).contiguous()
+    want, *_ = run_decode(rep)
+    ref = O.decode_explicit(Lh["q"], Lh["B_K"], Lh["B_V"], Lh["k_cache"], Lh["v_cache"],
+                            Lh["tables"], Lh["seq_lens"], Lh["scale"])
+    assert_close({b: got[b] for b in range(wl.batch)}, {b: ref[b] for b in range(wl.batch)})
+    assert_close({b: want[b] for b in range(wl.batch)}, {b: ref[b] for b in range(wl.batch)})
+
+
+def test_grouped_query_descriptor_checks():
+    d = S.layer_desc(32, 128, 64, 512, 100, 8, num_kv_heads=12)        # not a power of two
+    assert S.starkv_decode_workspace_bytes(d, 4, 100) == 0
+    d = S.layer_desc(8, 128, 64, 512, 100, 8, num_kv_heads=16)         # more KV than query heads
+    assert S.starkv_decode_workspace_bytes(d, 4, 100) == 0
+    d = S.layer_desc(32, 128, 64, 512, 100, 8, num_kv_heads=8)
+    assert S.starkv_decode_workspace_bytes(d, 4, 100) > 0
+
+
 def test_decode_and_append_batch_over_256():
     """300 short sequences: several 256-row batch tiles in the append GEMM and the up-projection."""
     sh = W.LayerShape(32, 128, 64, 2048)
@@ -387,6 +449,7 @@ def test_decode_and_append_batch_over_256():
     (4, 2, [11, 40]),                   #   r=96 / R=3072
     (5, 0, [0, 7]),                     # 32-layer 7B attention path, first layer
     (5, 31, [3]),                       #   last layer
+    (6, 0, [0, 21, 63]),                # grouped-query layer, batch 64, context 8192
 ])
 def test_decode_full_size_sampled(idx, layer, sample):
     """Full-size workloads in the benchmark's launch configuration, sampled rows."""
