@@ -413,20 +413,21 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
 
 // ============================================================== kpass (tensor)
 // Grouped-query K pass on tcgen05.  With G = H/Hkv query heads per KV head the
-// logits of a run of tokens are a small GEMM, S[(j,t), h] = c_K[t, j] . q~_h.
+// logits of a run of tokens are a small GEMM, S[(t,j), h] = c_K[t, j] . q~_h.
 // A tile is 128 code rows: tpt = 128/Hkv tokens of one sequence times the Hkv
-// KV heads, head-major (row j*tpt + t), loaded by TMA as 3-D boxes
-// {64 codes, 1 head, min(16, tpt) tokens} with the 128-byte swizzle, which is
-// the K-major operand layout.  B holds the sequence's absorbed queries for all
-// H heads split into an fp16 high part (row h) and the fp16 rounding of the
-// remainder (row H+h), so D[row, h] + D[row, H+h] is c_K . q~_h with q~ carried
-// to about 22 bits and fp32 accumulation.  A row uses only the G columns of its
-// own KV head; the tensor cores compute all 2H, which at G >= 2 still costs
-// less than the HBM time of the tile.  The epilogue (4 warps, one TMEM lane
-// quarter each) adds hi + lo, stores each row's G logits as one contiguous
-// vector and keeps the row's running maxima, merged per (sequence, CTA)
-// segment in shared memory.  Several accumulators let the tensor cores run
-// ahead of the epilogue.
+// KV heads in page order (row t*Hkv + j), brought in by one 3-D TMA box per
+// page {64 codes, Hkv heads, min(16, tpt) tokens} with the 128-byte swizzle,
+// which is the K-major operand layout.  B holds the sequence's absorbed
+// queries for all H heads split into an fp16 high part (row h) and the fp16
+// rounding of the remainder (row H+h), so D[row, h] + D[row, H+h] is
+// c_K . q~_h with q~ carried to about 22 bits and fp32 accumulation; it is
+// loaded once per (sequence, CTA) segment into one of two slots.  A row uses
+// only the G columns of its own KV head; the tensor cores compute all 2H,
+// which at G >= 2 still costs less than the HBM time of the tile.  The
+// epilogue (4 warps, one TMEM lane quarter each) adds hi + lo for its row's G
+// heads, stores them as one contiguous vector (a warp writes whole logit rows)
+// and keeps running maxima, merged per segment in shared memory.  Several
+// accumulators let the tensor cores run ahead of the epilogue.
 struct KPassTCParams {
   const int32_t* tables;      // [B][MB]
   const int32_t* teff;        // [B]
@@ -434,14 +435,12 @@ struct KPassTCParams {
   float* logits;              // [B][t_pad][H]
   float* mpart;               // [k_slots][H]
   int32_t* status;
-  int B, H, log2G, log2Hkv, MB, NB, t_pad;
+  int B, log2G, log2Hkv, MB, NB, t_pad;
   int log2tpt;                // tokens per tile = 128 / Hkv
   int ksteps;                 // UMMA K steps of 16 codes: ceil(r/16)
   int kb;                     // 64-code column blocks: ceil(r/64)
   int npad;                   // UMMA N = max(16, 2H)
-  int acc_cols;               // TMEM columns per accumulator (npad + 16 of slack for the epilogue reads)
-  int nacc;                   // accumulators in TMEM (2..4)
-  int ncol;                   // query-head columns of one lane quarter: max(G, H/4)
+  int nacc;                   // accumulators in TMEM (2..4), npad columns each
   int stages;
   uint32_t a_bytes;           // kb * 128 rows * 128 bytes
   uint32_t b_bytes;           // kb * npad * 128 bytes
@@ -451,9 +450,10 @@ struct KPassTCParams {
 constexpr int kKTCThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kKTCSegBufs = 6;     // segment-maximum buffers (warps run at most nacc <= 4 tiles apart)
 
-// Calls f(b, t0, nt, last) for the K-pass tiles of pages [p0, p1) in order:
-// tokens [t0, t0+nt) of sequence b, `last` on the final tile of the
-// (sequence, CTA) segment.  Stops when f returns false.
+// Calls f(b, t0, nt, x0, first, last) for the K-pass tiles of pages [p0, p1)
+// in order: tokens [t0, t0+nt) of sequence b, whose first token lies in global
+// page x0, `first` / `last` on the first and final tile of the (sequence, CTA)
+// segment.  Stops when f returns false.
 template <typename F>
 __device__ __forceinline__ void for_each_k_tile(const KPassTCParams& p, int64_t p0, int64_t p1, F&& f) {
   const int tpt = 1 << p.log2tpt;
@@ -466,7 +466,7 @@ __device__ __forceinline__ void for_each_k_tile(const KPassTCParams& p, int64_t 
     const int32_t ts = static_cast<int32_t>(x - base) * kBlock;
     const int32_t te = min(static_cast<int32_t>(seg_end - base) * kBlock, p.teff[b]);
     for (int32_t t0 = ts; t0 < te; t0 += tpt)
-      if (!f(b, t0, min(tpt, te - t0), t0 + tpt >= te)) return;
+      if (!f(b, t0, min(tpt, te - t0), static_cast<int64_t>(base) + (t0 >> 4), t0 == ts, t0 + tpt >= te)) return;
     x = seg_end;
   }
 }
@@ -478,33 +478,36 @@ __device__ __forceinline__ void smem_atomic_max_f32(float* addr, float v) {
   else atomicMin(reinterpret_cast<unsigned int*>(addr), __float_as_uint(v));
 }
 
-template <int G>   // query heads per KV head
+template <int G, int H>   // query heads per KV head, query heads
 __global__ void __launch_bounds__(kKTCThreads, 1)
 kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                 KPassTCParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages;
-  const uint32_t stage_bytes = p.a_bytes + p.b_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * stage_bytes);
+  uint8_t* bslot = smem + static_cast<size_t>(S) * p.a_bytes;                    // [2] query tiles
+  uint64_t* full = reinterpret_cast<uint64_t*>(bslot + 2 * static_cast<size_t>(p.b_bytes));
   uint64_t* empty = full + S;
-  uint64_t* tfull = empty + S;     // [4] accumulator ready
+  uint64_t* bfull = empty + S;     // [2] query tile landed
+  uint64_t* bempty = bfull + 2;    // [2] query tile no longer read by the tensor cores
+  uint64_t* tfull = bempty + 2;    // [4] accumulator ready
   uint64_t* tempty = tfull + 4;    // [4] accumulator drained (4 epilogue warps)
   uint64_t* mmadone = tempty + 4;
   float* segmax = reinterpret_cast<float*>(mmadone + 1);          // [kKTCSegBufs][H]
-  int32_t* segcnt = reinterpret_cast<int32_t*>(segmax + kKTCSegBufs * p.H);
+  int32_t* segcnt = reinterpret_cast<int32_t*>(segmax + kKTCSegBufs * H);
   __shared__ uint32_t taddr_s;
   __shared__ volatile int32_t abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&bfull[a], 1); mbar_init(&bempty[a], 1); }
     for (int a = 0; a < 4; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
     mbar_init(mmadone, 1);
     abort_flag = 0;
     fence_mbar_init();
   }
-  for (int i = tid; i < kKTCSegBufs * p.H; i += kKTCThreads) segmax[i] = -INFINITY;
+  for (int i = tid; i < kKTCSegBufs * H; i += kKTCThreads) segmax[i] = -INFINITY;
   if (tid < kKTCSegBufs) segcnt[tid] = 0;
   griddep_wait();
   griddep_launch_dependents();
@@ -523,71 +526,105 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   const uint32_t taddr = taddr_s;
   const int64_t p0 = part_begin(cta, pt), p1 = part_begin(cta + 1, pt);
   const int tpt = 1 << p.log2tpt;
-  const int tb = tpt < kBlock ? tpt : kBlock;       // tokens per TMA box
   const int Hkv = 1 << p.log2Hkv;
+  const int tb = tpt < kBlock ? tpt : kBlock;       // tokens per TMA box (one page, or half of one)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // The whole warp walks the tiles; lane i reads ahead the block-table entry
+    // of page cbase + i so that lane 0 never waits on a table load per page.
     if (lane == 0) {
       prefetch_tensormap(&kmap);
       prefetch_tensormap(&qmap);
-      const uint64_t stream = policy_evict_first();
-      const uint64_t reuse = policy_evict_last();   // q~ tiles: read again for every tile
-      const uint32_t box_bytes = static_cast<uint32_t>(tb) * 128u;
-      uint32_t k = 0;
-      bool ok = true;
-      for_each_k_tile(p, p0, p1, [&](int32_t b, int32_t t0, int32_t nt, bool) {
-        const int s = k % S;
-        if (k >= static_cast<uint32_t>(S) && !mbar_wait(&empty[s], ((k / S) - 1) & 1)) { ok = false; return false; }
-        uint8_t* st = smem + static_cast<size_t>(s) * stage_bytes;
-        const int nbox = (nt + tb - 1) / tb;
-        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox * Hkv * p.kb) * box_bytes + p.b_bytes);
-        for (int c = 0; c < nbox; ++c) {
-          const int32_t t = t0 + c * tb;
-          int32_t phys = p.tables[static_cast<size_t>(b) * p.MB + (t >> 4)];
+    }
+    const uint64_t stream = policy_evict_first();
+    const uint64_t reuse = policy_evict_last();
+    const uint32_t box_bytes = static_cast<uint32_t>(tb) * Hkv * 128u;
+    int64_t cbase = -64;
+    int32_t cphys = 0;
+    int32_t cb = 0;
+    uint32_t k = 0, seg = 0;
+    bool ok = true;
+    for_each_k_tile(p, p0, p1, [&](int32_t b, int32_t t0, int32_t nt, int64_t x0, bool first, bool last) {
+      if (first) {
+        const int bs = seg & 1;
+        if (lane == 0) {
+          if (seg >= 2 && !mbar_wait(&bempty[bs], ((seg >> 1) - 1) & 1)) {
+            ok = false;
+          } else {
+            mbar_arrive_expect_tx(&bfull[bs], p.b_bytes);
+            for (int a = 0; a < p.kb; ++a)
+              tma_load_2d(bslot + bs * static_cast<size_t>(p.b_bytes) + static_cast<size_t>(a) * p.npad * 128, &qmap,
+                          a * 64, b * 2 * H, &bfull[bs], reuse);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) return false;
+      }
+      const int s = k % S;
+      if (lane == 0 && k >= static_cast<uint32_t>(S) && !mbar_wait(&empty[s], ((k / S) - 1) & 1)) ok = false;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) return false;
+      uint8_t* st = smem + static_cast<size_t>(s) * p.a_bytes;
+      const int nbox = (nt + tb - 1) / tb;
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox * p.kb) * box_bytes);
+      for (int c = 0; c < nbox; ++c) {
+        const int32_t t = t0 + c * tb;
+        const int64_t x = x0 + (((t0 & (kBlock - 1)) + c * tb) >> 4);      // global page index
+        if (x < cbase || x >= cbase + 32) {                                  // uniform over the warp
+          cbase = x;
+          cb = b;
+          const int64_t xi = x + lane;
+          int32_t bi = b;
+          while (bi < p.B - 1 && p.prefix[bi + 1] <= xi) ++bi;
+          cphys = xi < p1 ? p.tables[static_cast<size_t>(bi) * p.MB + static_cast<int32_t>(xi - p.prefix[bi])] : 0;
+        }
+        int32_t phys = __shfl_sync(0xffffffffu, cphys, static_cast<int>(x - cbase));
+        if (lane == 0) {
           if (phys < 0 || phys >= p.NB) { set_flag(p.status, STARKV_FLAG_BAD_BLOCK_ID); phys = 0; }
           const int32_t row = phys * kBlock + (t & (kBlock - 1));
-          for (int j = 0; j < Hkv; ++j)
-            for (int a = 0; a < p.kb; ++a)
-              tma_load_3d(st + static_cast<size_t>(a) * 16384 + static_cast<size_t>((j << p.log2tpt) + c * tb) * 128,
-                          &kmap, a * 64, j, row, &full[s], stream);
+          for (int a = 0; a < p.kb; ++a)
+            tma_load_3d(st + static_cast<size_t>(a) * 16384 + static_cast<size_t>(c) * box_bytes, &kmap, a * 64, 0,
+                        row, &full[s], stream);
         }
-        for (int a = 0; a < p.kb; ++a)
-          tma_load_2d(st + p.a_bytes + static_cast<size_t>(a) * p.npad * 128, &qmap, a * 64, b * 2 * p.H,
-                      &full[s], reuse);
-        ++k;
-        return true;
-      });
-      if (!ok) {
-        set_timeout(p.status, kSiteKEmpty);
-        abort_flag = 1;
-        const uint32_t first = k > static_cast<uint32_t>(S) ? k - S : 0;
-        for (uint32_t kk = first; kk < k; ++kk) mbar_wait(&full[kk % S], (kk / S) & 1);
       }
+      ++k;
+      if (last) ++seg;
+      return true;
+    });
+    (void)cb;
+    if (!ok && lane == 0) {
+      set_timeout(p.status, kSiteKEmpty);
+      abort_flag = 1;
+      const uint32_t first = k > static_cast<uint32_t>(S) ? k - S : 0;
+      for (uint32_t kk = first; kk < k; ++kk) mbar_wait(&full[kk % S], (kk / S) & 1);
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(128, p.npad, /*a_mn_major=*/false, /*b_mn_major=*/false);
-      uint32_t k = 0;
+      uint32_t k = 0, seg = 0;
       bool ok = true;
-      for_each_k_tile(p, p0, p1, [&](int32_t, int32_t, int32_t, bool) {
+      for_each_k_tile(p, p0, p1, [&](int32_t, int32_t, int32_t, int64_t, bool first, bool last) {
         const int s = k % S;
+        const int bs = seg & 1;
         const uint32_t acc = k % p.nacc, use = k / p.nacc;
+        if (first && !mbar_wait(&bfull[bs], (seg >> 1) & 1)) { ok = false; return false; }
         if (use > 0 && !mbar_wait(&tempty[acc], (use - 1) & 1)) { ok = false; return false; }
         if (!mbar_wait(&full[s], (k / S) & 1) || abort_flag) { ok = false; return false; }
         tc_fence_after();
-        const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
-        const uint32_t sb = sa + p.a_bytes;
-        const uint32_t d = taddr + static_cast<uint32_t>(acc * p.acc_cols);
+        // descriptors of the stage / query slot; a K step adds its byte offset >> 4 to the start field
+        const uint64_t da = smem_desc(smem_u32(smem + static_cast<size_t>(s) * p.a_bytes), 16u, 1024u, kSwizzle128B);
+        const uint64_t db = smem_desc(smem_u32(bslot + bs * static_cast<size_t>(p.b_bytes)), 16u, 1024u, kSwizzle128B);
+        const uint32_t d = taddr + acc * static_cast<uint32_t>(p.npad);
+        const uint32_t b_atom = static_cast<uint32_t>(p.npad) * 8u;     // npad * 128 bytes >> 4
         for (int ks = 0; ks < p.ksteps; ++ks) {
           const uint32_t a = ks >> 2, kk = ks & 3;
-          umma_f16_ss(d, smem_desc(sa + a * 16384u + kk * 32u, 16u, 1024u, kSwizzle128B),
-                      smem_desc(sb + a * static_cast<uint32_t>(p.npad) * 128u + kk * 32u, 16u, 1024u, kSwizzle128B),
-                      idesc, ks > 0 ? 1u : 0u);
+          umma_f16_ss(d, da + (a * 1024u + kk * 2u), db + (a * b_atom + kk * 2u), idesc, ks > 0 ? 1u : 0u);
         }
         umma_commit(&empty[s]);
         umma_commit(&tfull[acc]);
+        if (last) { umma_commit(&bempty[bs]); ++seg; }
         ++k;
         return true;
       });
@@ -597,76 +634,74 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // Columns [col0, col0 + ncol) of a lane quarter are the query heads of its
-    // KV heads; the lane owns the G of them at offset jl*G.
-    constexpr int NCH = G >= 16 ? G / 16 : 1;        // 16-column chunks read per tile
-    constexpr int HQ = G >= 16 ? 1 : 16 / G;         // KV heads a 16-column chunk spans
+    // Row rho of a tile is token rho / Hkv, KV head j = rho % Hkv; the row's
+    // logits are D columns [j*G, j*G + G) (hi) plus H + the same (lo).
     const int q = warp & 3;                          // TMEM lane quarter of this warp
-    const int rho = q * 32 + lane;                   // tile row
-    const int jq = (q * 32) >> p.log2tpt;            // first KV head of the quarter
-    const int jl = (rho >> p.log2tpt) - jq;          // this row's KV head, relative to jq
-    const int tl = rho & (tpt - 1);                  // token of this row within the tile
-    const int col0 = jq * G;                         // first query head of the quarter
+    const int rho = q * 32 + lane;
+    const int j = rho & (Hkv - 1);
+    const int tl = rho >> p.log2Hkv;
     const uint64_t keep = policy_evict_last();       // logits: read back by the V pass
     float m[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) m[g] = -INFINITY;
     uint32_t k = 0, seg = 0;
     bool ok = true;
-    for_each_k_tile(p, p0, p1, [&](int32_t b, int32_t t0, int32_t nt, bool last) {
+    for_each_k_tile(p, p0, p1, [&](int32_t b, int32_t t0, int32_t nt, int64_t, bool, bool last) {
       const uint32_t acc = k % p.nacc, use = k / p.nacc;
       if (!mbar_wait(&tfull[acc], use & 1) || abort_flag) { ok = false; return false; }
       tc_fence_after();
-      const bool valid = tl < nt;
-      float* lrow = p.logits + (static_cast<size_t>(b) * p.t_pad + t0 + tl) * p.H + col0 + jl * G;
-      const uint32_t tbase = taddr + (static_cast<uint32_t>(q * 32) << 16) + acc * p.acc_cols + col0;
+      const uint32_t tbase = taddr + (static_cast<uint32_t>(q * 32) << 16) + acc * static_cast<uint32_t>(p.npad);
+      float o[G];
+      if constexpr (H >= 32) {
 #pragma unroll
-      for (int ch = 0; ch < NCH; ++ch) {
-        uint32_t hi[32], lo[32];
-        tmem_ld_32x32b_x16(tbase + ch * 16, hi);
-        tmem_ld_32x32b_x16(tbase + p.H + ch * 16, lo);
-        tmem_ld_wait();
-        float v[16];
+        for (int ch = 0; ch < H / 32; ++ch) {     // hi and lo of 32 heads per round, one wait
+          uint32_t hi[32], lo[32];
+          tmem_ld_32x32b_x32(tbase + ch * 32, hi);
+          tmem_ld_32x32b_x32(tbase + H + ch * 32, lo);
+          tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 16; ++c) v[c] = __uint_as_float(hi[c]) + __uint_as_float(lo[c]);
-        constexpr int GC = G >= 16 ? 16 : G;          // owned values in this chunk
-        float o[GC];
-#pragma unroll
-        for (int g = 0; g < GC; ++g) o[g] = v[g];
-#pragma unroll
-        for (int x = 1; x < HQ; ++x)
-          if (jl == x) {
-#pragma unroll
-            for (int g = 0; g < GC; ++g) o[g] = v[x * GC + g];
-          }
-        if (valid) {
-#pragma unroll
-          for (int g = 0; g < GC; ++g) m[ch * 16 + g] = fmaxf(m[ch * 16 + g], o[g]);
-          if constexpr (GC >= 4) {
-#pragma unroll
-            for (int g = 0; g < GC; g += 4)
-              st_global_hint(reinterpret_cast<float4*>(lrow + ch * 16 + g),
-                             make_float4(o[g], o[g + 1], o[g + 2], o[g + 3]), keep);
-          } else {
-            st_global_hint(reinterpret_cast<uint2*>(lrow), make_uint2(__float_as_uint(o[0]), __float_as_uint(o[1])),
-                           keep);
+          for (int c = 0; c < 32; ++c) {
+            const int col = ch * 32 + c;
+            if ((col / G) == j) o[col % G] = __uint_as_float(hi[c]) + __uint_as_float(lo[c]);
           }
         }
+      } else if constexpr (H == 16) {
+        uint32_t v[32];                              // columns [0, 16) hi, [16, 32) lo
+        tmem_ld_32x32b_x32(tbase, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          if ((c / G) == j) o[c % G] = __uint_as_float(v[c]) + __uint_as_float(v[16 + c]);
+      } else {
+        uint32_t v[32];                              // columns [0, H) hi, [H, 2H) lo
+        tmem_ld_32x32b_x16(tbase, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < H; ++c)
+          if ((c / G) == j) o[c % G] = __uint_as_float(v[c]) + __uint_as_float(v[H + c]);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (tl < nt) {
+        float* lrow = p.logits + (static_cast<size_t>(b) * p.t_pad + t0 + tl) * H + j * G;
+#pragma unroll
+        for (int g = 0; g < G; ++g) m[g] = fmaxf(m[g], o[g]);
+        if constexpr (G >= 4) {
+#pragma unroll
+          for (int g = 0; g < G; g += 4)
+            st_global_hint(reinterpret_cast<float4*>(lrow + g), make_float4(o[g], o[g + 1], o[g + 2], o[g + 3]), keep);
+        } else {
+          st_global_hint(reinterpret_cast<uint2*>(lrow), make_uint2(__float_as_uint(o[0]), __float_as_uint(o[1])), keep);
+        }
+      }
       if (last) {
-        // merge the quarter's maxima into the segment buffer; the last warp writes the segment out
-        float* sm = segmax + (seg % kKTCSegBufs) * p.H;
-        const int n_own = (p.ncol + G - 1) / G;       // KV heads in this quarter
+        // merge this warp's maxima into the segment buffer; the last warp writes the segment out
+        float* sm = segmax + (seg % kKTCSegBufs) * H;
 #pragma unroll
-        for (int x = 0; x < HQ; ++x) {
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const float w = warp_max_f32(jl == x ? m[g] : -INFINITY);
-            if (lane == 0 && x < n_own && w > -INFINITY) smem_atomic_max_f32(sm + col0 + x * G + g, w);
-          }
+        for (int h = 0; h < H; ++h) {
+          const float w = warp_max_f32((h / G) == j ? m[h % G] : -INFINITY);
+          if (lane == 0 && w > -INFINITY) smem_atomic_max_f32(sm + h, w);
         }
 #pragma unroll
         for (int g = 0; g < G; ++g) m[g] = -INFINITY;
@@ -678,8 +713,8 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         }
         prev = __shfl_sync(0xffffffffu, prev, 0);
         if (prev == 3) {
-          for (int h = lane; h < p.H; h += 32) {
-            p.mpart[static_cast<size_t>(b + cta) * p.H + h] = sm[h];
+          for (int h = lane; h < H; h += 32) {
+            p.mpart[static_cast<size_t>(b + cta) * H + h] = sm[h];
             sm[h] = -INFINITY;
           }
           __syncwarp();

@@ -21,8 +21,11 @@
 #ifndef STARKV_K_STAGE_CAP
 #define STARKV_K_STAGE_CAP 65536
 #endif
-#ifndef STARKV_KTC_RING_BYTES
-#define STARKV_KTC_RING_BYTES (192 * 1024)
+#ifndef STARKV_KTC_CTAS_PER_SM
+#define STARKV_KTC_CTAS_PER_SM 2
+#endif
+#ifndef STARKV_KTC_SMEM_BYTES
+#define STARKV_KTC_SMEM_BYTES (216 * 1024)   // stage ring + query slots of the CTAs on one SM
 #endif
 #ifndef STARKV_K_RING_BYTES
 #define STARKV_K_RING_BYTES (200 * 1024 / STARKV_K_CTAS_PER_SM)
@@ -85,7 +88,7 @@ struct DecodePlan {
   size_t k_smem;
   // K pass on tensor cores (grouped queries)
   bool ktc;
-  int ktc_log2tpt, ktc_ksteps, ktc_kb, ktc_npad, ktc_acc_cols, ktc_nacc, ktc_ncol, ktc_stages;
+  int ktc_log2tpt, ktc_ksteps, ktc_kb, ktc_npad, ktc_nacc, ktc_stages;
   uint32_t ktc_a_bytes, ktc_b_bytes, ktc_tmem;
   size_t ktc_smem;
   // V pass
@@ -147,30 +150,32 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
              2 * p.k_stages * sizeof(uint64_t) + (kKConsumers / p.L) * sizeof(float);
   p.k_ctas = sms * STARKV_K_CTAS_PER_SM;
 
-  // Grouped queries (G >= 2) with at most 16 KV heads: the K pass runs on the
-  // tensor cores when two stages fit in shared memory.
+  // Grouped queries (G >= 2, H >= 4) with at most 16 KV heads: the K pass runs
+  // on the tensor cores, with STARKV_KTC_CTAS_PER_SM CTAs per SM when their
+  // rings (>= 2 stages) and accumulators fit, else with one.
   p.ktc = false;
-  if (p.log2G >= 1 && p.Hkv <= 16) {
+  if (p.log2G >= 1 && p.H >= 4 && p.Hkv <= 16) {
     int log2Hkv = 0;
     while ((1 << log2Hkv) < p.Hkv) ++log2Hkv;
     p.ktc_log2tpt = 7 - log2Hkv;
     p.ktc_ksteps = (p.r + 15) / 16;
     p.ktc_kb = (p.r + 63) / 64;
     p.ktc_npad = 2 * p.H < 16 ? 16 : 2 * p.H;
-    p.ktc_acc_cols = p.ktc_npad + 16;
-    const int G = 1 << p.log2G;
-    p.ktc_ncol = G > p.H / 4 ? G : p.H / 4;
-    p.ktc_nacc = 512 / p.ktc_acc_cols;
-    if (p.ktc_nacc > 4) p.ktc_nacc = 4;
     p.ktc_a_bytes = static_cast<uint32_t>(p.ktc_kb) * 128u * 128u;
     p.ktc_b_bytes = static_cast<uint32_t>(p.ktc_kb) * p.ktc_npad * 128u;
-    const uint32_t stage = p.ktc_a_bytes + p.ktc_b_bytes;
-    p.ktc_stages = static_cast<int>(static_cast<uint32_t>(STARKV_KTC_RING_BYTES) / stage);
-    if (p.ktc_stages > 8) p.ktc_stages = 8;
-    p.ktc_tmem = static_cast<uint32_t>(pow2_ceil(p.ktc_nacc * p.ktc_acc_cols));
-    p.ktc_smem = 1024 + static_cast<size_t>(p.ktc_stages) * stage + (2 * p.ktc_stages + 9) * sizeof(uint64_t) +
-                 (kKTCSegBufs * p.H + kKTCSegBufs) * sizeof(float);
-    p.ktc = p.ktc_stages >= 2 && p.ktc_nacc >= 2 && p.ktc_tmem <= 512;
+    for (int ctas = STARKV_KTC_CTAS_PER_SM; ctas >= 1 && !p.ktc; ctas = ctas > 1 ? 1 : 0) {
+      const uint32_t budget = static_cast<uint32_t>(STARKV_KTC_SMEM_BYTES) / ctas;
+      p.ktc_nacc = 512 / ctas / p.ktc_npad;
+      if (p.ktc_nacc > 4) p.ktc_nacc = 4;
+      p.ktc_stages = budget > 2u * p.ktc_b_bytes ? static_cast<int>((budget - 2u * p.ktc_b_bytes) / p.ktc_a_bytes) : 0;
+      if (p.ktc_stages > 12) p.ktc_stages = 12;
+      p.ktc_tmem = static_cast<uint32_t>(pow2_ceil(p.ktc_nacc * p.ktc_npad < 32 ? 32 : p.ktc_nacc * p.ktc_npad));
+      p.ktc_smem = 1024 + static_cast<size_t>(p.ktc_stages) * p.ktc_a_bytes + 2u * p.ktc_b_bytes +
+                   (2 * p.ktc_stages + 13) * sizeof(uint64_t) + (kKTCSegBufs * p.H + kKTCSegBufs) * sizeof(float);
+      p.ktc = p.ktc_stages >= 2 && p.ktc_nacc >= 2 && p.ktc_tmem * ctas <= 512 &&
+              p.ktc_smem * ctas <= 227u * 1024u;
+      if (p.ktc) p.k_ctas = sms * ctas;
+    }
   }
 
   // V pass: R split into ranges of <= 1024 rows (128-row UMMA tiles)
@@ -300,15 +305,15 @@ bool encode_vpool_map(CUtensorMap* map, const void* v_cache, int R, int NB) {
 }
 
 // K pool [num_blocks*16 tokens][Hkv][r] fp16 as a 3-D tensor map {r, Hkv,
-// tokens} with boxes {64 codes, 1 head, box_tokens} and the 128-byte swizzle
-// (codes past r read as zero).
+// tokens} with boxes {64 codes, all Hkv heads, box_tokens} and the 128-byte
+// swizzle (codes past r read as zero).
 bool encode_kpool_map(CUtensorMap* map, const void* k_cache, int r, int Hkv, int NB, uint32_t box_tokens) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(r), static_cast<cuuint64_t>(Hkv),
                         static_cast<cuuint64_t>(NB) * 16};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(r) * 2, static_cast<cuuint64_t>(Hkv) * r * 2};
-  cuuint32_t box[3] = {64, 1, box_tokens};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(Hkv), box_tokens};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult res = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(k_cache), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -369,22 +374,37 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
   return e;
 }
 
-template <int G>
-cudaError_t launch_kpass_tc_g(const DecodePlan& pl, const CUtensorMap& kmap, const CUtensorMap& qmap,
+template <int G, int H>
+cudaError_t launch_kpass_tc_gh(const DecodePlan& pl, const CUtensorMap& kmap, const CUtensorMap& qmap,
+                               const KPassTCParams& tp, cudaStream_t s) {
+  if (!set_smem(kpass_tc_kernel<G, H>, pl.ktc_smem)) return cudaErrorInvalidValue;
+  return launch(kpass_tc_kernel<G, H>, dim3(pl.k_ctas), dim3(kKTCThreads), pl.ktc_smem, s, 1, kmap, qmap, tp);
+}
+
+template <int H>
+cudaError_t launch_kpass_tc_h(const DecodePlan& pl, const CUtensorMap& kmap, const CUtensorMap& qmap,
                               const KPassTCParams& tp, cudaStream_t s) {
-  if (!set_smem(kpass_tc_kernel<G>, pl.ktc_smem)) return cudaErrorInvalidValue;
-  return launch(kpass_tc_kernel<G>, dim3(pl.k_ctas), dim3(kKTCThreads), pl.ktc_smem, s, 1, kmap, qmap, tp);
+  // G = H / Hkv with 1 <= Hkv <= 16 and G >= 2
+  switch (pl.log2G) {
+    case 1: if constexpr (H / 2 <= 16) return launch_kpass_tc_gh<2, H>(pl, kmap, qmap, tp, s); break;
+    case 2: if constexpr (H >= 4) return launch_kpass_tc_gh<(H >= 4 ? 4 : H), H>(pl, kmap, qmap, tp, s); break;
+    case 3: if constexpr (H >= 8) return launch_kpass_tc_gh<(H >= 8 ? 8 : H), H>(pl, kmap, qmap, tp, s); break;
+    case 4: if constexpr (H >= 16) return launch_kpass_tc_gh<(H >= 16 ? 16 : H), H>(pl, kmap, qmap, tp, s); break;
+    case 5: if constexpr (H >= 32) return launch_kpass_tc_gh<(H >= 32 ? 32 : H), H>(pl, kmap, qmap, tp, s); break;
+    case 6: if constexpr (H >= 64) return launch_kpass_tc_gh<(H >= 64 ? 64 : H), H>(pl, kmap, qmap, tp, s); break;
+    default: break;
+  }
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_kpass_tc(const DecodePlan& pl, const CUtensorMap& kmap, const CUtensorMap& qmap,
                             const KPassTCParams& tp, cudaStream_t s) {
-  switch (pl.log2G) {
-    case 1: return launch_kpass_tc_g<2>(pl, kmap, qmap, tp, s);
-    case 2: return launch_kpass_tc_g<4>(pl, kmap, qmap, tp, s);
-    case 3: return launch_kpass_tc_g<8>(pl, kmap, qmap, tp, s);
-    case 4: return launch_kpass_tc_g<16>(pl, kmap, qmap, tp, s);
-    case 5: return launch_kpass_tc_g<32>(pl, kmap, qmap, tp, s);
-    default: return launch_kpass_tc_g<64>(pl, kmap, qmap, tp, s);
+  switch (pl.H) {
+    case 4: return launch_kpass_tc_h<4>(pl, kmap, qmap, tp, s);
+    case 8: return launch_kpass_tc_h<8>(pl, kmap, qmap, tp, s);
+    case 16: return launch_kpass_tc_h<16>(pl, kmap, qmap, tp, s);
+    case 32: return launch_kpass_tc_h<32>(pl, kmap, qmap, tp, s);
+    default: return launch_kpass_tc_h<64>(pl, kmap, qmap, tp, s);
   }
 }
 
@@ -625,10 +645,10 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
     KPassTCParams tp;
     tp.tables = block_tables; tp.teff = teff; tp.prefix = prefix;
     tp.logits = logits; tp.mpart = mpart; tp.status = status;
-    tp.B = batch; tp.H = pl.H; tp.log2G = pl.log2G; tp.log2Hkv = pl.log2H - pl.log2G;
+    tp.B = batch; tp.log2G = pl.log2G; tp.log2Hkv = pl.log2H - pl.log2G;
     tp.MB = pl.MB; tp.NB = pl.NB; tp.t_pad = pl.t_pad;
     tp.log2tpt = pl.ktc_log2tpt; tp.ksteps = pl.ktc_ksteps; tp.kb = pl.ktc_kb; tp.npad = pl.ktc_npad;
-    tp.acc_cols = pl.ktc_acc_cols; tp.nacc = pl.ktc_nacc; tp.ncol = pl.ktc_ncol; tp.stages = pl.ktc_stages;
+    tp.nacc = pl.ktc_nacc; tp.stages = pl.ktc_stages;
     tp.a_bytes = pl.ktc_a_bytes; tp.b_bytes = pl.ktc_b_bytes; tp.tmem_cols = pl.ktc_tmem;
     e = launch_kpass_tc(pl, kmap, qmap, tp, s);
   } else if (pl.L == 1 && pl.CPT == 4) e = launch_kpass<1, 4>(pl, kp, s);

@@ -373,6 +373,27 @@ def test_compress_store_prefill_then_decode():
     assert_close({0: got[0]}, {0: ref[0]})
 
 
+@pytest.mark.parametrize("kv_heads", [0, 8])
+def test_decode_independent_of_workspace_contents(kv_heads):
+    """Two runs over a workspace pre-filled with 0x00 and with 0xFF (NaN) bytes agree bit for bit."""
+    sh = W.LayerShape(32, 128, 64, 512, num_kv_heads=kv_heads)
+    wl = W.custom("ws", 4040 + kv_heads, sh, [1, 15, 16, 17, 300, 0, 1000, 129], append=False)
+    Ld = D.device_layer(wl, 0)
+    desc = desc_of(Ld)
+    B, T = wl.batch, wl.max_seq_len
+    wsb = S.starkv_decode_workspace_bytes(desc, B, T)
+    outs = []
+    for fill in (0x00, 0xFF):
+        ws = torch.full((wsb,), fill, dtype=torch.uint8, device="cuda")
+        out = torch.full((B, Ld["H"], Ld["d"]), float("nan"), dtype=torch.float16, device="cuda")
+        S.starkv_paged_decode(desc, B, T, Ld["q"], Ld["B_K"], Ld["B_V"], Ld["k_cache"], Ld["v_cache"],
+                              Ld["tables"], Ld["seq_lens"], Ld["scale"], ws, wsb, out)
+        st, flags = S.starkv_decode_check(ws)
+        assert st == 0, (S.STATUS[st], flags)
+        outs.append(out.cpu().numpy())
+    assert np.array_equal(outs[0].view(np.uint16), outs[1].view(np.uint16))
+
+
 # ------------------------------------------------ grouped-query attention
 
 @pytest.mark.parametrize("H,Hkv,d,r,R", [
@@ -427,9 +448,14 @@ def test_grouped_query_descriptor_checks():
     assert S.starkv_decode_workspace_bytes(d, 4, 100) > 0
 
 
-def test_decode_and_append_batch_over_256():
-    """300 short sequences: several 256-row batch tiles in the append GEMM and the up-projection."""
-    sh = W.LayerShape(32, 128, 64, 2048)
+@pytest.mark.parametrize("kv_heads", [0, 8])
+def test_decode_and_append_batch_over_256(kv_heads):
+    """300 short sequences: several 256-row batch tiles in the append GEMM and the up-projection.
+
+    With 8 KV heads, most K-pass segments are one page long, so the query tiles
+    change slot at almost every tile.
+    """
+    sh = W.LayerShape(32, 128, 64, 2048 if not kv_heads else 512, num_kv_heads=kv_heads)
     rng = np.random.default_rng(5)
     wl = W.custom("wide", 5150, sh, rng.integers(1, 48, size=300), append=True)
     Lh, Ld, appended = _append_check(wl)
