@@ -419,14 +419,17 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
 // page {64 codes, Hkv heads, min(16, tpt) tokens} with the 128-byte swizzle,
 // which is the K-major operand layout.  B holds the sequence's absorbed
 // queries for all H heads split into an fp16 high part (row h) and the fp16
-// rounding of the remainder (row H+h), so D[row, h] + D[row, H+h] is
-// c_K . q~_h with q~ carried to about 22 bits and fp32 accumulation; it is
-// loaded once per (sequence, CTA) segment into one of two slots.  A row uses
-// only the G columns of its own KV head; the tensor cores compute all 2H,
-// which at G >= 2 still costs less than the HBM time of the tile.  The
-// epilogue (4 warps, one TMEM lane quarter each) adds hi + lo for its row's G
-// heads, stores them as one contiguous vector (a warp writes whole logit rows)
-// and keeps running maxima, merged per segment in shared memory.  Several
+// rounding of the remainder (row H+h); each K step issues one MMA against the
+// high rows and one against the low rows into the same accumulator, so
+// D[row, h] = c_K . q~_h with q~ carried to about 22 bits and fp32
+// accumulation; it is
+// loaded once per (sequence, CTA) segment into one of nbs slots (with one
+// slot, a new segment's queries wait until the previous segment's MMAs end).
+// A row uses only the G columns of its own KV head; the tensor cores compute
+// all H, which at G >= 2 still costs less than the HBM time of the tile.  The
+// epilogue (4 warps, one TMEM lane quarter each) picks its row's G columns,
+// stores them as one contiguous vector (a warp writes whole logit rows) and
+// keeps running maxima, merged per segment in shared memory.  Several
 // accumulators let the tensor cores run ahead of the epilogue.
 struct KPassTCParams {
   const int32_t* tables;      // [B][MB]
@@ -439,11 +442,13 @@ struct KPassTCParams {
   int log2tpt;                // tokens per tile = 128 / Hkv
   int ksteps;                 // UMMA K steps of 16 codes: ceil(r/16)
   int kb;                     // 64-code column blocks: ceil(r/64)
-  int npad;                   // UMMA N = max(16, 2H)
-  int nacc;                   // accumulators in TMEM (2..4), npad columns each
+  int nmma;                   // UMMA N = max(16, H): TMEM columns per accumulator
+  int brows;                  // rows of a query tile: 2H (H >= 16) or 32
+  int nacc;                   // accumulators in TMEM (2..4)
+  int nbs;                    // query-tile slots (1 or 2)
   int stages;
   uint32_t a_bytes;           // kb * 128 rows * 128 bytes
-  uint32_t b_bytes;           // kb * npad * 128 bytes
+  uint32_t b_bytes;           // kb * brows * 128 bytes
   uint32_t tmem_cols;
 };
 
@@ -485,8 +490,8 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages;
-  uint8_t* bslot = smem + static_cast<size_t>(S) * p.a_bytes;                    // [2] query tiles
-  uint64_t* full = reinterpret_cast<uint64_t*>(bslot + 2 * static_cast<size_t>(p.b_bytes));
+  uint8_t* bslot = smem + static_cast<size_t>(S) * p.a_bytes;                    // [nbs] query tiles
+  uint64_t* full = reinterpret_cast<uint64_t*>(bslot + p.nbs * static_cast<size_t>(p.b_bytes));
   uint64_t* empty = full + S;
   uint64_t* bfull = empty + S;     // [2] query tile landed
   uint64_t* bempty = bfull + 2;    // [2] query tile no longer read by the tensor cores
@@ -547,14 +552,14 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
     bool ok = true;
     for_each_k_tile(p, p0, p1, [&](int32_t b, int32_t t0, int32_t nt, int64_t x0, bool first, bool last) {
       if (first) {
-        const int bs = seg & 1;
+        const uint32_t bs = seg % p.nbs, buse = seg / p.nbs;
         if (lane == 0) {
-          if (seg >= 2 && !mbar_wait(&bempty[bs], ((seg >> 1) - 1) & 1)) {
+          if (buse > 0 && !mbar_wait(&bempty[bs], (buse - 1) & 1)) {
             ok = false;
           } else {
             mbar_arrive_expect_tx(&bfull[bs], p.b_bytes);
             for (int a = 0; a < p.kb; ++a)
-              tma_load_2d(bslot + bs * static_cast<size_t>(p.b_bytes) + static_cast<size_t>(a) * p.npad * 128, &qmap,
+              tma_load_2d(bslot + bs * static_cast<size_t>(p.b_bytes) + static_cast<size_t>(a) * p.brows * 128, &qmap,
                           a * 64, b * 2 * H, &bfull[bs], reuse);
           }
         }
@@ -602,25 +607,27 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
-      const uint32_t idesc = idesc_f16_f32(128, p.npad, /*a_mn_major=*/false, /*b_mn_major=*/false);
+      const uint32_t idesc = idesc_f16_f32(128, p.nmma, /*a_mn_major=*/false, /*b_mn_major=*/false);
       uint32_t k = 0, seg = 0;
       bool ok = true;
       for_each_k_tile(p, p0, p1, [&](int32_t, int32_t, int32_t, int64_t, bool first, bool last) {
         const int s = k % S;
-        const int bs = seg & 1;
+        const uint32_t bs = seg % p.nbs;
         const uint32_t acc = k % p.nacc, use = k / p.nacc;
-        if (first && !mbar_wait(&bfull[bs], (seg >> 1) & 1)) { ok = false; return false; }
+        if (first && !mbar_wait(&bfull[bs], (seg / p.nbs) & 1)) { ok = false; return false; }
         if (use > 0 && !mbar_wait(&tempty[acc], (use - 1) & 1)) { ok = false; return false; }
         if (!mbar_wait(&full[s], (k / S) & 1) || abort_flag) { ok = false; return false; }
         tc_fence_after();
         // descriptors of the stage / query slot; a K step adds its byte offset >> 4 to the start field
         const uint64_t da = smem_desc(smem_u32(smem + static_cast<size_t>(s) * p.a_bytes), 16u, 1024u, kSwizzle128B);
         const uint64_t db = smem_desc(smem_u32(bslot + bs * static_cast<size_t>(p.b_bytes)), 16u, 1024u, kSwizzle128B);
-        const uint32_t d = taddr + acc * static_cast<uint32_t>(p.npad);
-        const uint32_t b_atom = static_cast<uint32_t>(p.npad) * 8u;     // npad * 128 bytes >> 4
+        const uint32_t d = taddr + acc * static_cast<uint32_t>(p.nmma);
+        const uint32_t b_atom = static_cast<uint32_t>(p.brows) * 8u;    // brows * 128 bytes >> 4
         for (int ks = 0; ks < p.ksteps; ++ks) {
           const uint32_t a = ks >> 2, kk = ks & 3;
-          umma_f16_ss(d, da + (a * 1024u + kk * 2u), db + (a * b_atom + kk * 2u), idesc, ks > 0 ? 1u : 0u);
+          const uint64_t dak = da + (a * 1024u + kk * 2u), dbk = db + (a * b_atom + kk * 2u);
+          umma_f16_ss(d, dak, dbk, idesc, ks > 0 ? 1u : 0u);                    // high parts (rows 0..)
+          umma_f16_ss(d, dak, dbk + static_cast<uint32_t>(H) * 8u, idesc, 1u);  // low parts (rows H..)
         }
         umma_commit(&empty[s]);
         umma_commit(&tfull[acc]);
@@ -650,35 +657,18 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       const uint32_t acc = k % p.nacc, use = k / p.nacc;
       if (!mbar_wait(&tfull[acc], use & 1) || abort_flag) { ok = false; return false; }
       tc_fence_after();
-      const uint32_t tbase = taddr + (static_cast<uint32_t>(q * 32) << 16) + acc * static_cast<uint32_t>(p.npad);
+      const uint32_t tbase = taddr + (static_cast<uint32_t>(q * 32) << 16) + acc * static_cast<uint32_t>(p.nmma);
       float o[G];
-      if constexpr (H >= 32) {
 #pragma unroll
-        for (int ch = 0; ch < H / 32; ++ch) {     // hi and lo of 32 heads per round, one wait
-          uint32_t hi[32], lo[32];
-          tmem_ld_32x32b_x32(tbase + ch * 32, hi);
-          tmem_ld_32x32b_x32(tbase + H + ch * 32, lo);
-          tmem_ld_wait();
+      for (int ch = 0; ch < (H + 15) / 16; ++ch) {   // 16 query heads per load
+        uint32_t v[32];
+        tmem_ld_32x32b_x16(tbase + ch * 16, v);
+        tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int col = ch * 32 + c;
-            if ((col / G) == j) o[col % G] = __uint_as_float(hi[c]) + __uint_as_float(lo[c]);
-          }
+        for (int c = 0; c < 16; ++c) {
+          const int col = ch * 16 + c;
+          if (col < H && (col / G) == j) o[col % G] = __uint_as_float(v[c]);
         }
-      } else if constexpr (H == 16) {
-        uint32_t v[32];                              // columns [0, 16) hi, [16, 32) lo
-        tmem_ld_32x32b_x32(tbase, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          if ((c / G) == j) o[c % G] = __uint_as_float(v[c]) + __uint_as_float(v[16 + c]);
-      } else {
-        uint32_t v[32];                              // columns [0, H) hi, [H, 2H) lo
-        tmem_ld_32x32b_x16(tbase, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < H; ++c)
-          if ((c / G) == j) o[c % G] = __uint_as_float(v[c]) + __uint_as_float(v[H + c]);
       }
       tc_fence_before();
       __syncwarp();
@@ -821,36 +811,55 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tensormap(&vmap);
-      const uint64_t pol_codes = policy_evict_first();
-      const uint64_t pol_logits = policy_evict_first();
-      uint32_t k = 0;
-      bool ok = true;
-      int32_t b = seq_of_page(p.prefix, p.B, p0);
-      const int c_base = rr * (p.r_range / 64);
-      const int n_ch = min(p.n_chunks, (p.R - rr * p.r_range + 63) / 64);
-      for (int64_t pg_g = p0; pg_g < p1; ++pg_g, ++k) {
-        while (p.prefix[b + 1] <= pg_g) ++b;
-        const int32_t pg = static_cast<int32_t>(pg_g - p.prefix[b]);
-        const int32_t npg = p.prefix[b + 1] - p.prefix[b];
-        const int32_t T = p.teff[b];
-        int32_t phys = p.tables[static_cast<size_t>(b) * p.MB + pg];
+    // The whole warp walks the pages; lane i reads ahead the block-table entry
+    // of page cbase + i, so lane 0 issues copies without a dependent global
+    // load per page.  Sequence bounds are reloaded only when the walk enters
+    // the next sequence.
+    if (lane == 0) prefetch_tensormap(&vmap);
+    const uint64_t pol_codes = policy_evict_first();
+    const uint64_t pol_logits = policy_evict_first();
+    uint32_t k = 0;
+    bool ok = true;
+    int32_t b = seq_of_page(p.prefix, p.B, p0);
+    int32_t sbeg = p.prefix[b], send = p.prefix[b + 1], T = p.teff[b];
+    int64_t cbase = -64;
+    int32_t cphys = 0;
+    const int c_base = rr * (p.r_range / 64);
+    for (int64_t pg_g = p0; pg_g < p1; ++pg_g, ++k) {
+      while (send <= pg_g) { ++b; sbeg = send; send = p.prefix[b + 1]; T = p.teff[b]; }
+      if (pg_g >= cbase + 32) {
+        cbase = pg_g;
+        const int64_t xi = pg_g + lane;
+        int32_t bi = b;
+        while (bi < p.B - 1 && p.prefix[bi + 1] <= xi) ++bi;
+        cphys = xi < p1 ? p.tables[static_cast<size_t>(bi) * p.MB + static_cast<int32_t>(xi - p.prefix[bi])] : 0;
+      }
+      int32_t phys = __shfl_sync(0xffffffffu, cphys, static_cast<int>(pg_g - cbase));
+      if (lane == 0) {
+        const int32_t pg = static_cast<int32_t>(pg_g - sbeg);
+        const int32_t npg = send - sbeg;
         if (phys < 0 || phys >= p.NB) { set_flag(p.status, STARKV_FLAG_BAD_BLOCK_ID); phys = 0; }
         const int s = k % S;
-        if (k >= static_cast<uint32_t>(S) && !mbar_wait(&empty[s], ((k / S) - 1) & 1)) { ok = false; break; }
-        int32_t fl = 0;
-        if (pg_g == p0 || pg == 0) fl |= kFirst;
-        if (pg_g == p1 - 1 || pg == npg - 1) fl |= kLast;
-        meta[s] = StageMeta{b, pg * kBlock, min(kBlock, T - pg * kBlock), fl};
-        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(n_ch) * 2048u + p.ltile_bytes);
-        uint8_t* vt = vtiles + static_cast<size_t>(s) * p.vtile_bytes;
-        for (int c = 0; c < n_ch; ++c)
-          tma_load_2d(vt + c * 2048, &vmap, (c_base + c) * 64, phys * kBlock, &full[s], pol_codes);
-        bulk_g2s(ltiles + static_cast<size_t>(s) * p.ltile_bytes,
-                 p.logits + (static_cast<size_t>(b) * p.t_pad + pg * kBlock) * p.H, p.ltile_bytes,
-                 &full[s], pol_logits);
+        if (k >= static_cast<uint32_t>(S) && !mbar_wait(&empty[s], ((k / S) - 1) & 1)) {
+          ok = false;
+        } else {
+          int32_t fl = 0;
+          if (pg_g == p0 || pg == 0) fl |= kFirst;
+          if (pg_g == p1 - 1 || pg == npg - 1) fl |= kLast;
+          meta[s] = StageMeta{b, pg * kBlock, min(kBlock, T - pg * kBlock), fl};
+          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(p.n_chunks) * 2048u + p.ltile_bytes);
+          // the page's R range in one box of n_chunks 64-code blocks
+          tma_load_3d(vtiles + static_cast<size_t>(s) * p.vtile_bytes, &vmap, 0, phys * kBlock, c_base, &full[s],
+                      pol_codes);
+          bulk_g2s(ltiles + static_cast<size_t>(s) * p.ltile_bytes,
+                   p.logits + (static_cast<size_t>(b) * p.t_pad + pg * kBlock) * p.H, p.ltile_bytes,
+                   &full[s], pol_logits);
+        }
       }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+    }
+    if (lane == 0) {
       if (ok) {
         const int s = k % S;
         if (k >= static_cast<uint32_t>(S) && !mbar_wait(&empty[s], ((k / S) - 1) & 1)) ok = false;

@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstring>
 #include <map>
+#include <tuple>
 #include <mutex>
 #include <utility>
 
@@ -22,10 +23,10 @@
 #define STARKV_K_STAGE_CAP 65536
 #endif
 #ifndef STARKV_KTC_CTAS_PER_SM
-#define STARKV_KTC_CTAS_PER_SM 2
+#define STARKV_KTC_CTAS_PER_SM 3
 #endif
 #ifndef STARKV_KTC_SMEM_BYTES
-#define STARKV_KTC_SMEM_BYTES (216 * 1024)   // stage ring + query slots of the CTAs on one SM
+#define STARKV_KTC_SMEM_BYTES (208 * 1024)   // shared memory of the K-pass CTAs on one SM
 #endif
 #ifndef STARKV_K_RING_BYTES
 #define STARKV_K_RING_BYTES (200 * 1024 / STARKV_K_CTAS_PER_SM)
@@ -88,7 +89,7 @@ struct DecodePlan {
   size_t k_smem;
   // K pass on tensor cores (grouped queries)
   bool ktc;
-  int ktc_log2tpt, ktc_ksteps, ktc_kb, ktc_npad, ktc_nacc, ktc_stages;
+  int ktc_log2tpt, ktc_ksteps, ktc_kb, ktc_nmma, ktc_brows, ktc_nacc, ktc_nbs, ktc_stages;
   uint32_t ktc_a_bytes, ktc_b_bytes, ktc_tmem;
   size_t ktc_smem;
   // V pass
@@ -110,6 +111,85 @@ void plan_kpass_shape(int r, int* L, int* CPT) {
   else if (cp <= 12) { *L = 1; *CPT = 12; } // r <= 96
   else if (cp <= 16) { *L = 2; *CPT = 8; }  // r <= 128
   else { *L = 4; *CPT = 8; }                // r <= 256
+}
+
+// ------------------------------------------------------ kernel attributes
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device), and
+// again only when a larger size is needed.
+template <typename K>
+bool set_smem(K kernel, size_t bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> set_bytes;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return false; }
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = set_bytes.find(key);
+  if (it != set_bytes.end() && it->second >= static_cast<int>(bytes)) return true;
+  // the largest shared-memory carveout, so that as many CTAs as the plan
+  // counts on fit on one SM
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           static_cast<int>(cudaSharedmemCarveoutMaxShared)) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  set_bytes[key] = static_cast<int>(bytes);
+  return true;
+}
+
+// CTAs of the tensor-core K pass (instance <G, H>) that fit on one SM by
+// registers (the kernel's count, allocated per warp in units of 256) and by
+// shared memory (`smem` bytes each within STARKV_KTC_SMEM_BYTES per SM).
+template <int G, int H>
+int ktc_occupancy(size_t smem) {
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kpass_tc_kernel<G, H>) != cudaSuccess) { cudaGetLastError(); return 0; }
+  // 10% margin: an instance at 109 registers measured at two resident CTAs, not three
+  const int per_warp = (fa.numRegs * 32 + 255) / 256 * 256;
+  const int by_regs = 65536 * 10 / (per_warp * (kKTCThreads / 32) * 11);
+  const int by_smem = static_cast<int>(static_cast<size_t>(STARKV_KTC_SMEM_BYTES) / (smem + 1024));
+  return by_regs < by_smem ? by_regs : by_smem;
+}
+
+template <int H>
+int ktc_occupancy_h(int log2G, size_t smem) {
+  switch (log2G) {
+    case 1: if constexpr (H / 2 <= 16) return ktc_occupancy<2, H>(smem); break;
+    case 2: if constexpr (H >= 4 && H / 4 <= 16) return ktc_occupancy<(H >= 4 ? 4 : H), H>(smem); break;
+    case 3: if constexpr (H >= 8) return ktc_occupancy<(H >= 8 ? 8 : H), H>(smem); break;
+    case 4: if constexpr (H >= 16) return ktc_occupancy<(H >= 16 ? 16 : H), H>(smem); break;
+    case 5: if constexpr (H >= 32) return ktc_occupancy<(H >= 32 ? 32 : H), H>(smem); break;
+    case 6: if constexpr (H >= 64) return ktc_occupancy<(H >= 64 ? 64 : H), H>(smem); break;
+    default: break;
+  }
+  return 0;
+}
+
+int ktc_resident_ctas(int log2G, int H, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, size_t, int>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return 0; }
+  const auto key = std::make_tuple(log2G, H, smem, dev);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  int n = 0;
+  switch (H) {
+    case 4: n = ktc_occupancy_h<4>(log2G, smem); break;
+    case 8: n = ktc_occupancy_h<8>(log2G, smem); break;
+    case 16: n = ktc_occupancy_h<16>(log2G, smem); break;
+    case 32: n = ktc_occupancy_h<32>(log2G, smem); break;
+    case 64: n = ktc_occupancy_h<64>(log2G, smem); break;
+    default: break;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = n;
+  return n;
 }
 
 starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_seq_len, DecodePlan* pl) {
@@ -151,30 +231,39 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   p.k_ctas = sms * STARKV_K_CTAS_PER_SM;
 
   // Grouped queries (G >= 2, H >= 4) with at most 16 KV heads: the K pass runs
-  // on the tensor cores, with STARKV_KTC_CTAS_PER_SM CTAs per SM when their
-  // rings (>= 2 stages) and accumulators fit, else with one.
+  // on the tensor cores.  Its per-CTA pipeline (one page per stage, one tile in
+  // the epilogue at a time) is latency-bound, so the plan takes the most CTAs
+  // per SM that fit (registers of the kernel instance, shared memory, TMEM),
+  // each with at least three stages (two for a single CTA), and two query
+  // slots where they fit.
   p.ktc = false;
-  if (p.log2G >= 1 && p.H >= 4 && p.Hkv <= 16) {
+  if (p.log2G >= 1 && p.H >= 8 && p.Hkv <= 16) {
     int log2Hkv = 0;
     while ((1 << log2Hkv) < p.Hkv) ++log2Hkv;
     p.ktc_log2tpt = 7 - log2Hkv;
     p.ktc_ksteps = (p.r + 15) / 16;
     p.ktc_kb = (p.r + 63) / 64;
-    p.ktc_npad = 2 * p.H < 16 ? 16 : 2 * p.H;
+    p.ktc_nmma = p.H < 16 ? 16 : p.H;
+    p.ktc_brows = p.H < 16 ? 32 : 2 * p.H;   // the low-part MMA reads rows [H, H + nmma)
     p.ktc_a_bytes = static_cast<uint32_t>(p.ktc_kb) * 128u * 128u;
-    p.ktc_b_bytes = static_cast<uint32_t>(p.ktc_kb) * p.ktc_npad * 128u;
-    for (int ctas = STARKV_KTC_CTAS_PER_SM; ctas >= 1 && !p.ktc; ctas = ctas > 1 ? 1 : 0) {
-      const uint32_t budget = static_cast<uint32_t>(STARKV_KTC_SMEM_BYTES) / ctas;
-      p.ktc_nacc = 512 / ctas / p.ktc_npad;
-      if (p.ktc_nacc > 4) p.ktc_nacc = 4;
-      p.ktc_stages = budget > 2u * p.ktc_b_bytes ? static_cast<int>((budget - 2u * p.ktc_b_bytes) / p.ktc_a_bytes) : 0;
-      if (p.ktc_stages > 12) p.ktc_stages = 12;
-      p.ktc_tmem = static_cast<uint32_t>(pow2_ceil(p.ktc_nacc * p.ktc_npad < 32 ? 32 : p.ktc_nacc * p.ktc_npad));
-      p.ktc_smem = 1024 + static_cast<size_t>(p.ktc_stages) * p.ktc_a_bytes + 2u * p.ktc_b_bytes +
-                   (2 * p.ktc_stages + 13) * sizeof(uint64_t) + (kKTCSegBufs * p.H + kKTCSegBufs) * sizeof(float);
-      p.ktc = p.ktc_stages >= 2 && p.ktc_nacc >= 2 && p.ktc_tmem * ctas <= 512 &&
-              p.ktc_smem * ctas <= 227u * 1024u;
-      if (p.ktc) p.k_ctas = sms * ctas;
+    p.ktc_b_bytes = static_cast<uint32_t>(p.ktc_kb) * p.ktc_brows * 128u;
+    for (int ctas = STARKV_KTC_CTAS_PER_SM; ctas >= 1 && !p.ktc; --ctas) {
+      for (int nbs = 2; nbs >= 1 && !p.ktc; --nbs) {
+        const uint32_t budget = static_cast<uint32_t>(STARKV_KTC_SMEM_BYTES) / ctas - 1024u;
+        const uint32_t fixed = 1024u + nbs * p.ktc_b_bytes + 13u * 8u + (kKTCSegBufs * p.H + kKTCSegBufs) * 4u;
+        if (budget <= fixed) continue;
+        int stages = static_cast<int>((budget - fixed) / (p.ktc_a_bytes + 16u));
+        if (stages > 12) stages = 12;
+        int nacc = 512 / ctas / p.ktc_nmma;
+        if (nacc > 4) nacc = 4;
+        const uint32_t tmem = static_cast<uint32_t>(pow2_ceil(nacc * p.ktc_nmma < 32 ? 32 : nacc * p.ktc_nmma));
+        if (stages < (ctas > 1 ? 3 : 2) || nacc < 2 || tmem * ctas > 512) continue;
+        const size_t smem = fixed + static_cast<size_t>(stages) * (p.ktc_a_bytes + 16u);
+        if (ktc_resident_ctas(p.log2G, p.H, smem) < ctas) continue;
+        p.ktc = true;
+        p.ktc_stages = stages; p.ktc_nacc = nacc; p.ktc_nbs = nbs; p.ktc_tmem = tmem; p.ktc_smem = smem;
+        p.k_ctas = sms * ctas;
+      }
     }
   }
 
@@ -298,10 +387,22 @@ bool encode_2d_map(CUtensorMap* map, const void* base, uint64_t cols, uint64_t r
   return r == CUDA_SUCCESS;
 }
 
-// V pool viewed as a 2-D matrix [num_blocks*16 rows][R] of fp16; boxes of
-// 64 columns x 16 rows (one page, one 128-byte-wide chunk).
-bool encode_vpool_map(CUtensorMap* map, const void* v_cache, int R, int NB) {
-  return encode_2d_map(map, v_cache, static_cast<uint64_t>(R), static_cast<uint64_t>(NB) * 16, 64, 16);
+// V pool [num_blocks*16 tokens][R] fp16 as a 3-D tensor map {64 codes, tokens,
+// R/64 column blocks} (strides: a token row, then 128 bytes per block) with
+// boxes {64, 16 tokens, box_chunks}: one copy brings a page's R range as
+// box_chunks consecutive 64-code x 16-token blocks of 2 KiB, each already the
+// 128B-swizzled MN-major operand slice; blocks past R read as zero.
+bool encode_vpool_map(CUtensorMap* map, const void* v_cache, int R, int NB, uint32_t box_chunks) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(NB) * 16, static_cast<cuuint64_t>(R) / 64};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(R) * 2, 128};
+  cuuint32_t box[3] = {64, 16, box_chunks};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult res = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(v_cache), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return res == CUDA_SUCCESS;
 }
 
 // K pool [num_blocks*16 tokens][Hkv][r] fp16 as a 3-D tensor map {r, Hkv,
@@ -319,28 +420,6 @@ bool encode_kpool_map(CUtensorMap* map, const void* k_cache, int r, int Hkv, int
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return res == CUDA_SUCCESS;
-}
-
-// ------------------------------------------------------ kernel attributes
-// Raises a kernel's dynamic shared-memory limit once per (kernel, device), and
-// again only when a larger size is needed.
-template <typename K>
-bool set_smem(K kernel, size_t bytes) {
-  static std::mutex mu;
-  static std::map<std::pair<const void*, int>, int> set_bytes;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return false; }
-  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
-  std::lock_guard<std::mutex> lock(mu);
-  auto it = set_bytes.find(key);
-  if (it != set_bytes.end() && it->second >= static_cast<int>(bytes)) return true;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
-      cudaSuccess) {
-    cudaGetLastError();
-    return false;
-  }
-  set_bytes[key] = static_cast<int>(bytes);
-  return true;
 }
 
 // Every kernel is launched with programmatic stream serialisation: the grid may
@@ -595,7 +674,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   __half* zhi = reinterpret_cast<__half*>(ws + pl.ws.zhi_off);
   __half* zlo = reinterpret_cast<__half*>(ws + pl.ws.zlo_off);
   CUtensorMap vmap, bvmap, zhimap, zlomap;
-  if (!encode_vpool_map(&vmap, v_cache, pl.R, pl.NB)) return STARKV_ERR_CUDA;
+  if (!encode_vpool_map(&vmap, v_cache, pl.R, pl.NB, static_cast<uint32_t>(pl.n_chunks))) return STARKV_ERR_CUDA;
   if (!encode_2d_map(&bvmap, B_V, static_cast<uint64_t>(pl.Hkv) * pl.d, static_cast<uint64_t>(pl.R), 64, kUpKC) ||
       !encode_2d_map(&zhimap, zhi, static_cast<uint64_t>(pl.R), static_cast<uint64_t>(pl.H) * batch, 64,
                      static_cast<uint32_t>(pl.up_npad)) ||
@@ -640,15 +719,16 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
     const uint32_t tpt = 1u << pl.ktc_log2tpt;
     if (!encode_kpool_map(&kmap, k_cache, pl.r, pl.Hkv, pl.NB, tpt < 16 ? tpt : 16) ||
         !encode_2d_map(&qmap, qth, static_cast<uint64_t>(pl.r), static_cast<uint64_t>(batch) * 2 * pl.H, 64,
-                       static_cast<uint32_t>(pl.ktc_npad)))
+                       static_cast<uint32_t>(pl.ktc_brows)))
       return STARKV_ERR_CUDA;
     KPassTCParams tp;
     tp.tables = block_tables; tp.teff = teff; tp.prefix = prefix;
     tp.logits = logits; tp.mpart = mpart; tp.status = status;
     tp.B = batch; tp.log2G = pl.log2G; tp.log2Hkv = pl.log2H - pl.log2G;
     tp.MB = pl.MB; tp.NB = pl.NB; tp.t_pad = pl.t_pad;
-    tp.log2tpt = pl.ktc_log2tpt; tp.ksteps = pl.ktc_ksteps; tp.kb = pl.ktc_kb; tp.npad = pl.ktc_npad;
-    tp.nacc = pl.ktc_nacc; tp.stages = pl.ktc_stages;
+    tp.log2tpt = pl.ktc_log2tpt; tp.ksteps = pl.ktc_ksteps; tp.kb = pl.ktc_kb;
+    tp.nmma = pl.ktc_nmma; tp.brows = pl.ktc_brows;
+    tp.nacc = pl.ktc_nacc; tp.nbs = pl.ktc_nbs; tp.stages = pl.ktc_stages;
     tp.a_bytes = pl.ktc_a_bytes; tp.b_bytes = pl.ktc_b_bytes; tp.tmem_cols = pl.ktc_tmem;
     e = launch_kpass_tc(pl, kmap, qmap, tp, s);
   } else if (pl.L == 1 && pl.CPT == 4) e = launch_kpass<1, 4>(pl, kp, s);
