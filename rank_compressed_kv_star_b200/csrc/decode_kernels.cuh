@@ -82,6 +82,8 @@ struct AbsorbParams {
   int32_t* prefix;        // [B+1]
   int32_t* teff;          // [B] clamped lengths
   int32_t* status;
+  float* mpart_init;      // [n_mpart] set to -inf (segment maxima merged by atomics later); may be null
+  int n_mpart;
   int B, H, d, r, cap;    // cap = min(max_seq_len, max_blocks_per_seq*16)
   int log2G;              // query heads per KV head = 1 << log2G
   float coef;             // scale * log2(e)
@@ -128,6 +130,11 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbParams p) {
       p.prefix[b] = acc;
       acc += (p.teff[b] + kBlock - 1) / kBlock;
     }
+  }
+  if (p.mpart_init) {
+    const int nthr = gridDim.x * gridDim.y * 256;
+    for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * 256 + tid; i < p.n_mpart; i += nthr)
+      p.mpart_init[i] = -INFINITY;
   }
   __shared__ __align__(16) __half qs[kAbsBT * D];
   const int bt0 = blockIdx.y * kAbsBT;
@@ -422,21 +429,24 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
 // rounding of the remainder (row H+h); each K step issues one MMA against the
 // high rows and one against the low rows into the same accumulator, so
 // D[row, h] = c_K . q~_h with q~ carried to about 22 bits and fp32
-// accumulation; it is
-// loaded once per (sequence, CTA) segment into one of nbs slots (with one
-// slot, a new segment's queries wait until the previous segment's MMAs end).
-// A row uses only the G columns of its own KV head; the tensor cores compute
-// all H, which at G >= 2 still costs less than the HBM time of the tile.  The
-// epilogue (4 warps, one TMEM lane quarter each) picks its row's G columns,
+// accumulation.  B is loaded once per (sequence, CTA) segment into one of nbs
+// slots.  A row uses only the G columns of its own KV head; the tensor cores
+// compute all H, which at G >= 2 costs less than the HBM time of the tile.
+//
+// One CTA streams a long ring of pages; the tiles are dealt round-robin to NG
+// consumer groups, each with its own MMA warp, TMEM accumulators and four
+// epilogue warps (one TMEM lane quarter each), so that per-tile latencies of
+// different groups overlap.  An epilogue warp picks its row's G columns,
 // stores them as one contiguous vector (a warp writes whole logit rows) and
-// keeps running maxima, merged per segment in shared memory.  Several
-// accumulators let the tensor cores run ahead of the epilogue.
+// keeps running maxima; at the end of every segment each warp merges them into
+// the segment's maxima in global memory (float max through integer atomics,
+// initialised to -inf by the absorb kernel).
 struct KPassTCParams {
   const int32_t* tables;      // [B][MB]
   const int32_t* teff;        // [B]
   const int32_t* prefix;      // [B+1]
   float* logits;              // [B][t_pad][H]
-  float* mpart;               // [k_slots][H]
+  float* mpart;               // [k_slots][H], -inf on entry
   int32_t* status;
   int B, log2G, log2Hkv, MB, NB, t_pad;
   int log2tpt;                // tokens per tile = 128 / Hkv
@@ -444,7 +454,8 @@ struct KPassTCParams {
   int kb;                     // 64-code column blocks: ceil(r/64)
   int nmma;                   // UMMA N = max(16, H): TMEM columns per accumulator
   int brows;                  // rows of a query tile: 2H (H >= 16) or 32
-  int nacc;                   // accumulators in TMEM (2..4)
+  int ng;                     // consumer groups (1..4)
+  int nacc;                   // accumulators per group
   int nbs;                    // query-tile slots (1 or 2)
   int stages;
   uint32_t a_bytes;           // kb * 128 rows * 128 bytes
@@ -452,8 +463,9 @@ struct KPassTCParams {
   uint32_t tmem_cols;
 };
 
-constexpr int kKTCThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
-constexpr int kKTCSegBufs = 6;     // segment-maximum buffers (warps run at most nacc <= 4 tiles apart)
+constexpr int kKTCMaxGroups = 4;
+constexpr int kKTCMaxAcc = 4;
+__host__ __device__ constexpr int ktc_threads(int ng) { return 32 * (1 + 5 * ng); }
 
 // Calls f(b, t0, nt, x0, first, last) for the K-pass tiles of pages [p0, p1)
 // in order: tokens [t0, t0+nt) of sequence b, whose first token lies in global
@@ -476,44 +488,41 @@ __device__ __forceinline__ void for_each_k_tile(const KPassTCParams& p, int64_t 
   }
 }
 
-// Float maximum into shared memory through the integer atomics (ordered bit
-// patterns: max over signed ints for v >= 0, min over unsigned for v < 0).
-__device__ __forceinline__ void smem_atomic_max_f32(float* addr, float v) {
+// Float maximum through the integer atomics (ordered bit patterns: max over
+// signed ints for v >= 0, min over unsigned for v < 0); works on shared or
+// global memory.
+__device__ __forceinline__ void atomic_max_f32(float* addr, float v) {
   if (__float_as_int(v) >= 0) atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));
   else atomicMin(reinterpret_cast<unsigned int*>(addr), __float_as_uint(v));
 }
 
 template <int G, int H>   // query heads per KV head, query heads
-__global__ void __launch_bounds__(kKTCThreads, 1)
+__global__ void __launch_bounds__(ktc_threads(kKTCMaxGroups), 1)
 kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                 KPassTCParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int S = p.stages;
+  const int S = p.stages, NG = p.ng;
   uint8_t* bslot = smem + static_cast<size_t>(S) * p.a_bytes;                    // [nbs] query tiles
   uint64_t* full = reinterpret_cast<uint64_t*>(bslot + p.nbs * static_cast<size_t>(p.b_bytes));
   uint64_t* empty = full + S;
-  uint64_t* bfull = empty + S;     // [2] query tile landed
-  uint64_t* bempty = bfull + 2;    // [2] query tile no longer read by the tensor cores
-  uint64_t* tfull = bempty + 2;    // [4] accumulator ready
-  uint64_t* tempty = tfull + 4;    // [4] accumulator drained (4 epilogue warps)
-  uint64_t* mmadone = tempty + 4;
-  float* segmax = reinterpret_cast<float*>(mmadone + 1);          // [kKTCSegBufs][H]
-  int32_t* segcnt = reinterpret_cast<int32_t*>(segmax + kKTCSegBufs * H);
+  uint64_t* bfull = empty + S;                     // [2] query tile landed
+  uint64_t* bempty = bfull + 2;                    // [2] query tile no longer read (one commit per group)
+  uint64_t* tfull = bempty + 2;                    // [NG][kKTCMaxAcc] accumulator ready
+  uint64_t* tempty = tfull + kKTCMaxGroups * kKTCMaxAcc;   // [NG][kKTCMaxAcc] accumulator drained
+  uint64_t* mmadone = tempty + kKTCMaxGroups * kKTCMaxAcc; // [NG]
   __shared__ uint32_t taddr_s;
   __shared__ volatile int32_t abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&bfull[a], 1); mbar_init(&bempty[a], 1); }
-    for (int a = 0; a < 4; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
-    mbar_init(mmadone, 1);
+    for (int a = 0; a < 2; ++a) { mbar_init(&bfull[a], 1); mbar_init(&bempty[a], NG); }
+    for (int a = 0; a < kKTCMaxGroups * kKTCMaxAcc; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
+    for (int g = 0; g < kKTCMaxGroups; ++g) mbar_init(&mmadone[g], 1);
     abort_flag = 0;
     fence_mbar_init();
   }
-  for (int i = tid; i < kKTCSegBufs * H; i += kKTCThreads) segmax[i] = -INFINITY;
-  if (tid < kKTCSegBufs) segcnt[tid] = 0;
   griddep_wait();
   griddep_launch_dependents();
   Partition pt;
@@ -534,185 +543,171 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   const int Hkv = 1 << p.log2Hkv;
   const int tb = tpt < kBlock ? tpt : kBlock;       // tokens per TMA box (one page, or half of one)
 
+  // Ring positions are advanced incrementally (no divisions per tile): a ring
+  // of n slots at position (i, u) is slot i in its u-th use.
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // The whole warp walks the tiles; lane i reads ahead the block-table entry
-    // of page cbase + i so that lane 0 never waits on a table load per page.
     if (lane == 0) {
       prefetch_tensormap(&kmap);
       prefetch_tensormap(&qmap);
-    }
-    const uint64_t stream = policy_evict_first();
-    const uint64_t reuse = policy_evict_last();
-    const uint32_t box_bytes = static_cast<uint32_t>(tb) * Hkv * 128u;
-    int64_t cbase = -64;
-    int32_t cphys = 0;
-    int32_t cb = 0;
-    uint32_t k = 0, seg = 0;
-    bool ok = true;
-    for_each_k_tile(p, p0, p1, [&](int32_t b, int32_t t0, int32_t nt, int64_t x0, bool first, bool last) {
-      if (first) {
-        const uint32_t bs = seg % p.nbs, buse = seg / p.nbs;
-        if (lane == 0) {
-          if (buse > 0 && !mbar_wait(&bempty[bs], (buse - 1) & 1)) {
-            ok = false;
-          } else {
-            mbar_arrive_expect_tx(&bfull[bs], p.b_bytes);
-            for (int a = 0; a < p.kb; ++a)
-              tma_load_2d(bslot + bs * static_cast<size_t>(p.b_bytes) + static_cast<size_t>(a) * p.brows * 128, &qmap,
-                          a * 64, b * 2 * H, &bfull[bs], reuse);
-          }
+      const uint64_t stream = policy_evict_first();
+      const uint64_t reuse = policy_evict_last();
+      const uint32_t box_bytes = static_cast<uint32_t>(tb) * Hkv * 128u;
+      const int log2tb = tpt < kBlock ? p.log2tpt : 4;
+      int si = 0, bi = 0;
+      uint32_t su = 0, bu = 0, issued = 0;
+      bool ok = true;
+      for_each_k_tile(p, p0, p1, [&](int32_t b, int32_t t0, int32_t nt, int64_t x0, bool first, bool last) {
+        if (first) {
+          if (bu > 0 && !mbar_wait(&bempty[bi], (bu - 1) & 1)) { ok = false; return false; }
+          mbar_arrive_expect_tx(&bfull[bi], p.b_bytes);
+          for (int a = 0; a < p.kb; ++a)
+            tma_load_2d(bslot + bi * static_cast<size_t>(p.b_bytes) + static_cast<size_t>(a) * p.brows * 128, &qmap,
+                        a * 64, b * 2 * H, &bfull[bi], reuse);
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) return false;
-      }
-      const int s = k % S;
-      if (lane == 0 && k >= static_cast<uint32_t>(S) && !mbar_wait(&empty[s], ((k / S) - 1) & 1)) ok = false;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) return false;
-      uint8_t* st = smem + static_cast<size_t>(s) * p.a_bytes;
-      const int nbox = (nt + tb - 1) / tb;
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox * p.kb) * box_bytes);
-      for (int c = 0; c < nbox; ++c) {
-        const int32_t t = t0 + c * tb;
-        const int64_t x = x0 + (((t0 & (kBlock - 1)) + c * tb) >> 4);      // global page index
-        if (x < cbase || x >= cbase + 32) {                                  // uniform over the warp
-          cbase = x;
-          cb = b;
-          const int64_t xi = x + lane;
-          int32_t bi = b;
-          while (bi < p.B - 1 && p.prefix[bi + 1] <= xi) ++bi;
-          cphys = xi < p1 ? p.tables[static_cast<size_t>(bi) * p.MB + static_cast<int32_t>(xi - p.prefix[bi])] : 0;
-        }
-        int32_t phys = __shfl_sync(0xffffffffu, cphys, static_cast<int>(x - cbase));
-        if (lane == 0) {
+        if (su > 0 && !mbar_wait(&empty[si], (su - 1) & 1)) { ok = false; return false; }
+        uint8_t* st = smem + static_cast<size_t>(si) * p.a_bytes;
+        const int nbox = (nt + tb - 1) >> log2tb;
+        mbar_arrive_expect_tx(&full[si], static_cast<uint32_t>(nbox * p.kb) * box_bytes);
+        const int32_t* trow = p.tables + static_cast<size_t>(b) * p.MB;
+        for (int c = 0; c < nbox; ++c) {
+          const int32_t t = t0 + c * tb;
+          int32_t phys = trow[t >> 4];
           if (phys < 0 || phys >= p.NB) { set_flag(p.status, STARKV_FLAG_BAD_BLOCK_ID); phys = 0; }
           const int32_t row = phys * kBlock + (t & (kBlock - 1));
           for (int a = 0; a < p.kb; ++a)
             tma_load_3d(st + static_cast<size_t>(a) * 16384 + static_cast<size_t>(c) * box_bytes, &kmap, a * 64, 0,
-                        row, &full[s], stream);
+                        row, &full[si], stream);
+        }
+        ++issued;
+        if (++si == S) { si = 0; ++su; }
+        if (last && ++bi == p.nbs) { bi = 0; ++bu; }
+        return true;
+      });
+      if (!ok) {
+        set_timeout(p.status, kSiteKEmpty);
+        abort_flag = 1;
+        // let the copies in flight land: the last min(issued, S) stages
+        int i = si;
+        uint32_t u = su;
+        for (uint32_t n = 0; n < issued && n < static_cast<uint32_t>(S); ++n) {
+          if (--i < 0) { i = S - 1; --u; }
+          mbar_wait(&full[i], u & 1);
         }
       }
-      ++k;
-      if (last) ++seg;
-      return true;
-    });
-    (void)cb;
-    if (!ok && lane == 0) {
-      set_timeout(p.status, kSiteKEmpty);
-      abort_flag = 1;
-      const uint32_t first = k > static_cast<uint32_t>(S) ? k - S : 0;
-      for (uint32_t kk = first; kk < k; ++kk) mbar_wait(&full[kk % S], (kk / S) & 1);
     }
-  } else if (warp == 1) {
+  } else if (warp <= NG) {
     // ----------------------------------------------------------------- MMA
+    // Group g = warp - 1 issues the MMAs of tiles k = g (mod NG); every group
+    // commits to the query slot's empty barrier at every segment end.
     if (lane == 0) {
+      const int g = warp - 1;
       const uint32_t idesc = idesc_f16_f32(128, p.nmma, /*a_mn_major=*/false, /*b_mn_major=*/false);
-      uint32_t k = 0, seg = 0;
+      const uint32_t b_atom = static_cast<uint32_t>(p.brows) * 8u;    // brows * 128 bytes >> 4
+      const uint32_t tcol0 = taddr + static_cast<uint32_t>(g * p.nacc * p.nmma);
+      int r = 0, si = 0, bi = 0, ai = 0;
+      uint32_t su = 0, bu = 0, au = 0;
       bool ok = true;
       for_each_k_tile(p, p0, p1, [&](int32_t, int32_t, int32_t, int64_t, bool first, bool last) {
-        const int s = k % S;
-        const uint32_t bs = seg % p.nbs;
-        const uint32_t acc = k % p.nacc, use = k / p.nacc;
-        if (first && !mbar_wait(&bfull[bs], (seg / p.nbs) & 1)) { ok = false; return false; }
-        if (use > 0 && !mbar_wait(&tempty[acc], (use - 1) & 1)) { ok = false; return false; }
-        if (!mbar_wait(&full[s], (k / S) & 1) || abort_flag) { ok = false; return false; }
-        tc_fence_after();
-        // descriptors of the stage / query slot; a K step adds its byte offset >> 4 to the start field
-        const uint64_t da = smem_desc(smem_u32(smem + static_cast<size_t>(s) * p.a_bytes), 16u, 1024u, kSwizzle128B);
-        const uint64_t db = smem_desc(smem_u32(bslot + bs * static_cast<size_t>(p.b_bytes)), 16u, 1024u, kSwizzle128B);
-        const uint32_t d = taddr + acc * static_cast<uint32_t>(p.nmma);
-        const uint32_t b_atom = static_cast<uint32_t>(p.brows) * 8u;    // brows * 128 bytes >> 4
-        for (int ks = 0; ks < p.ksteps; ++ks) {
-          const uint32_t a = ks >> 2, kk = ks & 3;
-          const uint64_t dak = da + (a * 1024u + kk * 2u), dbk = db + (a * b_atom + kk * 2u);
-          umma_f16_ss(d, dak, dbk, idesc, ks > 0 ? 1u : 0u);                    // high parts (rows 0..)
-          umma_f16_ss(d, dak, dbk + static_cast<uint32_t>(H) * 8u, idesc, 1u);  // low parts (rows H..)
+        if (r == g) {
+          uint64_t* tf = &tfull[g * kKTCMaxAcc + ai];
+          uint64_t* te = &tempty[g * kKTCMaxAcc + ai];
+          if (!mbar_wait(&bfull[bi], bu & 1)) { ok = false; return false; }
+          if (au > 0 && !mbar_wait(te, (au - 1) & 1)) { ok = false; return false; }
+          if (!mbar_wait(&full[si], su & 1) || abort_flag) { ok = false; return false; }
+          tc_fence_after();
+          // descriptors of the stage / query slot; a K step adds its byte offset >> 4 to the start field
+          const uint64_t da = smem_desc(smem_u32(smem + static_cast<size_t>(si) * p.a_bytes), 16u, 1024u, kSwizzle128B);
+          const uint64_t db = smem_desc(smem_u32(bslot + bi * static_cast<size_t>(p.b_bytes)), 16u, 1024u, kSwizzle128B);
+          const uint32_t d = tcol0 + static_cast<uint32_t>(ai * p.nmma);
+          for (int ks = 0; ks < p.ksteps; ++ks) {
+            const uint32_t a = ks >> 2, kk = ks & 3;
+            const uint64_t dak = da + (a * 1024u + kk * 2u), dbk = db + (a * b_atom + kk * 2u);
+            umma_f16_ss(d, dak, dbk, idesc, ks > 0 ? 1u : 0u);                    // high parts (rows 0..)
+            umma_f16_ss(d, dak, dbk + static_cast<uint32_t>(H) * 8u, idesc, 1u);  // low parts (rows H..)
+          }
+          umma_commit(&empty[si]);
+          umma_commit(tf);
+          if (++ai == p.nacc) { ai = 0; ++au; }
         }
-        umma_commit(&empty[s]);
-        umma_commit(&tfull[acc]);
-        if (last) { umma_commit(&bempty[bs]); ++seg; }
-        ++k;
+        if (last) {
+          umma_commit(&bempty[bi]);
+          if (++bi == p.nbs) { bi = 0; ++bu; }
+        }
+        if (++si == S) { si = 0; ++su; }
+        if (++r == NG) r = 0;
         return true;
       });
       if (!ok) { set_timeout(p.status, kSiteKFull); abort_flag = 1; }
-      umma_commit(mmadone);
-      mbar_wait(mmadone, 0);
+      umma_commit(&mmadone[g]);
+      mbar_wait(&mmadone[g], 0);
     }
   } else {
     // ------------------------------------------------------------ epilogue
     // Row rho of a tile is token rho / Hkv, KV head j = rho % Hkv; the row's
-    // logits are D columns [j*G, j*G + G) (hi) plus H + the same (lo).
+    // logits are accumulator columns [j*G, j*G + G).
+    const int e = warp - 1 - NG;                     // epilogue warp index
+    const int g = e >> 2;                            // its group
     const int q = warp & 3;                          // TMEM lane quarter of this warp
     const int rho = q * 32 + lane;
     const int j = rho & (Hkv - 1);
     const int tl = rho >> p.log2Hkv;
     const uint64_t keep = policy_evict_last();       // logits: read back by the V pass
+    const uint32_t tq = taddr + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(g * p.nacc * p.nmma);
     float m[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) m[g] = -INFINITY;
-    uint32_t k = 0, seg = 0;
+    for (int gg = 0; gg < G; ++gg) m[gg] = -INFINITY;
+    int r = 0, ai = 0;
+    uint32_t au = 0;
     bool ok = true;
     for_each_k_tile(p, p0, p1, [&](int32_t b, int32_t t0, int32_t nt, int64_t, bool, bool last) {
-      const uint32_t acc = k % p.nacc, use = k / p.nacc;
-      if (!mbar_wait(&tfull[acc], use & 1) || abort_flag) { ok = false; return false; }
-      tc_fence_after();
-      const uint32_t tbase = taddr + (static_cast<uint32_t>(q * 32) << 16) + acc * static_cast<uint32_t>(p.nmma);
-      float o[G];
+      if (r == g) {
+        if (!mbar_wait(&tfull[g * kKTCMaxAcc + ai], au & 1) || abort_flag) { ok = false; return false; }
+        tc_fence_after();
+        const uint32_t tbase = tq + static_cast<uint32_t>(ai * p.nmma);
+        float o[G];
 #pragma unroll
-      for (int ch = 0; ch < (H + 15) / 16; ++ch) {   // 16 query heads per load
-        uint32_t v[32];
-        tmem_ld_32x32b_x16(tbase + ch * 16, v);
-        tmem_ld_wait();
+        for (int ch = 0; ch < (H + 15) / 16; ++ch) {   // 16 query heads per load
+          uint32_t v[32];
+          tmem_ld_32x32b_x16(tbase + ch * 16, v);
+          tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int col = ch * 16 + c;
-          if (col < H && (col / G) == j) o[col % G] = __uint_as_float(v[c]);
+          for (int c = 0; c < 16; ++c) {
+            const int col = ch * 16 + c;
+            if (col < H && (col / G) == j) o[col % G] = __uint_as_float(v[c]);
+          }
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
-      if (tl < nt) {
-        float* lrow = p.logits + (static_cast<size_t>(b) * p.t_pad + t0 + tl) * H + j * G;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[g * kKTCMaxAcc + ai]);
+        if (++ai == p.nacc) { ai = 0; ++au; }
+        if (tl < nt) {
+          float* lrow = p.logits + (static_cast<size_t>(b) * p.t_pad + t0 + tl) * H + j * G;
 #pragma unroll
-        for (int g = 0; g < G; ++g) m[g] = fmaxf(m[g], o[g]);
-        if constexpr (G >= 4) {
+          for (int gg = 0; gg < G; ++gg) m[gg] = fmaxf(m[gg], o[gg]);
+          if constexpr (G >= 4) {
 #pragma unroll
-          for (int g = 0; g < G; g += 4)
-            st_global_hint(reinterpret_cast<float4*>(lrow + g), make_float4(o[g], o[g + 1], o[g + 2], o[g + 3]), keep);
-        } else {
-          st_global_hint(reinterpret_cast<uint2*>(lrow), make_uint2(__float_as_uint(o[0]), __float_as_uint(o[1])), keep);
+            for (int gg = 0; gg < G; gg += 4)
+              st_global_hint(reinterpret_cast<float4*>(lrow + gg), make_float4(o[gg], o[gg + 1], o[gg + 2], o[gg + 3]),
+                             keep);
+          } else {
+            st_global_hint(reinterpret_cast<uint2*>(lrow), make_uint2(__float_as_uint(o[0]), __float_as_uint(o[1])),
+                           keep);
+          }
         }
       }
       if (last) {
-        // merge this warp's maxima into the segment buffer; the last warp writes the segment out
-        float* sm = segmax + (seg % kKTCSegBufs) * H;
+        // this warp's maxima of the segment (all of its tiles precede this one in the walk)
+        float* mp = p.mpart + static_cast<size_t>(b + cta) * H;
 #pragma unroll
         for (int h = 0; h < H; ++h) {
           const float w = warp_max_f32((h / G) == j ? m[h % G] : -INFINITY);
-          if (lane == 0 && w > -INFINITY) smem_atomic_max_f32(sm + h, w);
+          if (lane == 0 && w > -INFINITY) atomic_max_f32(mp + h, w);
         }
 #pragma unroll
-        for (int g = 0; g < G; ++g) m[g] = -INFINITY;
-        int32_t prev = 0;
-        if (lane == 0) {
-          __threadfence_block();
-          prev = atomicAdd(&segcnt[seg % kKTCSegBufs], 1);
-          __threadfence_block();
-        }
-        prev = __shfl_sync(0xffffffffu, prev, 0);
-        if (prev == 3) {
-          for (int h = lane; h < H; h += 32) {
-            p.mpart[static_cast<size_t>(b + cta) * H + h] = sm[h];
-            sm[h] = -INFINITY;
-          }
-          __syncwarp();
-          if (lane == 0) segcnt[seg % kKTCSegBufs] = 0;
-        }
-        ++seg;
+        for (int gg = 0; gg < G; ++gg) m[gg] = -INFINITY;
       }
-      ++k;
+      if (++r == NG) r = 0;
       return true;
     });
     if (!ok) set_timeout(p.status, kSiteKFull);

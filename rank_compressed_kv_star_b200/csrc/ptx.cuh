@@ -45,10 +45,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same test, but a thread whose phase is not complete is suspended until it
+// completes or `hint_ns` elapse (it does not spin, so waiting warps leave the
+// issue slots to the warps that work).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Upper bounds of every wait: about two seconds of wall time and a hard cap on
 // polls, whichever comes first.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kWaitLimitPolls = 1u << 26;
+constexpr uint32_t kWaitSleepNs = 20000;   // one suspended poll: at most 20 us
 
 // Waits for the phase with parity `parity` to complete.  Returns false when
 // the bound ran out (the caller records a timeout and stops).
@@ -56,8 +72,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 0; i < kWaitLimitPolls; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+    if ((i & 7u) == 7u && globaltimer_ns() - t0 > kWaitLimitNs) return false;
   }
   return false;
 }

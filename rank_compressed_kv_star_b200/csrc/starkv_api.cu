@@ -26,7 +26,7 @@
 #define STARKV_KTC_CTAS_PER_SM 3
 #endif
 #ifndef STARKV_KTC_SMEM_BYTES
-#define STARKV_KTC_SMEM_BYTES (208 * 1024)   // shared memory of the K-pass CTAs on one SM
+#define STARKV_KTC_SMEM_BYTES (212 * 1024)   // shared memory of the K-pass CTAs on one SM
 #endif
 #ifndef STARKV_K_RING_BYTES
 #define STARKV_K_RING_BYTES (200 * 1024 / STARKV_K_CTAS_PER_SM)
@@ -89,7 +89,7 @@ struct DecodePlan {
   size_t k_smem;
   // K pass on tensor cores (grouped queries)
   bool ktc;
-  int ktc_log2tpt, ktc_ksteps, ktc_kb, ktc_nmma, ktc_brows, ktc_nacc, ktc_nbs, ktc_stages;
+  int ktc_log2tpt, ktc_ksteps, ktc_kb, ktc_nmma, ktc_brows, ktc_ng, ktc_nacc, ktc_nbs, ktc_stages;
   uint32_t ktc_a_bytes, ktc_b_bytes, ktc_tmem;
   size_t ktc_smem;
   // V pass
@@ -139,57 +139,36 @@ bool set_smem(K kernel, size_t bytes) {
   return true;
 }
 
-// CTAs of the tensor-core K pass (instance <G, H>) that fit on one SM by
-// registers (the kernel's count, allocated per warp in units of 256) and by
-// shared memory (`smem` bytes each within STARKV_KTC_SMEM_BYTES per SM).
+// Registers per thread of the tensor-core K pass instance <G, H> (0 if unknown).
 template <int G, int H>
-int ktc_occupancy(size_t smem) {
+int ktc_regs() {
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, kpass_tc_kernel<G, H>) != cudaSuccess) { cudaGetLastError(); return 0; }
-  // 10% margin: an instance at 109 registers measured at two resident CTAs, not three
-  const int per_warp = (fa.numRegs * 32 + 255) / 256 * 256;
-  const int by_regs = 65536 * 10 / (per_warp * (kKTCThreads / 32) * 11);
-  const int by_smem = static_cast<int>(static_cast<size_t>(STARKV_KTC_SMEM_BYTES) / (smem + 1024));
-  return by_regs < by_smem ? by_regs : by_smem;
+  return fa.numRegs;
 }
 
 template <int H>
-int ktc_occupancy_h(int log2G, size_t smem) {
+int ktc_regs_h(int log2G) {
   switch (log2G) {
-    case 1: if constexpr (H / 2 <= 16) return ktc_occupancy<2, H>(smem); break;
-    case 2: if constexpr (H >= 4 && H / 4 <= 16) return ktc_occupancy<(H >= 4 ? 4 : H), H>(smem); break;
-    case 3: if constexpr (H >= 8) return ktc_occupancy<(H >= 8 ? 8 : H), H>(smem); break;
-    case 4: if constexpr (H >= 16) return ktc_occupancy<(H >= 16 ? 16 : H), H>(smem); break;
-    case 5: if constexpr (H >= 32) return ktc_occupancy<(H >= 32 ? 32 : H), H>(smem); break;
-    case 6: if constexpr (H >= 64) return ktc_occupancy<(H >= 64 ? 64 : H), H>(smem); break;
+    case 1: if constexpr (H / 2 <= 16) return ktc_regs<2, H>(); break;
+    case 2: if constexpr (H >= 4 && H / 4 <= 16) return ktc_regs<(H >= 4 ? 4 : H), H>(); break;
+    case 3: if constexpr (H >= 8) return ktc_regs<(H >= 8 ? 8 : H), H>(); break;
+    case 4: if constexpr (H >= 16) return ktc_regs<(H >= 16 ? 16 : H), H>(); break;
+    case 5: if constexpr (H >= 32) return ktc_regs<(H >= 32 ? 32 : H), H>(); break;
+    case 6: if constexpr (H >= 64) return ktc_regs<(H >= 64 ? 64 : H), H>(); break;
     default: break;
   }
   return 0;
 }
 
-int ktc_resident_ctas(int log2G, int H, size_t smem) {
-  static std::mutex mu;
-  static std::map<std::tuple<int, int, size_t, int>, int> cache;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return 0; }
-  const auto key = std::make_tuple(log2G, H, smem, dev);
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    auto it = cache.find(key);
-    if (it != cache.end()) return it->second;
-  }
-  int n = 0;
+int ktc_num_regs(int log2G, int H) {
   switch (H) {
-    case 4: n = ktc_occupancy_h<4>(log2G, smem); break;
-    case 8: n = ktc_occupancy_h<8>(log2G, smem); break;
-    case 16: n = ktc_occupancy_h<16>(log2G, smem); break;
-    case 32: n = ktc_occupancy_h<32>(log2G, smem); break;
-    case 64: n = ktc_occupancy_h<64>(log2G, smem); break;
-    default: break;
+    case 8: return ktc_regs_h<8>(log2G);
+    case 16: return ktc_regs_h<16>(log2G);
+    case 32: return ktc_regs_h<32>(log2G);
+    case 64: return ktc_regs_h<64>(log2G);
+    default: return 0;
   }
-  std::lock_guard<std::mutex> lock(mu);
-  cache[key] = n;
-  return n;
 }
 
 starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_seq_len, DecodePlan* pl) {
@@ -230,12 +209,12 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
              2 * p.k_stages * sizeof(uint64_t) + (kKConsumers / p.L) * sizeof(float);
   p.k_ctas = sms * STARKV_K_CTAS_PER_SM;
 
-  // Grouped queries (G >= 2, H >= 4) with at most 16 KV heads: the K pass runs
-  // on the tensor cores.  Its per-CTA pipeline (one page per stage, one tile in
-  // the epilogue at a time) is latency-bound, so the plan takes the most CTAs
-  // per SM that fit (registers of the kernel instance, shared memory, TMEM),
-  // each with at least three stages (two for a single CTA), and two query
-  // slots where they fit.
+  // Grouped queries (G >= 2, H >= 8) with at most 16 KV heads: the K pass runs
+  // on the tensor cores.  A CTA's single producer thread and per-tile chain are
+  // serial, so the plan spreads the SM over up to STARKV_KTC_CTAS_PER_SM CTAs
+  // of one consumer group each, most CTAs first, that fit by registers (the
+  // instance's count), shared memory (>= 3 ring stages, 4 for a single CTA)
+  // and TMEM (>= 2 accumulators).
   p.ktc = false;
   if (p.log2G >= 1 && p.H >= 8 && p.Hkv <= 16) {
     int log2Hkv = 0;
@@ -247,22 +226,28 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
     p.ktc_brows = p.H < 16 ? 32 : 2 * p.H;   // the low-part MMA reads rows [H, H + nmma)
     p.ktc_a_bytes = static_cast<uint32_t>(p.ktc_kb) * 128u * 128u;
     p.ktc_b_bytes = static_cast<uint32_t>(p.ktc_kb) * p.ktc_brows * 128u;
+    const int regs = ktc_num_regs(p.log2G, p.H);
     for (int ctas = STARKV_KTC_CTAS_PER_SM; ctas >= 1 && !p.ktc; --ctas) {
-      for (int nbs = 2; nbs >= 1 && !p.ktc; --nbs) {
-        const uint32_t budget = static_cast<uint32_t>(STARKV_KTC_SMEM_BYTES) / ctas - 1024u;
-        const uint32_t fixed = 1024u + nbs * p.ktc_b_bytes + 13u * 8u + (kKTCSegBufs * p.H + kKTCSegBufs) * 4u;
-        if (budget <= fixed) continue;
-        int stages = static_cast<int>((budget - fixed) / (p.ktc_a_bytes + 16u));
-        if (stages > 12) stages = 12;
-        int nacc = 512 / ctas / p.ktc_nmma;
-        if (nacc > 4) nacc = 4;
-        const uint32_t tmem = static_cast<uint32_t>(pow2_ceil(nacc * p.ktc_nmma < 32 ? 32 : nacc * p.ktc_nmma));
-        if (stages < (ctas > 1 ? 3 : 2) || nacc < 2 || tmem * ctas > 512) continue;
-        const size_t smem = fixed + static_cast<size_t>(stages) * (p.ktc_a_bytes + 16u);
-        if (ktc_resident_ctas(p.log2G, p.H, smem) < ctas) continue;
-        p.ktc = true;
-        p.ktc_stages = stages; p.ktc_nacc = nacc; p.ktc_nbs = nbs; p.ktc_tmem = tmem; p.ktc_smem = smem;
-        p.k_ctas = sms * ctas;
+      for (int ng = 1; ng >= 1 && !p.ktc; --ng) {
+        const int per_warp = (regs * 32 + 255) / 256 * 256;
+        if (regs <= 0 || per_warp * (ktc_threads(ng) / 32) * ctas * 11 > 65536 * 10) continue;  // 10% margin
+        int nacc = 512 / (ctas * ng * p.ktc_nmma);
+        if (nacc > kKTCMaxAcc) nacc = kKTCMaxAcc;
+        if (nacc < 2) continue;
+        for (int nbs = 2; nbs >= 1 && !p.ktc; --nbs) {
+          const uint32_t fixed =
+              1024u + nbs * p.ktc_b_bytes + (4 + 2 * kKTCMaxGroups * kKTCMaxAcc + kKTCMaxGroups) * 8u;
+          const uint32_t budget = static_cast<uint32_t>(STARKV_KTC_SMEM_BYTES) / ctas - (ctas > 1 ? 1024u : 0u);
+          if (budget <= fixed) continue;
+          int stages = static_cast<int>((budget - fixed) / (p.ktc_a_bytes + 16u));
+          if (stages > 12) stages = 12;
+          if (stages < (ctas > 1 ? 3 : 4)) continue;
+          p.ktc = true;
+          p.ktc_ng = ng; p.ktc_nacc = nacc; p.ktc_nbs = nbs; p.ktc_stages = stages;
+          p.ktc_tmem = static_cast<uint32_t>(pow2_ceil(ng * nacc * p.ktc_nmma < 32 ? 32 : ng * nacc * p.ktc_nmma));
+          p.ktc_smem = fixed + static_cast<size_t>(stages) * (p.ktc_a_bytes + 16u);
+          p.k_ctas = sms * ctas;
+        }
       }
     }
   }
@@ -457,7 +442,8 @@ template <int G, int H>
 cudaError_t launch_kpass_tc_gh(const DecodePlan& pl, const CUtensorMap& kmap, const CUtensorMap& qmap,
                                const KPassTCParams& tp, cudaStream_t s) {
   if (!set_smem(kpass_tc_kernel<G, H>, pl.ktc_smem)) return cudaErrorInvalidValue;
-  return launch(kpass_tc_kernel<G, H>, dim3(pl.k_ctas), dim3(kKTCThreads), pl.ktc_smem, s, 1, kmap, qmap, tp);
+  return launch(kpass_tc_kernel<G, H>, dim3(pl.k_ctas), dim3(ktc_threads(pl.ktc_ng)), pl.ktc_smem, s, 1, kmap, qmap,
+                tp);
 }
 
 template <int H>
@@ -479,7 +465,6 @@ cudaError_t launch_kpass_tc_h(const DecodePlan& pl, const CUtensorMap& kmap, con
 cudaError_t launch_kpass_tc(const DecodePlan& pl, const CUtensorMap& kmap, const CUtensorMap& qmap,
                             const KPassTCParams& tp, cudaStream_t s) {
   switch (pl.H) {
-    case 4: return launch_kpass_tc_h<4>(pl, kmap, qmap, tp, s);
     case 8: return launch_kpass_tc_h<8>(pl, kmap, qmap, tp, s);
     case 16: return launch_kpass_tc_h<16>(pl, kmap, qmap, tp, s);
     case 32: return launch_kpass_tc_h<32>(pl, kmap, qmap, tp, s);
@@ -693,6 +678,8 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   ap.qt = qt; ap.prefix = prefix; ap.teff = teff; ap.status = status;
   __half* qth = pl.ktc ? reinterpret_cast<__half*>(ws + pl.ws.qth_off) : nullptr;
   ap.qth = qth;
+  ap.mpart_init = pl.ktc ? mpart : nullptr;   // the tensor-core K pass merges segment maxima by atomics
+  ap.n_mpart = pl.ws.k_slots * pl.H;
   ap.B = batch; ap.H = pl.H; ap.d = pl.d; ap.r = pl.r; ap.cap = pl.cap; ap.log2G = pl.log2G;
   ap.coef = scale * kLog2e;
   {
@@ -728,7 +715,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
     tp.MB = pl.MB; tp.NB = pl.NB; tp.t_pad = pl.t_pad;
     tp.log2tpt = pl.ktc_log2tpt; tp.ksteps = pl.ktc_ksteps; tp.kb = pl.ktc_kb;
     tp.nmma = pl.ktc_nmma; tp.brows = pl.ktc_brows;
-    tp.nacc = pl.ktc_nacc; tp.nbs = pl.ktc_nbs; tp.stages = pl.ktc_stages;
+    tp.ng = pl.ktc_ng; tp.nacc = pl.ktc_nacc; tp.nbs = pl.ktc_nbs; tp.stages = pl.ktc_stages;
     tp.a_bytes = pl.ktc_a_bytes; tp.b_bytes = pl.ktc_b_bytes; tp.tmem_cols = pl.ktc_tmem;
     e = launch_kpass_tc(pl, kmap, qmap, tp, s);
   } else if (pl.L == 1 && pl.CPT == 4) e = launch_kpass<1, 4>(pl, kp, s);
