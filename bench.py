@@ -79,15 +79,19 @@ def whole_job_tokens_per_s(world: int, batch_per_rank: int, ms_per_step_max: flo
     return world * batch_per_rank / (ms_per_step_max * 1e-3)
 
 
-# DRAM bytes (read + write) per processed token measured by one ncu capture of
-# the streaming kernels on the batch-32, context-8192 case (32 heads, K rank 64,
-# V rank 2048); traffic grows in proportion to the tokens processed.  Valid
-# only for that geometry and for the kernels as they were captured.
+# DRAM bytes (read + write) per processed token of the two streaming kernels,
+# from ncu captures (dram__bytes_read.sum + dram__bytes_write.sum of one
+# launch); traffic grows in proportion to the tokens processed.  Keyed by
+# layer geometry (query heads, KV heads, K rank, V rank); valid only for the
+# kernels as they were captured (the summaries under profiles/ give the
+# commands).
 NCU_TRAFFIC_PER_TOKEN = {
-    "kpass": (1.074168e9 + 6.671104e6) / (32 * 8192),
-    "vpass": (1.107514e9 + 5.822976e6) / (32 * 8192),
+    # batch 32, context 8192 (MHA): CUDA-core K pass, V pass
+    (32, 32, 64, 2048): {"kpass": (1074215168 + 6370048) / (32 * 8192),
+                         "vpass": (1108390400 + 4740096) / (32 * 8192)},
+    # batch 64, context 8192 (32 query heads over 8 KV heads): tensor-core K pass
+    (32, 8, 64, 512): {"kpass": (537.648640e6 + 8.424192e6) / (64 * 8192)},
 }
-NCU_TRAFFIC_GEOMETRY = (32, 32, 64, 2048)   # (query heads, KV heads, K rank, V rank)
 
 
 def measured_peaks():
@@ -179,8 +183,9 @@ def run_ours(args):
 
     wl = W.workload(args.workload)
     if args.batch:
-        wl = W.Workload(f"{wl.name} (override: batch {args.batch}, length {args.seq})", wl.seed,
-                        args.batch, wl.layers[:1], np.full(args.batch, args.seq - 1, dtype=np.int64))
+        seq = args.seq or wl.max_seq_len      # length defaults to the workload's own
+        wl = W.Workload(f"{wl.name} (override: batch {args.batch}, length {seq})", wl.seed,
+                        args.batch, wl.layers[:1], np.full(args.batch, seq - 1, dtype=np.int64))
     layers = []
     for li in range(len(wl.layers)):
         Ld = D.device_layer(wl, li)
@@ -288,8 +293,9 @@ def run_ours(args):
     dom = "kpass" if per["kpass"] >= per["vpass"] else "vpass"
     dom_bytes, dom_gbs = (k_bytes, kp_gbs) if dom == "kpass" else (v_bytes, vp_gbs)
     traffic = None
-    if len(layers) == 1 and (layers[0]["H"], layers[0]["Hkv"], layers[0]["r"], layers[0]["R"]) == NCU_TRAFFIC_GEOMETRY:
-        traffic = round(NCU_TRAFFIC_PER_TOKEN[dom] * T_sum)
+    geom = (layers[0]["H"], layers[0]["Hkv"], layers[0]["r"], layers[0]["R"])
+    if len(layers) == 1 and dom in NCU_TRAFFIC_PER_TOKEN.get(geom, {}):
+        traffic = round(NCU_TRAFFIC_PER_TOKEN[geom][dom] * T_sum)
 
     # ---------------- end to end through the public API with host buffers
     Ke = max(1, min(args.e2e_steps, K))
