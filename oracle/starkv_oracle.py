@@ -266,6 +266,38 @@ def attention_uncompressed(q, k_list, v_list, scale):
     return out
 
 
+def prefill_attention(q, B_K, B_V, k_cache, v_cache, tables, starts, chunk_lens, scale):
+    """Causal attention of prefill chunks over the paged codes (chunked prefill).
+
+    The README has STAR-KV served by dedicated kernels over the compressed
+    pages (method paragraph) and gives no formula; the reading taken is the
+    autoregressive one: query token ``i`` of sequence ``b`` (row
+    ``sum(chunk_lens[:b]) + i`` of ``q``) attends over the sequence's tokens
+    ``0 .. starts[b] + i``, whose codes (the chunk's own included) are in the
+    cache.  Keys and values are decompressed explicitly as in
+    :func:`decode_explicit`.  Returns fp64 ``[n_rows][H][d]``.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    n_rows, H, d = q.shape
+    Hkv = np.shape(B_K)[0]
+    out = np.zeros((n_rows, H, d))
+    row = 0
+    for b, n in enumerate(chunk_lens):
+        n = int(n)
+        t_end = int(starts[b]) + n
+        if n == 0:
+            continue
+        k_hat = decompress_k(gather(k_cache, tables[b], t_end), B_K)
+        v_hat = decompress_v(gather(v_cache, tables[b], t_end), B_V).reshape(t_end, Hkv, d)
+        for i in range(n):
+            T = int(starts[b]) + i + 1
+            for h in range(H):
+                j = kv_head(h, H, Hkv)
+                out[row, h] = attention_head(q[row, h], k_hat[:T, j, :], v_hat[:T, j, :], scale)
+            row += 1
+    return out
+
+
 def decode_stages(q_b, B_K, B_V, c_K, c_V, scale):
     """Intermediate quantities of one sequence in absorbed form, for diagnosis.
 

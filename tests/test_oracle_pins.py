@@ -120,6 +120,69 @@ def test_grouped_query_equals_mha_with_repeated_kv_heads():
                            L["seq_lens"], L["scale"]), want, rtol=0, atol=1e-12 * np.abs(want).max())
 
 
+def check_prefill_causal_full_rank(prefill=None):
+    """Chunks over a full-rank cache equal torch's attention with the causal mask of each chunk."""
+    H, Hkv, d = 4, 2, 16
+    starts, chunks = [0, 7, 30], [5, 9, 1]
+    lens = [s + c for s, c in zip(starts, chunks)]
+    c = _full_rank_case(seed=12, H=H, Hkv=Hkv, d=d, lens=tuple(lens))
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((sum(chunks), H, d))
+    prefill = prefill or O.prefill_attention
+    got = prefill(q, c["B_K"], c["B_V"], c["kc"], c["vc"], c["tables"], starts, chunks, c["scale"])
+    row = 0
+    for b, (s0, n) in enumerate(zip(starts, chunks)):
+        T = s0 + n
+        mask = torch.from_numpy(np.arange(T)[None, :] <= (s0 + np.arange(n))[:, None])      # [n][T]
+        qt = torch.from_numpy(np.transpose(q[row:row + n], (1, 0, 2)).copy())                 # [H][n][d]
+        kt = torch.from_numpy(np.transpose(c["k_full"][b], (1, 0, 2)).copy())                # [Hkv][T][d]
+        vt = torch.from_numpy(np.transpose(c["v_full"][b], (1, 0, 2)).copy())
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=c["scale"],
+                                                               enable_gqa=True)
+        np.testing.assert_allclose(got[row:row + n], np.transpose(ref.numpy(), (1, 0, 2)), rtol=0, atol=1e-12)
+        row += n
+
+
+def test_prefill_causal_full_rank_equals_library_attention():
+    check_prefill_causal_full_rank()
+
+
+def test_prefill_single_token_chunks_equal_decode():
+    wl = W.workload(1)
+    L = W.host_layer(wl, 0)
+    T = L["seq_lens"]
+    q = L["q"]
+    got = O.prefill_attention(q, L["B_K"], L["B_V"], L["k_cache"], L["v_cache"], L["tables"], T - 1,
+                              [1] * wl.batch, L["scale"])
+    want = O.decode_explicit(q, L["B_K"], L["B_V"], L["k_cache"], L["v_cache"], L["tables"], T, L["scale"])
+    np.testing.assert_array_equal(got, want)
+
+
+def test_planted_acausal_prefill_is_caught():
+    """A chunk token that also sees the next token must fail the causal pin."""
+    with pytest.raises(AssertionError):
+        check_prefill_causal_full_rank(_leaky_prefill)
+
+
+def _leaky_prefill(q, B_K, B_V, kc, vc, tables, starts, chunks, scale):
+    q = np.asarray(q, float)
+    n_rows, H, d = q.shape
+    Hkv = np.shape(B_K)[0]
+    out = np.zeros((n_rows, H, d))
+    row = 0
+    for b, n in enumerate(chunks):
+        t_end = starts[b] + n
+        k_hat = O.decompress_k(O.gather(kc, tables[b], t_end), B_K)
+        v_hat = O.decompress_v(O.gather(vc, tables[b], t_end), B_V).reshape(t_end, Hkv, d)
+        for i in range(n):
+            T = min(t_end, starts[b] + i + 2)          # one token too many
+            for h in range(H):
+                j = O.kv_head(h, H, Hkv)
+                out[row, h] = O.attention_head(q[row, h], k_hat[:T, j], v_hat[:T, j], scale)
+            row += 1
+    return out
+
+
 def test_uncompressed_attention_matches_library():
     c = _full_rank_case(seed=9, lens=(3, 33))
     got = O.attention_uncompressed(c["q"], c["k_full"], c["v_full"], c["scale"])
