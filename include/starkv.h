@@ -162,6 +162,41 @@ starkv_status starkv_paged_decode(const starkv_layer_desc* desc, int32_t batch, 
                                   void* workspace, size_t workspace_bytes, void* out, void* stream);
 
 /*
+ * starkv_paged_prefill -- causal attention of prefill chunks over the paged
+ * codes (chunked prefill).  The step that precedes decode: a prompt is
+ * compressed into the cache chunk by chunk (starkv_compress_store) and each
+ * chunk's queries attend over everything cached so far plus their own chunk.
+ * The README describes STAR-KV as served by dedicated kernels over the
+ * compressed pages ("Low-rank KV Cache Compression for vLLM", method
+ * paragraph); no formula is given, so this is causal softmax attention with
+ * the decode formulation above: query token i of sequence b (row
+ * row_offsets[b] + i) attends over the tokens 0 .. starts[b] + i of b, whose
+ * codes (the chunk's own included) must already be in the cache.
+ *
+ *   n_seqs        sequences with a chunk in this call
+ *   n_rows        query tokens in total = row_offsets[n_seqs] (host value)
+ *   max_seq_len   host-side upper bound of starts[b] + chunk length
+ *   q             fp16 [n_rows][H][d], the chunks back to back
+ *   block_tables  int32 [n_seqs][max_blocks_per_seq]
+ *   starts        int32 [n_seqs] (device): position of each chunk's first token
+ *   row_offsets   int32 [n_seqs + 1] (device): first row of each chunk,
+ *                 non-decreasing from 0 to n_rows
+ *   workspace     at least starkv_prefill_workspace_bytes(desc, n_rows,
+ *                 max_seq_len) bytes, 256-byte aligned
+ *   out           fp16 [n_rows][H][d]
+ *
+ * Every row is evaluated as one decode row (its own length, the sequence's
+ * block table), so a chunk's rows read the sequence's pages once per row:
+ * cost grows with rows x context.  Errors as starkv_paged_decode.
+ */
+size_t starkv_prefill_workspace_bytes(const starkv_layer_desc* desc, int32_t n_rows, int32_t max_seq_len);
+starkv_status starkv_paged_prefill(const starkv_layer_desc* desc, int32_t n_seqs, int32_t n_rows,
+                                   int32_t max_seq_len, const void* q, const void* B_K, const void* B_V,
+                                   const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                                   const int32_t* starts, const int32_t* row_offsets, float scale,
+                                   void* workspace, size_t workspace_bytes, void* out, void* stream);
+
+/*
  * starkv_paged_decode_profiled -- starkv_paged_decode that also records CUDA
  * events on `stream` around its kernels, for per-kernel timing.
  * stage_events: HOST array of 6 cudaEvent_t (as void*; a NULL entry is

@@ -92,6 +92,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                                  P, SZ, P, P, ctypes.POINTER(P)]
     lib.starkv_paged_decode_profiled.restype = ctypes.c_int
     lib.starkv_paged_decode_static.argtypes = [DP, I32, I32, P, P, P, P, P, P, P, ctypes.c_float, P, P]
+    lib.starkv_prefill_workspace_bytes.argtypes = [DP, I32, I32]
+    lib.starkv_prefill_workspace_bytes.restype = ctypes.c_size_t
+    lib.starkv_paged_prefill.argtypes = [DP, I32, I32, I32, P, P, P, P, P, P, P, P, ctypes.c_float, P,
+                                         ctypes.c_size_t, P, P]
+    lib.starkv_paged_prefill.restype = ctypes.c_int
     lib.starkv_paged_decode_static.restype = ctypes.c_int
     lib.starkv_decode_check.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
     lib.starkv_decode_check.restype = ctypes.c_int
@@ -180,6 +185,22 @@ def starkv_paged_decode(desc: LayerDesc, batch: int, max_seq_len: int, q, B_K, B
         int(workspace_bytes), _ptr(out), _stream(stream))
     if check:
         _check(st, "starkv_paged_decode")
+    return st
+
+
+def starkv_prefill_workspace_bytes(desc: LayerDesc, n_rows: int, max_seq_len: int) -> int:
+    return int(load_library().starkv_prefill_workspace_bytes(_desc_ref(desc), n_rows, max_seq_len))
+
+
+def starkv_paged_prefill(desc: LayerDesc, n_seqs: int, n_rows: int, max_seq_len: int, q, B_K, B_V,
+                         k_cache, v_cache, block_tables, starts, row_offsets, scale: float, workspace,
+                         workspace_bytes: int, out, stream=None, check: bool = True) -> int:
+    st = load_library().starkv_paged_prefill(
+        _desc_ref(desc), n_seqs, n_rows, max_seq_len, _ptr(q), _ptr(B_K), _ptr(B_V), _ptr(k_cache),
+        _ptr(v_cache), _ptr(block_tables), _ptr(starts), _ptr(row_offsets), float(scale),
+        _ptr(workspace), int(workspace_bytes), _ptr(out), _stream(stream))
+    if check:
+        _check(st, "starkv_paged_prefill")
     return st
 
 

@@ -62,6 +62,12 @@ __device__ __forceinline__ int32_t seq_of_page(const int32_t* prefix, int32_t B,
 
 __device__ __forceinline__ void set_flag(int32_t* status, int32_t f) { atomicOr(status, f); }
 
+// Block-table row of decode row b: row b itself, or, for rows that are query
+// tokens of a prefill chunk, the row of the sequence row_seq[b].
+__device__ __forceinline__ const int32_t* table_row(const int32_t* tables, const int32_t* row_seq, int32_t b, int MB) {
+  return tables + static_cast<size_t>(row_seq ? row_seq[b] : b) * MB;
+}
+
 // Timeout at pipeline wait `site`: the timeout bit plus a per-site bit (8..15)
 // that tells where the pipeline stopped.
 enum WaitSite : int32_t {
@@ -70,6 +76,33 @@ enum WaitSite : int32_t {
 };
 __device__ __forceinline__ void set_timeout(int32_t* status, WaitSite site) {
   atomicOr(status, STARKV_FLAG_TIMEOUT | (1 << (8 + site)));
+}
+
+// ================================================================ prefill rows
+// Rows of a chunked prefill: query token i of sequence b (rows
+// row_offsets[b] .. row_offsets[b+1]-1) attends over the sequence's tokens
+// 0 .. starts[b] + i, so it is decode row r with the sequence's block table
+// and length starts[b] + i + 1.
+struct PrefillRowsParams {
+  const int32_t* starts;       // [n_seqs] position of each chunk's first token
+  const int32_t* row_offsets;  // [n_seqs + 1] first row of each sequence's chunk
+  int32_t* row_seq;            // [n_rows] out
+  int32_t* row_len;            // [n_rows] out
+  int n_seqs, n_rows;
+};
+
+__global__ void __launch_bounds__(256) prefill_rows_kernel(PrefillRowsParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int r = blockIdx.x * 256 + threadIdx.x;
+  if (r >= p.n_rows) return;
+  int lo = 0, hi = p.n_seqs - 1;     // largest b with row_offsets[b] <= r
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.row_offsets[mid] <= r) lo = mid; else hi = mid - 1;
+  }
+  p.row_seq[r] = lo;
+  p.row_len[r] = p.starts[lo] + (r - p.row_offsets[lo]) + 1;
 }
 
 // ====================================================================== absorb
@@ -184,7 +217,8 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbParams p) {
 // ======================================================================= kpass
 struct KPassParams {
   const __half* k_cache;      // [NB][16][H][r]
-  const int32_t* tables;      // [B][MB]
+  const int32_t* tables;      // [B][MB] (or [n_seqs][MB] with row_seq)
+  const int32_t* row_seq;     // [B] sequence of each row, or null (row b is sequence b)
   const int32_t* teff;        // [B]
   const int32_t* prefix;      // [B+1]
   const float* qt;            // [B][H][r]
@@ -238,13 +272,15 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
   StageMeta* meta = reinterpret_cast<StageMeta*>(smem + static_cast<size_t>(S) * p.stage_bytes);
   uint64_t* full = reinterpret_cast<uint64_t*>(meta + S);
   uint64_t* empty = full + S;
-  float* red = reinterpret_cast<float*>(empty + S);         // [kKConsumers / L]
+  uint64_t* cbar = empty + S;                                // the consumers' segment-end sync
+  float* red = reinterpret_cast<float*>(cbar + 1);          // [kKConsumers / L]
   __shared__ volatile int32_t abort_flag;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], kKConsumers / 32); }
+    mbar_init(cbar, kKConsumers);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -275,7 +311,7 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
           while (p.prefix[b + 1] <= pg_g) ++b;
           const int32_t pg = static_cast<int32_t>(pg_g - p.prefix[b]);
           const int32_t T = p.teff[b];
-          int32_t phys = p.tables[static_cast<size_t>(b) * p.MB + pg];
+          int32_t phys = table_row(p.tables, p.row_seq, b, p.MB)[pg];
           if (phys < 0 || phys >= p.NB) { set_flag(p.status, STARKV_FLAG_BAD_BLOCK_ID); phys = 0; }
           const int32_t tend = min(pg * kBlock + kBlock, T);
           for (int32_t t0 = pg * kBlock; t0 < tend; t0 += p.tps, ++k) {
@@ -308,7 +344,7 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
           meta[s] = StageMeta{b, t0, nt, 0};
           mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nt) * tok_bytes);
           for (int i = 0; i < n_pg; ++i) {
-            int32_t phys = p.tables[static_cast<size_t>(b) * p.MB + pg + i];
+            int32_t phys = table_row(p.tables, p.row_seq, b, p.MB)[pg + i];
             if (phys < 0 || phys >= p.NB) { set_flag(p.status, STARKV_FLAG_BAD_BLOCK_ID); phys = 0; }
             const int32_t ti = min(kBlock, nt - i * kBlock);
             bulk_g2s(ring + static_cast<size_t>(s) * p.stage_bytes + static_cast<size_t>(i) * kBlock * tok_bytes,
@@ -346,6 +382,7 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
   float2 qv[CPT * 4];
   float m = -INFINITY;
   int cur_b = -1;
+  uint32_t cphase = 0;
   const uint64_t keep = policy_evict_last();   // logits: read back by the V pass
 
   for (uint32_t k = 0;; ++k) {
@@ -359,13 +396,13 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
       if (cur_b >= 0) {
         // per-segment max for every head: slot = sequence + CTA
         if (sub == 0) red[pair0] = m;
-        named_bar_sync(1, kKConsumers);
+        if (!group_sync(cbar, cphase)) { set_timeout(p.status, kSiteKFull); abort_flag = 1; break; }
         if (tid < p.H) {
           float M = -INFINITY;
           for (int g = tid; g < kPairsPerPass; g += p.H) M = fmaxf(M, red[g]);
           p.mpart[static_cast<size_t>(cur_b + cta) * p.H + tid] = M;
         }
-        named_bar_sync(1, kKConsumers);
+        if (!group_sync(cbar, cphase)) { set_timeout(p.status, kSiteKFull); abort_flag = 1; break; }
       }
       if (mt.b < 0) break;
       cur_b = mt.b;
@@ -442,7 +479,8 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
 // the segment's maxima in global memory (float max through integer atomics,
 // initialised to -inf by the absorb kernel).
 struct KPassTCParams {
-  const int32_t* tables;      // [B][MB]
+  const int32_t* tables;      // [B][MB] (or [n_seqs][MB] with row_seq)
+  const int32_t* row_seq;     // [B] sequence of each row, or null
   const int32_t* teff;        // [B]
   const int32_t* prefix;      // [B+1]
   float* logits;              // [B][t_pad][H]
@@ -569,7 +607,7 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         uint8_t* st = smem + static_cast<size_t>(si) * p.a_bytes;
         const int nbox = (nt + tb - 1) >> log2tb;
         mbar_arrive_expect_tx(&full[si], static_cast<uint32_t>(nbox * p.kb) * box_bytes);
-        const int32_t* trow = p.tables + static_cast<size_t>(b) * p.MB;
+        const int32_t* trow = table_row(p.tables, p.row_seq, b, p.MB);
         for (int c = 0; c < nbox; ++c) {
           const int32_t t = t0 + c * tb;
           int32_t phys = trow[t >> 4];
@@ -728,6 +766,7 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
 // block per 128 rows of the R range.
 struct VPassParams {
   const int32_t* tables;
+  const int32_t* row_seq;   // [B] sequence of each row, or null
   const int32_t* teff;
   const int32_t* prefix;
   const float* logits;    // [B][t_pad][H]
@@ -763,7 +802,8 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
   uint64_t* zdone = empty + S;
   uint64_t* tfree = zdone + 1;
   uint64_t* mdone = tfree + 1;
-  float* sM = reinterpret_cast<float*>(mdone + 1);                      // [npad]
+  uint64_t* pbar = mdone + 1;                                           // the weight warps' sync
+  float* sM = reinterpret_cast<float*>(pbar + 1);                       // [npad]
   float* sRed = sM + p.npad;                                            // [128]
   __shared__ uint32_t taddr_s;
   __shared__ volatile int32_t abort_flag;
@@ -790,6 +830,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
     mbar_init(zdone, 1);
     mbar_init(tfree, 128);
     mbar_init(mdone, 1);
+    mbar_init(pbar, 128);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -827,7 +868,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
         const int64_t xi = pg_g + lane;
         int32_t bi = b;
         while (bi < p.B - 1 && p.prefix[bi + 1] <= xi) ++bi;
-        cphys = xi < p1 ? p.tables[static_cast<size_t>(bi) * p.MB + static_cast<int32_t>(xi - p.prefix[bi])] : 0;
+        cphys = xi < p1 ? table_row(p.tables, p.row_seq, bi, p.MB)[static_cast<int32_t>(xi - p.prefix[bi])] : 0;
       }
       int32_t phys = __shfl_sync(0xffffffffu, cphys, static_cast<int>(pg_g - cbase));
       if (lane == 0) {
@@ -909,7 +950,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
     const int t_w0 = et / p.npad;
     const int t_step = 128 / p.npad;
     float lsum = 0.f;
-    uint32_t seg = 0;
+    uint32_t seg = 0, pphase = 0;
     const uint64_t keep = policy_evict_last();   // Z partials: read back by zfinal
     for (uint32_t k = 0;; ++k) {
       const int s = k % S;
@@ -921,7 +962,8 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
       const StageMeta mt = meta[s];
       if (mt.b < 0) { mbar_arrive(&pready[s]); break; }
       if (mt.flags & kFirst) {
-        named_bar_sync(2, 128);  // everyone is done with the previous segment's max
+        // everyone is done with the previous segment's max
+        if (!group_sync(pbar, pphase)) { set_timeout(p.status, kSiteVFull); abort_flag = 1; break; }
         // max of the sequence's logits: the split reduction over its K-pass segments
         const int32_t f0 = p.prefix[mt.b], f1 = p.prefix[mt.b + 1];
         const int32_t i0 = part_owner(f0, ptk), i1 = part_owner(f1 - 1, ptk);
@@ -933,7 +975,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
           }
           sM[h] = M;
         }
-        named_bar_sync(2, 128);
+        if (!group_sync(pbar, pphase)) { set_timeout(p.status, kSiteVFull); abort_flag = 1; break; }
         lsum = 0.f;
       }
       const float* lt = reinterpret_cast<const float*>(ltiles + static_cast<size_t>(s) * p.ltile_bytes);
@@ -992,13 +1034,13 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
         mbar_arrive(tfree);
         // per-segment normaliser of every head
         sRed[et] = lsum;
-        named_bar_sync(2, 128);
+        if (!group_sync(pbar, pphase)) { set_timeout(p.status, kSiteVFull); abort_flag = 1; break; }
         if (rr == 0 && et < p.H) {
           float Ls = 0.f;
           for (int i = et; i < 128; i += p.npad) Ls += sRed[i];
           p.lpart[slot * p.H + et] = Ls;
         }
-        named_bar_sync(2, 128);
+        if (!group_sync(pbar, pphase)) { set_timeout(p.status, kSiteVFull); abort_flag = 1; break; }
         ++seg;
       }
     }

@@ -170,6 +170,18 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Bounded barrier of a thread group on an mbarrier initialised with the
+// group's size: every member arrives, then waits for the phase `phase` (its own
+// count of the group's syncs so far).  Writes to shared memory before the sync
+// are visible after it (arrive releases, the wait acquires).  Returns false if
+// the wait ran out (a member stopped early); the caller records a timeout.
+__device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase) {
+  mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, phase & 1);
+  ++phase;
+  return ok;
+}
+
 // ------------------------------------------------ programmatic dependent launch
 // A grid launched with programmatic stream serialisation may start before the
 // previous grid in the stream has finished.  griddep_wait() blocks until that

@@ -206,7 +206,7 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   if (p.k_stages > 8) p.k_stages = 8;
   if (p.k_stages < 2) p.k_stages = 2;
   p.k_smem = static_cast<size_t>(p.k_stages) * p.k_stage_bytes + p.k_stages * sizeof(StageMeta) +
-             2 * p.k_stages * sizeof(uint64_t) + (kKConsumers / p.L) * sizeof(float);
+             (2 * p.k_stages + 1) * sizeof(uint64_t) + (kKConsumers / p.L) * sizeof(float);
   p.k_ctas = sms * STARKV_K_CTAS_PER_SM;
 
   // Grouped queries (G >= 2, H >= 8) with at most 16 KV heads: the K pass runs
@@ -270,7 +270,7 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   if (p.v_stages > 8) p.v_stages = 8;
   if (p.v_stages < 2) p.v_stages = 2;
   p.v_smem = 1024 + static_cast<size_t>(p.v_stages) * stage + p.v_stages * sizeof(StageMeta) +
-             (3 * p.v_stages + 3) * sizeof(uint64_t) + (p.npad + 128) * sizeof(float);
+             (3 * p.v_stages + 4) * sizeof(uint64_t) + (p.npad + 128) * sizeof(float);
   int per_sm = static_cast<int>((227u * 1024u) / (p.v_smem + 1024));
   if (per_sm > static_cast<int>(512 / p.tmem_cols)) per_sm = 512 / p.tmem_cols;
   if (per_sm < 1) per_sm = 1;
@@ -624,7 +624,8 @@ namespace {
 starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len, const void* q,
                           const void* B_K, const void* B_V, const void* k_cache, const void* v_cache,
                           const int32_t* block_tables, const int32_t* seq_lens, float scale, void* workspace,
-                          size_t workspace_bytes, void* out, void* stream, void* const* stage_events) {
+                          size_t workspace_bytes, void* out, void* stream, void* const* stage_events,
+                          const int32_t* row_seq = nullptr) {
   DecodePlan pl;
   starkv_status st = make_plan(desc, batch, max_seq_len, &pl);
   if (st != STARKV_OK) return st;
@@ -695,7 +696,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
 
   KPassParams kp;
   kp.k_cache = static_cast<const __half*>(k_cache);
-  kp.tables = block_tables; kp.teff = teff; kp.prefix = prefix; kp.qt = qt;
+  kp.tables = block_tables; kp.row_seq = row_seq; kp.teff = teff; kp.prefix = prefix; kp.qt = qt;
   kp.logits = logits; kp.mpart = mpart; kp.status = status;
   kp.B = batch; kp.H = pl.H; kp.log2H = pl.log2H; kp.r = pl.r; kp.MB = pl.MB; kp.NB = pl.NB; kp.t_pad = pl.t_pad;
   kp.Hkv = pl.Hkv; kp.log2G = pl.log2G;
@@ -709,7 +710,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
                        static_cast<uint32_t>(pl.ktc_brows)))
       return STARKV_ERR_CUDA;
     KPassTCParams tp;
-    tp.tables = block_tables; tp.teff = teff; tp.prefix = prefix;
+    tp.tables = block_tables; tp.row_seq = row_seq; tp.teff = teff; tp.prefix = prefix;
     tp.logits = logits; tp.mpart = mpart; tp.status = status;
     tp.B = batch; tp.log2G = pl.log2G; tp.log2Hkv = pl.log2H - pl.log2G;
     tp.MB = pl.MB; tp.NB = pl.NB; tp.t_pad = pl.t_pad;
@@ -727,7 +728,8 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   mark(2);
 
   VPassParams vp;
-  vp.tables = block_tables; vp.teff = teff; vp.prefix = prefix; vp.logits = logits; vp.mpart = mpart;
+  vp.tables = block_tables; vp.row_seq = row_seq; vp.teff = teff; vp.prefix = prefix; vp.logits = logits;
+  vp.mpart = mpart;
   vp.zpart = zpart; vp.lpart = lpart; vp.status = status;
   vp.B = batch; vp.H = pl.H; vp.npad = pl.npad; vp.MB = pl.MB; vp.NB = pl.NB; vp.R = pl.R;
   vp.t_pad = pl.t_pad; vp.r_range = pl.r_range; vp.n_rr = pl.n_rr; vp.v_slots = pl.ws.v_slots;
@@ -767,6 +769,43 @@ starkv_status starkv_paged_decode(const starkv_layer_desc* desc, int32_t batch, 
                                   float scale, void* workspace, size_t workspace_bytes, void* out, void* stream) {
   return decode_impl(desc, batch, max_seq_len, q, B_K, B_V, k_cache, v_cache, block_tables, seq_lens, scale,
                      workspace, workspace_bytes, out, stream, nullptr);
+}
+
+// Prefill workspace: the decode workspace of n_rows rows, then the rows'
+// sequence map and lengths (int32 [n_rows] each).
+size_t prefill_rows_offset(const DecodePlan& pl) { return align_up(pl.ws.total_bytes, 256); }
+
+size_t starkv_prefill_workspace_bytes(const starkv_layer_desc* desc, int32_t n_rows, int32_t max_seq_len) {
+  DecodePlan pl;
+  if (n_rows < 0 || make_plan(desc, n_rows, max_seq_len, &pl) != STARKV_OK) return 0;
+  return prefill_rows_offset(pl) + align_up(static_cast<size_t>(n_rows) * 8, 256);
+}
+
+starkv_status starkv_paged_prefill(const starkv_layer_desc* desc, int32_t n_seqs, int32_t n_rows, int32_t max_seq_len,
+                                   const void* q, const void* B_K, const void* B_V, const void* k_cache,
+                                   const void* v_cache, const int32_t* block_tables, const int32_t* starts,
+                                   const int32_t* row_offsets, float scale, void* workspace, size_t workspace_bytes,
+                                   void* out, void* stream) {
+  DecodePlan pl;
+  if (n_seqs < 0 || n_rows < 0) return STARKV_ERR_INVALID_ARG;
+  starkv_status st = make_plan(desc, n_rows, max_seq_len, &pl);
+  if (st != STARKV_OK) return st;
+  if (n_rows == 0) return STARKV_OK;
+  if (n_seqs == 0 || !starts || !row_offsets || (reinterpret_cast<uintptr_t>(starts) & 3u) ||
+      (reinterpret_cast<uintptr_t>(row_offsets) & 3u))
+    return STARKV_ERR_INVALID_ARG;
+  const size_t need = prefill_rows_offset(pl) + align_up(static_cast<size_t>(n_rows) * 8, 256);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return STARKV_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* row_seq = reinterpret_cast<int32_t*>(ws + prefill_rows_offset(pl));
+  int32_t* row_len = row_seq + n_rows;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  PrefillRowsParams rp{starts, row_offsets, row_seq, row_len, n_seqs, n_rows};
+  if (launch(prefill_rows_kernel, dim3((n_rows + 255) / 256), dim3(256), 0, s, 1, rp) != cudaSuccess)
+    return STARKV_ERR_CUDA;
+  return decode_impl(desc, n_rows, max_seq_len, q, B_K, B_V, k_cache, v_cache, block_tables, row_len, scale,
+                     workspace, workspace_bytes, out, stream, nullptr, row_seq);
 }
 
 starkv_status starkv_paged_decode_profiled(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len,

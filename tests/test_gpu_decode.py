@@ -394,6 +394,48 @@ def test_decode_independent_of_workspace_contents(kv_heads):
     assert np.array_equal(outs[0].view(np.uint16), outs[1].view(np.uint16))
 
 
+# ------------------------------------------------------ chunked prefill
+
+def _prefill_check(kv_heads, starts, chunks, seed):
+    H, d = 32, 128
+    sh = W.LayerShape(H, d, 64, 512 if kv_heads else 2048, num_kv_heads=kv_heads)
+    starts = np.asarray(starts, np.int64)
+    chunks = np.asarray(chunks, np.int64)
+    # every chunk's codes are in the cache: the context is start + chunk tokens
+    wl = W.custom("prefill", seed, sh, starts + chunks, append=False)
+    Lh = W.host_layer(wl, 0)
+    Ld = D.device_layer(wl, 0, tables=Lh["tables"], nb=Lh["nb"])
+    n_rows = int(chunks.sum())
+    q = gen.codes_f16(gen.stream_key(seed, 77), n_rows, H * d, None).reshape(n_rows, H, d)
+    offsets = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    desc = desc_of(Ld)
+    max_len = int((starts + chunks).max())
+    wsb = S.starkv_prefill_workspace_bytes(desc, n_rows, max_len)
+    ws = torch.full((wsb,), 0xFF, dtype=torch.uint8, device="cuda")
+    out = torch.full((n_rows, H, d), float("nan"), dtype=torch.float16, device="cuda")
+    S.starkv_paged_prefill(desc, len(chunks), n_rows, max_len, dev(q), Ld["B_K"], Ld["B_V"], Ld["k_cache"],
+                           Ld["v_cache"], Ld["tables"], dev(starts.astype(np.int32)), dev(offsets), Ld["scale"],
+                           ws, wsb, out)
+    st, flags = S.starkv_decode_check(ws)
+    assert st == 0, (S.STATUS[st], flags)
+    got = out.float().cpu().numpy().astype(np.float64)
+    ref = O.prefill_attention(q, Lh["B_K"], Lh["B_V"], Lh["k_cache"], Lh["v_cache"], Lh["tables"], starts,
+                              chunks, Lh["scale"])
+    assert_close({r: got[r] for r in range(n_rows)}, {r: ref[r] for r in range(n_rows)})
+
+
+@pytest.mark.parametrize("kv_heads", [0, 8])
+def test_prefill_chunks_causal(kv_heads):
+    """A first chunk, an empty chunk, a mid-prompt chunk, a one-token chunk and a 64-token tail chunk."""
+    _prefill_check(kv_heads, starts=[0, 5, 200, 1000, 37], chunks=[37, 0, 150, 1, 64], seed=6060 + kv_heads)
+
+
+def test_prefill_rows_of_one_sequence_span_tiles():
+    """One sequence, a 300-token chunk after 700 cached tokens: rows span several K/V partitions."""
+    _prefill_check(0, starts=[700], chunks=[300], seed=6161)
+
+
 # ------------------------------------------------ grouped-query attention
 
 @pytest.mark.parametrize("H,Hkv,d,r,R", [
