@@ -62,6 +62,14 @@ __device__ __forceinline__ int32_t seq_of_page(const int32_t* prefix, int32_t B,
 
 __device__ __forceinline__ void set_flag(int32_t* status, int32_t f) { atomicOr(status, f); }
 
+// Float maximum through the integer atomics (ordered bit patterns: max over
+// signed ints for v >= 0, min over unsigned for v < 0); works on shared or
+// global memory.
+__device__ __forceinline__ void atomic_max_f32(float* addr, float v) {
+  if (__float_as_int(v) >= 0) atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));
+  else atomicMin(reinterpret_cast<unsigned int*>(addr), __float_as_uint(v));
+}
+
 // Block-table row of decode row b: row b itself, or, for rows that are query
 // tokens of a prefill chunk, the row of the sequence row_seq[b].
 __device__ __forceinline__ const int32_t* table_row(const int32_t* tables, const int32_t* row_seq, int32_t b, int MB) {
@@ -223,7 +231,7 @@ struct KPassParams {
   const int32_t* prefix;      // [B+1]
   const float* qt;            // [B][H][r]
   float* logits;              // [B][t_pad][H]
-  float* mpart;               // [k_slots][H]: max of the base-2 logits per segment
+  float* mpart;               // [k_slots][H]: max of the base-2 logits per segment (-inf on entry)
   int32_t* status;
   int B, H, log2H, r, MB, NB, t_pad;
   int Hkv, log2G;             // KV heads (codes per token) and log2(query heads per KV head)
@@ -272,15 +280,13 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
   StageMeta* meta = reinterpret_cast<StageMeta*>(smem + static_cast<size_t>(S) * p.stage_bytes);
   uint64_t* full = reinterpret_cast<uint64_t*>(meta + S);
   uint64_t* empty = full + S;
-  uint64_t* cbar = empty + S;                                // the consumers' segment-end sync
-  float* red = reinterpret_cast<float*>(cbar + 1);          // [kKConsumers / L]
+
   __shared__ volatile int32_t abort_flag;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], kKConsumers / 32); }
-    mbar_init(cbar, kKConsumers);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -382,7 +388,6 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
   float2 qv[CPT * 4];
   float m = -INFINITY;
   int cur_b = -1;
-  uint32_t cphase = 0;
   const uint64_t keep = policy_evict_last();   // logits: read back by the V pass
 
   for (uint32_t k = 0;; ++k) {
@@ -393,17 +398,9 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
     }
     const StageMeta mt = meta[s];
     if (mt.b != cur_b || mt.b < 0) {   // new sequence, or the end marker (b < 0)
-      if (cur_b >= 0) {
-        // per-segment max for every head: slot = sequence + CTA
-        if (sub == 0) red[pair0] = m;
-        if (!group_sync(cbar, cphase)) { set_timeout(p.status, kSiteKFull); abort_flag = 1; break; }
-        if (tid < p.H) {
-          float M = -INFINITY;
-          for (int g = tid; g < kPairsPerPass; g += p.H) M = fmaxf(M, red[g]);
-          p.mpart[static_cast<size_t>(cur_b + cta) * p.H + tid] = M;
-        }
-        if (!group_sync(cbar, cphase)) { set_timeout(p.status, kSiteKFull); abort_flag = 1; break; }
-      }
+      // per-segment max of every head (slot = sequence + CTA, -inf on entry),
+      // merged across this CTA's consumers by float-max atomics
+      if (cur_b >= 0 && sub == 0 && m > -INFINITY) atomic_max_f32(&p.mpart[static_cast<size_t>(cur_b + cta) * p.H + head], m);
       if (mt.b < 0) break;
       cur_b = mt.b;
       m = -INFINITY;
@@ -524,14 +521,6 @@ __device__ __forceinline__ void for_each_k_tile(const KPassTCParams& p, int64_t 
       if (!f(b, t0, min(tpt, te - t0), static_cast<int64_t>(base) + (t0 >> 4), t0 == ts, t0 + tpt >= te)) return;
     x = seg_end;
   }
-}
-
-// Float maximum through the integer atomics (ordered bit patterns: max over
-// signed ints for v >= 0, min over unsigned for v < 0); works on shared or
-// global memory.
-__device__ __forceinline__ void atomic_max_f32(float* addr, float v) {
-  if (__float_as_int(v) >= 0) atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));
-  else atomicMin(reinterpret_cast<unsigned int*>(addr), __float_as_uint(v));
 }
 
 template <int G, int H>   // query heads per KV head, query heads

@@ -206,7 +206,7 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   if (p.k_stages > 8) p.k_stages = 8;
   if (p.k_stages < 2) p.k_stages = 2;
   p.k_smem = static_cast<size_t>(p.k_stages) * p.k_stage_bytes + p.k_stages * sizeof(StageMeta) +
-             (2 * p.k_stages + 1) * sizeof(uint64_t) + (kKConsumers / p.L) * sizeof(float);
+             2 * p.k_stages * sizeof(uint64_t);
   p.k_ctas = sms * STARKV_K_CTAS_PER_SM;
 
   // Grouped queries (G >= 2, H >= 8) with at most 16 KV heads: the K pass runs
@@ -679,7 +679,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   ap.qt = qt; ap.prefix = prefix; ap.teff = teff; ap.status = status;
   __half* qth = pl.ktc ? reinterpret_cast<__half*>(ws + pl.ws.qth_off) : nullptr;
   ap.qth = qth;
-  ap.mpart_init = pl.ktc ? mpart : nullptr;   // the tensor-core K pass merges segment maxima by atomics
+  ap.mpart_init = mpart;   // both K passes merge the segment maxima by float-max atomics
   ap.n_mpart = pl.ws.k_slots * pl.H;
   ap.B = batch; ap.H = pl.H; ap.d = pl.d; ap.r = pl.r; ap.cap = pl.cap; ap.log2G = pl.log2G;
   ap.coef = scale * kLog2e;
