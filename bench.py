@@ -60,6 +60,8 @@ def parse_args():
     ap.add_argument("--batch", type=int, default=0,
                     help="profiling only: override the batch with uniform lengths --seq")
     ap.add_argument("--seq", type=int, default=0)
+    ap.add_argument("--graph", action="store_true",
+                    help="time the step (every layer's append + decode) as one captured CUDA graph")
     ap.add_argument("--prefill-chunk", type=int, default=0,
                     help="instead of decode: a chunked-prefill step, each sequence compressing its last N "
                          "tokens into the cache and attending causally over its whole context")
@@ -92,8 +94,10 @@ NCU_TRAFFIC_PER_TOKEN = {
     # batch 32, context 8192 (MHA): CUDA-core K pass, V pass
     (32, 32, 64, 2048): {"kpass": (1074215168 + 6370048) / (32 * 8192),
                          "vpass": (1108390400 + 4740096) / (32 * 8192)},
-    # batch 64, context 8192 (32 query heads over 8 KV heads): tensor-core K pass
-    (32, 8, 64, 512): {"kpass": (537.648640e6 + 8.424192e6) / (64 * 8192)},
+    # batch 64, context 8192 (32 query heads over 8 KV heads): tensor-core K pass, V pass
+    # (cold replay: the V pass's figure includes the fp32 logits, read from L2 when live)
+    (32, 8, 64, 512): {"kpass": (537.648640e6 + 8.424192e6) / (64 * 8192),
+                       "vpass": (604.289792e6 + 6.300672e6) / (64 * 8192)},
 }
 
 
@@ -204,6 +208,7 @@ def run_ours(args):
     n_ev = 6
 
     def step(evs=None, app_evs=None, li_prof=None):
+        stream = torch.cuda.current_stream()       # the capture stream while a graph is recorded
         for li, L in enumerate(layers):
             if app_evs is not None:
                 app_evs[li][0].record(stream)
@@ -225,6 +230,18 @@ def run_ours(args):
     st, flags = S.starkv_decode_check(ws, stream)
     if st != 0:
         raise RuntimeError(f"device status {S.STATUS[st]} flags {flags}")
+    graph = None
+    if args.graph:
+        # the whole step (every layer) as one graph; the library makes no host
+        # round trips, allocations or synchronisations inside a call
+        graph = torch.cuda.CUDAGraph()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+    run_step = graph.replay if graph is not None else step
 
     # ---------------- device-timed region: inputs resident, codes >> L2 per step
     K = args.steps
@@ -242,7 +259,7 @@ def run_ours(args):
     time.sleep(0.3)
     t0.record(stream)
     for i in range(K):
-        step()
+        run_step()
     t1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -339,7 +356,8 @@ def run_ours(args):
                    "max_seq_len": max_len, "layers": len(layers),
                    "step": "compress-append of one token per sequence + paged decode, every layer",
                    "l2": "inputs larger than L2 (code pools of %.2f GiB read per step)" % ((k_bytes + v_bytes) / 2**30),
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "launch": "one CUDA graph per step" if graph is not None else "stream launches (PDL)"},
         "hbm": {"step_algorithmic_bytes": step_bytes,
                 "step_GBps": round(step_bytes / (ms * 1e-3) / 1e9, 1),
                 "frac_of_8TBps": round(step_bytes / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4),

@@ -394,6 +394,40 @@ def test_decode_independent_of_workspace_contents(kv_heads):
     assert np.array_equal(outs[0].view(np.uint16), outs[1].view(np.uint16))
 
 
+def test_append_and_decode_in_cuda_graph_match_stream_launches():
+    """Three layers of append + decode captured as one CUDA graph and replayed: bit-identical outputs."""
+    full = W.workload(4)
+    wl = W.Workload("cb-graph", full.seed, 6, full.layers, full.ctx_lens[:6])
+    layers = [D.device_layer(wl, li) for li in range(3)]
+    descs = [desc_of(L) for L in layers]
+    B, T = wl.batch, wl.max_seq_len
+    wsb = max(S.starkv_decode_workspace_bytes(dsc, B, T) for dsc in descs)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    pools = [(L["k_cache"].clone(), L["v_cache"].clone()) for L in layers]
+
+    def run(outs):
+        st = torch.cuda.current_stream()
+        for L, dsc, o, (kc, vc) in zip(layers, descs, outs, pools):
+            S.starkv_compress_append(dsc, B, L["k"], L["v"], L["A_K"], L["A_V"], L["tables"], L["ctx_lens"],
+                                     kc, vc, stream=st)
+            S.starkv_paged_decode(dsc, B, T, L["q"], L["B_K"], L["B_V"], kc, vc, L["tables"], L["seq_lens"],
+                                  L["scale"], ws, wsb, o, stream=st)
+
+    eager = [torch.empty((B, L["H"], L["d"]), dtype=torch.float16, device="cuda") for L in layers]
+    run(eager)
+    torch.cuda.synchronize()
+    graphed = [torch.full_like(o, float("nan")) for o in eager]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run(graphed)
+    g.replay()
+    torch.cuda.synchronize()
+    st, flags = S.starkv_decode_check(ws)
+    assert st == 0, (S.STATUS[st], flags)
+    for a, b in zip(eager, graphed):
+        assert np.array_equal(a.cpu().numpy().view(np.uint16), b.cpu().numpy().view(np.uint16))
+
+
 # ------------------------------------------------------ chunked prefill
 
 def _prefill_check(kv_heads, starts, chunks, seed):
