@@ -133,3 +133,34 @@ def test_compress_store_argument_errors(lib):
     a = list(args); a[1] = 0
     assert S.starkv_compress_store(*a, stream=0, check=False) == 0
     assert S.starkv_compress_store(_desc(block_size=8), *args[1:], stream=0, check=False) == 2
+
+
+@pytest.mark.parametrize("kv,expect", [(-1, 1), (12, 2), (64, 2), (3, 2)])
+def test_kv_head_count_validation(lib, kv, expect):
+    d = _desc(num_kv_heads=kv)
+    fake = 1 << 20
+    st = S.starkv_paged_decode(d, 1, 16, fake, fake, fake, fake, fake, fake, fake, 0.1, fake,
+                               1 << 30, fake, stream=0, check=False)
+    assert st == expect
+    assert S.starkv_decode_workspace_bytes(d, 1, 16) == 0
+
+
+def test_prefill_argument_errors(lib):
+    d = _desc()
+    fake = 1 << 20
+    need = S.starkv_prefill_workspace_bytes(d, 40, 1024)
+    assert need > S.starkv_decode_workspace_bytes(d, 40, 1024) > 0
+    args = [d, 2, 40, 1024, fake, fake, fake, fake, fake, fake, fake, fake, 0.1, fake, need, fake]
+
+    def call(i, v):
+        a = list(args); a[i] = v
+        return S.starkv_paged_prefill(*a, stream=0, check=False)
+    assert call(1, -1) == 1                      # negative sequence count
+    assert call(2, -5) == 1                      # negative row count
+    assert call(1, 0) == 1                       # rows but no sequences
+    assert call(10, None) == 1                   # null starts
+    assert call(11, fake + 2) == 1               # misaligned row offsets
+    assert call(14, need - 1) == 3               # workspace too small for the row arrays
+    assert call(3, 64 * 16 + 1) == 1             # length bound above table capacity
+    assert call(2, 0) == 0                       # no rows: no-op
+    assert S.starkv_prefill_workspace_bytes(d, -1, 1024) == 0
