@@ -629,6 +629,8 @@ def run_prefill(args):
 
 def main():
     args = parse_args()
+    if args.impl == "reference" and args.prefill_chunk:
+        raise SystemExit("the reference arm times the decode step; run --prefill-chunk with --impl ours")
     if args.impl == "reference":
         run_reference(args)
     elif args.prefill_chunk:

@@ -63,3 +63,14 @@ def test_capacity_helpers_reject_bad_input():
     assert S.starkv_num_blocks(-1, 10, 16) == -1
     assert S.starkv_num_blocks(100, 0, 16) == -1
     assert S.starkv_num_blocks(0, 10, 16) == 0
+
+
+def test_grouped_query_cache_costs_kv_heads_only():
+    """With grouped queries a token stores codes per KV head: a Llama-3-8B-shaped model (32 layers of
+    8 KV heads, d = 128) costs 2 * 32 * (8*128 + 8*128) bytes per token at full rank, a quarter of
+    the 32-head cost, and 2 * 32 * (8*64 + 512) at the 50% ranks of the grouped-query workload."""
+    full = ([8] * 32, [128] * 32, [8 * 128] * 32)
+    assert O.kv_bytes_per_token(*full) == S.starkv_kv_bytes_per_token(*full) == 2 * 32 * 2048
+    assert O.kv_bytes_per_token([32] * 32, [128] * 32, [4096] * 32) == 4 * O.kv_bytes_per_token(*full)
+    half = ([8] * 32, [64] * 32, [512] * 32)
+    assert O.kv_bytes_per_token(*half) == S.starkv_kv_bytes_per_token(*half) == 2 * 32 * 1024
