@@ -157,16 +157,31 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbParams p) {
       p.teff[b] = T;
       s += (T + kBlock - 1) / kBlock;
     }
-    part[tid] = s;
+    // exclusive scan of the 256 per-thread page counts: warp scans, then the warp totals
+    const int lane = tid & 31, warp = tid >> 5;
+    int32_t v = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (lane == 31) part[warp] = v;
     __syncthreads();
-    if (tid == 0) {
-      int32_t acc = 0;
-      for (int i = 0; i < 256; ++i) { int32_t v = part[i]; part[i] = acc; acc += v; }
-      p.prefix[p.B] = acc;
-      *p.status = bad ? STARKV_FLAG_BAD_SEQ_LEN : 0;
+    if (warp == 0) {
+      int32_t w = lane < 8 ? part[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      if (lane < 8) part[8 + lane] = w;       // inclusive totals of warps 0..lane
     }
     __syncthreads();
-    int32_t acc = part[tid];
+    int32_t acc = v - s + (warp > 0 ? part[8 + warp - 1] : 0);
+    if (tid == 255) {
+      p.prefix[p.B] = acc + s;
+      *p.status = bad ? STARKV_FLAG_BAD_SEQ_LEN : 0;
+    }
     for (int b = b0; b < b0 + per && b < p.B; ++b) {
       p.prefix[b] = acc;
       acc += (p.teff[b] + kBlock - 1) / kBlock;
