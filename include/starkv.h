@@ -5,12 +5,16 @@
  * the full-dimension cache: head-wise for K and joint across heads for V,
  * kept in a compressed paged format (Proxima README, "Low-rank KV Cache
  * Compression for vLLM", opening method paragraph; tenosra.com/proxima, first
- * paragraph).  This library implements the two per-token steps of that cache:
+ * paragraph).  This library implements the steps that read and write that
+ * cache on the GPU:
  *
  *   compress-and-append : codes of each sequence's new token written into the
- *                         paged pools;
+ *                         paged pools (and compress-store: many rows at
+ *                         explicit slots, e.g. a prompt chunk);
  *   paged decode        : single-query attention computed straight from the
- *                         codes, never materialising full keys or values.
+ *                         codes, never materialising full keys or values;
+ *   chunked prefill     : causal attention of prompt chunks over the codes;
+ * plus host helpers for rank selection and cache capacity.
  *
  * Formulation (head_dim d, H query heads, Hkv KV heads with query head h
  * reading KV head g(h) = h / (H/Hkv), K rank r per KV head, V joint rank R):

@@ -29,6 +29,7 @@ EXPORTED = (
     "starkv_paged_decode_profiled", "starkv_paged_decode_static",
     "starkv_decode_check", "starkv_decode_workspace_layout", "starkv_status_string",
     "starkv_rank_from_spectrum", "starkv_version", "starkv_kv_bytes_per_token", "starkv_num_blocks",
+    "starkv_prefill_workspace_bytes", "starkv_paged_prefill",
 )
 
 

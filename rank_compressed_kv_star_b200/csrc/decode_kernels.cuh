@@ -2,13 +2,19 @@
 //
 // One decode is five launches on the caller's stream, each launched with
 // programmatic stream serialisation (see griddep_wait):
-//   1. absorb      q~ = log2(e)*scale * q . B_K[h]^T; page prefix sums; status reset
+//   1. absorb      q~ = log2(e)*scale * q . B_K[g(h)]^T; page prefix sums; status
+//                  reset; segment maxima set to -inf
 //   2. kpass       base-2 logits s = q~ . c_K over the K pages, per-segment max
+//                  (kpass_kernel on CUDA cores for multi-head attention,
+//                  kpass_tc_kernel on tcgen05 for grouped queries)
 //   3. vpass       split reduction M = max over the sequence's K segments, then
 //                  Z = sum_t w c_V on tcgen05 tensor cores with w = fp16(exp2(s - M)),
 //                  and the normaliser L = sum_t w
 //   4. zfinal      Z / L summed over segments, split into fp16 hi + lo
-//   5. upproj      out_h = (Z_h / L) . B_V[:, h*d:(h+1)*d] on tcgen05 -> fp16
+//   5. upproj      out_h = (Z_h / L) . B_V[:, g(h)*d:(g(h)+1)*d] on tcgen05 -> fp16
+// with g(h) = h / (H / Hkv) the KV head of query head h (g(h) = h without
+// grouping).  A chunked prefill adds prefill_rows_kernel in front: each query
+// token of a chunk becomes a decode row of its sequence.
 //
 // The formulation (head-wise K with the query absorbed, joint V applied after
 // the weighted sum of codes) follows the STAR-KV description in the Proxima

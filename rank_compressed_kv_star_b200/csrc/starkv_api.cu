@@ -498,7 +498,7 @@ const char* starkv_status_string(starkv_status s) {
   return "STARKV_UNKNOWN_STATUS";
 }
 
-int32_t starkv_version(void) { return 100; }
+int32_t starkv_version(void) { return 200; }
 
 int64_t starkv_kv_bytes_per_token(int32_t n_layers, const int32_t* num_heads, const int32_t* k_ranks,
                                   const int32_t* v_ranks) {
