@@ -478,6 +478,8 @@ def test_prefill_rows_of_one_sequence_span_tiles():
     (16, 1, 128, 64, 128),      # one KV head (multi-query)
     (64, 8, 128, 128, 1024),    # 8 per KV head, r = d
     (8, 2, 64, 16, 128),        # small pages: 8-page K stages
+    (64, 32, 64, 64, 1024),     # 32 KV heads: the CUDA-core K pass with 2 query heads per KV head
+    (4, 2, 64, 16, 64),         # 4 query heads: the CUDA-core K pass
 ])
 def test_decode_grouped_query(H, Hkv, d, r, R):
     sh = W.LayerShape(H, d, r, R, num_kv_heads=Hkv)
