@@ -508,3 +508,24 @@ def test_slot_mapped_store_equals_block_table_append():
     s = O.compress_store(L["k"], L["v"], L["A_K"], L["A_V"], slots, L["k_cache"], L["v_cache"])
     for x, y in zip(a[2:], s[2:]):
         assert np.array_equal(x.view(np.uint16), y.view(np.uint16))
+
+
+def test_grouped_query_store_equals_append_and_contiguous_equals_paged():
+    """With 2 KV heads under 8 query heads: slot-mapped store == block-table append (bitwise), and
+    decode over contiguous code arrays == decode through the block tables (bitwise)."""
+    sh = W.LayerShape(8, 32, 16, 64, num_kv_heads=2)
+    wl = W.custom("gqa-store", 43, sh, [37, 100, 0, 15], append=True)
+    L = W.host_layer(wl, 0)
+    pos = L["ctx_lens"]
+    slots = [int(L["tables"][b][pos[b] // 16]) * 16 + int(pos[b] % 16) for b in range(wl.batch)]
+    a = O.compress_append(L["k"], L["v"], L["A_K"], L["A_V"], L["tables"], pos, L["k_cache"], L["v_cache"])
+    s = O.compress_store(L["k"], L["v"], L["A_K"], L["A_V"], slots, L["k_cache"], L["v_cache"])
+    for x, y in zip(a[2:], s[2:]):
+        assert np.array_equal(x.view(np.uint16), y.view(np.uint16))
+    kc, vc = a[2], a[3]
+    T = L["seq_lens"]
+    paged = O.decode_explicit(L["q"], L["B_K"], L["B_V"], kc, vc, L["tables"], T, L["scale"])
+    contig = O.decode_contiguous(L["q"], L["B_K"], L["B_V"],
+                                 [O.gather(kc, L["tables"][b], int(T[b])) for b in range(wl.batch)],
+                                 [O.gather(vc, L["tables"][b], int(T[b])) for b in range(wl.batch)], L["scale"])
+    assert np.array_equal(paged, contig)
