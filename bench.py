@@ -87,18 +87,13 @@ def whole_job_tokens_per_s(world: int, batch_per_rank: int, ms_per_step_max: flo
 # DRAM bytes (read + write) per processed token of the two streaming kernels,
 # from ncu captures (dram__bytes_read.sum + dram__bytes_write.sum of one
 # launch); traffic grows in proportion to the tokens processed.  Keyed by
-# layer geometry (query heads, KV heads, K rank, V rank); valid only for the
-# kernels as they were captured (the summaries under profiles/ give the
-# commands).
-NCU_TRAFFIC_PER_TOKEN = {
-    # batch 32, context 8192 (MHA): CUDA-core K pass, V pass
-    (32, 32, 64, 2048): {"kpass": (1074215168 + 6370048) / (32 * 8192),
-                         "vpass": (1108390400 + 4740096) / (32 * 8192)},
-    # batch 64, context 8192 (32 query heads over 8 KV heads): tensor-core K pass, V pass
-    # (cold replay: the V pass's figure includes the fp32 logits, read from L2 when live)
-    (32, 8, 64, 512): {"kpass": (537.648640e6 + 8.424192e6) / (64 * 8192),
-                       "vpass": (604.289792e6 + 6.300672e6) / (64 * 8192)},
-}
+# layer geometry (query heads, KV heads, K rank, V rank).  A figure is only
+# valid for the kernels as they were captured, so an entry is emptied when its
+# kernel changes and refilled from a new capture (the summaries under
+# profiles/ give the commands).  Both passes have changed since the last
+# captures (segment maxima by atomics, bounded V-pass syncs, the block-table
+# indirection for prefill rows), so no geometry has a current figure.
+NCU_TRAFFIC_PER_TOKEN: dict = {}
 
 
 def measured_peaks():
