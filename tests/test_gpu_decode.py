@@ -173,6 +173,13 @@ def test_decode_rank_variants(r, R):
     _full_check(wl)
 
 
+def test_decode_largest_head_dim_and_k_rank():
+    """head_dim 256 and K rank 256 (the largest the kernels take), V rank 4096, ragged lengths."""
+    sh = W.LayerShape(16, 256, 256, 4096)
+    wl = W.custom("d256", 256, sh, [1, 17, 100], append=False)
+    _full_check(wl)
+
+
 def test_decode_small_heads_and_dims():
     sh = W.LayerShape(8, 64, 32, 256)
     wl = W.custom("h8", 55, sh, [3, 64, 129], append=False)
