@@ -48,6 +48,8 @@
  *    outside [0, num_blocks), a length above the table's capacity, a timed-out
  *    internal wait) set bits of a device status word that
  *    starkv_decode_check() reads back; the affected output is undefined.
+ *  - The library keeps no state between calls, except the process-wide test
+ *    hook set by starkv_set_wait_test_hook() (off unless a test sets it).
  */
 #ifndef STARKV_H_
 #define STARKV_H_
@@ -105,30 +107,40 @@ typedef struct {
  *   positions     int32 [batch]: the sequence length BEFORE this append
  *   k_cache       fp16 [num_blocks][16][Hkv][r]   (in/out)
  *   v_cache       fp16 [num_blocks][16][R]      (in/out)
+ *   status        optional device int32 (NULL: not reported), 4-byte aligned:
+ *                 every skipped target OR-s a flag into it --
+ *                 STARKV_FLAG_BAD_SEQ_LEN for a position outside [0,
+ *                 max_blocks_per_seq*16), STARKV_FLAG_BAD_BLOCK_ID for a block
+ *                 id outside [0, num_blocks).  The library never clears it:
+ *                 zero it before the calls it should cover, then read it with
+ *                 starkv_decode_check(status, ...).
  *
  * Targets must be distinct slots (no page shared between sequences).  A target
- * whose position or block id is out of range is skipped.  batch == 0 is a
- * no-op.  Cites: README method paragraph ("stored in a compressed paged format").
+ * whose position or block id is out of range is skipped (and flagged in
+ * `status`).  batch == 0 is a no-op.  Cites: README method paragraph ("stored
+ * in a compressed paged format").
  */
 starkv_status starkv_compress_append(const starkv_layer_desc* desc, int32_t batch, const void* k,
                                      const void* v, const void* A_K, const void* A_V,
                                      const int32_t* block_tables, const int32_t* positions,
-                                     void* k_cache, void* v_cache, void* stream);
+                                     void* k_cache, void* v_cache, int32_t* status, void* stream);
 
 /*
  * starkv_compress_store -- compress n_tokens rows of k, v (for instance a
  * prompt at prefill) and store each row's codes at an explicit flat slot:
  * slot_mapping[i] = page * 16 + offset, int32 [n_tokens].  Same arithmetic,
  * layouts and rounding as starkv_compress_append; rows whose slot is outside
- * [0, num_blocks*16) are skipped; targets must be distinct.  k, v fp16
- * [n_tokens][Hkv][d].  Cites: README method paragraph (codes "stored in a
- * compressed paged format"); the flat slot is the paged address
- * block_table[b][t/16]*16 + t%16 precomputed by the caller.
+ * [0, num_blocks*16) are skipped and, when `status` is non-NULL, flagged with
+ * STARKV_FLAG_BAD_BLOCK_ID (same convention as starkv_compress_append);
+ * targets must be distinct.  k, v fp16 [n_tokens][Hkv][d].  Cites: README
+ * method paragraph (codes "stored in a compressed paged format"); the flat
+ * slot is the paged address block_table[b][t/16]*16 + t%16 precomputed by
+ * the caller.
  */
 starkv_status starkv_compress_store(const starkv_layer_desc* desc, int32_t n_tokens, const void* k,
                                     const void* v, const void* A_K, const void* A_V,
                                     const int32_t* slot_mapping, void* k_cache, void* v_cache,
-                                    void* stream);
+                                    int32_t* status, void* stream);
 
 /*
  * starkv_decode_workspace_bytes -- device scratch needed by starkv_paged_decode
@@ -246,11 +258,34 @@ starkv_status starkv_paged_decode_static(const starkv_layer_desc* desc, int32_t 
 
 /*
  * starkv_decode_check -- synchronise `stream` and read the device status word
- * the last decode on `workspace` left.  *flags_out receives STARKV_FLAG_* bits
- * (0 when clean).  Returns STARKV_OK when clean, STARKV_ERR_TIMEOUT when the
- * timeout bit is set, STARKV_ERR_DEVICE_CHECK for other bits.
+ * at `workspace` (the first int32 of a decode or prefill workspace, or an
+ * append `status` word).  For a workspace it is the status of the last decode
+ * or prefill call that returned STARKV_OK with that workspace, calls with
+ * nothing to compute (batch 0, max_seq_len 0, n_rows 0) included: those clear
+ * the word.  *flags_out receives STARKV_FLAG_* bits (0 when clean).  Returns
+ * STARKV_OK when clean, STARKV_ERR_TIMEOUT when the timeout bit is set,
+ * STARKV_ERR_DEVICE_CHECK for other bits.
  */
 starkv_status starkv_decode_check(const void* workspace, void* stream, int32_t* flags_out);
+
+/*
+ * starkv_set_wait_test_hook -- TEST HOOK for the failure path of the device
+ * pipelines; leave it off in production.  Every internal pipeline wait is
+ * bounded (about two seconds by default) and, when the bound runs out, sets
+ * STARKV_FLAG_TIMEOUT plus a site bit and leaves its loop instead of hanging.
+ * To exercise that path without faulting anything, a test can
+ *   wait_limit_us  shorten the bound of every wait to this many microseconds on
+ *                  the CURRENT device (0 restores the default), and
+ *   drop_k_stage   make the K pass of every later decode skip the copy of its
+ *                  ring stage number drop_k_stage in every CTA (-1: off), so
+ *                  that the waits on that stage run out while no copy is in
+ *                  flight.
+ * Process-wide state; not to be changed while decodes are in flight.  Returns
+ * STARKV_ERR_INVALID_ARG for drop_k_stage < -1 and STARKV_ERR_CUDA when the
+ * device bound cannot be set.  The method pages have no counterpart to this
+ * entry point.
+ */
+starkv_status starkv_set_wait_test_hook(uint32_t wait_limit_us, int32_t drop_k_stage);
 
 /*
  * Workspace layout (byte offsets into the decode workspace), exposed so that

@@ -29,7 +29,7 @@ EXPORTED = (
     "starkv_paged_decode_profiled", "starkv_paged_decode_static",
     "starkv_decode_check", "starkv_decode_workspace_layout", "starkv_status_string",
     "starkv_rank_from_spectrum", "starkv_version", "starkv_kv_bytes_per_token", "starkv_num_blocks",
-    "starkv_prefill_workspace_bytes", "starkv_paged_prefill",
+    "starkv_prefill_workspace_bytes", "starkv_paged_prefill", "starkv_set_wait_test_hook",
 )
 
 
@@ -80,9 +80,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib = ctypes.CDLL(path)
     P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     DP = ctypes.POINTER(LayerDesc)
-    lib.starkv_compress_append.argtypes = [DP, I32, P, P, P, P, P, P, P, P, P]
+    lib.starkv_compress_append.argtypes = [DP, I32, P, P, P, P, P, P, P, P, P, P]
     lib.starkv_compress_append.restype = ctypes.c_int
-    lib.starkv_compress_store.argtypes = [DP, I32, P, P, P, P, P, P, P, P]
+    lib.starkv_compress_store.argtypes = [DP, I32, P, P, P, P, P, P, P, P, P]
     lib.starkv_compress_store.restype = ctypes.c_int
     lib.starkv_decode_workspace_bytes.argtypes = [DP, I32, I32]
     lib.starkv_decode_workspace_bytes.restype = SZ
@@ -113,6 +113,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.starkv_kv_bytes_per_token.restype = I64
     lib.starkv_num_blocks.argtypes = [I64, I64, I32]
     lib.starkv_num_blocks.restype = I64
+    lib.starkv_set_wait_test_hook.argtypes = [ctypes.c_uint32, I32]
+    lib.starkv_set_wait_test_hook.restype = ctypes.c_int
     lib.starkv_version.argtypes = []
     lib.starkv_version.restype = I32
     _lib = lib
@@ -146,20 +148,21 @@ def _check(status: int, where: str):
 
 
 def starkv_compress_append(desc: LayerDesc, batch: int, k, v, A_K, A_V, block_tables, positions,
-                           k_cache, v_cache, stream=None, check: bool = True) -> int:
+                           k_cache, v_cache, stream=None, check: bool = True, status=None) -> int:
+    """``status``: optional device int32 word that skipped targets flag (never cleared by the call)."""
     st = load_library().starkv_compress_append(
         _desc_ref(desc), batch, _ptr(k), _ptr(v), _ptr(A_K), _ptr(A_V), _ptr(block_tables),
-        _ptr(positions), _ptr(k_cache), _ptr(v_cache), _stream(stream))
+        _ptr(positions), _ptr(k_cache), _ptr(v_cache), _ptr(status), _stream(stream))
     if check:
         _check(st, "starkv_compress_append")
     return st
 
 
 def starkv_compress_store(desc: LayerDesc, n_tokens: int, k, v, A_K, A_V, slot_mapping, k_cache,
-                          v_cache, stream=None, check: bool = True) -> int:
+                          v_cache, stream=None, check: bool = True, status=None) -> int:
     st = load_library().starkv_compress_store(
         _desc_ref(desc), n_tokens, _ptr(k), _ptr(v), _ptr(A_K), _ptr(A_V), _ptr(slot_mapping),
-        _ptr(k_cache), _ptr(v_cache), _stream(stream))
+        _ptr(k_cache), _ptr(v_cache), _ptr(status), _stream(stream))
     if check:
         _check(st, "starkv_compress_store")
     return st
@@ -239,6 +242,14 @@ def starkv_decode_check(workspace, stream=None) -> tuple[int, int]:
     flags = ctypes.c_int32(0)
     st = load_library().starkv_decode_check(_ptr(workspace), _stream(stream), ctypes.byref(flags))
     return st, flags.value
+
+
+def starkv_set_wait_test_hook(wait_limit_us: int, drop_k_stage: int, check: bool = True) -> int:
+    """Test hook: shorten every device wait bound (0 = default) and drop one K-pass stage (-1 = off)."""
+    st = load_library().starkv_set_wait_test_hook(int(wait_limit_us), int(drop_k_stage))
+    if check:
+        _check(st, "starkv_set_wait_test_hook")
+    return st
 
 
 def starkv_status_string(status: int) -> str:

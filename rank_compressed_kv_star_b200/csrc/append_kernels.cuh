@@ -20,6 +20,7 @@
 #include <cuda_fp16.h>
 
 #include "ptx.cuh"
+#include "../../include/starkv.h"
 
 namespace starkv {
 
@@ -30,19 +31,27 @@ struct AppendTarget {
   const int32_t* tables;   // [B][MB]
   const int32_t* positions;
   int MB, NB;
+  int32_t* status;         // optional: flags of skipped targets are OR-ed in
 };
 
-// Physical row (page*16 + slot) of row b's target, or -1 when out of range.
+// Physical row (page*16 + slot) of row b's target, or a negated STARKV_FLAG_*
+// naming why the target is skipped: -STARKV_FLAG_BAD_SEQ_LEN for a position
+// outside the block table, -STARKV_FLAG_BAD_BLOCK_ID for a page outside the pool.
 __device__ __forceinline__ int64_t append_row(const AppendTarget& a, int b) {
   if (a.slots) {
     const int32_t sl = a.slots[b];
-    return (sl < 0 || sl >= a.NB * 16) ? -1 : static_cast<int64_t>(sl);
+    return (sl < 0 || sl >= a.NB * 16) ? -STARKV_FLAG_BAD_BLOCK_ID : static_cast<int64_t>(sl);
   }
   const int32_t pos = a.positions[b];
-  if (pos < 0 || pos / 16 >= a.MB) return -1;
+  if (pos < 0 || pos / 16 >= a.MB) return -STARKV_FLAG_BAD_SEQ_LEN;
   const int32_t phys = a.tables[static_cast<size_t>(b) * a.MB + pos / 16];
-  if (phys < 0 || phys >= a.NB) return -1;
+  if (phys < 0 || phys >= a.NB) return -STARKV_FLAG_BAD_BLOCK_ID;
   return static_cast<int64_t>(phys) * 16 + (pos % 16);
+}
+
+// Records a skipped target (called by one thread per row).
+__device__ __forceinline__ void append_skipped(const AppendTarget& a, int64_t why) {
+  if (a.status) atomicOr(a.status, static_cast<int32_t>(-why));
 }
 
 // ------------------------------------------------------------ V codes (TC)
@@ -165,6 +174,7 @@ append_v_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
     for (int c = 0; c < KS; ++c) acc += cluster.map_shared_rank(part, c)[n * 128 + rrow];
     const int64_t dst = append_row(p.tgt, b);
     if (dst >= 0) p.v_cache[dst * p.R + rg] = __float2half_rn(acc);
+    else if (rg == 0) append_skipped(p.tgt, dst);
   }
   cluster.sync();   // nobody leaves while others still read its partials
   if (warp == 1) {
@@ -219,6 +229,7 @@ __global__ void __launch_bounds__(256) append_k_kernel(AppendKParams p) {
     }
     const int64_t row = append_row(p.tgt, bt0 + b);
     if (row >= 0) p.k_cache[(row * p.H + h) * p.r + i] = __float2half_rn((a0 + a1) + (a2 + a3));
+    else if (h == 0 && i == 0) append_skipped(p.tgt, row);
   }
 }
 

@@ -259,6 +259,7 @@ struct KPassParams {
   int tps;                    // tokens per ring stage (> 16: whole pages of one sequence)
   int stages;
   uint32_t stage_bytes;       // tps*Hkv*r*2
+  int drop_stage;             // test hook: this CTA-local stage is never copied (-1: off)
 };
 
 constexpr int kKConsumers = 256;            // 8 warps of dot products
@@ -344,6 +345,7 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
           for (int32_t t0 = pg * kBlock; t0 < tend; t0 += p.tps, ++k) {
             const int s = k % S;
             if (k >= static_cast<uint32_t>(S) && !mbar_wait(&empty[s], ((k / S) - 1) & 1)) { ok = false; break; }
+            if (static_cast<int>(k) == p.drop_stage) continue;
             const int32_t nt = min(p.tps, tend - t0);
             meta[s] = StageMeta{b, t0, nt, 0};
             const uint32_t bytes = static_cast<uint32_t>(nt) * tok_bytes;
@@ -368,9 +370,12 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
           const int32_t nt = min(n_pg * kBlock, T - t0);
           const int s = k % S;
           if (k >= static_cast<uint32_t>(S) && !mbar_wait(&empty[s], ((k / S) - 1) & 1)) { ok = false; break; }
-          meta[s] = StageMeta{b, t0, nt, 0};
-          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nt) * tok_bytes);
-          for (int i = 0; i < n_pg; ++i) {
+          const bool drop = static_cast<int>(k) == p.drop_stage;
+          if (!drop) {
+            meta[s] = StageMeta{b, t0, nt, 0};
+            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nt) * tok_bytes);
+          }
+          for (int i = 0; i < n_pg && !drop; ++i) {
             int32_t phys = table_row(p.tables, p.row_seq, b, p.MB)[pg + i];
             if (phys < 0 || phys >= p.NB) { set_flag(p.status, STARKV_FLAG_BAD_BLOCK_ID); phys = 0; }
             const int32_t ti = min(kBlock, nt - i * kBlock);
@@ -391,10 +396,13 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
     if (!ok) {
       set_timeout(p.status, kSiteKEmpty);
       abort_flag = 1;
-      // let copies already in flight land before the CTA can exit
-      const uint32_t first = k > static_cast<uint32_t>(S) ? k - S : 0;
-      for (uint32_t kk = first; kk < k; ++kk) mbar_wait(&full[kk % S], (kk / S) & 1);
     }
+    // Copies still in flight land before the CTA can exit (consumers that gave
+    // up do not wait for them): the last uses of the ring slots, i.e. stages
+    // [k - S, k), minus stage k - S when the end marker reused its slot (that
+    // stage was consumed, so it had landed).
+    const uint32_t first = k >= static_cast<uint32_t>(S) ? k - S + (ok ? 1u : 0u) : 0u;
+    for (uint32_t kk = first; kk < k; ++kk) mbar_wait(&full[kk % S], (kk / S) & 1);
     return;
   }
 
@@ -413,7 +421,9 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
 
   for (uint32_t k = 0;; ++k) {
     const int s = k % S;
-    if (!mbar_wait(&full[s], (k / S) & 1) || abort_flag) {
+    // warp-uniform decision: the lanes below shuffle with a full mask
+    const bool landed = mbar_wait(&full[s], (k / S) & 1);
+    if (!__all_sync(0xffffffffu, landed && !abort_flag)) {
       set_timeout(p.status, kSiteKFull);
       break;
     }
@@ -488,14 +498,14 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
 // slots.  A row uses only the G columns of its own KV head; the tensor cores
 // compute all H, which at G >= 2 costs less than the HBM time of the tile.
 //
-// One CTA streams a long ring of pages; the tiles are dealt round-robin to NG
-// consumer groups, each with its own MMA warp, TMEM accumulators and four
-// epilogue warps (one TMEM lane quarter each), so that per-tile latencies of
-// different groups overlap.  An epilogue warp picks its row's G columns,
-// stores them as one contiguous vector (a warp writes whole logit rows) and
-// keeps running maxima; at the end of every segment each warp merges them into
-// the segment's maxima in global memory (float max through integer atomics,
-// initialised to -inf by the absorb kernel).
+// Warp roles: warp 0 (one thread) issues the TMA copies, warp 1 (one thread)
+// the MMAs into a ring of nacc TMEM accumulators, warps 2..5 (one TMEM lane
+// quarter each) drain them.  Several CTAs share an SM so that the per-tile
+// latency chains of different CTAs overlap.  An epilogue warp picks its row's
+// G columns, stores them as one contiguous vector (a warp writes whole logit
+// rows) and keeps running maxima; at the end of every segment each warp merges
+// them into the segment's maxima in global memory (float max through integer
+// atomics, initialised to -inf by the absorb kernel).
 struct KPassTCParams {
   const int32_t* tables;      // [B][MB] (or [n_seqs][MB] with row_seq)
   const int32_t* row_seq;     // [B] sequence of each row, or null
@@ -510,18 +520,17 @@ struct KPassTCParams {
   int kb;                     // 64-code column blocks: ceil(r/64)
   int nmma;                   // UMMA N = max(16, H): TMEM columns per accumulator
   int brows;                  // rows of a query tile: 2H (H >= 16) or 32
-  int ng;                     // consumer groups (1..4)
-  int nacc;                   // accumulators per group
+  int nacc;                   // TMEM accumulators (ring)
   int nbs;                    // query-tile slots (1 or 2)
   int stages;
   uint32_t a_bytes;           // kb * 128 rows * 128 bytes
   uint32_t b_bytes;           // kb * brows * 128 bytes
   uint32_t tmem_cols;
+  int drop_stage;             // test hook: this CTA-local tile is never copied (-1: off)
 };
 
-constexpr int kKTCMaxGroups = 4;
 constexpr int kKTCMaxAcc = 4;
-__host__ __device__ constexpr int ktc_threads(int ng) { return 32 * (1 + 5 * ng); }
+constexpr int kKTCThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 
 // Calls f(b, t0, nt, x0, first, last) for the K-pass tiles of pages [p0, p1)
 // in order: tokens [t0, t0+nt) of sequence b, whose first token lies in global
@@ -545,29 +554,29 @@ __device__ __forceinline__ void for_each_k_tile(const KPassTCParams& p, int64_t 
 }
 
 template <int G, int H>   // query heads per KV head, query heads
-__global__ void __launch_bounds__(ktc_threads(kKTCMaxGroups), 1)
+__global__ void __launch_bounds__(kKTCThreads, 1)
 kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                 KPassTCParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int S = p.stages, NG = p.ng;
+  const int S = p.stages;
   uint8_t* bslot = smem + static_cast<size_t>(S) * p.a_bytes;                    // [nbs] query tiles
   uint64_t* full = reinterpret_cast<uint64_t*>(bslot + p.nbs * static_cast<size_t>(p.b_bytes));
   uint64_t* empty = full + S;
   uint64_t* bfull = empty + S;                     // [2] query tile landed
-  uint64_t* bempty = bfull + 2;                    // [2] query tile no longer read (one commit per group)
-  uint64_t* tfull = bempty + 2;                    // [NG][kKTCMaxAcc] accumulator ready
-  uint64_t* tempty = tfull + kKTCMaxGroups * kKTCMaxAcc;   // [NG][kKTCMaxAcc] accumulator drained
-  uint64_t* mmadone = tempty + kKTCMaxGroups * kKTCMaxAcc; // [NG]
+  uint64_t* bempty = bfull + 2;                    // [2] query tile no longer read
+  uint64_t* tfull = bempty + 2;                    // [kKTCMaxAcc] accumulator ready
+  uint64_t* tempty = tfull + kKTCMaxAcc;           // [kKTCMaxAcc] accumulator drained
+  uint64_t* mmadone = tempty + kKTCMaxAcc;         // every MMA issued has completed
   __shared__ uint32_t taddr_s;
   __shared__ volatile int32_t abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&bfull[a], 1); mbar_init(&bempty[a], NG); }
-    for (int a = 0; a < kKTCMaxGroups * kKTCMaxAcc; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
-    for (int g = 0; g < kKTCMaxGroups; ++g) mbar_init(&mmadone[g], 1);
+    for (int a = 0; a < 2; ++a) { mbar_init(&bfull[a], 1); mbar_init(&bempty[a], 1); }
+    for (int a = 0; a < kKTCMaxAcc; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
+    mbar_init(mmadone, 1);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -604,10 +613,12 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       const int log2tb = tpt < kBlock ? p.log2tpt : 4;
       int si = 0, bi = 0;
       uint32_t su = 0, bu = 0, issued = 0;
+      int32_t bpar[2] = {-1, -1};   // parity of each query slot's latest load (-1: none)
       bool ok = true;
       for_each_k_tile(p, p0, p1, [&](int32_t b, int32_t t0, int32_t nt, int64_t x0, bool first, bool last) {
         if (first) {
           if (bu > 0 && !mbar_wait(&bempty[bi], (bu - 1) & 1)) { ok = false; return false; }
+          bpar[bi] = static_cast<int32_t>(bu & 1);
           mbar_arrive_expect_tx(&bfull[bi], p.b_bytes);
           for (int a = 0; a < p.kb; ++a)
             tma_load_2d(bslot + bi * static_cast<size_t>(p.b_bytes) + static_cast<size_t>(a) * p.brows * 128, &qmap,
@@ -615,8 +626,9 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         }
         if (su > 0 && !mbar_wait(&empty[si], (su - 1) & 1)) { ok = false; return false; }
         uint8_t* st = smem + static_cast<size_t>(si) * p.a_bytes;
-        const int nbox = (nt + tb - 1) >> log2tb;
-        mbar_arrive_expect_tx(&full[si], static_cast<uint32_t>(nbox * p.kb) * box_bytes);
+        const bool drop = static_cast<int>(issued) == p.drop_stage;
+        const int nbox = drop ? 0 : (nt + tb - 1) >> log2tb;
+        if (!drop) mbar_arrive_expect_tx(&full[si], static_cast<uint32_t>(nbox * p.kb) * box_bytes);
         const int32_t* trow = table_row(p.tables, p.row_seq, b, p.MB);
         for (int c = 0; c < nbox; ++c) {
           const int32_t t = t0 + c * tb;
@@ -635,82 +647,78 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       if (!ok) {
         set_timeout(p.status, kSiteKEmpty);
         abort_flag = 1;
-        // let the copies in flight land: the last min(issued, S) stages
-        int i = si;
-        uint32_t u = su;
-        for (uint32_t n = 0; n < issued && n < static_cast<uint32_t>(S); ++n) {
-          if (--i < 0) { i = S - 1; --u; }
-          mbar_wait(&full[i], u & 1);
-        }
       }
+      // copies still in flight land before the CTA can exit (the MMA and
+      // epilogue warps may have given up): the last min(issued, S) stages and
+      // the latest load of each query slot
+      int i = si;
+      uint32_t u = su;
+      for (uint32_t n = 0; n < issued && n < static_cast<uint32_t>(S); ++n) {
+        if (--i < 0) { i = S - 1; --u; }
+        mbar_wait(&full[i], u & 1);
+      }
+      for (int a = 0; a < 2; ++a)
+        if (bpar[a] >= 0) mbar_wait(&bfull[a], static_cast<uint32_t>(bpar[a]));
     }
-  } else if (warp <= NG) {
+  } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    // Group g = warp - 1 issues the MMAs of tiles k = g (mod NG); every group
-    // commits to the query slot's empty barrier at every segment end.
+    // The query slot is released by a commit at every segment end.
     if (lane == 0) {
-      const int g = warp - 1;
       const uint32_t idesc = idesc_f16_f32(128, p.nmma, /*a_mn_major=*/false, /*b_mn_major=*/false);
       const uint32_t b_atom = static_cast<uint32_t>(p.brows) * 8u;    // brows * 128 bytes >> 4
-      const uint32_t tcol0 = taddr + static_cast<uint32_t>(g * p.nacc * p.nmma);
-      int r = 0, si = 0, bi = 0, ai = 0;
+      int si = 0, bi = 0, ai = 0;
       uint32_t su = 0, bu = 0, au = 0;
       bool ok = true;
-      for_each_k_tile(p, p0, p1, [&](int32_t, int32_t, int32_t, int64_t, bool first, bool last) {
-        if (r == g) {
-          uint64_t* tf = &tfull[g * kKTCMaxAcc + ai];
-          uint64_t* te = &tempty[g * kKTCMaxAcc + ai];
-          if (!mbar_wait(&bfull[bi], bu & 1)) { ok = false; return false; }
-          if (au > 0 && !mbar_wait(te, (au - 1) & 1)) { ok = false; return false; }
-          if (!mbar_wait(&full[si], su & 1) || abort_flag) { ok = false; return false; }
-          tc_fence_after();
-          // descriptors of the stage / query slot; a K step adds its byte offset >> 4 to the start field
-          const uint64_t da = smem_desc(smem_u32(smem + static_cast<size_t>(si) * p.a_bytes), 16u, 1024u, kSwizzle128B);
-          const uint64_t db = smem_desc(smem_u32(bslot + bi * static_cast<size_t>(p.b_bytes)), 16u, 1024u, kSwizzle128B);
-          const uint32_t d = tcol0 + static_cast<uint32_t>(ai * p.nmma);
-          for (int ks = 0; ks < p.ksteps; ++ks) {
-            const uint32_t a = ks >> 2, kk = ks & 3;
-            const uint64_t dak = da + (a * 1024u + kk * 2u), dbk = db + (a * b_atom + kk * 2u);
-            umma_f16_ss(d, dak, dbk, idesc, ks > 0 ? 1u : 0u);                    // high parts (rows 0..)
-            umma_f16_ss(d, dak, dbk + static_cast<uint32_t>(H) * 8u, idesc, 1u);  // low parts (rows H..)
-          }
-          umma_commit(&empty[si]);
-          umma_commit(tf);
-          if (++ai == p.nacc) { ai = 0; ++au; }
+      for_each_k_tile(p, p0, p1, [&](int32_t, int32_t, int32_t, int64_t, bool, bool last) {
+        if (!mbar_wait(&bfull[bi], bu & 1)) { ok = false; return false; }
+        if (au > 0 && !mbar_wait(&tempty[ai], (au - 1) & 1)) { ok = false; return false; }
+        if (!mbar_wait(&full[si], su & 1) || abort_flag) { ok = false; return false; }
+        tc_fence_after();
+        // descriptors of the stage / query slot; a K step adds its byte offset >> 4 to the start field
+        const uint64_t da = smem_desc(smem_u32(smem + static_cast<size_t>(si) * p.a_bytes), 16u, 1024u, kSwizzle128B);
+        const uint64_t db = smem_desc(smem_u32(bslot + bi * static_cast<size_t>(p.b_bytes)), 16u, 1024u, kSwizzle128B);
+        const uint32_t d = taddr + static_cast<uint32_t>(ai * p.nmma);
+        for (int ks = 0; ks < p.ksteps; ++ks) {
+          const uint32_t a = ks >> 2, kk = ks & 3;
+          const uint64_t dak = da + (a * 1024u + kk * 2u), dbk = db + (a * b_atom + kk * 2u);
+          umma_f16_ss(d, dak, dbk, idesc, ks > 0 ? 1u : 0u);                    // high parts (rows 0..)
+          umma_f16_ss(d, dak, dbk + static_cast<uint32_t>(H) * 8u, idesc, 1u);  // low parts (rows H..)
         }
+        umma_commit(&empty[si]);
+        umma_commit(&tfull[ai]);
+        if (++ai == p.nacc) { ai = 0; ++au; }
         if (last) {
           umma_commit(&bempty[bi]);
           if (++bi == p.nbs) { bi = 0; ++bu; }
         }
         if (++si == S) { si = 0; ++su; }
-        if (++r == NG) r = 0;
         return true;
       });
       if (!ok) { set_timeout(p.status, kSiteKFull); abort_flag = 1; }
-      umma_commit(&mmadone[g]);
-      mbar_wait(&mmadone[g], 0);
+      umma_commit(mmadone);
+      mbar_wait(mmadone, 0);
     }
   } else {
     // ------------------------------------------------------------ epilogue
     // Row rho of a tile is token rho / Hkv, KV head j = rho % Hkv; the row's
     // logits are accumulator columns [j*G, j*G + G).
-    const int e = warp - 1 - NG;                     // epilogue warp index
-    const int g = e >> 2;                            // its group
     const int q = warp & 3;                          // TMEM lane quarter of this warp
     const int rho = q * 32 + lane;
     const int j = rho & (Hkv - 1);
     const int tl = rho >> p.log2Hkv;
     const uint64_t keep = policy_evict_last();       // logits: read back by the V pass
-    const uint32_t tq = taddr + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(g * p.nacc * p.nmma);
+    const uint32_t tq = taddr + (static_cast<uint32_t>(q * 32) << 16);
     float m[G];
 #pragma unroll
     for (int gg = 0; gg < G; ++gg) m[gg] = -INFINITY;
-    int r = 0, ai = 0;
+    int ai = 0;
     uint32_t au = 0;
     bool ok = true;
     for_each_k_tile(p, p0, p1, [&](int32_t b, int32_t t0, int32_t nt, int64_t, bool, bool last) {
-      if (r == g) {
-        if (!mbar_wait(&tfull[g * kKTCMaxAcc + ai], au & 1) || abort_flag) { ok = false; return false; }
+      {
+        // warp-uniform decision: the TMEM loads below are .sync.aligned
+        const bool ready = mbar_wait(&tfull[ai], au & 1);
+        if (!__all_sync(0xffffffffu, ready && !abort_flag)) { ok = false; return false; }
         tc_fence_after();
         const uint32_t tbase = tq + static_cast<uint32_t>(ai * p.nmma);
         float o[G];
@@ -727,7 +735,7 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[g * kKTCMaxAcc + ai]);
+        if (lane == 0) mbar_arrive(&tempty[ai]);
         if (++ai == p.nacc) { ai = 0; ++au; }
         if (tl < nt) {
           float* lrow = p.logits + (static_cast<size_t>(b) * p.t_pad + t0 + tl) * H + j * G;
@@ -755,7 +763,6 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
 #pragma unroll
         for (int gg = 0; gg < G; ++gg) m[gg] = -INFINITY;
       }
-      if (++r == NG) r = 0;
       return true;
     });
     if (!ok) set_timeout(p.status, kSiteKFull);
@@ -914,9 +921,11 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
       if (!ok) {
         set_timeout(p.status, kSiteVEmpty);
         abort_flag = 1;
-        const uint32_t first = k > static_cast<uint32_t>(S) ? k - S : 0;
-        for (uint32_t kk = first; kk < k; ++kk) mbar_wait(&full[kk % S], (kk / S) & 1);
       }
+      // copies still in flight land before the CTA can exit: the last uses of
+      // the ring slots (stage k - S's slot was reused by the end marker)
+      const uint32_t first = k >= static_cast<uint32_t>(S) ? k - S + (ok ? 1u : 0u) : 0u;
+      for (uint32_t kk = first; kk < k; ++kk) mbar_wait(&full[kk % S], (kk / S) & 1);
     }
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer
@@ -964,7 +973,9 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
     const uint64_t keep = policy_evict_last();   // Z partials: read back by zfinal
     for (uint32_t k = 0;; ++k) {
       const int s = k % S;
-      if (!mbar_wait(&full[s], (k / S) & 1) || abort_flag) {
+      // warp-uniform decisions: the TMEM loads of the epilogue are .sync.aligned
+      const bool landed = mbar_wait(&full[s], (k / S) & 1);
+      if (!__all_sync(0xffffffffu, landed && !abort_flag)) {
         set_timeout(p.status, kSiteVFull);
         abort_flag = 1;
         break;
@@ -1017,7 +1028,8 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
       fence_proxy_async_smem();
       mbar_arrive(&pready[s]);
       if (mt.flags & kLast) {
-        if (!mbar_wait(zdone, seg & 1)) {
+        const bool done = mbar_wait(zdone, seg & 1);
+        if (!__all_sync(0xffffffffu, done)) {
           set_timeout(p.status, kSiteVZdone);
           abort_flag = 1;
           break;

@@ -61,19 +61,23 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 }
 
 // Upper bounds of every wait: about two seconds of wall time and a hard cap on
-// polls, whichever comes first.
+// polls, whichever comes first.  The wall-time bound is a device variable so
+// that a test can shorten it (starkv_set_wait_test_hook); it is read only once
+// a wait has already failed its first poll.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kWaitLimitPolls = 1u << 26;
 constexpr uint32_t kWaitSleepNs = 20000;   // one suspended poll: at most 20 us
+__device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
 
 // Waits for the phase with parity `parity` to complete.  Returns false when
 // the bound ran out (the caller records a timeout and stops).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = *const_cast<const volatile uint64_t*>(&g_wait_limit_ns);
   for (uint32_t i = 0; i < kWaitLimitPolls; ++i) {
     if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
-    if ((i & 7u) == 7u && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if ((i & 7u) == 7u && globaltimer_ns() - t0 > limit) return false;
   }
   return false;
 }

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -89,7 +90,7 @@ struct DecodePlan {
   size_t k_smem;
   // K pass on tensor cores (grouped queries)
   bool ktc;
-  int ktc_log2tpt, ktc_ksteps, ktc_kb, ktc_nmma, ktc_brows, ktc_ng, ktc_nacc, ktc_nbs, ktc_stages;
+  int ktc_log2tpt, ktc_ksteps, ktc_kb, ktc_nmma, ktc_brows, ktc_nacc, ktc_nbs, ktc_stages;
   uint32_t ktc_a_bytes, ktc_b_bytes, ktc_tmem;
   size_t ktc_smem;
   // V pass
@@ -211,10 +212,9 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
 
   // Grouped queries (G >= 2, H >= 8) with at most 16 KV heads: the K pass runs
   // on the tensor cores.  A CTA's single producer thread and per-tile chain are
-  // serial, so the plan spreads the SM over up to STARKV_KTC_CTAS_PER_SM CTAs
-  // of one consumer group each, most CTAs first, that fit by registers (the
-  // instance's count), shared memory (>= 3 ring stages, 4 for a single CTA)
-  // and TMEM (>= 2 accumulators).
+  // serial, so the plan spreads the SM over up to STARKV_KTC_CTAS_PER_SM CTAs,
+  // most CTAs first, that fit by registers (the instance's count), shared
+  // memory (>= 3 ring stages, 4 for a single CTA) and TMEM (>= 2 accumulators).
   p.ktc = false;
   if (p.log2G >= 1 && p.H >= 8 && p.Hkv <= 16) {
     int log2Hkv = 0;
@@ -228,26 +228,24 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
     p.ktc_b_bytes = static_cast<uint32_t>(p.ktc_kb) * p.ktc_brows * 128u;
     const int regs = ktc_num_regs(p.log2G, p.H);
     for (int ctas = STARKV_KTC_CTAS_PER_SM; ctas >= 1 && !p.ktc; --ctas) {
-      for (int ng = 1; ng >= 1 && !p.ktc; --ng) {
-        const int per_warp = (regs * 32 + 255) / 256 * 256;
-        if (regs <= 0 || per_warp * (ktc_threads(ng) / 32) * ctas * 11 > 65536 * 10) continue;  // 10% margin
-        int nacc = 512 / (ctas * ng * p.ktc_nmma);
-        if (nacc > kKTCMaxAcc) nacc = kKTCMaxAcc;
-        if (nacc < 2) continue;
-        for (int nbs = 2; nbs >= 1 && !p.ktc; --nbs) {
-          const uint32_t fixed =
-              1024u + nbs * p.ktc_b_bytes + (4 + 2 * kKTCMaxGroups * kKTCMaxAcc + kKTCMaxGroups) * 8u;
-          const uint32_t budget = static_cast<uint32_t>(STARKV_KTC_SMEM_BYTES) / ctas - (ctas > 1 ? 1024u : 0u);
-          if (budget <= fixed) continue;
-          int stages = static_cast<int>((budget - fixed) / (p.ktc_a_bytes + 16u));
-          if (stages > 12) stages = 12;
-          if (stages < (ctas > 1 ? 3 : 4)) continue;
-          p.ktc = true;
-          p.ktc_ng = ng; p.ktc_nacc = nacc; p.ktc_nbs = nbs; p.ktc_stages = stages;
-          p.ktc_tmem = static_cast<uint32_t>(pow2_ceil(ng * nacc * p.ktc_nmma < 32 ? 32 : ng * nacc * p.ktc_nmma));
-          p.ktc_smem = fixed + static_cast<size_t>(stages) * (p.ktc_a_bytes + 16u);
-          p.k_ctas = sms * ctas;
-        }
+      const int per_warp = (regs * 32 + 255) / 256 * 256;
+      if (regs <= 0 || per_warp * (kKTCThreads / 32) * ctas * 11 > 65536 * 10) continue;  // 10% margin
+      int nacc = 512 / (ctas * p.ktc_nmma);
+      if (nacc > kKTCMaxAcc) nacc = kKTCMaxAcc;
+      if (nacc < 2) continue;
+      for (int nbs = 2; nbs >= 1 && !p.ktc; --nbs) {
+        // query slots, then full/empty per stage, bfull/bempty[2], tfull/tempty per accumulator, mmadone
+        const uint32_t fixed = 1024u + nbs * p.ktc_b_bytes + (4 + 2 * kKTCMaxAcc + 1) * 8u;
+        const uint32_t budget = static_cast<uint32_t>(STARKV_KTC_SMEM_BYTES) / ctas - (ctas > 1 ? 1024u : 0u);
+        if (budget <= fixed) continue;
+        int stages = static_cast<int>((budget - fixed) / (p.ktc_a_bytes + 16u));
+        if (stages > 12) stages = 12;
+        if (stages < (ctas > 1 ? 3 : 4)) continue;
+        p.ktc = true;
+        p.ktc_nacc = nacc; p.ktc_nbs = nbs; p.ktc_stages = stages;
+        p.ktc_tmem = static_cast<uint32_t>(pow2_ceil(nacc * p.ktc_nmma < 32 ? 32 : nacc * p.ktc_nmma));
+        p.ktc_smem = fixed + static_cast<size_t>(stages) * (p.ktc_a_bytes + 16u);
+        p.k_ctas = sms * ctas;
       }
     }
   }
@@ -442,8 +440,7 @@ template <int G, int H>
 cudaError_t launch_kpass_tc_gh(const DecodePlan& pl, const CUtensorMap& kmap, const CUtensorMap& qmap,
                                const KPassTCParams& tp, cudaStream_t s) {
   if (!set_smem(kpass_tc_kernel<G, H>, pl.ktc_smem)) return cudaErrorInvalidValue;
-  return launch(kpass_tc_kernel<G, H>, dim3(pl.k_ctas), dim3(ktc_threads(pl.ktc_ng)), pl.ktc_smem, s, 1, kmap, qmap,
-                tp);
+  return launch(kpass_tc_kernel<G, H>, dim3(pl.k_ctas), dim3(kKTCThreads), pl.ktc_smem, s, 1, kmap, qmap, tp);
 }
 
 template <int H>
@@ -588,20 +585,39 @@ starkv_status compress_store_impl(const starkv_layer_desc* desc, int32_t batch, 
 
 starkv_status starkv_compress_append(const starkv_layer_desc* desc, int32_t batch, const void* k, const void* v,
                                      const void* A_K, const void* A_V, const int32_t* block_tables,
-                                     const int32_t* positions, void* k_cache, void* v_cache, void* stream) {
+                                     const int32_t* positions, void* k_cache, void* v_cache, int32_t* status,
+                                     void* stream) {
   if (batch > 0 && (!block_tables || !positions)) return STARKV_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(status) & 3u) return STARKV_ERR_INVALID_ARG;
   AppendTarget tgt{nullptr, block_tables, positions, desc ? desc->max_blocks_per_seq : 0,
-                   desc ? desc->num_blocks : 0};
+                   desc ? desc->num_blocks : 0, status};
   return compress_store_impl(desc, batch, k, v, A_K, A_V, tgt, k_cache, v_cache, stream);
 }
 
 starkv_status starkv_compress_store(const starkv_layer_desc* desc, int32_t n_tokens, const void* k, const void* v,
                                     const void* A_K, const void* A_V, const int32_t* slot_mapping, void* k_cache,
-                                    void* v_cache, void* stream) {
+                                    void* v_cache, int32_t* status, void* stream) {
   if (n_tokens > 0 && !slot_mapping) return STARKV_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(status) & 3u) return STARKV_ERR_INVALID_ARG;
   AppendTarget tgt{slot_mapping, nullptr, nullptr, desc ? desc->max_blocks_per_seq : 0,
-                   desc ? desc->num_blocks : 0};
+                   desc ? desc->num_blocks : 0, status};
   return compress_store_impl(desc, n_tokens, k, v, A_K, A_V, tgt, k_cache, v_cache, stream);
+}
+
+// Test hook state: the dropped K-pass stage applies to every later decode.
+namespace {
+std::atomic<int> g_drop_k_stage{-1};
+}
+
+starkv_status starkv_set_wait_test_hook(uint32_t wait_limit_us, int32_t drop_k_stage) {
+  if (drop_k_stage < -1) return STARKV_ERR_INVALID_ARG;
+  const uint64_t ns = wait_limit_us ? static_cast<uint64_t>(wait_limit_us) * 1000ull : kWaitLimitNs;
+  if (cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof(ns)) != cudaSuccess) {
+    cudaGetLastError();
+    return STARKV_ERR_CUDA;
+  }
+  g_drop_k_stage.store(drop_k_stage);
+  return STARKV_OK;
 }
 
 size_t starkv_decode_workspace_bytes(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len) {
@@ -621,6 +637,19 @@ starkv_status starkv_decode_workspace_layout(const starkv_layer_desc* desc, int3
 }
 
 namespace {
+// A call with nothing to compute still leaves a clean status word in the
+// workspace it was given, so that starkv_decode_check() after any successful
+// call reads this call's status and not stale bytes.
+starkv_status clear_status(void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace || workspace_bytes < sizeof(int32_t)) return STARKV_OK;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u)) return STARKV_ERR_WORKSPACE;
+  if (cudaMemsetAsync(workspace, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return STARKV_ERR_CUDA;
+  }
+  return STARKV_OK;
+}
+
 starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len, const void* q,
                           const void* B_K, const void* B_V, const void* k_cache, const void* v_cache,
                           const int32_t* block_tables, const int32_t* seq_lens, float scale, void* workspace,
@@ -630,7 +659,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   starkv_status st = make_plan(desc, batch, max_seq_len, &pl);
   if (st != STARKV_OK) return st;
   if (!(std::isfinite(scale) && scale > 0.f)) return STARKV_ERR_INVALID_ARG;
-  if (batch == 0) return STARKV_OK;
+  if (batch == 0) return clear_status(workspace, workspace_bytes, stream);
   if (!q || !B_K || !B_V || !k_cache || !v_cache || !block_tables || !seq_lens || !out)
     return STARKV_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(B_K) || !aligned16(B_V) || !aligned16(k_cache) || !aligned16(v_cache) ||
@@ -701,6 +730,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   kp.B = batch; kp.H = pl.H; kp.log2H = pl.log2H; kp.r = pl.r; kp.MB = pl.MB; kp.NB = pl.NB; kp.t_pad = pl.t_pad;
   kp.Hkv = pl.Hkv; kp.log2G = pl.log2G;
   kp.tps = pl.tps; kp.stages = pl.k_stages; kp.stage_bytes = pl.k_stage_bytes;
+  kp.drop_stage = g_drop_k_stage.load(std::memory_order_relaxed);
   cudaError_t e;
   if (pl.ktc) {
     CUtensorMap kmap, qmap;
@@ -716,8 +746,9 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
     tp.MB = pl.MB; tp.NB = pl.NB; tp.t_pad = pl.t_pad;
     tp.log2tpt = pl.ktc_log2tpt; tp.ksteps = pl.ktc_ksteps; tp.kb = pl.ktc_kb;
     tp.nmma = pl.ktc_nmma; tp.brows = pl.ktc_brows;
-    tp.ng = pl.ktc_ng; tp.nacc = pl.ktc_nacc; tp.nbs = pl.ktc_nbs; tp.stages = pl.ktc_stages;
+    tp.nacc = pl.ktc_nacc; tp.nbs = pl.ktc_nbs; tp.stages = pl.ktc_stages;
     tp.a_bytes = pl.ktc_a_bytes; tp.b_bytes = pl.ktc_b_bytes; tp.tmem_cols = pl.ktc_tmem;
+    tp.drop_stage = kp.drop_stage;
     e = launch_kpass_tc(pl, kmap, qmap, tp, s);
   } else if (pl.L == 1 && pl.CPT == 4) e = launch_kpass<1, 4>(pl, kp, s);
   else if (pl.L == 1 && pl.CPT == 8) e = launch_kpass<1, 8>(pl, kp, s);
@@ -790,7 +821,7 @@ starkv_status starkv_paged_prefill(const starkv_layer_desc* desc, int32_t n_seqs
   if (n_seqs < 0 || n_rows < 0) return STARKV_ERR_INVALID_ARG;
   starkv_status st = make_plan(desc, n_rows, max_seq_len, &pl);
   if (st != STARKV_OK) return st;
-  if (n_rows == 0) return STARKV_OK;
+  if (n_rows == 0) return clear_status(workspace, workspace_bytes, stream);
   if (n_seqs == 0 || !starts || !row_offsets || (reinterpret_cast<uintptr_t>(starts) & 3u) ||
       (reinterpret_cast<uintptr_t>(row_offsets) & 3u))
     return STARKV_ERR_INVALID_ARG;

@@ -89,6 +89,8 @@ def test_decode_argument_errors(lib):
     assert call(3, None) == 1                    # null q
     assert call(3, fake + 2) == 1                # misaligned q
     assert call(12, need - 1) == 3               # workspace too small
+    a = list(args); a[1] = 0; a[11] = None       # empty batch without a workspace: a no-op
+    assert S.starkv_paged_decode(*a, stream=0, check=False) == 0
     assert call(11, None) == 3                   # null workspace
     assert call(11, fake + 128) == 3             # workspace not 256-byte aligned
     assert S.starkv_paged_decode(None, 4, 1024, *args[3:], stream=0, check=False) == 1
@@ -105,6 +107,8 @@ def test_append_argument_errors(lib):
     assert S.starkv_compress_append(*a, stream=0, check=False) == 1
     a = list(args); a[1] = 0
     assert S.starkv_compress_append(*a, stream=0, check=False) == 0   # empty batch: no-op
+    a = list(args)                                                      # misaligned status word
+    assert S.starkv_compress_append(*a, stream=0, check=False, status=fake + 2) == 1
 
 
 def test_workspace_layout_is_consistent(lib):
@@ -162,5 +166,12 @@ def test_prefill_argument_errors(lib):
     assert call(11, fake + 2) == 1               # misaligned row offsets
     assert call(14, need - 1) == 3               # workspace too small for the row arrays
     assert call(3, 64 * 16 + 1) == 1             # length bound above table capacity
-    assert call(2, 0) == 0                       # no rows: no-op
+    a = list(args); a[2] = 0; a[13] = None       # no rows and no workspace: a no-op
+    assert S.starkv_paged_prefill(*a, stream=0, check=False) == 0
+    a = list(args); a[2] = 0; a[13] = fake + 128  # no rows, misaligned workspace: refused
+    assert S.starkv_paged_prefill(*a, stream=0, check=False) == 3
     assert S.starkv_prefill_workspace_bytes(d, -1, 1024) == 0
+
+
+def test_wait_test_hook_rejects_bad_stage(lib):
+    assert S.starkv_set_wait_test_hook(0, -2, check=False) == 1

@@ -74,3 +74,60 @@ def test_grouped_query_cache_costs_kv_heads_only():
     assert O.kv_bytes_per_token([32] * 32, [128] * 32, [4096] * 32) == 4 * O.kv_bytes_per_token(*full)
     half = ([8] * 32, [64] * 32, [512] * 32)
     assert O.kv_bytes_per_token(*half) == S.starkv_kv_bytes_per_token(*half) == 2 * 32 * 1024
+
+
+BLOCKS = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "block_count_table.txt")
+
+
+def _block_table():
+    rows = {}
+    for line in open(BLOCKS):
+        if line.startswith("#") or not line.strip():
+            continue
+        name, blocks = line.split()
+        rows[name] = int(blocks)
+    return rows
+
+
+def test_block_count_table_756_to_2353():
+    """The pages' 756 -> 2353 (3.11x) block counts in one memory budget.
+
+    Plain blocks cost 16 tokens x 512 KiB, so 756 whole blocks pin the budget
+    to [756, 757) x 8 MiB.  2353 whole STAR-KV blocks in that budget pin the
+    compressed bytes per token to (756*8 MiB / (16*2354), 757*8 MiB /
+    (16*2353)], about 164.4-164.7 KiB: 2631-2635 fp16 codes per layer on
+    average (H*r + R), a ratio of 3.11 to the 512 KiB of the full cache, within
+    0.3% of the ~165 KiB per token of the README's boot logs.  A profile that
+    the kernels accept (K ranks multiples of 16, V ranks multiples of 64) falls
+    in that interval and reproduces both counts through the capacity helpers.
+    """
+    t = _block_table()
+    plain_tok = O.kv_bytes_per_token([32] * 32, [128] * 32, [4096] * 32)
+    assert plain_tok == 512 * 1024
+    block = 16 * plain_tok
+    lo, hi = t["plain"] * block, (t["plain"] + 1) * block          # budget interval [lo, hi)
+    assert O.num_blocks(lo, plain_tok) == S.starkv_num_blocks(lo, plain_tok, 16) == t["plain"]
+    assert O.num_blocks(hi - 1, plain_tok) == t["plain"] and O.num_blocks(hi, plain_tok) == t["plain"] + 1
+    # per-token bytes b with floor(budget / (16 b)) == 2353 for some budget in [lo, hi)
+    b_min, b_max = lo / (16 * (t["starkv"] + 1)), (hi - 1) / (16 * t["starkv"])
+    assert 164.4 * 1024 < b_min < b_max < 164.8 * 1024
+    ratio = plain_tok / np.array([b_max, b_min])
+    assert np.all(np.abs(ratio - 3.11) < 0.005)                      # the printed "3.11x"
+    codes_per_layer = np.array([b_min, b_max]) / (2 * 32)
+    assert 2630 < codes_per_layer[0] < codes_per_layer[1] < 2636
+    boot = _boot_log()
+    per_tok_boot = boot["starkv_8192"][0] * GIB / boot["starkv_8192"][1]
+    assert abs(per_tok_boot - b_max) / per_tok_boot < 3e-3
+    # a kernel-compatible profile: K rank 32 per head in every layer, V ranks
+    # 1600 in 28 layers and 1664 in 4 (2 * (32*32*32 + 51456) = 168448 bytes)
+    prof = ([32] * 32, [32] * 32, [1600] * 28 + [1664] * 4)
+    per_tok = O.kv_bytes_per_token(*prof)
+    assert per_tok == S.starkv_kv_bytes_per_token(*prof) == 168448
+    assert b_min < per_tok <= b_max
+    # budgets giving both printed counts: [lo, min(hi, 2354 * 16 * per_tok)), not empty
+    both = (lo, min(hi, (t["starkv"] + 1) * 16 * per_tok))
+    assert both[0] < both[1]
+    for budget in (both[0], both[1] - 1):
+        assert O.num_blocks(budget, plain_tok) == S.starkv_num_blocks(budget, plain_tok, 16) == t["plain"]
+        assert O.num_blocks(budget, per_tok) == S.starkv_num_blocks(budget, per_tok, 16) == t["starkv"]
+    assert round(t["starkv"] / t["plain"], 2) == 3.11

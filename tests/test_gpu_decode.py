@@ -1,12 +1,10 @@
-"""GPU parity of the C-ABI path against the CPU fp64 oracle (B200, sm_100a).
+"""GPU parity of the C-ABI path against the CPU fp64 oracle (B200, sm_100a):
+edge cases, paging invariances, shapes, errors, chunked prefill, graphs.
 
-Tolerances (stated for the fp16-output path with fp32 accumulation): for
-decode outputs, max |gpu - oracle| <= 2e-3 and relative L2 error <= 1e-3 over
-the compared rows.  Appended codes: placement and every untouched byte
-bit-exact; code values within one fp16 ulp of the fp64 code plus the fp32
-dot-product rounding bound (which only matters for codes near zero), and
-within the same max-abs / rel-L2 bounds.  Paging
-invariances (page permutation, identity vs shuffled table) are bit-exact.
+The graded workloads, append bit-exactness and grouped-query parity run
+first, from test_gpu_0_graded.py.  Tolerances are stated in ``gpu_common``:
+decode max |err| <= 2e-3 and relative L2 <= 1e-3; paging invariances (page
+permutation, identity vs shuffled table) are bit-exact.
 """
 import numpy as np
 import pytest
@@ -15,75 +13,15 @@ import torch
 import rank_compressed_kv_star_b200 as S
 from oracle import starkv_oracle as O
 from starkv_inputs import device as D, gen, workloads as W
+from gpu_common import (MAX_ABS, REL_L2, POISON, append_check, assert_close, desc_of, full_check, load,
+                        oracle_rows, rel_l2, run_decode)
 
 pytestmark = pytest.mark.gpu
-
-MAX_ABS, REL_L2 = 2e-3, 1e-3
-
-
-def rel_l2(got, ref):
-    return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
-
-
-def desc_of(L):
-    return S.layer_desc(L["H"], L["d"], L["r"], L["R"], L["nb"], L["tables"].shape[1],
-                        num_kv_heads=L.get("Hkv", 0))
-
-
-def run_decode(L, seq_lens=None, max_seq_len=None, q=None):
-    seq_lens = L["seq_lens"] if seq_lens is None else seq_lens
-    B = seq_lens.shape[0]
-    if max_seq_len is None:
-        max_seq_len = int(seq_lens.max().item()) if B else 0
-    desc = desc_of(L)
-    wsb = S.starkv_decode_workspace_bytes(desc, B, max_seq_len)
-    ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device="cuda")
-    out = torch.full((B, L["H"], L["d"]), float("nan"), dtype=torch.float16, device="cuda")
-    S.starkv_paged_decode(desc, B, max_seq_len, L["q"] if q is None else q, L["B_K"], L["B_V"],
-                          L["k_cache"], L["v_cache"], L["tables"], seq_lens, L["scale"], ws, wsb, out)
-    st, flags = S.starkv_decode_check(ws)
-    assert st == 0, (S.STATUS[st], flags)
-    return out.float().cpu().numpy().astype(np.float64), ws, desc
-
-
-def oracle_rows(wl, layer, L_host_q, A_np, bs, seq_lens, appended=None, q=None):
-    """fp64 oracle for sequences `bs` (codes regenerated on the host)."""
-    A_K, A_V, B_K, B_V = A_np
-    qn = L_host_q if q is None else q
-    out = {}
-    for b in bs:
-        T = int(seq_lens[b])
-        if T == 0:
-            out[b] = np.zeros(qn.shape[1:])
-            continue
-        ctx = int(wl.ctx_lens[b])
-        cK, cV = W.seq_codes(wl, layer, b, min(ctx, T))
-        cK, cV = cK.astype(np.float64), cV.astype(np.float64)
-        if T > ctx:  # the step's appended token (oracle's own fp16 codes)
-            aK, aV = appended
-            cK = np.concatenate([cK, aK[b][None].astype(np.float64)])
-            cV = np.concatenate([cV, aV[b][None].astype(np.float64)])
-        out[b] = O.attend_codes_reordered(qn[b], B_K, B_V, cK, cV, 1.0 / np.sqrt(qn.shape[2]))
-    return out
-
-
-def assert_close(got_rows, ref_rows):
-    g = np.stack([got_rows[b] for b in sorted(ref_rows)])
-    r = np.stack([ref_rows[b] for b in sorted(ref_rows)])
-    err = np.abs(g - r).max()
-    rl = rel_l2(g, r)
-    assert np.isfinite(g).all()
-    assert err <= MAX_ABS, err
-    assert rl <= REL_L2, rl
-    return err, rl
 
 
 @pytest.fixture(scope="module", autouse=True)
 def _built(cuda_ok):
-    from rank_compressed_kv_star_b200 import build
-    build.build()
-    build.build_inputs()
-    S.load_library()
+    load()
 
 
 # ------------------------------------------------------------- generator twin
@@ -107,20 +45,6 @@ def test_device_pools_match_host_pools():
 
 
 # ------------------------------------------------------------------ decode
-
-def _full_check(wl, layer=0):
-    Lh = W.host_layer(wl, layer)
-    Ld = D.device_layer(wl, layer, tables=Lh["tables"], nb=Lh["nb"])
-    got, ws, desc = run_decode(Ld)
-    ref = O.decode_explicit(Lh["q"], Lh["B_K"], Lh["B_V"], Lh["k_cache"], Lh["v_cache"],
-                            Lh["tables"], Lh["seq_lens"], Lh["scale"])
-    err, rl = assert_close({b: got[b] for b in range(wl.batch)}, {b: ref[b] for b in range(wl.batch)})
-    return Lh, Ld, got, ws, desc, err, rl
-
-
-def test_decode_tiny_workload():
-    _full_check(W.workload(1))
-
 
 @pytest.mark.parametrize("gqa", [False, True])
 def test_decode_tiny_intermediates(gqa):
@@ -163,33 +87,33 @@ def test_decode_tiny_intermediates(gqa):
 def test_decode_ragged_multitile():
     sh = W.LayerShape(32, 128, 64, 2048)
     wl = W.custom("ragged", 2024, sh, [1, 15, 16, 17, 300, 0, 1000], append=False)
-    _full_check(wl)
+    full_check(wl)
 
 
 @pytest.mark.parametrize("r,R", [(32, 1024), (96, 3072), (16, 64), (128, 512)])
 def test_decode_rank_variants(r, R):
     sh = W.LayerShape(32, 128, r, R)
     wl = W.custom(f"r{r}", 300 + r, sh, [5, 33, 160, 511], append=False)
-    _full_check(wl)
+    full_check(wl)
 
 
 def test_decode_largest_head_dim_and_k_rank():
     """head_dim 256 and K rank 256 (the largest the kernels take), V rank 4096, ragged lengths."""
     sh = W.LayerShape(16, 256, 256, 4096)
     wl = W.custom("d256", 256, sh, [1, 17, 100], append=False)
-    _full_check(wl)
+    full_check(wl)
 
 
 def test_decode_small_heads_and_dims():
     sh = W.LayerShape(8, 64, 32, 256)
     wl = W.custom("h8", 55, sh, [3, 64, 129], append=False)
-    _full_check(wl)
+    full_check(wl)
 
 
 def test_decode_empty_and_zero_batch():
     sh = W.LayerShape(32, 128, 64, 2048)
     wl = W.custom("empties", 7, sh, [0, 0, 40, 0], append=False)
-    Lh, Ld, got, *_ = _full_check(wl)
+    Lh, Ld, got, *_ = full_check(wl)
     assert np.array_equal(got[[0, 1, 3]], np.zeros_like(got[[0, 1, 3]]))
     # batch 0 and max_seq_len 0 are accepted and launch nothing / zero the output
     z = torch.zeros(0, dtype=torch.int32, device="cuda")
@@ -197,6 +121,44 @@ def test_decode_empty_and_zero_batch():
     zeros4 = torch.zeros(4, dtype=torch.int32, device="cuda")
     out, *_ = run_decode(Ld, seq_lens=zeros4, max_seq_len=0)
     assert np.array_equal(out, np.zeros_like(out))
+    # a prefill call with no rows also leaves a clean status word in a poisoned workspace
+    desc = desc_of(Ld)
+    wsb = S.starkv_prefill_workspace_bytes(desc, 0, 0)
+    ws = torch.full((max(wsb, 256),), POISON, dtype=torch.uint8, device="cuda")
+    S.starkv_paged_prefill(desc, 0, 0, 0, None, None, None, None, None, None, None, None, 0.1, ws, wsb, None)
+    assert S.starkv_decode_check(ws) == (0, 0)
+
+
+def test_append_flags_skipped_targets():
+    """Out-of-range positions and block ids are skipped and reported; the other rows are written."""
+    sh = W.LayerShape(32, 128, 64, 2048)
+    wl = W.custom("skips", 96, sh, [37, 100, 5, 64], append=True)
+    Ld = D.device_layer(wl, 0)
+    desc = desc_of(Ld)
+    before_k, before_v = Ld["k_cache"].clone(), Ld["v_cache"].clone()
+    pos = Ld["ctx_lens"].clone()
+    tables = Ld["tables"].clone()
+    pos[1] = Ld["tables"].shape[1] * 16          # past the block table
+    tables[2, 0] = Ld["nb"] + 3                  # page outside the pool
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    S.starkv_compress_append(desc, wl.batch, Ld["k"], Ld["v"], Ld["A_K"], Ld["A_V"], tables, pos,
+                             Ld["k_cache"], Ld["v_cache"], status=status)
+    st, flags = S.starkv_decode_check(status)
+    assert S.STATUS[st] == "STARKV_ERR_DEVICE_CHECK"
+    assert flags == S.FLAG_BAD_SEQ_LEN | S.FLAG_BAD_BLOCK_ID
+    tab = Ld["tables_np"]
+    written = [int(tab[b][wl.ctx_lens[b] // 16]) * 16 + int(wl.ctx_lens[b] % 16) for b in (0, 3)]
+    kf, vf = Ld["k_cache"].view(-1, 32 * 64), Ld["v_cache"].view(-1, 2048)
+    changed_k = (kf.view(torch.int16) != before_k.view(-1, 32 * 64).view(torch.int16)).any(1)
+    changed_v = (vf.view(torch.int16) != before_v.view(-1, 2048).view(torch.int16)).any(1)
+    assert sorted(torch.nonzero(changed_k).flatten().tolist()) == sorted(written)
+    assert sorted(torch.nonzero(changed_v).flatten().tolist()) == sorted(written)
+    # compress-store: a slot outside the pool is skipped and flagged the same way
+    status.zero_()
+    slots = torch.tensor([written[0], Ld["nb"] * 16 + 7], dtype=torch.int32, device="cuda")
+    S.starkv_compress_store(desc, 2, Ld["k"][:2], Ld["v"][:2], Ld["A_K"], Ld["A_V"], slots, Ld["k_cache"],
+                            Ld["v_cache"], status=status)
+    assert S.starkv_decode_check(status) == (5, S.FLAG_BAD_BLOCK_ID)
 
 
 def test_decode_page_permutation_bit_identical():
@@ -291,61 +253,6 @@ def test_host_side_errors_launch_nothing():
 
 
 # ------------------------------------------------------------------ append
-
-def _append_check(wl, layer=0):
-    Lh = W.host_layer(wl, layer)
-    Ld = D.device_layer(wl, layer, tables=Lh["tables"], nb=Lh["nb"])
-    desc = desc_of(Ld)
-    before_k = Ld["k_cache"].clone()
-    before_v = Ld["v_cache"].clone()
-    S.starkv_compress_append(desc, wl.batch, Ld["k"], Ld["v"], Ld["A_K"], Ld["A_V"], Ld["tables"],
-                             Ld["ctx_lens"], Ld["k_cache"], Ld["v_cache"])
-    torch.cuda.synchronize()
-    cK, cV = O.compress(Lh["k"], Lh["v"], Lh["A_K"], Lh["A_V"])
-    pos = wl.ctx_lens
-    rows = np.array([Lh["tables"][b][pos[b] // 16] * 16 + pos[b] % 16 for b in range(wl.batch)])
-    Hkv = Lh["Hkv"]
-    kf_new = Ld["k_cache"].view(-1, Hkv * Lh["r"]).cpu().numpy()
-    vf_new = Ld["v_cache"].view(-1, Lh["R"]).cpu().numpy()
-    kf_old = before_k.view(-1, Hkv * Lh["r"]).cpu().numpy()
-    vf_old = before_v.view(-1, Lh["R"]).cpu().numpy()
-    mask = np.ones(kf_new.shape[0], bool)
-    mask[rows] = False
-    assert np.array_equal(kf_new[mask].view(np.uint16), kf_old[mask].view(np.uint16))
-    assert np.array_equal(vf_new[mask].view(np.uint16), vf_old[mask].view(np.uint16))
-    # bound: one fp16 ulp of the exact code plus the fp32 dot-product error bound
-    # gamma(K) * sum|terms| (K = length of the contraction), doubled for the
-    # order-free accumulation
-    kk, vv = Lh["k"].astype(np.float64), Lh["v"].astype(np.float64)
-    absK = np.stack([np.abs(kk[:, h, :]) @ np.abs(Lh["A_K"][h].astype(np.float64))
-                     for h in range(Hkv)], axis=1).reshape(wl.batch, -1)
-    absV = np.abs(vv.reshape(wl.batch, -1)) @ np.abs(Lh["A_V"].astype(np.float64))
-    for want, got, absum, K in ((cK.reshape(wl.batch, -1), kf_new[rows], absK, Lh["d"]),
-                                (cV, vf_new[rows], absV, Hkv * Lh["d"])):
-        got = got.astype(np.float64)
-        ulp = np.spacing(np.abs(want).astype(np.float16)).astype(np.float64)
-        gamma = K * 2.0 ** -24 / (1 - K * 2.0 ** -24)
-        bound = ulp + 2 * gamma * absum
-        assert np.all(np.abs(got - want) <= bound), np.max(np.abs(got - want) / bound)
-        assert np.abs(got - want).max() <= MAX_ABS
-        assert rel_l2(got, want) <= REL_L2
-    return Lh, Ld, (cK.astype(np.float16), cV.astype(np.float16))
-
-
-def test_append_tiny():
-    _append_check(W.custom("app", 31, W.LayerShape(4, 64, 16, 64), [37, 100, 0, 15]))
-
-
-@pytest.mark.parametrize("layer", [0, 1, 2])
-def test_append_then_decode_continuous_batching_subset(layer):
-    """Batch-48 mixed-length workload's three rank profiles, first 6 sequences."""
-    full = W.workload(4)
-    wl = W.Workload("cb-subset", full.seed, 6, full.layers, full.ctx_lens[:6])
-    Lh, Ld, appended = _append_check(wl, layer)
-    got, *_ = run_decode(Ld)
-    ref = oracle_rows(wl, layer, Lh["q"], Ld["A_np"], range(6), wl.seq_lens, appended)
-    assert_close({b: got[b] for b in range(6)}, ref)
-
 
 def test_compress_store_prefill_then_decode():
     """A 600-token prompt compressed by slot mapping (three 256-row tiles), then decoded."""
@@ -479,30 +386,6 @@ def test_prefill_rows_of_one_sequence_span_tiles():
 
 # ------------------------------------------------ grouped-query attention
 
-@pytest.mark.parametrize("H,Hkv,d,r,R", [
-    (32, 8, 128, 64, 512),      # Llama-3-8B-like heads, 4 query heads per KV head
-    (32, 16, 128, 64, 1024),    # 2 per KV head
-    (16, 1, 128, 64, 128),      # one KV head (multi-query)
-    (64, 8, 128, 128, 1024),    # 8 per KV head, r = d
-    (8, 2, 64, 16, 128),        # small pages: 8-page K stages
-    (64, 32, 64, 64, 1024),     # 32 KV heads: the CUDA-core K pass with 2 query heads per KV head
-    (4, 2, 64, 16, 64),         # 4 query heads: the CUDA-core K pass
-])
-def test_decode_grouped_query(H, Hkv, d, r, R):
-    sh = W.LayerShape(H, d, r, R, num_kv_heads=Hkv)
-    wl = W.custom(f"gqa{H}x{Hkv}", 600 + H + Hkv, sh, [1, 15, 16, 17, 300, 0, 1000, 129], append=False)
-    _full_check(wl)
-
-
-def test_append_then_decode_grouped_query():
-    sh = W.LayerShape(32, 128, 64, 512, num_kv_heads=8)
-    wl = W.custom("gqa-app", 777, sh, [37, 100, 0, 15, 2000, 4095], append=True)
-    Lh, Ld, appended = _append_check(wl)
-    got, *_ = run_decode(Ld)
-    ref = oracle_rows(wl, 0, Lh["q"], Ld["A_np"], range(wl.batch), wl.seq_lens, appended)
-    assert_close({b: got[b] for b in range(wl.batch)}, ref)
-
-
 def test_decode_grouped_query_equals_repeated_kv_heads_on_gpu():
     """Hkv KV heads against the same inputs repeated to H KV heads: the MHA kernels' output."""
     H, Hkv, d, r, R = 16, 4, 64, 32, 256
@@ -543,37 +426,8 @@ def test_decode_and_append_batch_over_256(kv_heads):
     sh = W.LayerShape(32, 128, 64, 2048 if not kv_heads else 512, num_kv_heads=kv_heads)
     rng = np.random.default_rng(5)
     wl = W.custom("wide", 5150, sh, rng.integers(1, 48, size=300), append=True)
-    Lh, Ld, appended = _append_check(wl)
+    Ld, appended = append_check(wl)
     got, *_ = run_decode(Ld)
     sample = [0, 1, 255, 256, 257, 299]
-    ref = oracle_rows(wl, 0, Lh["q"], Ld["A_np"], sample, wl.seq_lens, appended)
+    ref = oracle_rows(wl, 0, W.activation(wl, 0, W.ACT_Q), Ld["A_np"], sample, wl.seq_lens, appended)
     assert_close({b: got[b] for b in sample}, ref)
-
-
-# ---------------------------------------------------- full-size workloads
-
-@pytest.mark.parametrize("idx,layer,sample", [
-    (2, 0, list(range(16))),            # batch 16, context 2048: every sequence
-    (3, 0, [0, 31, 63]),                # batch 64, context 8192
-    (4, 0, [0, 17, 47]),                # batch 48, mixed lengths, r=32 / R=1024
-    (4, 1, [5, 23]),                    #   r=64 / R=2048
-    (4, 2, [11, 40]),                   #   r=96 / R=3072
-    (5, 0, [0, 7]),                     # 32-layer 7B attention path, first layer
-    (5, 31, [3]),                       #   last layer
-    (6, 0, [0, 21, 63]),                # grouped-query layer, batch 64, context 8192
-])
-def test_decode_full_size_sampled(idx, layer, sample):
-    """Full-size workloads in the benchmark's launch configuration, sampled rows."""
-    wl = W.workload(idx)
-    Ld = D.device_layer(wl, layer)
-    S.starkv_compress_append(desc_of(Ld), wl.batch, Ld["k"], Ld["v"], Ld["A_K"], Ld["A_V"],
-                             Ld["tables"], Ld["ctx_lens"], Ld["k_cache"], Ld["v_cache"])
-    got, *_ = run_decode(Ld)
-    A_K, A_V, B_K, B_V = Ld["A_np"]
-    cK, cV = O.compress(Ld["k"].cpu().numpy(), Ld["v"].cpu().numpy(), A_K, A_V)
-    ref = oracle_rows(wl, layer, Ld["q"].cpu().numpy(), Ld["A_np"], sample, wl.seq_lens,
-                      (cK.astype(np.float16), cV.astype(np.float16)))
-    assert_close({b: got[b] for b in sample}, ref)
-    assert np.isfinite(got).all()
-    del Ld
-    torch.cuda.empty_cache()
