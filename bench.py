@@ -200,25 +200,25 @@ def run_ours(args):
     ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
     outs = [torch.empty((B, L["H"], L["d"]), dtype=torch.float16, device="cuda") for L in layers]
     stream = torch.cuda.current_stream()
-    n_ev = 6
+    n_ev = 5
 
-    def step(evs=None, app_evs=None, li_prof=None):
+    def step(evs=None, app_evs=None):
+        """One step: every layer's append + decode as one starkv_append_decode call, or, when timing
+        the kernels one by one, starkv_compress_append then starkv_paged_decode_profiled."""
         stream = torch.cuda.current_stream()       # the capture stream while a graph is recorded
         for li, L in enumerate(layers):
-            if app_evs is not None:
-                app_evs[li][0].record(stream)
+            if evs is None:
+                S.starkv_append_decode(L["desc"], B, max_len, L["k"], L["v"], L["A_K"], L["A_V"], L["ctx_lens"],
+                                       L["q"], L["B_K"], L["B_V"], L["k_cache"], L["v_cache"], L["tables"],
+                                       L["seq_lens"], L["scale"], ws, wsb, outs[li], stream=stream)
+                continue
+            app_evs[li][0].record(stream)
             S.starkv_compress_append(L["desc"], B, L["k"], L["v"], L["A_K"], L["A_V"], L["tables"],
                                      L["ctx_lens"], L["k_cache"], L["v_cache"], stream=stream)
-            if app_evs is not None:
-                app_evs[li][1].record(stream)
-            if evs is not None:
-                S.starkv_paged_decode_profiled(L["desc"], B, max_len, L["q"], L["B_K"], L["B_V"],
-                                               L["k_cache"], L["v_cache"], L["tables"], L["seq_lens"],
-                                               L["scale"], ws, wsb, outs[li], evs[li], stream=stream)
-            else:
-                S.starkv_paged_decode(L["desc"], B, max_len, L["q"], L["B_K"], L["B_V"], L["k_cache"],
-                                      L["v_cache"], L["tables"], L["seq_lens"], L["scale"], ws, wsb,
-                                      outs[li], stream=stream)
+            app_evs[li][1].record(stream)
+            S.starkv_paged_decode_profiled(L["desc"], B, max_len, L["q"], L["B_K"], L["B_V"],
+                                           L["k_cache"], L["v_cache"], L["tables"], L["seq_lens"],
+                                           L["scale"], ws, wsb, outs[li], evs[li], stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -281,7 +281,7 @@ def run_ours(args):
     for i in range(Kp):
         step(evs[i], app_evs[i])
     torch.cuda.synchronize()
-    names = ["absorb", "kpass", "vpass", "zfinal", "upproj"]
+    names = ["absorb", "kpass", "vpass", "finish"]
     per = {n: 0.0 for n in names}
     per["append"] = 0.0
     for i in range(Kp):
@@ -349,7 +349,8 @@ def run_ours(args):
         "config": {"workload": (f"cfg{args.workload}: {WORKLOAD_NAMES[args.workload]}" if not args.batch
                                 else wl.name), "batch": B,
                    "max_seq_len": max_len, "layers": len(layers),
-                   "step": "compress-append of one token per sequence + paged decode, every layer",
+                   "step": "compress-append of one token per sequence + paged decode, every layer "
+                           "(one starkv_append_decode call per layer)",
                    "l2": "inputs larger than L2 (code pools of %.2f GiB read per step)" % ((k_bytes + v_bytes) / 2**30),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "launch": "one CUDA graph per step" if graph is not None else "stream launches (PDL)"},
@@ -361,11 +362,14 @@ def run_ours(args):
                      "unit": "GB/s", "frac": round(dom_gbs / peak, 4), "traffic": traffic,
                      "algorithmic_bytes_per_launch": dom_bytes // len(layers), "peak_kind": peak_kind},
         "kernels_ms_per_step": {n: round(v, 5) for n, v in per.items()},
-        "kernels_timing": f"CUDA events between kernels over {Kp} further steps (vpass includes the split reduction)",
+        "kernels_timing": f"CUDA events between kernels over {Kp} further steps of separate append and decode "
+                          f"calls (append = the prep kernel with the V and K codes; absorb = the prep kernel "
+                          f"with the query absorption; vpass includes the split reduction of the maxima; "
+                          f"finish = split reduction of Z / L + up-projection)",
         "kernels_GBps": {"kpass": round(kp_gbs, 1), "vpass": round(vp_gbs, 1)},
         "e2e": {"value": round(whole_job_tokens_per_s(world, B, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
-        "gpu_launches": K * len(layers) * 7,   # append: V GEMM + K codes; decode: 5
+        "gpu_launches": K * len(layers) * 4,   # per layer: prep (append + absorb), K pass, V pass, finish
         "clocks": clk,
     }
     if cpu is not None:

@@ -178,6 +178,32 @@ starkv_status starkv_paged_decode(const starkv_layer_desc* desc, int32_t batch, 
                                   void* workspace, size_t workspace_bytes, void* out, void* stream);
 
 /*
+ * starkv_append_decode -- one decode step of a layer: starkv_compress_append of
+ * the new token of every sequence, then starkv_paged_decode over the updated
+ * cache, with the same results as those two calls in that order (the cache
+ * write comes before the attention that reads it, as in a serving engine's
+ * decode step).  The new tokens' K/V codes and the query absorption run in
+ * one launch, which saves two kernel boundaries per step.
+ *
+ *   k, v, A_K, A_V, positions, append_status   as in starkv_compress_append
+ *   q, B_K, B_V, block_tables, seq_lens, scale,
+ *   max_seq_len, workspace, out                 as in starkv_paged_decode
+ *   k_cache, v_cache                            written by the append, then read
+ *
+ * seq_lens are the lengths after the append (normally positions + 1).
+ * Errors as the two calls; nothing is launched when either set of arguments
+ * is invalid.  Cites: README method paragraph (codes written into the
+ * compressed paged cache and read by dedicated decode kernels).
+ */
+starkv_status starkv_append_decode(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len,
+                                   const void* k, const void* v, const void* A_K, const void* A_V,
+                                   const int32_t* positions, const void* q, const void* B_K,
+                                   const void* B_V, void* k_cache, void* v_cache,
+                                   const int32_t* block_tables, const int32_t* seq_lens, float scale,
+                                   void* workspace, size_t workspace_bytes, void* out,
+                                   int32_t* append_status, void* stream);
+
+/*
  * starkv_paged_prefill -- causal attention of prefill chunks over the paged
  * codes (chunked prefill).  The step that precedes decode: a prompt is
  * compressed into the cache chunk by chunk (starkv_compress_store) and each
@@ -215,10 +241,11 @@ starkv_status starkv_paged_prefill(const starkv_layer_desc* desc, int32_t n_seqs
 /*
  * starkv_paged_decode_profiled -- starkv_paged_decode that also records CUDA
  * events on `stream` around its kernels, for per-kernel timing.
- * stage_events: HOST array of 6 cudaEvent_t (as void*; a NULL entry is
+ * stage_events: HOST array of 5 cudaEvent_t (as void*; a NULL entry is
  * skipped) recorded before the query absorption, after it, after the K pass,
- * after the V pass (which includes the split reduction), after the Z
- * finalisation and after the up-projection.  Events between the kernels keep
+ * after the V pass (which includes the split reduction of the maxima) and
+ * after the finish kernel (the split reduction of Z / L and the
+ * up-projection).  Events between the kernels keep
  * them from overlapping their launches, so this variant can be slightly slower
  * than starkv_paged_decode.  The events are not recorded when the call returns
  * an error before launching or when max_seq_len == 0.  Otherwise identical to
@@ -300,9 +327,7 @@ typedef struct {
   size_t logits_off;  /* fp32 [batch][t_pad][H]: base-2 logits s*log2(e) */
   size_t mpart_off;   /* fp32 [k_slots][H]: max of the base-2 logits per segment */
   size_t lpart_off;   /* fp32 [v_slots][H]: per segment, sum of the fp16 weights exp2(s - max) */
-  size_t zpart_off;   /* fp32 [n_rranges][v_slots][H][r_range]: per segment, sum_t w c_V */
-  size_t zhi_off;     /* fp16 [H][batch][R]: Z/L rounded to fp16 */
-  size_t zlo_off;     /* fp16 [H][batch][R]: Z/L minus its fp16 rounding, in fp16 */
+  size_t zpart_off;   /* fp32 [n_rranges][H][v_slots][r_range]: per segment, sum_t w c_V */
   int32_t t_pad;      /* logits row capacity (multiple of 16) */
   int32_t k_ctas;     /* CTAs of the K pass (stream partition) */
   int32_t k_slots;    /* k_ctas + batch */

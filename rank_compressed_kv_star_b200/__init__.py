@@ -25,7 +25,7 @@ FLAG_BAD_BLOCK_ID, FLAG_BAD_SEQ_LEN, FLAG_TIMEOUT = 1, 2, 4
 
 EXPORTED = (
     "starkv_compress_append", "starkv_compress_store", "starkv_decode_workspace_bytes",
-    "starkv_paged_decode",
+    "starkv_paged_decode", "starkv_append_decode",
     "starkv_paged_decode_profiled", "starkv_paged_decode_static",
     "starkv_decode_check", "starkv_decode_workspace_layout", "starkv_status_string",
     "starkv_rank_from_spectrum", "starkv_version", "starkv_kv_bytes_per_token", "starkv_num_blocks",
@@ -51,8 +51,7 @@ class WorkspaceLayout(ctypes.Structure):
                 ("prefix_off", ctypes.c_size_t), ("qt_off", ctypes.c_size_t),
                 ("logits_off", ctypes.c_size_t), ("mpart_off", ctypes.c_size_t),
                 ("lpart_off", ctypes.c_size_t),
-                ("zpart_off", ctypes.c_size_t), ("zhi_off", ctypes.c_size_t),
-                ("zlo_off", ctypes.c_size_t),
+                ("zpart_off", ctypes.c_size_t),
                 ("t_pad", ctypes.c_int32), ("k_ctas", ctypes.c_int32), ("k_slots", ctypes.c_int32),
                 ("v_ctas", ctypes.c_int32), ("v_slots", ctypes.c_int32),
                 ("n_rranges", ctypes.c_int32), ("r_range", ctypes.c_int32),
@@ -89,6 +88,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.starkv_paged_decode.argtypes = [DP, I32, I32, P, P, P, P, P, P, P, ctypes.c_float,
                                         P, SZ, P, P]
     lib.starkv_paged_decode.restype = ctypes.c_int
+    lib.starkv_append_decode.argtypes = [DP, I32, I32, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_float,
+                                         P, SZ, P, P, P]
+    lib.starkv_append_decode.restype = ctypes.c_int
     lib.starkv_paged_decode_profiled.argtypes = [DP, I32, I32, P, P, P, P, P, P, P, ctypes.c_float,
                                                  P, SZ, P, P, ctypes.POINTER(P)]
     lib.starkv_paged_decode_profiled.restype = ctypes.c_int
@@ -192,6 +194,19 @@ def starkv_paged_decode(desc: LayerDesc, batch: int, max_seq_len: int, q, B_K, B
     return st
 
 
+def starkv_append_decode(desc: LayerDesc, batch: int, max_seq_len: int, k, v, A_K, A_V, positions, q, B_K,
+                         B_V, k_cache, v_cache, block_tables, seq_lens, scale: float, workspace,
+                         workspace_bytes: int, out, stream=None, check: bool = True, append_status=None) -> int:
+    """compress-append of the new tokens then paged decode, in one call (one launch fewer per kernel pair)."""
+    st = load_library().starkv_append_decode(
+        _desc_ref(desc), batch, max_seq_len, _ptr(k), _ptr(v), _ptr(A_K), _ptr(A_V), _ptr(positions), _ptr(q),
+        _ptr(B_K), _ptr(B_V), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), float(scale),
+        _ptr(workspace), int(workspace_bytes), _ptr(out), _ptr(append_status), _stream(stream))
+    if check:
+        _check(st, "starkv_append_decode")
+    return st
+
+
 def starkv_prefill_workspace_bytes(desc: LayerDesc, n_rows: int, max_seq_len: int) -> int:
     return int(load_library().starkv_prefill_workspace_bytes(_desc_ref(desc), n_rows, max_seq_len))
 
@@ -212,10 +227,10 @@ def starkv_paged_decode_profiled(desc: LayerDesc, batch: int, max_seq_len: int, 
                                  k_cache, v_cache, block_tables, seq_lens, scale: float, workspace,
                                  workspace_bytes: int, out, stage_events, stream=None,
                                  check: bool = True) -> int:
-    """``stage_events``: six ``torch.cuda.Event`` (or raw cudaEvent_t ints / None)."""
+    """``stage_events``: five ``torch.cuda.Event`` (or raw cudaEvent_t ints / None)."""
     raw = [None if e is None else (e if isinstance(e, int) else e.cuda_event) for e in stage_events]
-    assert len(raw) == 6
-    arr = (ctypes.c_void_p * 6)(*raw)
+    assert len(raw) == 5
+    arr = (ctypes.c_void_p * 5)(*raw)
     st = load_library().starkv_paged_decode_profiled(
         _desc_ref(desc), batch, max_seq_len, _ptr(q), _ptr(B_K), _ptr(B_V), _ptr(k_cache),
         _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), float(scale), _ptr(workspace),

@@ -13,7 +13,11 @@
 // boxes of the batch's v rows (K-major, 128B swizzle), the fp32 accumulator
 // lives in tensor memory.  The K ranges of one R tile form a thread-block
 // cluster and are summed through distributed shared memory in a fixed order,
-// so the result does not depend on scheduling.
+// so the result does not depend on scheduling.  The head-wise K codes are
+// small per-head products on the CUDA cores.
+//
+// Both run as tile bodies of the prep kernel (decode_kernels.cuh), which can
+// put them in one launch with the decode's query absorption.
 #pragma once
 #include <cooperative_groups.h>
 #include <cstdint>
@@ -65,17 +69,19 @@ struct AppendVParams {
   uint32_t tmem_cols;
 };
 
-constexpr int kAppThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kPrepThreads = 256;  // threads of every prep-kernel CTA
 constexpr int kAppKC = 64;         // rows of H*d per pipeline stage
 
-// grid (ceil(R/128), KS, ceil(B/256)), cluster (1, KS, 1)
-__global__ void __launch_bounds__(kAppThreads, 1)
-append_v_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap vmap,
-                AppendVParams p) {
+// One tile of the V-code GEMM: rows [128 mt, 128 mt + 128) of R, the ks-th of
+// KS K ranges (the CTA's rank in its (1, KS, 1) cluster), batch tile bt of
+// 256 sequences.  Warp 0 issues the TMA copies, warp 1 the MMAs, warps 2..5
+// drain the accumulator; all kPrepThreads threads take part in the
+// cluster-wide reduction.  `smem` is the 1024-aligned dynamic shared memory.
+__device__ __forceinline__ void append_v_tile(const CUtensorMap* amap, const CUtensorMap* vmap,
+                                              const AppendVParams& p, int mt, int ks, int KS, int bt,
+                                              uint8_t* smem) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages;
   const uint32_t a_bytes = 2u * kAppKC * 128u;                 // two 64x64 fp16 boxes
   const uint32_t b_bytes = static_cast<uint32_t>(p.npad) * 128u;
@@ -87,10 +93,7 @@ append_v_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
   __shared__ uint32_t taddr_s;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int mt = blockIdx.x;                  // 128-row tile of R
-  const int ks = blockIdx.y;                  // K range (cluster rank)
-  const int KS = gridDim.y;
-  const int b0 = blockIdx.z * 256;
+  const int b0 = bt * 256;
   const int k0 = ks * p.k_per_cta;
   const int k1 = min(p.HD, k0 + p.k_per_cta);
   const int n_stages = k1 > k0 ? (k1 - k0 + kAppKC - 1) / kAppKC : 0;
@@ -113,8 +116,8 @@ append_v_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
   griddep_launch_dependents();
 
   if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&amap);
-    prefetch_tensormap(&vmap);
+    prefetch_tensormap(amap);
+    prefetch_tensormap(vmap);
     const uint64_t pol = policy_evict_last();
     for (int i = 0; i < n_stages; ++i) {
       const int s = i % S;
@@ -122,9 +125,9 @@ append_v_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
       uint8_t* st = smem + static_cast<size_t>(s) * stage_bytes;
       const int kr = k0 + i * kAppKC;
       mbar_arrive_expect_tx(&full[s], stage_bytes);
-      tma_load_2d(st, &amap, mt * 128, kr, &full[s], pol);
-      tma_load_2d(st + kAppKC * 128, &amap, mt * 128 + 64, kr, &full[s], pol);
-      tma_load_2d(st + a_bytes, &vmap, kr, b0, &full[s], pol);
+      tma_load_2d(st, amap, mt * 128, kr, &full[s], pol);
+      tma_load_2d(st + kAppKC * 128, amap, mt * 128 + 64, kr, &full[s], pol);
+      tma_load_2d(st + a_bytes, vmap, kr, b0, &full[s], pol);
     }
   } else if (warp == 1 && lane == 0) {
     const uint32_t idesc = idesc_f16_f32(128, p.npad, /*a_mn_major=*/true, /*b_mn_major=*/false);
@@ -148,7 +151,7 @@ append_v_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
   // every warp observes the accumulator completion (or an empty K range)
   if (!mbar_wait(done, 0)) ok = false;
   tc_fence_after();
-  if (warp >= 2) {
+  if (warp >= 2 && warp < 6) {
     const int q = warp & 3;
     const int row = q * 32 + lane;            // row of the R tile
     for (int c0 = 0; c0 < p.npad; c0 += 16) {
@@ -165,7 +168,7 @@ append_v_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant_
   // rank ks sums rows (batch entries) [ks*npad/KS, (ks+1)*npad/KS) over the cluster, in rank order
   const int per = (p.npad + KS - 1) / KS;
   const int n_lo = ks * per, n_hi = min(p.npad, n_lo + per);
-  for (int x = tid; x < (n_hi - n_lo) * 128; x += kAppThreads) {
+  for (int x = tid; x < (n_hi - n_lo) * 128; x += kPrepThreads) {
     const int n = n_lo + x / 128, rrow = x % 128;
     const int b = b0 + n;
     const int rg = mt * 128 + rrow;
@@ -190,32 +193,29 @@ struct AppendKParams {
   const __half* A_K;       // [H][d][r]
   __half* k_cache;         // [NB][16][H][r]
   int B, H, d, r;
+  int tile;                // sequences per item (<= kAppKB)
 };
 
-// grid (H, ceil(B/kAppKB)), 256 threads; dynamic smem: A_K[h] (d*r halves) +
-// the tile's k[:, h, :] rows (kAppKB*d halves).  Thread = (rank index, lane
-// over the tile's sequences).
-constexpr int kAppKB = 8;
+// One item: head h, sequences [b0, b0 + tile).  A_K[h] and the tile's k[:, h, :]
+// rows are staged in shared memory (`smem`: d*r + kAppKB*d halves); thread =
+// (rank index, lane over the tile's sequences).
+constexpr int kAppKB = 64;
 
-__global__ void __launch_bounds__(256) append_k_kernel(AppendKParams p) {
-  extern __shared__ __align__(16) uint8_t ks_smem[];
-  __half* As = reinterpret_cast<__half*>(ks_smem);              // [d][r]
+__device__ __forceinline__ void append_k_item(const AppendKParams& p, int h, int b0, uint8_t* smem) {
+  __half* As = reinterpret_cast<__half*>(smem);                 // [d][r]
   __half* ksm = As + static_cast<size_t>(p.d) * p.r;            // [kAppKB][d]
-  const int h = blockIdx.x, tid = threadIdx.x;
-  griddep_wait();
-  griddep_launch_dependents();
-  const int bt0 = blockIdx.y * kAppKB;
-  const int nb = min(kAppKB, p.B - bt0);
+  const int tid = threadIdx.x;
+  const int nb = min(p.tile, p.B - b0);
   const uint4* asrc = reinterpret_cast<const uint4*>(p.A_K + static_cast<size_t>(h) * p.d * p.r);
-  for (int x = tid; x < p.d * p.r / 8; x += 256) reinterpret_cast<uint4*>(As)[x] = asrc[x];
-  for (int x = tid; x < nb * p.d / 8; x += 256) {
+  for (int x = tid; x < p.d * p.r / 8; x += kPrepThreads) reinterpret_cast<uint4*>(As)[x] = asrc[x];
+  for (int x = tid; x < nb * p.d / 8; x += kPrepThreads) {
     const int b = x / (p.d / 8), c = x % (p.d / 8);
     reinterpret_cast<uint4*>(ksm)[x] =
-        reinterpret_cast<const uint4*>(p.k + (static_cast<size_t>(bt0 + b) * p.H + h) * p.d)[c];
+        reinterpret_cast<const uint4*>(p.k + (static_cast<size_t>(b0 + b) * p.H + h) * p.d)[c];
   }
   __syncthreads();
   const int i = tid % p.r;
-  const int bpar = 256 / p.r;
+  const int bpar = kPrepThreads / p.r;
   const int bs = tid / p.r;
   if (bs >= bpar) return;
   for (int b = bs; b < nb; b += bpar) {
@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(256) append_k_kernel(AppendKParams p) {
       a2 = fmaf(__half2float(kr[j + 2]), __half2float(As[(j + 2) * p.r + i]), a2);
       a3 = fmaf(__half2float(kr[j + 3]), __half2float(As[(j + 3) * p.r + i]), a3);
     }
-    const int64_t row = append_row(p.tgt, bt0 + b);
+    const int64_t row = append_row(p.tgt, b0 + b);
     if (row >= 0) p.k_cache[(row * p.H + h) * p.r + i] = __float2half_rn((a0 + a1) + (a2 + a3));
     else if (h == 0 && i == 0) append_skipped(p.tgt, row);
   }

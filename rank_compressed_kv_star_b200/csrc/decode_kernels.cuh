@@ -1,6 +1,6 @@
 // Decode kernels of the STAR-KV paged low-rank cache (sm_100a).
 //
-// One decode is five launches on the caller's stream, each launched with
+// One decode is four launches on the caller's stream, each launched with
 // programmatic stream serialisation (see griddep_wait):
 //   1. absorb      q~ = log2(e)*scale * q . B_K[g(h)]^T; page prefix sums; status
 //                  reset; segment maxima set to -inf
@@ -9,9 +9,9 @@
 //                  kpass_tc_kernel on tcgen05 for grouped queries)
 //   3. vpass       split reduction M = max over the sequence's K segments, then
 //                  Z = sum_t w c_V on tcgen05 tensor cores with w = fp16(exp2(s - M)),
-//                  and the normaliser L = sum_t w
-//   4. zfinal      Z / L summed over segments, split into fp16 hi + lo
-//   5. upproj      out_h = (Z_h / L) . B_V[:, g(h)*d:(g(h)+1)*d] on tcgen05 -> fp16
+//                  and the normaliser L = sum_t w, per segment
+//   4. finish      Z / L summed over the segments and split into fp16 hi + lo,
+//                  then out_h = (Z_h / L) . B_V[:, g(h)*d:(g(h)+1)*d] on tcgen05 -> fp16
 // with g(h) = h / (H / Hkv) the KV head of query head h (g(h) = h without
 // grouping).  A chunked prefill adds prefill_rows_kernel in front: each query
 // token of a chunk becomes a decode row of its sequence.
@@ -36,6 +36,7 @@
 #include <cuda_fp16.h>
 
 #include "ptx.cuh"
+#include "append_kernels.cuh"
 #include "../../include/starkv.h"
 
 namespace starkv {
@@ -136,20 +137,20 @@ struct AbsorbParams {
   float coef;             // scale * log2(e)
 };
 
-// grid (H, ceil(B/16)), 256 threads.  CTA (0, 0) also writes the page prefix
-// sums and resets the status word (every later kernel of the decode runs after
-// this one).  Thread = (rank index i, lane over the tile's sequences); its row
-// B_K[h][i][:] is held in registers and the tile's q rows are staged in shared
-// memory.
-constexpr int kAbsBT = 16;
+// One item: query head h, sequences [b0, b0 + tile) (tile <= kAbsBT).  Item 0
+// also writes the page prefix sums and resets the status word (every later
+// kernel of the decode runs after this one); all items share setting the
+// segment-max slots to -inf.  Thread = (rank index i, lane over the tile's
+// sequences); its row B_K[g(h)][i][:] is held in registers and the tile's q
+// rows are staged in shared memory (`smem`, tile*D halves).
+constexpr int kAbsBT = 64;
 
 template <int D>
-__global__ void __launch_bounds__(256) absorb_kernel(AbsorbParams p) {
-  const int h = blockIdx.x;
+__device__ __forceinline__ void absorb_item(const AbsorbParams& p, int item, int n_items, int tile, uint8_t* smem) {
+  const int h = item % p.H;
+  const int bt0 = (item / p.H) * tile;
   const int tid = threadIdx.x;
-  griddep_wait();
-  griddep_launch_dependents();
-  if (h == 0 && blockIdx.y == 0) {
+  if (item == 0) {
     __shared__ int32_t part[256];
     __shared__ int32_t bad;
     if (tid == 0) bad = 0;
@@ -194,20 +195,18 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbParams p) {
     }
   }
   if (p.mpart_init) {
-    const int nthr = gridDim.x * gridDim.y * 256;
-    for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * 256 + tid; i < p.n_mpart; i += nthr)
-      p.mpart_init[i] = -INFINITY;
+    const int nthr = n_items * 256;
+    for (int i = item * 256 + tid; i < p.n_mpart; i += nthr) p.mpart_init[i] = -INFINITY;
   }
-  __shared__ __align__(16) __half qs[kAbsBT * D];
-  const int bt0 = blockIdx.y * kAbsBT;
-  const int nb = min(kAbsBT, p.B - bt0);
+  __half* qs = reinterpret_cast<__half*>(smem);    // [tile][D]
+  const int nb = min(tile, p.B - bt0);
   for (int x = tid; x < nb * (D / 8); x += 256) {
     const int bb = x / (D / 8), c = x % (D / 8);
     reinterpret_cast<uint4*>(qs)[x] =
         reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(bt0 + bb) * p.H + h) * D)[c];
   }
   __syncthreads();
-  // q~[b,h,i] = coef * sum_j q[b,h,j] * B_K[h][i][j]
+  // q~[b,h,i] = coef * sum_j q[b,h,j] * B_K[g(h)][i][j]
   const int i = tid % p.r;
   const int bpar = 256 / p.r;
   const int bs = tid / p.r;
@@ -241,6 +240,48 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbParams p) {
       row[static_cast<size_t>(p.H) * p.r] = __float2half_rn(v - __half2float(hi));
     }
   }
+}
+
+// ======================================================================== prep
+// One launch for the small per-token work of a step, by CTA role along x
+// (clusters of KS CTAs along y):
+//   x <  v_cols            tiles of the V-code GEMM of the new tokens (append)
+//   x <  v_cols + k_cols   K-code items (head, batch tile) of the new tokens
+//   the rest               query-absorption items (head, batch tile) of a decode
+// A call runs any subset: the compress-and-append alone (V + K codes), the
+// decode's absorption alone, or both at once for a whole step.  The roles read
+// and write disjoint data, so they need no order among themselves.
+struct PrepParams {
+  AppendVParams v;
+  AppendKParams k;
+  AbsorbParams a;
+  int v_mt, v_cols;        // 128-row tiles of R; grid columns of V-code tiles (v_mt * batch tiles)
+  int k_items, k_cols;     // K-code items (heads x batch tiles) and their grid columns
+  int a_items, a_tile;     // absorption items (heads x batch tiles of a_tile sequences)
+};
+
+template <int D>
+__global__ void __launch_bounds__(kPrepThreads, 1)
+prep_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap vmap, PrepParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int KS = gridDim.y;
+  int x = blockIdx.x;
+  if (x < p.v_cols) {
+    append_v_tile(&amap, &vmap, p.v, x % p.v_mt, blockIdx.y, KS, x / p.v_mt, smem);
+    return;
+  }
+  x -= p.v_cols;
+  griddep_wait();
+  griddep_launch_dependents();
+  if (x < p.k_cols) {
+    const int it = x * KS + blockIdx.y;
+    if (it < p.k_items) append_k_item(p.k, it % p.k.H, (it / p.k.H) * p.k.tile, smem);
+    return;
+  }
+  x -= p.k_cols;
+  const int it = x * KS + blockIdx.y;
+  if (it < p.a_items) absorb_item<D>(p.a, it, p.a_items, p.a_tile, smem);
 }
 
 // ======================================================================= kpass
@@ -788,7 +829,7 @@ struct VPassParams {
   const int32_t* prefix;
   const float* logits;    // [B][t_pad][H]
   const float* mpart;     // [k_slots][H]: K-pass per-segment max of the logits
-  float* zpart;           // [n_rr][v_slots][H][r_range]: sum_t w c_V per segment
+  float* zpart;           // [n_rr][H][v_slots][r_range]: sum_t w c_V per segment
   float* lpart;           // [v_slots][H]: sum_t w per segment (written by R range 0)
   int32_t* status;
   int B, H, npad, MB, NB, R, t_pad, r_range, n_rr, v_slots, stages;
@@ -970,7 +1011,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
     const int t_step = 128 / p.npad;
     float lsum = 0.f;
     uint32_t seg = 0, pphase = 0;
-    const uint64_t keep = policy_evict_last();   // Z partials: read back by zfinal
+    const uint64_t keep = policy_evict_last();   // Z partials: read back by the finish kernel
     for (uint32_t k = 0;; ++k) {
       const int s = k % S;
       // warp-uniform decisions: the TMEM loads of the epilogue are .sync.aligned
@@ -1036,7 +1077,8 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
         }
         tc_fence_after();
         const size_t slot = static_cast<size_t>(mt.b) + cta;
-        float* zb = p.zpart + (static_cast<size_t>(rr) * p.v_slots + slot) * p.H * p.r_range;
+        // partial rows [R range][head][slot][r_range]: head h0+hh's row of this slot
+        float* zb = p.zpart + ((static_cast<size_t>(rr) * p.H) * p.v_slots + slot) * p.r_range;
         for (int m = 0; m < p.n_mtiles; ++m) {
           uint32_t v[32];
           const uint32_t ta = taddr + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(m * p.npad);
@@ -1048,7 +1090,8 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
             if (j < p.r_range && rr * p.r_range + j < p.R) {
               const int hn = min(32, p.H - h0);
               for (int hh = 0; hh < hn; ++hh)
-                st_global_hint(zb + static_cast<size_t>(h0 + hh) * p.r_range + j, __uint_as_float(v[hh]), keep);
+                st_global_hint(zb + static_cast<size_t>(h0 + hh) * p.v_slots * p.r_range + j, __uint_as_float(v[hh]),
+                               keep);
             }
           }
         }
@@ -1074,133 +1117,75 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
   }
 }
 
-// ==================================================================== zfinal
-// Z / L per (sequence, head): the V-pass partials of the sequence's segments
-// summed in segment order, scaled by 1/L (L = the summed fp16 weights), and
-// split into fp16 hi + lo halves for the up-projection's B operand (hi + lo
-// keeps about 22 bits of the fp32 value).  Z / L is a convex combination of
-// fp16 codes, so both halves are in range.  Layout [H][B][R] (head-major) so
-// that one head's rows of a batch tile are contiguous.
-struct ZFinalParams {
-  const float* zpart;     // [n_rr][v_slots][H][r_range]
-  const float* lpart;     // [v_slots][H]
-  const int32_t* prefix;
-  __half* zhi;            // [H][B][R]
-  __half* zlo;            // [H][B][R]
-  int B, H, R, r_range, v_slots, v_grid;
-};
-
-// grid (ceil(R/2048), B*H), 256 threads x 8 consecutive rows of R.  Thread 0
-// looks up the sequence's segments and 1/L once for the CTA.
-__global__ void __launch_bounds__(256) zfinal_kernel(ZFinalParams p) {
-  griddep_wait();
-  __shared__ int32_t s_i0, s_i1;
-  __shared__ float s_il;
-  const int bh = blockIdx.y;
-  const int b = bh / p.H, h = bh % p.H;
-  if (threadIdx.x == 0) {
-    const int32_t f0 = p.prefix[b], f1 = p.prefix[b + 1];
-    int32_t i0 = 0, i1 = -1;
-    float il = 0.f;
-    if (f1 > f0) {
-      Partition pt;
-      pt.P = p.prefix[p.B];
-      pt.G = static_cast<int32_t>(pt.P < p.v_grid ? pt.P : p.v_grid);
-      i0 = part_owner(f0, pt);
-      i1 = part_owner(f1 - 1, pt);
-      float Ls = 0.f;
-      for (int32_t i = i0; i <= i1; ++i) Ls += p.lpart[static_cast<size_t>(b + i) * p.H + h];
-      il = 1.f / Ls;
-    }
-    s_i0 = i0;
-    s_i1 = i1;
-    s_il = il;
-  }
-  __syncthreads();
-  const int j = (blockIdx.x * 256 + threadIdx.x) * 8;
-  if (j >= p.R) return;
-  const int32_t i0 = s_i0, i1 = s_i1;
-  float z[8];
-#pragma unroll
-  for (int u = 0; u < 8; ++u) z[u] = 0.f;
-  if (i1 >= i0) {
-    const int rrg = j / p.r_range, jj = j % p.r_range;
-    const size_t stride = static_cast<size_t>(p.H) * p.r_range;
-    const float* src = p.zpart + ((static_cast<size_t>(rrg) * p.v_slots + b + i0) * p.H + h) * p.r_range + jj;
-    // all loads of up to four segments are issued before they are summed in segment order
-    for (int32_t i = i0; i <= i1; i += 4) {
-      float4 v[4][2];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float4* q = reinterpret_cast<const float4*>(src + static_cast<size_t>(i - i0 + u) * stride);
-        const bool in = i + u <= i1;
-        v[u][0] = in ? q[0] : make_float4(0.f, 0.f, 0.f, 0.f);
-        v[u][1] = in ? q[1] : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (i + u <= i1) {
-          z[0] += v[u][0].x; z[1] += v[u][0].y; z[2] += v[u][0].z; z[3] += v[u][0].w;
-          z[4] += v[u][1].x; z[5] += v[u][1].y; z[6] += v[u][1].z; z[7] += v[u][1].w;
-        }
-      }
-    }
-    const float il = s_il;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) z[u] *= il;
-  }
-  uint4 hv, lv;
-  uint32_t* hw = reinterpret_cast<uint32_t*>(&hv);
-  uint32_t* lw = reinterpret_cast<uint32_t*>(&lv);
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const __half2 hh = __floats2half2_rn(z[2 * u], z[2 * u + 1]);
-    const float2 g = __half22float2(hh);
-    const __half2 ll = __floats2half2_rn(z[2 * u] - g.x, z[2 * u + 1] - g.y);
-    hw[u] = *reinterpret_cast<const uint32_t*>(&hh);
-    lw[u] = *reinterpret_cast<const uint32_t*>(&ll);
-  }
-  const size_t dst = (static_cast<size_t>(h) * p.B + b) * p.R + j;
-  *reinterpret_cast<uint4*>(p.zhi + dst) = hv;
-  *reinterpret_cast<uint4*>(p.zlo + dst) = lv;
-}
-
-// ====================================================================== upproj
+// ==================================================================== finish
 // out_h^T (d x B) = B_V^h^T (d x R) . (Z_h / L)^T (R x B) on tcgen05 tensor
-// cores, two MMAs per K step (hi and lo halves of Z / L).  A = B_V^h^T from
-// 64x64 TMA boxes of B_V (MN-major, 128B swizzle); B from 64-column boxes of
-// the head's Z rows (K-major, 128B swizzle).  R is split over a cluster whose
-// partial sums are added through distributed shared memory in rank order.
-struct UpProjParams {
+// cores, with Z / L formed on the fly from the V pass's per-segment partials
+// (the split reduction of Z and the up-projection in one kernel).
+//
+// Partials are laid out [R range][head][slot][r_range] (fp32), so for one
+// head and one R range the slots of consecutive sequences are consecutive
+// rows: sequence b owns slots b + i0 .. b + i1 (the V-pass CTAs i0..i1 that
+// overlapped it), and those runs are ordered and disjoint.  A batch tile of
+// sequences therefore needs one contiguous block of partial rows, brought in
+// per stage (64 rows of R) by 2-D TMA boxes of 32 partial rows x 64 values.
+// Four converter warps sum each sequence's rows in segment order, scale by
+// 1/L (L = the summed fp16 weights of all its segments) and split the result
+// into fp16 hi + lo halves (about 22 bits of the fp32 value), written straight
+// into the MMA's B operand (K-major, 128-byte swizzle).  Z / L is a convex
+// combination of fp16 codes, so both halves are in range.  A = B_V^h^T from
+// 64x64 TMA boxes of B_V (MN-major, 128B swizzle); two MMAs per K step (hi
+// and lo).  R is split over a cluster whose partial sums are added through
+// distributed shared memory in rank order.
+struct FinishParams {
   __half* out;            // [B][H][d]
+  const float* lpart;     // [v_slots][H]
+  const int32_t* prefix;  // [B+1]
   int B, H, d, R;
   int log2G;              // query head h reads B_V columns of KV head h >> log2G
+  int r_range, v_slots, v_grid;
   int n_mt;               // 128-row tiles of d
+  int bt_rows;            // sequences per batch tile
   int k_per_cta;          // rows of R per CTA (multiple of 64)
   int npad;               // UMMA N (batch tile padded to 16)
   int stages;
+  int zrows;              // partial rows reserved per stage (multiple of kFinZBox, >= any tile's need)
+  uint32_t stage_bytes;
   uint32_t tmem_cols;
 };
 
-constexpr int kUpThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
-constexpr int kUpKC = 64;        // rows of R per stage
+constexpr int kFinThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 convert, then epilogue
+constexpr int kFinKC = 64;        // rows of R per stage
+constexpr int kFinZBox = 32;      // partial rows per TMA box
+constexpr int kFinMaxRows = 256;  // sequences per batch tile at most
+
+// First slot (a lower bound) and slot count of the partials of sequences
+// [b0, b1) for a V-pass partition pt (P > 0).
+__device__ __forceinline__ void tile_slots(const int32_t* prefix, const Partition& pt, int b0, int b1,
+                                           int32_t* lo, int32_t* n) {
+  const int64_t f0 = min(static_cast<int64_t>(prefix[b0]), pt.P - 1);
+  const int64_t f1 = min(max(static_cast<int64_t>(prefix[b1]) - 1, int64_t{0}), pt.P - 1);
+  *lo = b0 + part_owner(f0, pt);
+  *n = (b1 - 1 + part_owner(f1, pt)) - *lo + 1;
+}
 
 // grid (H * n_mt * n_bt, KS), cluster (1, KS, 1)
-__global__ void __launch_bounds__(kUpThreads, 1)
-upproj_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__ CUtensorMap zhimap,
-              const __grid_constant__ CUtensorMap zlomap, UpProjParams p) {
+__global__ void __launch_bounds__(kFinThreads, 1)
+finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__ CUtensorMap zmap, FinishParams p) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages;
-  const uint32_t a_bytes = 2u * kUpKC * 128u;                 // two 64x64 boxes of B_V
-  const uint32_t z_bytes = static_cast<uint32_t>(p.npad) * 128u;  // one 64-column box of Z rows
-  const uint32_t stage_bytes = a_bytes + 2 * z_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * stage_bytes);
-  uint64_t* empty = full + S;
+  const uint32_t a_bytes = 2u * kFinKC * 128u;                      // two 64x64 boxes of B_V
+  const uint32_t half_bytes = static_cast<uint32_t>(p.npad) * 128u;  // one hi or lo operand tile
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * p.stage_bytes);
+  uint64_t* conv = full + S;
+  uint64_t* empty = conv + S;
   uint64_t* done = empty + S;
-  float* part = reinterpret_cast<float*>(smem);              // [npad][128], reuses the ring
+  int32_t* s_row = reinterpret_cast<int32_t*>(done + 1);            // [kFinMaxRows] first partial row
+  int32_t* s_nseg = s_row + kFinMaxRows;                            // [kFinMaxRows] segments
+  float* s_il = reinterpret_cast<float*>(s_nseg + kFinMaxRows);     // [kFinMaxRows] 1/L
+  float* part = reinterpret_cast<float*>(smem);                     // [npad][128], reuses the ring
   __shared__ uint32_t taddr_s;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1209,13 +1194,14 @@ upproj_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
   const int mt = xi % p.n_mt;
   const int bt = xi / p.n_mt;
   const int ks = blockIdx.y, KS = gridDim.y;
-  const int b0 = bt * 256;
+  const int b0 = bt * p.bt_rows;
+  const int nb = min(p.bt_rows, p.B - b0);
   const int k0 = ks * p.k_per_cta;
   const int k1 = min(p.R, k0 + p.k_per_cta);
-  const int n_stages = k1 > k0 ? (k1 - k0 + kUpKC - 1) / kUpKC : 0;
+  const int n_stages = k1 > k0 ? (k1 - k0 + kFinKC - 1) / kFinKC : 0;
 
   if (tid == 0) {
-    for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&conv[s], 128); mbar_init(&empty[s], 1); }
     mbar_init(done, 1);
     fence_mbar_init();
   }
@@ -1231,42 +1217,127 @@ upproj_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
   griddep_wait();
   griddep_launch_dependents();
 
-  if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&bvmap);
-    prefetch_tensormap(&zhimap);
-    prefetch_tensormap(&zlomap);
-    const uint64_t pol = policy_evict_first();
-    const int col = (h >> p.log2G) * p.d + mt * 128;
-    const int zrow = h * p.B + b0;
-    for (int i = 0; i < n_stages; ++i) {
-      const int s = i % S;
-      if (i >= S && !mbar_wait(&empty[s], ((i / S) - 1) & 1)) { ok = false; break; }
-      uint8_t* st = smem + static_cast<size_t>(s) * stage_bytes;
-      const int kr = k0 + i * kUpKC;
-      mbar_arrive_expect_tx(&full[s], stage_bytes);
-      tma_load_2d(st, &bvmap, col, kr, &full[s], pol);
-      tma_load_2d(st + kUpKC * 128, &bvmap, col + 64, kr, &full[s], pol);
-      tma_load_2d(st + a_bytes, &zhimap, kr, zrow, &full[s], pol);
-      tma_load_2d(st + a_bytes + z_bytes, &zlomap, kr, zrow, &full[s], pol);
-    }
-  } else if (warp == 1 && lane == 0) {
-    const uint32_t idesc = idesc_f16_f32(128, p.npad, /*a_mn_major=*/true, /*b_mn_major=*/false);
-    for (int i = 0; i < n_stages; ++i) {
-      const int s = i % S;
-      if (!mbar_wait(&full[s], (i / S) & 1)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
-      const uint32_t shi = sa + a_bytes, slo = shi + z_bytes;
-#pragma unroll
-      for (int kk = 0; kk < kUpKC / 16; ++kk) {
-        const uint64_t adesc = smem_desc(sa + kk * 16u * 128u, kUpKC * 128u, 1024u, kSwizzle128B);
-        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-        umma_f16_ss(taddr, adesc, smem_desc(shi + kk * 32u, 16u, 1024u, kSwizzle128B), idesc, acc);
-        umma_f16_ss(taddr, adesc, smem_desc(slo + kk * 32u, 16u, 1024u, kSwizzle128B), idesc, 1u);
+  Partition pt;
+  pt.P = p.prefix[p.B];
+  pt.G = static_cast<int32_t>(pt.P < p.v_grid ? pt.P : p.v_grid);
+  int32_t slot_lo = 0, n_slots = 0;
+  if (pt.P > 0) tile_slots(p.prefix, pt, b0, b0 + nb, &slot_lo, &n_slots);
+  const int n_box = n_slots > 0 ? (min(n_slots, p.zrows) + kFinZBox - 1) / kFinZBox : 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      prefetch_tensormap(&bvmap);
+      prefetch_tensormap(&zmap);
+      const uint64_t pol = policy_evict_first();
+      const int col = (h >> p.log2G) * p.d + mt * 128;
+      for (int i = 0; i < n_stages; ++i) {
+        const int s = i % S;
+        if (i >= S && !mbar_wait(&empty[s], ((i / S) - 1) & 1)) { ok = false; break; }
+        uint8_t* st = smem + static_cast<size_t>(s) * p.stage_bytes;
+        const int kr = k0 + i * kFinKC;
+        const int rr = kr / p.r_range, jj = kr - rr * p.r_range;
+        mbar_arrive_expect_tx(&full[s], a_bytes + static_cast<uint32_t>(n_box) * kFinZBox * 256u);
+        tma_load_2d(st, &bvmap, col, kr, &full[s], pol);
+        tma_load_2d(st + kFinKC * 128, &bvmap, col + 64, kr, &full[s], pol);
+        const int zrow = (rr * p.H + h) * p.v_slots + slot_lo;
+        uint8_t* zdst = st + a_bytes + 2u * half_bytes;
+        for (int z = 0; z < n_box; ++z)
+          tma_load_2d(zdst + static_cast<size_t>(z) * kFinZBox * 256, &zmap, jj, zrow + z * kFinZBox, &full[s], pol);
       }
-      umma_commit(&empty[s]);
     }
-    umma_commit(done);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ----------------------------------------------------------------- MMA
+      const uint32_t idesc = idesc_f16_f32(128, p.npad, /*a_mn_major=*/true, /*b_mn_major=*/false);
+      for (int i = 0; i < n_stages; ++i) {
+        const int s = i % S;
+        if (!mbar_wait(&conv[s], (i / S) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * p.stage_bytes);
+        const uint32_t shi = sa + a_bytes, slo = shi + half_bytes;
+#pragma unroll
+        for (int kk = 0; kk < kFinKC / 16; ++kk) {
+          const uint64_t adesc = smem_desc(sa + kk * 16u * 128u, kFinKC * 128u, 1024u, kSwizzle128B);
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          umma_f16_ss(taddr, adesc, smem_desc(shi + kk * 32u, 16u, 1024u, kSwizzle128B), idesc, acc);
+          umma_f16_ss(taddr, adesc, smem_desc(slo + kk * 32u, 16u, 1024u, kSwizzle128B), idesc, 1u);
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(done);
+    }
+  } else {
+    // ------------------------------------------------------------ converters
+    const int et = tid - 64;                 // 0..127
+    // each sequence's partial rows (relative to the tile's first slot) and 1/L;
+    // L sums the per-segment normalisers in segment order
+    for (int bl = et; bl < p.npad; bl += 128) {
+      int32_t row = 0, nseg = 0;
+      float il = 0.f;
+      if (bl < nb && pt.P > 0) {
+        const int b = b0 + bl;
+        const int32_t f0 = p.prefix[b], f1 = p.prefix[b + 1];
+        if (f1 > f0) {
+          const int32_t i0 = part_owner(f0, pt), i1 = part_owner(f1 - 1, pt);
+          float Ls = 0.f;
+          for (int32_t i = i0; i <= i1; ++i) Ls += p.lpart[static_cast<size_t>(b + i) * p.H + h];
+          il = 1.f / Ls;
+          row = b + i0 - slot_lo;
+          nseg = i1 - i0 + 1;
+          if (row < 0 || row + nseg > n_box * kFinZBox) nseg = 0;   // cannot happen: the plan bounds the tile
+        }
+      }
+      s_row[bl] = row;
+      s_nseg[bl] = nseg;
+      s_il[bl] = il;
+    }
+    named_bar_sync(1, 128);
+    for (int i = 0; i < n_stages; ++i) {
+      const int s = i % S;
+      const bool landed = mbar_wait(&full[s], (i / S) & 1);
+      if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }
+      uint8_t* st = smem + static_cast<size_t>(s) * p.stage_bytes;
+      uint8_t* hi_t = st + a_bytes;
+      const uint8_t* zt = st + a_bytes + 2u * half_bytes;
+      // item = (sequence row bl of the tile, 8-value chunk c of the stage's 64 rows of R)
+      for (int item = et; item < p.npad * 8; item += 128) {
+        const int bl = item >> 3, c = item & 7;
+        float z[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) z[u] = 0.f;
+        const int nseg = s_nseg[bl];
+        if (nseg > 0) {
+          const float* src = reinterpret_cast<const float*>(zt + static_cast<size_t>(s_row[bl]) * 256) + c * 8;
+          for (int g = 0; g < nseg; ++g) {
+            const float4 v0 = reinterpret_cast<const float4*>(src + g * 64)[0];
+            const float4 v1 = reinterpret_cast<const float4*>(src + g * 64)[1];
+            z[0] += v0.x; z[1] += v0.y; z[2] += v0.z; z[3] += v0.w;
+            z[4] += v1.x; z[5] += v1.y; z[6] += v1.z; z[7] += v1.w;
+          }
+          const float il = s_il[bl];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) z[u] *= il;
+        }
+        uint4 hv, lv;
+        uint32_t* hw = reinterpret_cast<uint32_t*>(&hv);
+        uint32_t* lw = reinterpret_cast<uint32_t*>(&lv);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const __half2 hh = __floats2half2_rn(z[2 * u], z[2 * u + 1]);
+          const float2 g = __half22float2(hh);
+          const __half2 ll = __floats2half2_rn(z[2 * u] - g.x, z[2 * u + 1] - g.y);
+          hw[u] = *reinterpret_cast<const uint32_t*>(&hh);
+          lw[u] = *reinterpret_cast<const uint32_t*>(&ll);
+        }
+        // K-major operand row bl, 16-byte chunk c at its 128B-swizzled position
+        const uint32_t off = static_cast<uint32_t>(bl) * 128u + (static_cast<uint32_t>(c ^ (bl & 7)) << 4);
+        *reinterpret_cast<uint4*>(hi_t + off) = hv;
+        *reinterpret_cast<uint4*>(hi_t + half_bytes + off) = lv;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&conv[s]);
+    }
   }
   __syncthreads();
   if (!mbar_wait(done, 0)) ok = false;
@@ -1287,11 +1358,11 @@ upproj_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
   cluster.sync();
   const int per = (p.npad + KS - 1) / KS;
   const int n_lo = ks * per, n_hi = min(p.npad, n_lo + per);
-  for (int x = tid; x < (n_hi - n_lo) * 128; x += kUpThreads) {
+  for (int x = tid; x < (n_hi - n_lo) * 128; x += kFinThreads) {
     const int n = n_lo + x / 128, m = x % 128;
     const int b = b0 + n;
     const int dm = mt * 128 + m;
-    if (b >= p.B || dm >= p.d) continue;
+    if (n >= nb || dm >= p.d) continue;
     float acc = 0.f;
     for (int c = 0; c < KS; ++c) acc += cluster.map_shared_rank(part, c)[n * 128 + m];
     p.out[(static_cast<size_t>(b) * p.H + h) * p.d + dm] = __float2half_rn(acc);

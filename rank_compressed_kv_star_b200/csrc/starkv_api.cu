@@ -38,9 +38,6 @@
 #ifndef STARKV_V_RING_BYTES
 #define STARKV_V_RING_BYTES (105 * 1024)
 #endif
-#ifndef STARKV_UP_CTAS_PER_SM
-#define STARKV_UP_CTAS_PER_SM 1
-#endif
 
 namespace starkv {
 namespace {
@@ -97,9 +94,9 @@ struct DecodePlan {
   int n_rr, r_range, r_range_pad, n_chunks, n_mtiles, v_stages, v_ctas, v_per_sm;
   uint32_t vtile, ltile, ptile, tmem_cols;
   size_t v_smem;
-  // up-projection (tcgen05, split-K cluster)
-  int up_mt, up_bt, up_npad, up_ks, up_kpc, up_stages;
-  uint32_t up_tmem;
+  // finish: Z / L from the partials and the up-projection (tcgen05, split-K cluster)
+  int up_mt, up_bt_rows, up_bt, up_npad, up_ks, up_kpc, up_stages, up_zrows;
+  uint32_t up_stage_bytes, up_tmem;
   size_t up_smem;
   starkv_workspace_layout ws;
 };
@@ -277,28 +274,31 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   p.v_ctas = sms * per_sm / p.n_rr;
   if (p.v_ctas < 1) p.v_ctas = 1;
 
+  // finish: a stage holds two 64x64 B_V boxes, the hi and lo operand tiles
+  // (npad rows x 128 B each) and the partial rows a batch tile can need (its
+  // sequences plus one per V-pass CTA boundary, 256 B each); two stages.  The
+  // batch tile is the largest (<= 256 sequences, halving) whose stages fit.
+  // The epilogue's [npad][128] fp32 sums reuse the ring (two stages hold them).
   p.up_mt = (p.d + 127) / 128;    // 128-row tiles of d (rows past d are ignored)
-  p.up_bt = (batch + 255) / 256;
-  {
-    const int rows = batch < 256 ? batch : 256;
-    p.up_npad = rows < 16 ? 16 : (rows + 15) / 16 * 16;
+  p.up_stages = 2;
+  p.up_bt_rows = batch < kFinMaxRows ? (batch > 0 ? batch : 1) : kFinMaxRows;
+  for (;;) {
+    p.up_npad = p.up_bt_rows < 16 ? 16 : (p.up_bt_rows + 15) / 16 * 16;
+    const int need = p.up_bt_rows + p.v_ctas - 1;
+    p.up_zrows = (need + kFinZBox - 1) / kFinZBox * kFinZBox;
+    p.up_stage_bytes = static_cast<uint32_t>(
+        align_up(2u * kFinKC * 128u + 2u * static_cast<size_t>(p.up_npad) * 128u + p.up_zrows * 256u, 1024));
+    p.up_smem = 1024 + static_cast<size_t>(p.up_stages) * p.up_stage_bytes + (3 * p.up_stages + 1) * sizeof(uint64_t) +
+                3 * kFinMaxRows * 4;
+    if (p.up_smem <= 220u * 1024u || p.up_bt_rows <= 16) break;
+    p.up_bt_rows = p.up_bt_rows / 2 < 16 ? 16 : p.up_bt_rows / 2 / 16 * 16;
   }
+  p.up_bt = batch > 0 ? (batch + p.up_bt_rows - 1) / p.up_bt_rows : 1;
   p.up_ks = 1;
-  while (p.up_ks < 8 && p.H * p.up_mt * p.up_bt * p.up_ks * 2 <= sms * STARKV_UP_CTAS_PER_SM &&
-         p.R / kUpKC >= p.up_ks * 2)
+  while (p.up_ks < 8 && p.H * p.up_mt * p.up_bt * p.up_ks * 2 <= sms && p.R / kFinKC >= p.up_ks * 2)
     p.up_ks *= 2;
-  p.up_kpc = ((p.R + p.up_ks * kUpKC - 1) / (p.up_ks * kUpKC)) * kUpKC;
-  {
-    // stage: two 64x64 B_V boxes + hi and lo Z boxes (npad rows x 128 B); the
-    // epilogue's [npad][128] fp32 partial reuses the ring (>= 2 stages always hold it)
-    const size_t stage = 2u * kUpKC * 128u + 2u * static_cast<size_t>(p.up_npad) * 128u;
-    p.up_stages = static_cast<int>((160u * 1024u / STARKV_UP_CTAS_PER_SM) / stage);
-    if (p.up_stages > 4) p.up_stages = 4;
-    if (p.up_stages < 2) p.up_stages = 2;
-    while (static_cast<size_t>(p.up_stages) * stage < static_cast<size_t>(p.up_npad) * 512u) ++p.up_stages;
-    p.up_tmem = static_cast<uint32_t>(pow2_ceil(p.up_npad < 32 ? 32 : p.up_npad));
-    p.up_smem = 1024 + p.up_stages * stage + (2 * p.up_stages + 1) * sizeof(uint64_t);
-  }
+  p.up_kpc = ((p.R + p.up_ks * kFinKC - 1) / (p.up_ks * kFinKC)) * kFinKC;
+  p.up_tmem = static_cast<uint32_t>(pow2_ceil(p.up_npad < 32 ? 32 : p.up_npad));
 
   // workspace layout
   starkv_workspace_layout& w = p.ws;
@@ -319,8 +319,6 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   w.r_range = p.r_range;
   w.zpart_off = off;
   off = align_up(off + static_cast<size_t>(p.n_rr) * w.v_slots * p.H * p.r_range * 4, 256);
-  w.zhi_off = off; off = align_up(off + static_cast<size_t>(p.H) * batch * p.R * 2, 256);
-  w.zlo_off = off; off = align_up(off + static_cast<size_t>(p.H) * batch * p.R * 2, 256);
   w.k_tensor = p.ktc ? 1 : 0;
   w.qth_off = 0;
   if (p.ktc) { w.qth_off = off; off = align_up(off + static_cast<size_t>(batch) * 2 * p.H * p.r * 2, 256); }
@@ -366,6 +364,22 @@ bool encode_2d_map(CUtensorMap* map, const void* base, uint64_t cols, uint64_t r
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Row-major fp32 matrix [rows][cols] as a 2-D tensor map with boxes of
+// box_cols x box_rows, no swizzle (rows land back to back in shared memory).
+bool encode_f32_rows_map(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                         uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -522,14 +536,19 @@ int32_t starkv_rank_from_spectrum(const double* s, int32_t n, double tau) {
 }
 
 namespace {
-// Compress rows of k, v and store their codes at the target rows (see AppendTarget).
-starkv_status compress_store_impl(const starkv_layer_desc* desc, int32_t batch, const void* k, const void* v,
-                                  const void* A_K, const void* A_V, AppendTarget tgt, void* k_cache,
-                                  void* v_cache, void* stream) {
-  starkv_status st = check_desc(desc);
-  if (st != STARKV_OK) return st;
-  if (batch < 0) return STARKV_ERR_INVALID_ARG;
-  if (batch == 0) return STARKV_OK;
+// Launch plan of the append roles of the prep kernel: the V-code GEMM tiles
+// and the K-code items of `batch` new rows of k, v stored at `tgt`.
+struct AppendPlan {
+  CUtensorMap amap, vmap;
+  AppendVParams vp;
+  AppendKParams kp;
+  int v_mt, v_cols, KS;
+  size_t v_smem, k_smem;
+};
+
+starkv_status plan_append(const starkv_layer_desc* desc, int32_t batch, const void* k, const void* v,
+                          const void* A_K, const void* A_V, AppendTarget tgt, void* k_cache, void* v_cache,
+                          AppendPlan* ap) {
   if (!k || !v || !A_K || !A_V || !k_cache || !v_cache) return STARKV_ERR_INVALID_ARG;
   if (!tgt.slots && (!tgt.tables || !tgt.positions)) return STARKV_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v) || !aligned16(A_K) || !aligned16(A_V) || !aligned16(k_cache) ||
@@ -538,22 +557,21 @@ starkv_status compress_store_impl(const starkv_layer_desc* desc, int32_t batch, 
     return STARKV_ERR_INVALID_ARG;
   const int H = kv_heads(desc), d = desc->head_dim, r = desc->k_rank, R = desc->v_rank;   // codes per KV head
   const int HD = H * d;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-
-  // ---- joint V codes: tcgen05 GEMM, split-K over a cluster
-  CUtensorMap amap, vmap;
+  // joint V codes: tcgen05 GEMM, split-K over a cluster
   const int n_bt = (batch + 255) / 256;
   const int bt_rows = batch < 256 ? batch : 256;
   const int npad = (bt_rows + 15) / 16 * 16;
-  if (!encode_2d_map(&amap, A_V, static_cast<uint64_t>(R), static_cast<uint64_t>(HD), 64, kAppKC) ||
-      !encode_2d_map(&vmap, v, static_cast<uint64_t>(HD), static_cast<uint64_t>(batch), 64,
+  if (!encode_2d_map(&ap->amap, A_V, static_cast<uint64_t>(R), static_cast<uint64_t>(HD), 64, kAppKC) ||
+      !encode_2d_map(&ap->vmap, v, static_cast<uint64_t>(HD), static_cast<uint64_t>(batch), 64,
                      static_cast<uint32_t>(npad)))
     return STARKV_ERR_CUDA;
-  const int n_mt = (R + 127) / 128;
+  ap->v_mt = (R + 127) / 128;
+  ap->v_cols = ap->v_mt * n_bt;
   const int sms = device_sm_count();
   int KS = 1;
-  while (KS < 8 && n_mt * n_bt * KS * 2 <= sms && (HD / kAppKC) >= KS * 2) KS *= 2;
-  AppendVParams vp;
+  while (KS < 8 && ap->v_cols * KS * 2 <= sms && (HD / kAppKC) >= KS * 2) KS *= 2;
+  ap->KS = KS;
+  AppendVParams& vp = ap->vp;
   vp.tgt = tgt;
   vp.v_cache = static_cast<__half*>(v_cache);
   vp.B = batch; vp.HD = HD; vp.R = R;
@@ -562,24 +580,87 @@ starkv_status compress_store_impl(const starkv_layer_desc* desc, int32_t batch, 
   vp.stages = 4;
   vp.tmem_cols = static_cast<uint32_t>(pow2_ceil(npad < 32 ? 32 : npad));
   const size_t stage_bytes = 2u * kAppKC * 128u + static_cast<size_t>(npad) * 128u;
-  const size_t smem = 1024 + vp.stages * stage_bytes + (2 * vp.stages + 1) * sizeof(uint64_t);
-  if (!set_smem(append_v_kernel, smem)) return STARKV_ERR_CUDA;
-  if (launch(append_v_kernel, dim3(n_mt, KS, n_bt), dim3(kAppThreads), smem, s, KS, amap, vmap, vp) != cudaSuccess)
-    return STARKV_ERR_CUDA;
-
-  // ---- head-wise K codes
-  AppendKParams kp;
+  ap->v_smem = vp.stages * stage_bytes + (2 * vp.stages + 1) * sizeof(uint64_t);
+  // head-wise K codes
+  AppendKParams& kp = ap->kp;
   kp.tgt = tgt;
   kp.k = static_cast<const __half*>(k);
   kp.A_K = static_cast<const __half*>(A_K);
   kp.k_cache = static_cast<__half*>(k_cache);
   kp.H = H; kp.d = d; kp.r = r;
   kp.B = batch;
-  const size_t ksm = (static_cast<size_t>(d) * r + static_cast<size_t>(kAppKB) * d) * 2;
-  if (!set_smem(append_k_kernel, ksm)) return STARKV_ERR_CUDA;
-  if (launch(append_k_kernel, dim3(H, (batch + kAppKB - 1) / kAppKB), dim3(256), ksm, s, 1, kp) != cudaSuccess)
-    return STARKV_ERR_CUDA;
+  kp.tile = kAppKB;
+  ap->k_smem = (static_cast<size_t>(d) * r + static_cast<size_t>(kAppKB) * d) * 2;
   return STARKV_OK;
+}
+
+extern "C++" {
+template <int D>
+cudaError_t launch_prep_d(const PrepParams& pp, const CUtensorMap& amap, const CUtensorMap& vmap, dim3 grid,
+                          size_t smem, int KS, cudaStream_t s) {
+  if (!set_smem(prep_kernel<D>, smem)) return cudaErrorInvalidValue;
+  return launch(prep_kernel<D>, grid, dim3(kPrepThreads), smem, s, KS, amap, vmap, pp);
+}
+}
+
+// One prep launch: the append roles of `app` (null: none) and the query
+// absorption `abs` (null: none) over `batch` rows.  Small items are sized so
+// that the grid stays within about one CTA per SM.
+starkv_status launch_prep(int d, const AppendPlan* app, const AbsorbParams* abs, int batch, cudaStream_t s) {
+  PrepParams pp;
+  std::memset(&pp, 0, sizeof(pp));
+  const int KS = app ? app->KS : 1;
+  const int sms = device_sm_count();
+  const int v_ctas = app ? app->v_cols * KS : 0;
+  const int spare = sms - v_ctas > 2 * KS ? sms - v_ctas : 2 * KS;
+  const int k_heads = app ? app->kp.H : 0;
+  const int a_heads = abs ? abs->H : 0;
+  int tile = 16;
+  while (tile < kAbsBT && (k_heads + a_heads) * ((batch + tile - 1) / tile) > spare) tile *= 2;
+  size_t smem = 0;
+  CUtensorMap none;
+  std::memset(&none, 0, sizeof(none));
+  if (app) {
+    pp.v = app->vp;
+    pp.k = app->kp;
+    pp.k.tile = tile;
+    pp.v_mt = app->v_mt;
+    pp.v_cols = app->v_cols;
+    pp.k_items = k_heads * ((batch + tile - 1) / tile);
+    pp.k_cols = (pp.k_items + KS - 1) / KS;
+    smem = app->v_smem > app->k_smem ? app->v_smem : app->k_smem;
+  }
+  if (abs) {
+    pp.a = *abs;
+    pp.a_tile = tile;
+    pp.a_items = a_heads * ((batch + tile - 1) / tile);
+    const size_t qs = static_cast<size_t>(tile) * d * 2;
+    if (qs > smem) smem = qs;
+  }
+  smem += 1024;   // room to align the dynamic shared memory to 1024 bytes
+  const dim3 grid(pp.v_cols + pp.k_cols + (pp.a_items + KS - 1) / KS, KS);
+  const CUtensorMap& amap = app ? app->amap : none;
+  const CUtensorMap& vmap = app ? app->vmap : none;
+  cudaError_t e;
+  if (d == 32) e = launch_prep_d<32>(pp, amap, vmap, grid, smem, KS, s);
+  else if (d == 64) e = launch_prep_d<64>(pp, amap, vmap, grid, smem, KS, s);
+  else if (d == 128) e = launch_prep_d<128>(pp, amap, vmap, grid, smem, KS, s);
+  else e = launch_prep_d<256>(pp, amap, vmap, grid, smem, KS, s);
+  return e == cudaSuccess ? STARKV_OK : STARKV_ERR_CUDA;
+}
+
+// Compress rows of k, v and store their codes at the target rows (see AppendTarget).
+starkv_status compress_store_impl(const starkv_layer_desc* desc, int32_t batch, const void* k, const void* v,
+                                  const void* A_K, const void* A_V, AppendTarget tgt, void* k_cache,
+                                  void* v_cache, void* stream) {
+  starkv_status st = check_desc(desc);
+  if (st != STARKV_OK) return st;
+  if (batch < 0) return STARKV_ERR_INVALID_ARG;
+  if (batch == 0) return STARKV_OK;
+  AppendPlan ap;
+  st = plan_append(desc, batch, k, v, A_K, A_V, tgt, k_cache, v_cache, &ap);
+  if (st != STARKV_OK) return st;
+  return launch_prep(desc->head_dim, &ap, nullptr, batch, static_cast<cudaStream_t>(stream));
 }
 }  // namespace
 
@@ -654,7 +735,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
                           const void* B_K, const void* B_V, const void* k_cache, const void* v_cache,
                           const int32_t* block_tables, const int32_t* seq_lens, float scale, void* workspace,
                           size_t workspace_bytes, void* out, void* stream, void* const* stage_events,
-                          const int32_t* row_seq = nullptr) {
+                          const int32_t* row_seq = nullptr, const AppendPlan* app = nullptr) {
   DecodePlan pl;
   starkv_status st = make_plan(desc, batch, max_seq_len, &pl);
   if (st != STARKV_OK) return st;
@@ -680,21 +761,18 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   float* zpart = reinterpret_cast<float*>(ws + pl.ws.zpart_off);
 
   if (max_seq_len == 0) {
+    if (app && launch_prep(pl.d, app, nullptr, batch, s) != STARKV_OK) return STARKV_ERR_CUDA;
     if (cudaMemsetAsync(status, 0, 4, s) != cudaSuccess ||
         cudaMemsetAsync(out, 0, static_cast<size_t>(batch) * pl.H * pl.d * 2, s) != cudaSuccess)
       return STARKV_ERR_CUDA;
     return STARKV_OK;
   }
 
-  __half* zhi = reinterpret_cast<__half*>(ws + pl.ws.zhi_off);
-  __half* zlo = reinterpret_cast<__half*>(ws + pl.ws.zlo_off);
-  CUtensorMap vmap, bvmap, zhimap, zlomap;
+  CUtensorMap vmap, bvmap, zmap;
   if (!encode_vpool_map(&vmap, v_cache, pl.R, pl.NB, static_cast<uint32_t>(pl.n_chunks))) return STARKV_ERR_CUDA;
-  if (!encode_2d_map(&bvmap, B_V, static_cast<uint64_t>(pl.Hkv) * pl.d, static_cast<uint64_t>(pl.R), 64, kUpKC) ||
-      !encode_2d_map(&zhimap, zhi, static_cast<uint64_t>(pl.R), static_cast<uint64_t>(pl.H) * batch, 64,
-                     static_cast<uint32_t>(pl.up_npad)) ||
-      !encode_2d_map(&zlomap, zlo, static_cast<uint64_t>(pl.R), static_cast<uint64_t>(pl.H) * batch, 64,
-                     static_cast<uint32_t>(pl.up_npad)))
+  if (!encode_2d_map(&bvmap, B_V, static_cast<uint64_t>(pl.Hkv) * pl.d, static_cast<uint64_t>(pl.R), 64, kFinKC) ||
+      !encode_f32_rows_map(&zmap, zpart, static_cast<uint64_t>(pl.r_range),
+                           static_cast<uint64_t>(pl.n_rr) * pl.H * pl.ws.v_slots, 64, kFinZBox))
     return STARKV_ERR_CUDA;
   auto mark = [&](int i) {
     if (stage_events && stage_events[i]) cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), s);
@@ -712,15 +790,8 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   ap.n_mpart = pl.ws.k_slots * pl.H;
   ap.B = batch; ap.H = pl.H; ap.d = pl.d; ap.r = pl.r; ap.cap = pl.cap; ap.log2G = pl.log2G;
   ap.coef = scale * kLog2e;
-  {
-    const dim3 grid(pl.H, (batch + kAbsBT - 1) / kAbsBT);
-    cudaError_t ea;
-    if (pl.d == 32) ea = launch(absorb_kernel<32>, grid, dim3(256), 0, s, 1, ap);
-    else if (pl.d == 64) ea = launch(absorb_kernel<64>, grid, dim3(256), 0, s, 1, ap);
-    else if (pl.d == 128) ea = launch(absorb_kernel<128>, grid, dim3(256), 0, s, 1, ap);
-    else ea = launch(absorb_kernel<256>, grid, dim3(256), 0, s, 1, ap);
-    if (ea != cudaSuccess) return STARKV_ERR_CUDA;
-  }
+  // the query absorption, with the step's compress-and-append in the same launch when fused
+  if (launch_prep(pl.d, app, &ap, batch, s) != STARKV_OK) return STARKV_ERR_CUDA;
   mark(1);
 
   KPassParams kp;
@@ -772,24 +843,18 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
     return STARKV_ERR_CUDA;
   mark(3);
 
-  ZFinalParams zf;
-  zf.zpart = zpart; zf.lpart = lpart; zf.prefix = prefix; zf.zhi = zhi; zf.zlo = zlo;
-  zf.B = batch; zf.H = pl.H; zf.R = pl.R; zf.r_range = pl.r_range; zf.v_slots = pl.ws.v_slots;
-  zf.v_grid = pl.v_ctas;
-  if (launch(zfinal_kernel, dim3((pl.R + 2047) / 2048, batch * pl.H), dim3(256), 0, s, 1, zf) != cudaSuccess)
+  FinishParams fp;
+  fp.out = static_cast<__half*>(out);
+  fp.lpart = lpart; fp.prefix = prefix;
+  fp.B = batch; fp.H = pl.H; fp.d = pl.d; fp.R = pl.R; fp.log2G = pl.log2G;
+  fp.r_range = pl.r_range; fp.v_slots = pl.ws.v_slots; fp.v_grid = pl.v_ctas;
+  fp.n_mt = pl.up_mt; fp.bt_rows = pl.up_bt_rows; fp.k_per_cta = pl.up_kpc; fp.npad = pl.up_npad;
+  fp.stages = pl.up_stages; fp.zrows = pl.up_zrows; fp.stage_bytes = pl.up_stage_bytes; fp.tmem_cols = pl.up_tmem;
+  if (!set_smem(finish_kernel, pl.up_smem)) return STARKV_ERR_CUDA;
+  if (launch(finish_kernel, dim3(pl.H * pl.up_mt * pl.up_bt, pl.up_ks), dim3(kFinThreads), pl.up_smem, s, pl.up_ks,
+             bvmap, zmap, fp) != cudaSuccess)
     return STARKV_ERR_CUDA;
   mark(4);
-
-  UpProjParams up;
-  up.out = static_cast<__half*>(out);
-  up.B = batch; up.H = pl.H; up.d = pl.d; up.R = pl.R; up.log2G = pl.log2G;
-  up.n_mt = pl.up_mt; up.k_per_cta = pl.up_kpc; up.npad = pl.up_npad;
-  up.stages = pl.up_stages; up.tmem_cols = pl.up_tmem;
-  if (!set_smem(upproj_kernel, pl.up_smem)) return STARKV_ERR_CUDA;
-  if (launch(upproj_kernel, dim3(pl.H * pl.up_mt * pl.up_bt, pl.up_ks), dim3(kUpThreads), pl.up_smem, s, pl.up_ks,
-             bvmap, zhimap, zlomap, up) != cudaSuccess)
-    return STARKV_ERR_CUDA;
-  mark(5);
   return STARKV_OK;
 }
 }  // namespace
@@ -800,6 +865,25 @@ starkv_status starkv_paged_decode(const starkv_layer_desc* desc, int32_t batch, 
                                   float scale, void* workspace, size_t workspace_bytes, void* out, void* stream) {
   return decode_impl(desc, batch, max_seq_len, q, B_K, B_V, k_cache, v_cache, block_tables, seq_lens, scale,
                      workspace, workspace_bytes, out, stream, nullptr);
+}
+
+starkv_status starkv_append_decode(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len,
+                                   const void* k, const void* v, const void* A_K, const void* A_V,
+                                   const int32_t* positions, const void* q, const void* B_K, const void* B_V,
+                                   void* k_cache, void* v_cache, const int32_t* block_tables,
+                                   const int32_t* seq_lens, float scale, void* workspace, size_t workspace_bytes,
+                                   void* out, int32_t* append_status, void* stream) {
+  starkv_status st = check_desc(desc);
+  if (st != STARKV_OK) return st;
+  if (batch < 0) return STARKV_ERR_INVALID_ARG;
+  if (batch == 0) return clear_status(workspace, workspace_bytes, stream);
+  if (!block_tables || !positions || (reinterpret_cast<uintptr_t>(append_status) & 3u)) return STARKV_ERR_INVALID_ARG;
+  AppendTarget tgt{nullptr, block_tables, positions, desc->max_blocks_per_seq, desc->num_blocks, append_status};
+  AppendPlan ap;
+  st = plan_append(desc, batch, k, v, A_K, A_V, tgt, k_cache, v_cache, &ap);
+  if (st != STARKV_OK) return st;
+  return decode_impl(desc, batch, max_seq_len, q, B_K, B_V, k_cache, v_cache, block_tables, seq_lens, scale,
+                     workspace, workspace_bytes, out, stream, nullptr, nullptr, &ap);
 }
 
 // Prefill workspace: the decode workspace of n_rows rows, then the rows'

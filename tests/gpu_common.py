@@ -87,14 +87,35 @@ def full_check(wl, layer=0):
     return Lh, Ld, got, ws, desc, err, rl
 
 
-def append_check(wl, layer=0, Ld=None):
+def append_only(Ld, desc, status, B):
+    S.starkv_compress_append(desc, B, Ld["k"], Ld["v"], Ld["A_K"], Ld["A_V"], Ld["tables"], Ld["ctx_lens"],
+                             Ld["k_cache"], Ld["v_cache"], status=status)
+
+
+def append_then_decode(Ld, desc, status, B):
+    """The step as one call (starkv_append_decode): returns the decode output and its workspace."""
+    T = int(Ld["seq_lens"].max().item())
+    wsb = S.starkv_decode_workspace_bytes(desc, B, T)
+    ws = torch.full((max(wsb, 256),), POISON, dtype=torch.uint8, device="cuda")
+    out = torch.full((B, Ld["H"], Ld["d"]), float("nan"), dtype=torch.float16, device="cuda")
+    S.starkv_append_decode(desc, B, T, Ld["k"], Ld["v"], Ld["A_K"], Ld["A_V"], Ld["ctx_lens"], Ld["q"], Ld["B_K"],
+                           Ld["B_V"], Ld["k_cache"], Ld["v_cache"], Ld["tables"], Ld["seq_lens"], Ld["scale"],
+                           ws, wsb, out, append_status=status)
+    st, flags = S.starkv_decode_check(ws)
+    assert st == 0, (S.STATUS[st], flags)
+    return out.float().cpu().numpy().astype(np.float64), ws
+
+
+def append_check(wl, layer=0, Ld=None, run=append_only):
     """Compress-and-append of one token per sequence through the C ABI, whole batch.
 
-    Bit-exact: every byte of both pools outside the batch's target slots is
-    unchanged (compared on the device), and the status word reports no skipped
-    target.  Values: each target slot's codes against the oracle's fp64 codes
-    of the same fp16 inputs, within one fp16 ulp plus the fp32 dot-product
-    bound.  Returns the device layer and the oracle's fp16 codes.
+    ``run(Ld, desc, status, batch)`` makes the call that appends (by default
+    starkv_compress_append alone).  Bit-exact: every byte of both pools
+    outside the batch's target slots is unchanged (compared on the device),
+    and the status word reports no skipped target.  Values: each target
+    slot's codes against the oracle's fp64 codes of the same fp16 inputs,
+    within one fp16 ulp plus the fp32 dot-product bound.  Returns the device
+    layer, the oracle's fp16 codes and what ``run`` returned.
     """
     if Ld is None:
         Ld = D.device_layer(wl, layer)
@@ -104,8 +125,7 @@ def append_check(wl, layer=0, Ld=None):
     vf = Ld["v_cache"].view(-1, R)
     before_k, before_v = kf.clone(), vf.clone()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    S.starkv_compress_append(desc, wl.batch, Ld["k"], Ld["v"], Ld["A_K"], Ld["A_V"], Ld["tables"],
-                             Ld["ctx_lens"], Ld["k_cache"], Ld["v_cache"], status=status)
+    ran = run(Ld, desc, status, wl.batch)
     st, flags = S.starkv_decode_check(status)
     assert st == 0 and flags == 0, (S.STATUS[st], flags)
     pos = wl.ctx_lens
@@ -140,7 +160,7 @@ def append_check(wl, layer=0, Ld=None):
         assert np.all(np.abs(got - want) <= bound), np.max(np.abs(got - want) / bound)
         assert np.abs(got - want).max() <= MAX_ABS
         assert rel_l2(got, want) <= REL_L2
-    return Ld, (cK.astype(np.float16), cV.astype(np.float16))
+    return Ld, (cK.astype(np.float16), cV.astype(np.float16)), ran
 
 
 def load():

@@ -116,7 +116,7 @@ def test_workspace_layout_is_consistent(lib):
     lay = S.starkv_decode_workspace_layout(d, 64, 8192)
     assert lay.total_bytes == S.starkv_decode_workspace_bytes(d, 64, 8192)
     offs = [lay.status_off, lay.prefix_off, lay.qt_off, lay.logits_off, lay.mpart_off,
-            lay.lpart_off, lay.zpart_off, lay.zhi_off, lay.zlo_off]
+            lay.lpart_off, lay.zpart_off]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     assert lay.t_pad == 8192 and lay.k_slots == lay.k_ctas + 64 and lay.v_slots == lay.v_ctas + 64
     assert lay.n_rranges * lay.r_range >= 2048

@@ -11,7 +11,8 @@ import pytest
 import torch
 
 from starkv_inputs import workloads as W
-from gpu_common import (append_check, assert_close, full_check, load, oracle_rows, run_decode)
+from gpu_common import (append_check, append_then_decode, assert_close, full_check, load, oracle_rows,
+                        run_decode)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,14 +38,13 @@ def test_decode_tiny_workload():
     (6, 0, [0, 21, 63]),                # grouped-query layer, batch 64, context 8192
 ])
 def test_full_size_append_then_decode(idx, layer, sample):
-    """Full-size workloads in the benchmark's launch configuration.
+    """Full-size workloads in the benchmark's launch configuration (one starkv_append_decode per step).
 
     The whole batch's append is checked (placement and untouched bytes
     bit-exact, codes against the oracle), then decode on sampled sequences.
     """
     wl = W.workload(idx)
-    Ld, appended = append_check(wl, layer)
-    got, *_ = run_decode(Ld)
+    Ld, appended, (got, _) = append_check(wl, layer, run=append_then_decode)
     ref = oracle_rows(wl, layer, W.activation(wl, layer, W.ACT_Q), Ld["A_np"], sample, wl.seq_lens,
                       appended)
     assert_close({b: got[b] for b in sample}, ref)
@@ -56,6 +56,21 @@ def test_full_size_append_then_decode(idx, layer, sample):
 def test_append_tiny_ragged():
     """Positions 37, 100, 0 and 15: mid-page, page start of a new page, the first slot, a page's last slot."""
     append_check(W.custom("app", 31, W.LayerShape(4, 64, 16, 64), [37, 100, 0, 15]))
+
+
+@pytest.mark.parametrize("kv_heads", [0, 8])
+def test_fused_step_equals_append_then_decode_calls(kv_heads):
+    """starkv_append_decode against starkv_compress_append + starkv_paged_decode: identical pools and outputs."""
+    sh = W.LayerShape(32, 128, 64, 2048 if not kv_heads else 512, num_kv_heads=kv_heads)
+    wl = W.custom("fused", 4141 + kv_heads, sh, [37, 100, 0, 15, 700, 2047, 31], append=True)
+    La, appended, _ = append_check(wl)
+    sep, *_ = run_decode(La)
+    Lb, _, (fused, _) = append_check(wl, run=append_then_decode)
+    assert torch.equal(La["k_cache"].view(torch.int16), Lb["k_cache"].view(torch.int16))
+    assert torch.equal(La["v_cache"].view(torch.int16), Lb["v_cache"].view(torch.int16))
+    assert np.array_equal(sep, fused)
+    ref = oracle_rows(wl, 0, W.activation(wl, 0, W.ACT_Q), La["A_np"], range(wl.batch), wl.seq_lens, appended)
+    assert_close({b: fused[b] for b in range(wl.batch)}, ref)
 
 
 @pytest.mark.parametrize("H,Hkv,d,r,R", [
@@ -76,7 +91,7 @@ def test_decode_grouped_query(H, Hkv, d, r, R):
 def test_append_then_decode_grouped_query():
     sh = W.LayerShape(32, 128, 64, 512, num_kv_heads=8)
     wl = W.custom("gqa-app", 777, sh, [37, 100, 0, 15, 2000, 4095], append=True)
-    Ld, appended = append_check(wl)
+    Ld, appended, _ = append_check(wl)
     got, *_ = run_decode(Ld)
     ref = oracle_rows(wl, 0, W.activation(wl, 0, W.ACT_Q), Ld["A_np"], range(wl.batch), wl.seq_lens,
                       appended)

@@ -426,7 +426,7 @@ def test_decode_and_append_batch_over_256(kv_heads):
     sh = W.LayerShape(32, 128, 64, 2048 if not kv_heads else 512, num_kv_heads=kv_heads)
     rng = np.random.default_rng(5)
     wl = W.custom("wide", 5150, sh, rng.integers(1, 48, size=300), append=True)
-    Ld, appended = append_check(wl)
+    Ld, appended, _ = append_check(wl)
     got, *_ = run_decode(Ld)
     sample = [0, 1, 255, 256, 257, 299]
     ref = oracle_rows(wl, 0, W.activation(wl, 0, W.ACT_Q), Ld["A_np"], sample, wl.seq_lens, appended)
