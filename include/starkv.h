@@ -204,6 +204,30 @@ starkv_status starkv_append_decode(const starkv_layer_desc* desc, int32_t batch,
                                    int32_t* append_status, void* stream);
 
 /*
+ * starkv_append_decode_host -- starkv_append_decode for a caller whose step
+ * inputs are in HOST memory (pinned memory lets the copies overlap): the new
+ * tokens' k, v, their positions, the queries, the block tables and the
+ * lengths are copied to `staging` (caller-owned DEVICE memory of at least
+ * starkv_host_staging_bytes(desc, batch) bytes, 256-byte aligned) with one
+ * cudaMemcpyAsync each on `stream`, the step runs there, and `out` is copied
+ * back to the HOST array out_host (fp16 [batch][H][d]).  Everything is
+ * enqueued asynchronously: out_host is valid after the stream synchronises.
+ * The projections, pools and workspace are device memory as in
+ * starkv_append_decode; argument errors return before anything is enqueued.
+ * (Same method passage as starkv_append_decode.)
+ */
+size_t starkv_host_staging_bytes(const starkv_layer_desc* desc, int32_t batch);
+starkv_status starkv_append_decode_host(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len,
+                                        const void* k_host, const void* v_host,
+                                        const int32_t* positions_host, const void* q_host,
+                                        const int32_t* block_tables_host, const int32_t* seq_lens_host,
+                                        const void* A_K, const void* A_V, const void* B_K,
+                                        const void* B_V, void* k_cache, void* v_cache, float scale,
+                                        void* staging, size_t staging_bytes, void* workspace,
+                                        size_t workspace_bytes, void* out_host, int32_t* append_status,
+                                        void* stream);
+
+/*
  * starkv_paged_prefill -- causal attention of prefill chunks over the paged
  * codes (chunked prefill).  The step that precedes decode: a prompt is
  * compressed into the cache chunk by chunk (starkv_compress_store) and each

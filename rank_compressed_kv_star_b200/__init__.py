@@ -25,7 +25,7 @@ FLAG_BAD_BLOCK_ID, FLAG_BAD_SEQ_LEN, FLAG_TIMEOUT = 1, 2, 4
 
 EXPORTED = (
     "starkv_compress_append", "starkv_compress_store", "starkv_decode_workspace_bytes",
-    "starkv_paged_decode", "starkv_append_decode",
+    "starkv_paged_decode", "starkv_append_decode", "starkv_append_decode_host", "starkv_host_staging_bytes",
     "starkv_paged_decode_profiled", "starkv_paged_decode_static",
     "starkv_decode_check", "starkv_decode_workspace_layout", "starkv_status_string",
     "starkv_rank_from_spectrum", "starkv_version", "starkv_kv_bytes_per_token", "starkv_num_blocks",
@@ -91,6 +91,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.starkv_append_decode.argtypes = [DP, I32, I32, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_float,
                                          P, SZ, P, P, P]
     lib.starkv_append_decode.restype = ctypes.c_int
+    lib.starkv_host_staging_bytes.argtypes = [DP, I32]
+    lib.starkv_host_staging_bytes.restype = SZ
+    lib.starkv_append_decode_host.argtypes = [DP, I32, I32, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_float,
+                                              P, SZ, P, SZ, P, P, P]
+    lib.starkv_append_decode_host.restype = ctypes.c_int
     lib.starkv_paged_decode_profiled.argtypes = [DP, I32, I32, P, P, P, P, P, P, P, ctypes.c_float,
                                                  P, SZ, P, P, ctypes.POINTER(P)]
     lib.starkv_paged_decode_profiled.restype = ctypes.c_int
@@ -204,6 +209,25 @@ def starkv_append_decode(desc: LayerDesc, batch: int, max_seq_len: int, k, v, A_
         _ptr(workspace), int(workspace_bytes), _ptr(out), _ptr(append_status), _stream(stream))
     if check:
         _check(st, "starkv_append_decode")
+    return st
+
+
+def starkv_host_staging_bytes(desc: LayerDesc, batch: int) -> int:
+    return int(load_library().starkv_host_staging_bytes(_desc_ref(desc), batch))
+
+
+def starkv_append_decode_host(desc: LayerDesc, batch: int, max_seq_len: int, k_host, v_host, positions_host,
+                              q_host, block_tables_host, seq_lens_host, A_K, A_V, B_K, B_V, k_cache, v_cache,
+                              scale: float, staging, staging_bytes: int, workspace, workspace_bytes: int,
+                              out_host, stream=None, check: bool = True, append_status=None) -> int:
+    """The step from host buffers (``*_host``: pinned CPU tensors or addresses); copies run in the call."""
+    st = load_library().starkv_append_decode_host(
+        _desc_ref(desc), batch, max_seq_len, _ptr(k_host), _ptr(v_host), _ptr(positions_host), _ptr(q_host),
+        _ptr(block_tables_host), _ptr(seq_lens_host), _ptr(A_K), _ptr(A_V), _ptr(B_K), _ptr(B_V),
+        _ptr(k_cache), _ptr(v_cache), float(scale), _ptr(staging), int(staging_bytes), _ptr(workspace),
+        int(workspace_bytes), _ptr(out_host), _ptr(append_status), _stream(stream))
+    if check:
+        _check(st, "starkv_append_decode_host")
     return st
 
 

@@ -886,6 +886,85 @@ starkv_status starkv_append_decode(const starkv_layer_desc* desc, int32_t batch,
                      workspace, workspace_bytes, out, stream, nullptr, nullptr, &ap);
 }
 
+// Staging layout of starkv_append_decode_host: the step's inputs and output
+// as device copies, each 256-byte aligned.
+struct HostStaging {
+  size_t k, v, q, pos, lens, tables, out, total;
+};
+
+bool host_staging(const starkv_layer_desc* desc, int32_t batch, HostStaging* st) {
+  if (check_desc(desc) != STARKV_OK || batch < 0) return false;
+  const size_t B = static_cast<size_t>(batch);
+  const size_t kv = B * kv_heads(desc) * desc->head_dim * 2, qo = B * desc->num_heads * desc->head_dim * 2;
+  size_t off = 0;
+  st->k = off; off = align_up(off + kv, 256);
+  st->v = off; off = align_up(off + kv, 256);
+  st->q = off; off = align_up(off + qo, 256);
+  st->pos = off; off = align_up(off + B * 4, 256);
+  st->lens = off; off = align_up(off + B * 4, 256);
+  st->tables = off; off = align_up(off + B * desc->max_blocks_per_seq * 4, 256);
+  st->out = off; off = align_up(off + qo, 256);
+  st->total = off > 256 ? off : 256;
+  return true;
+}
+
+size_t starkv_host_staging_bytes(const starkv_layer_desc* desc, int32_t batch) {
+  HostStaging st;
+  return host_staging(desc, batch, &st) ? st.total : 0;
+}
+
+starkv_status starkv_append_decode_host(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len,
+                                        const void* k_host, const void* v_host, const int32_t* positions_host,
+                                        const void* q_host, const int32_t* block_tables_host,
+                                        const int32_t* seq_lens_host, const void* A_K, const void* A_V,
+                                        const void* B_K, const void* B_V, void* k_cache, void* v_cache,
+                                        float scale, void* staging, size_t staging_bytes, void* workspace,
+                                        size_t workspace_bytes, void* out_host, int32_t* append_status,
+                                        void* stream) {
+  HostStaging st;
+  if (!host_staging(desc, batch, &st)) return check_desc(desc) != STARKV_OK ? check_desc(desc) : STARKV_ERR_INVALID_ARG;
+  if (batch == 0) return clear_status(workspace, workspace_bytes, stream);
+  if (!k_host || !v_host || !positions_host || !q_host || !block_tables_host || !seq_lens_host || !out_host)
+    return STARKV_ERR_INVALID_ARG;
+  if (!staging || staging_bytes < st.total || (reinterpret_cast<uintptr_t>(staging) & 255u))
+    return STARKV_ERR_WORKSPACE;
+  // the decode's own argument checks run before any copy is enqueued
+  DecodePlan pl;
+  starkv_status ps = make_plan(desc, batch, max_seq_len, &pl);
+  if (ps != STARKV_OK) return ps;
+  if (!(std::isfinite(scale) && scale > 0.f)) return STARKV_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < pl.ws.total_bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return STARKV_ERR_WORKSPACE;
+  if (!A_K || !A_V || !B_K || !B_V || !k_cache || !v_cache || !aligned16(A_K) || !aligned16(A_V) ||
+      !aligned16(B_K) || !aligned16(B_V) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(append_status) & 3u))
+    return STARKV_ERR_INVALID_ARG;
+  uint8_t* sg = static_cast<uint8_t*>(staging);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t B = static_cast<size_t>(batch);
+  const size_t kv = B * kv_heads(desc) * desc->head_dim * 2, qo = B * desc->num_heads * desc->head_dim * 2;
+  // one copy per input (no batched-copy call)
+  const struct { size_t off; const void* src; size_t bytes; } in[] = {
+      {st.k, k_host, kv}, {st.v, v_host, kv}, {st.q, q_host, qo}, {st.pos, positions_host, B * 4},
+      {st.lens, seq_lens_host, B * 4}, {st.tables, block_tables_host, B * desc->max_blocks_per_seq * 4}};
+  for (const auto& c : in)
+    if (cudaMemcpyAsync(sg + c.off, c.src, c.bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+      cudaGetLastError();
+      return STARKV_ERR_CUDA;
+    }
+  const starkv_status ds = starkv_append_decode(
+      desc, batch, max_seq_len, sg + st.k, sg + st.v, A_K, A_V, reinterpret_cast<const int32_t*>(sg + st.pos),
+      sg + st.q, B_K, B_V, k_cache, v_cache, reinterpret_cast<const int32_t*>(sg + st.tables),
+      reinterpret_cast<const int32_t*>(sg + st.lens), scale, workspace, workspace_bytes, sg + st.out,
+      append_status, stream);
+  if (ds != STARKV_OK) return ds;
+  if (cudaMemcpyAsync(out_host, sg + st.out, qo, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+    cudaGetLastError();
+    return STARKV_ERR_CUDA;
+  }
+  return STARKV_OK;
+}
+
 // Prefill workspace: the decode workspace of n_rows rows, then the rows'
 // sequence map and lengths (int32 [n_rows] each).
 size_t prefill_rows_offset(const DecodePlan& pl) { return align_up(pl.ws.total_bytes, 256); }

@@ -175,3 +175,28 @@ def test_prefill_argument_errors(lib):
 
 def test_wait_test_hook_rejects_bad_stage(lib):
     assert S.starkv_set_wait_test_hook(0, -2, check=False) == 1
+
+
+def test_host_step_argument_errors(lib):
+    """starkv_append_decode_host refuses bad arguments before it enqueues any copy."""
+    d = _desc()
+    fake = 1 << 20
+    stg = S.starkv_host_staging_bytes(d, 4)
+    ws = S.starkv_decode_workspace_bytes(d, 4, 1024)
+    assert stg >= 4 * 32 * 128 * 2 * 4 and ws > 0
+    args = [d, 4, 1024] + [fake] * 6 + [fake] * 6 + [0.1, fake, stg, fake, ws, fake]
+
+    def call(i, v):
+        a = list(args); a[i] = v
+        return S.starkv_append_decode_host(*a, stream=0, check=False)
+    # indices: 3..8 host k, v, positions, q, tables, lengths; 9..14 device A_K, A_V, B_K, B_V, pools;
+    # 15 scale, 16/17 staging and its size, 18/19 workspace and its size, 20 host out
+    assert call(3, None) == 1                    # no host k
+    assert call(20, None) == 1                   # no host output
+    assert call(17, stg - 1) == 3                # staging too small
+    assert call(16, fake + 64) == 3              # staging not 256-byte aligned
+    assert call(19, ws - 1) == 3                 # workspace too small
+    assert call(2, 64 * 16 + 1) == 1             # length bound above table capacity
+    assert call(15, float("nan")) == 1           # bad scale
+    assert call(9, None) == 1 and call(13, fake + 8) == 1   # no A_K; misaligned K pool
+    assert S.starkv_host_staging_bytes(_desc(block_size=8), 4) == 0

@@ -96,3 +96,31 @@ def test_append_then_decode_grouped_query():
     ref = oracle_rows(wl, 0, W.activation(wl, 0, W.ACT_Q), Ld["A_np"], range(wl.batch), wl.seq_lens,
                       appended)
     assert_close({b: got[b] for b in range(wl.batch)}, ref)
+
+
+def test_step_from_host_buffers_equals_device_call():
+    """starkv_append_decode_host (inputs and output in pinned host memory) against starkv_append_decode."""
+    import rank_compressed_kv_star_b200 as S
+    from gpu_common import POISON, desc_of
+    from starkv_inputs import device as D
+    sh = W.LayerShape(32, 128, 64, 2048)
+    wl = W.custom("host", 4343, sh, [37, 100, 0, 15, 700], append=True)
+    La = D.device_layer(wl, 0)
+    Lb = D.device_layer(wl, 0)
+    desc = desc_of(La)
+    B, T = wl.batch, wl.max_seq_len
+    dev_out, _ = append_then_decode(La, desc, None, B)
+    wsb = S.starkv_decode_workspace_bytes(desc, B, T)
+    ws = torch.full((wsb,), POISON, dtype=torch.uint8, device="cuda")
+    stg = S.starkv_host_staging_bytes(desc, B)
+    staging = torch.full((stg,), POISON, dtype=torch.uint8, device="cuda")
+    h = {n: Lb[n].cpu().pin_memory() for n in ("q", "k", "v", "tables", "seq_lens", "ctx_lens")}
+    out_host = torch.full((B, 32, 128), float("nan"), dtype=torch.float16).pin_memory()
+    S.starkv_append_decode_host(desc, B, T, h["k"], h["v"], h["ctx_lens"], h["q"], h["tables"], h["seq_lens"],
+                                Lb["A_K"], Lb["A_V"], Lb["B_K"], Lb["B_V"], Lb["k_cache"], Lb["v_cache"],
+                                Lb["scale"], staging, stg, ws, wsb, out_host)
+    torch.cuda.synchronize()
+    assert S.starkv_decode_check(ws) == (0, 0)
+    assert np.array_equal(out_host.float().numpy().astype(np.float64), dev_out)
+    assert torch.equal(La["k_cache"].view(torch.int16), Lb["k_cache"].view(torch.int16))
+    assert torch.equal(La["v_cache"].view(torch.int16), Lb["v_cache"].view(torch.int16))
