@@ -168,21 +168,83 @@ __device__ __forceinline__ void append_v_tile(const CUtensorMap* amap, const CUt
   // rank ks sums rows (batch entries) [ks*npad/KS, (ks+1)*npad/KS) over the cluster, in rank order
   const int per = (p.npad + KS - 1) / KS;
   const int n_lo = ks * per, n_hi = min(p.npad, n_lo + per);
-  for (int x = tid; x < (n_hi - n_lo) * 128; x += kPrepThreads) {
-    const int n = n_lo + x / 128, rrow = x % 128;
+  // four consecutive rows of R per thread, all ranks' loads issued before the
+  // adds (in rank order)
+  for (int x = tid; x < (n_hi - n_lo) * 32; x += kPrepThreads) {
+    const int n = n_lo + x / 32, rrow = (x % 32) * 4;
     const int b = b0 + n;
     const int rg = mt * 128 + rrow;
     if (b >= p.B || rg >= p.R) continue;
-    float acc = 0.f;
-    for (int c = 0; c < KS; ++c) acc += cluster.map_shared_rank(part, c)[n * 128 + rrow];
+    float4 v[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      if (c < KS) v[c] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(part, c) + n * 128 + rrow);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      if (c < KS) { acc.x += v[c].x; acc.y += v[c].y; acc.z += v[c].z; acc.w += v[c].w; }
     const int64_t dst = append_row(p.tgt, b);
-    if (dst >= 0) p.v_cache[dst * p.R + rg] = __float2half_rn(acc);
-    else if (rg == 0) append_skipped(p.tgt, dst);
+    if (dst >= 0) {
+      const __half2 lo = __floats2half2_rn(acc.x, acc.y), hi = __floats2half2_rn(acc.z, acc.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(p.v_cache + dst * p.R + rg) = pk;
+    } else if (rg == 0) {
+      append_skipped(p.tgt, dst);
+    }
   }
   cluster.sync();   // nobody leaves while others still read its partials
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(taddr, p.tmem_cols);
+  }
+}
+
+// ------------------------------------------------------------ small products
+// out[b][i] = sum_j x[b][j] * W[j][i] for nb rows of x (fp16 [nb][d]) and W
+// (fp16 [d][r]), both staged in shared memory, with fp32 accumulation.
+// Thread = (column pair p: columns 2p and 2p+1; row lane bl); each step of 8
+// along j it reads 8 column pairs of W (4-byte reads, consecutive across a
+// warp) and 8 values of each of up to kProjRows rows (16-byte broadcast
+// reads), and accumulates with packed FMAs.  emit(b, i, v_i, v_i+1) receives
+// the two columns of row b.  r must be a multiple of 16 (r/2 divides 256).
+constexpr int kProjRows = 4;
+
+template <typename Emit>
+__device__ __forceinline__ void small_proj(const __half* Ws, const __half* xs, int nb, int d, int r, Emit&& emit) {
+  const int np = r >> 1;
+  const int nbl = kPrepThreads / np;
+  const int p = static_cast<int>(threadIdx.x) % np, bl = static_cast<int>(threadIdx.x) / np;
+  for (int b0 = bl; b0 < nb; b0 += nbl * kProjRows) {
+    float2 acc[kProjRows];
+#pragma unroll
+    for (int s = 0; s < kProjRows; ++s) acc[s] = make_float2(0.f, 0.f);
+    for (int j = 0; j < d; j += 8) {
+      float2 w[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        w[u] = __half22float2(*reinterpret_cast<const __half2*>(Ws + static_cast<size_t>(j + u) * r + 2 * p));
+#pragma unroll
+      for (int s = 0; s < kProjRows; ++s) {
+        const int b = b0 + s * nbl;
+        if (b < nb) {
+          const uint4 xv = *reinterpret_cast<const uint4*>(xs + static_cast<size_t>(b) * d + j);
+          const __half2* x2 = reinterpret_cast<const __half2*>(&xv);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 xf = __half22float2(x2[u]);
+            acc[s] = ffma2(make_float2(xf.x, xf.x), w[2 * u], acc[s]);
+            acc[s] = ffma2(make_float2(xf.y, xf.y), w[2 * u + 1], acc[s]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int s = 0; s < kProjRows; ++s) {
+      const int b = b0 + s * nbl;
+      if (b < nb) emit(b, 2 * p, acc[s].x, acc[s].y);
+    }
   }
 }
 
@@ -196,10 +258,10 @@ struct AppendKParams {
   int tile;                // sequences per item (<= kAppKB)
 };
 
-// One item: head h, sequences [b0, b0 + tile).  A_K[h] and the tile's k[:, h, :]
-// rows are staged in shared memory (`smem`: d*r + kAppKB*d halves); thread =
-// (rank index, lane over the tile's sequences).
-constexpr int kAppKB = 64;
+// One item: head h, sequences [b0, b0 + tile).  A_K[h] ([d][r]) and the
+// tile's k[:, h, :] rows are staged in shared memory (`smem`: d*r + kAppKB*d
+// halves) for the small-product routine; codes are stored as fp16 pairs.
+constexpr int kAppKB = 32;
 
 __device__ __forceinline__ void append_k_item(const AppendKParams& p, int h, int b0, uint8_t* smem) {
   __half* As = reinterpret_cast<__half*>(smem);                 // [d][r]
@@ -214,23 +276,12 @@ __device__ __forceinline__ void append_k_item(const AppendKParams& p, int h, int
         reinterpret_cast<const uint4*>(p.k + (static_cast<size_t>(b0 + b) * p.H + h) * p.d)[c];
   }
   __syncthreads();
-  const int i = tid % p.r;
-  const int bpar = kPrepThreads / p.r;
-  const int bs = tid / p.r;
-  if (bs >= bpar) return;
-  for (int b = bs; b < nb; b += bpar) {
-    const __half* kr = ksm + static_cast<size_t>(b) * p.d;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    for (int j = 0; j < p.d; j += 4) {
-      a0 = fmaf(__half2float(kr[j]), __half2float(As[j * p.r + i]), a0);
-      a1 = fmaf(__half2float(kr[j + 1]), __half2float(As[(j + 1) * p.r + i]), a1);
-      a2 = fmaf(__half2float(kr[j + 2]), __half2float(As[(j + 2) * p.r + i]), a2);
-      a3 = fmaf(__half2float(kr[j + 3]), __half2float(As[(j + 3) * p.r + i]), a3);
-    }
+  small_proj(As, ksm, nb, p.d, p.r, [&](int b, int i, float v0, float v1) {
     const int64_t row = append_row(p.tgt, b0 + b);
-    if (row >= 0) p.k_cache[(row * p.H + h) * p.r + i] = __float2half_rn((a0 + a1) + (a2 + a3));
+    if (row >= 0)
+      *reinterpret_cast<__half2*>(p.k_cache + (row * p.H + h) * p.r + i) = __floats2half2_rn(v0, v1);
     else if (h == 0 && i == 0) append_skipped(p.tgt, row);
-  }
+  });
 }
 
 }  // namespace starkv

@@ -140,12 +140,11 @@ struct AbsorbParams {
 // One item: query head h, sequences [b0, b0 + tile) (tile <= kAbsBT).  Item 0
 // also writes the page prefix sums and resets the status word (every later
 // kernel of the decode runs after this one); all items share setting the
-// segment-max slots to -inf.  Thread = (rank index i, lane over the tile's
-// sequences); its row B_K[g(h)][i][:] is held in registers and the tile's q
-// rows are staged in shared memory (`smem`, tile*D halves).
-constexpr int kAbsBT = 64;
+// segment-max slots to -inf.  B_K[g(h)] is staged transposed ([d][r]) and the
+// tile's q rows as they are, both in shared memory (`smem`: d*r + tile*d
+// halves), for the shared small-product routine.
+constexpr int kAbsBT = 32;
 
-template <int D>
 __device__ __forceinline__ void absorb_item(const AbsorbParams& p, int item, int n_items, int tile, uint8_t* smem) {
   const int h = item % p.H;
   const int bt0 = (item / p.H) * tile;
@@ -198,48 +197,38 @@ __device__ __forceinline__ void absorb_item(const AbsorbParams& p, int item, int
     const int nthr = n_items * 256;
     for (int i = item * 256 + tid; i < p.n_mpart; i += nthr) p.mpart_init[i] = -INFINITY;
   }
-  __half* qs = reinterpret_cast<__half*>(smem);    // [tile][D]
+  const int D = p.d, r = p.r;
+  __half* Ws = reinterpret_cast<__half*>(smem);                 // [d][r]: B_K[g(h)] transposed
+  __half* qs = Ws + static_cast<size_t>(D) * r;                 // [tile][d]
   const int nb = min(tile, p.B - bt0);
-  for (int x = tid; x < nb * (D / 8); x += 256) {
+  const __half* bk = p.B_K + static_cast<size_t>(h >> p.log2G) * r * D;   // [r][d]
+  for (int x = tid; x < r * (D / 8); x += kPrepThreads) {
+    const int i = x % r, jb = x / r;          // consecutive threads: consecutive rank indices
+    const uint4 v = *reinterpret_cast<const uint4*>(bk + static_cast<size_t>(i) * D + jb * 8);
+    const __half* hv = reinterpret_cast<const __half*>(&v);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) Ws[(jb * 8 + u) * r + i] = hv[u];
+  }
+  for (int x = tid; x < nb * (D / 8); x += kPrepThreads) {
     const int bb = x / (D / 8), c = x % (D / 8);
     reinterpret_cast<uint4*>(qs)[x] =
         reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(bt0 + bb) * p.H + h) * D)[c];
   }
   __syncthreads();
   // q~[b,h,i] = coef * sum_j q[b,h,j] * B_K[g(h)][i][j]
-  const int i = tid % p.r;
-  const int bpar = 256 / p.r;
-  const int bs = tid / p.r;
-  if (bs >= bpar) return;
-  uint4 brow[D / 8];
-  const uint4* bsrc = reinterpret_cast<const uint4*>(p.B_K + (static_cast<size_t>(h >> p.log2G) * p.r + i) * D);
-#pragma unroll
-  for (int c = 0; c < D / 8; ++c) brow[c] = bsrc[c];
-  for (int bb = bs; bb < nb; bb += bpar) {
-    const uint4* qrow = reinterpret_cast<const uint4*>(qs + bb * D);
-    float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-      const uint4 qw = qrow[c];
-      const __half2* b2 = reinterpret_cast<const __half2*>(&brow[c]);
-      const __half2* q2 = reinterpret_cast<const __half2*>(&qw);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float2 bf = __half22float2(b2[u]);
-        const float2 qf = __half22float2(q2[u]);
-        a0 = fmaf(qf.x, bf.x, a0);
-        a1 = fmaf(qf.y, bf.y, a1);
-      }
-    }
-    const float v = (a0 + a1) * p.coef;
-    p.qt[(static_cast<size_t>(bt0 + bb) * p.H + h) * p.r + i] = v;
+  small_proj(Ws, qs, nb, D, r, [&](int bb, int i, float v0, float v1) {
+    v0 *= p.coef;
+    v1 *= p.coef;
+    const size_t o = (static_cast<size_t>(bt0 + bb) * p.H + h) * r + i;
+    *reinterpret_cast<float2*>(p.qt + o) = make_float2(v0, v1);
     if (p.qth) {
-      const __half hi = __float2half_rn(v);
-      __half* row = p.qth + (static_cast<size_t>(bt0 + bb) * 2 * p.H + h) * p.r + i;
-      row[0] = hi;
-      row[static_cast<size_t>(p.H) * p.r] = __float2half_rn(v - __half2float(hi));
+      const __half2 hi = __floats2half2_rn(v0, v1);
+      const float2 hf = __half22float2(hi);
+      __half* row = p.qth + (static_cast<size_t>(bt0 + bb) * 2 * p.H + h) * r + i;
+      *reinterpret_cast<__half2*>(row) = hi;
+      *reinterpret_cast<__half2*>(row + static_cast<size_t>(p.H) * r) = __floats2half2_rn(v0 - hf.x, v1 - hf.y);
     }
-  }
+  });
 }
 
 // ======================================================================== prep
@@ -260,8 +249,7 @@ struct PrepParams {
   int a_items, a_tile;     // absorption items (heads x batch tiles of a_tile sequences)
 };
 
-template <int D>
-__global__ void __launch_bounds__(kPrepThreads, 1)
+__global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap vmap, PrepParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -281,7 +269,7 @@ prep_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CU
   }
   x -= p.k_cols;
   const int it = x * KS + blockIdx.y;
-  if (it < p.a_items) absorb_item<D>(p.a, it, p.a_items, p.a_tile, smem);
+  if (it < p.a_items) absorb_item(p.a, it, p.a_items, p.a_tile, smem);
 }
 
 // ======================================================================= kpass
@@ -307,15 +295,6 @@ constexpr int kKConsumers = 256;            // 8 warps of dot products
 constexpr int kKThreads = kKConsumers + 32; // + one producer warp
 
 struct StageMeta { int32_t b, t0, nt, flags; };
-
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;"
-      : "=l"(d)
-      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)),
-        "l"(*reinterpret_cast<uint64_t*>(&c)));
-  return *reinterpret_cast<float2*>(&d);
-}
 
 // First chunk a thread visits, chosen so that the 8 threads sharing a
 // shared-memory wavefront (8 consecutive rows of r*2 bytes, 16-byte reads)
@@ -449,6 +428,7 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
 
   // -------------------------------------------------------------- consumers
   constexpr int kPairsPerPass = kKConsumers / L;
+  constexpr int kRP = CPT <= 4 ? 4 : (CPT <= 8 ? 2 : 1);   // passes held in registers at a time
   const int pair0 = tid / L;
   const int sub = tid % L;
   const int head = pair0 & (p.H - 1);
@@ -487,40 +467,57 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
                                   : make_float2(0.f, 0.f);
       }
     }
+    // The rows of up to kRP passes are copied into registers first; once the
+    // last pass's rows are in registers the stage goes back to the producer,
+    // so the ring refills while the dot products run (a stage is held only
+    // for its shared-memory reads, which keeps more copies in flight).
     const uint8_t* st = ring + static_cast<size_t>(s) * p.stage_bytes;
-    for (int ps = 0; ps < passes; ++ps) {
-      const int pair = ps * kPairsPerPass + pair0;
-      const int t = pair >> p.log2H;     // token within the stage; pair & (H-1) == head
-      const bool valid = t < mt.nt;
-      float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
-      if (valid) {
-        // code row (token t, KV head of this query head); rows are r*2 bytes
-        const uint8_t* row = st + static_cast<size_t>((t << (p.log2H - p.log2G)) + (head >> p.log2G)) * p.r * 2;
+    for (int ps0 = 0; ps0 < passes; ps0 += kRP) {
+      uint4 w[kRP][CPT];
+      int tt[kRP];
 #pragma unroll
-        for (int c = 0; c < CPT; ++c) {
-          const int cc = c + rot < CPT ? c + rot : c + rot - CPT;
-          const int ch = sub * CPT + cc;
-          if (ch < cp) {
-            const uint4 w = *reinterpret_cast<const uint4*>(row + ch * 16);
-            const __half2* h2 = reinterpret_cast<const __half2*>(&w);
+      for (int u = 0; u < kRP; ++u) {
+        const int t = ((ps0 + u) * kPairsPerPass + pair0) >> p.log2H;   // token within the stage
+        tt[u] = (ps0 + u < passes && t < mt.nt) ? t : -1;
+        if (tt[u] >= 0) {
+          // code row (token t, KV head of this query head); rows are r*2 bytes
+          const uint8_t* row = st + static_cast<size_t>((t << (p.log2H - p.log2G)) + (head >> p.log2G)) * p.r * 2;
+#pragma unroll
+          for (int c = 0; c < CPT; ++c) {
+            const int cc = c + rot < CPT ? c + rot : c + rot - CPT;
+            const int ch = sub * CPT + cc;
+            w[u][c] = ch < cp ? *reinterpret_cast<const uint4*>(row + ch * 16) : make_uint4(0, 0, 0, 0);
+          }
+        }
+      }
+      if (ps0 + kRP >= passes) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+#pragma unroll
+      for (int u = 0; u < kRP; ++u) {
+        float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
+        if (tt[u] >= 0) {
+#pragma unroll
+          for (int c = 0; c < CPT; ++c) {
+            const __half2* h2 = reinterpret_cast<const __half2*>(&w[u][c]);
             a0 = ffma2(__half22float2(h2[0]), qv[c * 4 + 0], a0);
             a1 = ffma2(__half22float2(h2[1]), qv[c * 4 + 1], a1);
             a2 = ffma2(__half22float2(h2[2]), qv[c * 4 + 2], a2);
             a3 = ffma2(__half22float2(h2[3]), qv[c * 4 + 3], a3);
           }
         }
-      }
-      float acc = ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
+        float acc = ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
 #pragma unroll
-      for (int o = L / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (valid) {
-        if (sub == 0)
-          st_global_hint(p.logits + (static_cast<size_t>(cur_b) * p.t_pad + mt.t0 + t) * p.H + head, acc, keep);
-        m = fmaxf(m, acc);
+        for (int o = L / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (tt[u] >= 0) {
+          if (sub == 0)
+            st_global_hint(p.logits + (static_cast<size_t>(cur_b) * p.t_pad + mt.t0 + tt[u]) * p.H + head, acc,
+                           keep);
+          m = fmaxf(m, acc);
+        }
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
   }
 }
 
@@ -763,16 +760,22 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         tc_fence_after();
         const uint32_t tbase = tq + static_cast<uint32_t>(ai * p.nmma);
         float o[G];
-#pragma unroll
-        for (int ch = 0; ch < (H + 15) / 16; ++ch) {   // 16 query heads per load
-          uint32_t v[32];
-          tmem_ld_32x32b_x16(tbase + ch * 16, v);
+        if constexpr (H >= 32) {
+          // all loads of the row's H columns in flight before a single wait
+          uint32_t v0[32], v1[32];
+          tmem_ld_32x32b_x32(tbase, v0);
+          if constexpr (H == 64) tmem_ld_32x32b_x32(tbase + 32, v1);
           tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int col = ch * 16 + c;
-            if (col < H && (col / G) == j) o[col % G] = __uint_as_float(v[c]);
-          }
+          for (int col = 0; col < H; ++col)
+            if ((col / G) == j) o[col % G] = __uint_as_float(col < 32 ? v0[col] : v1[col - 32]);
+        } else {
+          uint32_t v[32];
+          tmem_ld_32x32b_x16(tbase, v);             // H <= 16 heads: one 16-column load
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            if (c < H && (c / G) == j) o[c % G] = __uint_as_float(v[c]);
         }
         tc_fence_before();
         __syncwarp();
@@ -1356,16 +1359,27 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
   }
   tc_fence_before();
   cluster.sync();
+  // rank ks sums rows [ks*npad/KS, (ks+1)*npad/KS) over the cluster in rank
+  // order, four consecutive outputs per thread (all ranks' loads issued first)
   const int per = (p.npad + KS - 1) / KS;
   const int n_lo = ks * per, n_hi = min(p.npad, n_lo + per);
-  for (int x = tid; x < (n_hi - n_lo) * 128; x += kFinThreads) {
-    const int n = n_lo + x / 128, m = x % 128;
-    const int b = b0 + n;
+  for (int x = tid; x < (n_hi - n_lo) * 32; x += kFinThreads) {
+    const int n = n_lo + x / 32, m = (x % 32) * 4;
     const int dm = mt * 128 + m;
     if (n >= nb || dm >= p.d) continue;
-    float acc = 0.f;
-    for (int c = 0; c < KS; ++c) acc += cluster.map_shared_rank(part, c)[n * 128 + m];
-    p.out[(static_cast<size_t>(b) * p.H + h) * p.d + dm] = __float2half_rn(acc);
+    float4 v[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      if (c < KS) v[c] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(part, c) + n * 128 + m);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      if (c < KS) { acc.x += v[c].x; acc.y += v[c].y; acc.z += v[c].z; acc.w += v[c].w; }
+    const __half2 lo = __floats2half2_rn(acc.x, acc.y), hi = __floats2half2_rn(acc.z, acc.w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(p.out + (static_cast<size_t>(b0 + n) * p.H + h) * p.d + dm) = pk;
   }
   cluster.sync();
   if (warp == 1) {

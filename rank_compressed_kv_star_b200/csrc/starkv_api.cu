@@ -569,7 +569,7 @@ starkv_status plan_append(const starkv_layer_desc* desc, int32_t batch, const vo
   ap->v_cols = ap->v_mt * n_bt;
   const int sms = device_sm_count();
   int KS = 1;
-  while (KS < 8 && ap->v_cols * KS * 2 <= sms && (HD / kAppKC) >= KS * 2) KS *= 2;
+  while (KS < 8 && ap->v_cols * KS * 2 <= 2 * sms && (HD / kAppKC) >= KS * 2) KS *= 2;   // <= one wave at 2 CTAs/SM
   ap->KS = KS;
   AppendVParams& vp = ap->vp;
   vp.tgt = tgt;
@@ -594,29 +594,21 @@ starkv_status plan_append(const starkv_layer_desc* desc, int32_t batch, const vo
   return STARKV_OK;
 }
 
-extern "C++" {
-template <int D>
-cudaError_t launch_prep_d(const PrepParams& pp, const CUtensorMap& amap, const CUtensorMap& vmap, dim3 grid,
-                          size_t smem, int KS, cudaStream_t s) {
-  if (!set_smem(prep_kernel<D>, smem)) return cudaErrorInvalidValue;
-  return launch(prep_kernel<D>, grid, dim3(kPrepThreads), smem, s, KS, amap, vmap, pp);
-}
-}
-
 // One prep launch: the append roles of `app` (null: none) and the query
-// absorption `abs` (null: none) over `batch` rows.  Small items are sized so
-// that the grid stays within about one CTA per SM.
+// absorption `abs` (null: none) over `batch` rows.  Item tiles of 16 rows are
+// used when they keep the grid within one wave of two CTAs per SM, else 32.
 starkv_status launch_prep(int d, const AppendPlan* app, const AbsorbParams* abs, int batch, cudaStream_t s) {
   PrepParams pp;
   std::memset(&pp, 0, sizeof(pp));
   const int KS = app ? app->KS : 1;
   const int sms = device_sm_count();
   const int v_ctas = app ? app->v_cols * KS : 0;
-  const int spare = sms - v_ctas > 2 * KS ? sms - v_ctas : 2 * KS;
+  const int spare = 2 * sms - v_ctas > 2 * KS ? 2 * sms - v_ctas : 2 * KS;
   const int k_heads = app ? app->kp.H : 0;
   const int a_heads = abs ? abs->H : 0;
+  const int r = app ? app->kp.r : abs->r;
   int tile = 16;
-  while (tile < kAbsBT && (k_heads + a_heads) * ((batch + tile - 1) / tile) > spare) tile *= 2;
+  if ((k_heads + a_heads) * ((batch + tile - 1) / tile) > spare) tile = kAbsBT;
   size_t smem = 0;
   CUtensorMap none;
   std::memset(&none, 0, sizeof(none));
@@ -634,19 +626,16 @@ starkv_status launch_prep(int d, const AppendPlan* app, const AbsorbParams* abs,
     pp.a = *abs;
     pp.a_tile = tile;
     pp.a_items = a_heads * ((batch + tile - 1) / tile);
-    const size_t qs = static_cast<size_t>(tile) * d * 2;
-    if (qs > smem) smem = qs;
+    const size_t ws = (static_cast<size_t>(d) * r + static_cast<size_t>(tile) * d) * 2;   // B_K^T + q rows
+    if (ws > smem) smem = ws;
   }
   smem += 1024;   // room to align the dynamic shared memory to 1024 bytes
   const dim3 grid(pp.v_cols + pp.k_cols + (pp.a_items + KS - 1) / KS, KS);
   const CUtensorMap& amap = app ? app->amap : none;
   const CUtensorMap& vmap = app ? app->vmap : none;
-  cudaError_t e;
-  if (d == 32) e = launch_prep_d<32>(pp, amap, vmap, grid, smem, KS, s);
-  else if (d == 64) e = launch_prep_d<64>(pp, amap, vmap, grid, smem, KS, s);
-  else if (d == 128) e = launch_prep_d<128>(pp, amap, vmap, grid, smem, KS, s);
-  else e = launch_prep_d<256>(pp, amap, vmap, grid, smem, KS, s);
-  return e == cudaSuccess ? STARKV_OK : STARKV_ERR_CUDA;
+  if (!set_smem(prep_kernel, smem)) return STARKV_ERR_CUDA;
+  return launch(prep_kernel, grid, dim3(kPrepThreads), smem, s, KS, amap, vmap, pp) == cudaSuccess ? STARKV_OK
+                                                                                                   : STARKV_ERR_CUDA;
 }
 
 // Compress rows of k, v and store their codes at the target rows (see AppendTarget).
