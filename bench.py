@@ -538,7 +538,7 @@ def run_prefill(args):
     qd, kd, vd, sd = dev(q), dev(kx), dev(vx), dev(slots)
     st_d, of_d = dev(starts.astype(np.int32)), dev(offs)
     max_len = int(T.max())
-    wsb = S.starkv_prefill_workspace_bytes(desc, n_rows, max_len)
+    wsb = S.starkv_prefill_workspace_bytes(desc, B, n_rows, max_len)
     ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
     out = torch.empty((n_rows, H, d), dtype=torch.float16, device="cuda")
     stream = torch.cuda.current_stream()

@@ -247,15 +247,21 @@ starkv_status starkv_append_decode_host(const starkv_layer_desc* desc, int32_t b
  *   starts        int32 [n_seqs] (device): position of each chunk's first token
  *   row_offsets   int32 [n_seqs + 1] (device): first row of each chunk,
  *                 non-decreasing from 0 to n_rows
- *   workspace     at least starkv_prefill_workspace_bytes(desc, n_rows,
+ *   workspace     at least starkv_prefill_workspace_bytes(desc, n_seqs, n_rows,
  *                 max_seq_len) bytes, 256-byte aligned
  *   out           fp16 [n_rows][H][d]
  *
- * Every row is evaluated as one decode row (its own length, the sequence's
- * block table), so a chunk's rows read the sequence's pages once per row:
- * cost grows with rows x context.  Errors as starkv_paged_decode.
+ * When the KV heads come in groups of 8 and H / Hkv <= 16, a chunk is read
+ * once: its rows are taken nq = 16 / (H / Hkv) at a time, and each group of
+ * nq rows streams the sequence's K and V pages once for all of its rows (the
+ * rows' query heads act as nq x H query heads with per-row causal limits).
+ * Other shapes evaluate every row as one decode row (its own length, the
+ * sequence's block table), reading the pages once per row.  The workspace
+ * holds logits of every virtual head: it grows with (n_rows / nq + n_seqs) x
+ * max_seq_len x H x nq.  Errors as starkv_paged_decode.
  */
-size_t starkv_prefill_workspace_bytes(const starkv_layer_desc* desc, int32_t n_rows, int32_t max_seq_len);
+size_t starkv_prefill_workspace_bytes(const starkv_layer_desc* desc, int32_t n_seqs, int32_t n_rows,
+                                      int32_t max_seq_len);
 starkv_status starkv_paged_prefill(const starkv_layer_desc* desc, int32_t n_seqs, int32_t n_rows,
                                    int32_t max_seq_len, const void* q, const void* B_K, const void* B_V,
                                    const void* k_cache, const void* v_cache, const int32_t* block_tables,

@@ -100,7 +100,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                                  P, SZ, P, P, ctypes.POINTER(P)]
     lib.starkv_paged_decode_profiled.restype = ctypes.c_int
     lib.starkv_paged_decode_static.argtypes = [DP, I32, I32, P, P, P, P, P, P, P, ctypes.c_float, P, P]
-    lib.starkv_prefill_workspace_bytes.argtypes = [DP, I32, I32]
+    lib.starkv_prefill_workspace_bytes.argtypes = [DP, I32, I32, I32]
     lib.starkv_prefill_workspace_bytes.restype = ctypes.c_size_t
     lib.starkv_paged_prefill.argtypes = [DP, I32, I32, I32, P, P, P, P, P, P, P, P, ctypes.c_float, P,
                                          ctypes.c_size_t, P, P]
@@ -231,8 +231,8 @@ def starkv_append_decode_host(desc: LayerDesc, batch: int, max_seq_len: int, k_h
     return st
 
 
-def starkv_prefill_workspace_bytes(desc: LayerDesc, n_rows: int, max_seq_len: int) -> int:
-    return int(load_library().starkv_prefill_workspace_bytes(_desc_ref(desc), n_rows, max_seq_len))
+def starkv_prefill_workspace_bytes(desc: LayerDesc, n_seqs: int, n_rows: int, max_seq_len: int) -> int:
+    return int(load_library().starkv_prefill_workspace_bytes(_desc_ref(desc), n_seqs, n_rows, max_seq_len))
 
 
 def starkv_paged_prefill(desc: LayerDesc, n_seqs: int, n_rows: int, max_seq_len: int, q, B_K, B_V,

@@ -120,6 +120,77 @@ __global__ void __launch_bounds__(256) prefill_rows_kernel(PrefillRowsParams p) 
   p.row_len[r] = p.starts[lo] + (r - p.row_offsets[lo]) + 1;
 }
 
+// ================================================================ chunk table
+// Read-once chunked prefill: the rows of a sequence's chunk are taken nq at a
+// time as one virtual sequence whose query heads are the virtual heads
+// (h, i) = query head h of the chunk's row i.  Virtual sequence v covers rows
+// vs_row0[v] .. + vs_nrows[v] - 1 (consecutive positions starting at
+// vs_len[v] - vs_nrows[v]) and attends over tokens [0, vs_len[v]): row i over
+// tokens [0, vs_len[v] - vs_nrows[v] + i] (causal).  Entries past the last
+// virtual sequence get zero rows and zero length.
+struct ChunkTableParams {
+  const int32_t* starts;       // [n_seqs] position of each chunk's first token
+  const int32_t* row_offsets;  // [n_seqs + 1] first row of each sequence's chunk
+  int32_t* vs_seq;             // [nv_max] sequence (block-table row) of each virtual sequence
+  int32_t* vs_row0;            // [nv_max]
+  int32_t* vs_nrows;           // [nv_max]
+  int32_t* vs_len;             // [nv_max]
+  int n_seqs, nv_max, log2nq;
+};
+
+// one CTA of 256 threads: per-sequence counts, a block-wide scan, the entries
+__global__ void __launch_bounds__(256) chunk_table_kernel(ChunkTableParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
+  __shared__ int32_t part[16];
+  __shared__ int32_t total;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nq = 1 << p.log2nq;
+  const int per = (p.n_seqs + 255) / 256;
+  const int b0 = tid * per;
+  int32_t s = 0;
+  for (int b = b0; b < b0 + per && b < p.n_seqs; ++b) {
+    const int32_t c = p.row_offsets[b + 1] - p.row_offsets[b];
+    s += c > 0 ? (c + nq - 1) >> p.log2nq : 0;
+  }
+  int32_t v = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
+  }
+  if (lane == 31) part[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = lane < 8 ? part[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < 8) part[8 + lane] = w;
+    if (lane == 7) total = w;
+  }
+  __syncthreads();
+  int32_t at = v - s + (warp > 0 ? part[8 + warp - 1] : 0);
+  for (int b = b0; b < b0 + per && b < p.n_seqs; ++b) {
+    const int32_t r0 = p.row_offsets[b], c = p.row_offsets[b + 1] - r0;
+    for (int32_t js = 0; js * nq < c && at < p.nv_max; ++js, ++at) {
+      const int32_t n = min(nq, c - js * nq);
+      p.vs_seq[at] = b;
+      p.vs_row0[at] = r0 + js * nq;
+      p.vs_nrows[at] = n;
+      p.vs_len[at] = p.starts[b] + js * nq + n;
+    }
+  }
+  for (int32_t e = total + tid; e < p.nv_max; e += 256) {
+    p.vs_seq[e] = 0;
+    p.vs_row0[e] = 0;
+    p.vs_nrows[e] = 0;
+    p.vs_len[e] = 0;
+  }
+}
+
 // ====================================================================== absorb
 struct AbsorbParams {
   const __half* q;        // [B][H][d]
@@ -135,6 +206,12 @@ struct AbsorbParams {
   int B, H, d, r, cap;    // cap = min(max_seq_len, max_blocks_per_seq*16)
   int log2G;              // query heads per KV head = 1 << log2G
   float coef;             // scale * log2(e)
+  // chunked prefill read once (null vs_row0: decode rows): B counts virtual
+  // sequences of 1 << log2nq query rows each, seq_lens are their lengths, and
+  // qth is laid out [B][2][H << log2nq][r] with virtual head h * nq + i
+  const int32_t* vs_row0; // [B] first query row of each virtual sequence
+  const int32_t* vs_nrows;// [B] its rows (0: unused entry)
+  int log2nq;
 };
 
 // One item: query head h, sequences [b0, b0 + tile) (tile <= kAbsBT).  Item 0
@@ -200,7 +277,9 @@ __device__ __forceinline__ void absorb_item(const AbsorbParams& p, int item, int
   const int D = p.d, r = p.r;
   __half* Ws = reinterpret_cast<__half*>(smem);                 // [d][r]: B_K[g(h)] transposed
   __half* qs = Ws + static_cast<size_t>(D) * r;                 // [tile][d]
-  const int nb = min(tile, p.B - bt0);
+  // rows of the item: sequences, or (virtual sequence, row) pairs in chunk mode
+  const int n_rows_all = p.vs_row0 ? (p.B << p.log2nq) : p.B;
+  const int nb = min(tile, n_rows_all - bt0);
   const __half* bk = p.B_K + static_cast<size_t>(h >> p.log2G) * r * D;   // [r][d]
   for (int x = tid; x < r * (D / 8); x += kPrepThreads) {
     const int i = x % r, jb = x / r;          // consecutive threads: consecutive rank indices
@@ -211,14 +290,31 @@ __device__ __forceinline__ void absorb_item(const AbsorbParams& p, int item, int
   }
   for (int x = tid; x < nb * (D / 8); x += kPrepThreads) {
     const int bb = x / (D / 8), c = x % (D / 8);
+    int64_t qrow = bt0 + bb;
+    if (p.vs_row0) {   // row i of virtual sequence v, or a zero row past its chunk
+      const int v = (bt0 + bb) >> p.log2nq, i = (bt0 + bb) & ((1 << p.log2nq) - 1);
+      qrow = i < p.vs_nrows[v] ? static_cast<int64_t>(p.vs_row0[v]) + i : -1;
+    }
     reinterpret_cast<uint4*>(qs)[x] =
-        reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(bt0 + bb) * p.H + h) * D)[c];
+        qrow >= 0 ? reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(qrow) * p.H + h) * D)[c]
+                  : make_uint4(0, 0, 0, 0);
   }
   __syncthreads();
   // q~[b,h,i] = coef * sum_j q[b,h,j] * B_K[g(h)][i][j]
   small_proj(Ws, qs, nb, D, r, [&](int bb, int i, float v0, float v1) {
     v0 *= p.coef;
     v1 *= p.coef;
+    if (p.vs_row0) {
+      // B-operand rows of the read-once K pass: virtual head h * nq + row, hi then lo block
+      const int vr = bt0 + bb, v = vr >> p.log2nq, row = vr & ((1 << p.log2nq) - 1);
+      const size_t hv = static_cast<size_t>(p.H) << p.log2nq;
+      const __half2 hi = __floats2half2_rn(v0, v1);
+      const float2 hf = __half22float2(hi);
+      __half* dst = p.qth + (static_cast<size_t>(v) * 2 * hv + (static_cast<size_t>(h) << p.log2nq) + row) * r + i;
+      *reinterpret_cast<__half2*>(dst) = hi;
+      *reinterpret_cast<__half2*>(dst + hv * r) = __floats2half2_rn(v0 - hf.x, v1 - hf.y);
+      return;
+    }
     const size_t o = (static_cast<size_t>(bt0 + bb) * p.H + h) * r + i;
     *reinterpret_cast<float2*>(p.qt + o) = make_float2(v0, v1);
     if (p.qth) {
@@ -818,6 +914,278 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   }
 }
 
+// ============================================================ kpass (chunks)
+// Read-once K pass of a chunked prefill on tcgen05.  The virtual heads (h, i)
+// of a virtual sequence (query head h of its chunk row i) that share KV head
+// g(h) share its K codes, so with 16 virtual heads per KV head (G query heads
+// x nq rows) a tile is one page of a group of 8 KV heads (row 8 t + j: token
+// t, KV head j of the group), one 3-D TMA box {64 codes, 8 heads, 16 tokens}
+// per 64 codes, and B holds the 128 virtual heads of the group (rows: fp16
+// high parts, then the low parts), loaded once per (segment, group).  A CTA
+// walks each virtual sequence of its page range once per group, so every K
+// page is read once in total.  An epilogue warp owns four tokens of the tile
+// (32 rows, all 8 KV heads): four 32-column TMEM loads per tile, each lane
+// keeps its KV head's 16 columns, sets logits past a row's causal limit to
+// -inf, stores the 16 as consecutive logits and keeps running maxima that are
+// merged into the segment slots (float max) at the end of each pass.
+struct KPassChunkParams {
+  const int32_t* tables;      // [n_seqs][MB]
+  const int32_t* vs_seq;      // [B] sequence of each virtual sequence
+  const int32_t* vs_nrows;    // [B] rows of each virtual sequence
+  const int32_t* teff;        // [B] lengths
+  const int32_t* prefix;      // [B+1]
+  float* logits;              // [B][n_vg][t_pad][lw]
+  float* mpart;               // [k_slots][Hv], -inf on entry
+  int32_t* status;
+  int B, MB, NB, t_pad;
+  int Hv, n_vg, log2lw;       // virtual heads, groups of lw = min(256, Hv) of them
+  int n_groups;               // KV-head groups of 8
+  int log2nq;
+  int ksteps, kb;             // UMMA K steps of 16 codes; 64-code column blocks
+  int nacc, nbs, stages;
+  uint32_t a_bytes;           // kb * 16 KiB
+  uint32_t b_bytes;           // kb * 256 rows * 128 B
+  uint32_t tmem_cols;
+  int drop_stage;             // test hook (-1: off)
+};
+
+constexpr int kKChunkCols = 128;   // virtual heads of a KV-head group (8 x 16): UMMA N
+
+// Calls f(v, pg, nt, g, first, last) for the tiles of pages [p0, p1): page pg
+// (tokens [16 pg, 16 pg + nt)) of virtual sequence v for KV-head group g,
+// each (v, g) pass over the CTA's pages of v in page order, `first` / `last`
+// on the pass's first and final tile.  Stops when f returns false.
+template <typename F>
+__device__ __forceinline__ void for_each_chunk_tile(const KPassChunkParams& p, int64_t p0, int64_t p1, F&& f) {
+  int32_t v = seq_of_page(p.prefix, p.B, p0);
+  int64_t x = p0;
+  while (x < p1) {
+    while (p.prefix[v + 1] <= x) ++v;
+    const int64_t seg_end = min(p1, static_cast<int64_t>(p.prefix[v + 1]));
+    const int32_t base = p.prefix[v];
+    const int32_t T = p.teff[v];
+    for (int g = 0; g < p.n_groups; ++g)
+      for (int64_t y = x; y < seg_end; ++y) {
+        const int32_t pg = static_cast<int32_t>(y - base);
+        if (!f(v, pg, min(kBlock, T - pg * kBlock), g, y == x, y == seg_end - 1)) return;
+      }
+    x = seg_end;
+  }
+}
+
+__global__ void __launch_bounds__(kKTCThreads, 1)
+kpass_chunk_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                   KPassChunkParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages;
+  uint8_t* bslot = smem + static_cast<size_t>(S) * p.a_bytes;                    // [nbs] query tiles
+  uint64_t* full = reinterpret_cast<uint64_t*>(bslot + p.nbs * static_cast<size_t>(p.b_bytes));
+  uint64_t* empty = full + S;
+  uint64_t* bfull = empty + S;
+  uint64_t* bempty = bfull + 2;
+  uint64_t* tfull = bempty + 2;
+  uint64_t* tempty = tfull + kKTCMaxAcc;
+  uint64_t* mmadone = tempty + kKTCMaxAcc;
+  __shared__ uint32_t taddr_s;
+  __shared__ volatile int32_t abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&bfull[a], 1); mbar_init(&bempty[a], 1); }
+    for (int a = 0; a < kKTCMaxAcc; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
+    mbar_init(mmadone, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  griddep_wait();
+  griddep_launch_dependents();
+  Partition pt;
+  pt.P = p.prefix[p.B];
+  pt.G = static_cast<int32_t>(pt.P < gridDim.x ? pt.P : gridDim.x);
+  const int cta = blockIdx.x;
+  if (cta >= pt.G) return;   // uniform over the CTA
+  if (warp == 1) {
+    tmem_alloc(&taddr_s, p.tmem_cols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t taddr = taddr_s;
+  const int64_t p0 = part_begin(cta, pt), p1 = part_begin(cta + 1, pt);
+  const int nq1 = (1 << p.log2nq) - 1;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&kmap);
+      prefetch_tensormap(&qmap);
+      const uint64_t stream = policy_evict_first();
+      const uint64_t reuse = policy_evict_last();
+      int si = 0, bi = 0;
+      uint32_t su = 0, bu = 0, issued = 0;
+      int32_t bpar[2] = {-1, -1};
+      bool ok = true;
+      for_each_chunk_tile(p, p0, p1, [&](int32_t v, int32_t pg, int32_t, int g, bool first, bool last) {
+        if (first) {
+          if (bu > 0 && !mbar_wait(&bempty[bi], (bu - 1) & 1)) { ok = false; return false; }
+          bpar[bi] = static_cast<int32_t>(bu & 1);
+          mbar_arrive_expect_tx(&bfull[bi], p.b_bytes);
+          const int hi_row = v * 2 * p.Hv + g * kKChunkCols;
+          for (int a = 0; a < p.kb; ++a) {
+            uint8_t* dst = bslot + bi * static_cast<size_t>(p.b_bytes) + static_cast<size_t>(a) * 256 * 128;
+            tma_load_2d(dst, &qmap, a * 64, hi_row, &bfull[bi], reuse);
+            tma_load_2d(dst + kKChunkCols * 128, &qmap, a * 64, hi_row + p.Hv, &bfull[bi], reuse);
+          }
+        }
+        if (su > 0 && !mbar_wait(&empty[si], (su - 1) & 1)) { ok = false; return false; }
+        uint8_t* st = smem + static_cast<size_t>(si) * p.a_bytes;
+        const bool drop = static_cast<int>(issued) == p.drop_stage;
+        if (!drop) {
+          mbar_arrive_expect_tx(&full[si], static_cast<uint32_t>(p.kb) * 16384u);
+          int32_t phys = table_row(p.tables, p.vs_seq, v, p.MB)[pg];
+          if (phys < 0 || phys >= p.NB) { set_flag(p.status, STARKV_FLAG_BAD_BLOCK_ID); phys = 0; }
+          for (int a = 0; a < p.kb; ++a)
+            tma_load_3d(st + static_cast<size_t>(a) * 16384, &kmap, a * 64, g * 8, phys * kBlock, &full[si], stream);
+        }
+        ++issued;
+        if (++si == S) { si = 0; ++su; }
+        if (last && ++bi == p.nbs) { bi = 0; ++bu; }
+        return true;
+      });
+      if (!ok) {
+        set_timeout(p.status, kSiteKEmpty);
+        abort_flag = 1;
+      }
+      int i = si;
+      uint32_t u = su;
+      for (uint32_t n = 0; n < issued && n < static_cast<uint32_t>(S); ++n) {
+        if (--i < 0) { i = S - 1; --u; }
+        mbar_wait(&full[i], u & 1);
+      }
+      for (int a = 0; a < 2; ++a)
+        if (bpar[a] >= 0) mbar_wait(&bfull[a], static_cast<uint32_t>(bpar[a]));
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16_f32(128, kKChunkCols, /*a_mn_major=*/false, /*b_mn_major=*/false);
+      const uint32_t b_atom = 256u * 8u;    // one 64-code block of B: 256 rows * 128 bytes >> 4
+      int si = 0, bi = 0, ai = 0;
+      uint32_t su = 0, bu = 0, au = 0;
+      bool ok = true;
+      for_each_chunk_tile(p, p0, p1, [&](int32_t, int32_t, int32_t, int, bool, bool last) {
+        if (!mbar_wait(&bfull[bi], bu & 1)) { ok = false; return false; }
+        if (au > 0 && !mbar_wait(&tempty[ai], (au - 1) & 1)) { ok = false; return false; }
+        if (!mbar_wait(&full[si], su & 1) || abort_flag) { ok = false; return false; }
+        tc_fence_after();
+        const uint64_t da = smem_desc(smem_u32(smem + static_cast<size_t>(si) * p.a_bytes), 16u, 1024u, kSwizzle128B);
+        const uint64_t db = smem_desc(smem_u32(bslot + bi * static_cast<size_t>(p.b_bytes)), 16u, 1024u, kSwizzle128B);
+        const uint32_t d = taddr + static_cast<uint32_t>(ai * kKChunkCols);
+        for (int ks = 0; ks < p.ksteps; ++ks) {
+          const uint32_t a = ks >> 2, kk = ks & 3;
+          const uint64_t dak = da + (a * 1024u + kk * 2u), dbk = db + (a * b_atom + kk * 2u);
+          umma_f16_ss(d, dak, dbk, idesc, ks > 0 ? 1u : 0u);                           // high parts
+          umma_f16_ss(d, dak, dbk + static_cast<uint32_t>(kKChunkCols) * 8u, idesc, 1u);  // low parts
+        }
+        umma_commit(&empty[si]);
+        umma_commit(&tfull[ai]);
+        if (++ai == p.nacc) { ai = 0; ++au; }
+        if (last) {
+          umma_commit(&bempty[bi]);
+          if (++bi == p.nbs) { bi = 0; ++bu; }
+        }
+        if (++si == S) { si = 0; ++su; }
+        return true;
+      });
+      if (!ok) { set_timeout(p.status, kSiteKFull); abort_flag = 1; }
+      umma_commit(mmadone);
+      mbar_wait(mmadone, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // warp quarter q holds rows 32q..32q+31: tokens 4q..4q+3, all 8 KV heads;
+    // lane L: token 4q + L/8, KV head L % 8 of the group (columns 16 j .. 16 j + 15)
+    const int q = warp & 3;
+    const int jl = lane & 7;
+    const int t = 4 * q + (lane >> 3);
+    const uint64_t keep = policy_evict_last();       // logits: read back by the V pass
+    const uint32_t tq = taddr + (static_cast<uint32_t>(q * 32) << 16);
+    float m[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) m[c] = -INFINITY;
+    int ai = 0;
+    uint32_t au = 0;
+    bool ok = true;
+    for_each_chunk_tile(p, p0, p1, [&](int32_t v, int32_t pg, int32_t nt, int g, bool, bool last) {
+      const bool ready = mbar_wait(&tfull[ai], au & 1);
+      if (!__all_sync(0xffffffffu, ready && !abort_flag)) { ok = false; return false; }
+      tc_fence_after();
+      float xs[16];
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {   // columns 32 c4 .. 32 c4 + 31: KV heads 2 c4, 2 c4 + 1
+        uint32_t w[32];
+        tmem_ld_32x32b_x32(tq + static_cast<uint32_t>(ai * kKChunkCols + 32 * c4), w);
+        tmem_ld_wait();
+        if ((jl >> 1) == c4) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) xs[c] = __uint_as_float((jl & 1) ? w[16 + c] : w[c]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[ai]);
+      if (++ai == p.nacc) { ai = 0; ++au; }
+      const int kv = g * 8 + jl;                     // KV head of this lane's row
+      if (t < nt) {
+        const int32_t tabs = pg * kBlock + t;
+        const int32_t nrows = p.vs_nrows[v];
+        const int32_t rel = tabs - (p.teff[v] - nrows);   // rows i >= rel see this token
+        float o[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int i = c & nq1;
+          o[c] = (i < nrows && i >= rel) ? xs[c] : -INFINITY;
+          m[c] = fmaxf(m[c], o[c]);
+        }
+        const int vh = kv * 16;                       // 16 consecutive virtual heads, in one group
+        const size_t lrow_idx = (static_cast<size_t>(v) * p.n_vg + (vh >> p.log2lw)) * p.t_pad + tabs;
+        float* lrow = p.logits + (lrow_idx << p.log2lw) + (vh & ((1 << p.log2lw) - 1));
+#pragma unroll
+        for (int c = 0; c < 16; c += 4)
+          st_global_hint(reinterpret_cast<float4*>(lrow + c), make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]), keep);
+      }
+      if (last) {
+        // the maxima of this (segment, group) pass: over the warp's 4 tokens (lanes jl, jl+8, jl+16, jl+24)
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          float x = m[c];
+          x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
+          x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
+          m[c] = x;
+        }
+        if (lane < 8) {
+          float* mp = p.mpart + static_cast<size_t>(v + cta) * p.Hv + kv * 16;
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            if (m[c] > -INFINITY) atomic_max_f32(mp + c, m[c]);
+        }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) m[c] = -INFINITY;
+      }
+      return true;
+    });
+    if (!ok) set_timeout(p.status, kSiteKFull);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(taddr, p.tmem_cols);
+  }
+}
+
 // ======================================================================= vpass
 // Z^T (R-range rows x heads) += C_V^T (R-range x 16 tokens) . P^T (16 x heads)
 // per page, with A = the V page slice as an MN-major 128B-swizzled operand
@@ -843,11 +1211,18 @@ struct VPassParams {
   uint32_t vtile_bytes;   // r_range_pad*16*2
   uint32_t ltile_bytes;   // 16*H*4
   uint32_t ptile_bytes;   // npad*16*2
+  // read-once chunked prefill (vpass_kernel<true>): B counts virtual sequences,
+  // logits are [B][n_vg][t_pad][256], the columns are virtual heads h * nq + i
+  // (Hv of them, 256 per group: grid y = R range + n_rr * group), and the
+  // partials of virtual head (h, i) sit at row (slot * nq + i) of head h
+  int Hv, n_vg, log2nq;
+  int lw;                 // chunk mode: logits row width = virtual heads per group (npad)
 };
 
 constexpr int kVThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 weights + epilogue
 constexpr int32_t kFirst = 1, kLast = 2;
 
+template <bool kChunk>
 __global__ void __launch_bounds__(kVThreads, 1)
 vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -879,7 +1254,8 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
   ptk.P = pt.P;
   ptk.G = static_cast<int32_t>(pt.P < p.k_grid ? pt.P : p.k_grid);
   const int cta = blockIdx.x;
-  const int rr = blockIdx.y;
+  const int rr = kChunk ? static_cast<int>(blockIdx.y) % p.n_rr : static_cast<int>(blockIdx.y);
+  const int vg = kChunk ? static_cast<int>(blockIdx.y) / p.n_rr : 0;   // group of virtual heads (chunk mode)
   if (cta >= pt.G) return;  // uniform across the CTA: nothing allocated yet
 
   if (tid == 0) {
@@ -948,9 +1324,10 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
           // the page's R range in one box of n_chunks 64-code blocks
           tma_load_3d(vtiles + static_cast<size_t>(s) * p.vtile_bytes, &vmap, 0, phys * kBlock, c_base, &full[s],
                       pol_codes);
-          bulk_g2s(ltiles + static_cast<size_t>(s) * p.ltile_bytes,
-                   p.logits + (static_cast<size_t>(b) * p.t_pad + pg * kBlock) * p.H, p.ltile_bytes,
-                   &full[s], pol_logits);
+          const float* lsrc =
+              kChunk ? p.logits + ((static_cast<size_t>(b) * p.n_vg + vg) * p.t_pad + pg * kBlock) * p.lw
+                     : p.logits + (static_cast<size_t>(b) * p.t_pad + pg * kBlock) * p.H;
+          bulk_g2s(ltiles + static_cast<size_t>(s) * p.ltile_bytes, lsrc, p.ltile_bytes, &full[s], pol_logits);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -1013,6 +1390,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
     const int t_w0 = et / p.npad;
     const int t_step = 128 / p.npad;
     float lsum = 0.f;
+    float lsum2[2] = {0.f, 0.f};           // chunk mode: columns et and et + 128
     uint32_t seg = 0, pphase = 0;
     const uint64_t keep = policy_evict_last();   // Z partials: read back by the finish kernel
     for (uint32_t k = 0;; ++k) {
@@ -1034,7 +1412,13 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
         const int32_t i0 = part_owner(f0, ptk), i1 = part_owner(f1 - 1, ptk);
         for (int h = et; h < p.npad; h += 128) {
           float M = 0.f;
-          if (h < p.H) {
+          if constexpr (kChunk) {
+            const int col = vg * p.lw + h;
+            if (col < p.Hv) {
+              M = -INFINITY;   // stays -inf for a virtual head with no visible token (weights 0)
+              for (int32_t i = i0; i <= i1; ++i) M = fmaxf(M, p.mpart[static_cast<size_t>(mt.b + i) * p.Hv + col]);
+            }
+          } else if (h < p.H) {
             M = -INFINITY;
             for (int32_t i = i0; i <= i1; ++i) M = fmaxf(M, p.mpart[static_cast<size_t>(mt.b + i) * p.H + h]);
           }
@@ -1042,19 +1426,46 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
         }
         if (!group_sync(pbar, pphase)) { set_timeout(p.status, kSiteVFull); abort_flag = 1; break; }
         lsum = 0.f;
+        lsum2[0] = lsum2[1] = 0.f;
       }
       const float* lt = reinterpret_cast<const float*>(ltiles + static_cast<size_t>(s) * p.ltile_bytes);
       uint8_t* pt_s = ptiles + static_cast<size_t>(s) * p.ptile_bytes;
-      const float m_h = sM[h_w];
-      for (int t = t_w0; t < kBlock; t += t_step) {
-        // unnormalised weight exp2(s - M) <= 1, rounded to fp16 for the MMA; the
-        // normaliser sums exactly the rounded weights
-        __half w = __float2half_rn(0.f);
-        if (t < mt.nt && h_w < p.H) w = __float2half_rn(exp2f(lt[t * p.H + h_w] - m_h));
-        lsum += __half2float(w);
-        const uint32_t off = static_cast<uint32_t>(t >> 3) * lbo_b + static_cast<uint32_t>(h_w >> 3) * 128u +
-                             static_cast<uint32_t>(h_w & 7) * 16u + static_cast<uint32_t>(t & 7) * 2u;
-        *reinterpret_cast<__half*>(pt_s + off) = w;
+      if constexpr (kChunk) {
+        // columns et and et + 128, all 16 tokens; a logit of -inf (past a row's
+        // causal limit, or a virtual head with no row) weighs exactly 0
+#pragma unroll
+        for (int k2 = 0; k2 < 2; ++k2) {
+          const int col = et + 128 * k2;
+          if (col < p.npad) {
+            const float mh = sM[col];
+            const bool live = vg * p.lw + col < p.Hv;
+            float acc = 0.f;
+            for (int t = 0; t < kBlock; ++t) {
+              __half w = __float2half_rn(0.f);
+              if (live && t < mt.nt) {
+                const float x = lt[t * p.lw + col];
+                if (x > -INFINITY) w = __float2half_rn(exp2f(x - mh));
+              }
+              acc += __half2float(w);
+              const uint32_t off = static_cast<uint32_t>(t >> 3) * lbo_b + static_cast<uint32_t>(col >> 3) * 128u +
+                                   static_cast<uint32_t>(col & 7) * 16u + static_cast<uint32_t>(t & 7) * 2u;
+              *reinterpret_cast<__half*>(pt_s + off) = w;
+            }
+            lsum2[k2] += acc;
+          }
+        }
+      } else {
+        const float m_h = sM[h_w];
+        for (int t = t_w0; t < kBlock; t += t_step) {
+          // unnormalised weight exp2(s - M) <= 1, rounded to fp16 for the MMA; the
+          // normaliser sums exactly the rounded weights
+          __half w = __float2half_rn(0.f);
+          if (t < mt.nt && h_w < p.H) w = __float2half_rn(exp2f(lt[t * p.H + h_w] - m_h));
+          lsum += __half2float(w);
+          const uint32_t off = static_cast<uint32_t>(t >> 3) * lbo_b + static_cast<uint32_t>(h_w >> 3) * 128u +
+                               static_cast<uint32_t>(h_w & 7) * 16u + static_cast<uint32_t>(t & 7) * 2u;
+          *reinterpret_cast<__half*>(pt_s + off) = w;
+        }
       }
       if (mt.nt < kBlock) {
         // tokens past the sequence end: zero their rows of the V tile so that
@@ -1082,7 +1493,31 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
         const size_t slot = static_cast<size_t>(mt.b) + cta;
         // partial rows [R range][head][slot][r_range]: head h0+hh's row of this slot
         float* zb = p.zpart + ((static_cast<size_t>(rr) * p.H) * p.v_slots + slot) * p.r_range;
-        for (int m = 0; m < p.n_mtiles; ++m) {
+        if constexpr (kChunk) {
+          // virtual head (h, i): row slot * nq + i of head h
+          for (int m = 0; m < p.n_mtiles; ++m) {
+            uint32_t v[32];
+            const uint32_t ta = taddr + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(m * p.npad);
+            const int j = m * 128 + q * 32 + lane;
+            for (int h0 = 0; h0 < p.npad; h0 += 32) {
+              if (p.npad - h0 >= 32) tmem_ld_32x32b_x32(ta + h0, v);
+              else tmem_ld_32x32b_x16(ta + h0, v);
+              tmem_ld_wait();
+              if (j < p.r_range && rr * p.r_range + j < p.R) {
+                const int hn = min(32, p.npad - h0);
+                for (int hh = 0; hh < hn; ++hh) {
+                  const int col = vg * p.lw + h0 + hh;
+                  if (col >= p.Hv) break;
+                  const size_t row = ((static_cast<size_t>(rr) * p.H + (col >> p.log2nq)) * p.v_slots + slot)
+                                         << p.log2nq;
+                  st_global_hint(p.zpart + (row + (col & ((1 << p.log2nq) - 1))) * p.r_range + j,
+                                 __uint_as_float(v[hh]), keep);
+                }
+              }
+            }
+          }
+        }
+        for (int m = 0; m < (kChunk ? 0 : p.n_mtiles); ++m) {
           uint32_t v[32];
           const uint32_t ta = taddr + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(m * p.npad);
           const int j = m * 128 + q * 32 + lane;
@@ -1100,6 +1535,16 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
         }
         tc_fence_before();
         mbar_arrive(tfree);
+        if constexpr (kChunk) {
+          // per-segment normaliser of every virtual head (one thread per column)
+          if (rr == 0)
+            for (int k2 = 0; k2 < 2; ++k2) {
+              const int col = et + 128 * k2;
+              if (col < p.npad && vg * p.lw + col < p.Hv) p.lpart[slot * p.Hv + vg * p.lw + col] = lsum2[k2];
+            }
+          ++seg;
+          continue;
+        }
         // per-segment normaliser of every head
         sRed[et] = lsum;
         if (!group_sync(pbar, pphase)) { set_timeout(p.status, kSiteVFull); abort_flag = 1; break; }
@@ -1154,6 +1599,14 @@ struct FinishParams {
   int zrows;              // partial rows reserved per stage (multiple of kFinZBox, >= any tile's need)
   uint32_t stage_bytes;
   uint32_t tmem_cols;
+  // read-once chunked prefill: the "sequences" are virtual sequences of
+  // 1 << log2nq query rows; B-operand row v * nq + i is row i of virtual
+  // sequence v (output row vs_row0[v] + i, present while i < vs_nrows[v]),
+  // its partials are rows slot * nq + i of head h, its normalisers are
+  // lpart[slot][h * nq + i] (row width Hv).  log2nq = 0, vs_row0 = null: decode.
+  const int32_t* vs_row0;
+  const int32_t* vs_nrows;
+  int log2nq, Hv;
 };
 
 constexpr int kFinThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 convert, then epilogue
@@ -1197,8 +1650,9 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
   const int mt = xi % p.n_mt;
   const int bt = xi / p.n_mt;
   const int ks = blockIdx.y, KS = gridDim.y;
-  const int b0 = bt * p.bt_rows;
+  const int b0 = bt * p.bt_rows;                      // first (virtual) sequence of the tile
   const int nb = min(p.bt_rows, p.B - b0);
+  const int nq = 1 << p.log2nq;
   const int k0 = ks * p.k_per_cta;
   const int k1 = min(p.R, k0 + p.k_per_cta);
   const int n_stages = k1 > k0 ? (k1 - k0 + kFinKC - 1) / kFinKC : 0;
@@ -1225,7 +1679,7 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
   pt.G = static_cast<int32_t>(pt.P < p.v_grid ? pt.P : p.v_grid);
   int32_t slot_lo = 0, n_slots = 0;
   if (pt.P > 0) tile_slots(p.prefix, pt, b0, b0 + nb, &slot_lo, &n_slots);
-  const int n_box = n_slots > 0 ? (min(n_slots, p.zrows) + kFinZBox - 1) / kFinZBox : 0;
+  const int n_box = n_slots > 0 ? (min(n_slots << p.log2nq, p.zrows) + kFinZBox - 1) / kFinZBox : 0;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -1243,7 +1697,7 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
         mbar_arrive_expect_tx(&full[s], a_bytes + static_cast<uint32_t>(n_box) * kFinZBox * 256u);
         tma_load_2d(st, &bvmap, col, kr, &full[s], pol);
         tma_load_2d(st + kFinKC * 128, &bvmap, col + 64, kr, &full[s], pol);
-        const int zrow = (rr * p.H + h) * p.v_slots + slot_lo;
+        const int zrow = ((rr * p.H + h) * p.v_slots + slot_lo) << p.log2nq;
         uint8_t* zdst = st + a_bytes + 2u * half_bytes;
         for (int z = 0; z < n_box; ++z)
           tma_load_2d(zdst + static_cast<size_t>(z) * kFinZBox * 256, &zmap, jj, zrow + z * kFinZBox, &full[s], pol);
@@ -1278,17 +1732,20 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
     for (int bl = et; bl < p.npad; bl += 128) {
       int32_t row = 0, nseg = 0;
       float il = 0.f;
-      if (bl < nb && pt.P > 0) {
-        const int b = b0 + bl;
+      const int vb = bl >> p.log2nq, qi = bl & (nq - 1);   // (virtual) sequence of the tile, its row
+      if (vb < nb && pt.P > 0 && (!p.vs_nrows || qi < p.vs_nrows[b0 + vb])) {
+        const int b = b0 + vb;
         const int32_t f0 = p.prefix[b], f1 = p.prefix[b + 1];
         if (f1 > f0) {
           const int32_t i0 = part_owner(f0, pt), i1 = part_owner(f1 - 1, pt);
+          const int col = p.vs_row0 ? (h << p.log2nq) + qi : h;
+          const int lw = p.vs_row0 ? p.Hv : p.H;
           float Ls = 0.f;
-          for (int32_t i = i0; i <= i1; ++i) Ls += p.lpart[static_cast<size_t>(b + i) * p.H + h];
+          for (int32_t i = i0; i <= i1; ++i) Ls += p.lpart[static_cast<size_t>(b + i) * lw + col];
           il = 1.f / Ls;
-          row = b + i0 - slot_lo;
+          row = ((b + i0 - slot_lo) << p.log2nq) + qi;
           nseg = i1 - i0 + 1;
-          if (row < 0 || row + nseg > n_box * kFinZBox) nseg = 0;   // cannot happen: the plan bounds the tile
+          if (row < 0 || row + ((nseg - 1) << p.log2nq) >= n_box * kFinZBox) nseg = 0;   // cannot happen: the plan bounds the tile
         }
       }
       s_row[bl] = row;
@@ -1312,9 +1769,9 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
         const int nseg = s_nseg[bl];
         if (nseg > 0) {
           const float* src = reinterpret_cast<const float*>(zt + static_cast<size_t>(s_row[bl]) * 256) + c * 8;
-          for (int g = 0; g < nseg; ++g) {
-            const float4 v0 = reinterpret_cast<const float4*>(src + g * 64)[0];
-            const float4 v1 = reinterpret_cast<const float4*>(src + g * 64)[1];
+          for (int g = 0; g < nseg; ++g) {   // segment g: nq partial rows further on
+            const float4 v0 = reinterpret_cast<const float4*>(src + (g << p.log2nq) * 64)[0];
+            const float4 v1 = reinterpret_cast<const float4*>(src + (g << p.log2nq) * 64)[1];
             z[0] += v0.x; z[1] += v0.y; z[2] += v0.z; z[3] += v0.w;
             z[4] += v1.x; z[5] += v1.y; z[6] += v1.z; z[7] += v1.w;
           }
@@ -1366,7 +1823,10 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
   for (int x = tid; x < (n_hi - n_lo) * 32; x += kFinThreads) {
     const int n = n_lo + x / 32, m = (x % 32) * 4;
     const int dm = mt * 128 + m;
-    if (n >= nb || dm >= p.d) continue;
+    const int vb = n >> p.log2nq, qi = n & (nq - 1);
+    if (vb >= nb || dm >= p.d) continue;
+    if (p.vs_nrows && qi >= p.vs_nrows[b0 + vb]) continue;
+    const int64_t orow = p.vs_row0 ? static_cast<int64_t>(p.vs_row0[b0 + vb]) + qi : b0 + n;
     float4 v[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c)
@@ -1379,7 +1839,7 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
     uint2 pk;
     pk.x = *reinterpret_cast<const uint32_t*>(&lo);
     pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-    *reinterpret_cast<uint2*>(p.out + (static_cast<size_t>(b0 + n) * p.H + h) * p.d + dm) = pk;
+    *reinterpret_cast<uint2*>(p.out + (static_cast<size_t>(orow) * p.H + h) * p.d + dm) = pk;
   }
   cluster.sync();
   if (warp == 1) {

@@ -403,15 +403,16 @@ bool encode_vpool_map(CUtensorMap* map, const void* v_cache, int R, int NB, uint
 }
 
 // K pool [num_blocks*16 tokens][Hkv][r] fp16 as a 3-D tensor map {r, Hkv,
-// tokens} with boxes {64 codes, all Hkv heads, box_tokens} and the 128-byte
+// tokens} with boxes {64 codes, box_heads heads, box_tokens} and the 128-byte
 // swizzle (codes past r read as zero).
-bool encode_kpool_map(CUtensorMap* map, const void* k_cache, int r, int Hkv, int NB, uint32_t box_tokens) {
+bool encode_kpool_map(CUtensorMap* map, const void* k_cache, int r, int Hkv, int NB, uint32_t box_heads,
+                      uint32_t box_tokens) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(r), static_cast<cuuint64_t>(Hkv),
                         static_cast<cuuint64_t>(NB) * 16};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(r) * 2, static_cast<cuuint64_t>(Hkv) * r * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(Hkv), box_tokens};
+  cuuint32_t box[3] = {64, box_heads, box_tokens};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult res = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(k_cache), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -795,7 +796,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   if (pl.ktc) {
     CUtensorMap kmap, qmap;
     const uint32_t tpt = 1u << pl.ktc_log2tpt;
-    if (!encode_kpool_map(&kmap, k_cache, pl.r, pl.Hkv, pl.NB, tpt < 16 ? tpt : 16) ||
+    if (!encode_kpool_map(&kmap, k_cache, pl.r, pl.Hkv, pl.NB, static_cast<uint32_t>(pl.Hkv), tpt < 16 ? tpt : 16) ||
         !encode_2d_map(&qmap, qth, static_cast<uint64_t>(pl.r), static_cast<uint64_t>(batch) * 2 * pl.H, 64,
                        static_cast<uint32_t>(pl.ktc_brows)))
       return STARKV_ERR_CUDA;
@@ -827,8 +828,8 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   vp.k_grid = pl.k_ctas;
   vp.stages = pl.v_stages; vp.n_chunks = pl.n_chunks; vp.n_mtiles = pl.n_mtiles; vp.tmem_cols = pl.tmem_cols;
   vp.vtile_bytes = pl.vtile; vp.ltile_bytes = pl.ltile; vp.ptile_bytes = pl.ptile;
-  if (!set_smem(vpass_kernel, pl.v_smem)) return STARKV_ERR_CUDA;
-  if (launch(vpass_kernel, dim3(pl.v_ctas, pl.n_rr), dim3(kVThreads), pl.v_smem, s, 1, vmap, vp) != cudaSuccess)
+  if (!set_smem(vpass_kernel<false>, pl.v_smem)) return STARKV_ERR_CUDA;
+  if (launch(vpass_kernel<false>, dim3(pl.v_ctas, pl.n_rr), dim3(kVThreads), pl.v_smem, s, 1, vmap, vp) != cudaSuccess)
     return STARKV_ERR_CUDA;
   mark(3);
 
@@ -958,9 +959,262 @@ starkv_status starkv_append_decode_host(const starkv_layer_desc* desc, int32_t b
 // sequence map and lengths (int32 [n_rows] each).
 size_t prefill_rows_offset(const DecodePlan& pl) { return align_up(pl.ws.total_bytes, 256); }
 
-size_t starkv_prefill_workspace_bytes(const starkv_layer_desc* desc, int32_t n_rows, int32_t max_seq_len) {
+namespace {
+// ------------------------------------------------- read-once chunked prefill
+// A chunk's rows are taken nq = 16 / G at a time as virtual sequences whose
+// query heads are the virtual heads (h, i); every K and V page of a virtual
+// sequence is then streamed once for all of its rows (see kpass_chunk_kernel).
+// Shapes: KV heads in groups of 8 (Hkv % 8 == 0), G = H / Hkv <= 16.
+struct ChunkPlan {
+  int H, Hkv, d, r, R, G, nq, log2nq, Hv, lw, n_vg, nv_max, n_groups, t_pad, MB, NB, n_rows, n_seqs;
+  // K pass
+  int k_ctas, kb, ksteps, k_stages, nacc, nbs;
+  uint32_t a_bytes, b_bytes, k_tmem;
+  size_t k_smem;
+  // V pass
+  int r_range, r_range_pad, n_rr, n_chunks, n_mtiles, v_ctas, v_stages, v_slots, k_slots;
+  uint32_t vtile, ltile, ptile, v_tmem;
+  size_t v_smem;
+  // finish
+  int up_mt, up_bt_rows, up_bt, up_npad, up_ks, up_kpc, up_zrows;
+  uint32_t up_stage_bytes, up_tmem;
+  size_t up_smem;
+  // workspace
+  size_t status_off, prefix_off, teff_off, vs_seq_off, vs_row0_off, vs_nrows_off, vs_len_off, qth_off, logits_off,
+      mpart_off, lpart_off, zpart_off, total;
+};
+
+bool chunk_eligible(const starkv_layer_desc* d) {
+  const int Hkv = kv_heads(d);
+  return Hkv % 8 == 0 && d->num_heads / Hkv <= 16;
+}
+
+starkv_status make_chunk_plan(const starkv_layer_desc* d, int32_t n_seqs, int32_t n_rows, int32_t max_seq_len,
+                              ChunkPlan* cp) {
+  starkv_status st = check_desc(d);
+  if (st != STARKV_OK) return st;
+  if (n_seqs < 0 || n_rows < 0 || max_seq_len < 0) return STARKV_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(max_seq_len) > static_cast<int64_t>(d->max_blocks_per_seq) * 16)
+    return STARKV_ERR_INVALID_ARG;
+  if (!chunk_eligible(d)) return STARKV_ERR_UNSUPPORTED;
+  ChunkPlan& c = *cp;
+  std::memset(&c, 0, sizeof(c));
+  c.H = d->num_heads; c.Hkv = kv_heads(d); c.d = d->head_dim; c.r = d->k_rank; c.R = d->v_rank;
+  c.G = c.H / c.Hkv; c.nq = 16 / c.G;
+  while ((1 << c.log2nq) < c.nq) ++c.log2nq;
+  c.Hv = c.H * c.nq;
+  c.lw = c.Hv < 256 ? c.Hv : 256;
+  c.n_vg = c.Hv / c.lw;
+  c.n_rows = n_rows; c.n_seqs = n_seqs;
+  {
+    const int64_t bound = static_cast<int64_t>(n_rows) / c.nq + n_seqs;
+    c.nv_max = static_cast<int>(bound < n_rows ? bound : n_rows);
+    if (c.nv_max < 1) c.nv_max = 1;
+  }
+  c.n_groups = c.Hkv / 8;
+  c.t_pad = (max_seq_len + 15) / 16 * 16;
+  c.MB = d->max_blocks_per_seq; c.NB = d->num_blocks;
+  const int sms = device_sm_count();
+  // K pass: one CTA per SM, two query-tile slots, up to 8 stages, 4 accumulators of 128 columns
+  c.kb = (c.r + 63) / 64;
+  c.ksteps = (c.r + 15) / 16;
+  c.a_bytes = static_cast<uint32_t>(c.kb) * 16384u;
+  c.b_bytes = static_cast<uint32_t>(c.kb) * 256u * 128u;
+  c.nbs = 2;
+  c.nacc = 4;
+  c.k_tmem = 512;
+  {
+    const size_t fixed = 1024 + c.nbs * static_cast<size_t>(c.b_bytes) + (4 + 2 * kKTCMaxAcc + 1) * 8;
+    int stages = static_cast<int>((200u * 1024u - fixed) / (c.a_bytes + 16u));
+    if (stages > 8) stages = 8;
+    if (stages < 2) return STARKV_ERR_UNSUPPORTED;
+    c.k_stages = stages;
+    c.k_smem = fixed + static_cast<size_t>(stages) * (c.a_bytes + 16u);
+  }
+  c.k_ctas = sms;
+  // V pass: lw virtual heads per CTA and mt 128-row M tiles of R (TMEM: mt * lw
+  // columns).  The CTAs of one (R range, virtual-head group) are capped so that
+  // the finish kernel's tile of one virtual sequence can hold all the partial
+  // rows it may need (v_ctas * nq rows of 256 bytes in each of two stages).
+  {
+    // two stages of at most 107 KiB (with barriers and per-row arrays: <= 220 KiB), each
+    // holding B_V boxes, hi/lo tiles of 16 rows and whole 32-row boxes of partial rows
+    const int z_cap = static_cast<int>((107u * 1024u - 2u * kFinKC * 128u - 2u * 16u * 128u) / 256u) /
+                      kFinZBox * kFinZBox;
+    const int cap = z_cap / c.nq > 1 ? z_cap / c.nq : 1;
+    const int rpad = (c.R + 127) / 128 * 128;
+    int best_total = -1;
+    for (int mt = 512 / c.lw; mt >= 1; mt /= 2) {
+      const int rr = mt * 128 < rpad ? mt * 128 : rpad;
+      const int n_rr = (c.R + rr - 1) / rr;
+      const int per_sm = 512 / (mt * c.lw) < 2 ? 512 / (mt * c.lw) : 2;
+      const uint32_t stage = static_cast<uint32_t>(rr) * 32u + 64u * c.lw + 32u * c.lw;   // V tile, logits, weights
+      const int stages = static_cast<int>((200u * 1024u / per_sm) / stage);
+      if (per_sm < 1 || stages < 2) continue;
+      int v_ctas = sms * per_sm / (n_rr * c.n_vg);
+      if (v_ctas > cap) v_ctas = cap;
+      if (v_ctas < 1) v_ctas = 1;
+      const int total = v_ctas * n_rr * c.n_vg;
+      if (best_total >= sms || total <= best_total) continue;   // the widest R range that fills the GPU
+      best_total = total;
+      c.r_range = rr; c.n_rr = n_rr; c.v_ctas = v_ctas;
+      c.v_stages = stages > 8 ? 8 : stages;
+    }
+    if (best_total < 0) return STARKV_ERR_UNSUPPORTED;
+    c.r_range_pad = c.r_range;
+    c.n_chunks = c.r_range_pad / 64;
+    c.n_mtiles = c.r_range_pad / 128;
+    c.vtile = static_cast<uint32_t>(c.r_range_pad) * 16 * 2;
+    c.ltile = 16u * c.lw * 4;
+    c.ptile = static_cast<uint32_t>(c.lw) * 16 * 2;
+    c.v_tmem = static_cast<uint32_t>(pow2_ceil(c.n_mtiles * c.lw < 32 ? 32 : c.n_mtiles * c.lw));
+    c.v_smem = 1024 + static_cast<size_t>(c.v_stages) * (c.vtile + c.ltile + c.ptile) + c.v_stages * sizeof(StageMeta) +
+               (3 * c.v_stages + 4) * sizeof(uint64_t) + (c.lw + 128) * sizeof(float);
+  }
+  c.k_slots = c.k_ctas + c.nv_max;
+  c.v_slots = c.v_ctas + c.nv_max;
+  // finish: tiles of virtual sequences (nq rows each)
+  c.up_mt = (c.d + 127) / 128;
+  c.up_bt_rows = 256 / c.nq;
+  if (c.up_bt_rows > c.nv_max) c.up_bt_rows = c.nv_max;
+  for (int tries = 0; tries < 16; ++tries) {
+    const int rows = c.up_bt_rows * c.nq;
+    c.up_npad = rows < 16 ? 16 : (rows + 15) / 16 * 16;
+    const int need = (c.up_bt_rows + c.v_ctas - 1) * c.nq;
+    c.up_zrows = (need + kFinZBox - 1) / kFinZBox * kFinZBox;
+    c.up_stage_bytes = static_cast<uint32_t>(
+        align_up(2u * kFinKC * 128u + 2u * static_cast<size_t>(c.up_npad) * 128u + c.up_zrows * 256u, 1024));
+    c.up_smem = 1024 + 2 * static_cast<size_t>(c.up_stage_bytes) + 7 * sizeof(uint64_t) + 3 * kFinMaxRows * 4;
+    if (c.up_smem <= 220u * 1024u) break;
+    if (c.up_bt_rows == 1) return STARKV_ERR_UNSUPPORTED;
+    c.up_bt_rows /= 2;
+  }
+  if (c.up_smem > 220u * 1024u) return STARKV_ERR_UNSUPPORTED;
+  c.up_bt = (c.nv_max + c.up_bt_rows - 1) / c.up_bt_rows;
+  c.up_ks = 1;
+  while (c.up_ks < 8 && c.H * c.up_mt * c.up_bt * c.up_ks * 2 <= sms && c.R / kFinKC >= c.up_ks * 2) c.up_ks *= 2;
+  c.up_kpc = ((c.R + c.up_ks * kFinKC - 1) / (c.up_ks * kFinKC)) * kFinKC;
+  c.up_tmem = static_cast<uint32_t>(pow2_ceil(c.up_npad < 32 ? 32 : c.up_npad));
+  // workspace
+  size_t off = 0;
+  const size_t nv = static_cast<size_t>(c.nv_max);
+  c.status_off = off; off += 256;
+  c.prefix_off = off; off = align_up(off + (nv + 1) * 4, 256);
+  c.teff_off = off; off = align_up(off + nv * 4, 256);
+  c.vs_seq_off = off; off = align_up(off + nv * 4, 256);
+  c.vs_row0_off = off; off = align_up(off + nv * 4, 256);
+  c.vs_nrows_off = off; off = align_up(off + nv * 4, 256);
+  c.vs_len_off = off; off = align_up(off + nv * 4, 256);
+  c.qth_off = off; off = align_up(off + nv * 2 * c.Hv * c.r * 2, 256);
+  c.logits_off = off; off = align_up(off + nv * c.n_vg * c.t_pad * static_cast<size_t>(c.lw) * 4, 256);
+  c.mpart_off = off; off = align_up(off + static_cast<size_t>(c.k_slots) * c.Hv * 4, 256);
+  c.lpart_off = off; off = align_up(off + static_cast<size_t>(c.v_slots) * c.Hv * 4, 256);
+  c.zpart_off = off;
+  off = align_up(off + static_cast<size_t>(c.n_rr) * c.H * c.v_slots * c.nq * c.r_range * 4, 256);
+  c.total = off;
+  return STARKV_OK;
+}
+
+starkv_status chunk_prefill(const ChunkPlan& c, const void* q, const void* B_K, const void* B_V, const void* k_cache,
+                            const void* v_cache, const int32_t* block_tables, const int32_t* starts,
+                            const int32_t* row_offsets, float scale, uint8_t* ws, void* out, cudaStream_t s) {
+  int32_t* status = reinterpret_cast<int32_t*>(ws + c.status_off);
+  int32_t* prefix = reinterpret_cast<int32_t*>(ws + c.prefix_off);
+  int32_t* teff = reinterpret_cast<int32_t*>(ws + c.teff_off);
+  int32_t* vs_seq = reinterpret_cast<int32_t*>(ws + c.vs_seq_off);
+  int32_t* vs_row0 = reinterpret_cast<int32_t*>(ws + c.vs_row0_off);
+  int32_t* vs_nrows = reinterpret_cast<int32_t*>(ws + c.vs_nrows_off);
+  int32_t* vs_len = reinterpret_cast<int32_t*>(ws + c.vs_len_off);
+  __half* qth = reinterpret_cast<__half*>(ws + c.qth_off);
+  float* logits = reinterpret_cast<float*>(ws + c.logits_off);
+  float* mpart = reinterpret_cast<float*>(ws + c.mpart_off);
+  float* lpart = reinterpret_cast<float*>(ws + c.lpart_off);
+  float* zpart = reinterpret_cast<float*>(ws + c.zpart_off);
+
+  CUtensorMap kmap, qmap, vmap, bvmap, zmap;
+  if (!encode_kpool_map(&kmap, k_cache, c.r, c.Hkv, c.NB, 8, 16) ||
+      !encode_2d_map(&qmap, qth, static_cast<uint64_t>(c.r), static_cast<uint64_t>(c.nv_max) * 2 * c.Hv, 64,
+                     kKChunkCols) ||
+      !encode_vpool_map(&vmap, v_cache, c.R, c.NB, static_cast<uint32_t>(c.n_chunks)) ||
+      !encode_2d_map(&bvmap, B_V, static_cast<uint64_t>(c.Hkv) * c.d, static_cast<uint64_t>(c.R), 64, kFinKC) ||
+      !encode_f32_rows_map(&zmap, zpart, static_cast<uint64_t>(c.r_range),
+                           static_cast<uint64_t>(c.n_rr) * c.H * c.v_slots * c.nq, 64, kFinZBox))
+    return STARKV_ERR_CUDA;
+
+  ChunkTableParams tp{starts, row_offsets, vs_seq, vs_row0, vs_nrows, vs_len, c.n_seqs, c.nv_max, c.log2nq};
+  if (launch(chunk_table_kernel, dim3(1), dim3(256), 0, s, 1, tp) != cudaSuccess) return STARKV_ERR_CUDA;
+
+  AbsorbParams ap;
+  std::memset(&ap, 0, sizeof(ap));
+  ap.q = static_cast<const __half*>(q);
+  ap.B_K = static_cast<const __half*>(B_K);
+  ap.seq_lens = vs_len;
+  ap.qt = nullptr; ap.qth = qth; ap.prefix = prefix; ap.teff = teff; ap.status = status;
+  ap.mpart_init = mpart;
+  ap.n_mpart = c.k_slots * c.Hv;
+  ap.B = c.nv_max; ap.H = c.H; ap.d = c.d; ap.r = c.r; ap.cap = c.t_pad;
+  {
+    int lg = 0;
+    while ((c.Hkv << lg) < c.H) ++lg;
+    ap.log2G = lg;
+  }
+  ap.coef = scale * kLog2e;
+  ap.vs_row0 = vs_row0; ap.vs_nrows = vs_nrows; ap.log2nq = c.log2nq;
+  if (launch_prep(c.d, nullptr, &ap, c.nv_max << c.log2nq, s) != STARKV_OK) return STARKV_ERR_CUDA;
+
+  KPassChunkParams kp;
+  kp.tables = block_tables; kp.vs_seq = vs_seq; kp.vs_nrows = vs_nrows; kp.teff = teff; kp.prefix = prefix;
+  kp.logits = logits; kp.mpart = mpart; kp.status = status;
+  kp.B = c.nv_max; kp.MB = c.MB; kp.NB = c.NB; kp.t_pad = c.t_pad;
+  kp.Hv = c.Hv; kp.n_vg = c.n_vg; kp.n_groups = c.n_groups; kp.log2nq = c.log2nq;
+  kp.log2lw = 0;
+  while ((1 << kp.log2lw) < c.lw) ++kp.log2lw;
+  kp.ksteps = c.ksteps; kp.kb = c.kb; kp.nacc = c.nacc; kp.nbs = c.nbs; kp.stages = c.k_stages;
+  kp.a_bytes = c.a_bytes; kp.b_bytes = c.b_bytes; kp.tmem_cols = c.k_tmem;
+  kp.drop_stage = g_drop_k_stage.load(std::memory_order_relaxed);
+  if (!set_smem(kpass_chunk_kernel, c.k_smem)) return STARKV_ERR_CUDA;
+  if (launch(kpass_chunk_kernel, dim3(c.k_ctas), dim3(kKTCThreads), c.k_smem, s, 1, kmap, qmap, kp) != cudaSuccess)
+    return STARKV_ERR_CUDA;
+
+  VPassParams vp;
+  std::memset(&vp, 0, sizeof(vp));
+  vp.tables = block_tables; vp.row_seq = vs_seq; vp.teff = teff; vp.prefix = prefix; vp.logits = logits;
+  vp.mpart = mpart; vp.zpart = zpart; vp.lpart = lpart; vp.status = status;
+  vp.B = c.nv_max; vp.H = c.H; vp.npad = c.lw; vp.MB = c.MB; vp.NB = c.NB; vp.R = c.R;
+  vp.t_pad = c.t_pad; vp.r_range = c.r_range; vp.n_rr = c.n_rr; vp.v_slots = c.v_slots;
+  vp.k_grid = c.k_ctas;
+  vp.stages = c.v_stages; vp.n_chunks = c.n_chunks; vp.n_mtiles = c.n_mtiles; vp.tmem_cols = c.v_tmem;
+  vp.vtile_bytes = c.vtile; vp.ltile_bytes = c.ltile; vp.ptile_bytes = c.ptile;
+  vp.Hv = c.Hv; vp.n_vg = c.n_vg; vp.log2nq = c.log2nq; vp.lw = c.lw;
+  if (!set_smem(vpass_kernel<true>, c.v_smem)) return STARKV_ERR_CUDA;
+  if (launch(vpass_kernel<true>, dim3(c.v_ctas, c.n_rr * c.n_vg), dim3(kVThreads), c.v_smem, s, 1, vmap, vp) !=
+      cudaSuccess)
+    return STARKV_ERR_CUDA;
+
+  FinishParams fp;
+  std::memset(&fp, 0, sizeof(fp));
+  fp.out = static_cast<__half*>(out);
+  fp.lpart = lpart; fp.prefix = prefix;
+  fp.B = c.nv_max; fp.H = c.H; fp.d = c.d; fp.R = c.R;
+  fp.log2G = ap.log2G;
+  fp.r_range = c.r_range; fp.v_slots = c.v_slots; fp.v_grid = c.v_ctas;
+  fp.n_mt = c.up_mt; fp.bt_rows = c.up_bt_rows; fp.k_per_cta = c.up_kpc; fp.npad = c.up_npad;
+  fp.stages = 2; fp.zrows = c.up_zrows; fp.stage_bytes = c.up_stage_bytes; fp.tmem_cols = c.up_tmem;
+  fp.vs_row0 = vs_row0; fp.vs_nrows = vs_nrows; fp.log2nq = c.log2nq; fp.Hv = c.Hv;
+  if (!set_smem(finish_kernel, c.up_smem)) return STARKV_ERR_CUDA;
+  if (launch(finish_kernel, dim3(c.H * c.up_mt * c.up_bt, c.up_ks), dim3(kFinThreads), c.up_smem, s, c.up_ks,
+             bvmap, zmap, fp) != cudaSuccess)
+    return STARKV_ERR_CUDA;
+  return STARKV_OK;
+}
+}  // namespace
+
+size_t starkv_prefill_workspace_bytes(const starkv_layer_desc* desc, int32_t n_seqs, int32_t n_rows,
+                                      int32_t max_seq_len) {
   DecodePlan pl;
-  if (n_rows < 0 || make_plan(desc, n_rows, max_seq_len, &pl) != STARKV_OK) return 0;
+  if (n_seqs < 0 || n_rows < 0 || make_plan(desc, n_rows, max_seq_len, &pl) != STARKV_OK) return 0;
+  ChunkPlan cp;
+  if (chunk_eligible(desc)) return make_chunk_plan(desc, n_seqs, n_rows, max_seq_len, &cp) == STARKV_OK ? cp.total : 0;
   return prefill_rows_offset(pl) + align_up(static_cast<size_t>(n_rows) * 8, 256);
 }
 
@@ -977,13 +1231,25 @@ starkv_status starkv_paged_prefill(const starkv_layer_desc* desc, int32_t n_seqs
   if (n_seqs == 0 || !starts || !row_offsets || (reinterpret_cast<uintptr_t>(starts) & 3u) ||
       (reinterpret_cast<uintptr_t>(row_offsets) & 3u))
     return STARKV_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ChunkPlan cp;
+  if (chunk_eligible(desc)) {
+    if (make_chunk_plan(desc, n_seqs, n_rows, max_seq_len, &cp) != STARKV_OK) return STARKV_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < cp.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+      return STARKV_ERR_WORKSPACE;
+    if (!q || !B_K || !B_V || !k_cache || !v_cache || !block_tables || !out || !aligned16(q) || !aligned16(B_K) ||
+        !aligned16(B_V) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) || !(std::isfinite(scale) && scale > 0.f))
+      return STARKV_ERR_INVALID_ARG;
+    return chunk_prefill(cp, q, B_K, B_V, k_cache, v_cache, block_tables, starts, row_offsets, scale,
+                         static_cast<uint8_t*>(workspace), out, s);
+  }
   const size_t need = prefill_rows_offset(pl) + align_up(static_cast<size_t>(n_rows) * 8, 256);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return STARKV_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* row_seq = reinterpret_cast<int32_t*>(ws + prefill_rows_offset(pl));
   int32_t* row_len = row_seq + n_rows;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   PrefillRowsParams rp{starts, row_offsets, row_seq, row_len, n_seqs, n_rows};
   if (launch(prefill_rows_kernel, dim3((n_rows + 255) / 256), dim3(256), 0, s, 1, rp) != cudaSuccess)
     return STARKV_ERR_CUDA;

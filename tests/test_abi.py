@@ -152,7 +152,7 @@ def test_kv_head_count_validation(lib, kv, expect):
 def test_prefill_argument_errors(lib):
     d = _desc()
     fake = 1 << 20
-    need = S.starkv_prefill_workspace_bytes(d, 40, 1024)
+    need = S.starkv_prefill_workspace_bytes(d, 2, 40, 1024)
     assert need > S.starkv_decode_workspace_bytes(d, 40, 1024) > 0
     args = [d, 2, 40, 1024, fake, fake, fake, fake, fake, fake, fake, fake, 0.1, fake, need, fake]
 
@@ -170,7 +170,8 @@ def test_prefill_argument_errors(lib):
     assert S.starkv_paged_prefill(*a, stream=0, check=False) == 0
     a = list(args); a[2] = 0; a[13] = fake + 128  # no rows, misaligned workspace: refused
     assert S.starkv_paged_prefill(*a, stream=0, check=False) == 3
-    assert S.starkv_prefill_workspace_bytes(d, -1, 1024) == 0
+    assert S.starkv_prefill_workspace_bytes(d, 2, -1, 1024) == 0
+    assert S.starkv_prefill_workspace_bytes(d, -1, 40, 1024) == 0
 
 
 def test_wait_test_hook_rejects_bad_stage(lib):

@@ -123,7 +123,7 @@ def test_decode_empty_and_zero_batch():
     assert np.array_equal(out, np.zeros_like(out))
     # a prefill call with no rows also leaves a clean status word in a poisoned workspace
     desc = desc_of(Ld)
-    wsb = S.starkv_prefill_workspace_bytes(desc, 0, 0)
+    wsb = S.starkv_prefill_workspace_bytes(desc, 0, 0, 0)
     ws = torch.full((max(wsb, 256),), POISON, dtype=torch.uint8, device="cuda")
     S.starkv_paged_prefill(desc, 0, 0, 0, None, None, None, None, None, None, None, None, 0.1, ws, wsb, None)
     assert S.starkv_decode_check(ws) == (0, 0)
@@ -344,9 +344,9 @@ def test_append_and_decode_in_cuda_graph_match_stream_launches():
 
 # ------------------------------------------------------ chunked prefill
 
-def _prefill_check(kv_heads, starts, chunks, seed):
-    H, d = 32, 128
-    sh = W.LayerShape(H, d, 64, 512 if kv_heads else 2048, num_kv_heads=kv_heads)
+def _prefill_check(kv_heads, starts, chunks, seed, H=32, d=128, r=64, R=None):
+    R = R or (512 if kv_heads else 2048)
+    sh = W.LayerShape(H, d, r, R, num_kv_heads=kv_heads)
     starts = np.asarray(starts, np.int64)
     chunks = np.asarray(chunks, np.int64)
     # every chunk's codes are in the cache: the context is start + chunk tokens
@@ -359,7 +359,7 @@ def _prefill_check(kv_heads, starts, chunks, seed):
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     desc = desc_of(Ld)
     max_len = int((starts + chunks).max())
-    wsb = S.starkv_prefill_workspace_bytes(desc, n_rows, max_len)
+    wsb = S.starkv_prefill_workspace_bytes(desc, len(chunks), n_rows, max_len)
     ws = torch.full((wsb,), 0xFF, dtype=torch.uint8, device="cuda")
     out = torch.full((n_rows, H, d), float("nan"), dtype=torch.float16, device="cuda")
     S.starkv_paged_prefill(desc, len(chunks), n_rows, max_len, dev(q), Ld["B_K"], Ld["B_V"], Ld["k_cache"],
@@ -382,6 +382,18 @@ def test_prefill_chunks_causal(kv_heads):
 def test_prefill_rows_of_one_sequence_span_tiles():
     """One sequence, a 300-token chunk after 700 cached tokens: rows span several K/V partitions."""
     _prefill_check(0, starts=[700], chunks=[300], seed=6161)
+
+
+def test_prefill_read_once_shapes():
+    """Read-once path with 8 query heads per KV head (2 rows per virtual sequence), and 16-row chunks
+    of several sequences over long contexts (the benchmark's chunk size)."""
+    _prefill_check(8, starts=[0, 333, 1500], chunks=[5, 16, 33], seed=6262, H=64, r=64, R=512)
+    _prefill_check(0, starts=[2048, 700, 1601, 16], chunks=[16, 16, 16, 16], seed=6363)
+
+
+def test_prefill_row_wise_path():
+    """KV heads not in groups of 8 (8 query heads over 2 KV heads): every row runs as a decode row."""
+    _prefill_check(2, starts=[0, 5, 200, 37], chunks=[37, 0, 150, 64], seed=6464, H=8, d=64, r=16, R=128)
 
 
 # ------------------------------------------------ grouped-query attention
