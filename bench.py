@@ -86,14 +86,16 @@ def whole_job_tokens_per_s(world: int, batch_per_rank: int, ms_per_step_max: flo
 
 # DRAM bytes (read + write) per processed token of the two streaming kernels,
 # from ncu captures (dram__bytes_read.sum + dram__bytes_write.sum of one
-# launch); traffic grows in proportion to the tokens processed.  Keyed by
-# layer geometry (query heads, KV heads, K rank, V rank).  A figure is only
-# valid for the kernels as they were captured, so an entry is emptied when its
-# kernel changes and refilled from a new capture (the summaries under
-# profiles/ give the commands).  Both passes have changed since the last
-# captures (segment maxima by atomics, bounded V-pass syncs, the block-table
-# indirection for prefill rows), so no geometry has a current figure.
-NCU_TRAFFIC_PER_TOKEN: dict = {}
+# launch at batch 32, context 8192, divided by its 262,144 tokens); traffic
+# grows in proportion to the tokens processed.  Keyed by layer geometry
+# (query heads, KV heads, K rank, V rank).  A figure is only valid for the
+# kernels as they were captured: profiles/streaming_traffic_b32_t8192.md and
+# profiles/gqa_streaming_b32_t8192_full.md give the commands; an entry is
+# emptied when its kernel changes.
+NCU_TRAFFIC_PER_TOKEN: dict = {
+    (32, 32, 64, 2048): {"kpass": 4123.2, "vpass": 4259.4},
+    (32, 8, 64, 512): {"kpass": 1049.6, "vpass": 1167.1},
+}
 
 
 def measured_peaks():
