@@ -541,8 +541,8 @@ namespace {
 // and the K-code items of `batch` new rows of k, v stored at `tgt`.
 struct AppendPlan {
   CUtensorMap amap, vmap;
-  AppendVParams vp;
-  AppendKParams kp;
+  AppendVParams vp{};
+  AppendKParams kp{};
   int v_mt, v_cols, KS;
   size_t v_smem, k_smem;
 };
@@ -599,7 +599,7 @@ starkv_status plan_append(const starkv_layer_desc* desc, int32_t batch, const vo
 // absorption `abs` (null: none) over `batch` rows.  Item tiles of 16 rows are
 // used when they keep the grid within one wave of two CTAs per SM, else 32.
 starkv_status launch_prep(int d, const AppendPlan* app, const AbsorbParams* abs, int batch, cudaStream_t s) {
-  PrepParams pp;
+  PrepParams pp{};
   std::memset(&pp, 0, sizeof(pp));
   const int KS = app ? app->KS : 1;
   const int sms = device_sm_count();
@@ -647,7 +647,7 @@ starkv_status compress_store_impl(const starkv_layer_desc* desc, int32_t batch, 
   if (st != STARKV_OK) return st;
   if (batch < 0) return STARKV_ERR_INVALID_ARG;
   if (batch == 0) return STARKV_OK;
-  AppendPlan ap;
+  AppendPlan ap{};
   st = plan_append(desc, batch, k, v, A_K, A_V, tgt, k_cache, v_cache, &ap);
   if (st != STARKV_OK) return st;
   return launch_prep(desc->head_dim, &ap, nullptr, batch, static_cast<cudaStream_t>(stream));
@@ -692,7 +692,7 @@ starkv_status starkv_set_wait_test_hook(uint32_t wait_limit_us, int32_t drop_k_s
 }
 
 size_t starkv_decode_workspace_bytes(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len) {
-  DecodePlan pl;
+  DecodePlan pl{};
   if (make_plan(desc, batch, max_seq_len, &pl) != STARKV_OK) return 0;
   return pl.ws.total_bytes;
 }
@@ -700,7 +700,7 @@ size_t starkv_decode_workspace_bytes(const starkv_layer_desc* desc, int32_t batc
 starkv_status starkv_decode_workspace_layout(const starkv_layer_desc* desc, int32_t batch, int32_t max_seq_len,
                                              starkv_workspace_layout* out) {
   if (!out) return STARKV_ERR_INVALID_ARG;
-  DecodePlan pl;
+  DecodePlan pl{};
   starkv_status st = make_plan(desc, batch, max_seq_len, &pl);
   if (st != STARKV_OK) return st;
   *out = pl.ws;
@@ -726,7 +726,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
                           const int32_t* block_tables, const int32_t* seq_lens, float scale, void* workspace,
                           size_t workspace_bytes, void* out, void* stream, void* const* stage_events,
                           const int32_t* row_seq = nullptr, const AppendPlan* app = nullptr) {
-  DecodePlan pl;
+  DecodePlan pl{};
   starkv_status st = make_plan(desc, batch, max_seq_len, &pl);
   if (st != STARKV_OK) return st;
   if (!(std::isfinite(scale) && scale > 0.f)) return STARKV_ERR_INVALID_ARG;
@@ -769,7 +769,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   };
   mark(0);
 
-  AbsorbParams ap;
+  AbsorbParams ap{};
   ap.q = static_cast<const __half*>(q);
   ap.B_K = static_cast<const __half*>(B_K);
   ap.seq_lens = seq_lens;
@@ -784,7 +784,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   if (launch_prep(pl.d, app, &ap, batch, s) != STARKV_OK) return STARKV_ERR_CUDA;
   mark(1);
 
-  KPassParams kp;
+  KPassParams kp{};
   kp.k_cache = static_cast<const __half*>(k_cache);
   kp.tables = block_tables; kp.row_seq = row_seq; kp.teff = teff; kp.prefix = prefix; kp.qt = qt;
   kp.logits = logits; kp.mpart = mpart; kp.status = status;
@@ -800,7 +800,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
         !encode_2d_map(&qmap, qth, static_cast<uint64_t>(pl.r), static_cast<uint64_t>(batch) * 2 * pl.H, 64,
                        static_cast<uint32_t>(pl.ktc_brows)))
       return STARKV_ERR_CUDA;
-    KPassTCParams tp;
+    KPassTCParams tp{};
     tp.tables = block_tables; tp.row_seq = row_seq; tp.teff = teff; tp.prefix = prefix;
     tp.logits = logits; tp.mpart = mpart; tp.status = status;
     tp.B = batch; tp.log2G = pl.log2G; tp.log2Hkv = pl.log2H - pl.log2G;
@@ -819,7 +819,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   if (e != cudaSuccess) return STARKV_ERR_CUDA;
   mark(2);
 
-  VPassParams vp;
+  VPassParams vp{};
   vp.tables = block_tables; vp.row_seq = row_seq; vp.teff = teff; vp.prefix = prefix; vp.logits = logits;
   vp.mpart = mpart;
   vp.zpart = zpart; vp.lpart = lpart; vp.status = status;
@@ -833,7 +833,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
     return STARKV_ERR_CUDA;
   mark(3);
 
-  FinishParams fp;
+  FinishParams fp{};
   fp.out = static_cast<__half*>(out);
   fp.lpart = lpart; fp.prefix = prefix;
   fp.B = batch; fp.H = pl.H; fp.d = pl.d; fp.R = pl.R; fp.log2G = pl.log2G;
@@ -869,7 +869,7 @@ starkv_status starkv_append_decode(const starkv_layer_desc* desc, int32_t batch,
   if (batch == 0) return clear_status(workspace, workspace_bytes, stream);
   if (!block_tables || !positions || (reinterpret_cast<uintptr_t>(append_status) & 3u)) return STARKV_ERR_INVALID_ARG;
   AppendTarget tgt{nullptr, block_tables, positions, desc->max_blocks_per_seq, desc->num_blocks, append_status};
-  AppendPlan ap;
+  AppendPlan ap{};
   st = plan_append(desc, batch, k, v, A_K, A_V, tgt, k_cache, v_cache, &ap);
   if (st != STARKV_OK) return st;
   return decode_impl(desc, batch, max_seq_len, q, B_K, B_V, k_cache, v_cache, block_tables, seq_lens, scale,
@@ -919,7 +919,7 @@ starkv_status starkv_append_decode_host(const starkv_layer_desc* desc, int32_t b
   if (!staging || staging_bytes < st.total || (reinterpret_cast<uintptr_t>(staging) & 255u))
     return STARKV_ERR_WORKSPACE;
   // the decode's own argument checks run before any copy is enqueued
-  DecodePlan pl;
+  DecodePlan pl{};
   starkv_status ps = make_plan(desc, batch, max_seq_len, &pl);
   if (ps != STARKV_OK) return ps;
   if (!(std::isfinite(scale) && scale > 0.f)) return STARKV_ERR_INVALID_ARG;
@@ -1144,7 +1144,7 @@ starkv_status chunk_prefill(const ChunkPlan& c, const void* q, const void* B_K, 
   ChunkTableParams tp{starts, row_offsets, vs_seq, vs_row0, vs_nrows, vs_len, c.n_seqs, c.nv_max, c.log2nq};
   if (launch(chunk_table_kernel, dim3(1), dim3(256), 0, s, 1, tp) != cudaSuccess) return STARKV_ERR_CUDA;
 
-  AbsorbParams ap;
+  AbsorbParams ap{};
   std::memset(&ap, 0, sizeof(ap));
   ap.q = static_cast<const __half*>(q);
   ap.B_K = static_cast<const __half*>(B_K);
@@ -1162,7 +1162,7 @@ starkv_status chunk_prefill(const ChunkPlan& c, const void* q, const void* B_K, 
   ap.vs_row0 = vs_row0; ap.vs_nrows = vs_nrows; ap.log2nq = c.log2nq;
   if (launch_prep(c.d, nullptr, &ap, c.nv_max << c.log2nq, s) != STARKV_OK) return STARKV_ERR_CUDA;
 
-  KPassChunkParams kp;
+  KPassChunkParams kp{};
   kp.tables = block_tables; kp.vs_seq = vs_seq; kp.vs_nrows = vs_nrows; kp.teff = teff; kp.prefix = prefix;
   kp.logits = logits; kp.mpart = mpart; kp.status = status;
   kp.B = c.nv_max; kp.MB = c.MB; kp.NB = c.NB; kp.t_pad = c.t_pad;
@@ -1176,7 +1176,7 @@ starkv_status chunk_prefill(const ChunkPlan& c, const void* q, const void* B_K, 
   if (launch(kpass_chunk_kernel, dim3(c.k_ctas), dim3(kKTCThreads), c.k_smem, s, 1, kmap, qmap, kp) != cudaSuccess)
     return STARKV_ERR_CUDA;
 
-  VPassParams vp;
+  VPassParams vp{};
   std::memset(&vp, 0, sizeof(vp));
   vp.tables = block_tables; vp.row_seq = vs_seq; vp.teff = teff; vp.prefix = prefix; vp.logits = logits;
   vp.mpart = mpart; vp.zpart = zpart; vp.lpart = lpart; vp.status = status;
@@ -1191,7 +1191,7 @@ starkv_status chunk_prefill(const ChunkPlan& c, const void* q, const void* B_K, 
       cudaSuccess)
     return STARKV_ERR_CUDA;
 
-  FinishParams fp;
+  FinishParams fp{};
   std::memset(&fp, 0, sizeof(fp));
   fp.out = static_cast<__half*>(out);
   fp.lpart = lpart; fp.prefix = prefix;
@@ -1211,9 +1211,9 @@ starkv_status chunk_prefill(const ChunkPlan& c, const void* q, const void* B_K, 
 
 size_t starkv_prefill_workspace_bytes(const starkv_layer_desc* desc, int32_t n_seqs, int32_t n_rows,
                                       int32_t max_seq_len) {
-  DecodePlan pl;
+  DecodePlan pl{};
   if (n_seqs < 0 || n_rows < 0 || make_plan(desc, n_rows, max_seq_len, &pl) != STARKV_OK) return 0;
-  ChunkPlan cp;
+  ChunkPlan cp{};
   if (chunk_eligible(desc)) return make_chunk_plan(desc, n_seqs, n_rows, max_seq_len, &cp) == STARKV_OK ? cp.total : 0;
   return prefill_rows_offset(pl) + align_up(static_cast<size_t>(n_rows) * 8, 256);
 }
@@ -1223,7 +1223,7 @@ starkv_status starkv_paged_prefill(const starkv_layer_desc* desc, int32_t n_seqs
                                    const void* v_cache, const int32_t* block_tables, const int32_t* starts,
                                    const int32_t* row_offsets, float scale, void* workspace, size_t workspace_bytes,
                                    void* out, void* stream) {
-  DecodePlan pl;
+  DecodePlan pl{};
   if (n_seqs < 0 || n_rows < 0) return STARKV_ERR_INVALID_ARG;
   starkv_status st = make_plan(desc, n_rows, max_seq_len, &pl);
   if (st != STARKV_OK) return st;
@@ -1232,7 +1232,7 @@ starkv_status starkv_paged_prefill(const starkv_layer_desc* desc, int32_t n_seqs
       (reinterpret_cast<uintptr_t>(row_offsets) & 3u))
     return STARKV_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  ChunkPlan cp;
+  ChunkPlan cp{};
   if (chunk_eligible(desc)) {
     if (make_chunk_plan(desc, n_seqs, n_rows, max_seq_len, &cp) != STARKV_OK) return STARKV_ERR_UNSUPPORTED;
     if (!workspace || workspace_bytes < cp.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -1303,7 +1303,7 @@ starkv_status starkv_paged_decode_static(const starkv_layer_desc* desc, int32_t 
                                          const void* q, const void* B_K, const void* B_V, const void* k_cache,
                                          const void* v_cache, const int32_t* block_tables,
                                          const int32_t* seq_lens, float scale, void* out, void* stream) {
-  DecodePlan pl;
+  DecodePlan pl{};
   starkv_status st = make_plan(desc, batch, max_seq_len, &pl);
   if (st != STARKV_OK) return st;
   if (pl.ws.total_bytes > STARKV_STATIC_WS_BYTES) return STARKV_ERR_WORKSPACE;
