@@ -1609,7 +1609,8 @@ struct FinishParams {
   int log2nq, Hv;
 };
 
-constexpr int kFinThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 convert, then epilogue
+constexpr int kFinThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 convert; warps 2..5 drain TMEM
+constexpr int kFinConv = kFinThreads - 64;
 constexpr int kFinKC = 64;        // rows of R per stage
 constexpr int kFinZBox = 32;      // partial rows per TMA box
 constexpr int kFinMaxRows = 256;  // sequences per batch tile at most
@@ -1658,7 +1659,7 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
   const int n_stages = k1 > k0 ? (k1 - k0 + kFinKC - 1) / kFinKC : 0;
 
   if (tid == 0) {
-    for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&conv[s], 128); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&conv[s], kFinConv); mbar_init(&empty[s], 1); }
     mbar_init(done, 1);
     fence_mbar_init();
   }
@@ -1726,10 +1727,10 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
     }
   } else {
     // ------------------------------------------------------------ converters
-    const int et = tid - 64;                 // 0..127
+    const int et = tid - 64;                 // 0 .. kFinConv-1
     // each sequence's partial rows (relative to the tile's first slot) and 1/L;
     // L sums the per-segment normalisers in segment order
-    for (int bl = et; bl < p.npad; bl += 128) {
+    for (int bl = et; bl < p.npad; bl += kFinConv) {
       int32_t row = 0, nseg = 0;
       float il = 0.f;
       const int vb = bl >> p.log2nq, qi = bl & (nq - 1);   // (virtual) sequence of the tile, its row
@@ -1741,7 +1742,14 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
           const int col = p.vs_row0 ? (h << p.log2nq) + qi : h;
           const int lw = p.vs_row0 ? p.Hv : p.H;
           float Ls = 0.f;
-          for (int32_t i = i0; i <= i1; ++i) Ls += p.lpart[static_cast<size_t>(b + i) * lw + col];
+          for (int32_t i = i0; i <= i1; i += 4) {   // four loads issued before they are added in order
+            float l4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) l4[u] = i + u <= i1 ? p.lpart[static_cast<size_t>(b + i + u) * lw + col] : 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (i + u <= i1) Ls += l4[u];
+          }
           il = 1.f / Ls;
           row = ((b + i0 - slot_lo) << p.log2nq) + qi;
           nseg = i1 - i0 + 1;
@@ -1752,7 +1760,7 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
       s_nseg[bl] = nseg;
       s_il[bl] = il;
     }
-    named_bar_sync(1, 128);
+    named_bar_sync(1, kFinConv);
     for (int i = 0; i < n_stages; ++i) {
       const int s = i % S;
       const bool landed = mbar_wait(&full[s], (i / S) & 1);
@@ -1761,7 +1769,7 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
       uint8_t* hi_t = st + a_bytes;
       const uint8_t* zt = st + a_bytes + 2u * half_bytes;
       // item = (sequence row bl of the tile, 8-value chunk c of the stage's 64 rows of R)
-      for (int item = et; item < p.npad * 8; item += 128) {
+      for (int item = et; item < p.npad * 8; item += kFinConv) {
         const int bl = item >> 3, c = item & 7;
         float z[8];
 #pragma unroll
@@ -1802,7 +1810,7 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
   __syncthreads();
   if (!mbar_wait(done, 0)) ok = false;
   tc_fence_after();
-  if (warp >= 2) {
+  if (warp >= 2 && warp < 6) {
     const int q = warp & 3;
     const int row = q * 32 + lane;
     for (int c0 = 0; c0 < p.npad; c0 += 16) {

@@ -27,7 +27,7 @@
 #define STARKV_KTC_CTAS_PER_SM 3
 #endif
 #ifndef STARKV_KTC_SMEM_BYTES
-#define STARKV_KTC_SMEM_BYTES (212 * 1024)   // shared memory of the K-pass CTAs on one SM
+#define STARKV_KTC_SMEM_BYTES (224 * 1024)   // shared memory of the K-pass CTAs on one SM (228 KB less 1 KB per CTA)
 #endif
 #ifndef STARKV_K_RING_BYTES
 #define STARKV_K_RING_BYTES (200 * 1024 / STARKV_K_CTAS_PER_SM)
@@ -230,18 +230,25 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
       int nacc = 512 / (ctas * p.ktc_nmma);
       if (nacc > kKTCMaxAcc) nacc = kKTCMaxAcc;
       if (nacc < 2) continue;
-      for (int nbs = 2; nbs >= 1 && !p.ktc; --nbs) {
+      // one or two query-tile slots: two hide the reload at a segment boundary, one
+      // leaves room for another ring stage (more bytes in flight); a CTA crosses
+      // only a few segment boundaries, so the extra stage wins when there is one
+      int best_stages = 0, best_nbs = 0;
+      uint32_t best_fixed = 0;
+      for (int nbs = 2; nbs >= 1; --nbs) {
         // query slots, then full/empty per stage, bfull/bempty[2], tfull/tempty per accumulator, mmadone
         const uint32_t fixed = 1024u + nbs * p.ktc_b_bytes + (4 + 2 * kKTCMaxAcc + 1) * 8u;
         const uint32_t budget = static_cast<uint32_t>(STARKV_KTC_SMEM_BYTES) / ctas - (ctas > 1 ? 1024u : 0u);
         if (budget <= fixed) continue;
         int stages = static_cast<int>((budget - fixed) / (p.ktc_a_bytes + 16u));
         if (stages > 12) stages = 12;
-        if (stages < (ctas > 1 ? 3 : 4)) continue;
+        if (stages > best_stages) { best_stages = stages; best_nbs = nbs; best_fixed = fixed; }
+      }
+      if (best_stages >= (ctas > 1 ? 3 : 4)) {
         p.ktc = true;
-        p.ktc_nacc = nacc; p.ktc_nbs = nbs; p.ktc_stages = stages;
+        p.ktc_nacc = nacc; p.ktc_nbs = best_nbs; p.ktc_stages = best_stages;
         p.ktc_tmem = static_cast<uint32_t>(pow2_ceil(nacc * p.ktc_nmma < 32 ? 32 : nacc * p.ktc_nmma));
-        p.ktc_smem = fixed + static_cast<size_t>(stages) * (p.ktc_a_bytes + 16u);
+        p.ktc_smem = best_fixed + static_cast<size_t>(best_stages) * (p.ktc_a_bytes + 16u);
         p.k_ctas = sms * ctas;
       }
     }
