@@ -519,6 +519,10 @@ def run_prefill(args):
     S.load_library()
     N = args.prefill_chunk
     wl = W.workload(args.workload)
+    if args.batch:   # profiling only: fewer sequences of a uniform length
+        seq = args.seq or wl.max_seq_len
+        wl = W.Workload(f"{wl.name} (override: batch {args.batch}, length {seq})", wl.seed, args.batch, wl.layers[:1],
+                        np.full(args.batch, seq, dtype=np.int64), append=False)
     wl = W.Workload(wl.name + f" (chunked prefill: last {N} tokens)", wl.seed, wl.batch, wl.layers[:1],
                     wl.seq_lens.copy(), append=False)
     L = D.device_layer(wl, 0)
