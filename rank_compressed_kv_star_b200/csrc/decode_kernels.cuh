@@ -1139,7 +1139,8 @@ kpass_chunk_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
       if (lane == 0) mbar_arrive(&tempty[ai]);
       if (++ai == p.nacc) { ai = 0; ++au; }
       const int kv = g * 8 + jl;                     // KV head of this lane's row
-      if (t < nt) {
+      {
+        // every slot of the page gets a logit: -inf past the sequence end too
         const int32_t tabs = pg * kBlock + t;
         const int32_t nrows = p.vs_nrows[v];
         const int32_t rel = tabs - (p.teff[v] - nrows);   // rows i >= rel see this token
@@ -1147,7 +1148,7 @@ kpass_chunk_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const int i = c & nq1;
-          o[c] = (i < nrows && i >= rel) ? xs[c] : -INFINITY;
+          o[c] = (t < nt && i < nrows && i >= rel) ? xs[c] : -INFINITY;
           m[c] = fmaxf(m[c], o[c]);
         }
         const int vh = kv * 16;                       // 16 consecutive virtual heads, in one group
@@ -1186,13 +1187,122 @@ kpass_chunk_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
   }
 }
 
+// ============================================================ chunk weights
+// Read-once chunked prefill, between the K and V passes: the attention
+// weights of every virtual head, once.  CTA (v, pc, vg) owns pages
+// [pc * kCwPages, (pc + 1) * kCwPages) of virtual sequence v for the lw
+// virtual heads of group vg.  M = the max over the K pass's segments of v;
+// w = fp16(exp2(s - M)) (0 for a logit of -inf: past the row's causal limit,
+// or no row).  A page's 16 x lw weights go, in the V pass's B-operand layout
+// (K-major core matrices of 8 tokens x 8 heads, i.e. halves [t / 8][head][t %
+// 8]), to the page's tile of wts.  The normaliser partial
+// of the CTA (the rounded weights summed per page lane in token order, then
+// over the page lanes in order) goes to lwpart[v][pc][Hv].
+constexpr int kCwPages = 32;
+struct ChunkWeightsParams {
+  const float* logits;        // [B][n_vg][t_pad][lw]
+  __half* wts;                // [B][n_vg][t_pad][lw] fp16: each page's 16 x lw tile in the B-operand layout
+  const float* mpart;         // [k_slots][Hv]
+  const int32_t* teff;        // [B]
+  const int32_t* prefix;      // [B+1]
+  float* lwpart;              // [B][n_pc][Hv]: per page chunk sums of the weights of each virtual head
+  int B, Hv, n_vg, lw, log2lw, t_pad, k_grid, n_pc;
+};
+
+// Thread = (page lane, 4 consecutive virtual heads): 16 float4 loads take a
+// page's logits of its heads, and 8 16-byte stores write their weights.
+// Hv is a multiple of lw (both powers of two), so every head is live; the K
+// pass wrote -inf for every logit that has no weight (past a row's causal
+// limit or the sequence end), and ex2 of -inf is exactly 0.
+__global__ void __launch_bounds__(256) chunk_weights_kernel(ChunkWeightsParams p) {
+  __shared__ float4 sL[256];
+  griddep_wait();
+  griddep_launch_dependents();
+  const int v = blockIdx.x, pc = blockIdx.y, vg = blockIdx.z, tid = threadIdx.x;
+  const int log2tpp = p.log2lw - 2;                 // threads per page: lw / 4
+  const int c4 = tid & ((1 << log2tpp) - 1), lane_pg = tid >> log2tpp;
+  const int gp = 256 >> log2tpp;                    // pages handled side by side
+  const int32_t T = p.teff[v];
+  const int n_pages = T > 0 ? (T + kBlock - 1) / kBlock : 0;
+  const int pg0 = pc * kCwPages, pg1 = min(n_pages, pg0 + kCwPages);   // uniform over the CTA
+  const int hcol = vg * p.lw + 4 * c4;
+  float M[4] = {0.f, 0.f, 0.f, 0.f};
+  if (pg0 < pg1) {
+    Partition ptk;
+    ptk.P = p.prefix[p.B];
+    ptk.G = static_cast<int32_t>(ptk.P < p.k_grid ? ptk.P : p.k_grid);
+    const int32_t i0 = part_owner(p.prefix[v], ptk), i1 = part_owner(p.prefix[v + 1] - 1, ptk);
+    float4 m = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    for (int32_t i = i0; i <= i1; ++i) {
+      const float4 x = *reinterpret_cast<const float4*>(p.mpart + static_cast<size_t>(v + i) * p.Hv + hcol);
+      m = make_float4(fmaxf(m.x, x.x), fmaxf(m.y, x.y), fmaxf(m.z, x.z), fmaxf(m.w, x.w));
+    }
+    // a head with no visible token keeps M = 0: all its logits are -inf
+    M[0] = m.x > -INFINITY ? m.x : 0.f;
+    M[1] = m.y > -INFINITY ? m.y : 0.f;
+    M[2] = m.z > -INFINITY ? m.z : 0.f;
+    M[3] = m.w > -INFINITY ? m.w : 0.f;
+  }
+  const size_t seq_off = (static_cast<size_t>(v) * p.n_vg + vg) * p.t_pad * p.lw;
+  const float* seq_logits = p.logits + seq_off;
+  __half* seq_wts = p.wts + seq_off;
+  const int row4 = p.lw >> 2;                       // float4 per token row
+  float L[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int pgb = pg0; pgb < pg1; pgb += gp) {
+    const int pg = pgb + lane_pg;
+    const bool have = pg < pg1;
+    const float4* lt = reinterpret_cast<const float4*>(seq_logits + static_cast<size_t>(pg) * kBlock * p.lw) + c4;
+    float4 x[kBlock];
+#pragma unroll
+    for (int t = 0; t < kBlock; ++t)
+      x[t] = have ? lt[t * row4] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    if (have) {
+      uint32_t w[4][kBlock / 2];
+#pragma unroll
+      for (int t2 = 0; t2 < kBlock / 2; ++t2) {
+        const float4 a = x[2 * t2], b = x[2 * t2 + 1];
+        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half2 h = __floats2half2_rn(ex2_approx(av[j] - M[j]), ex2_approx(bv[j] - M[j]));
+          const float2 f = __half22float2(h);
+          L[j] += f.x;
+          L[j] += f.y;
+          w[j][t2] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+      }
+      uint8_t* dst = reinterpret_cast<uint8_t*>(seq_wts + static_cast<size_t>(pg) * kBlock * p.lw);
+      uint8_t* lo = dst + (4 * c4) * 16;
+      uint8_t* hi = dst + p.lw * 16 + (4 * c4) * 16;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        *reinterpret_cast<uint4*>(lo + j * 16) = make_uint4(w[j][0], w[j][1], w[j][2], w[j][3]);
+        *reinterpret_cast<uint4*>(hi + j * 16) = make_uint4(w[j][4], w[j][5], w[j][6], w[j][7]);
+      }
+    }
+  }
+  sL[tid] = make_float4(L[0], L[1], L[2], L[3]);
+  __syncthreads();
+  if (lane_pg == 0) {
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < gp; ++j) {
+      const float4 x = sL[(j << log2tpp) + c4];
+      s.x += x.x; s.y += x.y; s.z += x.z; s.w += x.w;
+    }
+    *reinterpret_cast<float4*>(p.lwpart + (static_cast<size_t>(v) * p.n_pc + pc) * p.Hv + hcol) = s;
+  }
+}
+
 // ======================================================================= vpass
 // Z^T (R-range rows x heads) += C_V^T (R-range x 16 tokens) . P^T (16 x heads)
 // per page, with A = the V page slice as an MN-major 128B-swizzled operand
 // (exactly the layout TMA writes for 64-element x 16-token boxes) and B = the
 // fp16 attention weights in a K-major, unswizzled layout written by the
-// P warps.  The accumulator lives in tensor memory: one 128-lane x npad-column
-// block per 128 rows of the R range.
+// P warps (chunked prefill: by chunk_weights_kernel).  The accumulator lives in
+// tensor memory: one 128-lane x npad-column block per 128 rows of the R range.
+// A ring stage holds up to pps consecutive pages of one segment, so that the
+// per-stage work of the single issuing threads (barrier waits, bookkeeping)
+// is shared by several pages' copies and MMAs.
 struct VPassParams {
   const int32_t* tables;
   const int32_t* row_seq;   // [B] sequence of each row, or null
@@ -1217,7 +1327,10 @@ struct VPassParams {
   // partials of virtual head (h, i) sit at row (slot * nq + i) of head h
   int Hv, n_vg, log2nq;
   int lw;                 // chunk mode: logits row width = virtual heads per group (npad)
+  int pps;                // pages per ring stage (1..kMaxPPS)
+  const __half* wts;      // chunk mode: [B][n_vg][t_pad][lw] fp16 weights, each page's tile in the B layout
 };
+constexpr int kMaxPPS = 8;
 
 constexpr int kVThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 weights + epilogue
 constexpr int32_t kFirst = 1, kLast = 2;
@@ -1227,11 +1340,12 @@ __global__ void __launch_bounds__(kVThreads, 1)
 vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int S = p.stages;
-  uint8_t* vtiles = smem;                                               // S x vtile_bytes (1024-aligned)
-  uint8_t* ltiles = vtiles + static_cast<size_t>(S) * p.vtile_bytes;    // S x ltile_bytes
-  uint8_t* ptiles = ltiles + static_cast<size_t>(S) * p.ltile_bytes;    // S x ptile_bytes
-  StageMeta* meta = reinterpret_cast<StageMeta*>(ptiles + static_cast<size_t>(S) * p.ptile_bytes);
+  const int S = p.stages, PPS = p.pps;
+  const uint32_t vstage = PPS * p.vtile_bytes, lstage = PPS * p.ltile_bytes, pstage = PPS * p.ptile_bytes;
+  uint8_t* vtiles = smem;                                               // S x vstage (1024-aligned)
+  uint8_t* ltiles = vtiles + static_cast<size_t>(S) * vstage;           // S x lstage
+  uint8_t* ptiles = ltiles + static_cast<size_t>(S) * lstage;           // S x pstage
+  StageMeta* meta = reinterpret_cast<StageMeta*>(ptiles + static_cast<size_t>(S) * pstage);
   uint64_t* full = reinterpret_cast<uint64_t*>(meta + S);
   uint64_t* pready = full + S;
   uint64_t* empty = pready + S;
@@ -1287,56 +1401,76 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
     // The whole warp walks the pages; lane i reads ahead the block-table entry
     // of page cbase + i, so lane 0 issues copies without a dependent global
     // load per page.  Sequence bounds are reloaded only when the walk enters
-    // the next sequence.
+    // the next sequence.  A stage takes the next min(pps, pages left in the
+    // segment) pages: one box per page, one bulk copy for their weights.
     if (lane == 0) prefetch_tensormap(&vmap);
     const uint64_t pol_codes = policy_evict_first();
     const uint64_t pol_logits = policy_evict_first();
-    uint32_t k = 0;
+    uint32_t k = 0;             // stages issued
+    int s = 0;                  // ring slot of stage k
+    uint32_t ph = 0;            // parity of that slot's current use
     bool ok = true;
     int32_t b = seq_of_page(p.prefix, p.B, p0);
     int32_t sbeg = p.prefix[b], send = p.prefix[b + 1], T = p.teff[b];
     int64_t cbase = -64;
     int32_t cphys = 0;
     const int c_base = rr * (p.r_range / 64);
-    for (int64_t pg_g = p0; pg_g < p1; ++pg_g, ++k) {
+    for (int64_t pg_g = p0; pg_g < p1;) {
       while (send <= pg_g) { ++b; sbeg = send; send = p.prefix[b + 1]; T = p.teff[b]; }
-      if (pg_g >= cbase + 32) {
+      const int32_t pg = static_cast<int32_t>(pg_g - sbeg);
+      const int64_t left = (send < p1 ? static_cast<int64_t>(send) : p1) - pg_g;   // pages left in the segment
+      const int np = left < PPS ? static_cast<int>(left) : PPS;
+      if (pg_g + np > cbase + 32) {
         cbase = pg_g;
         const int64_t xi = pg_g + lane;
         int32_t bi = b;
         while (bi < p.B - 1 && p.prefix[bi + 1] <= xi) ++bi;
         cphys = xi < p1 ? table_row(p.tables, p.row_seq, bi, p.MB)[static_cast<int32_t>(xi - p.prefix[bi])] : 0;
       }
-      int32_t phys = __shfl_sync(0xffffffffu, cphys, static_cast<int>(pg_g - cbase));
+      const int w0 = static_cast<int>(pg_g - cbase);
+      int32_t phys[kMaxPPS];
+#pragma unroll
+      for (int j = 0; j < kMaxPPS; ++j) phys[j] = __shfl_sync(0xffffffffu, cphys, (w0 + j) & 31);
       if (lane == 0) {
-        const int32_t pg = static_cast<int32_t>(pg_g - sbeg);
-        const int32_t npg = send - sbeg;
-        if (phys < 0 || phys >= p.NB) { set_flag(p.status, STARKV_FLAG_BAD_BLOCK_ID); phys = 0; }
-        const int s = k % S;
-        if (k >= static_cast<uint32_t>(S) && !mbar_wait(&empty[s], ((k / S) - 1) & 1)) {
+        if (k >= static_cast<uint32_t>(S) && !mbar_wait(&empty[s], ph ^ 1u)) {
           ok = false;
         } else {
           int32_t fl = 0;
           if (pg_g == p0 || pg == 0) fl |= kFirst;
-          if (pg_g == p1 - 1 || pg == npg - 1) fl |= kLast;
-          meta[s] = StageMeta{b, pg * kBlock, min(kBlock, T - pg * kBlock), fl};
-          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(p.n_chunks) * 2048u + p.ltile_bytes);
-          // the page's R range in one box of n_chunks 64-code blocks
-          tma_load_3d(vtiles + static_cast<size_t>(s) * p.vtile_bytes, &vmap, 0, phys * kBlock, c_base, &full[s],
-                      pol_codes);
-          const float* lsrc =
-              kChunk ? p.logits + ((static_cast<size_t>(b) * p.n_vg + vg) * p.t_pad + pg * kBlock) * p.lw
-                     : p.logits + (static_cast<size_t>(b) * p.t_pad + pg * kBlock) * p.H;
-          bulk_g2s(ltiles + static_cast<size_t>(s) * p.ltile_bytes, lsrc, p.ltile_bytes, &full[s], pol_logits);
+          if (np == left) fl |= kLast;   // the stage ends the segment
+          const int32_t t0 = pg * kBlock;
+          meta[s] = StageMeta{b, t0, min(np * kBlock, T - t0), fl};
+          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(np) * (static_cast<uint32_t>(p.n_chunks) * 2048u +
+                                                                       (kChunk ? p.ptile_bytes : p.ltile_bytes)));
+          uint8_t* vt = vtiles + static_cast<size_t>(s) * vstage;
+#pragma unroll
+          for (int j = 0; j < kMaxPPS; ++j) {
+            if (j < np) {
+              int32_t pj = phys[j];
+              if (pj < 0 || pj >= p.NB) { set_flag(p.status, STARKV_FLAG_BAD_BLOCK_ID); pj = 0; }
+              // the page's R range in one box of n_chunks 64-code blocks
+              tma_load_3d(vt + j * p.vtile_bytes, &vmap, 0, pj * kBlock, c_base, &full[s], pol_codes);
+            }
+          }
+          if constexpr (kChunk) {
+            // the pages' weights, already in the B-operand layout (chunk_weights_kernel)
+            const __half* wsrc = p.wts + ((static_cast<size_t>(b) * p.n_vg + vg) * p.t_pad + t0) * p.lw;
+            bulk_g2s(ptiles + static_cast<size_t>(s) * pstage, wsrc, np * p.ptile_bytes, &full[s], pol_logits);
+          } else {
+            bulk_g2s(ltiles + static_cast<size_t>(s) * lstage, p.logits + (static_cast<size_t>(b) * p.t_pad + t0) * p.H,
+                     np * p.ltile_bytes, &full[s], pol_logits);
+          }
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
+      pg_g += np;
+      ++k;
+      if (++s == S) { s = 0; ph ^= 1u; }
     }
     if (lane == 0) {
       if (ok) {
-        const int s = k % S;
-        if (k >= static_cast<uint32_t>(S) && !mbar_wait(&empty[s], ((k / S) - 1) & 1)) ok = false;
+        if (k >= static_cast<uint32_t>(S) && !mbar_wait(&empty[s], ph ^ 1u)) ok = false;
         if (ok) { meta[s] = StageMeta{-1, 0, 0, 0}; mbar_arrive(&full[s]); }
       }
       if (!ok) {
@@ -1353,11 +1487,17 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(128, p.npad, /*a_mn_major=*/true, /*b_mn_major=*/false);
       const uint32_t lbo_b = static_cast<uint32_t>(p.npad / 8) * 128u;
+      // descriptors of ring slot 0's first page; the start address field
+      // (address / 16, 14 bits) advances by plain addition: shared memory
+      // addresses stay below 256 KB, so the sum never carries out of it
+      const uint64_t adesc0 = smem_desc(smem_u32(vtiles), 2048u, 1024u, kSwizzle128B);
+      const uint64_t bdesc0 = smem_desc(smem_u32(ptiles), lbo_b, 128u, kSwizzleNone);
       uint32_t seg = 0;
       uint32_t accumulate = 0;
-      for (uint32_t k = 0;; ++k) {
-        const int s = k % S;
-        if (!mbar_wait(&pready[s], (k / S) & 1) || abort_flag) { set_timeout(p.status, kSiteVPready); break; }
+      int s = 0;
+      uint32_t ph = 0;
+      for (;;) {
+        if (!mbar_wait(&pready[s], ph) || abort_flag) { set_timeout(p.status, kSiteVPready); break; }
         const StageMeta mt = meta[s];
         if (mt.b < 0) break;
         if (mt.flags & kFirst) {
@@ -1365,16 +1505,20 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
           accumulate = 0;
         }
         tc_fence_after();
-        const uint32_t va = smem_u32(vtiles + static_cast<size_t>(s) * p.vtile_bytes);
-        const uint32_t pa = smem_u32(ptiles + static_cast<size_t>(s) * p.ptile_bytes);
-        const uint64_t bdesc = smem_desc(pa, lbo_b, 128u, kSwizzleNone);
-        for (int m = 0; m < p.n_mtiles; ++m) {
-          const uint64_t adesc = smem_desc(va + m * 4096u, 2048u, 1024u, kSwizzle128B);
-          umma_f16_ss(taddr + static_cast<uint32_t>(m * p.npad), adesc, bdesc, idesc, accumulate);
+        const int np = (mt.nt + kBlock - 1) >> 4;
+        const uint64_t as = adesc0 + ((static_cast<uint32_t>(s) * vstage) >> 4);
+        const uint64_t bs = bdesc0 + ((static_cast<uint32_t>(s) * pstage) >> 4);
+        for (int j = 0; j < np; ++j) {
+          const uint64_t bj = bs + ((static_cast<uint32_t>(j) * p.ptile_bytes) >> 4);
+          const uint64_t aj = as + ((static_cast<uint32_t>(j) * p.vtile_bytes) >> 4);
+          for (int m = 0; m < p.n_mtiles; ++m)
+            umma_f16_ss(taddr + static_cast<uint32_t>(m * p.npad), aj + static_cast<uint32_t>(m * 256), bj, idesc,
+                        accumulate);
+          accumulate = 1;
         }
-        accumulate = 1;
         umma_commit(&empty[s]);
         if (mt.flags & kLast) { umma_commit(zdone); ++seg; }
+        if (++s == S) { s = 0; ph ^= 1u; }
       }
       // every MMA issued has completed before the CTA can release TMEM
       umma_commit(mdone);
@@ -1390,13 +1534,16 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
     const int t_w0 = et / p.npad;
     const int t_step = 128 / p.npad;
     float lsum = 0.f;
-    float lsum2[2] = {0.f, 0.f};           // chunk mode: columns et and et + 128
     uint32_t seg = 0, pphase = 0;
     const uint64_t keep = policy_evict_last();   // Z partials: read back by the finish kernel
-    for (uint32_t k = 0;; ++k) {
-      const int s = k % S;
+    int s_next = 0;
+    uint32_t ph_next = 0;
+    for (;;) {
+      const int s = s_next;
+      const uint32_t ph = ph_next;
+      if (++s_next == S) { s_next = 0; ph_next ^= 1u; }
       // warp-uniform decisions: the TMEM loads of the epilogue are .sync.aligned
-      const bool landed = mbar_wait(&full[s], (k / S) & 1);
+      const bool landed = mbar_wait(&full[s], ph);
       if (!__all_sync(0xffffffffu, landed && !abort_flag)) {
         set_timeout(p.status, kSiteVFull);
         abort_flag = 1;
@@ -1404,7 +1551,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
       }
       const StageMeta mt = meta[s];
       if (mt.b < 0) { mbar_arrive(&pready[s]); break; }
-      if (mt.flags & kFirst) {
+      if (!kChunk && (mt.flags & kFirst)) {   // (chunk mode: the weights arrive with the stage)
         // everyone is done with the previous segment's max
         if (!group_sync(pbar, pphase)) { set_timeout(p.status, kSiteVFull); abort_flag = 1; break; }
         // max of the sequence's logits: the split reduction over its K-pass segments
@@ -1412,13 +1559,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
         const int32_t i0 = part_owner(f0, ptk), i1 = part_owner(f1 - 1, ptk);
         for (int h = et; h < p.npad; h += 128) {
           float M = 0.f;
-          if constexpr (kChunk) {
-            const int col = vg * p.lw + h;
-            if (col < p.Hv) {
-              M = -INFINITY;   // stays -inf for a virtual head with no visible token (weights 0)
-              for (int32_t i = i0; i <= i1; ++i) M = fmaxf(M, p.mpart[static_cast<size_t>(mt.b + i) * p.Hv + col]);
-            }
-          } else if (h < p.H) {
+          if (h < p.H) {
             M = -INFINITY;
             for (int32_t i = i0; i <= i1; ++i) M = fmaxf(M, p.mpart[static_cast<size_t>(mt.b + i) * p.H + h]);
           }
@@ -1426,57 +1567,39 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
         }
         if (!group_sync(pbar, pphase)) { set_timeout(p.status, kSiteVFull); abort_flag = 1; break; }
         lsum = 0.f;
-        lsum2[0] = lsum2[1] = 0.f;
       }
-      const float* lt = reinterpret_cast<const float*>(ltiles + static_cast<size_t>(s) * p.ltile_bytes);
-      uint8_t* pt_s = ptiles + static_cast<size_t>(s) * p.ptile_bytes;
-      if constexpr (kChunk) {
-        // columns et and et + 128, all 16 tokens; a logit of -inf (past a row's
-        // causal limit, or a virtual head with no row) weighs exactly 0
-#pragma unroll
-        for (int k2 = 0; k2 < 2; ++k2) {
-          const int col = et + 128 * k2;
-          if (col < p.npad) {
-            const float mh = sM[col];
-            const bool live = vg * p.lw + col < p.Hv;
-            float acc = 0.f;
-            for (int t = 0; t < kBlock; ++t) {
-              __half w = __float2half_rn(0.f);
-              if (live && t < mt.nt) {
-                const float x = lt[t * p.lw + col];
-                if (x > -INFINITY) w = __float2half_rn(exp2f(x - mh));
-              }
-              acc += __half2float(w);
-              const uint32_t off = static_cast<uint32_t>(t >> 3) * lbo_b + static_cast<uint32_t>(col >> 3) * 128u +
-                                   static_cast<uint32_t>(col & 7) * 16u + static_cast<uint32_t>(t & 7) * 2u;
-              *reinterpret_cast<__half*>(pt_s + off) = w;
-            }
-            lsum2[k2] += acc;
+      const int np = (mt.nt + kBlock - 1) >> 4;
+      const int ntl = mt.nt - ((np - 1) << 4);   // valid tokens of the stage's last page
+      if constexpr (!kChunk) {
+        const float m_h = sM[h_w];
+        for (int j = 0; j < np; ++j) {
+          const float* lt = reinterpret_cast<const float*>(ltiles + static_cast<size_t>(s) * lstage +
+                                                           static_cast<size_t>(j) * p.ltile_bytes);
+          uint8_t* pt_j = ptiles + static_cast<size_t>(s) * pstage + static_cast<size_t>(j) * p.ptile_bytes;
+          const int ntj = j == np - 1 ? ntl : kBlock;
+          for (int t = t_w0; t < kBlock; t += t_step) {
+            // unnormalised weight exp2(s - M) <= 1, rounded to fp16 for the MMA; the
+            // normaliser sums exactly the rounded weights
+            __half w = __float2half_rn(0.f);
+            if (t < ntj && h_w < p.H) w = __float2half_rn(exp2f(lt[t * p.H + h_w] - m_h));
+            lsum += __half2float(w);
+            const uint32_t off = static_cast<uint32_t>(t >> 3) * lbo_b + static_cast<uint32_t>(h_w >> 3) * 128u +
+                                 static_cast<uint32_t>(h_w & 7) * 16u + static_cast<uint32_t>(t & 7) * 2u;
+            *reinterpret_cast<__half*>(pt_j + off) = w;
           }
         }
-      } else {
-        const float m_h = sM[h_w];
-        for (int t = t_w0; t < kBlock; t += t_step) {
-          // unnormalised weight exp2(s - M) <= 1, rounded to fp16 for the MMA; the
-          // normaliser sums exactly the rounded weights
-          __half w = __float2half_rn(0.f);
-          if (t < mt.nt && h_w < p.H) w = __float2half_rn(exp2f(lt[t * p.H + h_w] - m_h));
-          lsum += __half2float(w);
-          const uint32_t off = static_cast<uint32_t>(t >> 3) * lbo_b + static_cast<uint32_t>(h_w >> 3) * 128u +
-                               static_cast<uint32_t>(h_w & 7) * 16u + static_cast<uint32_t>(t & 7) * 2u;
-          *reinterpret_cast<__half*>(pt_s + off) = w;
-        }
       }
-      if (mt.nt < kBlock) {
-        // tokens past the sequence end: zero their rows of the V tile so that
-        // whatever the unused slots hold (NaN included) contributes exactly 0
-        uint8_t* vt = vtiles + static_cast<size_t>(s) * p.vtile_bytes;
-        const int nrows = kBlock - mt.nt;
+      if (ntl < kBlock) {
+        // tokens past the sequence end: zero their rows of the last page's V
+        // tile so that whatever the unused slots hold (NaN included)
+        // contributes exactly 0
+        uint8_t* vt = vtiles + static_cast<size_t>(s) * vstage + static_cast<size_t>(np - 1) * p.vtile_bytes;
+        const int nrows = kBlock - ntl;
         const int n_ch = min(p.n_chunks, (p.R - rr * p.r_range + 63) / 64);
         const int nst = n_ch * nrows * 8;  // 16-byte stores
         for (int x = et; x < nst; x += 128) {
           const int c = x / (nrows * 8), rem = x % (nrows * 8);
-          const int t = mt.nt + rem / 8, u = rem % 8;
+          const int t = ntl + rem / 8, u = rem % 8;
           *reinterpret_cast<uint4*>(vt + c * 2048 + t * 128 + u * 16) = make_uint4(0, 0, 0, 0);
         }
       }
@@ -1535,13 +1658,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
         }
         tc_fence_before();
         mbar_arrive(tfree);
-        if constexpr (kChunk) {
-          // per-segment normaliser of every virtual head (one thread per column)
-          if (rr == 0)
-            for (int k2 = 0; k2 < 2; ++k2) {
-              const int col = et + 128 * k2;
-              if (col < p.npad && vg * p.lw + col < p.Hv) p.lpart[slot * p.Hv + vg * p.lw + col] = lsum2[k2];
-            }
+        if constexpr (kChunk) {   // the normalisers were summed once by chunk_weights_kernel
           ++seg;
           continue;
         }
@@ -1586,6 +1703,7 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
 // distributed shared memory in rank order.
 struct FinishParams {
   __half* out;            // [B][H][d]
+  const float* zpart;     // the V-pass partials (read directly for tiles too wide to stage)
   const float* lpart;     // [v_slots][H]
   const int32_t* prefix;  // [B+1]
   int B, H, d, R;
@@ -1607,6 +1725,8 @@ struct FinishParams {
   const int32_t* vs_row0;
   const int32_t* vs_nrows;
   int log2nq, Hv;
+  const float* lwpart;    // chunk mode: [B][n_pc][Hv] normaliser partials of each virtual head
+  int n_pc;
 };
 
 constexpr int kFinThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 convert; warps 2..5 drain TMEM
@@ -1680,7 +1800,10 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
   pt.G = static_cast<int32_t>(pt.P < p.v_grid ? pt.P : p.v_grid);
   int32_t slot_lo = 0, n_slots = 0;
   if (pt.P > 0) tile_slots(p.prefix, pt, b0, b0 + nb, &slot_lo, &n_slots);
-  const int n_box = n_slots > 0 ? (min(n_slots << p.log2nq, p.zrows) + kFinZBox - 1) / kFinZBox : 0;
+  // the tile's partial rows are staged by TMA when they fit the stage, else
+  // the converters read them from global memory (an unusually skewed tile)
+  const bool staged = (n_slots << p.log2nq) <= p.zrows;
+  const int n_box = (n_slots > 0 && staged) ? ((n_slots << p.log2nq) + kFinZBox - 1) / kFinZBox : 0;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -1739,21 +1862,24 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
         const int32_t f0 = p.prefix[b], f1 = p.prefix[b + 1];
         if (f1 > f0) {
           const int32_t i0 = part_owner(f0, pt), i1 = part_owner(f1 - 1, pt);
-          const int col = p.vs_row0 ? (h << p.log2nq) + qi : h;
-          const int lw = p.vs_row0 ? p.Hv : p.H;
           float Ls = 0.f;
-          for (int32_t i = i0; i <= i1; i += 4) {   // four loads issued before they are added in order
-            float l4[4];
+          if (p.lwpart) {
+            const float* lp = p.lwpart + static_cast<size_t>(b) * p.n_pc * p.Hv + (h << p.log2nq) + qi;
+            for (int j = 0; j < p.n_pc; ++j) Ls += lp[static_cast<size_t>(j) * p.Hv];
+          } else {
+            for (int32_t i = i0; i <= i1; i += 4) {   // four loads issued before they are added in order
+              float l4[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) l4[u] = i + u <= i1 ? p.lpart[static_cast<size_t>(b + i + u) * lw + col] : 0.f;
+              for (int u = 0; u < 4; ++u) l4[u] = i + u <= i1 ? p.lpart[static_cast<size_t>(b + i + u) * p.H + h] : 0.f;
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-              if (i + u <= i1) Ls += l4[u];
+              for (int u = 0; u < 4; ++u)
+                if (i + u <= i1) Ls += l4[u];
+            }
           }
           il = 1.f / Ls;
           row = ((b + i0 - slot_lo) << p.log2nq) + qi;
           nseg = i1 - i0 + 1;
-          if (row < 0 || row + ((nseg - 1) << p.log2nq) >= n_box * kFinZBox) nseg = 0;   // cannot happen: the plan bounds the tile
+          if (row < 0 || (staged && row + ((nseg - 1) << p.log2nq) >= n_box * kFinZBox)) nseg = 0;   // cannot happen
         }
       }
       s_row[bl] = row;
@@ -1768,6 +1894,12 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
       uint8_t* st = smem + static_cast<size_t>(s) * p.stage_bytes;
       uint8_t* hi_t = st + a_bytes;
       const uint8_t* zt = st + a_bytes + 2u * half_bytes;
+      // partial rows of this stage: staged rows of 64 values, or global rows of r_range values
+      const int kr = k0 + i * kFinKC;
+      const int rr = kr / p.r_range;
+      const float* zg = p.zpart + ((static_cast<size_t>((rr * p.H + h) * p.v_slots + slot_lo) << p.log2nq) * p.r_range) +
+                        (kr - rr * p.r_range);
+      const int zstride = staged ? 64 : p.r_range;
       // item = (sequence row bl of the tile, 8-value chunk c of the stage's 64 rows of R)
       for (int item = et; item < p.npad * 8; item += kFinConv) {
         const int bl = item >> 3, c = item & 7;
@@ -1776,10 +1908,11 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
         for (int u = 0; u < 8; ++u) z[u] = 0.f;
         const int nseg = s_nseg[bl];
         if (nseg > 0) {
-          const float* src = reinterpret_cast<const float*>(zt + static_cast<size_t>(s_row[bl]) * 256) + c * 8;
+          const float* src = (staged ? reinterpret_cast<const float*>(zt) : zg) +
+                             static_cast<size_t>(s_row[bl]) * zstride + c * 8;
           for (int g = 0; g < nseg; ++g) {   // segment g: nq partial rows further on
-            const float4 v0 = reinterpret_cast<const float4*>(src + (g << p.log2nq) * 64)[0];
-            const float4 v1 = reinterpret_cast<const float4*>(src + (g << p.log2nq) * 64)[1];
+            const float4 v0 = reinterpret_cast<const float4*>(src + static_cast<size_t>(g << p.log2nq) * zstride)[0];
+            const float4 v1 = reinterpret_cast<const float4*>(src + static_cast<size_t>(g << p.log2nq) * zstride)[1];
             z[0] += v0.x; z[1] += v0.y; z[2] += v0.z; z[3] += v0.w;
             z[4] += v1.x; z[5] += v1.y; z[6] += v1.z; z[7] += v1.w;
           }

@@ -125,6 +125,15 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   return *reinterpret_cast<float2*>(&d);
 }
 
+// 2^x by the hardware approximation (PTX ex2.approx.ftz: relative error near
+// 2^-22, +0 for x = -inf, subnormal results flushed to 0); ample for weights
+// that are rounded to fp16 next.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Maximum of a float over the full warp (every lane receives it).
 __device__ __forceinline__ float warp_max_f32(float x) {
   float r;

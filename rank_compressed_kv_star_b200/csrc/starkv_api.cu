@@ -35,6 +35,18 @@
 #ifndef STARKV_V_RRANGE
 #define STARKV_V_RRANGE 1024
 #endif
+#ifndef STARKV_CV_STAGE_CAP
+#define STARKV_CV_STAGE_CAP 8   // ring stages of the chunked-prefill V pass
+#endif
+#ifndef STARKV_CV_LW_MAX
+#define STARKV_CV_LW_MAX 256    // widest group of virtual heads of one chunked-prefill V-pass CTA
+#endif
+#ifndef STARKV_CV_PPS
+#define STARKV_CV_PPS 4         // pages per ring stage of the chunked-prefill V pass (at most)
+#endif
+#ifndef STARKV_V_PPS
+#define STARKV_V_PPS 1          // pages per ring stage of the decode V pass (at most)
+#endif
 #ifndef STARKV_V_RING_BYTES
 #define STARKV_V_RING_BYTES (105 * 1024)
 #endif
@@ -91,7 +103,7 @@ struct DecodePlan {
   uint32_t ktc_a_bytes, ktc_b_bytes, ktc_tmem;
   size_t ktc_smem;
   // V pass
-  int n_rr, r_range, r_range_pad, n_chunks, n_mtiles, v_stages, v_ctas, v_per_sm;
+  int n_rr, r_range, r_range_pad, n_chunks, n_mtiles, v_stages, v_ctas, v_per_sm, v_pps;
   uint32_t vtile, ltile, ptile, tmem_cols;
   size_t v_smem;
   // finish: Z / L from the partials and the up-projection (tcgen05, split-K cluster)
@@ -267,7 +279,12 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   p.ltile = 16u * p.H * 4;
   p.ptile = static_cast<uint32_t>(p.npad) * 16 * 2;
   p.tmem_cols = static_cast<uint32_t>(pow2_ceil(p.n_mtiles * p.npad < 32 ? 32 : p.n_mtiles * p.npad));
-  const uint32_t stage = p.vtile + p.ltile + p.ptile;
+  // pages per ring stage: at most STARKV_V_PPS, fewer while a ring of 3 stages would not fit
+  p.v_pps = STARKV_V_PPS < kMaxPPS ? STARKV_V_PPS : kMaxPPS;
+  while (p.v_pps > 1 &&
+         3u * p.v_pps * (p.vtile + p.ltile + p.ptile) > static_cast<uint32_t>(STARKV_V_RING_BYTES))
+    --p.v_pps;
+  const uint32_t stage = p.v_pps * (p.vtile + p.ltile + p.ptile);
   p.v_stages = static_cast<int>(static_cast<uint32_t>(STARKV_V_RING_BYTES) / stage);
   if (p.v_stages > 8) p.v_stages = 8;
   if (p.v_stages < 2) p.v_stages = 2;
@@ -834,7 +851,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   vp.t_pad = pl.t_pad; vp.r_range = pl.r_range; vp.n_rr = pl.n_rr; vp.v_slots = pl.ws.v_slots;
   vp.k_grid = pl.k_ctas;
   vp.stages = pl.v_stages; vp.n_chunks = pl.n_chunks; vp.n_mtiles = pl.n_mtiles; vp.tmem_cols = pl.tmem_cols;
-  vp.vtile_bytes = pl.vtile; vp.ltile_bytes = pl.ltile; vp.ptile_bytes = pl.ptile;
+  vp.vtile_bytes = pl.vtile; vp.ltile_bytes = pl.ltile; vp.ptile_bytes = pl.ptile; vp.pps = pl.v_pps;
   if (!set_smem(vpass_kernel<false>, pl.v_smem)) return STARKV_ERR_CUDA;
   if (launch(vpass_kernel<false>, dim3(pl.v_ctas, pl.n_rr), dim3(kVThreads), pl.v_smem, s, 1, vmap, vp) != cudaSuccess)
     return STARKV_ERR_CUDA;
@@ -842,7 +859,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
 
   FinishParams fp{};
   fp.out = static_cast<__half*>(out);
-  fp.lpart = lpart; fp.prefix = prefix;
+  fp.zpart = zpart; fp.lpart = lpart; fp.prefix = prefix;
   fp.B = batch; fp.H = pl.H; fp.d = pl.d; fp.R = pl.R; fp.log2G = pl.log2G;
   fp.r_range = pl.r_range; fp.v_slots = pl.ws.v_slots; fp.v_grid = pl.v_ctas;
   fp.n_mt = pl.up_mt; fp.bt_rows = pl.up_bt_rows; fp.k_per_cta = pl.up_kpc; fp.npad = pl.up_npad;
@@ -973,13 +990,13 @@ namespace {
 // sequence is then streamed once for all of its rows (see kpass_chunk_kernel).
 // Shapes: KV heads in groups of 8 (Hkv % 8 == 0), G = H / Hkv <= 16.
 struct ChunkPlan {
-  int H, Hkv, d, r, R, G, nq, log2nq, Hv, lw, n_vg, nv_max, n_groups, t_pad, MB, NB, n_rows, n_seqs;
+  int H, Hkv, d, r, R, G, nq, log2nq, Hv, lw, n_vg, nv_max, n_groups, t_pad, MB, NB, n_rows, n_seqs, n_pc;
   // K pass
   int k_ctas, kb, ksteps, k_stages, nacc, nbs;
   uint32_t a_bytes, b_bytes, k_tmem;
   size_t k_smem;
   // V pass
-  int r_range, r_range_pad, n_rr, n_chunks, n_mtiles, v_ctas, v_stages, v_slots, k_slots;
+  int r_range, r_range_pad, n_rr, n_chunks, n_mtiles, v_ctas, v_stages, v_slots, k_slots, v_pps;
   uint32_t vtile, ltile, ptile, v_tmem;
   size_t v_smem;
   // finish
@@ -988,7 +1005,7 @@ struct ChunkPlan {
   size_t up_smem;
   // workspace
   size_t status_off, prefix_off, teff_off, vs_seq_off, vs_row0_off, vs_nrows_off, vs_len_off, qth_off, logits_off,
-      mpart_off, lpart_off, zpart_off, total;
+      mpart_off, lpart_off, lwpart_off, wts_off, zpart_off, total;
 };
 
 bool chunk_eligible(const starkv_layer_desc* d) {
@@ -1040,62 +1057,68 @@ starkv_status make_chunk_plan(const starkv_layer_desc* d, int32_t n_seqs, int32_
   }
   c.k_ctas = sms;
   // V pass: lw virtual heads per CTA and mt 128-row M tiles of R (TMEM: mt * lw
-  // columns).  The CTAs of one (R range, virtual-head group) are capped so that
-  // the finish kernel's tile of one virtual sequence can hold all the partial
-  // rows it may need (v_ctas * nq rows of 256 bytes in each of two stages).
+  // columns <= 512).  Per token, the V codes are read once per group of
+  // virtual heads (Hv / lw groups) and the fp16 weights once per R range (R /
+  // (128 mt) ranges): the split with the fewest bytes per token wins (the
+  // larger lw on a tie).  The logits, and the weights written over them, are
+  // laid out in rows of lw virtual heads.
   {
-    // two stages of at most 107 KiB (with barriers and per-row arrays: <= 220 KiB), each
-    // holding B_V boxes, hi/lo tiles of 16 rows and whole 32-row boxes of partial rows
-    const int z_cap = static_cast<int>((107u * 1024u - 2u * kFinKC * 128u - 2u * 16u * 128u) / 256u) /
-                      kFinZBox * kFinZBox;
-    const int cap = z_cap / c.nq > 1 ? z_cap / c.nq : 1;
     const int rpad = (c.R + 127) / 128 * 128;
-    int best_total = -1;
-    for (int mt = 512 / c.lw; mt >= 1; mt /= 2) {
-      const int rr = mt * 128 < rpad ? mt * 128 : rpad;
-      const int n_rr = (c.R + rr - 1) / rr;
-      const int per_sm = 512 / (mt * c.lw) < 2 ? 512 / (mt * c.lw) : 2;
-      const uint32_t stage = static_cast<uint32_t>(rr) * 32u + 64u * c.lw + 32u * c.lw;   // V tile, logits, weights
-      const int stages = static_cast<int>((200u * 1024u / per_sm) / stage);
-      if (per_sm < 1 || stages < 2) continue;
-      int v_ctas = sms * per_sm / (n_rr * c.n_vg);
-      if (v_ctas > cap) v_ctas = cap;
-      if (v_ctas < 1) v_ctas = 1;
-      const int total = v_ctas * n_rr * c.n_vg;
-      if (best_total >= sms || total <= best_total) continue;   // the widest R range that fills the GPU
-      best_total = total;
-      c.r_range = rr; c.n_rr = n_rr; c.v_ctas = v_ctas;
-      c.v_stages = stages > 8 ? 8 : stages;
-    }
-    if (best_total < 0) return STARKV_ERR_UNSUPPORTED;
+    int64_t best = -1;
+    for (int lw = c.Hv < STARKV_CV_LW_MAX ? c.Hv : STARKV_CV_LW_MAX; lw >= 16; lw /= 2)
+      for (int mt = 512 / lw; mt >= 1; mt /= 2) {
+        if (mt * 128 > rpad && mt > 1) continue;
+        const int n_vg = c.Hv / lw;
+        const int n_rr = (c.R + mt * 128 - 1) / (mt * 128);
+        const int64_t cost = static_cast<int64_t>(n_vg) * c.R * 2 + static_cast<int64_t>(n_rr) * c.Hv * 2;
+        if (best >= 0 && cost >= best) continue;
+        best = cost;
+        c.lw = lw; c.n_vg = n_vg; c.n_rr = n_rr; c.r_range = mt * 128 < rpad ? mt * 128 : rpad;
+      }
     c.r_range_pad = c.r_range;
     c.n_chunks = c.r_range_pad / 64;
     c.n_mtiles = c.r_range_pad / 128;
     c.vtile = static_cast<uint32_t>(c.r_range_pad) * 16 * 2;
-    c.ltile = 16u * c.lw * 4;
+    c.ltile = 0;   // the weights arrive as fp16 tiles (chunk_weights_kernel)
     c.ptile = static_cast<uint32_t>(c.lw) * 16 * 2;
     c.v_tmem = static_cast<uint32_t>(pow2_ceil(c.n_mtiles * c.lw < 32 ? 32 : c.n_mtiles * c.lw));
-    c.v_smem = 1024 + static_cast<size_t>(c.v_stages) * (c.vtile + c.ltile + c.ptile) + c.v_stages * sizeof(StageMeta) +
+    const int per_sm = 512 / static_cast<int>(c.v_tmem) < 2 ? 512 / static_cast<int>(c.v_tmem) : 2;
+    // pages per ring stage: at most STARKV_CV_PPS, fewer while a ring of 3 stages would not fit
+    c.v_pps = STARKV_CV_PPS < kMaxPPS ? STARKV_CV_PPS : kMaxPPS;
+    while (c.v_pps > 1 && 3u * c.v_pps * (c.vtile + c.ltile + c.ptile) > 200u * 1024u / per_sm) --c.v_pps;
+    const uint32_t stage = c.v_pps * (c.vtile + c.ltile + c.ptile);
+    c.v_stages = static_cast<int>((200u * 1024u / per_sm) / stage);
+    if (c.v_stages > STARKV_CV_STAGE_CAP) c.v_stages = STARKV_CV_STAGE_CAP;
+    if (c.v_stages < 2) return STARKV_ERR_UNSUPPORTED;
+    c.v_smem = 1024 + static_cast<size_t>(c.v_stages) * stage + c.v_stages * sizeof(StageMeta) +
                (3 * c.v_stages + 4) * sizeof(uint64_t) + (c.lw + 128) * sizeof(float);
+    c.v_ctas = sms * per_sm / (c.n_rr * c.n_vg);
+    if (c.v_ctas < 1) c.v_ctas = 1;
   }
   c.k_slots = c.k_ctas + c.nv_max;
   c.v_slots = c.v_ctas + c.nv_max;
   // finish: tiles of virtual sequences (nq rows each)
   c.up_mt = (c.d + 127) / 128;
+  // tiles of up to 256 / nq virtual sequences (64 when shared memory is
+  // short); a stage stages at most the partial rows that fit (107 KiB stages),
+  // wider tiles read theirs from global memory
   c.up_bt_rows = 256 / c.nq;
   if (c.up_bt_rows > c.nv_max) c.up_bt_rows = c.nv_max;
   for (int tries = 0; tries < 16; ++tries) {
     const int rows = c.up_bt_rows * c.nq;
     c.up_npad = rows < 16 ? 16 : (rows + 15) / 16 * 16;
     const int need = (c.up_bt_rows + c.v_ctas - 1) * c.nq;
+    const int cap = static_cast<int>((107u * 1024u - 2u * kFinKC * 128u - 2u * c.up_npad * 128u) / 256u) /
+                    kFinZBox * kFinZBox;
     c.up_zrows = (need + kFinZBox - 1) / kFinZBox * kFinZBox;
-    c.up_stage_bytes = static_cast<uint32_t>(
-        align_up(2u * kFinKC * 128u + 2u * static_cast<size_t>(c.up_npad) * 128u + c.up_zrows * 256u, 1024));
-    c.up_smem = 1024 + 2 * static_cast<size_t>(c.up_stage_bytes) + 7 * sizeof(uint64_t) + 3 * kFinMaxRows * 4;
-    if (c.up_smem <= 220u * 1024u) break;
-    if (c.up_bt_rows == 1) return STARKV_ERR_UNSUPPORTED;
+    if (c.up_zrows > cap) c.up_zrows = cap;
+    if (c.up_zrows >= 2 * kFinZBox || c.up_bt_rows == 1) break;
     c.up_bt_rows /= 2;
   }
+  if (c.up_zrows < kFinZBox) return STARKV_ERR_UNSUPPORTED;
+  c.up_stage_bytes = static_cast<uint32_t>(
+      align_up(2u * kFinKC * 128u + 2u * static_cast<size_t>(c.up_npad) * 128u + c.up_zrows * 256u, 1024));
+  c.up_smem = 1024 + 2 * static_cast<size_t>(c.up_stage_bytes) + 7 * sizeof(uint64_t) + 3 * kFinMaxRows * 4;
   if (c.up_smem > 220u * 1024u) return STARKV_ERR_UNSUPPORTED;
   c.up_bt = (c.nv_max + c.up_bt_rows - 1) / c.up_bt_rows;
   c.up_ks = 1;
@@ -1114,8 +1137,11 @@ starkv_status make_chunk_plan(const starkv_layer_desc* d, int32_t n_seqs, int32_
   c.vs_len_off = off; off = align_up(off + nv * 4, 256);
   c.qth_off = off; off = align_up(off + nv * 2 * c.Hv * c.r * 2, 256);
   c.logits_off = off; off = align_up(off + nv * c.n_vg * c.t_pad * static_cast<size_t>(c.lw) * 4, 256);
+  c.wts_off = off; off = align_up(off + nv * c.n_vg * c.t_pad * static_cast<size_t>(c.lw) * 2, 256);
   c.mpart_off = off; off = align_up(off + static_cast<size_t>(c.k_slots) * c.Hv * 4, 256);
   c.lpart_off = off; off = align_up(off + static_cast<size_t>(c.v_slots) * c.Hv * 4, 256);
+  c.n_pc = static_cast<int>((c.t_pad / kBlock + kCwPages - 1) / kCwPages);
+  c.lwpart_off = off; off = align_up(off + nv * c.n_pc * c.Hv * 4, 256);
   c.zpart_off = off;
   off = align_up(off + static_cast<size_t>(c.n_rr) * c.H * c.v_slots * c.nq * c.r_range * 4, 256);
   c.total = off;
@@ -1136,6 +1162,8 @@ starkv_status chunk_prefill(const ChunkPlan& c, const void* q, const void* B_K, 
   float* logits = reinterpret_cast<float*>(ws + c.logits_off);
   float* mpart = reinterpret_cast<float*>(ws + c.mpart_off);
   float* lpart = reinterpret_cast<float*>(ws + c.lpart_off);
+  float* lwpart = reinterpret_cast<float*>(ws + c.lwpart_off);
+  __half* wts = reinterpret_cast<__half*>(ws + c.wts_off);
   float* zpart = reinterpret_cast<float*>(ws + c.zpart_off);
 
   CUtensorMap kmap, qmap, vmap, bvmap, zmap;
@@ -1183,6 +1211,11 @@ starkv_status chunk_prefill(const ChunkPlan& c, const void* q, const void* B_K, 
   if (launch(kpass_chunk_kernel, dim3(c.k_ctas), dim3(kKTCThreads), c.k_smem, s, 1, kmap, qmap, kp) != cudaSuccess)
     return STARKV_ERR_CUDA;
 
+  ChunkWeightsParams wp{logits, wts,  mpart,   teff,  prefix,   lwpart,
+                        c.nv_max, c.Hv, c.n_vg, c.lw, kp.log2lw, c.t_pad, c.k_ctas, c.n_pc};
+  if (launch(chunk_weights_kernel, dim3(c.nv_max, c.n_pc, c.n_vg), dim3(256), 0, s, 1, wp) != cudaSuccess)
+    return STARKV_ERR_CUDA;
+
   VPassParams vp{};
   std::memset(&vp, 0, sizeof(vp));
   vp.tables = block_tables; vp.row_seq = vs_seq; vp.teff = teff; vp.prefix = prefix; vp.logits = logits;
@@ -1191,7 +1224,7 @@ starkv_status chunk_prefill(const ChunkPlan& c, const void* q, const void* B_K, 
   vp.t_pad = c.t_pad; vp.r_range = c.r_range; vp.n_rr = c.n_rr; vp.v_slots = c.v_slots;
   vp.k_grid = c.k_ctas;
   vp.stages = c.v_stages; vp.n_chunks = c.n_chunks; vp.n_mtiles = c.n_mtiles; vp.tmem_cols = c.v_tmem;
-  vp.vtile_bytes = c.vtile; vp.ltile_bytes = c.ltile; vp.ptile_bytes = c.ptile;
+  vp.vtile_bytes = c.vtile; vp.ltile_bytes = c.ltile; vp.ptile_bytes = c.ptile; vp.pps = c.v_pps; vp.wts = wts;
   vp.Hv = c.Hv; vp.n_vg = c.n_vg; vp.log2nq = c.log2nq; vp.lw = c.lw;
   if (!set_smem(vpass_kernel<true>, c.v_smem)) return STARKV_ERR_CUDA;
   if (launch(vpass_kernel<true>, dim3(c.v_ctas, c.n_rr * c.n_vg), dim3(kVThreads), c.v_smem, s, 1, vmap, vp) !=
@@ -1201,13 +1234,13 @@ starkv_status chunk_prefill(const ChunkPlan& c, const void* q, const void* B_K, 
   FinishParams fp{};
   std::memset(&fp, 0, sizeof(fp));
   fp.out = static_cast<__half*>(out);
-  fp.lpart = lpart; fp.prefix = prefix;
+  fp.zpart = zpart; fp.lpart = lpart; fp.prefix = prefix;
   fp.B = c.nv_max; fp.H = c.H; fp.d = c.d; fp.R = c.R;
   fp.log2G = ap.log2G;
   fp.r_range = c.r_range; fp.v_slots = c.v_slots; fp.v_grid = c.v_ctas;
   fp.n_mt = c.up_mt; fp.bt_rows = c.up_bt_rows; fp.k_per_cta = c.up_kpc; fp.npad = c.up_npad;
   fp.stages = 2; fp.zrows = c.up_zrows; fp.stage_bytes = c.up_stage_bytes; fp.tmem_cols = c.up_tmem;
-  fp.vs_row0 = vs_row0; fp.vs_nrows = vs_nrows; fp.log2nq = c.log2nq; fp.Hv = c.Hv;
+  fp.vs_row0 = vs_row0; fp.vs_nrows = vs_nrows; fp.log2nq = c.log2nq; fp.Hv = c.Hv; fp.lwpart = lwpart; fp.n_pc = c.n_pc;
   if (!set_smem(finish_kernel, c.up_smem)) return STARKV_ERR_CUDA;
   if (launch(finish_kernel, dim3(c.H * c.up_mt * c.up_bt, c.up_ks), dim3(kFinThreads), c.up_smem, s, c.up_ks,
              bvmap, zmap, fp) != cudaSuccess)
