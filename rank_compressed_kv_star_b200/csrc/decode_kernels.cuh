@@ -1616,43 +1616,52 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
         const size_t slot = static_cast<size_t>(mt.b) + cta;
         // partial rows [R range][head][slot][r_range]: head h0+hh's row of this slot
         float* zb = p.zpart + ((static_cast<size_t>(rr) * p.H) * p.v_slots + slot) * p.r_range;
+        // every (m, h0) block: 32 TMEM columns into registers, then 32 stores
+        // with constant register indices (fully unrolled), each a 128-byte
+        // row piece across the warp's lanes
         if constexpr (kChunk) {
-          // virtual head (h, i): row slot * nq + i of head h
+          // virtual head (h, i): row slot * nq + i of head h (npad = lw, a multiple of 32)
+          const uint32_t nqm = (1u << p.log2nq) - 1u;
           for (int m = 0; m < p.n_mtiles; ++m) {
-            uint32_t v[32];
             const uint32_t ta = taddr + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(m * p.npad);
             const int j = m * 128 + q * 32 + lane;
+            const bool jok = j < p.r_range && rr * p.r_range + j < p.R;
+            float* zj = p.zpart + j;
             for (int h0 = 0; h0 < p.npad; h0 += 32) {
-              if (p.npad - h0 >= 32) tmem_ld_32x32b_x32(ta + h0, v);
-              else tmem_ld_32x32b_x16(ta + h0, v);
+              uint32_t v[32];
+              tmem_ld_32x32b_x32(ta + h0, v);
               tmem_ld_wait();
-              if (j < p.r_range && rr * p.r_range + j < p.R) {
-                const int hn = min(32, p.npad - h0);
-                for (int hh = 0; hh < hn; ++hh) {
-                  const int col = vg * p.lw + h0 + hh;
-                  if (col >= p.Hv) break;
-                  const size_t row = ((static_cast<size_t>(rr) * p.H + (col >> p.log2nq)) * p.v_slots + slot)
-                                         << p.log2nq;
-                  st_global_hint(p.zpart + (row + (col & ((1 << p.log2nq) - 1))) * p.r_range + j,
-                                 __uint_as_float(v[hh]), keep);
+              if (jok) {
+                const uint32_t c0 = static_cast<uint32_t>(vg * p.lw + h0);
+#pragma unroll
+                for (int hh = 0; hh < 32; ++hh) {
+                  const uint32_t col = c0 + hh;
+                  const size_t row =
+                      ((static_cast<size_t>(rr * p.H + static_cast<int>(col >> p.log2nq)) * p.v_slots + slot)
+                       << p.log2nq) + (col & nqm);
+                  st_global_hint_free(zj + row * p.r_range, __uint_as_float(v[hh]), keep);
                 }
               }
             }
           }
-        }
-        for (int m = 0; m < (kChunk ? 0 : p.n_mtiles); ++m) {
-          uint32_t v[32];
-          const uint32_t ta = taddr + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(m * p.npad);
-          const int j = m * 128 + q * 32 + lane;
-          for (int h0 = 0; h0 < p.H; h0 += 32) {
-            if (p.npad - h0 >= 32) tmem_ld_32x32b_x32(ta + h0, v);
-            else tmem_ld_32x32b_x16(ta + h0, v);
-            tmem_ld_wait();
-            if (j < p.r_range && rr * p.r_range + j < p.R) {
-              const int hn = min(32, p.H - h0);
-              for (int hh = 0; hh < hn; ++hh)
-                st_global_hint(zb + static_cast<size_t>(h0 + hh) * p.v_slots * p.r_range + j, __uint_as_float(v[hh]),
-                               keep);
+        } else {
+          for (int m = 0; m < p.n_mtiles; ++m) {
+            const uint32_t ta = taddr + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(m * p.npad);
+            const int j = m * 128 + q * 32 + lane;
+            const bool jok = j < p.r_range && rr * p.r_range + j < p.R;
+            const size_t hstride = static_cast<size_t>(p.v_slots) * p.r_range;
+            for (int h0 = 0; h0 < p.H; h0 += 32) {
+              uint32_t v[32];
+              if (p.npad - h0 >= 32) tmem_ld_32x32b_x32(ta + h0, v);
+              else tmem_ld_32x32b_x16(ta + h0, v);
+              tmem_ld_wait();
+              if (jok) {
+                const int hn = min(32, p.H - h0);
+                float* zr = zb + static_cast<size_t>(h0) * hstride + j;
+#pragma unroll
+                for (int hh = 0; hh < 32; ++hh)
+                  if (hh < hn) st_global_hint_free(zr + hh * hstride, __uint_as_float(v[hh]), keep);
+              }
             }
           }
         }

@@ -171,6 +171,12 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
 __device__ __forceinline__ void st_global_hint(float* p, float v, uint64_t policy) {
   asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(policy) : "memory");
 }
+// The same store without a compiler memory barrier: for results that nothing
+// in the same kernel reads back, so that the compiler may schedule freely
+// around a long run of them.
+__device__ __forceinline__ void st_global_hint_free(float* p, float v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(policy));
+}
 __device__ __forceinline__ void st_global_hint(uint2* p, uint2 v, uint64_t policy) {
   asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;" ::"l"(p), "r"(v.x), "r"(v.y), "l"(policy)
                : "memory");

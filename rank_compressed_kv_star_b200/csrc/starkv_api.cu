@@ -1065,7 +1065,7 @@ starkv_status make_chunk_plan(const starkv_layer_desc* d, int32_t n_seqs, int32_
   {
     const int rpad = (c.R + 127) / 128 * 128;
     int64_t best = -1;
-    for (int lw = c.Hv < STARKV_CV_LW_MAX ? c.Hv : STARKV_CV_LW_MAX; lw >= 16; lw /= 2)
+    for (int lw = c.Hv < STARKV_CV_LW_MAX ? c.Hv : STARKV_CV_LW_MAX; lw >= 32; lw /= 2)
       for (int mt = 512 / lw; mt >= 1; mt /= 2) {
         if (mt * 128 > rpad && mt > 1) continue;
         const int n_vg = c.Hv / lw;
