@@ -31,6 +31,7 @@ sys.path.insert(0, ROOT)
 METRIC = "compressed-KV paged decode tokens/s at 1 B200; HBM GB/s as % of ~8 TB/s peak"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_F16_TFLOPS = 1590.0   # dense fp16/bf16 tensor throughput (burst) of the profiling recipe
 WORKLOAD_NAMES = {
     2: "single-layer decode: 32 heads, head_size 128, K rank 64/head, V joint rank 2048, fp16, "
        "block_size 16, batch 16, seq_len 2048",
@@ -93,8 +94,8 @@ def whole_job_tokens_per_s(world: int, batch_per_rank: int, ms_per_step_max: flo
 # profiles/gqa_streaming_b32_t8192_full.md give the commands; an entry is
 # emptied when its kernel changes.
 NCU_TRAFFIC_PER_TOKEN: dict = {
-    (32, 32, 64, 2048): {"kpass": 4123.2, "vpass": 4259.4},
-    (32, 8, 64, 512): {"kpass": 1049.6, "vpass": 1167.1},
+    (32, 32, 64, 2048): {"kpass": 4122.6, "vpass": 4247.5},
+    (32, 8, 64, 512): {"kpass": 1047.0, "vpass": 1164.1},
 }
 
 
@@ -106,6 +107,17 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense fp16 tensor TFLOP/s: the measured bf16 burst figure (same rate for fp16), else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_F16_TFLOPS, "fallback"
 
 
 # --------------------------------------------------------------- clocks
@@ -604,6 +616,20 @@ def run_prefill(args):
                   + (L["A_K"].numel() + L["A_V"].numel() + L["B_K"].numel() + L["B_V"].numel()) * 2)
     peak, peak_kind = measured_peaks()
     achieved = step_bytes / (ms * 1e-3) / 1e9
+    # useful tensor work of the read-once path per context token: the K logits of
+    # the chunk's rows (2 * N * H * r) and the weighted sum of the V codes
+    # (2 * N * H * R); the larger of the two roof times sets the bound
+    step_flops = int(T.sum()) * 2 * N * H * (r + R)
+    tpeak, tpeak_kind = measured_tensor_peak()
+    t_flops = step_flops / (tpeak * 1e12)
+    t_bytes = step_bytes / (peak * 1e9)
+    tensor_bound = t_flops > t_bytes
+    achieved_tf = step_flops / (ms * 1e-3) / 1e12
+    G = H // Hkv
+    read_note = ("every page of a sequence is read once per step: the chunk's rows are the extra N columns "
+                 "of the tensor-core K and V passes (one virtual sequence of 16 rows)" if G == 1 else
+                 f"grouped queries: a chunk's 16 rows form {G} virtual sequences of {16 // G} rows (16 virtual "
+                 f"heads per KV head), each reading the sequence's pages, so pages are read {G} times per step")
 
     # the oracle on one sequence's chunk
     b0 = 0
@@ -621,14 +647,24 @@ def run_prefill(args):
         "config": {"workload": wl.name, "batch": B, "chunk": N, "context": max_len, "layers": 1,
                    "step": "compress-store of the chunk + causal attention of its queries over the context",
                    "l2": f"code pools of {code_bytes / 2**30:.2f} GiB read per step"},
-        "roofline": {"kernel": "prefill step", "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
-                     "algorithmic_bytes_per_launch": step_bytes, "peak_kind": peak_kind,
-                     "note": "each query row reads its sequence's pages: traffic is about chunk x the "
-                             "algorithmic bytes"},
+        "roofline": ({"kernel": "prefill step", "bound": "tensor", "achieved": round(achieved_tf, 1),
+                      "peak": tpeak, "unit": "TFLOP/s", "frac": round(achieved_tf / tpeak, 4), "traffic": None,
+                      "algorithmic_flops_per_step": step_flops, "peak_kind": tpeak_kind,
+                      "hbm": {"achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                              "frac": round(achieved / peak, 4), "algorithmic_bytes_per_step": step_bytes,
+                              "peak_kind": peak_kind},
+                      "note": read_note}
+                     if tensor_bound else
+                     {"kernel": "prefill step", "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                      "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                      "algorithmic_bytes_per_launch": step_bytes, "peak_kind": peak_kind,
+                      "tensor": {"achieved": round(achieved_tf, 1), "peak": tpeak, "unit": "TFLOP/s",
+                                 "frac": round(achieved_tf / tpeak, 4), "algorithmic_flops_per_step": step_flops,
+                                 "peak_kind": tpeak_kind},
+                      "note": read_note}),
         "e2e": {"value": round(n_rows / (ms_e2e * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 5)},
-        "gpu_launches": K * 8,
+        "gpu_launches": K * 7,   # compress-store + chunk table, absorb, K pass, weights, V pass, finish
         "clocks": clk,
         "cpu_baseline": {"value": round(N / cpu_s, 4), "unit": "tokens/s", "cores": _blas_threads(),
                          "kind": "oracle",
