@@ -351,16 +351,17 @@ starkv_status starkv_set_wait_test_hook(uint32_t wait_limit_us, int32_t drop_k_s
  */
 typedef struct {
   size_t total_bytes;
-  size_t status_off;  /* int32 status word */
+  size_t status_off;  /* int32 status word; status_off + 64: uint32 counter of the page chunks the K
+                         pass has handed out (set to 0 by the query absorption of every call) */
   size_t prefix_off;  /* int32 [batch+1] prefix sums of pages per sequence */
   size_t qt_off;      /* fp32 [batch][H][r]: log2(e)*scale*q.B_K^T */
   size_t logits_off;  /* fp32 [batch][t_pad][H]: base-2 logits s*log2(e) */
-  size_t mpart_off;   /* fp32 [k_slots][H]: max of the base-2 logits per segment */
+  size_t mpart_off;   /* fp32 [k_slots][H]: max of each sequence's base-2 logits */
   size_t lpart_off;   /* fp32 [v_slots][H]: per segment, sum of the fp16 weights exp2(s - max) */
   size_t zpart_off;   /* fp32 [n_rranges][H][v_slots][r_range]: per segment, sum_t w c_V */
   int32_t t_pad;      /* logits row capacity (multiple of 16) */
-  int32_t k_ctas;     /* CTAs of the K pass (stream partition) */
-  int32_t k_slots;    /* k_ctas + batch */
+  int32_t k_ctas;     /* CTAs of the K pass (they take page chunks from the counter) */
+  int32_t k_slots;    /* batch: one maximum slot per sequence */
   int32_t v_ctas;     /* CTAs of the V pass per R range */
   int32_t v_slots;    /* v_ctas + batch */
   int32_t n_rranges;  /* R ranges of the V pass */

@@ -3,12 +3,12 @@
 // One decode is four launches on the caller's stream, each launched with
 // programmatic stream serialisation (see griddep_wait):
 //   1. absorb      q~ = log2(e)*scale * q . B_K[g(h)]^T; page prefix sums; status
-//                  reset; segment maxima set to -inf
-//   2. kpass       base-2 logits s = q~ . c_K over the K pages, per-segment max
-//                  (kpass_kernel on CUDA cores for multi-head attention,
+//                  and page-chunk counter reset; per-sequence maxima set to -inf
+//   2. kpass       base-2 logits s = q~ . c_K over the K pages, each sequence's
+//                  max M merged by float-max atomics (kpass_kernel on CUDA cores
+//                  for multi-head attention, taking page chunks from a counter;
 //                  kpass_tc_kernel on tcgen05 for grouped queries)
-//   3. vpass       split reduction M = max over the sequence's K segments, then
-//                  Z = sum_t w c_V on tcgen05 tensor cores with w = fp16(exp2(s - M)),
+//   3. vpass       Z = sum_t w c_V on tcgen05 tensor cores with w = fp16(exp2(s - M)),
 //                  and the normaliser L = sum_t w, per segment
 //   4. finish      Z / L summed over the segments and split into fp16 hi + lo,
 //                  then out_h = (Z_h / L) . B_V[:, g(h)*d:(g(h)+1)*d] on tcgen05 -> fp16
@@ -201,8 +201,9 @@ struct AbsorbParams {
   int32_t* prefix;        // [B+1]
   int32_t* teff;          // [B] clamped lengths
   int32_t* status;
-  float* mpart_init;      // [n_mpart] set to -inf (segment maxima merged by atomics later); may be null
+  float* mpart_init;      // [n_mpart] set to -inf (maxima merged by atomics later); may be null
   int n_mpart;
+  uint32_t* work_ctr;     // the K pass's page-chunk counter, set to 0 by item 0; may be null
   int B, H, d, r, cap;    // cap = min(max_seq_len, max_blocks_per_seq*16)
   int log2G;              // query heads per KV head = 1 << log2G
   float coef;             // scale * log2(e)
@@ -264,6 +265,7 @@ __device__ __forceinline__ void absorb_item(const AbsorbParams& p, int item, int
     if (tid == 255) {
       p.prefix[p.B] = acc + s;
       *p.status = bad ? STARKV_FLAG_BAD_SEQ_LEN : 0;
+      if (p.work_ctr) *p.work_ctr = 0u;
     }
     for (int b = b0; b < b0 + per && b < p.B; ++b) {
       p.prefix[b] = acc;
@@ -377,8 +379,10 @@ struct KPassParams {
   const int32_t* prefix;      // [B+1]
   const float* qt;            // [B][H][r]
   float* logits;              // [B][t_pad][H]
-  float* mpart;               // [k_slots][H]: max of the base-2 logits per segment (-inf on entry)
+  float* mpart;               // [B][H]: max of each sequence's base-2 logits (-inf on entry)
   int32_t* status;
+  uint32_t* work_ctr;         // next page chunk to hand out (0 on entry)
+  int chunk_pages;            // pages per chunk
   int B, H, log2H, r, MB, NB, t_pad;
   int Hkv, log2G;             // KV heads (codes per token) and log2(query heads per KV head)
   int tps;                    // tokens per ring stage (> 16: whole pages of one sequence)
@@ -432,23 +436,29 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
   griddep_wait();
   griddep_launch_dependents();
 
-  Partition pt;
-  pt.P = p.prefix[p.B];
-  pt.G = static_cast<int32_t>(pt.P < gridDim.x ? pt.P : gridDim.x);
-  const int cta = blockIdx.x;
-  const bool has_work = cta < pt.G;
-
   if (warp == kKConsumers / 32) {
     // ------------------------------------------------------------ producer
+    // Pages are handed out in chunks of chunk_pages from a counter in the
+    // workspace, so that a CTA on an SM that streams faster takes more of
+    // them (equal static ranges leave the grid waiting for its slowest CTA).
+    // The only per-CTA results are the per-sequence maxima, merged by atomics,
+    // so which CTA reads a page does not change any result.  A CTA's chunks
+    // come in increasing order, so its walk over the sequences only moves on.
     if (lane != 0) return;
     const uint64_t pol = policy_evict_first();
     const uint32_t tok_bytes = static_cast<uint32_t>(p.Hkv) * p.r * 2;
     uint32_t k = 0;
     bool ok = true;
-    if (has_work) {
-      const int64_t p0 = part_begin(cta, pt), p1 = part_begin(cta + 1, pt);
-      int32_t b = seq_of_page(p.prefix, p.B, p0);
-      const size_t page_elems = static_cast<size_t>(kBlock) * p.Hkv * p.r;
+    const int64_t P = p.prefix[p.B];
+    const int64_t C = p.chunk_pages;
+    const int64_t n_chunks = (P + C - 1) / C;
+    const size_t page_elems = static_cast<size_t>(kBlock) * p.Hkv * p.r;
+    int32_t b = -1;
+    uint32_t c = atomicAdd(p.work_ctr, 1u);
+    while (ok && static_cast<int64_t>(c) < n_chunks) {
+      const uint32_t c_next = atomicAdd(p.work_ctr, 1u);   // in flight while this chunk is issued
+      const int64_t p0 = static_cast<int64_t>(c) * C, p1 = min(P, p0 + C);
+      if (b < 0) b = seq_of_page(p.prefix, p.B, p0);
       if (p.tps <= kBlock) {
         // a page is split over several stages
         for (int64_t pg_g = p0; pg_g < p1 && ok; ++pg_g) {
@@ -503,6 +513,7 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
           pg_g += n_pg;
         }
       }
+      c = c_next;
     }
     if (ok) {
       const int s = k % S;
@@ -546,9 +557,9 @@ __global__ void __launch_bounds__(kKThreads, STARKV_K_CTAS_PER_SM) kpass_kernel(
     }
     const StageMeta mt = meta[s];
     if (mt.b != cur_b || mt.b < 0) {   // new sequence, or the end marker (b < 0)
-      // per-segment max of every head (slot = sequence + CTA, -inf on entry),
-      // merged across this CTA's consumers by float-max atomics
-      if (cur_b >= 0 && sub == 0 && m > -INFINITY) atomic_max_f32(&p.mpart[static_cast<size_t>(cur_b + cta) * p.H + head], m);
+      // the sequence's max of every head (-inf on entry), merged across all
+      // consumers of all CTAs by float-max atomics
+      if (cur_b >= 0 && sub == 0 && m > -INFINITY) atomic_max_f32(&p.mpart[static_cast<size_t>(cur_b) * p.H + head], m);
       if (mt.b < 0) break;
       cur_b = mt.b;
       m = -INFINITY;
@@ -646,7 +657,7 @@ struct KPassTCParams {
   const int32_t* teff;        // [B]
   const int32_t* prefix;      // [B+1]
   float* logits;              // [B][t_pad][H]
-  float* mpart;               // [k_slots][H], -inf on entry
+  float* mpart;               // [B][H]: each sequence's maxima, -inf on entry
   int32_t* status;
   int B, log2G, log2Hkv, MB, NB, t_pad;
   int log2tpt;                // tokens per tile = 128 / Hkv
@@ -894,7 +905,7 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       }
       if (last) {
         // this warp's maxima of the segment (all of its tiles precede this one in the walk)
-        float* mp = p.mpart + static_cast<size_t>(b + cta) * H;
+        float* mp = p.mpart + static_cast<size_t>(b) * H;   // the sequence's maxima
 #pragma unroll
         for (int h = 0; h < H; ++h) {
           const float w = warp_max_f32((h / G) == j ? m[h % G] : -INFINITY);
@@ -1309,12 +1320,11 @@ struct VPassParams {
   const int32_t* teff;
   const int32_t* prefix;
   const float* logits;    // [B][t_pad][H]
-  const float* mpart;     // [k_slots][H]: K-pass per-segment max of the logits
+  const float* mpart;     // [B][H]: each sequence's max of the logits (decode)
   float* zpart;           // [n_rr][H][v_slots][r_range]: sum_t w c_V per segment
   float* lpart;           // [v_slots][H]: sum_t w per segment (written by R range 0)
   int32_t* status;
   int B, H, npad, MB, NB, R, t_pad, r_range, n_rr, v_slots, stages;
-  int k_grid;             // CTAs of the K pass (its partition gives the segments to reduce)
   int n_chunks;           // 64-wide chunks per R range (r_range_pad/64); the last range may hold fewer
   int n_mtiles;           // r_range_pad / 128
   uint32_t tmem_cols;
@@ -1364,9 +1374,6 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
   Partition pt;
   pt.P = p.prefix[p.B];
   pt.G = static_cast<int32_t>(pt.P < gridDim.x ? pt.P : gridDim.x);
-  Partition ptk;            // the K pass's partition of the same pages
-  ptk.P = pt.P;
-  ptk.G = static_cast<int32_t>(pt.P < p.k_grid ? pt.P : p.k_grid);
   const int cta = blockIdx.x;
   const int rr = kChunk ? static_cast<int>(blockIdx.y) % p.n_rr : static_cast<int>(blockIdx.y);
   const int vg = kChunk ? static_cast<int>(blockIdx.y) / p.n_rr : 0;   // group of virtual heads (chunk mode)
@@ -1554,17 +1561,8 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
       if (!kChunk && (mt.flags & kFirst)) {   // (chunk mode: the weights arrive with the stage)
         // everyone is done with the previous segment's max
         if (!group_sync(pbar, pphase)) { set_timeout(p.status, kSiteVFull); abort_flag = 1; break; }
-        // max of the sequence's logits: the split reduction over its K-pass segments
-        const int32_t f0 = p.prefix[mt.b], f1 = p.prefix[mt.b + 1];
-        const int32_t i0 = part_owner(f0, ptk), i1 = part_owner(f1 - 1, ptk);
-        for (int h = et; h < p.npad; h += 128) {
-          float M = 0.f;
-          if (h < p.H) {
-            M = -INFINITY;
-            for (int32_t i = i0; i <= i1; ++i) M = fmaxf(M, p.mpart[static_cast<size_t>(mt.b + i) * p.H + h]);
-          }
-          sM[h] = M;
-        }
+        // max of the sequence's logits (merged by the K pass)
+        for (int h = et; h < p.npad; h += 128) sM[h] = h < p.H ? p.mpart[static_cast<size_t>(mt.b) * p.H + h] : 0.f;
         if (!group_sync(pbar, pphase)) { set_timeout(p.status, kSiteVFull); abort_flag = 1; break; }
         lsum = 0.f;
       }

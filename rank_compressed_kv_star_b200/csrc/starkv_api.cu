@@ -47,6 +47,9 @@
 #ifndef STARKV_V_PPS
 #define STARKV_V_PPS 1          // pages per ring stage of the decode V pass (at most)
 #endif
+#ifndef STARKV_K_CHUNK_BYTES
+#define STARKV_K_CHUNK_BYTES (1024 * 1024)   // codes per chunk of pages handed out by the K pass's counter
+#endif
 #ifndef STARKV_V_RING_BYTES
 #define STARKV_V_RING_BYTES (105 * 1024)
 #endif
@@ -94,7 +97,7 @@ starkv_status check_desc(const starkv_layer_desc* d) {
 struct DecodePlan {
   int H, Hkv, log2G, d, r, R, B, MB, NB, cap, n_pages_max, t_pad, npad;
   // K pass
-  int L, CPT, log2H, tps, k_stages, k_ctas;
+  int L, CPT, log2H, tps, k_stages, k_ctas, k_chunk_pages;
   uint32_t k_stage_bytes;
   size_t k_smem;
   // K pass on tensor cores (grouped queries)
@@ -218,6 +221,10 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   p.k_smem = static_cast<size_t>(p.k_stages) * p.k_stage_bytes + p.k_stages * sizeof(StageMeta) +
              2 * p.k_stages * sizeof(uint64_t);
   p.k_ctas = sms * STARKV_K_CTAS_PER_SM;
+  // pages per chunk handed out by the K pass's counter: about 1 MiB of codes (smaller chunks
+  // balance better but make a CTA change sequence, and reload its queries, more often)
+  p.k_chunk_pages = static_cast<int>(static_cast<uint32_t>(STARKV_K_CHUNK_BYTES) / (16u * tok));
+  if (p.k_chunk_pages < 1) p.k_chunk_pages = 1;
 
   // Grouped queries (G >= 2, H >= 8) with at most 16 KV heads: the K pass runs
   // on the tensor cores.  A CTA's single producer thread and per-tile chain are
@@ -334,7 +341,7 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   w.qt_off = off; off = align_up(off + static_cast<size_t>(batch) * p.H * p.r * 4, 256);
   w.logits_off = off; off = align_up(off + static_cast<size_t>(batch) * p.t_pad * p.H * 4, 256);
   w.k_ctas = p.k_ctas;
-  w.k_slots = p.k_ctas + batch;
+  w.k_slots = batch;   // one maximum per (sequence, head)
   w.mpart_off = off; off = align_up(off + static_cast<size_t>(w.k_slots) * p.H * 4, 256);
   w.v_ctas = p.v_ctas;
   w.v_slots = p.v_ctas + batch;
@@ -350,6 +357,10 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   w.total_bytes = off;
   return STARKV_OK;
 }
+
+// The K pass's page-chunk counter sits in the workspace's status area, 64
+// bytes after the status word; the absorption kernel sets it to 0.
+constexpr size_t kWorkCtrOffset = 64;
 
 size_t teff_offset(const DecodePlan& p) {
   return align_up(p.ws.prefix_off + (static_cast<size_t>(p.B) + 1) * 4, 256);
@@ -773,6 +784,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   float* mpart = reinterpret_cast<float*>(ws + pl.ws.mpart_off);
   float* lpart = reinterpret_cast<float*>(ws + pl.ws.lpart_off);
   float* zpart = reinterpret_cast<float*>(ws + pl.ws.zpart_off);
+  uint32_t* work_ctr = reinterpret_cast<uint32_t*>(ws + pl.ws.status_off + kWorkCtrOffset);
 
   if (max_seq_len == 0) {
     if (app && launch_prep(pl.d, app, nullptr, batch, s) != STARKV_OK) return STARKV_ERR_CUDA;
@@ -800,8 +812,9 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   ap.qt = qt; ap.prefix = prefix; ap.teff = teff; ap.status = status;
   __half* qth = pl.ktc ? reinterpret_cast<__half*>(ws + pl.ws.qth_off) : nullptr;
   ap.qth = qth;
-  ap.mpart_init = mpart;   // both K passes merge the segment maxima by float-max atomics
+  ap.mpart_init = mpart;   // both K passes merge each sequence's maxima by float-max atomics
   ap.n_mpart = pl.ws.k_slots * pl.H;
+  ap.work_ctr = work_ctr;
   ap.B = batch; ap.H = pl.H; ap.d = pl.d; ap.r = pl.r; ap.cap = pl.cap; ap.log2G = pl.log2G;
   ap.coef = scale * kLog2e;
   // the query absorption, with the step's compress-and-append in the same launch when fused
@@ -812,6 +825,7 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   kp.k_cache = static_cast<const __half*>(k_cache);
   kp.tables = block_tables; kp.row_seq = row_seq; kp.teff = teff; kp.prefix = prefix; kp.qt = qt;
   kp.logits = logits; kp.mpart = mpart; kp.status = status;
+  kp.work_ctr = work_ctr; kp.chunk_pages = pl.k_chunk_pages;
   kp.B = batch; kp.H = pl.H; kp.log2H = pl.log2H; kp.r = pl.r; kp.MB = pl.MB; kp.NB = pl.NB; kp.t_pad = pl.t_pad;
   kp.Hkv = pl.Hkv; kp.log2G = pl.log2G;
   kp.tps = pl.tps; kp.stages = pl.k_stages; kp.stage_bytes = pl.k_stage_bytes;
@@ -849,7 +863,6 @@ starkv_status decode_impl(const starkv_layer_desc* desc, int32_t batch, int32_t 
   vp.zpart = zpart; vp.lpart = lpart; vp.status = status;
   vp.B = batch; vp.H = pl.H; vp.npad = pl.npad; vp.MB = pl.MB; vp.NB = pl.NB; vp.R = pl.R;
   vp.t_pad = pl.t_pad; vp.r_range = pl.r_range; vp.n_rr = pl.n_rr; vp.v_slots = pl.ws.v_slots;
-  vp.k_grid = pl.k_ctas;
   vp.stages = pl.v_stages; vp.n_chunks = pl.n_chunks; vp.n_mtiles = pl.n_mtiles; vp.tmem_cols = pl.tmem_cols;
   vp.vtile_bytes = pl.vtile; vp.ltile_bytes = pl.ltile; vp.ptile_bytes = pl.ptile; vp.pps = pl.v_pps;
   if (!set_smem(vpass_kernel<false>, pl.v_smem)) return STARKV_ERR_CUDA;
@@ -1222,7 +1235,6 @@ starkv_status chunk_prefill(const ChunkPlan& c, const void* q, const void* B_K, 
   vp.mpart = mpart; vp.zpart = zpart; vp.lpart = lpart; vp.status = status;
   vp.B = c.nv_max; vp.H = c.H; vp.npad = c.lw; vp.MB = c.MB; vp.NB = c.NB; vp.R = c.R;
   vp.t_pad = c.t_pad; vp.r_range = c.r_range; vp.n_rr = c.n_rr; vp.v_slots = c.v_slots;
-  vp.k_grid = c.k_ctas;
   vp.stages = c.v_stages; vp.n_chunks = c.n_chunks; vp.n_mtiles = c.n_mtiles; vp.tmem_cols = c.v_tmem;
   vp.vtile_bytes = c.vtile; vp.ltile_bytes = c.ltile; vp.ptile_bytes = c.ptile; vp.pps = c.v_pps; vp.wts = wts;
   vp.Hv = c.Hv; vp.n_vg = c.n_vg; vp.log2nq = c.log2nq; vp.lw = c.lw;

@@ -118,7 +118,7 @@ def test_workspace_layout_is_consistent(lib):
     offs = [lay.status_off, lay.prefix_off, lay.qt_off, lay.logits_off, lay.mpart_off,
             lay.lpart_off, lay.zpart_off]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
-    assert lay.t_pad == 8192 and lay.k_slots == lay.k_ctas + 64 and lay.v_slots == lay.v_ctas + 64
+    assert lay.t_pad == 8192 and lay.k_slots == 64 and lay.v_slots == lay.v_ctas + 64
     assert lay.n_rranges * lay.r_range >= 2048
     assert lay.logits_off + 64 * 8192 * 32 * 4 <= lay.mpart_off
     # grows with batch and length
