@@ -1576,10 +1576,11 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
           uint8_t* pt_j = ptiles + static_cast<size_t>(s) * pstage + static_cast<size_t>(j) * p.ptile_bytes;
           const int ntj = j == np - 1 ? ntl : kBlock;
           for (int t = t_w0; t < kBlock; t += t_step) {
-            // unnormalised weight exp2(s - M) <= 1, rounded to fp16 for the MMA; the
-            // normaliser sums exactly the rounded weights
+            // unnormalised weight exp2(s - M) <= 1 (hardware ex2: about 2^-22
+            // relative error, far below the fp16 rounding that follows), rounded
+            // to fp16 for the MMA; the normaliser sums exactly the rounded weights
             __half w = __float2half_rn(0.f);
-            if (t < ntj && h_w < p.H) w = __float2half_rn(exp2f(lt[t * p.H + h_w] - m_h));
+            if (t < ntj && h_w < p.H) w = __float2half_rn(ex2_approx(lt[t * p.H + h_w] - m_h));
             lsum += __half2float(w);
             const uint32_t off = static_cast<uint32_t>(t >> 3) * lbo_b + static_cast<uint32_t>(h_w >> 3) * 128u +
                                  static_cast<uint32_t>(h_w & 7) * 16u + static_cast<uint32_t>(t & 7) * 2u;
