@@ -928,17 +928,19 @@ kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
 // ============================================================ kpass (chunks)
 // Read-once K pass of a chunked prefill on tcgen05.  The virtual heads (h, i)
 // of a virtual sequence (query head h of its chunk row i) that share KV head
-// g(h) share its K codes, so with 16 virtual heads per KV head (G query heads
-// x nq rows) a tile is one page of a group of 8 KV heads (row 8 t + j: token
-// t, KV head j of the group), one 3-D TMA box {64 codes, 8 heads, 16 tokens}
-// per 64 codes, and B holds the 128 virtual heads of the group (rows: fp16
-// high parts, then the low parts), loaded once per (segment, group).  A CTA
-// walks each virtual sequence of its page range once per group, so every K
-// page is read once in total.  An epilogue warp owns four tokens of the tile
-// (32 rows, all 8 KV heads): four 32-column TMEM loads per tile, each lane
-// keeps its KV head's 16 columns, sets logits past a row's causal limit to
-// -inf, stores the 16 as consecutive logits and keeps running maxima that are
-// merged into the segment slots (float max) at the end of each pass.
+// g(h) share its K codes: VPK = G x nq of them per KV head, with nq = 16 rows
+// per virtual sequence for G <= 4 (a 16-row chunk is one virtual sequence and
+// every page is read once) and VPK = 64 above (nq = 64 / G).  A tile is 128
+// rows (token, KV head) of KVT KV heads: one page of 8 KV heads (VPK <= 32),
+// or two pages of 4 KV heads (VPK = 64), one 3-D TMA box {64 codes, KVT
+// heads, 16 tokens} per page and 64 codes; B holds the KVT x VPK virtual heads
+// of the group (rows: fp16 high parts, then the low parts), loaded once per
+// (segment, group), and the MMA has N = KVT x VPK (128 or 256).  A CTA walks
+// each virtual sequence of its page range once per group.  An epilogue lane
+// owns one row: it keeps its KV head's VPK columns, sets logits past the
+// row's causal limit or the sequence end to -inf, stores them as consecutive
+// logits and keeps running maxima that are merged into the segment slots
+// (float max) at the end of each pass.
 struct KPassChunkParams {
   const int32_t* tables;      // [n_seqs][MB]
   const int32_t* vs_seq;      // [B] sequence of each virtual sequence
@@ -949,25 +951,34 @@ struct KPassChunkParams {
   float* mpart;               // [k_slots][Hv], -inf on entry
   int32_t* status;
   int B, MB, NB, t_pad;
-  int Hv, n_vg, log2lw;       // virtual heads, groups of lw = min(256, Hv) of them
-  int n_groups;               // KV-head groups of 8
+  int Hv, n_vg, log2lw;       // virtual heads, groups of lw of them (lw >= VPK)
+  int n_groups;               // KV-head groups of KVT
   int log2nq;
   int ksteps, kb;             // UMMA K steps of 16 codes; 64-code column blocks
   int nacc, nbs, stages;
   uint32_t a_bytes;           // kb * 16 KiB
-  uint32_t b_bytes;           // kb * 256 rows * 128 B
+  uint32_t b_bytes;           // kb * 2 * N rows * 128 B
   uint32_t tmem_cols;
   int drop_stage;             // test hook (-1: off)
 };
 
-constexpr int kKChunkCols = 128;   // virtual heads of a KV-head group (8 x 16): UMMA N
+// Tile geometry for VPK virtual heads per KV head.
+template <int VPK>
+struct ChunkTile {
+  static constexpr int kKvt = VPK >= 64 ? 4 : 8;    // KV heads per tile
+  static constexpr int kCols = kKvt * VPK;           // UMMA N (128 or 256)
+  static constexpr int kTokens = 128 / kKvt;          // tokens per tile (16 or 32)
+  static constexpr int kPages = kTokens / kBlock;    // pages per tile (1 or 2)
+};
 
-// Calls f(v, pg, nt, g, first, last) for the tiles of pages [p0, p1): page pg
-// (tokens [16 pg, 16 pg + nt)) of virtual sequence v for KV-head group g,
-// each (v, g) pass over the CTA's pages of v in page order, `first` / `last`
-// on the pass's first and final tile.  Stops when f returns false.
+// Calls f(v, pg, np, nt, g, first, last) for the tiles of pages [p0, p1): np
+// (<= ppt) consecutive pages from page pg of virtual sequence v (tokens [16 pg,
+// 16 pg + nt)) for KV-head group g, each (v, g) pass over the CTA's pages of
+// v in page order, `first` / `last` on the pass's first and final tile.  Stops
+// when f returns false.
 template <typename F>
-__device__ __forceinline__ void for_each_chunk_tile(const KPassChunkParams& p, int64_t p0, int64_t p1, F&& f) {
+__device__ __forceinline__ void for_each_chunk_tile(const KPassChunkParams& p, int64_t p0, int64_t p1, int ppt,
+                                                    F&& f) {
   int32_t v = seq_of_page(p.prefix, p.B, p0);
   int64_t x = p0;
   while (x < p1) {
@@ -976,17 +987,21 @@ __device__ __forceinline__ void for_each_chunk_tile(const KPassChunkParams& p, i
     const int32_t base = p.prefix[v];
     const int32_t T = p.teff[v];
     for (int g = 0; g < p.n_groups; ++g)
-      for (int64_t y = x; y < seg_end; ++y) {
+      for (int64_t y = x; y < seg_end; y += ppt) {
         const int32_t pg = static_cast<int32_t>(y - base);
-        if (!f(v, pg, min(kBlock, T - pg * kBlock), g, y == x, y == seg_end - 1)) return;
+        const int np = static_cast<int>(min(static_cast<int64_t>(ppt), seg_end - y));
+        if (!f(v, pg, np, min(np * kBlock, T - pg * kBlock), g, y == x, y + ppt >= seg_end)) return;
       }
     x = seg_end;
   }
 }
 
+template <int VPK>
 __global__ void __launch_bounds__(kKTCThreads, 1)
 kpass_chunk_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                    KPassChunkParams p) {
+  using Geo = ChunkTile<VPK>;
+  constexpr int KVT = Geo::kKvt, NCOL = Geo::kCols, PPT = Geo::kPages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages;
@@ -1027,6 +1042,7 @@ kpass_chunk_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
   const uint32_t taddr = taddr_s;
   const int64_t p0 = part_begin(cta, pt), p1 = part_begin(cta + 1, pt);
   const int nq1 = (1 << p.log2nq) - 1;
+  constexpr uint32_t kBoxBytes = static_cast<uint32_t>(KVT) * kBlock * 128u;   // one page of KVT heads, 64 codes
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -1039,27 +1055,31 @@ kpass_chunk_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
       uint32_t su = 0, bu = 0, issued = 0;
       int32_t bpar[2] = {-1, -1};
       bool ok = true;
-      for_each_chunk_tile(p, p0, p1, [&](int32_t v, int32_t pg, int32_t, int g, bool first, bool last) {
+      for_each_chunk_tile(p, p0, p1, PPT, [&](int32_t v, int32_t pg, int np, int32_t, int g, bool first, bool last) {
         if (first) {
           if (bu > 0 && !mbar_wait(&bempty[bi], (bu - 1) & 1)) { ok = false; return false; }
           bpar[bi] = static_cast<int32_t>(bu & 1);
           mbar_arrive_expect_tx(&bfull[bi], p.b_bytes);
-          const int hi_row = v * 2 * p.Hv + g * kKChunkCols;
+          const int hi_row = v * 2 * p.Hv + g * NCOL;
           for (int a = 0; a < p.kb; ++a) {
-            uint8_t* dst = bslot + bi * static_cast<size_t>(p.b_bytes) + static_cast<size_t>(a) * 256 * 128;
+            uint8_t* dst = bslot + bi * static_cast<size_t>(p.b_bytes) + static_cast<size_t>(a) * 2 * NCOL * 128;
             tma_load_2d(dst, &qmap, a * 64, hi_row, &bfull[bi], reuse);
-            tma_load_2d(dst + kKChunkCols * 128, &qmap, a * 64, hi_row + p.Hv, &bfull[bi], reuse);
+            tma_load_2d(dst + NCOL * 128, &qmap, a * 64, hi_row + p.Hv, &bfull[bi], reuse);
           }
         }
         if (su > 0 && !mbar_wait(&empty[si], (su - 1) & 1)) { ok = false; return false; }
         uint8_t* st = smem + static_cast<size_t>(si) * p.a_bytes;
         const bool drop = static_cast<int>(issued) == p.drop_stage;
         if (!drop) {
-          mbar_arrive_expect_tx(&full[si], static_cast<uint32_t>(p.kb) * 16384u);
-          int32_t phys = table_row(p.tables, p.vs_seq, v, p.MB)[pg];
-          if (phys < 0 || phys >= p.NB) { set_flag(p.status, STARKV_FLAG_BAD_BLOCK_ID); phys = 0; }
-          for (int a = 0; a < p.kb; ++a)
-            tma_load_3d(st + static_cast<size_t>(a) * 16384, &kmap, a * 64, g * 8, phys * kBlock, &full[si], stream);
+          mbar_arrive_expect_tx(&full[si], static_cast<uint32_t>(np * p.kb) * kBoxBytes);
+          const int32_t* trow = table_row(p.tables, p.vs_seq, v, p.MB);
+          for (int pp = 0; pp < np; ++pp) {
+            int32_t phys = trow[pg + pp];
+            if (phys < 0 || phys >= p.NB) { set_flag(p.status, STARKV_FLAG_BAD_BLOCK_ID); phys = 0; }
+            for (int a = 0; a < p.kb; ++a)
+              tma_load_3d(st + static_cast<size_t>(a) * 16384 + static_cast<size_t>(pp) * kBoxBytes, &kmap, a * 64,
+                          g * KVT, phys * kBlock, &full[si], stream);
+          }
         }
         ++issued;
         if (++si == S) { si = 0; ++su; }
@@ -1082,24 +1102,24 @@ kpass_chunk_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
-      const uint32_t idesc = idesc_f16_f32(128, kKChunkCols, /*a_mn_major=*/false, /*b_mn_major=*/false);
-      const uint32_t b_atom = 256u * 8u;    // one 64-code block of B: 256 rows * 128 bytes >> 4
+      const uint32_t idesc = idesc_f16_f32(128, NCOL, /*a_mn_major=*/false, /*b_mn_major=*/false);
+      const uint32_t b_atom = 2u * NCOL * 8u;   // one 64-code block of B: 2N rows * 128 bytes >> 4
       int si = 0, bi = 0, ai = 0;
       uint32_t su = 0, bu = 0, au = 0;
       bool ok = true;
-      for_each_chunk_tile(p, p0, p1, [&](int32_t, int32_t, int32_t, int, bool, bool last) {
+      for_each_chunk_tile(p, p0, p1, PPT, [&](int32_t, int32_t, int, int32_t, int, bool, bool last) {
         if (!mbar_wait(&bfull[bi], bu & 1)) { ok = false; return false; }
         if (au > 0 && !mbar_wait(&tempty[ai], (au - 1) & 1)) { ok = false; return false; }
         if (!mbar_wait(&full[si], su & 1) || abort_flag) { ok = false; return false; }
         tc_fence_after();
         const uint64_t da = smem_desc(smem_u32(smem + static_cast<size_t>(si) * p.a_bytes), 16u, 1024u, kSwizzle128B);
         const uint64_t db = smem_desc(smem_u32(bslot + bi * static_cast<size_t>(p.b_bytes)), 16u, 1024u, kSwizzle128B);
-        const uint32_t d = taddr + static_cast<uint32_t>(ai * kKChunkCols);
+        const uint32_t d = taddr + static_cast<uint32_t>(ai * NCOL);
         for (int ks = 0; ks < p.ksteps; ++ks) {
           const uint32_t a = ks >> 2, kk = ks & 3;
           const uint64_t dak = da + (a * 1024u + kk * 2u), dbk = db + (a * b_atom + kk * 2u);
-          umma_f16_ss(d, dak, dbk, idesc, ks > 0 ? 1u : 0u);                           // high parts
-          umma_f16_ss(d, dak, dbk + static_cast<uint32_t>(kKChunkCols) * 8u, idesc, 1u);  // low parts
+          umma_f16_ss(d, dak, dbk, idesc, ks > 0 ? 1u : 0u);                       // high parts
+          umma_f16_ss(d, dak, dbk + static_cast<uint32_t>(NCOL) * 8u, idesc, 1u);  // low parts
         }
         umma_commit(&empty[si]);
         umma_commit(&tfull[ai]);
@@ -1117,75 +1137,87 @@ kpass_chunk_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // warp quarter q holds rows 32q..32q+31: tokens 4q..4q+3, all 8 KV heads;
-    // lane L: token 4q + L/8, KV head L % 8 of the group (columns 16 j .. 16 j + 15)
+    // warp quarter q holds tile rows 32q..32q+31; lane L: row 32q + L = token
+    // (32q + L) / KVT of the tile, KV head (L % KVT) of the group, whose
+    // columns are [VPK j, VPK j + VPK)
     const int q = warp & 3;
-    const int jl = lane & 7;
-    const int t = 4 * q + (lane >> 3);
+    const int row = 32 * q + lane;
+    const int jl = row % KVT;
+    const int t = row / KVT;
     const uint64_t keep = policy_evict_last();       // logits: read back by the V pass
     const uint32_t tq = taddr + (static_cast<uint32_t>(q * 32) << 16);
-    float m[16];
+    float m[VPK];
 #pragma unroll
-    for (int c = 0; c < 16; ++c) m[c] = -INFINITY;
+    for (int c = 0; c < VPK; ++c) m[c] = -INFINITY;
     int ai = 0;
     uint32_t au = 0;
     bool ok = true;
-    for_each_chunk_tile(p, p0, p1, [&](int32_t v, int32_t pg, int32_t nt, int g, bool, bool last) {
+    for_each_chunk_tile(p, p0, p1, PPT, [&](int32_t v, int32_t pg, int, int32_t nt, int g, bool, bool last) {
       const bool ready = mbar_wait(&tfull[ai], au & 1);
       if (!__all_sync(0xffffffffu, ready && !abort_flag)) { ok = false; return false; }
       tc_fence_after();
-      float xs[16];
+      float xs[VPK];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {   // columns 32 c4 .. 32 c4 + 31: KV heads 2 c4, 2 c4 + 1
+      for (int cb = 0; cb < NCOL / 32; ++cb) {   // columns 32 cb .. 32 cb + 31
         uint32_t w[32];
-        tmem_ld_32x32b_x32(tq + static_cast<uint32_t>(ai * kKChunkCols + 32 * c4), w);
+        tmem_ld_32x32b_x32(tq + static_cast<uint32_t>(ai * NCOL + 32 * cb), w);
         tmem_ld_wait();
-        if ((jl >> 1) == c4) {
+        if constexpr (VPK == 16) {             // two KV heads per block
+          if ((jl >> 1) == cb) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) xs[c] = __uint_as_float((jl & 1) ? w[16 + c] : w[c]);
+            for (int c = 0; c < 16; ++c) xs[c] = __uint_as_float((jl & 1) ? w[16 + c] : w[c]);
+          }
+        } else {                               // VPK / 32 blocks per KV head
+          if (jl == cb / (VPK / 32)) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) xs[(cb % (VPK / 32)) * 32 + c] = __uint_as_float(w[c]);
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[ai]);
       if (++ai == p.nacc) { ai = 0; ++au; }
-      const int kv = g * 8 + jl;                     // KV head of this lane's row
       {
-        // every slot of the page gets a logit: -inf past the sequence end too
+        // every token slot of the tile's pages gets a logit: -inf past the
+        // sequence end too
         const int32_t tabs = pg * kBlock + t;
         const int32_t nrows = p.vs_nrows[v];
         const int32_t rel = tabs - (p.teff[v] - nrows);   // rows i >= rel see this token
-        float o[16];
+        float o[VPK];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < VPK; ++c) {
           const int i = c & nq1;
           o[c] = (t < nt && i < nrows && i >= rel) ? xs[c] : -INFINITY;
           m[c] = fmaxf(m[c], o[c]);
         }
-        const int vh = kv * 16;                       // 16 consecutive virtual heads, in one group
-        const size_t lrow_idx = (static_cast<size_t>(v) * p.n_vg + (vh >> p.log2lw)) * p.t_pad + tabs;
-        float* lrow = p.logits + (lrow_idx << p.log2lw) + (vh & ((1 << p.log2lw) - 1));
+        if (t < ((nt + kBlock - 1) & ~(kBlock - 1))) {   // tokens of pages this tile loaded
+          const int vh = g * NCOL + jl * VPK;            // VPK consecutive virtual heads, in one group
+          const size_t lrow_idx = (static_cast<size_t>(v) * p.n_vg + (vh >> p.log2lw)) * p.t_pad + tabs;
+          float* lrow = p.logits + (lrow_idx << p.log2lw) + (vh & ((1 << p.log2lw) - 1));
 #pragma unroll
-        for (int c = 0; c < 16; c += 4)
-          st_global_hint(reinterpret_cast<float4*>(lrow + c), make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]), keep);
+          for (int c = 0; c < VPK; c += 4)
+            st_global_hint(reinterpret_cast<float4*>(lrow + c), make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]),
+                           keep);
+        }
       }
       if (last) {
-        // the maxima of this (segment, group) pass: over the warp's 4 tokens (lanes jl, jl+8, jl+16, jl+24)
+        // the maxima of this (segment, group) pass over the warp's rows of each KV head
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < VPK; ++c) {
           float x = m[c];
-          x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
-          x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
+#pragma unroll
+          for (int o2 = KVT; o2 < 32; o2 <<= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o2));
           m[c] = x;
         }
-        if (lane < 8) {
-          float* mp = p.mpart + static_cast<size_t>(v + cta) * p.Hv + kv * 16;
+        if (lane < KVT) {
+          float* mp = p.mpart + static_cast<size_t>(v + cta) * p.Hv + g * NCOL + jl * VPK;
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
+          for (int c = 0; c < VPK; ++c)
             if (m[c] > -INFINITY) atomic_max_f32(mp + c, m[c]);
         }
 #pragma unroll
-        for (int c = 0; c < 16; ++c) m[c] = -INFINITY;
+        for (int c = 0; c < VPK; ++c) m[c] = -INFINITY;
       }
       return true;
     });

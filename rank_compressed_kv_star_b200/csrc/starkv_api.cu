@@ -1004,6 +1004,7 @@ namespace {
 // Shapes: KV heads in groups of 8 (Hkv % 8 == 0), G = H / Hkv <= 16.
 struct ChunkPlan {
   int H, Hkv, d, r, R, G, nq, log2nq, Hv, lw, n_vg, nv_max, n_groups, t_pad, MB, NB, n_rows, n_seqs, n_pc;
+  int vpk, kvt, kcols;   // virtual heads per KV head, KV heads per K tile, its UMMA N
   // K pass
   int k_ctas, kb, ksteps, k_stages, nacc, nbs;
   uint32_t a_bytes, b_bytes, k_tmem;
@@ -1021,6 +1022,20 @@ struct ChunkPlan {
       mpart_off, lpart_off, lwpart_off, wts_off, zpart_off, total;
 };
 
+cudaError_t launch_kpass_chunk(int vpk, size_t smem, int ctas, const CUtensorMap& kmap, const CUtensorMap& qmap,
+                               const KPassChunkParams& kp, cudaStream_t s) {
+  if (vpk == 16) {
+    if (!set_smem(kpass_chunk_kernel<16>, smem)) return cudaErrorInvalidValue;
+    return launch(kpass_chunk_kernel<16>, dim3(ctas), dim3(kKTCThreads), smem, s, 1, kmap, qmap, kp);
+  }
+  if (vpk == 32) {
+    if (!set_smem(kpass_chunk_kernel<32>, smem)) return cudaErrorInvalidValue;
+    return launch(kpass_chunk_kernel<32>, dim3(ctas), dim3(kKTCThreads), smem, s, 1, kmap, qmap, kp);
+  }
+  if (!set_smem(kpass_chunk_kernel<64>, smem)) return cudaErrorInvalidValue;
+  return launch(kpass_chunk_kernel<64>, dim3(ctas), dim3(kKTCThreads), smem, s, 1, kmap, qmap, kp);
+}
+
 bool chunk_eligible(const starkv_layer_desc* d) {
   const int Hkv = kv_heads(d);
   return Hkv % 8 == 0 && d->num_heads / Hkv <= 16;
@@ -1037,7 +1052,13 @@ starkv_status make_chunk_plan(const starkv_layer_desc* d, int32_t n_seqs, int32_
   ChunkPlan& c = *cp;
   std::memset(&c, 0, sizeof(c));
   c.H = d->num_heads; c.Hkv = kv_heads(d); c.d = d->head_dim; c.r = d->k_rank; c.R = d->v_rank;
-  c.G = c.H / c.Hkv; c.nq = 16 / c.G;
+  // VPK virtual heads per KV head: all 16 rows of a chunk (one virtual
+  // sequence, pages read once) while G <= 4, 64 of them above (nq = 64 / G)
+  c.G = c.H / c.Hkv;
+  c.vpk = 16 * c.G < 64 ? 16 * c.G : 64;
+  c.nq = c.vpk / c.G;
+  c.kvt = c.vpk >= 64 ? 4 : 8;
+  c.kcols = c.kvt * c.vpk;
   while ((1 << c.log2nq) < c.nq) ++c.log2nq;
   c.Hv = c.H * c.nq;
   c.lw = c.Hv < 256 ? c.Hv : 256;
@@ -1048,17 +1069,17 @@ starkv_status make_chunk_plan(const starkv_layer_desc* d, int32_t n_seqs, int32_
     c.nv_max = static_cast<int>(bound < n_rows ? bound : n_rows);
     if (c.nv_max < 1) c.nv_max = 1;
   }
-  c.n_groups = c.Hkv / 8;
+  c.n_groups = c.Hkv / c.kvt;
   c.t_pad = (max_seq_len + 15) / 16 * 16;
   c.MB = d->max_blocks_per_seq; c.NB = d->num_blocks;
   const int sms = device_sm_count();
-  // K pass: one CTA per SM, two query-tile slots, up to 8 stages, 4 accumulators of 128 columns
+  // K pass: one CTA per SM, two query-tile slots, up to 8 stages, accumulators of kcols columns
   c.kb = (c.r + 63) / 64;
   c.ksteps = (c.r + 15) / 16;
   c.a_bytes = static_cast<uint32_t>(c.kb) * 16384u;
-  c.b_bytes = static_cast<uint32_t>(c.kb) * 256u * 128u;
+  c.b_bytes = static_cast<uint32_t>(c.kb) * 2u * c.kcols * 128u;
   c.nbs = 2;
-  c.nacc = 4;
+  c.nacc = 512 / c.kcols;
   c.k_tmem = 512;
   {
     const size_t fixed = 1024 + c.nbs * static_cast<size_t>(c.b_bytes) + (4 + 2 * kKTCMaxAcc + 1) * 8;
@@ -1078,7 +1099,7 @@ starkv_status make_chunk_plan(const starkv_layer_desc* d, int32_t n_seqs, int32_
   {
     const int rpad = (c.R + 127) / 128 * 128;
     int64_t best = -1;
-    for (int lw = c.Hv < STARKV_CV_LW_MAX ? c.Hv : STARKV_CV_LW_MAX; lw >= 32; lw /= 2)
+    for (int lw = c.Hv < STARKV_CV_LW_MAX ? c.Hv : STARKV_CV_LW_MAX; lw >= 32 && lw >= c.vpk; lw /= 2)
       for (int mt = 512 / lw; mt >= 1; mt /= 2) {
         if (mt * 128 > rpad && mt > 1) continue;
         const int n_vg = c.Hv / lw;
@@ -1180,9 +1201,9 @@ starkv_status chunk_prefill(const ChunkPlan& c, const void* q, const void* B_K, 
   float* zpart = reinterpret_cast<float*>(ws + c.zpart_off);
 
   CUtensorMap kmap, qmap, vmap, bvmap, zmap;
-  if (!encode_kpool_map(&kmap, k_cache, c.r, c.Hkv, c.NB, 8, 16) ||
+  if (!encode_kpool_map(&kmap, k_cache, c.r, c.Hkv, c.NB, static_cast<uint32_t>(c.kvt), 16) ||
       !encode_2d_map(&qmap, qth, static_cast<uint64_t>(c.r), static_cast<uint64_t>(c.nv_max) * 2 * c.Hv, 64,
-                     kKChunkCols) ||
+                     static_cast<uint32_t>(c.kcols)) ||
       !encode_vpool_map(&vmap, v_cache, c.R, c.NB, static_cast<uint32_t>(c.n_chunks)) ||
       !encode_2d_map(&bvmap, B_V, static_cast<uint64_t>(c.Hkv) * c.d, static_cast<uint64_t>(c.R), 64, kFinKC) ||
       !encode_f32_rows_map(&zmap, zpart, static_cast<uint64_t>(c.r_range),
@@ -1220,9 +1241,7 @@ starkv_status chunk_prefill(const ChunkPlan& c, const void* q, const void* B_K, 
   kp.ksteps = c.ksteps; kp.kb = c.kb; kp.nacc = c.nacc; kp.nbs = c.nbs; kp.stages = c.k_stages;
   kp.a_bytes = c.a_bytes; kp.b_bytes = c.b_bytes; kp.tmem_cols = c.k_tmem;
   kp.drop_stage = g_drop_k_stage.load(std::memory_order_relaxed);
-  if (!set_smem(kpass_chunk_kernel, c.k_smem)) return STARKV_ERR_CUDA;
-  if (launch(kpass_chunk_kernel, dim3(c.k_ctas), dim3(kKTCThreads), c.k_smem, s, 1, kmap, qmap, kp) != cudaSuccess)
-    return STARKV_ERR_CUDA;
+  if (launch_kpass_chunk(c.vpk, c.k_smem, c.k_ctas, kmap, qmap, kp, s) != cudaSuccess) return STARKV_ERR_CUDA;
 
   ChunkWeightsParams wp{logits, wts,  mpart,   teff,  prefix,   lwpart,
                         c.nv_max, c.Hv, c.n_vg, c.lw, kp.log2lw, c.t_pad, c.k_ctas, c.n_pc};

@@ -385,9 +385,14 @@ def test_prefill_rows_of_one_sequence_span_tiles():
 
 
 def test_prefill_read_once_shapes():
-    """Read-once path with 8 query heads per KV head (2 rows per virtual sequence), and 16-row chunks
-    of several sequences over long contexts (the benchmark's chunk size)."""
+    """Read-once path for every tile geometry: 8 query heads per KV head (64 virtual heads per KV
+    head, 8 rows per virtual sequence, K tiles of 4 KV heads over two pages), 2 per KV head (32
+    virtual heads, N = 256 tiles of 8 KV heads), 4 per KV head with odd page counts (two-page tiles
+    that end on one page), and 16-row chunks of several sequences over long contexts (the
+    benchmark's chunk size)."""
     _prefill_check(8, starts=[0, 333, 1500], chunks=[5, 16, 33], seed=6262, H=64, r=64, R=512)
+    _prefill_check(16, starts=[0, 333, 1500, 47], chunks=[5, 16, 33, 17], seed=6265, H=32, r=64, R=1024)
+    _prefill_check(8, starts=[1, 15, 16, 300, 4000], chunks=[16, 1, 16, 20, 3], seed=6266, H=32, r=32, R=512)
     _prefill_check(0, starts=[2048, 700, 1601, 16], chunks=[16, 16, 16, 16], seed=6363)
 
 
