@@ -636,20 +636,37 @@ def run_prefill(args):
     clk = clocks.stop()
     ms = t0.elapsed_time(t1) / K
 
-    # end to end: host chunk inputs in, outputs back, every step
+    # end to end: every step copies the chunk's inputs from pinned host memory,
+    # runs the step and copies its output back to pinned host memory; two sets
+    # of device buffers let a step's copies overlap the previous step's kernels
     hin = [x.cpu().pin_memory() for x in (qd, kd, vd, sd, st_d, of_d)]
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    dbuf = [torch.empty_like(x) for x in (qd, kd, vd, sd, st_d, of_d)]
+    dbuf = [[torch.empty_like(x) for x in (qd, kd, vd, sd, st_d, of_d)] for _ in range(2)]
+    dout = [torch.empty_like(out) for _ in range(2)]
+    copy_s, back_s = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in, ev_run, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
     Ke = max(1, min(args.e2e_steps, K))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(Ke):
-        for h, dd in zip(hin, dbuf):
-            dd.copy_(h, non_blocking=True)
-        step(*dbuf)
-        hout.copy_(out, non_blocking=True)
-    e1.record(stream)
+    e0.record(copy_s)
+    for i in range(Ke):
+        j = i % 2
+        with torch.cuda.stream(copy_s):
+            if i >= 2:
+                copy_s.wait_event(ev_run[j])
+            for h, dd in zip(hin, dbuf[j]):
+                dd.copy_(h, non_blocking=True)
+            ev_in[j].record(copy_s)
+        stream.wait_event(ev_in[j])
+        if i >= 2:
+            stream.wait_event(ev_out[j])
+        step(*dbuf[j], o=dout[j])
+        ev_run[j].record(stream)
+        with torch.cuda.stream(back_s):
+            back_s.wait_event(ev_run[j])
+            hout.copy_(dout[j], non_blocking=True)
+            ev_out[j].record(back_s)
+    e1.record(back_s)
     torch.cuda.synchronize()
     ms_e2e = e0.elapsed_time(e1) / Ke
     h2d = sum(x.numel() * x.element_size() for x in hin)

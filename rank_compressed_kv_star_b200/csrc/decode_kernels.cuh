@@ -215,13 +215,14 @@ struct AbsorbParams {
   int log2nq;
 };
 
-// One item: query head h, sequences [b0, b0 + tile) (tile <= kAbsBT).  Item 0
+// One item: query head h, sequences [b0, b0 + tile) (tile <= kAbsBigTile).  Item 0
 // also writes the page prefix sums and resets the status word (every later
 // kernel of the decode runs after this one); all items share setting the
 // segment-max slots to -inf.  B_K[g(h)] is staged transposed ([d][r]) and the
 // tile's q rows as they are, both in shared memory (`smem`: d*r + tile*d
 // halves), for the shared small-product routine.
 constexpr int kAbsBT = 32;
+constexpr int kAbsBigTile = 128;   // rows per absorption item when the absorption runs alone over many rows
 
 __device__ __forceinline__ void absorb_item(const AbsorbParams& p, int item, int n_items, int tile, uint8_t* smem) {
   const int h = item % p.H;

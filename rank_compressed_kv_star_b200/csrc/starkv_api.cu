@@ -645,6 +645,10 @@ starkv_status launch_prep(int d, const AppendPlan* app, const AbsorbParams* abs,
   const int r = app ? app->kp.r : abs->r;
   int tile = 16;
   if ((k_heads + a_heads) * ((batch + tile - 1) / tile) > spare) tile = kAbsBT;
+  // an absorption alone over many rows (a chunked prefill): items of 128 rows,
+  // so that each B_K slice is staged for 4x more rows and the grid stays
+  // within a few waves
+  if (!app && a_heads * ((batch + tile - 1) / tile) > 2 * spare) tile = kAbsBigTile;
   size_t smem = 0;
   CUtensorMap none;
   std::memset(&none, 0, sizeof(none));
