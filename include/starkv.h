@@ -251,13 +251,14 @@ starkv_status starkv_append_decode_host(const starkv_layer_desc* desc, int32_t b
  *                 max_seq_len) bytes, 256-byte aligned
  *   out           fp16 [n_rows][H][d]
  *
- * When the KV heads come in groups of 8 and H / Hkv <= 16, a chunk is read
- * once: its rows are taken nq = 16 / (H / Hkv) at a time, and each group of
+ * When the KV heads come in groups of 8 and G = H / Hkv <= 16, a chunk's rows
+ * are taken nq at a time (nq = 16 for G <= 4, 64 / G above), and each group of
  * nq rows streams the sequence's K and V pages once for all of its rows (the
- * rows' query heads act as nq x H query heads with per-row causal limits).
- * Other shapes evaluate every row as one decode row (its own length, the
- * sequence's block table), reading the pages once per row.  The workspace
- * holds logits of every virtual head: it grows with (n_rows / nq + n_seqs) x
+ * rows' query heads act as nq x H query heads with per-row causal limits): a
+ * chunk of up to 16 rows reads every page once when G <= 4.  Other shapes
+ * evaluate every row as one decode row (its own length, the sequence's block
+ * table), reading the pages once per row.  The workspace holds the logits and
+ * fp16 weights of every virtual head: it grows with (n_rows / nq + n_seqs) x
  * max_seq_len x H x nq.  Errors as starkv_paged_decode.
  */
 size_t starkv_prefill_workspace_bytes(const starkv_layer_desc* desc, int32_t n_seqs, int32_t n_rows,
