@@ -50,6 +50,9 @@
 #ifndef STARKV_K_CHUNK_BYTES
 #define STARKV_K_CHUNK_BYTES (1024 * 1024)   // codes per chunk of pages handed out by the K pass's counter
 #endif
+#ifndef STARKV_V_MIN_PAGES
+#define STARKV_V_MIN_PAGES 16   // fewest pages per decode V-pass CTA when a call has few pages
+#endif
 #ifndef STARKV_V_RING_BYTES
 #define STARKV_V_RING_BYTES (105 * 1024)
 #endif
@@ -222,8 +225,15 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
              2 * p.k_stages * sizeof(uint64_t);
   p.k_ctas = sms * STARKV_K_CTAS_PER_SM;
   // pages per chunk handed out by the K pass's counter: about 1 MiB of codes (smaller chunks
-  // balance better but make a CTA change sequence, and reload its queries, more often)
+  // balance better but make a CTA change sequence, and reload its queries, more often),
+  // and at least four chunks per CTA when the call has few pages
   p.k_chunk_pages = static_cast<int>(static_cast<uint32_t>(STARKV_K_CHUNK_BYTES) / (16u * tok));
+  {
+    const int64_t pages_max = static_cast<int64_t>(batch) * ((p.cap + 15) / 16);
+    const int64_t per_cta =
+        (pages_max + 4 * static_cast<int64_t>(p.k_ctas) - 1) / (4 * static_cast<int64_t>(p.k_ctas));
+    if (per_cta < p.k_chunk_pages) p.k_chunk_pages = static_cast<int>(per_cta);
+  }
   if (p.k_chunk_pages < 1) p.k_chunk_pages = 1;
 
   // Grouped queries (G >= 2, H >= 8) with at most 16 KV heads: the K pass runs
@@ -303,6 +313,14 @@ starkv_status make_plan(const starkv_layer_desc* d, int32_t batch, int32_t max_s
   if (per_sm > 2) per_sm = 2;
   p.v_per_sm = per_sm;
   p.v_ctas = sms * per_sm / p.n_rr;
+  // a call with few pages gives each CTA at least STARKV_V_MIN_PAGES of them:
+  // every CTA boundary inside a sequence costs a Z partial (H x R range fp32)
+  // that the finish reads back, which at batch 1 outweighs the pages' codes
+  {
+    const int64_t pages_max = static_cast<int64_t>(batch) * ((p.cap + 15) / 16);
+    const int64_t cap_ctas = (pages_max + STARKV_V_MIN_PAGES - 1) / STARKV_V_MIN_PAGES;
+    if (cap_ctas < p.v_ctas) p.v_ctas = static_cast<int>(cap_ctas);
+  }
   if (p.v_ctas < 1) p.v_ctas = 1;
 
   // finish: a stage holds two 64x64 B_V boxes, the hi and lo operand tiles
