@@ -351,7 +351,7 @@ struct PrepParams {
 __global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap vmap, PrepParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   const int KS = gridDim.y;
   int x = blockIdx.x;
   if (x < p.v_cols) {
@@ -704,7 +704,7 @@ __global__ void __launch_bounds__(kKTCThreads, 1)
 kpass_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                 KPassTCParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   const int S = p.stages;
   uint8_t* bslot = smem + static_cast<size_t>(S) * p.a_bytes;                    // [nbs] query tiles
   uint64_t* full = reinterpret_cast<uint64_t*>(bslot + p.nbs * static_cast<size_t>(p.b_bytes));
@@ -1004,7 +1004,7 @@ kpass_chunk_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
   using Geo = ChunkTile<VPK>;
   constexpr int KVT = Geo::kKvt, NCOL = Geo::kCols, PPT = Geo::kPages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   const int S = p.stages;
   uint8_t* bslot = smem + static_cast<size_t>(S) * p.a_bytes;                    // [nbs] query tiles
   uint64_t* full = reinterpret_cast<uint64_t*>(bslot + p.nbs * static_cast<size_t>(p.b_bytes));
@@ -1382,7 +1382,7 @@ template <bool kChunk>
 __global__ void __launch_bounds__(kVThreads, 1)
 vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   const int S = p.stages, PPS = p.pps;
   const uint32_t vstage = PPS * p.vtile_bytes, lstage = PPS * p.ltile_bytes, pstage = PPS * p.ptile_bytes;
   uint8_t* vtiles = smem;                                               // S x vstage (1024-aligned)
@@ -1775,6 +1775,7 @@ constexpr int kFinConv = kFinThreads - 64;
 constexpr int kFinKC = 64;        // rows of R per stage
 constexpr int kFinZBox = 32;      // partial rows per TMA box
 constexpr int kFinMaxRows = 256;  // sequences per batch tile at most
+constexpr int kFinSegBatch = 4;   // partial rows a converter loads before adding them
 
 // First slot (a lower bound) and slot count of the partials of sequences
 // [b0, b1) for a V-pass partition pt (P > 0).
@@ -1792,7 +1793,7 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   const int S = p.stages;
   const uint32_t a_bytes = 2u * kFinKC * 128u;                      // two 64x64 boxes of B_V
   const uint32_t half_bytes = static_cast<uint32_t>(p.npad) * 128u;  // one hi or lo operand tile
@@ -1951,15 +1952,35 @@ finish_kernel(const __grid_constant__ CUtensorMap bvmap, const __grid_constant__
         if (nseg > 0) {
           const float* src = (staged ? reinterpret_cast<const float*>(zt) : zg) +
                              static_cast<size_t>(s_row[bl]) * zstride + c * 8;
-          for (int g = 0; g < nseg; ++g) {   // segment g: nq partial rows further on
-            const float4 v0 = reinterpret_cast<const float4*>(src + static_cast<size_t>(g << p.log2nq) * zstride)[0];
-            const float4 v1 = reinterpret_cast<const float4*>(src + static_cast<size_t>(g << p.log2nq) * zstride)[1];
-            z[0] += v0.x; z[1] += v0.y; z[2] += v0.z; z[3] += v0.w;
-            z[4] += v1.x; z[5] += v1.y; z[6] += v1.z; z[7] += v1.w;
-          }
-          const float il = s_il[bl];
+          const size_t gstep = static_cast<size_t>(nq) * zstride;   // segment g: nq partial rows further on
+          // the eight threads of a quarter warp read one row's eight 32-byte
+          // items; items c >= 4 take their upper 16 bytes first, so that each
+          // load touches eight distinct bank groups.  Segments are loaded four
+          // at a time and then added in segment order.
+          const int h0 = c >> 2;
+          float4 a = make_float4(0.f, 0.f, 0.f, 0.f), e = a;
+          for (int g0 = 0; g0 < nseg; g0 += kFinSegBatch) {
+            float4 v0[kFinSegBatch], v1[kFinSegBatch];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) z[u] *= il;
+            for (int u = 0; u < kFinSegBatch; ++u) {
+              if (g0 + u < nseg) {
+                const float4* s4 = reinterpret_cast<const float4*>(src + (g0 + u) * gstep);
+                v0[u] = s4[h0];
+                v1[u] = s4[h0 ^ 1];
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < kFinSegBatch; ++u) {
+              if (g0 + u < nseg) {
+                a.x += v0[u].x; a.y += v0[u].y; a.z += v0[u].z; a.w += v0[u].w;
+                e.x += v1[u].x; e.y += v1[u].y; e.z += v1[u].z; e.w += v1[u].w;
+              }
+            }
+          }
+          const float4 lo4 = h0 ? e : a, hi4 = h0 ? a : e;
+          const float il = s_il[bl];
+          z[0] = lo4.x * il; z[1] = lo4.y * il; z[2] = lo4.z * il; z[3] = lo4.w * il;
+          z[4] = hi4.x * il; z[5] = hi4.y * il; z[6] = hi4.z * il; z[7] = hi4.w * il;
         }
         uint4 hv, lv;
         uint32_t* hw = reinterpret_cast<uint32_t*>(&hv);

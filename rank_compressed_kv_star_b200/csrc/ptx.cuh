@@ -13,6 +13,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// `base` (dynamic shared memory) advanced to the next 1024-byte boundary.  The
+// result is derived from `base` by pointer arithmetic, so the compiler still
+// knows it addresses shared memory and emits shared-memory loads and stores
+// through it (a round trip through an integer would leave generic accesses).
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* base) {
+  return base + ((1024u - (smem_u32(base) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -53,6 +53,9 @@
 #ifndef STARKV_V_MIN_PAGES
 #define STARKV_V_MIN_PAGES 16   // fewest pages per decode V-pass CTA when a call has few pages
 #endif
+#ifndef STARKV_APP_KS_MAX
+#define STARKV_APP_KS_MAX 4     // largest cluster splitting the V-code GEMM's K range
+#endif
 #ifndef STARKV_V_RING_BYTES
 #define STARKV_V_RING_BYTES (105 * 1024)
 #endif
@@ -623,7 +626,10 @@ starkv_status plan_append(const starkv_layer_desc* desc, int32_t batch, const vo
   ap->v_cols = ap->v_mt * n_bt;
   const int sms = device_sm_count();
   int KS = 1;
-  while (KS < 8 && ap->v_cols * KS * 2 <= 2 * sms && (HD / kAppKC) >= KS * 2) KS *= 2;   // <= one wave at 2 CTAs/SM
+  // <= one wave at 2 CTAs/SM, and clusters of at most 4: the whole prep grid
+  // (K-code and absorption items too) is launched in clusters of KS, and with
+  // 8 some of them found no free GPC slots until the V tiles had ended
+  while (KS < STARKV_APP_KS_MAX && ap->v_cols * KS * 2 <= 2 * sms && (HD / kAppKC) >= KS * 2) KS *= 2;
   ap->KS = KS;
   AppendVParams& vp = ap->vp;
   vp.tgt = tgt;
