@@ -1677,24 +1677,54 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
             }
           }
         } else {
-          for (int m = 0; m < p.n_mtiles; ++m) {
-            const uint32_t ta = taddr + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(m * p.npad);
-            const int j = m * 128 + q * 32 + lane;
-            const bool jok = j < p.r_range && rr * p.r_range + j < p.R;
-            const size_t hstride = static_cast<size_t>(p.v_slots) * p.r_range;
-            for (int h0 = 0; h0 < p.H; h0 += 32) {
-              uint32_t v[32];
-              if (p.npad - h0 >= 32) tmem_ld_32x32b_x32(ta + h0, v);
-              else tmem_ld_32x32b_x16(ta + h0, v);
-              tmem_ld_wait();
-              if (jok) {
-                const int hn = min(32, p.H - h0);
-                float* zr = zb + static_cast<size_t>(h0) * hstride + j;
+          // blocks of TMEM columns (M tile m, heads h0 .. h0 + 31), two loaded
+          // per wait.  A block is stored after a 4 x 4 transpose across each
+          // quad of lanes: lane 4g + i then holds head h0 + 4k + i at rows
+          // 4g .. 4g + 3 of the warp's 32, one 16-byte store, and a warp
+          // instruction writes 128 contiguous bytes of each of four heads' rows
+          const int nh = (p.H + 31) >> 5;
+          const int nblk = p.n_mtiles * nh;
+          const size_t hstride = static_cast<size_t>(p.v_slots) * p.r_range;
+          const int i4 = lane & 3;
+          const bool odd = (i4 & 1) != 0, upper = (i4 & 2) != 0;
+          auto load_blk = [&](int blk, uint32_t (&v)[32]) {
+            const int m = blk / nh, h0 = (blk - m * nh) << 5;
+            const uint32_t ta = taddr + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(m * p.npad + h0);
+            if (p.npad - h0 >= 32) tmem_ld_32x32b_x32(ta, v);
+            else tmem_ld_32x32b_x16(ta, v);
+          };
+          auto store_blk = [&](int blk, const uint32_t (&v)[32]) {
+            const int m = blk / nh, h0 = (blk - m * nh) << 5;
+            const int j0 = m * 128 + q * 32;   // the warp's first row of the R range
+            // warp-uniform: r_range and R are multiples of 64
+            if (j0 >= p.r_range || rr * p.r_range + j0 >= p.R) return;
+            const int kmax = p.npad - h0 >= 32 ? 8 : 4;   // quads of columns loaded
+            float* zq = zb + static_cast<size_t>(h0) * hstride + j0 + 4 * (lane >> 2);
 #pragma unroll
-                for (int hh = 0; hh < 32; ++hh)
-                  if (hh < hn) st_global_hint_free(zr + hh * hstride, __uint_as_float(v[hh]), keep);
+            for (int k = 0; k < 8; ++k) {
+              if (k < kmax) {
+                const float a0 = __uint_as_float(v[4 * k]), a1 = __uint_as_float(v[4 * k + 1]);
+                const float a2 = __uint_as_float(v[4 * k + 2]), a3 = __uint_as_float(v[4 * k + 3]);
+                // pairs of lanes swap the off-diagonal elements of their 2 x 2 blocks ...
+                const float y0 = __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
+                const float y1 = __shfl_xor_sync(0xffffffffu, odd ? a2 : a3, 1);
+                const float b0 = odd ? y0 : a0, b1 = odd ? a1 : y0, b2 = odd ? y1 : a2, b3 = odd ? a3 : y1;
+                // ... then lanes two apart swap the off-diagonal 2 x 2 blocks
+                const float z0 = __shfl_xor_sync(0xffffffffu, upper ? b0 : b2, 2);
+                const float z1 = __shfl_xor_sync(0xffffffffu, upper ? b1 : b3, 2);
+                const float4 f = upper ? make_float4(z0, z1, b2, b3) : make_float4(b0, b1, z0, z1);
+                const int hh = 4 * k + i4;
+                if (h0 + hh < p.H) st_global_hint_free(reinterpret_cast<float4*>(zq + hh * hstride), f, keep);
               }
             }
+          };
+          for (int blk = 0; blk < nblk; blk += 2) {
+            uint32_t va[32], vb[32];
+            load_blk(blk, va);
+            if (blk + 1 < nblk) load_blk(blk + 1, vb);
+            tmem_ld_wait();
+            store_blk(blk, va);
+            if (blk + 1 < nblk) store_blk(blk + 1, vb);
           }
         }
         tc_fence_before();

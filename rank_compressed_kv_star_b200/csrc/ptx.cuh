@@ -185,6 +185,10 @@ __device__ __forceinline__ void st_global_hint(float* p, float v, uint64_t polic
 __device__ __forceinline__ void st_global_hint_free(float* p, float v, uint64_t policy) {
   asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(policy));
 }
+__device__ __forceinline__ void st_global_hint_free(float4* p, float4 v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w), "l"(policy));
+}
 __device__ __forceinline__ void st_global_hint(uint2* p, uint2 v, uint64_t policy) {
   asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;" ::"l"(p), "r"(v.x), "r"(v.y), "l"(policy)
                : "memory");
