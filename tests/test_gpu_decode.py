@@ -110,6 +110,15 @@ def test_decode_small_heads_and_dims():
     full_check(wl)
 
 
+@pytest.mark.parametrize("H,Hkv", [(64, 0), (2, 0), (1, 0), (64, 16)])
+def test_decode_head_count_extremes(H, Hkv):
+    """64 query heads (two 32-column TMEM blocks per R tile in the V pass's drain), 1 and 2 heads (a partly
+    used quad of columns there), and 64 query heads over 16 KV heads (grouped queries at the most heads)."""
+    sh = W.LayerShape(H, 64, 16, min(256, 64 * H), num_kv_heads=Hkv)   # the joint V rank is at most H * d
+    wl = W.custom(f"h{H}kv{Hkv}", 640 + H + Hkv, sh, [3, 70, 300], append=False)
+    full_check(wl)
+
+
 def test_decode_empty_and_zero_batch():
     sh = W.LayerShape(32, 128, 64, 2048)
     wl = W.custom("empties", 7, sh, [0, 0, 40, 0], append=False)
