@@ -1378,6 +1378,20 @@ constexpr int kMaxPPS = 8;
 constexpr int kVThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 weights + epilogue
 constexpr int32_t kFirst = 1, kLast = 2;
 
+// 4 x 4 transpose across a quad of lanes (i = lane & 3): on entry a lane holds
+// row i, columns 0..3 of its quad's block; on return rows 0..3 of column i.
+// Pairs of lanes first swap the off-diagonal elements of their 2 x 2 blocks,
+// then lanes two apart swap the off-diagonal 2 x 2 blocks.
+__device__ __forceinline__ float4 quad_transpose(float a0, float a1, float a2, float a3, int i) {
+  const bool odd = (i & 1) != 0, upper = (i & 2) != 0;
+  const float y0 = __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
+  const float y1 = __shfl_xor_sync(0xffffffffu, odd ? a2 : a3, 1);
+  const float b0 = odd ? y0 : a0, b1 = odd ? a1 : y0, b2 = odd ? y1 : a2, b3 = odd ? a3 : y1;
+  const float z0 = __shfl_xor_sync(0xffffffffu, upper ? b0 : b2, 2);
+  const float z1 = __shfl_xor_sync(0xffffffffu, upper ? b1 : b3, 2);
+  return upper ? make_float4(z0, z1, b2, b3) : make_float4(b0, b1, z0, z1);
+}
+
 template <bool kChunk>
 __global__ void __launch_bounds__(kVThreads, 1)
 vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
@@ -1648,17 +1662,21 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
         const size_t slot = static_cast<size_t>(mt.b) + cta;
         // partial rows [R range][head][slot][r_range]: head h0+hh's row of this slot
         float* zb = p.zpart + ((static_cast<size_t>(rr) * p.H) * p.v_slots + slot) * p.r_range;
-        // every (m, h0) block: 32 TMEM columns into registers, then 32 stores
-        // with constant register indices (fully unrolled), each a 128-byte
-        // row piece across the warp's lanes
+        // A block of 32 TMEM columns is stored after a quad transpose
+        // (quad_transpose): lane 4g + i then holds column 4k + i of the block
+        // at rows 4g .. 4g + 3 of the warp's 32 rows of R, one 16-byte store,
+        // and a warp instruction writes 128 contiguous bytes of each of four
+        // columns' partial rows.  r_range and R are multiples of 64, so a
+        // warp's 32 rows are all inside the R range or all outside it.
+        const int i4 = lane & 3;
         if constexpr (kChunk) {
           // virtual head (h, i): row slot * nq + i of head h (npad = lw, a multiple of 32)
           const uint32_t nqm = (1u << p.log2nq) - 1u;
           for (int m = 0; m < p.n_mtiles; ++m) {
             const uint32_t ta = taddr + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(m * p.npad);
-            const int j = m * 128 + q * 32 + lane;
-            const bool jok = j < p.r_range && rr * p.r_range + j < p.R;
-            float* zj = p.zpart + j;
+            const int j0 = m * 128 + q * 32;   // the warp's first row of the R range
+            const bool jok = j0 < p.r_range && rr * p.r_range + j0 < p.R;
+            float* zq = p.zpart + j0 + 4 * (lane >> 2);
             for (int h0 = 0; h0 < p.npad; h0 += 32) {
               uint32_t v[32];
               tmem_ld_32x32b_x32(ta + h0, v);
@@ -1666,27 +1684,24 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
               if (jok) {
                 const uint32_t c0 = static_cast<uint32_t>(vg * p.lw + h0);
 #pragma unroll
-                for (int hh = 0; hh < 32; ++hh) {
-                  const uint32_t col = c0 + hh;
+                for (int k = 0; k < 8; ++k) {
+                  const float4 f = quad_transpose(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                                  __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]), i4);
+                  const uint32_t col = c0 + 4 * k + i4;
                   const size_t row =
                       ((static_cast<size_t>(rr * p.H + static_cast<int>(col >> p.log2nq)) * p.v_slots + slot)
                        << p.log2nq) + (col & nqm);
-                  st_global_hint_free(zj + row * p.r_range, __uint_as_float(v[hh]), keep);
+                  st_global_hint_free(reinterpret_cast<float4*>(zq + row * p.r_range), f, keep);
                 }
               }
             }
           }
         } else {
           // blocks of TMEM columns (M tile m, heads h0 .. h0 + 31), two loaded
-          // per wait.  A block is stored after a 4 x 4 transpose across each
-          // quad of lanes: lane 4g + i then holds head h0 + 4k + i at rows
-          // 4g .. 4g + 3 of the warp's 32, one 16-byte store, and a warp
-          // instruction writes 128 contiguous bytes of each of four heads' rows
+          // per wait
           const int nh = (p.H + 31) >> 5;
           const int nblk = p.n_mtiles * nh;
           const size_t hstride = static_cast<size_t>(p.v_slots) * p.r_range;
-          const int i4 = lane & 3;
-          const bool odd = (i4 & 1) != 0, upper = (i4 & 2) != 0;
           auto load_blk = [&](int blk, uint32_t (&v)[32]) {
             const int m = blk / nh, h0 = (blk - m * nh) << 5;
             const uint32_t ta = taddr + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(m * p.npad + h0);
@@ -1696,23 +1711,14 @@ vpass_kernel(const __grid_constant__ CUtensorMap vmap, VPassParams p) {
           auto store_blk = [&](int blk, const uint32_t (&v)[32]) {
             const int m = blk / nh, h0 = (blk - m * nh) << 5;
             const int j0 = m * 128 + q * 32;   // the warp's first row of the R range
-            // warp-uniform: r_range and R are multiples of 64
-            if (j0 >= p.r_range || rr * p.r_range + j0 >= p.R) return;
+            if (j0 >= p.r_range || rr * p.r_range + j0 >= p.R) return;   // warp-uniform
             const int kmax = p.npad - h0 >= 32 ? 8 : 4;   // quads of columns loaded
             float* zq = zb + static_cast<size_t>(h0) * hstride + j0 + 4 * (lane >> 2);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               if (k < kmax) {
-                const float a0 = __uint_as_float(v[4 * k]), a1 = __uint_as_float(v[4 * k + 1]);
-                const float a2 = __uint_as_float(v[4 * k + 2]), a3 = __uint_as_float(v[4 * k + 3]);
-                // pairs of lanes swap the off-diagonal elements of their 2 x 2 blocks ...
-                const float y0 = __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
-                const float y1 = __shfl_xor_sync(0xffffffffu, odd ? a2 : a3, 1);
-                const float b0 = odd ? y0 : a0, b1 = odd ? a1 : y0, b2 = odd ? y1 : a2, b3 = odd ? a3 : y1;
-                // ... then lanes two apart swap the off-diagonal 2 x 2 blocks
-                const float z0 = __shfl_xor_sync(0xffffffffu, upper ? b0 : b2, 2);
-                const float z1 = __shfl_xor_sync(0xffffffffu, upper ? b1 : b3, 2);
-                const float4 f = upper ? make_float4(z0, z1, b2, b3) : make_float4(b0, b1, z0, z1);
+                const float4 f = quad_transpose(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                                __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]), i4);
                 const int hh = 4 * k + i4;
                 if (h0 + hh < p.H) st_global_hint_free(reinterpret_cast<float4*>(zq + hh * hstride), f, keep);
               }
