@@ -94,8 +94,8 @@ def whole_job_tokens_per_s(world: int, batch_per_rank: int, ms_per_step_max: flo
 # profiles/gqa_streaming_b32_t8192_full.md give the commands; an entry is
 # emptied when its kernel changes.
 NCU_TRAFFIC_PER_TOKEN: dict = {
-    (32, 32, 64, 2048): {"kpass": 4124.2, "vpass": 4247.8},
-    (32, 8, 64, 512): {"kpass": 1049.3, "vpass": 1178.5},
+    (32, 32, 64, 2048): {"kpass": 4124.2, "vpass": 4252.5},
+    (32, 8, 64, 512): {"kpass": 1049.3, "vpass": 1163.9},
 }
 
 
